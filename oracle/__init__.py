@@ -1,0 +1,218 @@
+"""CPU oracle of the MSA routed-memory path (double precision).
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and bench.py's CPU baseline
+are the only code allowed to import this package. The CUDA library never imports it and
+shares no code with it; the two meet only through the seeded inputs of ``synth``.
+
+The arithmetic lives in ``msa_oracle.c`` (plain C, double precision, one output at a time);
+this module marshals numpy arrays into it. Storage rounding of the bf16 configuration is
+mirrored with the oracle's own round-to-nearest-even (``round_bf16``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+
+FP32, BF16 = 0, 1
+
+
+def build(force: bool = False, src: str | None = None, out: str | None = None) -> str:
+    """Compile the oracle with gcc (OpenMP). ``src``/``out`` let a test build a variant."""
+    src = src or _SRC
+    out = out or _SO
+    if force or not os.path.exists(out) or os.path.getmtime(src) > os.path.getmtime(out):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", out, src, "-lm"])
+    return out
+
+
+def _declare(L):
+    vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    L.orc_num_threads.restype = i32
+    L.orc_round_bf16.restype = ctypes.c_uint16
+    L.orc_round_bf16.argtypes = [dbl]
+    L.orc_round_bf16_array.restype = None
+    L.orc_round_bf16_array.argtypes = [vp, vp, i64]
+    L.orc_rope.restype = None
+    L.orc_rope.argtypes = [vp, i32, dbl, dbl]
+    L.orc_cosine.restype = dbl
+    L.orc_cosine.argtypes = [vp, vp, i32]
+    L.orc_encode_pool.restype = i64
+    L.orc_encode_pool.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, dbl, vp, vp, vp, vp]
+    L.orc_route.restype = i32
+    L.orc_route.argtypes = [i32, vp, i32, i32, i32, vp, i32, i32, vp, i32, i32, vp, vp, vp, vp]
+    L.orc_gather.restype = i32
+    L.orc_gather.argtypes = [vp, i32, i32, vp, i32, i32, vp, vp]
+    L.orc_attend.restype = i32
+    L.orc_attend.argtypes = [i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32, i32, i32,
+                             i32, dbl, dbl, vp]
+    return L
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def load_variant(path: str):
+    """Load a separately built copy of the oracle (used by the planted-mistake tests)."""
+    return _declare(ctypes.CDLL(path))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dt(x: np.ndarray) -> int:
+    if x.dtype == np.float32:
+        return FP32
+    if x.dtype == np.uint16:
+        return BF16
+    raise TypeError(f"oracle inputs are float32 or bf16 bits (uint16), got {x.dtype}")
+
+
+def _c(x):
+    return np.ascontiguousarray(x)
+
+
+def _same(*arrs) -> int:
+    """All tensor inputs of one oracle call share one storage type; return its code."""
+    codes = {_dt(a) for a in arrs}
+    if len(codes) != 1:
+        raise TypeError("oracle inputs of one call must share a dtype (float32 or bf16 bits)")
+    return codes.pop()
+
+
+def num_threads(L=None) -> int:
+    return (L or lib()).orc_num_threads()
+
+
+def round_bf16(x: np.ndarray, L=None) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    (L or lib()).orc_round_bf16_array(_p(x), _p(out), x.size)
+    return out
+
+
+def store_as(x: np.ndarray, dtype: str, L=None) -> np.ndarray:
+    """Round double results to the storage type of the configuration."""
+    return round_bf16(x, L) if dtype == "bf16" else np.asarray(x, dtype=np.float32)
+
+
+def rope(x: np.ndarray, pos: float, base: float, L=None) -> np.ndarray:
+    """RoPE of one head vector (copy, float64)."""
+    v = np.array(x, dtype=np.float64, copy=True)
+    (L or lib()).orc_rope(_p(v), v.shape[-1], float(pos), float(base))
+    return v
+
+
+def cosine(q, k, L=None) -> float:
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    return (L or lib()).orc_cosine(_p(q), _p(k), q.shape[-1])
+
+
+def encode_pool(K, V, K_r, doc_tok_off, chunk: int, rope_base: float, L=None):
+    """Doc-wise RoPE + chunk mean pooling. Returns (Kbar, Vbar, Krbar) float64
+    [n_chunks, h_kv, d] and doc_chunk_off [n_docs+1] int64."""
+    K, V, K_r = _c(K), _c(V), _c(K_r)
+    off = np.ascontiguousarray(doc_tok_off, dtype=np.int64)
+    n_docs = len(off) - 1
+    h_kv, d = K.shape[1], K.shape[2]
+    n_chunks = int(sum(-(-int(off[i + 1] - off[i]) // chunk) for i in range(n_docs)))
+    Kb = np.empty((n_chunks, h_kv, d))
+    Vb = np.empty_like(Kb)
+    Rb = np.empty_like(Kb)
+    coff = np.empty(n_docs + 1, dtype=np.int64)
+    r = (L or lib()).orc_encode_pool(_same(K, V, K_r), _p(K), _p(V), _p(K_r), _p(off), n_docs, chunk, h_kv,
+                                     d, float(rope_base), _p(Kb), _p(Vb), _p(Rb), _p(coff))
+    if r != n_chunks:
+        raise ValueError(f"orc_encode_pool returned {r}")
+    return Kb, Vb, Rb, coff
+
+
+def route(Q_r, Kbar_r, doc_chunk_off, k: int, exclude_bits=None, L=None):
+    """Cosine routing + top-k. Returns (top_ids int32 [B,k], top_scores f64 [B,k],
+    doc_scores f64 [B, n_docs])."""
+    Q_r, Kbar_r = _c(Q_r), _c(Kbar_r)
+    B, T, h_qr, d = Q_r.shape
+    h_kv = Kbar_r.shape[1]
+    coff = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
+    n_docs = len(coff) - 1
+    ids = np.empty((B, k), dtype=np.int32)
+    ts = np.empty((B, k))
+    ds = np.empty((B, n_docs))
+    ex = None if exclude_bits is None else np.ascontiguousarray(exclude_bits, dtype=np.uint32)
+    r = (L or lib()).orc_route(_same(Q_r, Kbar_r), _p(Q_r), B, T, h_qr, _p(Kbar_r), h_kv, d, _p(coff),
+                               n_docs, k, _p(ex), _p(ds), _p(ids), _p(ts))
+    if r != 0:
+        raise ValueError("orc_route: invalid arguments")
+    return ids, ts, ds
+
+
+def gather(top_ids, doc_chunk_off, max_ctx: int, L=None):
+    """Returns (gather_idx int32 [B, max_ctx], ctx_len int32 [B])."""
+    ids = np.ascontiguousarray(top_ids, dtype=np.int32)
+    B, k = ids.shape
+    coff = np.ascontiguousarray(doc_chunk_off, dtype=np.int64)
+    gi = np.empty((B, max_ctx), dtype=np.int32)
+    cl = np.empty(B, dtype=np.int32)
+    r = (L or lib()).orc_gather(_p(ids), B, k, _p(coff), len(coff) - 1, max_ctx, _p(gi), _p(cl))
+    if r != 0:
+        raise ValueError(f"orc_gather returned {r}")
+    return gi, cl
+
+
+def attend(Q, K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0: int, rope_base: float,
+           scale: float = 0.0, L=None):
+    """Global-RoPE GQA attention over [gathered memory ; causal local]. Returns O float64."""
+    Q, K_loc, V_loc, Kbar, Vbar = map(_c, (Q, K_loc, V_loc, Kbar, Vbar))
+    B, T, h_q, d = Q.shape
+    Lloc, h_kv = K_loc.shape[1], K_loc.shape[2]
+    gi = np.ascontiguousarray(gather_idx, dtype=np.int32)
+    cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+    O = np.empty((B, T, h_q, d))
+    r = (L or lib()).orc_attend(_same(Q, K_loc, V_loc, Kbar, Vbar), _p(Q), B, T, h_q, _p(K_loc), _p(V_loc), Lloc, _p(Kbar),
+                                _p(Vbar), _p(gi), _p(cl), gi.shape[1], h_kv, d, int(pos0),
+                                float(rope_base), float(scale), _p(O))
+    if r != 0:
+        raise ValueError("orc_attend: invalid arguments")
+    return O
+
+
+def pipeline(w, inp: dict, L=None) -> dict:
+    """Oracle of one routed layer: (encode →) route → gather → attend, with the storage
+    rounding of the configuration between steps. ``inp`` comes from synth."""
+    out = {}
+    dt = w.dtype
+    if "K" in inp:  # per-token inputs: offline encode first
+        Kb, Vb, Rb, coff = encode_pool(inp["K"], inp["V"], inp["K_r"], inp["doc_tok_off"],
+                                       w.chunk, w.rope_base, L)
+        out.update(Kbar64=Kb, Vbar64=Vb, Krbar64=Rb)
+        Kbar, Vbar, Krbar = (store_as(a, dt, L) for a in (Kb, Vb, Rb))
+        out.update(Kbar=Kbar, Vbar=Vbar, Kbar_r=Krbar, doc_chunk_off=coff)
+    else:
+        Kbar, Vbar, Krbar, coff = inp["Kbar"], inp["Vbar"], inp["Kbar_r"], inp["doc_chunk_off"]
+    ids, ts, ds = route(inp["Q_r"], Krbar, coff, w.k, inp.get("exclude_bits"), L)
+    out.update(top_ids=ids, top_scores=ts, doc_scores=ds)
+    cpd_max = int(np.max(np.diff(coff))) if len(coff) > 1 else 0
+    max_ctx = inp.get("max_ctx", w.k * cpd_max)
+    gi, cl = gather(ids, coff, max_ctx, L)
+    out.update(gather_idx=gi, ctx_len=cl)
+    O = attend(inp["Q"], inp["K_loc"], inp["V_loc"], Kbar, Vbar, gi, cl, pos0=w.k,
+               rope_base=w.rope_base, L=L)
+    out["O64"] = O
+    out["O"] = store_as(O, dt, L)
+    return out
