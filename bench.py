@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA routed-memory hot path on B200 (libmsa).
+
+Default workload: routed decode over a 100M-token memory bank on one GPU, 18 routed
+layers (200,000 docs x 500 tokens -> 1,600,000 chunks of 64; K̄_r bf16 [chunks, 8, 128] per
+layer resident in HBM, 3.28 GB per layer, 59 GB in total; K̄/V̄ bf16 in pinned host memory,
+the selected documents fetched per layer), batch of 4 decode queries (T = 1, 32 query
+heads, 8 KV heads, d = 128, k = 16, 2048-token local KV cache each).
+
+One step = for each routed layer: route + top-k over the whole bank (msa_route_topk),
+context assembly from the host bank (msa_fetch_begin/finish; copies overlap the next
+layer's scan), sparse attention (msa_sparse_attend). Queries/s = B / step time.
+
+``--workload bank10m`` runs the 10M-token single-layer decode (20,000 docs, B = 8, device
+bank) instead. ``--impl reference`` times the CPU oracle on the host cores (a bounded
+sample of the same workload). Under torchrun every rank runs an independent replica
+(the path does not shard: no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MSA routed-decode queries/s at 10M/100M-token bank; router-scan HBM GB/s"
+UNIT = "queries/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
+    ap.add_argument("--workload", default="bank100m", choices=["bank100m", "bank10m"])
+    ap.add_argument("--fetch", default="memcpy", choices=["memcpy", "zerocopy"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-layers", type=int, default=3,
+                    help="routed layers in the CPU-oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ workload
+class Decode:
+    """Routed decode over a memory bank: per layer route -> fetch/gather -> attend."""
+
+    def __init__(self, w, dev, fetch: str, rank: int):
+        import torch
+
+        import long_context_doc_b200 as msa
+        import synth
+        self.torch, self.msa, self.w, self.dev = torch, msa, w, dev
+        self.fetch = fetch if w.layers > 1 else "device"
+        self.L = w.layers
+        self.main = torch.cuda.current_stream()
+        self.copy = torch.cuda.Stream()
+        self.layers = []
+        seed_w = w.scaled(seed=w.seed + 1000 * rank)
+        self.sw = seed_w
+        for l in range(self.L):
+            dv = synth.dev_bank_workload(seed_w, dev, layer=l, with_kv=(self.fetch == "device"))
+            dv["inv"] = msa.kr_inv_norm(dv["Kbar_r"])
+            self.layers.append(dv)
+        self.coff_host = self.layers[0]["doc_chunk_off"]
+        self.coff = torch.from_numpy(self.coff_host).to(dev)
+        self.n_chunks = int(self.coff_host[-1])
+        self.n_docs = w.n_docs
+        self.max_ctx = w.k * int(np.max(np.diff(self.coff_host)))
+        if self.fetch != "device":
+            # one pinned host K̄/V̄ bank shared by the routed layers (only the selected rows
+            # ever cross the host link, so the fetch traffic does not depend on this)
+            self.Kh = torch.empty((self.n_chunks, w.h_kv, w.d), dtype=torch.bfloat16,
+                                  pin_memory=True)
+            self.Vh = torch.empty_like(self.Kh, pin_memory=True)
+            tmp = torch.empty((1 << 20, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)
+            row = w.h_kv * w.d
+            for name, dst in (("Kbar", self.Kh), ("Vbar", self.Vh)):
+                tid = synth.KBAR if name == "Kbar" else synth.VBAR
+                for c0 in range(0, self.n_chunks, tmp.shape[0]):
+                    n = min(tmp.shape[0], self.n_chunks - c0)
+                    t = tmp[:n]
+                    synth.dev_normal(t, seed_w.seed, synth.tag(tid, 0), first=c0 * row)
+                    dst[c0:c0 + n].copy_(t)
+            del tmp
+            self.fetchers = [msa.Fetcher(w.B, w.k) for _ in range(2)]
+        B, k = w.B, w.k
+        ws_r = msa.msa_route_topk_workspace(B, w.T, w.h_qr, w.h_kv, w.d, 1, self.n_docs,
+                                            self.n_chunks, k)
+        ws_a = msa.msa_sparse_attend_workspace(B, w.T, w.h_q, w.h_kv, w.d, self.max_ctx, w.L_loc)
+        self.buf = []
+        for _ in range(2):
+            self.buf.append(dict(
+                ws_r=torch.empty(ws_r, dtype=torch.uint8, device=dev),
+                ws_a=torch.empty(ws_a, dtype=torch.uint8, device=dev),
+                ws_g=torch.zeros(256, dtype=torch.uint8, device=dev),
+                ids=torch.empty((B, k), dtype=torch.int32, device=dev),
+                sc=torch.empty((B, k), dtype=torch.float32, device=dev),
+                gi=torch.empty((B, self.max_ctx), dtype=torch.int32, device=dev),
+                cl=torch.empty(B, dtype=torch.int32, device=dev),
+                cK=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev),
+                cV=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)))
+        self.O = [torch.empty((B, w.T, w.h_q, w.d), dtype=torch.bfloat16, device=dev)
+                  for _ in range(self.L)]
+        self.route_ev = None
+        # kernels per step (own kernels only; memsets and copies excluded)
+        att_plan_S = 1
+        self.kernels_per_layer = 1 + 1 + 1 + 1  # route scan, gather, rope table, attend
+        from long_context_doc_b200 import msa_sparse_attend_workspace  # noqa: F401
+
+    # per-layer pieces -------------------------------------------------------------
+    def route(self, l):
+        msa, d, bf = self.msa, self.layers[l], self.buf[l % 2]
+        if self.route_ev is not None:
+            self.route_ev[l][0].record(self.main)
+        msa.msa_route_topk(d["Q_r"], d["Kbar_r"], d["inv"], self.coff, self.w.k, None, bf["ids"],
+                           bf["sc"], None, bf["ws_r"], self.main)
+        if self.route_ev is not None:
+            self.route_ev[l][1].record(self.main)
+
+    def begin(self, l):
+        bf = self.buf[l % 2]
+        if self.fetch == "memcpy":
+            self.fetchers[l % 2].begin(bf["ids"], self.coff, self.max_ctx, bf["gi"], bf["cl"],
+                                       bf["ws_g"], self.main)
+        elif self.fetch == "zerocopy":
+            self.msa.msa_gather(bf["ids"], self.coff, self.Kh, self.Vh, self.max_ctx, bf["gi"],
+                                bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.main)
+        else:
+            d = self.layers[l]
+            self.msa.msa_gather(bf["ids"], self.coff, d["Kbar"], d["Vbar"], self.max_ctx,
+                                bf["gi"], bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.main)
+
+    def finish(self, l):
+        if self.fetch == "memcpy":
+            bf = self.buf[l % 2]
+            self.fetchers[l % 2].finish(self.coff_host, self.Kh, self.Vh, self.max_ctx, bf["cK"],
+                                        bf["cV"], self.main, self.copy, 10_000)
+
+    def attend(self, l):
+        d, bf, w = self.layers[l], self.buf[l % 2], self.w
+        self.msa.msa_sparse_attend(d["Q"], d["K_loc"], d["V_loc"], bf["cK"], bf["cV"], bf["cl"],
+                                   w.k, w.rope_base, 0.0, self.O[l], bf["ws_a"], self.main)
+
+    def step(self):
+        self.route(0)
+        self.begin(0)
+        for l in range(self.L):
+            if l + 1 < self.L:
+                self.route(l + 1)
+                self.begin(l + 1)
+            self.finish(l)
+            self.attend(l)
+
+    def scan_bytes(self):
+        w = self.w
+        return self.n_chunks * w.h_kv * w.d * 2 + self.n_chunks * w.h_kv * 4
+
+
+def run_libmsa(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    w = synth.C4 if args.workload == "bank100m" else synth.C3
+    wk = Decode(w, dev, args.fetch, rank)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        wk.step()
+    barrier()
+    # timed region: K steps, per-route events for the roofline
+    Kst = args.steps
+    wk.route_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(wk.L)] for _ in range(Kst)]
+    ev_route = wk.route_ev
+    route_ms = []
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record(wk.main)
+    for s in range(Kst):
+        wk.route_ev = ev_route[s]
+        wk.step()
+    t1.record(wk.main)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = t0.elapsed_time(t1) / Kst
+    for s in range(Kst):
+        for l in range(wk.L):
+            route_ms.append(ev_route[s][l][0].elapsed_time(ev_route[s][l][1]))
+    wk.route_ev = None
+    # end to end: per-step query inputs copied from pinned host memory, outputs read back
+    host_in = []
+    for l in range(wk.L):
+        d = wk.layers[l]
+        host_in.append([t.cpu().pin_memory() for t in (d["Q_r"], d["Q"], d["K_loc"][:, -1:],
+                                                        d["V_loc"][:, -1:])])
+    host_O = [o.cpu().pin_memory() for o in wk.O]
+    host_ids = [b["ids"].cpu().pin_memory() for b in wk.buf]
+    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs)
+    d2h = sum(o.numel() * o.element_size() for o in host_O) + wk.L * w.B * w.k * 4
+
+    def e2e_step():
+        for l in range(wk.L):
+            d = wk.layers[l]
+            qr, q, kn, vn = host_in[l]
+            d["Q_r"].copy_(qr, non_blocking=True)
+            d["Q"].copy_(q, non_blocking=True)
+            d["K_loc"][:, -1:].copy_(kn, non_blocking=True)
+            d["V_loc"][:, -1:].copy_(vn, non_blocking=True)
+        wk.step()
+        for l in range(wk.L):
+            host_O[l].copy_(wk.O[l], non_blocking=True)
+        host_ids[0].copy_(wk.buf[0]["ids"], non_blocking=True)
+        host_ids[1].copy_(wk.buf[1]["ids"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    Ke = max(5, Kst // 2)
+    e0.record(wk.main)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(wk.main)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([step_ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, e2e_ms = float(t[0]), float(t[1])
+    value = world * w.B / (step_ms / 1e3)
+    e2e_value = world * w.B / (e2e_ms / 1e3)
+    route_avg = statistics.mean(route_ms)
+    peak, peak_kind = peaks()
+    achieved = wk.scan_bytes() / (route_avg / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": Kst,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 normals, planted docs; no dataset)",
+        "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len, "n_docs": w.n_docs,
+                   "n_chunks": wk.n_chunks, "chunk": w.chunk, "routed_layers": wk.L,
+                   "batch": w.B, "T": w.T, "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d, "k": w.k,
+                   "local_kv": w.L_loc,
+                   "kv_bank": ("pinned host memory, one K̄/V̄ bank shared by the routed layers, "
+                               f"fetch={wk.fetch}") if wk.fetch != "device" else "HBM",
+                   "l2": "no flush: every layer scans a 3.28 GB K̄_r, far larger than the 126 MB L2"
+                   if wk.L > 1 else "no flush: the 328 MB K̄_r scan exceeds the 126 MB L2",
+                   "parallelism": f"replicas x{world}"},
+        "router_scan_gbs": round(achieved, 1),
+        "roofline": {"kernel": "route_scan (msa_route_topk: scan + fused top-k)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": None, "bytes_per_launch": wk.scan_bytes(),
+                     "avg_launch_ms": round(route_avg, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": Kst * wk.L * wk.kernels_per_layer,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_layers)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_layer_time(w, layer: int) -> float:
+    """Oracle time of one routed layer of the decode workload for the whole batch:
+    route over every document, gather, attend (inputs generated beforehand, untimed)."""
+    import oracle
+    import synth
+    inp = synth.make_bank_workload(w, layer, with_bank=False)
+    coff = inp["doc_chunk_off"]
+    Krb = synth.host_bank_rows(w, "Kbar_r", 0, int(coff[-1]), layer=layer, coff=coff,
+                               Q_r=inp["Q_r"])
+    t0 = time.perf_counter()
+    ids, _, _ = oracle.route(inp["Q_r"], Krb, coff, w.k)
+    max_ctx = w.k * int(np.max(np.diff(coff)))
+    gi, cl = oracle.gather(ids, coff, max_ctx)
+    t1 = time.perf_counter()
+    del Krb
+    # the gathered rows only (the oracle reads bank rows through the gather indices)
+    rows = np.unique(gi[gi >= 0])
+    remap = np.full(int(coff[-1]), -1, np.int64)
+    remap[rows] = np.arange(len(rows))
+    Kb = np.concatenate([synth.host_bank_rows(w, "Kbar", int(r), int(r) + 1, layer=0)
+                         for r in rows])
+    Vb = np.concatenate([synth.host_bank_rows(w, "Vbar", int(r), int(r) + 1, layer=0)
+                         for r in rows])
+    gi2 = np.where(gi >= 0, remap[np.maximum(gi, 0)], -1).astype(np.int32)
+    t2 = time.perf_counter()
+    oracle.attend(inp["Q"], inp["K_loc"], inp["V_loc"], Kb, Vb, gi2, cl, w.k, w.rope_base)
+    t3 = time.perf_counter()
+    return (t1 - t0) + (t3 - t2)
+
+
+def cpu_baseline(w, n_layers: int) -> dict:
+    import oracle
+    times = [oracle_layer_time(w, l) for l in range(n_layers)]
+    per_layer = sum(times) / len(times)
+    step = per_layer * w.layers
+    return {"value": round(w.B / step, 4), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"{n_layers} of {w.layers} routed layers of the same workload, each: route "
+                       f"over all {w.n_docs} docs + gather + attend for the batch of {w.B}; "
+                       f"step time = mean layer time x {w.layers}"),
+            "cpu_seconds": round(sum(times), 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    w = synth.C4 if args.workload == "bank100m" else synth.C3
+    for l in range(min(args.warmup, 1)):
+        oracle_layer_time(w.scaled(n_docs=2000), l)
+    times = []
+    for s in range(args.steps):
+        times.append(oracle_layer_time(w, s % w.layers) * w.layers)
+        if sum(times) / w.layers > 60:
+            break
+    step = statistics.mean(times)
+    value = w.B / step
+    line = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1,
+            "steps": len(times), "warmup": args.warmup, "ms_per_step": round(step * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len,
+                       "routed_layers": w.layers, "batch": w.B, "k": w.k},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": "each step = one routed layer (route over every doc + "
+                                       "gather + attend for the batch) x the layer count"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_libmsa(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+/*
+ * msa.h - C ABI of libmsa, the routed-memory hot path of Memory Sparse Attention (MSA)
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The method (as described on the pages about MSA):
+ *  - offline "global memory encoding": each document's per-token K, V and router keys K_r
+ *    are compressed by fixed-length chunk mean pooling into K̄, V̄, K̄_r, with document-wise
+ *    RoPE (positions restart at 0 in every document)
+ *      [news.neo-ai.one article, "全体設計 / アーキテクチャ" and "推論パイプライン" (Fig. 3);
+ *       ruixiangma.github.io blog "Memory-Sparse-Attention", "方法 / 稀疏注意力机制" and
+ *       "文档级RoPE"];
+ *  - online routing: the router query Q_r is matched against every chunk's K̄_r by cosine
+ *    similarity, averaged over heads, maximised over query tokens (and over a document's
+ *    chunks), and the top-k documents are selected
+ *      [news.neo-ai.one, "アーキテクチャ"; github-eval-reports "MSA 项目评测报告", "核心模块"];
+ *  - context assembly: only the selected K̄/V̄ are loaded (from GPU memory or, for very large
+ *    banks, from host memory, asynchronously) and concatenated with the query's local K/V
+ *      [news.neo-ai.one, "推論パイプライン"; ruixiangma blog, "Memory Parallel"];
+ *  - sparse generation: attention over [memory ; local] with "global RoPE" on the active
+ *    context, the query's start index shifted by k, the number of retrieved blocks
+ *      [news.neo-ai.one, "グローバル RoPE"; ai-papers.net summary, "MSAの提案手法"].
+ *
+ * Conventions (all entry points):
+ *  - Every call returns an msa_status; nothing aborts, exits or prints. Arguments are
+ *    validated on the host before any work is enqueued; on an error nothing is enqueued
+ *    and the outputs are left untouched. msa_last_error() gives a thread-local message.
+ *  - Tensors are caller-owned, dense, row-major, and DEVICE pointers unless marked "host".
+ *    The library allocates nothing on the hot path: scratch space is a caller-provided
+ *    workspace whose size the matching *_workspace() query returns (256-byte aligned).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). All
+ *    device work is asynchronous on that stream. The only host waits are in
+ *    msa_fetch_finish (bounded by timeout_ms) and msa_workspace_status.
+ *  - dtype: MSA_FP32 (float) or MSA_BF16 (bfloat16 bit patterns); all floating tensors of
+ *    one call share it, except the fp32 inverse norms and scores.
+ *  - Supported shapes: d in {64, 128}; h_q % h_kv == 0; h_qr % h_kv == 0; 1 <= k <= 32;
+ *    anything else returns MSA_ERR_UNSUPPORTED or MSA_ERR_INVALID_ARG.
+ *  - Calls are reentrant; two calls may run concurrently on different streams as long as
+ *    they do not share a workspace.
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent layout */
+    MSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (d, k, head counts, T) */
+    MSA_ERR_WORKSPACE = 3,     /* workspace missing, misaligned or smaller than required */
+    MSA_ERR_CUDA = 4,          /* a CUDA runtime call failed (message has the CUDA error) */
+    MSA_ERR_TIMEOUT = 5,       /* a bounded host wait or a bounded device wait expired */
+    MSA_ERR_DEVICE = 6         /* a kernel recorded an error in its workspace status word */
+} msa_status;
+
+typedef enum { MSA_FP32 = 0, MSA_BF16 = 1 } msa_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char* msa_status_string(int status);
+/* Thread-local description of the last failure in this thread ("" if none). */
+const char* msa_last_error(void);
+/* ABI version, (major << 16) | minor. */
+int msa_version(void);
+
+/* ------------------------------------------------------------------------------------
+ * Bank layout helper (host only, no device work).
+ * Number of chunks of a corpus whose document d owns tokens
+ * [doc_tok_off_host[d], doc_tok_off_host[d+1]): sum over docs of ceil(len / chunk).
+ * Chunks never cross documents; a partial last chunk counts as one chunk.
+ * Returns the count, or -1 if the offsets are not non-decreasing from 0 or chunk < 1.
+ */
+int64_t msa_count_chunks(const int64_t* doc_tok_off_host, int64_t n_docs, int32_t chunk);
+
+/* ------------------------------------------------------------------------------------
+ * msa_encode_pool - offline memory encoding: document-wise RoPE + chunk mean pooling.
+ *   [news.neo-ai.one, "アーキテクチャ": chunk-wise mean pooling compresses K/V/K_r;
+ *    "並列（ドキュメント単位）RoPE": positions restart at 0 per document;
+ *    ruixiangma blog, "稀疏注意力机制 / 分块压缩" and "文档级RoPE"]
+ *
+ * K, V, K_r        [n_tok, h_kv, d] per-token keys, values and router keys (dtype).
+ * doc_tok_off_host host [n_docs+1] token offsets (validated: starts at 0, non-decreasing,
+ *                  ends at n_tok, and sum of ceil(len/chunk) == n_chunks).
+ * doc_tok_off      device copy of the same offsets.
+ * rope_base        RoPE base (e.g. 1e6); <= 0 disables rotation. RoPE pairs element i with
+ *                  element i + d/2 ("rotate half") at angle pos * base^(-2i/d), pos = the
+ *                  token's index within its document. K and K_r are rotated, V is not.
+ * Kbar, Vbar, Kbar_r [n_chunks, h_kv, d] outputs (dtype): mean over each chunk's valid
+ *                  tokens, accumulated in fp32, stored with round-to-nearest-even.
+ * kr_inv_norm      [n_chunks, h_kv] fp32 output (nullable): 1/||Kbar_r[c,h]|| of the STORED
+ *                  row (0 for a zero row), consumed by msa_route_topk.
+ * doc_chunk_off    [n_docs+1] int64 output: chunk offsets (doc i owns chunks
+ *                  [doc_chunk_off[i], doc_chunk_off[i+1])).
+ * No workspace. Errors: INVALID_ARG (layout, null), UNSUPPORTED (d, dtype, h_kv*d).
+ */
+msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_t n_tok,
+                           const int64_t* doc_tok_off_host, const int64_t* doc_tok_off,
+                           int64_t n_docs, int32_t chunk, int32_t h_kv, int32_t d,
+                           int32_t dtype, float rope_base, void* Kbar, void* Vbar,
+                           void* Kbar_r, float* kr_inv_norm, int64_t* doc_chunk_off,
+                           int64_t n_chunks, void* stream);
+
+/* msa_kr_inv_norm - inverse L2 norms of a pre-pooled router-key bank (bank preparation for
+ * banks that were not produced by msa_encode_pool): out[c,h] = 1/||Kbar_r[c,h,:]|| (0 for a
+ * zero row), fp32 [n_chunks, h_kv]. */
+msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                           int32_t dtype, float* kr_inv_norm, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * msa_route_topk - online routing: cosine scoring of every chunk and exact top-k documents.
+ *   [news.neo-ai.one, "アーキテクチャ": the routing projector computes relevance by cosine
+ *    similarity (mean over attention heads, then max over tokens) and selects the Top-k
+ *    documents; github-eval-reports, "核心模块 / 路由投影器"; ruixiangma blog, "Top-k检索"]
+ *
+ * Q_r        [B, T, h_qr, d] router queries (dtype). Router head h uses router-key head
+ *            floor(h / (h_qr / h_kv)).
+ * Kbar_r     [n_chunks, h_kv, d] router-key bank (dtype), 16-byte aligned.
+ * kr_inv_norm [n_chunks, h_kv] fp32 inverse norms (from msa_encode_pool / msa_kr_inv_norm).
+ * doc_chunk_off [n_docs+1] device int64 chunk offsets (non-decreasing, ends at n_chunks).
+ * Score of doc i for query b:
+ *     S[b,i] = max_{c in doc i} max_t (1/h_qr) sum_h cos(Q_r[b,t,h], Kbar_r[c, g(h)])
+ *   (cosine of a zero vector = 0; a document without chunks scores -inf).
+ * exclude_bits (nullable) [B, ceil(n_docs/32)] uint32: bit i set = doc i is not eligible.
+ * top_ids    [B, k] int32 output: the k eligible docs with the largest S[b,.], score
+ *            descending, ties to the lower doc id (-0.0 ranks as +0.0); -1 when fewer than k
+ *            docs are eligible.
+ * top_scores [B, k] fp32 output (S of the selected docs; -inf in unused slots).
+ * doc_scores (nullable) [B, n_docs] fp32 output: every S[b,i] (for tests).
+ * Requires 1 <= k <= min(32, n_docs) and T <= 16 on the CUDA-core scan (B*T rows are
+ * processed in passes of up to 16 rows).
+ * ws         workspace of msa_route_topk_workspace(...) bytes; its first word is a device
+ *            status (see msa_workspace_status).
+ */
+size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv, int32_t d,
+                                int32_t dtype, int64_t n_docs, int64_t n_chunks, int32_t k);
+msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
+                          const void* Kbar_r, const float* kr_inv_norm,
+                          const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks,
+                          int32_t h_kv, int32_t d, int32_t dtype, int32_t k,
+                          const uint32_t* exclude_bits, int32_t* top_ids, float* top_scores,
+                          float* doc_scores, void* ws, size_t ws_bytes, void* stream);
+
+/* Read the device status word of a workspace (synchronises `stream`): *code = 0 if the
+ * kernels that used it recorded no error. Returns MSA_ERR_DEVICE if *code != 0. */
+msa_status msa_workspace_status(const void* ws, int32_t* code, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * msa_gather - context assembly from a bank the GPU can address (HBM, or pinned host memory
+ * reached directly over the host link).
+ *   [news.neo-ai.one, "推論パイプライン": only the selected K̄/V̄ are loaded and concatenated
+ *    with the local context]
+ *
+ * top_ids    [B, k] int32 (distinct ids; -1 entries are skipped).
+ * Context rows of query b: the selected docs in ascending doc id, each doc's chunks in
+ * order. gather_idx [B, max_ctx] int32 output: bank chunk row of each context row, -1
+ * past ctx_len[b]; ctx_len [B] int32 output.
+ * ctxK, ctxV [B, max_ctx, h_kv, d] outputs (dtype): copies of Kbar/Vbar rows; rows past
+ *            ctx_len[b] are not written.
+ * A context longer than max_ctx is truncated to max_ctx and flagged in the status word of
+ * `ws` (MSA_ERR_DEVICE via msa_workspace_status); ws must hold 256 bytes.
+ */
+msa_status msa_gather(const int32_t* top_ids, int32_t B, int32_t k,
+                      const int64_t* doc_chunk_off, int64_t n_docs, const void* Kbar,
+                      const void* Vbar, int32_t h_kv, int32_t d, int32_t dtype, int32_t max_ctx,
+                      int32_t* gather_idx, int32_t* ctx_len, void* ctxK, void* ctxV, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Asynchronous fetch from a bank in pinned host memory (tiered storage: router keys on the
+ * GPU, content K̄/V̄ in host DRAM, fetched on demand when selected).
+ *   [ruixiangma blog, "Memory Parallel / 分层内存存储"; news.neo-ai.one, "推論パイプライン"]
+ *
+ * msa_fetch_create allocates a context holding a pinned staging area for max_B*max_k ids
+ * and two CUDA events (set-up time, not the hot path); msa_fetch_destroy frees it.
+ * msa_fetch_begin enqueues on `stream`: the device gather indices (as msa_gather) and a
+ *   device-to-host copy of top_ids into the staging area, then records an event. It does
+ *   not wait.
+ * msa_fetch_finish waits on the host (polling, at most timeout_ms milliseconds; 0 = check
+ *   once) for that event, then issues one cudaMemcpyAsync per run of consecutive selected
+ *   chunks for K̄ and for V̄ from the host bank into ctxK/ctxV on `copy_stream`, records an
+ *   event there and makes `stream` wait for it. Kbar_host/Vbar_host are
+ *   [n_chunks, h_kv, d] pinned host arrays; doc_chunk_off_host is the host copy of the
+ *   chunk offsets. Returns MSA_ERR_TIMEOUT (nothing copied) if the ids are not ready in
+ *   time; the context stays usable.
+ */
+typedef struct msa_fetch msa_fetch;
+msa_status msa_fetch_create(int32_t max_B, int32_t max_k, msa_fetch** out);
+void msa_fetch_destroy(msa_fetch* f);
+msa_status msa_fetch_begin(msa_fetch* f, const int32_t* top_ids, int32_t B, int32_t k,
+                           const int64_t* doc_chunk_off, int64_t n_docs, int32_t max_ctx,
+                           int32_t* gather_idx, int32_t* ctx_len, void* ws, size_t ws_bytes,
+                           void* stream);
+msa_status msa_fetch_finish(msa_fetch* f, const int64_t* doc_chunk_off_host, int64_t n_docs,
+                            const void* Kbar_host, const void* Vbar_host, int32_t h_kv,
+                            int32_t d, int32_t dtype, int32_t max_ctx, void* ctxK, void* ctxV,
+                            void* stream, void* copy_stream, int32_t timeout_ms);
+
+/* ------------------------------------------------------------------------------------
+ * msa_sparse_attend - GQA softmax attention over [gathered memory ; causal local context]
+ * with global RoPE on the active context.
+ *   [news.neo-ai.one, "グローバル RoPE（アクティブコンテキスト）": the query's start index
+ *    is shifted by k (the number of Top-k retrieved blocks) to keep the causal order
+ *    background -> query -> generation; "推論パイプライン": sparse generation over the
+ *    assembled context]
+ *
+ * Q          [B, T, h_q, d]; query token t is local row L_loc - T + t.
+ * K_loc, V_loc [B, L_loc, h_kv, d]; K_loc before RoPE. Requires 1 <= T <= L_loc.
+ * ctxK, ctxV [B, max_ctx, h_kv, d] gathered memory rows; the first ctx_len[b] are used.
+ * Q and K_loc rows are rotated at position pos0 + (local row index) (pos0 = k); memory rows
+ * are used as stored. Query head h reads KV head floor(h / (h_q / h_kv)).
+ * O[b,t,h] = softmax over {memory rows j < ctx_len[b]} U {local rows j <= L_loc - T + t} of
+ *            scale * q.k, applied to the matching V rows; scale <= 0 means 1/sqrt(d).
+ * O          [B, T, h_q, d] output (dtype), fp32 accumulation and softmax.
+ * ws         msa_sparse_attend_workspace(...) bytes (split partials + the RoPE table).
+ */
+size_t msa_sparse_attend_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv, int32_t d,
+                                   int32_t max_ctx, int32_t L_loc);
+msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
+                             const void* K_loc, const void* V_loc, int32_t L_loc,
+                             const void* ctxK, const void* ctxV, const int32_t* ctx_len,
+                             int32_t max_ctx, int32_t h_kv, int32_t d, int32_t dtype,
+                             int32_t pos0, float rope_base, float scale, void* O, void* ws,
+                             size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H */

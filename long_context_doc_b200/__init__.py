@@ -1,0 +1,290 @@
+"""Python binding of libmsa, the B200 (sm_100a) routed-memory hot path of Memory Sparse
+Attention (MSA).
+
+The ``msa_*`` functions mirror the C ABI of ``include/msa.h`` one to one: they marshal
+torch tensors (device memory) into pointers and sizes and raise :class:`MSAError` when the
+library returns a non-zero status. Every step of the path runs in the library's CUDA
+kernels; torch only provides device memory and streams. There is no fallback: if
+``libmsa.so`` is missing or fails to load, importing this package raises.
+
+The lower-case helpers (``encode_pool``, ``route_topk``, ``gather``, ``sparse_attend``,
+``Fetcher``) allocate outputs and workspaces with torch and call the ``msa_*`` functions.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+MSA_FP32, MSA_BF16 = 0, 1
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_WORKSPACE",
+          4: "MSA_ERR_CUDA", 5: "MSA_ERR_TIMEOUT", 6: "MSA_ERR_DEVICE"}
+LIB_PATH = _build.LIB
+
+# every symbol include/msa.h declares
+SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chunks",
+           "msa_encode_pool", "msa_kr_inv_norm", "msa_route_topk_workspace", "msa_route_topk",
+           "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
+           "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
+           "msa_sparse_attend")
+
+
+class MSAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+        self.message = message
+
+
+def _load():
+    if not os.path.exists(LIB_PATH) or _build.stale():
+        _build.build()
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    L.msa_status_string.restype = ctypes.c_char_p
+    L.msa_status_string.argtypes = [ctypes.c_int]
+    L.msa_last_error.restype = ctypes.c_char_p
+    L.msa_last_error.argtypes = []
+    L.msa_version.restype = ctypes.c_int
+    L.msa_count_chunks.restype = i64
+    L.msa_count_chunks.argtypes = [vp, i64, i32]
+    L.msa_encode_pool.restype = ctypes.c_int
+    L.msa_encode_pool.argtypes = [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, f32, vp, vp,
+                                  vp, vp, vp, i64, vp]
+    L.msa_kr_inv_norm.restype = ctypes.c_int
+    L.msa_kr_inv_norm.argtypes = [vp, i64, i32, i32, i32, vp, vp]
+    L.msa_route_topk_workspace.restype = sz
+    L.msa_route_topk_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i64, i64, i32]
+    L.msa_route_topk.restype = ctypes.c_int
+    L.msa_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp,
+                                 vp, vp, vp, vp, sz, vp]
+    L.msa_workspace_status.restype = ctypes.c_int
+    L.msa_workspace_status.argtypes = [vp, vp, vp]
+    L.msa_gather.restype = ctypes.c_int
+    L.msa_gather.argtypes = [vp, i32, i32, vp, i64, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp,
+                             vp, sz, vp]
+    L.msa_fetch_create.restype = ctypes.c_int
+    L.msa_fetch_create.argtypes = [i32, i32, vp]
+    L.msa_fetch_destroy.restype = None
+    L.msa_fetch_destroy.argtypes = [vp]
+    L.msa_fetch_begin.restype = ctypes.c_int
+    L.msa_fetch_begin.argtypes = [vp, vp, i32, i32, vp, i64, i32, vp, vp, vp, sz, vp]
+    L.msa_fetch_finish.restype = ctypes.c_int
+    L.msa_fetch_finish.argtypes = [vp, vp, i64, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, i32]
+    L.msa_sparse_attend_workspace.restype = sz
+    L.msa_sparse_attend_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    L.msa_sparse_attend.restype = ctypes.c_int
+    L.msa_sparse_attend.argtypes = [vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32,
+                                    i32, f32, f32, vp, vp, sz, vp]
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int):
+    if status != 0:
+        raise MSAError(status, lib.msa_last_error().decode(errors="replace"))
+
+
+def _p(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _s(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MSA_FP32
+    if t.dtype == torch.bfloat16:
+        return MSA_BF16
+    raise TypeError(f"libmsa tensors are float32 or bfloat16, got {t.dtype}")
+
+
+# ----------------------------------------------------------------------------- raw ABI
+def msa_count_chunks(doc_tok_off_host: np.ndarray, chunk: int) -> int:
+    off = np.ascontiguousarray(doc_tok_off_host, dtype=np.int64)
+    return int(lib.msa_count_chunks(off.ctypes.data, len(off) - 1, chunk))
+
+
+def msa_encode_pool(K, V, K_r, doc_tok_off_host, doc_tok_off, chunk, rope_base, Kbar, Vbar,
+                    Kbar_r, kr_inv_norm, doc_chunk_off, stream=None):
+    off = np.ascontiguousarray(doc_tok_off_host, dtype=np.int64)
+    _check(lib.msa_encode_pool(_p(K), _p(V), _p(K_r), K.shape[0], off.ctypes.data,
+                               _p(doc_tok_off), len(off) - 1, chunk, K.shape[1], K.shape[2],
+                               dtype_code(K), rope_base, _p(Kbar), _p(Vbar), _p(Kbar_r),
+                               _p(kr_inv_norm), _p(doc_chunk_off), Kbar.shape[0], _s(stream)))
+
+
+def msa_kr_inv_norm(Kbar_r, out, stream=None):
+    n, h_kv, d = Kbar_r.shape
+    _check(lib.msa_kr_inv_norm(_p(Kbar_r), n, h_kv, d, dtype_code(Kbar_r), _p(out), _s(stream)))
+
+
+def msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k) -> int:
+    return int(lib.msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k))
+
+
+def msa_route_topk(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_bits, top_ids, top_scores,
+                   doc_scores, ws, stream=None):
+    B, T, h_qr, d = Q_r.shape
+    n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
+    _check(lib.msa_route_topk(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm), _p(doc_chunk_off),
+                              doc_chunk_off.shape[0] - 1, n_chunks, h_kv, d, dtype_code(Kbar_r), k,
+                              _p(exclude_bits), _p(top_ids), _p(top_scores), _p(doc_scores),
+                              _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_workspace_status(ws, stream=None) -> int:
+    code = ctypes.c_int32(0)
+    st = lib.msa_workspace_status(_p(ws), ctypes.addressof(code), _s(stream))
+    if st not in (0, 6):
+        _check(st)
+    return int(code.value)
+
+
+def msa_gather(top_ids, doc_chunk_off, Kbar, Vbar, max_ctx, gather_idx, ctx_len, ctxK, ctxV, ws,
+               stream=None):
+    B, k = top_ids.shape
+    _check(lib.msa_gather(_p(top_ids), B, k, _p(doc_chunk_off), doc_chunk_off.shape[0] - 1,
+                          _p(Kbar), _p(Vbar), Kbar.shape[1], Kbar.shape[2], dtype_code(Kbar),
+                          max_ctx, _p(gather_idx), _p(ctx_len), _p(ctxK), _p(ctxV), _p(ws),
+                          ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_sparse_attend_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc) -> int:
+    return int(lib.msa_sparse_attend_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc))
+
+
+def msa_sparse_attend(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0, rope_base, scale, O, ws,
+                      stream=None):
+    B, T, h_q, d = Q.shape
+    L_loc, h_kv = K_loc.shape[1], K_loc.shape[2]
+    max_ctx = ctxK.shape[1]
+    _check(lib.msa_sparse_attend(_p(Q), B, T, h_q, _p(K_loc), _p(V_loc), L_loc, _p(ctxK), _p(ctxV),
+                                 _p(ctx_len), max_ctx, h_kv, d, dtype_code(Q), pos0, rope_base,
+                                 scale, _p(O), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+# ----------------------------------------------------------------------------- helpers
+def _ws(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def encode_pool(K, V, K_r, doc_tok_off_host, chunk: int, rope_base: float, stream=None):
+    """Doc-wise RoPE + chunk pooling. Returns dict(Kbar, Vbar, Kbar_r, kr_inv_norm,
+    doc_chunk_off)."""
+    dev = K.device
+    off = np.ascontiguousarray(doc_tok_off_host, dtype=np.int64)
+    n_chunks = msa_count_chunks(off, chunk)
+    if n_chunks < 0:
+        raise MSAError(1, "invalid document offsets")
+    n, h_kv, d = K.shape
+    out = dict(Kbar=torch.empty((n_chunks, h_kv, d), dtype=K.dtype, device=dev),
+               Vbar=torch.empty((n_chunks, h_kv, d), dtype=K.dtype, device=dev),
+               Kbar_r=torch.empty((n_chunks, h_kv, d), dtype=K.dtype, device=dev),
+               kr_inv_norm=torch.empty((n_chunks, h_kv), dtype=torch.float32, device=dev),
+               doc_chunk_off=torch.empty(len(off), dtype=torch.int64, device=dev))
+    tok_off = torch.from_numpy(off).to(dev)
+    msa_encode_pool(K, V, K_r, off, tok_off, chunk, rope_base, out["Kbar"], out["Vbar"],
+                    out["Kbar_r"], out["kr_inv_norm"], out["doc_chunk_off"], stream)
+    return out
+
+
+def kr_inv_norm(Kbar_r, stream=None):
+    out = torch.empty(Kbar_r.shape[:2], dtype=torch.float32, device=Kbar_r.device)
+    msa_kr_inv_norm(Kbar_r, out, stream)
+    return out
+
+
+def route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k: int, exclude_bits=None,
+               doc_scores: bool = False, ws=None, stream=None):
+    """Returns (top_ids int32 [B,k], top_scores f32 [B,k], doc_scores f32 [B,n_docs] or None)."""
+    B, T, h_qr, d = Q_r.shape
+    n_chunks, h_kv = Kbar_r.shape[:2]
+    n_docs = doc_chunk_off.shape[0] - 1
+    dev = Q_r.device
+    if ws is None:
+        ws = _ws(msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype_code(Kbar_r), n_docs,
+                                          n_chunks, k), dev)
+    ids = torch.empty((B, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, k), dtype=torch.float32, device=dev)
+    ds = torch.empty((B, n_docs), dtype=torch.float32, device=dev) if doc_scores else None
+    msa_route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k, exclude_bits, ids, sc, ds, ws, stream)
+    return ids, sc, ds
+
+
+def gather(top_ids, doc_chunk_off, Kbar, Vbar, max_ctx: int, ws=None, stream=None):
+    """Returns (gather_idx [B,max_ctx], ctx_len [B], ctxK, ctxV [B,max_ctx,h_kv,d])."""
+    B = top_ids.shape[0]
+    dev = top_ids.device
+    h_kv, d = Kbar.shape[1], Kbar.shape[2]
+    gi = torch.empty((B, max_ctx), dtype=torch.int32, device=dev)
+    cl = torch.empty(B, dtype=torch.int32, device=dev)
+    cK = torch.empty((B, max_ctx, h_kv, d), dtype=Kbar.dtype, device=dev)
+    cV = torch.empty_like(cK)
+    if ws is None:
+        ws = _ws(256, dev)
+    msa_gather(top_ids, doc_chunk_off, Kbar, Vbar, max_ctx, gi, cl, cK, cV, ws, stream)
+    return gi, cl, cK, cV
+
+
+def sparse_attend(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0: int, rope_base: float,
+                  scale: float = 0.0, ws=None, stream=None):
+    B, T, h_q, d = Q.shape
+    if ws is None:
+        ws = _ws(msa_sparse_attend_workspace(B, T, h_q, K_loc.shape[2], d, ctxK.shape[1],
+                                             K_loc.shape[1]), Q.device)
+    O = torch.empty_like(Q)
+    msa_sparse_attend(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0, rope_base, scale, O, ws, stream)
+    return O
+
+
+class Fetcher:
+    """msa_fetch context: asynchronous fetch of selected K̄/V̄ from a pinned host bank."""
+
+    def __init__(self, max_B: int, max_k: int):
+        h = ctypes.c_void_p()
+        _check(lib.msa_fetch_create(max_B, max_k, ctypes.addressof(h)))
+        self.h = h
+        self.ws = None
+
+    def begin(self, top_ids, doc_chunk_off, max_ctx, gather_idx, ctx_len, ws, stream=None):
+        B, k = top_ids.shape
+        _check(lib.msa_fetch_begin(self.h, _p(top_ids), B, k, _p(doc_chunk_off),
+                                   doc_chunk_off.shape[0] - 1, max_ctx, _p(gather_idx),
+                                   _p(ctx_len), _p(ws), ws.numel() * ws.element_size(),
+                                   _s(stream)))
+
+    def finish(self, doc_chunk_off_host: np.ndarray, Kbar_host, Vbar_host, max_ctx, ctxK, ctxV,
+               stream=None, copy_stream=None, timeout_ms: int = 10000):
+        off = doc_chunk_off_host
+        h_kv, d = Kbar_host.shape[1], Kbar_host.shape[2]
+        _check(lib.msa_fetch_finish(self.h, off.ctypes.data, len(off) - 1, _p(Kbar_host),
+                                    _p(Vbar_host), h_kv, d, dtype_code(Kbar_host), max_ctx,
+                                    _p(ctxK), _p(ctxV), _s(stream), _s(copy_stream), timeout_ms))
+
+    def close(self):
+        if self.h:
+            lib.msa_fetch_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,472 @@
+// api.cu - the extern "C" boundary of libmsa (declared in include/msa.h): argument
+// validation, workspace sizing and kernel launches. No device memory is allocated here; the
+// only allocation is the pinned staging area of an msa_fetch context, made at set-up time.
+#include <algorithm>
+#include <cstdarg>
+#include <chrono>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "../../include/msa.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+msa_status fail(msa_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+msa_status fail(msa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+msa_status ok() {
+  g_err.clear();
+  return MSA_OK;
+}
+
+msa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(MSA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+    return 148;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+size_t esize(int dtype) { return dtype == MSA_BF16 ? 2 : 4; }
+
+constexpr size_t kHeader = 256;   // workspace header: [0] status word, [1..63] counters
+constexpr int kMaxPasses = 63;
+
+#define REQUIRE(cond, status, ...) \
+  do {                             \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+msa_status check_common(int32_t h_kv, int32_t d, int32_t dtype) {
+  REQUIRE(dtype == MSA_FP32 || dtype == MSA_BF16, MSA_ERR_UNSUPPORTED, "dtype %d", dtype);
+  REQUIRE(d == 64 || d == 128, MSA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+  REQUIRE(h_kv >= 1, MSA_ERR_INVALID_ARG, "h_kv %d", h_kv);
+  return MSA_OK;
+}
+
+// route pass geometry: queries per pass and number of passes
+void route_passes(int B, int T, int* bp, int* passes) {
+  int per = std::max(1, 16 / std::max(T, 1));
+  per = std::min(per, std::max(B, 1));
+  int np = (B + per - 1) / per;
+  per = (B + np - 1) / std::max(np, 1);
+  *bp = std::max(per, 1);
+  *passes = np;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* msa_status_string(int s) {
+  switch (s) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+    case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+    case MSA_ERR_TIMEOUT: return "MSA_ERR_TIMEOUT";
+    case MSA_ERR_DEVICE: return "MSA_ERR_DEVICE";
+    default: return "MSA_ERR_UNKNOWN";
+  }
+}
+
+const char* msa_last_error(void) { return g_err.c_str(); }
+
+int msa_version(void) { return (1 << 16) | 0; }
+
+int64_t msa_count_chunks(const int64_t* off, int64_t n_docs, int32_t chunk) {
+  if (off == nullptr || n_docs < 0 || chunk < 1) return -1;
+  if (off[0] != 0) return -1;
+  int64_t n = 0;
+  for (int64_t i = 0; i < n_docs; ++i) {
+    const int64_t len = off[i + 1] - off[i];
+    if (len < 0) return -1;
+    n += (len + chunk - 1) / chunk;
+  }
+  return n;
+}
+
+msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_t n_tok,
+                           const int64_t* doc_tok_off_host, const int64_t* doc_tok_off,
+                           int64_t n_docs, int32_t chunk, int32_t h_kv, int32_t d,
+                           int32_t dtype, float rope_base, void* Kbar, void* Vbar,
+                           void* Kbar_r, float* kr_inv_norm, int64_t* doc_chunk_off,
+                           int64_t n_chunks, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(n_docs >= 0 && n_tok >= 0 && n_chunks >= 0, MSA_ERR_INVALID_ARG, "negative size");
+  REQUIRE(chunk >= 1, MSA_ERR_INVALID_ARG, "chunk %d", chunk);
+  REQUIRE(doc_tok_off_host && doc_tok_off && doc_chunk_off, MSA_ERR_INVALID_ARG,
+          "null offset pointer");
+  REQUIRE(doc_tok_off_host[n_docs] == n_tok, MSA_ERR_INVALID_ARG,
+          "doc_tok_off[n_docs] = %lld != n_tok %lld", (long long)doc_tok_off_host[n_docs],
+          (long long)n_tok);
+  const int64_t nc = msa_count_chunks(doc_tok_off_host, n_docs, chunk);
+  REQUIRE(nc >= 0, MSA_ERR_INVALID_ARG, "doc_tok_off must start at 0 and not decrease");
+  REQUIRE(nc == n_chunks, MSA_ERR_INVALID_ARG, "n_chunks %lld != %lld implied by the offsets",
+          (long long)n_chunks, (long long)nc);
+  const int E = dtype == MSA_BF16 ? 8 : 4;
+  REQUIRE(pow2(h_kv) && h_kv * (d / 2) / E <= 256, MSA_ERR_UNSUPPORTED,
+          "encode needs h_kv a power of two with h_kv*d/2/%d <= 256 (h_kv=%d)", E, h_kv);
+  if (n_chunks > 0) {
+    REQUIRE(K && V && K_r && Kbar && Vbar && Kbar_r, MSA_ERR_INVALID_ARG, "null tensor");
+    REQUIRE(aligned16(K) && aligned16(V) && aligned16(K_r) && aligned16(Kbar) &&
+                aligned16(Vbar) && aligned16(Kbar_r),
+            MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  }
+  msa::EncodeParams p{K, V, K_r, doc_tok_off, doc_chunk_off, n_docs, n_chunks, chunk, h_kv,
+                      (double)rope_base, Kbar, Vbar, Kbar_r, kr_inv_norm};
+  cudaError_t e = msa::launch_encode_pool(p, dtype, d, sm_count(), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_encode_pool launch");
+  return ok();
+}
+
+msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                           int32_t dtype, float* out, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(n_chunks >= 0, MSA_ERR_INVALID_ARG, "negative n_chunks");
+  REQUIRE(n_chunks == 0 || (Kbar_r && out), MSA_ERR_INVALID_ARG, "null tensor");
+  cudaError_t e = msa::launch_inv_norm(Kbar_r, n_chunks, h_kv, d, dtype, out, sm_count(),
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_kr_inv_norm launch");
+  return ok();
+}
+
+size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv, int32_t d,
+                                int32_t dtype, int64_t n_docs, int64_t n_chunks, int32_t k) {
+  (void)h_qr;
+  (void)n_docs;
+  if (B < 1 || T < 1 || k < 1 || h_kv < 1 || d < 1) return kHeader;
+  int bp, passes;
+  route_passes(B, T, &bp, &passes);
+  const msa::RouteChoice c = msa::route_choose(dtype, bp * T, h_kv * d);
+  if (c.R == 0) return kHeader;
+  const int grid = msa::route_grid(dtype, c, h_kv * d, sm_count(), n_chunks);
+  if (grid < 1) return kHeader;
+  return kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
+}
+
+msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
+                          const void* Kbar_r, const float* kr_inv_norm,
+                          const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks,
+                          int32_t h_kv, int32_t d, int32_t dtype, int32_t k,
+                          const uint32_t* exclude_bits, int32_t* top_ids, float* top_scores,
+                          float* doc_scores, void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && T >= 1 && n_docs >= 1 && n_chunks >= 0, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d T=%d n_docs=%lld n_chunks=%lld)", B, T, (long long)n_docs,
+          (long long)n_chunks);
+  REQUIRE(h_qr >= 1 && h_qr % h_kv == 0, MSA_ERR_INVALID_ARG, "h_qr %d not a multiple of h_kv %d",
+          h_qr, h_kv);
+  REQUIRE(k >= 1 && k <= n_docs, MSA_ERR_INVALID_ARG, "k %d outside [1, n_docs=%lld]", k,
+          (long long)n_docs);
+  REQUIRE(k <= 32, MSA_ERR_UNSUPPORTED, "k %d > 32", k);
+  REQUIRE(T <= 16, MSA_ERR_UNSUPPORTED, "query length T=%d > 16 needs the tensor-core scan", T);
+  if (B == 0) return ok();
+  REQUIRE(Q_r && Kbar_r && kr_inv_norm && doc_chunk_off && top_ids && top_scores,
+          MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(aligned16(Kbar_r), MSA_ERR_INVALID_ARG, "Kbar_r must be 16-byte aligned");
+  int bp, passes;
+  route_passes(B, T, &bp, &passes);
+  REQUIRE(passes <= kMaxPasses, MSA_ERR_UNSUPPORTED, "B=%d needs %d passes (> %d)", B, passes,
+          kMaxPasses);
+  const int W = h_kv * d;
+  const msa::RouteChoice c = msa::route_choose(dtype, bp * T, W);
+  REQUIRE(c.R != 0, MSA_ERR_UNSUPPORTED, "router key row h_kv*d=%d not supported", W);
+  const int grid = msa::route_grid(dtype, c, W, sm_count(), n_chunks);
+  REQUIRE(grid >= 1, MSA_ERR_CUDA, "occupancy query failed");
+  const size_t need = kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
+  REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu (256-byte aligned)", ws_bytes,
+          ws, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeader, st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace header reset");
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  const int64_t words = (n_docs + 31) / 32;
+  const size_t qstride = (size_t)T * h_qr * d * esize(dtype);
+  for (int pass = 0; pass < passes; ++pass) {
+    const int b0 = pass * bp;
+    const int nb = std::min(bp, B - b0);
+    if (nb <= 0) break;
+    msa::RouteParams p{};
+    p.qr = static_cast<const unsigned char*>(Q_r) + (size_t)b0 * qstride;
+    p.kr = Kbar_r;
+    p.invk = kr_inv_norm;
+    p.coff = doc_chunk_off;
+    p.excl = exclude_bits ? exclude_bits + (size_t)b0 * words : nullptr;
+    p.n_docs = n_docs;
+    p.n_chunks = n_chunks;
+    p.words = words;
+    p.B = nb;
+    p.T = T;
+    p.h_qr = h_qr;
+    p.h_kv = h_kv;
+    p.d = d;
+    p.k = k;
+    p.top_ids = top_ids + (size_t)b0 * k;
+    p.top_scores = top_scores + (size_t)b0 * k;
+    p.doc_scores = doc_scores ? doc_scores + (size_t)b0 * n_docs : nullptr;
+    p.cand = reinterpret_cast<unsigned long long*>(base + kHeader) + (size_t)pass * grid * bp * k;
+    p.counter = reinterpret_cast<unsigned int*>(base) + 1 + pass;
+    p.err = reinterpret_cast<int*>(base);
+    e = msa::route_launch(dtype, c, p, grid, st);
+    if (e != cudaSuccess) return cuda_fail(e, "msa_route_topk launch");
+  }
+  return ok();
+}
+
+msa_status msa_workspace_status(const void* ws, int32_t* code, void* stream) {
+  REQUIRE(ws && code, MSA_ERR_INVALID_ARG, "null pointer");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_workspace_status");
+  *code = v;
+  if (v != 0) return fail(MSA_ERR_DEVICE, "device status %d recorded in the workspace", v);
+  return ok();
+}
+
+msa_status msa_gather(const int32_t* top_ids, int32_t B, int32_t k,
+                      const int64_t* doc_chunk_off, int64_t n_docs, const void* Kbar,
+                      const void* Vbar, int32_t h_kv, int32_t d, int32_t dtype, int32_t max_ctx,
+                      int32_t* gather_idx, int32_t* ctx_len, void* ctxK, void* ctxV, void* ws,
+                      size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && k >= 1 && k <= 32 && max_ctx >= 0 && n_docs >= 1, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d k=%d max_ctx=%d)", B, k, max_ctx);
+  REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "gather needs a 256-byte aligned workspace of >= 256 bytes");
+  if (B == 0) return ok();
+  REQUIRE(top_ids && doc_chunk_off && gather_idx && ctx_len && Kbar && Vbar && ctxK && ctxV,
+          MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(aligned16(Kbar) && aligned16(Vbar) && aligned16(ctxK) && aligned16(ctxV),
+          MSA_ERR_INVALID_ARG, "bank and context must be 16-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  msa::GatherParams p{top_ids, doc_chunk_off, n_docs, B, k, max_ctx,
+                      (int64_t)h_kv * d * (int64_t)esize(dtype), Kbar, Vbar, gather_idx,
+                      ctx_len, ctxK, ctxV, static_cast<int*>(ws)};
+  e = msa::launch_gather(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_gather launch");
+  return ok();
+}
+
+// ----------------------------------------------------------------------------- host fetch
+struct msa_fetch {
+  int32_t max_B = 0, max_k = 0;
+  int32_t* ids_host = nullptr;  // pinned
+  cudaEvent_t ids_ready = nullptr, copy_done = nullptr;
+  int32_t B = 0, k = 0;
+  bool pending = false;
+};
+
+msa_status msa_fetch_create(int32_t max_B, int32_t max_k, msa_fetch** out) {
+  REQUIRE(out && max_B >= 1 && max_k >= 1 && max_k <= 32, MSA_ERR_INVALID_ARG,
+          "bad fetch context sizes");
+  msa_fetch* f = new msa_fetch();
+  f->max_B = max_B;
+  f->max_k = max_k;
+  cudaError_t e = cudaHostAlloc(&f->ids_host, (size_t)max_B * max_k * sizeof(int32_t),
+                                cudaHostAllocDefault);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f->ids_ready, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f->copy_done, cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    msa_fetch_destroy(f);
+    return cuda_fail(e, "msa_fetch_create");
+  }
+  *out = f;
+  return ok();
+}
+
+void msa_fetch_destroy(msa_fetch* f) {
+  if (!f) return;
+  if (f->ids_host) cudaFreeHost(f->ids_host);
+  if (f->ids_ready) cudaEventDestroy(f->ids_ready);
+  if (f->copy_done) cudaEventDestroy(f->copy_done);
+  delete f;
+}
+
+msa_status msa_fetch_begin(msa_fetch* f, const int32_t* top_ids, int32_t B, int32_t k,
+                           const int64_t* doc_chunk_off, int64_t n_docs, int32_t max_ctx,
+                           int32_t* gather_idx, int32_t* ctx_len, void* ws, size_t ws_bytes,
+                           void* stream) {
+  REQUIRE(f, MSA_ERR_INVALID_ARG, "null fetch context");
+  REQUIRE(B >= 1 && B <= f->max_B && k >= 1 && k <= f->max_k && max_ctx >= 0 && n_docs >= 1,
+          MSA_ERR_INVALID_ARG, "B=%d k=%d outside the context's %d x %d", B, k, f->max_B,
+          f->max_k);
+  REQUIRE(top_ids && doc_chunk_off && gather_idx && ctx_len, MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "fetch needs a 256-byte aligned workspace of >= 256 bytes");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+  msa::GatherParams p{top_ids, doc_chunk_off, n_docs, B, k, max_ctx, 16, nullptr, nullptr,
+                      gather_idx, ctx_len, nullptr, nullptr, static_cast<int*>(ws)};
+  e = msa::launch_gather(p, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(f->ids_host, top_ids, (size_t)B * k * sizeof(int32_t),
+                        cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaEventRecord(f->ids_ready, st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_fetch_begin");
+  f->B = B;
+  f->k = k;
+  f->pending = true;
+  return ok();
+}
+
+msa_status msa_fetch_finish(msa_fetch* f, const int64_t* coff, int64_t n_docs,
+                            const void* Kbar_host, const void* Vbar_host, int32_t h_kv,
+                            int32_t d, int32_t dtype, int32_t max_ctx, void* ctxK, void* ctxV,
+                            void* stream, void* copy_stream, int32_t timeout_ms) {
+  REQUIRE(f && f->pending, MSA_ERR_INVALID_ARG, "msa_fetch_finish without msa_fetch_begin");
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(coff && Kbar_host && Vbar_host && ctxK && ctxV && max_ctx >= 0, MSA_ERR_INVALID_ARG,
+          "null pointer");
+  // bounded host wait for the selected ids
+  const auto t0 = std::chrono::steady_clock::now();
+  while (true) {
+    cudaError_t q = cudaEventQuery(f->ids_ready);
+    if (q == cudaSuccess) break;
+    if (q != cudaErrorNotReady) return cuda_fail(q, "waiting for the selected ids");
+    const auto ms = std::chrono::duration_cast<std::chrono::milliseconds>(
+                        std::chrono::steady_clock::now() - t0).count();
+    if (ms >= timeout_ms)
+      return fail(MSA_ERR_TIMEOUT, "selected ids not ready after %d ms", timeout_ms);
+    std::this_thread::yield();
+  }
+  f->pending = false;
+  cudaStream_t st = (cudaStream_t)stream, cst = (cudaStream_t)copy_stream;
+  cudaError_t e = cudaStreamWaitEvent(cst, f->ids_ready, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "copy stream wait");
+  const size_t row = (size_t)h_kv * d * esize(dtype);
+  const unsigned char* hk = static_cast<const unsigned char*>(Kbar_host);
+  const unsigned char* hv = static_cast<const unsigned char*>(Vbar_host);
+  unsigned char* dk = static_cast<unsigned char*>(ctxK);
+  unsigned char* dv = static_cast<unsigned char*>(ctxV);
+  std::vector<int32_t> ids;
+  ids.reserve(f->k);
+  for (int b = 0; b < f->B; ++b) {
+    ids.clear();
+    for (int j = 0; j < f->k; ++j) {
+      const int32_t id = f->ids_host[b * f->k + j];
+      if (id >= 0 && id < n_docs) ids.push_back(id);
+    }
+    std::sort(ids.begin(), ids.end());
+    int64_t off = 0;
+    size_t q = 0;
+    while (q < ids.size() && off < max_ctx) {
+      // merge docs whose chunk ranges are adjacent in the bank into one copy
+      int64_t src = coff[ids[q]], end = coff[ids[q] + 1];
+      size_t r = q + 1;
+      while (r < ids.size() && coff[ids[r]] == end) end = coff[ids[r++] + 1];
+      int64_t n = end - src;
+      if (off + n > max_ctx) n = max_ctx - off;
+      if (n > 0) {
+        const size_t dst = ((size_t)b * max_ctx + off) * row;
+        e = cudaMemcpyAsync(dk + dst, hk + src * row, n * row, cudaMemcpyHostToDevice, cst);
+        if (e == cudaSuccess)
+          e = cudaMemcpyAsync(dv + dst, hv + src * row, n * row, cudaMemcpyHostToDevice, cst);
+        if (e != cudaSuccess) return cuda_fail(e, "host bank fetch");
+      }
+      off += n;
+      q = r;
+    }
+  }
+  e = cudaEventRecord(f->copy_done, cst);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, f->copy_done, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "fetch completion event");
+  return ok();
+}
+
+// ----------------------------------------------------------------------------- attention
+size_t msa_sparse_attend_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv, int32_t d,
+                                   int32_t max_ctx, int32_t L_loc) {
+  if (B < 1 || T < 1 || h_q < 1 || h_kv < 1 || d < 2 || max_ctx < 0 || L_loc < 1) return kHeader;
+  const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
+  return kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes;
+}
+
+msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
+                             const void* K_loc, const void* V_loc, int32_t L_loc,
+                             const void* ctxK, const void* ctxV, const int32_t* ctx_len,
+                             int32_t max_ctx, int32_t h_kv, int32_t d, int32_t dtype,
+                             int32_t pos0, float rope_base, float scale, void* O, void* ws,
+                             size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && T >= 1 && L_loc >= T && max_ctx >= 0, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d T=%d L_loc=%d max_ctx=%d)", B, T, L_loc, max_ctx);
+  REQUIRE(h_q >= h_kv && h_q % h_kv == 0, MSA_ERR_INVALID_ARG, "h_q %d not a multiple of h_kv %d",
+          h_q, h_kv);
+  REQUIRE(pos0 >= 0, MSA_ERR_INVALID_ARG, "pos0 %d", pos0);
+  if (B == 0) return ok();
+  REQUIRE(Q && K_loc && V_loc && ctx_len && O, MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(max_ctx == 0 || (ctxK && ctxV), MSA_ERR_INVALID_ARG, "null context");
+  REQUIRE(aligned16(Q) && aligned16(K_loc) && aligned16(V_loc) &&
+              (max_ctx == 0 || (aligned16(ctxK) && aligned16(ctxV))),
+          MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
+  const size_t need = kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes;
+  REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+  unsigned char* base = static_cast<unsigned char*>(ws) + kHeader;
+  msa::AttendParams p{};
+  p.Q = Q;
+  p.Kl = K_loc;
+  p.Vl = V_loc;
+  p.cK = ctxK;
+  p.cV = ctxV;
+  p.ctx_len = ctx_len;
+  p.B = B;
+  p.T = T;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.d = d;
+  p.L = L_loc;
+  p.max_ctx = max_ctx;
+  p.rope = rope_base > 0.f ? 1 : 0;
+  p.cs = reinterpret_cast<const float2*>(base);
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.S = pl.S;
+  p.KPS = pl.KPS;
+  p.RB = pl.RB;
+  p.NRB = pl.NRB;
+  p.part_o = reinterpret_cast<float*>(base + pl.cs_bytes);
+  p.part_ml = reinterpret_cast<float*>(base + pl.cs_bytes + pl.part_o_bytes);
+  p.O = O;
+  cudaError_t e = msa::launch_attend(p, dtype, (double)rope_base, pos0, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,284 @@
+// encode_pool.cu - offline memory encoding of MSA: document-wise RoPE on K and K_r fused with
+// fixed-length chunk mean pooling of K, V and K_r, plus the fp32 inverse norms of the pooled
+// router keys. One streaming pass over the per-token tensors (HBM-bound).
+//
+// Method: chunk-wise mean pooling compresses each document's K/V/K_r
+//   [news.neo-ai.one article, "全体設計 / アーキテクチャ"; ruixiangma.github.io blog
+//    "Memory-Sparse-Attention", "稀疏注意力机制 / 分块压缩"], with document-wise ("parallel")
+//   RoPE whose positions restart at 0 in every document
+//   [news.neo-ai.one, "並列（ドキュメント単位）RoPE"; ruixiangma blog, "文档级RoPE"].
+//
+// Layout: one CTA per chunk (grid-stride). A thread owns one "pair group": E consecutive
+// elements of the first half of a head and the E elements they pair with in the second half
+// (RoPE rotates element i with i + d/2), for TP-strided tokens of the chunk; TP lanes that
+// share a pair group sit next to each other in the warp and are reduced with shuffles.
+// cos/sin of the chunk's positions are computed once per CTA in double precision into a
+// shared-memory table (padded rows: conflict-free 16-byte reads).
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace msa {
+
+
+template <typename T, int E, int D, int TP>
+__global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
+  constexpr int HALF = D / 2;
+  constexpr int SUBS = HALF / E;     // pair groups per head
+  constexpr int TB = 64;             // positions per cos/sin table block
+  constexpr int ROW = HALF + 2;      // padded table row (float2 units)
+  using V = Vec<T, E>;
+  using raw = typename V::raw;
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float2* cs = reinterpret_cast<float2*>(smem_raw);                 // [TB][ROW]
+  double* theta = reinterpret_cast<double*>(cs + TB * ROW);         // [HALF]
+  float* ssp = reinterpret_cast<float*>(theta + HALF);              // [PG] partial sum sq
+
+  const int PG = p.h_kv * SUBS;
+  const int tid = threadIdx.x;
+  const int tp = tid % TP;
+  const int pg = tid / TP;
+  const bool active = pg < PG;
+  const int h = pg / SUBS;
+  const int e1 = (pg % SUBS) * E;    // first-half element offset within the head
+  const int W = p.h_kv * D;          // row length
+  const bool rope = p.rope_base > 0.0;
+
+  if (rope) {
+    for (int i = tid; i < HALF; i += blockDim.x)
+      theta[i] = pow(p.rope_base, -2.0 * (double)i / (double)D);
+  }
+
+  const T* K = static_cast<const T*>(p.K);
+  const T* Vt = static_cast<const T*>(p.V);
+  const T* Kr = static_cast<const T*>(p.Kr);
+
+  for (int64_t c = blockIdx.x; c < p.n_chunks; c += gridDim.x) {
+    // document owning chunk c: off[i] <= c < off[i+1]
+    const int64_t doc = lower_bound_i64(p.chunk_off, p.n_docs, c + 1) - 1;
+    const int64_t j = c - p.chunk_off[doc];
+    const int64_t tdoc = p.tok_off[doc];
+    const int64_t t0 = tdoc + j * p.chunk;
+    int64_t t1 = t0 + p.chunk;
+    if (t1 > p.tok_off[doc + 1]) t1 = p.tok_off[doc + 1];
+    const int n = (int)(t1 - t0);
+    const int64_t pos0 = j * p.chunk;  // position of the chunk's first token in its doc
+
+    float k1[E], k2[E], r1[E], r2[E], v1[E], v2[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) k1[e] = k2[e] = r1[e] = r2[e] = v1[e] = v2[e] = 0.f;
+
+    for (int sb = 0; sb < n; sb += TB) {
+      const int nb = min(TB, n - sb);
+      if (rope) {
+        __syncthreads();  // the previous table block is no longer read
+        for (int idx = tid; idx < nb * HALF; idx += blockDim.x) {
+          const int pl = idx / HALF, i = idx % HALF;
+          double s, co;
+          sincos((double)(pos0 + sb + pl) * theta[i], &s, &co);
+          cs[pl * ROW + i] = make_float2((float)co, (float)s);
+        }
+        __syncthreads();
+      }
+      if (active) {
+#pragma unroll 2
+        for (int tl = tp; tl < nb; tl += TP) {
+          const int64_t base = (t0 + sb + tl) * (int64_t)W + (int64_t)h * D + e1;
+          float a1[E], a2[E], b1[E], b2[E], c1[E], c2[E];
+          V::unpack(*reinterpret_cast<const raw*>(K + base), a1);
+          V::unpack(*reinterpret_cast<const raw*>(K + base + HALF), a2);
+          V::unpack(*reinterpret_cast<const raw*>(Kr + base), b1);
+          V::unpack(*reinterpret_cast<const raw*>(Kr + base + HALF), b2);
+          V::unpack(*reinterpret_cast<const raw*>(Vt + base), c1);
+          V::unpack(*reinterpret_cast<const raw*>(Vt + base + HALF), c2);
+          if (rope) {
+            const float2* row = cs + tl * ROW + e1;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              const float2 t = row[e];
+              k1[e] += a1[e] * t.x - a2[e] * t.y;
+              k2[e] += a2[e] * t.x + a1[e] * t.y;
+              r1[e] += b1[e] * t.x - b2[e] * t.y;
+              r2[e] += b2[e] * t.x + b1[e] * t.y;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              k1[e] += a1[e]; k2[e] += a2[e]; r1[e] += b1[e]; r2[e] += b2[e];
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < E; ++e) { v1[e] += c1[e]; v2[e] += c2[e]; }
+        }
+      }
+    }
+
+    // reduce over the TP lanes sharing this pair group (adjacent lanes)
+#pragma unroll
+    for (int o = TP / 2; o > 0; o >>= 1) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        k1[e] += __shfl_xor_sync(0xffffffffu, k1[e], o);
+        k2[e] += __shfl_xor_sync(0xffffffffu, k2[e], o);
+        r1[e] += __shfl_xor_sync(0xffffffffu, r1[e], o);
+        r2[e] += __shfl_xor_sync(0xffffffffu, r2[e], o);
+        v1[e] += __shfl_xor_sync(0xffffffffu, v1[e], o);
+        v2[e] += __shfl_xor_sync(0xffffffffu, v2[e], o);
+      }
+    }
+
+    if (active) {
+      const float inv_n = 1.0f / (float)n;
+      const int64_t ob = c * (int64_t)W + (int64_t)h * D + e1;
+      T* Kb = static_cast<T*>(p.Kb);
+      T* Vb = static_cast<T*>(p.Vb);
+      T* Rb = static_cast<T*>(p.Rb);
+      float ss = 0.f;
+      // every lane of the TP group holds the totals; lane tp stores vectors tp, tp+TP, ...
+#pragma unroll
+      for (int vct = 0; vct < 6; ++vct) {
+        const bool mine = (vct % TP) == tp;
+        const float* src = vct == 0 ? k1 : vct == 1 ? k2 : vct == 2 ? r1 : vct == 3 ? r2
+                         : vct == 4 ? v1 : v2;
+        T* dst = (vct < 2 ? Kb : vct < 4 ? Rb : Vb) + ob + ((vct & 1) ? HALF : 0);
+        T out[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[e] = Elem<T>::from_f(src[e] * inv_n);
+        if (mine) *reinterpret_cast<raw*>(dst) = *reinterpret_cast<const raw*>(out);
+        if (vct == 2 || vct == 3) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            const float s = Elem<T>::to_f(out[e]);
+            ss += s * s;
+          }
+        }
+      }
+      if (tp == 0) ssp[pg] = ss;
+    }
+    __syncthreads();
+    if (p.inv_norm != nullptr) {
+      for (int hh = tid; hh < p.h_kv; hh += blockDim.x) {
+        float s = 0.f;
+        for (int q = 0; q < SUBS; ++q) s += ssp[hh * SUBS + q];
+        p.inv_norm[c * p.h_kv + hh] = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Inverse norms of a pre-pooled bank: one warp per (chunk, head) row.
+template <typename T>
+__global__ void __launch_bounds__(256) inv_norm_kernel(const T* __restrict__ R, int64_t rows,
+                                                       int d, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp; r < rows; r += nw) {
+    float s = 0.f;
+    for (int e = lane; e < d; e += 32) {
+      const float x = Elem<T>::to_f(R[r * d + e]);
+      s += x * x;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) out[r] = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
+  }
+}
+
+// chunk offsets: doc_chunk_off[i+1] = sum_{j<=i} ceil(len_j / chunk). One CTA of 1024.
+__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int64_t* __restrict__ tok_off,
+                                                             int64_t n_docs, int chunk,
+                                                             int64_t* __restrict__ out) {
+  __shared__ int64_t part[1024];
+  const int tid = threadIdx.x;
+  const int64_t per = (n_docs + blockDim.x - 1) / blockDim.x;
+  const int64_t a = min(n_docs, (int64_t)tid * per), b = min(n_docs, a + per);
+  int64_t s = 0;
+  for (int64_t i = a; i < b; ++i) s += (tok_off[i + 1] - tok_off[i] + chunk - 1) / chunk;
+  part[tid] = s;
+  __syncthreads();
+  for (int o = 1; o < (int)blockDim.x; o <<= 1) {  // inclusive scan
+    const int64_t v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  int64_t run = tid ? part[tid - 1] : 0;
+  if (tid == 0) out[0] = 0;
+  for (int64_t i = a; i < b; ++i) {
+    run += (tok_off[i + 1] - tok_off[i] + chunk - 1) / chunk;
+    out[i + 1] = run;
+  }
+}
+
+// ------------------------------------------------------------------------------- launch
+template <typename T, int E, int D, int TP>
+static cudaError_t launch_encode_t(const EncodeParams& p, int sms, cudaStream_t st) {
+  constexpr int HALF = D / 2;
+  const int PG = p.h_kv * (HALF / E);
+  const size_t smem = sizeof(float2) * 64 * (HALF + 2) + sizeof(double) * HALF +
+                      sizeof(float) * PG;
+  auto kfn = encode_pool_kernel<T, E, D, TP>;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  int64_t grid = p.n_chunks;
+  const int64_t cap = (int64_t)sms * 64;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  kfn<<<(unsigned)grid, PG * TP, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int E, int D>
+static cudaError_t launch_encode_e(const EncodeParams& p, int sms, cudaStream_t st) {
+  const int PG = p.h_kv * (D / 2 / E);
+  const int tp = 256 / PG;
+  switch (tp >= 32 ? 32 : tp) {
+    case 32: return launch_encode_t<T, E, D, 32>(p, sms, st);
+    case 16: return launch_encode_t<T, E, D, 16>(p, sms, st);
+    case 8: return launch_encode_t<T, E, D, 8>(p, sms, st);
+    case 4: return launch_encode_t<T, E, D, 4>(p, sms, st);
+    case 2: return launch_encode_t<T, E, D, 2>(p, sms, st);
+    case 1: return launch_encode_t<T, E, D, 1>(p, sms, st);
+    default: return cudaErrorInvalidConfiguration;
+  }
+}
+
+// Host entry (validated by the caller): dtype 0 fp32, 1 bf16; d 64 or 128; h_kv a power of
+// two with h_kv * (d/2) / E <= 256.
+cudaError_t launch_encode_pool(const EncodeParams& p, int dtype, int d, int sms,
+                               cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  if (p.n_docs > 0) {
+    chunk_offsets_kernel<<<1, 1024, 0, st>>>(p.tok_off, p.n_docs, p.chunk,
+                                             const_cast<int64_t*>(p.chunk_off));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.n_chunks == 0) return cudaSuccess;
+  if (dtype == 1) {
+    return d == 128 ? launch_encode_e<__nv_bfloat16, 8, 128>(p, sms, st)
+                    : launch_encode_e<__nv_bfloat16, 8, 64>(p, sms, st);
+  }
+  return d == 128 ? launch_encode_e<float, 4, 128>(p, sms, st)
+                  : launch_encode_e<float, 4, 64>(p, sms, st);
+}
+
+cudaError_t launch_inv_norm(const void* R, int64_t n_chunks, int h_kv, int d, int dtype,
+                            float* out, int sms, cudaStream_t st) {
+  const int64_t rows = n_chunks * h_kv;
+  if (rows == 0) return cudaSuccess;
+  int64_t grid = (rows * 32 + 255) / 256;
+  if (grid > (int64_t)sms * 32) grid = (int64_t)sms * 32;
+  if (dtype == 1)
+    inv_norm_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(R), rows, d, out);
+  else
+    inv_norm_kernel<float><<<(unsigned)grid, 256, 0, st>>>(static_cast<const float*>(R), rows,
+                                                           d, out);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

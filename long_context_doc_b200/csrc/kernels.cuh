@@ -1,0 +1,91 @@
+// kernels.cuh - parameter blocks and launchers of the libmsa kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace msa {
+
+// ---- encode_pool.cu
+struct EncodeParams {
+  const void* K;
+  const void* V;
+  const void* Kr;
+  const int64_t* tok_off;    // [n_docs+1]
+  const int64_t* chunk_off;  // [n_docs+1] (written by the chunk-offset kernel)
+  int64_t n_docs, n_chunks;
+  int chunk, h_kv;
+  double rope_base;          // <= 0: no rotation
+  void* Kb;
+  void* Vb;
+  void* Rb;
+  float* inv_norm;           // nullable
+};
+cudaError_t launch_encode_pool(const EncodeParams& p, int dtype, int d, int sms, cudaStream_t st);
+cudaError_t launch_inv_norm(const void* R, int64_t n_chunks, int h_kv, int d, int dtype, float* out,
+                            int sms, cudaStream_t st);
+
+// ---- route.cu
+struct RouteParams {
+  const void* qr;            // [B, T, h_qr, d] of this pass
+  const void* kr;            // [n_chunks, h_kv, d]
+  const float* invk;         // [n_chunks, h_kv]
+  const int64_t* coff;       // [n_docs + 1]
+  const uint32_t* excl;      // nullable [B, words] of this pass
+  int64_t n_docs, n_chunks, words;
+  int B, T, h_qr, h_kv, d, k;
+  int32_t* top_ids;          // [B, k] of this pass
+  float* top_scores;         // [B, k]
+  float* doc_scores;         // nullable [B, n_docs]
+  unsigned long long* cand;  // [grid, B, k]
+  unsigned int* counter;
+  int* err;
+};
+struct RouteChoice { int R, E; };
+RouteChoice route_choose(int dtype, int rows, int W);
+int route_grid(int dtype, RouteChoice c, int W, int sms, int64_t n_chunks);
+cudaError_t route_launch(int dtype, RouteChoice c, const RouteParams& p, int grid, cudaStream_t st);
+
+// ---- gather.cu
+struct GatherParams {
+  const int32_t* ids;      // [B, k]
+  const int64_t* coff;     // [n_docs + 1]
+  int64_t n_docs;
+  int B, k, max_ctx;
+  int64_t row_bytes;       // h_kv * d * sizeof(T), a multiple of 16
+  const void* Kb;          // nullable: index-only mode
+  const void* Vb;
+  int32_t* gidx;           // [B, max_ctx]
+  int32_t* ctx_len;        // [B]
+  void* ctxK;
+  void* ctxV;
+  int* err;
+};
+cudaError_t launch_gather(const GatherParams& p, cudaStream_t st);
+
+// ---- attend.cu
+struct AttendParams {
+  const void* Q;        // [B, T, h_q, d]
+  const void* Kl;       // [B, L, h_kv, d]
+  const void* Vl;
+  const void* cK;       // [B, max_ctx, h_kv, d]
+  const void* cV;
+  const int32_t* ctx_len;
+  int B, T, h_q, h_kv, d, L, max_ctx;
+  int rope;             // 0: no rotation
+  const float2* cs;     // [L][d/2] cos/sin at positions pos0 + j
+  float scale_log2;     // softmax scale * log2(e)
+  int S, KPS, RB, NRB;  // splits, keys per split, rows per CTA, row blocks
+  float* part_o;        // [B*T*h_q, S, d]
+  float* part_ml;       // [B*T*h_q, S, 2]
+  void* O;              // [B, T, h_q, d]
+};
+struct AttendPlan {
+  int RB, NRB, KPS, S;
+  size_t cs_bytes, part_o_bytes, part_ml_bytes;
+};
+AttendPlan attend_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
+cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0, cudaStream_t st);
+
+}  // namespace msa

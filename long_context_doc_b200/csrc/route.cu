@@ -1,0 +1,429 @@
+// route.cu - online routing of MSA: cosine scoring of every chunk of the router-key bank
+// against the router queries, document scores, and an exact top-k, in ONE kernel launch.
+//
+// Method: the router query Q_r is compared with every chunk's pooled router key K̄_r by
+// cosine similarity; the similarities are averaged over heads, the maximum is taken over
+// query tokens, and the Top-k documents are selected
+//   [news.neo-ai.one article, "全体設計 / アーキテクチャ"; github-eval-reports "MSA 项目评测报告",
+//    "核心模块 / 路由投影器"; ruixiangma.github.io blog, "稀疏注意力机制 / Top-k检索"].
+// A document's score is the maximum over its chunks.
+//
+// Design (the bank is streamed once per query batch; HBM-bound for short queries):
+//  * Persistent grid, one contiguous document-aligned chunk range per CTA (docs never straddle
+//    CTAs, so each CTA's candidate list is an exact superset of its share of the top-k).
+//  * K̄_r tiles (8-32 chunks, 16 KB) are staged into shared memory by 1-D bulk async copies
+//    (cp.async.bulk + mbarrier transaction counts), STAGES deep, issued by one thread.
+//  * The query side is folded once per CTA into q̃[r, g, :] = sum over the router heads h of
+//    KV head g of Q_r[r,h,:] / (||Q_r[r,h]|| * h_qr), kept in registers (E elements x R rows
+//    per thread). A chunk's score for row r is sum_g inv_norm[c,g] * <q̃[r,g], K̄_r[c,g]>.
+//  * Each thread owns E consecutive elements of a chunk row; partial dots of U chunks x R rows
+//    are reduced across the warp by a transposing butterfly (each halving step sends half of
+//    the values), then across the warps that share a chunk through shared memory.
+//  * Per tile: max over query tokens -> per-document max (segmented, with a carry for a
+//    document that continues into the next tile) -> warp-register top-k insertion per query
+//    (lane i holds the i-th best 64-bit key (score, ~doc id)).
+//  * The CTA writes its k candidates per query; the last CTA to finish (threadfence + atomic
+//    ticket, no spinning) merges all candidates into the final top-k.
+#include "common.cuh"
+#include "kernels.cuh"
+
+#include <type_traits>
+
+namespace msa {
+
+
+constexpr int kNT = 256;
+constexpr int kWarps = kNT / 32;
+constexpr int kU = 4;       // chunks per thread per tile
+constexpr int kStages = 4;  // bulk-copy pipeline depth
+
+// Transposing warp reduction of N values per lane (see header comment). After the call,
+// if N >= 32 lane l holds flat indices [l*N/32, (l+1)*N/32) in v[0..N/32); otherwise v[0]
+// holds index l / (32/N), summed over all 32 lanes.
+template <int N, int O>
+__device__ __forceinline__ void tr_reduce(float* v, int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (N >= 2) {
+      constexpr int H = N / 2;
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < H; ++i) {
+        const float send = up ? v[i] : v[i + H];
+        const float keep = up ? v[i + H] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      tr_reduce<H, O / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      tr_reduce<1, O / 2>(v, lane);
+    }
+  }
+}
+
+// Insert the lanes' candidate keys into the warp-held sorted list (lane i < k holds the
+// i-th largest key; 0 = empty).
+__device__ __forceinline__ void list_insert(unsigned long long& li, unsigned long long key,
+                                            int lane, int k) {
+  const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
+  unsigned m = __ballot_sync(0xffffffffu, key > thr);
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    const unsigned long long x = __shfl_sync(0xffffffffu, key, src);
+    const unsigned gt = __ballot_sync(0xffffffffu, lane < k && li > x);
+    const int pos = __popc(gt);
+    const unsigned long long up = __shfl_up_sync(0xffffffffu, li, 1);
+    if (pos < k) {
+      if (lane > pos && lane < k) li = up;
+      if (lane == pos) li = x;
+    }
+  }
+}
+
+template <typename T, int R, int E>
+__global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
+  using VecT = Vec<T, E>;
+  using raw = typename VecT::raw;
+  constexpr int V = kU * R;
+  constexpr int VPL = V >= 32 ? V / 32 : 1;  // values per lane after the warp reduction
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int W = p.h_kv * p.d;
+  const int LPC = W / E;          // threads per chunk (multiple of 32, <= 256)
+  const int CPG = kNT / LPC;      // chunk groups per CTA
+  const int NWG = LPC / 32;       // warps per chunk group
+  const int TC = kU * CPG;        // chunks per tile
+  const uint32_t tile_bytes = (uint32_t)(TC * W * (int)sizeof(T));
+
+  extern __shared__ __align__(128) unsigned char sm[];
+  unsigned char* stage = sm;                                            // [kStages][tile]
+  float* qt = reinterpret_cast<float*>(sm + kStages * tile_bytes);     // [R][W]
+  float* red = qt + R * W;                                              // [kWarps][V]
+  float* msc = red + kWarps * V;                                        // [TC][R]
+  unsigned long long* lists =
+      reinterpret_cast<unsigned long long*>(msc + ((TC * R + 1) & ~1));  // [R][32]
+  float* carry = reinterpret_cast<float*>(lists + R * 32);             // [R]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(carry + ((R + 1) & ~1) + 2);
+  int64_t* docs = reinterpret_cast<int64_t*>(mbar + kStages);          // [0] cur, [1] next
+  int* flags = reinterpret_cast<int*>(docs + 2);                       // [0] last
+
+  // ---- document-aligned chunk range of this CTA
+  const int64_t G = gridDim.x;
+  const int64_t i = blockIdx.x;
+  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (i * p.n_chunks) / G);
+  const int64_t D1 = (i == G - 1) ? p.n_docs : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
+  const int64_t cb = p.coff[D0], ce = p.coff[D1];
+  const int64_t n_tiles = (ce - cb + TC - 1) / TC;
+  const T* kr = static_cast<const T*>(p.kr);
+  const size_t row_bytes = (size_t)W * sizeof(T);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
+    fence_mbar_init();
+    docs[0] = D0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < kStages && s < n_tiles; ++s) {
+      const int64_t c0 = cb + (int64_t)s * TC;
+      const int64_t n = min((int64_t)TC, ce - c0);
+      mbar_arrive_expect_tx(&mbar[s], (uint32_t)(n * row_bytes));
+      bulk_g2s(stage + (size_t)s * tile_bytes, kr + c0 * W, (uint32_t)(n * row_bytes), &mbar[s]);
+    }
+  }
+
+  // ---- fold the router queries into q̃ (shared), then into registers
+  {
+    const T* q = static_cast<const T*>(p.qr);
+    const int rows = p.B * p.T;
+    const int m = p.h_qr / p.h_kv;
+    const float inv_h = 1.0f / (float)p.h_qr;
+    for (int pair = warp; pair < R * p.h_kv; pair += kWarps) {
+      const int r = pair / p.h_kv, g = pair % p.h_kv;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r < rows) {
+        for (int hm = 0; hm < m; ++hm) {
+          const int h = g * m + hm;
+          const T* qh = q + ((int64_t)r * p.h_qr + h) * p.d;
+          float x[4];
+          float ss = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = lane + 32 * j;
+            x[j] = e < p.d ? Elem<T>::to_f(qh[e]) : 0.f;
+            ss += x[j] * x[j];
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          const float sc = ss > 0.f ? (1.0f / sqrtf(ss)) * inv_h : 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[j] += x[j] * sc;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = lane + 32 * j;
+        if (e < p.d) qt[r * W + g * p.d + e] = acc[j];
+      }
+    }
+    for (int b = warp; b < R; b += kWarps) lists[b * 32 + lane] = 0ull;
+    if (tid < R) carry[tid] = -INFINITY;
+  }
+  __syncthreads();
+
+  const int cg = tid / LPC;
+  const int li = tid % LPC;
+  const int e0 = li * E;
+  const int g = e0 / p.d;
+  float qreg[R][E];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qreg[r][e] = qt[r * W + e0 + e];
+
+  bool failed = false;
+  int64_t it = 0;
+  for (; it < n_tiles; ++it) {
+    const int s = (int)(it % kStages);
+    const uint32_t par = (uint32_t)((it / kStages) & 1);
+    const int64_t c0 = cb + it * TC;
+    const int n = (int)min((int64_t)TC, ce - c0);
+    const bool ok = mbar_wait_bounded(&mbar[s], par, p.err);
+
+    float v[V];
+    const unsigned char* tile = stage + (size_t)s * tile_bytes;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int ci = u * CPG + cg;
+      float x[E];
+      float inv = 0.f;
+      if (ci < n) {
+        VecT::unpack(*reinterpret_cast<const raw*>(tile + ((size_t)ci * W + e0) * sizeof(T)), x);
+        inv = __ldg(p.invk + (c0 + ci) * p.h_kv + g);
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) x[e] = 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) a = fmaf(qreg[r][e], x[e], a);
+        v[u * R + r] = a * inv;
+      }
+    }
+    tr_reduce<V, 16>(v, lane);
+    if constexpr (V >= 32) {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) red[warp * V + lane * VPL + j] = v[j];
+    } else {
+      if ((lane % (32 / V)) == 0) red[warp * V + lane / (32 / V)] = v[0];
+    }
+    if (!__syncthreads_and(ok)) {  // (A) stage s and red are complete for every thread
+      failed = true;
+      break;
+    }
+    if (tid == 0 && it + kStages < n_tiles) {
+      fence_proxy_async_smem();
+      const int64_t cn = cb + (it + kStages) * TC;
+      const int64_t nn = min((int64_t)TC, ce - cn);
+      mbar_arrive_expect_tx(&mbar[s], (uint32_t)(nn * row_bytes));
+      bulk_g2s(stage + (size_t)s * tile_bytes, kr + cn * W, (uint32_t)(nn * row_bytes), &mbar[s]);
+    }
+    // chunk score per query: max over tokens of the sum over the group's warps
+    for (int idx = tid; idx < TC * p.B; idx += kNT) {
+      const int ci = idx / p.B, b = idx % p.B;
+      const int gi = ci % CPG, u = ci / CPG;
+      float mx = -INFINITY;
+      if (ci < n) {
+        for (int t = 0; t < p.T; ++t) {
+          const int f = u * R + b * p.T + t;
+          float sum = 0.f;
+          for (int w = 0; w < NWG; ++w) sum += red[(gi * NWG + w) * V + f];
+          mx = fmaxf(mx, sum);
+        }
+      }
+      msc[ci * R + b] = mx;
+    }
+    __syncthreads();  // (B)
+    // per-document max + top-k insertion; warp w serves queries w, w + 8, ...
+    const int64_t dcur = docs[it & 1];
+    const int64_t tend = c0 + n;
+    for (int b = warp; b < p.B; b += kWarps) {
+      unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
+      float cr = carry[b];
+      int64_t dd = dcur;
+      int64_t next = dcur;
+      while (true) {
+        const int64_t doc = dd + lane;
+        bool valid = doc < D1;
+        const int64_t ds = valid ? p.coff[doc] : 0;
+        const int64_t de = valid ? p.coff[doc + 1] : 0;
+        valid = valid && ds < tend;
+        bool fin = false;
+        float sc = -INFINITY;
+        if (valid) {
+          const int64_t lo = max(ds, c0), hi = min(de, tend);
+          for (int64_t c = lo; c < hi; ++c) sc = fmaxf(sc, msc[(c - c0) * R + b]);
+          if (ds < c0) sc = fmaxf(sc, cr);
+          fin = de <= tend;
+        }
+        unsigned long long key = 0ull;
+        if (fin) {
+          if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = sc;
+          const bool ex = p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
+          if (!ex) key = score_key(sc, (uint32_t)doc);
+        }
+        list_insert(lst, key, lane, p.k);
+        const unsigned cont = __ballot_sync(0xffffffffu, valid && !fin);
+        const unsigned vm = __ballot_sync(0xffffffffu, valid);
+        if (cont) {
+          const int src = __ffs(cont) - 1;
+          cr = __shfl_sync(0xffffffffu, sc, src);
+          next = dd + src;
+          break;
+        }
+        if (vm != 0xffffffffu) {
+          next = dd + __popc(vm);
+          break;
+        }
+        dd += 32;
+      }
+      if (lane < p.k) lists[b * 32 + lane] = lst;
+      if (lane == 0) carry[b] = cr;
+      if (b == 0 && lane == 0) docs[(it + 1) & 1] = next;
+    }
+    __syncthreads();  // (C)
+  }
+
+  if (failed) {
+    // drain the copies still in flight into this CTA's shared memory (bounded)
+    for (int64_t t = it; t < n_tiles && t < it + kStages; ++t)
+      mbar_wait_bounded(&mbar[t % kStages], (uint32_t)((t / kStages) & 1), p.err);
+    __syncthreads();
+  } else {
+    // documents without chunks at the end of the range score -inf
+    const int64_t dcur = docs[n_tiles & 1];
+    for (int b = warp; b < p.B; b += kWarps) {
+      unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
+      for (int64_t dd = dcur; dd < D1; dd += 32) {
+        const int64_t doc = dd + lane;
+        unsigned long long key = 0ull;
+        if (doc < D1) {
+          if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = -INFINITY;
+          const bool ex = p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
+          if (!ex) key = score_key(-INFINITY, (uint32_t)doc);
+        }
+        list_insert(lst, key, lane, p.k);
+      }
+      if (lane < p.k) lists[b * 32 + lane] = lst;
+    }
+    __syncthreads();
+  }
+
+  // ---- publish this CTA's candidates; the last CTA merges
+  for (int b = warp; b < p.B; b += kWarps)
+    if (lane < p.k) p.cand[(i * p.B + b) * p.k + lane] = lists[b * 32 + lane];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned t = atomicInc(p.counter, (unsigned)(G - 1));
+    flags[0] = (t == (unsigned)(G - 1));
+  }
+  __syncthreads();
+  if (!flags[0]) return;
+  __threadfence();
+  const int64_t total = G * p.k;
+  for (int b = warp; b < p.B; b += kWarps) {
+    unsigned long long lst = 0ull;
+    for (int64_t base = 0; base < total; base += 32) {
+      const int64_t idx = base + lane;
+      unsigned long long key = 0ull;
+      if (idx < total) {
+        const int64_t cta = idx / p.k, j = idx % p.k;
+        key = __ldcg(p.cand + (cta * p.B + b) * p.k + j);
+      }
+      list_insert(lst, key, lane, p.k);
+    }
+    if (lane < p.k) {
+      p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
+      p.top_scores[b * p.k + lane] = lst ? key_score(lst) : -INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------- launch
+template <typename T, int R, int E>
+static size_t route_smem_bytes(int W) {
+  const int LPC = W / E, CPG = kNT / LPC, TC = kU * CPG;
+  const size_t tile = (size_t)TC * W * sizeof(T);
+  size_t s = kStages * tile + sizeof(float) * ((size_t)R * W + kWarps * kU * R + ((TC * R + 1) & ~1));
+  s += sizeof(unsigned long long) * R * 32 + sizeof(float) * (((R + 1) & ~1) + 2);
+  s += sizeof(uint64_t) * kStages + sizeof(int64_t) * 2 + sizeof(int) * 4;
+  return (s + 127) & ~(size_t)127;
+}
+
+template <typename T, int R, int E>
+static cudaError_t route_launch_t(const RouteParams& p, int grid, cudaStream_t st) {
+  const size_t smem = route_smem_bytes<T, R, E>(p.h_kv * p.d);
+  auto kfn = route_scan_kernel<T, R, E>;
+  cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kfn<<<grid, kNT, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int R, int E>
+static int route_grid_t(int W, int sms, int64_t n_chunks) {
+  const size_t smem = route_smem_bytes<T, R, E>(W);
+  auto kfn = route_scan_kernel<T, R, E>;
+  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return -1;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kNT, smem) != cudaSuccess || per_sm < 1)
+    return -1;
+  const int TC = kU * (kNT / (W / E));
+  int64_t want = (n_chunks + 2 * TC - 1) / (2 * TC);  // at least two tiles per CTA
+  int64_t cap = (int64_t)per_sm * sms;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+// Dispatch on (dtype, rows per pass, vector width). Returns false if unsupported.
+
+RouteChoice route_choose(int dtype, int rows, int W) {
+  int R = 1;
+  while (R < rows) R <<= 1;
+  if (R > 16) return {0, 0};
+  int E = dtype == 1 ? (R <= 8 ? 8 : 4) : 4;
+  if (dtype == 1 && E == 8 && ((W / 8) % 32 != 0 || W / 8 > kNT)) E = 4;
+  if (W % E != 0 || (W / E) % 32 != 0 || W / E > kNT) return {0, 0};
+  return {R, E};
+}
+
+#define MSA_ROUTE_CASES(X)                                                              \
+  X(float, 1, 4) X(float, 2, 4) X(float, 4, 4) X(float, 8, 4) X(float, 16, 4)           \
+  X(__nv_bfloat16, 1, 8) X(__nv_bfloat16, 2, 8) X(__nv_bfloat16, 4, 8)                  \
+  X(__nv_bfloat16, 8, 8) X(__nv_bfloat16, 1, 4) X(__nv_bfloat16, 2, 4)                  \
+  X(__nv_bfloat16, 4, 4) X(__nv_bfloat16, 8, 4) X(__nv_bfloat16, 16, 4)
+
+int route_grid(int dtype, RouteChoice c, int W, int sms, int64_t n_chunks) {
+#define X(TT, RR, EE)                                                                     \
+  if ((dtype == 1) == std::is_same<TT, __nv_bfloat16>::value && c.R == RR && c.E == EE)   \
+    return route_grid_t<TT, RR, EE>(W, sms, n_chunks);
+  MSA_ROUTE_CASES(X)
+#undef X
+  return -1;
+}
+
+cudaError_t route_launch(int dtype, RouteChoice c, const RouteParams& p, int grid, cudaStream_t st) {
+#define X(TT, RR, EE)                                                                     \
+  if ((dtype == 1) == std::is_same<TT, __nv_bfloat16>::value && c.R == RR && c.E == EE)   \
+    return route_launch_t<TT, RR, EE>(p, grid, st);
+  MSA_ROUTE_CASES(X)
+#undef X
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace msa

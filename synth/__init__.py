@@ -332,3 +332,133 @@ def appended_doc_kv(w: Workload, layer: int, doc: int, dtype: str | None = None)
     k = normal(w.seed, tag(APPK, layer), (w.doc_len, w.h_kv, w.d), dt, first=doc * n)
     v = normal(w.seed, tag(APPV, layer), (w.doc_len, w.h_kv, w.d), dt, first=doc * n)
     return k, v
+
+
+# ----------------------------------------------------------------------------------------
+# device-side construction (bit-identical to the host arrays above)
+# ----------------------------------------------------------------------------------------
+def dev_normal(t, seed: int, tg: int, first: int = 0, scale: float = 1.0, stream=None):
+    """Fill the contiguous float32/bfloat16 device tensor ``t`` with normal(seed, tg, first+i)."""
+    import torch
+    assert t.is_contiguous() and t.dtype in (torch.float32, torch.bfloat16)
+    st = (stream or torch.cuda.current_stream()).cuda_stream
+    rc = lib_dev().synth_dev_fill_normal(t.data_ptr(), t.numel(),
+                                         0 if t.dtype == torch.float32 else 1, seed, tg, first,
+                                         scale, st)
+    if rc != 0:
+        raise RuntimeError(f"synth_dev_fill_normal failed with cudaError {rc}")
+    return t
+
+
+def _tdtype(dtype: str):
+    import torch
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def to_torch(x: np.ndarray, dev):
+    import torch
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(x).to(dev)
+
+
+def dev_token_workload(w: Workload, dev, layer: int = 0) -> dict:
+    """Device twin of make_token_workload: the same values, generated in place on the GPU
+    (queries and planted rows are small and built on the host)."""
+    import torch
+    s, dt = w.seed, w.dtype
+    td = _tdtype(dt)
+    off = doc_tok_offsets(w)
+    n_tok = int(off[-1])
+    out = dict(doc_tok_off=off, n_tok=n_tok)
+    for name, tid in (("K", K), ("V", V), ("K_r", KR)):
+        out[name] = dev_normal(torch.empty((n_tok, w.h_kv, w.d), dtype=td, device=dev), s,
+                               tag(tid, layer))
+    host = dict(Q_r=normal(s, tag(QR, layer), (w.B, w.T, w.h_qr, w.d), dt))
+    out["Q_r"] = to_torch(host["Q_r"], dev)
+    out["Q"] = dev_normal(torch.empty((w.B, w.T, w.h_q, w.d), dtype=td, device=dev), s,
+                          tag(Q, layer))
+    out["K_loc"] = dev_normal(torch.empty((w.B, w.L_loc, w.h_kv, w.d), dtype=td, device=dev), s,
+                              tag(KLOC, layer))
+    out["V_loc"] = dev_normal(torch.empty((w.B, w.L_loc, w.h_kv, w.d), dtype=td, device=dev), s,
+                              tag(VLOC, layer))
+    planted = np.sort(distinct(s, tag(PLANT_DOCS, layer), min(w.n_planted, w.n_docs),
+                               w.n_docs)) if w.n_planted else np.zeros(0, np.int64)
+    if len(planted):
+        u = planted_direction(as_f32(host["Q_r"][0], dt), w.h_kv)
+        for j, p in enumerate(planted):
+            a, b = int(off[p]), int(off[p + 1])
+            out["K_r"][a:b] = to_torch(planted_rows(s, layer, j, u, b - a, dt), dev)
+    out["planted"] = planted
+    return out
+
+
+def host_token_rows(w: Workload, name: str, t0: int, t1: int, layer: int = 0) -> np.ndarray:
+    """Host copy of token rows [t0, t1) of K / V / K_r (planted rows included)."""
+    tid = {"K": K, "V": V, "K_r": KR}[name]
+    row = w.h_kv * w.d
+    x = normal(w.seed, tag(tid, layer), (t1 - t0, w.h_kv, w.d), w.dtype, first=t0 * row)
+    if name == "K_r" and w.n_planted:
+        off = doc_tok_offsets(w)
+        planted = np.sort(distinct(w.seed, tag(PLANT_DOCS, layer), min(w.n_planted, w.n_docs),
+                                   w.n_docs))
+        qr = normal(w.seed, tag(QR, layer), (w.B, w.T, w.h_qr, w.d), w.dtype)
+        u = planted_direction(as_f32(qr[0], w.dtype), w.h_kv)
+        for j, p in enumerate(planted):
+            a, b = int(off[p]), int(off[p + 1])
+            lo, hi = max(a, t0), min(b, t1)
+            if lo < hi:
+                rows = planted_rows(w.seed, layer, j, u, b - a, w.dtype)
+                x[lo - t0:hi - t0] = rows[lo - a:hi - a]
+    return x
+
+
+def dev_bank_workload(w: Workload, dev, layer: int = 0, with_kv: bool = True) -> dict:
+    """Device twin of make_bank_workload (pre-pooled bank generated in place)."""
+    import torch
+    s, dt = w.seed, w.dtype
+    td = _tdtype(dt)
+    lens = (1 + uniform(s, tag(DOC_LEN), w.n_docs, 2 * w.doc_len - 1)) if w.ragged else \
+        np.full(w.n_docs, w.doc_len, dtype=np.int64)
+    coff = chunk_offsets_from_lengths(lens, w.chunk)
+    n_chunks = int(coff[-1])
+    out = dict(doc_chunk_off=coff, n_chunks=n_chunks, doc_len=lens)
+    qr = normal(s, tag(QR, layer), (w.B, w.T, w.h_qr, w.d), dt)
+    out["Q_r_host"] = qr
+    out["Q_r"] = to_torch(qr, dev)
+    out["Q"] = dev_normal(torch.empty((w.B, w.T, w.h_q, w.d), dtype=td, device=dev), s,
+                          tag(Q, layer))
+    out["K_loc"] = dev_normal(torch.empty((w.B, w.L_loc, w.h_kv, w.d), dtype=td, device=dev), s,
+                              tag(KLOC, layer))
+    out["V_loc"] = dev_normal(torch.empty((w.B, w.L_loc, w.h_kv, w.d), dtype=td, device=dev), s,
+                              tag(VLOC, layer))
+    Krb = dev_normal(torch.empty((n_chunks, w.h_kv, w.d), dtype=td, device=dev), s,
+                     tag(KRBAR, layer))
+    for _, p, rows in planted_bank_rows(w, layer, qr, coff):
+        Krb[int(coff[p]):int(coff[p + 1])] = to_torch(rows, dev)
+    out["Kbar_r"] = Krb
+    out["planted"] = plant_docs(w, layer)
+    if with_kv:
+        out["Kbar"] = dev_normal(torch.empty((n_chunks, w.h_kv, w.d), dtype=td, device=dev), s,
+                                 tag(KBAR, layer))
+        out["Vbar"] = dev_normal(torch.empty((n_chunks, w.h_kv, w.d), dtype=td, device=dev), s,
+                                 tag(VBAR, layer))
+    return out
+
+
+def host_bank_rows(w: Workload, name: str, c0: int, c1: int, layer: int = 0,
+                   coff: np.ndarray | None = None, Q_r: np.ndarray | None = None) -> np.ndarray:
+    """Host copy of bank rows [c0, c1) of K̄_r / K̄ / V̄ (planted K̄_r rows included)."""
+    tid = {"Kbar_r": KRBAR, "Kbar": KBAR, "Vbar": VBAR}[name]
+    row = w.h_kv * w.d
+    x = normal(w.seed, tag(tid, layer), (c1 - c0, w.h_kv, w.d), w.dtype, first=c0 * row)
+    if name == "Kbar_r" and w.n_planted:
+        if Q_r is None:
+            Q_r = normal(w.seed, tag(QR, layer), (w.B, w.T, w.h_qr, w.d), w.dtype)
+        for _, p, rows in planted_bank_rows(w, layer, Q_r, coff):
+            a, b = int(coff[p]), int(coff[p + 1])
+            lo, hi = max(a, c0), min(b, c1)
+            if lo < hi:
+                x[lo - c0:hi - c0] = rows[lo - a:hi - a]
+    return x

