@@ -165,7 +165,7 @@ size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv
   route_passes(B, T, &bp, &passes);
   const msa::RouteChoice c = msa::route_choose(dtype, bp * T, h_kv * d);
   if (c.R == 0) return kHeader;
-  const int grid = msa::route_grid(dtype, c, h_kv * d, sm_count(), n_chunks);
+  const int grid = msa::route_grid(dtype, c, h_kv * d, h_kv, sm_count(), n_chunks);
   if (grid < 1) return kHeader;
   return kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
 }
@@ -198,7 +198,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
   const int W = h_kv * d;
   const msa::RouteChoice c = msa::route_choose(dtype, bp * T, W);
   REQUIRE(c.R != 0, MSA_ERR_UNSUPPORTED, "router key row h_kv*d=%d not supported", W);
-  const int grid = msa::route_grid(dtype, c, W, sm_count(), n_chunks);
+  const int grid = msa::route_grid(dtype, c, W, h_kv, sm_count(), n_chunks);
   REQUIRE(grid >= 1, MSA_ERR_CUDA, "occupancy query failed");
   const size_t need = kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
   REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
@@ -235,6 +235,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
     p.cand = reinterpret_cast<unsigned long long*>(base + kHeader) + (size_t)pass * grid * bp * k;
     p.counter = reinterpret_cast<unsigned int*>(base) + 1 + pass;
     p.err = reinterpret_cast<int*>(base);
+    p.inv_bulk = (h_kv % 4 == 0 && aligned16(kr_inv_norm)) ? 1 : 0;
     e = msa::route_launch(dtype, c, p, grid, st);
     if (e != cudaSuccess) return cuda_fail(e, "msa_route_topk launch");
   }

@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
     }
 
     if (active) {
-      const float inv_n = 1.0f / (float)n;
+      const float fn = (float)n;
       const int64_t ob = c * (int64_t)W + (int64_t)h * D + e1;
       T* Kb = static_cast<T*>(p.Kb);
       T* Vb = static_cast<T*>(p.Vb);
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
         T* dst = (vct < 2 ? Kb : vct < 4 ? Rb : Vb) + ob + ((vct & 1) ? HALF : 0);
         T out[E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) out[e] = Elem<T>::from_f(src[e] * inv_n);
+        for (int e = 0; e < E; ++e) out[e] = Elem<T>::from_f(src[e] / fn);
         if (mine) *reinterpret_cast<raw*>(dst) = *reinterpret_cast<const raw*>(out);
         if (vct == 2 || vct == 3) {
 #pragma unroll

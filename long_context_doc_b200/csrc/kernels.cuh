@@ -41,10 +41,11 @@ struct RouteParams {
   unsigned long long* cand;  // [grid, B, k]
   unsigned int* counter;
   int* err;
+  int inv_bulk;              // inverse norms copied with each tile (h_kv % 4 == 0, aligned)
 };
 struct RouteChoice { int R, E; };
 RouteChoice route_choose(int dtype, int rows, int W);
-int route_grid(int dtype, RouteChoice c, int W, int sms, int64_t n_chunks);
+int route_grid(int dtype, RouteChoice c, int W, int h_kv, int sms, int64_t n_chunks);
 cudaError_t route_launch(int dtype, RouteChoice c, const RouteParams& p, int grid, cudaStream_t st);
 
 // ---- gather.cu

@@ -36,6 +36,7 @@ constexpr int kNT = 256;
 constexpr int kWarps = kNT / 32;
 constexpr int kU = 4;       // chunks per thread per tile
 constexpr int kStages = 4;  // bulk-copy pipeline depth
+constexpr int kWin = 1024;  // document offsets cached in shared memory
 
 // Transposing warp reduction of N values per lane (see header comment). After the call,
 // if N >= 32 lane l holds flat indices [l*N/32, (l+1)*N/32) in v[0..N/32); otherwise v[0]
@@ -81,11 +82,12 @@ __device__ __forceinline__ void list_insert(unsigned long long& li, unsigned lon
 }
 
 template <typename T, int R, int E>
-__global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(RouteParams p) {
   using VecT = Vec<T, E>;
   using raw = typename VecT::raw;
   constexpr int V = kU * R;
   constexpr int VPL = V >= 32 ? V / 32 : 1;  // values per lane after the warp reduction
+  constexpr int E2 = E / 2;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int W = p.h_kv * p.d;
@@ -94,45 +96,53 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
   const int NWG = LPC / 32;       // warps per chunk group
   const int TC = kU * CPG;        // chunks per tile
   const uint32_t tile_bytes = (uint32_t)(TC * W * (int)sizeof(T));
+  const uint32_t inv_bytes = (uint32_t)(TC * p.h_kv * 4);
 
   extern __shared__ __align__(128) unsigned char sm[];
-  unsigned char* stage = sm;                                            // [kStages][tile]
-  float* qt = reinterpret_cast<float*>(sm + kStages * tile_bytes);     // [R][W]
-  float* red = qt + R * W;                                              // [kWarps][V]
-  float* msc = red + kWarps * V;                                        // [TC][R]
-  unsigned long long* lists =
-      reinterpret_cast<unsigned long long*>(msc + ((TC * R + 1) & ~1));  // [R][32]
-  float* carry = reinterpret_cast<float*>(lists + R * 32);             // [R]
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(carry + ((R + 1) & ~1) + 2);
-  int64_t* docs = reinterpret_cast<int64_t*>(mbar + kStages);          // [0] cur, [1] next
-  int* flags = reinterpret_cast<int*>(docs + 2);                       // [0] last
+  unsigned char* stage = sm;                                                   // [S][tile]
+  float* invs = reinterpret_cast<float*>(sm + kStages * tile_bytes);          // [S][TC*h_kv]
+  float* qt = invs + kStages * TC * p.h_kv;                                    // [R][W]
+  float* red = qt + R * W;                                                     // [2][warps][V]
+  int64_t* win = reinterpret_cast<int64_t*>(red + 2 * kWarps * V);            // [kWin+1]
+  unsigned long long* lists = reinterpret_cast<unsigned long long*>(win + kWin + 1);  // [R][32]
+  float* carry = reinterpret_cast<float*>(lists + R * 32);                    // [R]
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(carry + ((R + 1) & ~1) + 2);   // [S]
+  int64_t* docs = reinterpret_cast<int64_t*>(mbar + kStages);                 // [0..1] cur, [2] win0
+  int* flags = reinterpret_cast<int*>(docs + 3);                              // [0] last
 
   // ---- document-aligned chunk range of this CTA
   const int64_t G = gridDim.x;
   const int64_t i = blockIdx.x;
   const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (i * p.n_chunks) / G);
-  const int64_t D1 = (i == G - 1) ? p.n_docs : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
+  const int64_t D1 = (i == G - 1) ? p.n_docs
+                                  : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
   const int64_t cb = p.coff[D0], ce = p.coff[D1];
   const int64_t n_tiles = (ce - cb + TC - 1) / TC;
   const T* kr = static_cast<const T*>(p.kr);
   const size_t row_bytes = (size_t)W * sizeof(T);
 
+  auto issue = [&](int s, int64_t t) {
+    const int64_t c0 = cb + t * TC;
+    const int64_t n = min((int64_t)TC, ce - c0);
+    const uint32_t kb = (uint32_t)(n * row_bytes);
+    const uint32_t ib = p.inv_bulk ? (uint32_t)(n * p.h_kv * 4) : 0u;
+    mbar_arrive_expect_tx(&mbar[s], kb + ib);
+    bulk_g2s(stage + (size_t)s * tile_bytes, kr + c0 * W, kb, &mbar[s]);
+    if (ib) bulk_g2s(invs + s * TC * p.h_kv, p.invk + c0 * p.h_kv, ib, &mbar[s]);
+  };
+
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
     fence_mbar_init();
     docs[0] = D0;
+    docs[2] = D0;
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int s = 0; s < kStages && s < n_tiles; ++s) {
-      const int64_t c0 = cb + (int64_t)s * TC;
-      const int64_t n = min((int64_t)TC, ce - c0);
-      mbar_arrive_expect_tx(&mbar[s], (uint32_t)(n * row_bytes));
-      bulk_g2s(stage + (size_t)s * tile_bytes, kr + c0 * W, (uint32_t)(n * row_bytes), &mbar[s]);
-    }
-  }
+  if (tid == 0)
+    for (int s = 0; s < kStages && s < n_tiles; ++s) issue(s, s);
 
-  // ---- fold the router queries into q̃ (shared), then into registers
+  // ---- doc-offset window, query fold (q̃ in shared, then registers)
+  for (int j = tid; j <= kWin; j += kNT) win[j] = (D0 + j <= D1) ? p.coff[D0 + j] : INT64_MAX;
   {
     const T* q = static_cast<const T*>(p.qr);
     const int rows = p.B * p.T;
@@ -175,11 +185,12 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
   const int li = tid % LPC;
   const int e0 = li * E;
   const int g = e0 / p.d;
-  float qreg[R][E];
+  float2 qreg[R][E2];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int e = 0; e < E; ++e) qreg[r][e] = qt[r * W + e0 + e];
+    for (int e = 0; e < E2; ++e)
+      qreg[r][e] = make_float2(qt[r * W + e0 + 2 * e], qt[r * W + e0 + 2 * e + 1]);
 
   bool failed = false;
   int64_t it = 0;
@@ -192,62 +203,56 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
 
     float v[V];
     const unsigned char* tile = stage + (size_t)s * tile_bytes;
+    const float* itile = invs + s * TC * p.h_kv;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int ci = u * CPG + cg;
-      float x[E];
+      float2 x2[E2];
       float inv = 0.f;
       if (ci < n) {
+        float x[E];
         VecT::unpack(*reinterpret_cast<const raw*>(tile + ((size_t)ci * W + e0) * sizeof(T)), x);
-        inv = __ldg(p.invk + (c0 + ci) * p.h_kv + g);
+#pragma unroll
+        for (int e = 0; e < E2; ++e) x2[e] = make_float2(x[2 * e], x[2 * e + 1]);
+        inv = p.inv_bulk ? itile[ci * p.h_kv + g] : __ldg(p.invk + (c0 + ci) * p.h_kv + g);
       } else {
 #pragma unroll
-        for (int e = 0; e < E; ++e) x[e] = 0.f;
+        for (int e = 0; e < E2; ++e) x2[e] = make_float2(0.f, 0.f);
       }
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float a = 0.f;
+        float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < E; ++e) a = fmaf(qreg[r][e], x[e], a);
-        v[u * R + r] = a * inv;
+        for (int e = 0; e < E2; ++e) a = __ffma2_rn(qreg[r][e], x2[e], a);
+        v[u * R + r] = (a.x + a.y) * inv;
       }
     }
     tr_reduce<V, 16>(v, lane);
+    float* rb = red + (int)(it & 1) * kWarps * V;
     if constexpr (V >= 32) {
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) red[warp * V + lane * VPL + j] = v[j];
+      for (int j = 0; j < VPL; ++j) rb[warp * V + lane * VPL + j] = v[j];
     } else {
-      if ((lane % (32 / V)) == 0) red[warp * V + lane / (32 / V)] = v[0];
+      if ((lane % (32 / V)) == 0) rb[warp * V + lane / (32 / V)] = v[0];
     }
-    if (!__syncthreads_and(ok)) {  // (A) stage s and red are complete for every thread
+    if (!__syncthreads_and(ok)) {  // the only block-wide barrier of a tile
       failed = true;
       break;
     }
     if (tid == 0 && it + kStages < n_tiles) {
       fence_proxy_async_smem();
-      const int64_t cn = cb + (it + kStages) * TC;
-      const int64_t nn = min((int64_t)TC, ce - cn);
-      mbar_arrive_expect_tx(&mbar[s], (uint32_t)(nn * row_bytes));
-      bulk_g2s(stage + (size_t)s * tile_bytes, kr + cn * W, (uint32_t)(nn * row_bytes), &mbar[s]);
+      issue(s, it + kStages);
     }
-    // chunk score per query: max over tokens of the sum over the group's warps
-    for (int idx = tid; idx < TC * p.B; idx += kNT) {
-      const int ci = idx / p.B, b = idx % p.B;
-      const int gi = ci % CPG, u = ci / CPG;
-      float mx = -INFINITY;
-      if (ci < n) {
-        for (int t = 0; t < p.T; ++t) {
-          const int f = u * R + b * p.T + t;
-          float sum = 0.f;
-          for (int w = 0; w < NWG; ++w) sum += red[(gi * NWG + w) * V + f];
-          mx = fmaxf(mx, sum);
-        }
-      }
-      msc[ci * R + b] = mx;
-    }
-    __syncthreads();  // (B)
-    // per-document max + top-k insertion; warp w serves queries w, w + 8, ...
+    // slide the doc-offset window when this tile's docs may run past it
     const int64_t dcur = docs[it & 1];
+    if (dcur + TC + 2 > docs[2] + kWin) {
+      for (int j = tid; j <= kWin; j += kNT) win[j] = (dcur + j <= D1) ? p.coff[dcur + j] : INT64_MAX;
+      __syncthreads();
+      if (tid == 0) docs[2] = dcur;
+      __syncthreads();
+    }
+    const int64_t w0 = docs[2];
+    // per-document max + top-k insertion; warp w serves queries w, w + 8, ...
     const int64_t tend = c0 + n;
     for (int b = warp; b < p.B; b += kWarps) {
       unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
@@ -257,14 +262,26 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
       while (true) {
         const int64_t doc = dd + lane;
         bool valid = doc < D1;
-        const int64_t ds = valid ? p.coff[doc] : 0;
-        const int64_t de = valid ? p.coff[doc + 1] : 0;
+        int64_t ds = 0, de = 0;
+        if (valid) {
+          ds = (doc - w0 < kWin) ? win[doc - w0] : __ldg(p.coff + doc);
+          de = (doc + 1 - w0 <= kWin) ? win[doc + 1 - w0] : __ldg(p.coff + doc + 1);
+        }
         valid = valid && ds < tend;
         bool fin = false;
         float sc = -INFINITY;
         if (valid) {
           const int64_t lo = max(ds, c0), hi = min(de, tend);
-          for (int64_t c = lo; c < hi; ++c) sc = fmaxf(sc, msc[(c - c0) * R + b]);
+          for (int64_t c = lo; c < hi; ++c) {
+            const int ci = (int)(c - c0);
+            const int gi = ci % CPG, u = ci / CPG;
+            for (int t = 0; t < p.T; ++t) {
+              const int f = u * R + b * p.T + t;
+              float sum = 0.f;
+              for (int w = 0; w < NWG; ++w) sum += rb[(gi * NWG + w) * V + f];
+              sc = fmaxf(sc, sum);
+            }
+          }
           if (ds < c0) sc = fmaxf(sc, cr);
           fin = de <= tend;
         }
@@ -293,8 +310,8 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
       if (lane == 0) carry[b] = cr;
       if (b == 0 && lane == 0) docs[(it + 1) & 1] = next;
     }
-    __syncthreads();  // (C)
   }
+  __syncthreads();
 
   if (failed) {
     // drain the copies still in flight into this CTA's shared memory (bounded)
@@ -354,18 +371,21 @@ __global__ void __launch_bounds__(kNT) route_scan_kernel(RouteParams p) {
 
 // ------------------------------------------------------------------------------- launch
 template <typename T, int R, int E>
-static size_t route_smem_bytes(int W) {
+static size_t route_smem_bytes(int W, int h_kv) {
   const int LPC = W / E, CPG = kNT / LPC, TC = kU * CPG;
   const size_t tile = (size_t)TC * W * sizeof(T);
-  size_t s = kStages * tile + sizeof(float) * ((size_t)R * W + kWarps * kU * R + ((TC * R + 1) & ~1));
-  s += sizeof(unsigned long long) * R * 32 + sizeof(float) * (((R + 1) & ~1) + 2);
-  s += sizeof(uint64_t) * kStages + sizeof(int64_t) * 2 + sizeof(int) * 4;
+  size_t s = kStages * tile + sizeof(float) * ((size_t)kStages * TC * h_kv + (size_t)R * W +
+                                               2 * kWarps * kU * R);
+  s = (s + 7) & ~(size_t)7;
+  s += sizeof(int64_t) * (kWin + 1) + sizeof(unsigned long long) * R * 32;
+  s += sizeof(float) * (((R + 1) & ~1) + 2);
+  s += sizeof(uint64_t) * kStages + sizeof(int64_t) * 3 + sizeof(int) * 4;
   return (s + 127) & ~(size_t)127;
 }
 
 template <typename T, int R, int E>
 static cudaError_t route_launch_t(const RouteParams& p, int grid, cudaStream_t st) {
-  const size_t smem = route_smem_bytes<T, R, E>(p.h_kv * p.d);
+  const size_t smem = route_smem_bytes<T, R, E>(p.h_kv * p.d, p.h_kv);
   auto kfn = route_scan_kernel<T, R, E>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -374,8 +394,8 @@ static cudaError_t route_launch_t(const RouteParams& p, int grid, cudaStream_t s
 }
 
 template <typename T, int R, int E>
-static int route_grid_t(int W, int sms, int64_t n_chunks) {
-  const size_t smem = route_smem_bytes<T, R, E>(W);
+static int route_grid_t(int W, int h_kv, int sms, int64_t n_chunks) {
+  const size_t smem = route_smem_bytes<T, R, E>(W, h_kv);
   auto kfn = route_scan_kernel<T, R, E>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return -1;
@@ -408,10 +428,10 @@ RouteChoice route_choose(int dtype, int rows, int W) {
   X(__nv_bfloat16, 8, 8) X(__nv_bfloat16, 1, 4) X(__nv_bfloat16, 2, 4)                  \
   X(__nv_bfloat16, 4, 4) X(__nv_bfloat16, 8, 4) X(__nv_bfloat16, 16, 4)
 
-int route_grid(int dtype, RouteChoice c, int W, int sms, int64_t n_chunks) {
+int route_grid(int dtype, RouteChoice c, int W, int h_kv, int sms, int64_t n_chunks) {
 #define X(TT, RR, EE)                                                                     \
   if ((dtype == 1) == std::is_same<TT, __nv_bfloat16>::value && c.R == RR && c.E == EE)   \
-    return route_grid_t<TT, RR, EE>(W, sms, n_chunks);
+    return route_grid_t<TT, RR, EE>(W, h_kv, sms, n_chunks);
   MSA_ROUTE_CASES(X)
 #undef X
   return -1;
