@@ -109,6 +109,13 @@ msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_
 msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
                            int32_t dtype, float* kr_inv_norm, void* stream);
 
+/* msa_kr_normalize - routing-only copy of a router-key bank for the tensor-core scan:
+ * out[c,h,:] = Kbar_r[c,h,:] / ||Kbar_r[c,h]|| rounded to bf16 (zero rows stay zero),
+ * [n_chunks, h_kv, d] bf16. Bank preparation, made once per bank; needed by msa_route_topk
+ * when T > 16 (long queries). */
+msa_status msa_kr_normalize(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                            int32_t dtype, void* Kbar_r_hat, void* stream);
+
 /* ------------------------------------------------------------------------------------
  * msa_route_topk - online routing: cosine scoring of every chunk and exact top-k documents.
  *   [news.neo-ai.one, "アーキテクチャ": the routing projector computes relevance by cosine
@@ -119,6 +126,11 @@ msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, i
  *            floor(h / (h_qr / h_kv)).
  * Kbar_r     [n_chunks, h_kv, d] router-key bank (dtype), 16-byte aligned.
  * kr_inv_norm [n_chunks, h_kv] fp32 inverse norms (from msa_encode_pool / msa_kr_inv_norm).
+ * Kbar_r_hat (nullable) [n_chunks, h_kv, d] bf16 per-head unit rows (msa_kr_normalize).
+ *            Queries with T <= 16 are scored on CUDA cores from Kbar_r and kr_inv_norm in
+ *            fp32 (B*T rows in passes of up to 16). Longer queries (17 <= T <= 256, bf16
+ *            banks) are scored on the tensor cores as one bf16 contraction of Kbar_r_hat with
+ *            the per-head normalised queries (fp32 accumulation); Kbar_r_hat is required there.
  * doc_chunk_off [n_docs+1] device int64 chunk offsets (non-decreasing, ends at n_chunks).
  * Score of doc i for query b:
  *     S[b,i] = max_{c in doc i} max_t (1/h_qr) sum_h cos(Q_r[b,t,h], Kbar_r[c, g(h)])
@@ -129,15 +141,15 @@ msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, i
  *            docs are eligible.
  * top_scores [B, k] fp32 output (S of the selected docs; -inf in unused slots).
  * doc_scores (nullable) [B, n_docs] fp32 output: every S[b,i] (for tests).
- * Requires 1 <= k <= min(32, n_docs) and T <= 16 on the CUDA-core scan (B*T rows are
- * processed in passes of up to 16 rows).
+ * Requires 1 <= k <= min(32, n_docs); T <= 16 (any dtype) or 17 <= T <= 256 (bf16 with
+ * Kbar_r_hat).
  * ws         workspace of msa_route_topk_workspace(...) bytes; its first word is a device
  *            status (see msa_workspace_status).
  */
 size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv, int32_t d,
                                 int32_t dtype, int64_t n_docs, int64_t n_chunks, int32_t k);
 msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
-                          const void* Kbar_r, const float* kr_inv_norm,
+                          const void* Kbar_r, const float* kr_inv_norm, const void* Kbar_r_hat,
                           const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks,
                           int32_t h_kv, int32_t d, int32_t dtype, int32_t k,
                           const uint32_t* exclude_bits, int32_t* top_ids, float* top_scores,

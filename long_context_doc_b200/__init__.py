@@ -28,7 +28,8 @@ LIB_PATH = _build.LIB
 
 # every symbol include/msa.h declares
 SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chunks",
-           "msa_encode_pool", "msa_kr_inv_norm", "msa_route_topk_workspace", "msa_route_topk",
+           "msa_encode_pool", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
+           "msa_route_topk",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
            "msa_sparse_attend")
@@ -59,11 +60,13 @@ def _load():
                                   vp, vp, vp, i64, vp]
     L.msa_kr_inv_norm.restype = ctypes.c_int
     L.msa_kr_inv_norm.argtypes = [vp, i64, i32, i32, i32, vp, vp]
+    L.msa_kr_normalize.restype = ctypes.c_int
+    L.msa_kr_normalize.argtypes = [vp, i64, i32, i32, i32, vp, vp]
     L.msa_route_topk_workspace.restype = sz
     L.msa_route_topk_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i64, i64, i32]
     L.msa_route_topk.restype = ctypes.c_int
-    L.msa_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp,
-                                 vp, vp, vp, vp, sz, vp]
+    L.msa_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32,
+                                 vp, vp, vp, vp, vp, sz, vp]
     L.msa_workspace_status.restype = ctypes.c_int
     L.msa_workspace_status.argtypes = [vp, vp, vp]
     L.msa_gather.restype = ctypes.c_int
@@ -135,15 +138,21 @@ def msa_kr_inv_norm(Kbar_r, out, stream=None):
     _check(lib.msa_kr_inv_norm(_p(Kbar_r), n, h_kv, d, dtype_code(Kbar_r), _p(out), _s(stream)))
 
 
+def msa_kr_normalize(Kbar_r, out, stream=None):
+    n, h_kv, d = Kbar_r.shape
+    _check(lib.msa_kr_normalize(_p(Kbar_r), n, h_kv, d, dtype_code(Kbar_r), _p(out), _s(stream)))
+
+
 def msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k) -> int:
     return int(lib.msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k))
 
 
 def msa_route_topk(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_bits, top_ids, top_scores,
-                   doc_scores, ws, stream=None):
+                   doc_scores, ws, stream=None, Kbar_r_hat=None):
     B, T, h_qr, d = Q_r.shape
     n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
-    _check(lib.msa_route_topk(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm), _p(doc_chunk_off),
+    _check(lib.msa_route_topk(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm), _p(Kbar_r_hat),
+                              _p(doc_chunk_off),
                               doc_chunk_off.shape[0] - 1, n_chunks, h_kv, d, dtype_code(Kbar_r), k,
                               _p(exclude_bits), _p(top_ids), _p(top_scores), _p(doc_scores),
                               _p(ws), ws.numel() * ws.element_size(), _s(stream)))
@@ -205,6 +214,12 @@ def encode_pool(K, V, K_r, doc_tok_off_host, chunk: int, rope_base: float, strea
     return out
 
 
+def kr_normalize(Kbar_r, stream=None):
+    out = torch.empty(Kbar_r.shape, dtype=torch.bfloat16, device=Kbar_r.device)
+    msa_kr_normalize(Kbar_r, out, stream)
+    return out
+
+
 def kr_inv_norm(Kbar_r, stream=None):
     out = torch.empty(Kbar_r.shape[:2], dtype=torch.float32, device=Kbar_r.device)
     msa_kr_inv_norm(Kbar_r, out, stream)
@@ -212,7 +227,7 @@ def kr_inv_norm(Kbar_r, stream=None):
 
 
 def route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k: int, exclude_bits=None,
-               doc_scores: bool = False, ws=None, stream=None):
+               doc_scores: bool = False, ws=None, stream=None, Kbar_r_hat=None):
     """Returns (top_ids int32 [B,k], top_scores f32 [B,k], doc_scores f32 [B,n_docs] or None)."""
     B, T, h_qr, d = Q_r.shape
     n_chunks, h_kv = Kbar_r.shape[:2]
@@ -224,7 +239,8 @@ def route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k: int, exclude_bits=None,
     ids = torch.empty((B, k), dtype=torch.int32, device=dev)
     sc = torch.empty((B, k), dtype=torch.float32, device=dev)
     ds = torch.empty((B, n_docs), dtype=torch.float32, device=dev) if doc_scores else None
-    msa_route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k, exclude_bits, ids, sc, ds, ws, stream)
+    msa_route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k, exclude_bits, ids, sc, ds, ws, stream,
+                   Kbar_r_hat)
     return ids, sc, ds
 
 

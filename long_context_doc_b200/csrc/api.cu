@@ -158,20 +158,35 @@ msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, i
 
 size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv, int32_t d,
                                 int32_t dtype, int64_t n_docs, int64_t n_chunks, int32_t k) {
-  (void)h_qr;
-  (void)n_docs;
   if (B < 1 || T < 1 || k < 1 || h_kv < 1 || d < 1) return kHeader;
+  if (T > 16) {
+    const msa::TcPlan pl = msa::tc_plan(B, T, h_kv, d, n_docs, n_chunks, k, sm_count());
+    if (!pl.ok) return kHeader;
+    return kHeader + pl.q_bytes + pl.m_bytes + pl.cand_bytes;
+  }
   int bp, passes;
   route_passes(B, T, &bp, &passes);
   const msa::RouteChoice c = msa::route_choose(dtype, bp * T, h_kv * d);
   if (c.R == 0) return kHeader;
-  const int grid = msa::route_grid(dtype, c, h_kv * d, h_kv, sm_count(), n_chunks);
+  const int grid = msa::route_grid(dtype, c, h_kv * d, h_kv, h_qr, sm_count(), n_chunks);
   if (grid < 1) return kHeader;
   return kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
 }
 
+msa_status msa_kr_normalize(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                            int32_t dtype, void* out, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(n_chunks >= 0, MSA_ERR_INVALID_ARG, "negative n_chunks");
+  REQUIRE(n_chunks == 0 || (Kbar_r && out), MSA_ERR_INVALID_ARG, "null tensor");
+  cudaError_t e = msa::launch_kr_normalize(Kbar_r, n_chunks, h_kv, d, dtype, out, sm_count(),
+                                           (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_kr_normalize launch");
+  return ok();
+}
+
 msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
-                          const void* Kbar_r, const float* kr_inv_norm,
+                          const void* Kbar_r, const float* kr_inv_norm, const void* Kbar_r_hat,
                           const int64_t* doc_chunk_off, int64_t n_docs, int64_t n_chunks,
                           int32_t h_kv, int32_t d, int32_t dtype, int32_t k,
                           const uint32_t* exclude_bits, int32_t* top_ids, float* top_scores,
@@ -186,11 +201,57 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
   REQUIRE(k >= 1 && k <= n_docs, MSA_ERR_INVALID_ARG, "k %d outside [1, n_docs=%lld]", k,
           (long long)n_docs);
   REQUIRE(k <= 32, MSA_ERR_UNSUPPORTED, "k %d > 32", k);
-  REQUIRE(T <= 16, MSA_ERR_UNSUPPORTED, "query length T=%d > 16 needs the tensor-core scan", T);
+  if (T > 16) {
+    REQUIRE(T <= 256, MSA_ERR_UNSUPPORTED, "query length T=%d > 256", T);
+    REQUIRE(dtype == MSA_BF16, MSA_ERR_UNSUPPORTED,
+            "queries with T=%d > 16 use the bf16 tensor-core scan (fp32 banks: T <= 16)", T);
+    REQUIRE(Kbar_r_hat != nullptr, MSA_ERR_INVALID_ARG,
+            "T=%d > 16 needs the normalised bank Kbar_r_hat (msa_kr_normalize)", T);
+  }
   if (B == 0) return ok();
   REQUIRE(Q_r && Kbar_r && kr_inv_norm && doc_chunk_off && top_ids && top_scores,
           MSA_ERR_INVALID_ARG, "null tensor");
   REQUIRE(aligned16(Kbar_r), MSA_ERR_INVALID_ARG, "Kbar_r must be 16-byte aligned");
+  if (T > 16) {
+    REQUIRE(aligned16(Kbar_r_hat) && aligned16(Q_r), MSA_ERR_INVALID_ARG,
+            "Kbar_r_hat and Q_r must be 16-byte aligned");
+    const msa::TcPlan pl = msa::tc_plan(B, T, h_kv, d, n_docs, n_chunks, k, sm_count());
+    REQUIRE(pl.ok, MSA_ERR_UNSUPPORTED, "tensor-core scan: h_kv*d=%d not a multiple of 64",
+            h_kv * d);
+    const size_t need = kHeader + pl.q_bytes + pl.m_bytes + pl.cand_bytes;
+    REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+            MSA_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu (256-byte aligned)",
+            ws_bytes, ws, need);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHeader, st);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace header reset");
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    msa::RouteTcArgs ta{};
+    ta.Q_r = Q_r;
+    ta.Kr_hat = Kbar_r_hat;
+    ta.coff = doc_chunk_off;
+    ta.excl = exclude_bits;
+    ta.n_docs = n_docs;
+    ta.n_chunks = n_chunks;
+    ta.B = B;
+    ta.T = T;
+    ta.h_qr = h_qr;
+    ta.h_kv = h_kv;
+    ta.d = d;
+    ta.k = k;
+    ta.dtype = dtype;
+    ta.top_ids = top_ids;
+    ta.top_scores = top_scores;
+    ta.doc_scores = doc_scores;
+    ta.q_hat = reinterpret_cast<__nv_bfloat16*>(base + kHeader);
+    ta.mscore = reinterpret_cast<float*>(base + kHeader + pl.q_bytes);
+    ta.cand = reinterpret_cast<unsigned long long*>(base + kHeader + pl.q_bytes + pl.m_bytes);
+    ta.counter = reinterpret_cast<unsigned int*>(base) + 1;
+    ta.err = reinterpret_cast<int*>(base);
+    e = msa::launch_route_tc(ta, pl, st);
+    if (e != cudaSuccess) return cuda_fail(e, "msa_route_topk (tensor-core scan) launch");
+    return ok();
+  }
   int bp, passes;
   route_passes(B, T, &bp, &passes);
   REQUIRE(passes <= kMaxPasses, MSA_ERR_UNSUPPORTED, "B=%d needs %d passes (> %d)", B, passes,
@@ -198,7 +259,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
   const int W = h_kv * d;
   const msa::RouteChoice c = msa::route_choose(dtype, bp * T, W);
   REQUIRE(c.R != 0, MSA_ERR_UNSUPPORTED, "router key row h_kv*d=%d not supported", W);
-  const int grid = msa::route_grid(dtype, c, W, h_kv, sm_count(), n_chunks);
+  const int grid = msa::route_grid(dtype, c, W, h_kv, h_qr, sm_count(), n_chunks);
   REQUIRE(grid >= 1, MSA_ERR_CUDA, "occupancy query failed");
   const size_t need = kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
   REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,

@@ -1,6 +1,7 @@
 // kernels.cuh - parameter blocks and launchers of the libmsa kernels (internal).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -45,8 +46,48 @@ struct RouteParams {
 };
 struct RouteChoice { int R, E; };
 RouteChoice route_choose(int dtype, int rows, int W);
-int route_grid(int dtype, RouteChoice c, int W, int h_kv, int sms, int64_t n_chunks);
+int route_grid(int dtype, RouteChoice c, int W, int h_kv, int h_qr, int sms, int64_t n_chunks);
 cudaError_t route_launch(int dtype, RouteChoice c, const RouteParams& p, int grid, cudaStream_t st);
+
+// ---- route_tc.cu (tensor-core scan for long queries)
+struct DocTopkParams {
+  const float* mscore;       // [B, n_chunks] chunk scores (max over tokens)
+  const int64_t* coff;
+  const uint32_t* excl;
+  int64_t n_docs, n_chunks, words;
+  int B, k;
+  int32_t* top_ids;
+  float* top_scores;
+  float* doc_scores;
+  unsigned long long* cand;  // [grid, B, k]
+  unsigned int* counter;
+};
+struct TcPlan {
+  bool ok;
+  int NQ, N, grid, topk_grid;
+  int64_t n_qtiles, n_ctiles;
+  size_t q_bytes, m_bytes, cand_bytes, smem;
+};
+struct RouteTcArgs {
+  const void* Q_r;
+  const void* Kr_hat;        // [n_chunks, h_kv * d] bf16 per-head unit rows
+  const int64_t* coff;
+  const uint32_t* excl;
+  int64_t n_docs, n_chunks;
+  int B, T, h_qr, h_kv, d, k, dtype;
+  int32_t* top_ids;
+  float* top_scores;
+  float* doc_scores;
+  __nv_bfloat16* q_hat;      // workspace [B*T, h_kv * d]
+  float* mscore;             // workspace [B, n_chunks]
+  unsigned long long* cand;  // workspace
+  unsigned int* counter;
+  int* err;
+};
+TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, int k, int sms);
+cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t st);
+cudaError_t launch_kr_normalize(const void* R, int64_t n_chunks, int h_kv, int d, int dtype,
+                                void* out, int sms, cudaStream_t st);
 
 // ---- gather.cu
 struct GatherParams {

@@ -32,10 +32,14 @@
 namespace msa {
 
 
-constexpr int kNT = 256;
+constexpr int kNT = 512;
 constexpr int kWarps = kNT / 32;
-constexpr int kU = 4;       // chunks per thread per tile
-constexpr int kStages = 4;  // bulk-copy pipeline depth
+// chunks per thread per sub-tile (one warp reduction each) and sub-tiles per tile; a tile is
+// kSub * kU = 8 vectors per thread (64 KB with 16-byte vectors). Wider query batches take
+// smaller sub-tiles to stay within 128 registers.
+template <int R> __host__ __device__ constexpr int kUof() { return R >= 8 ? 2 : 4; }
+template <int R> __host__ __device__ constexpr int kSubOf() { return 8 / kUof<R>(); }
+constexpr int kStages = 3;  // bulk-copy pipeline depth
 constexpr int kWin = 1024;  // document offsets cached in shared memory
 
 // Transposing warp reduction of N values per lane (see header comment). After the call,
@@ -82,28 +86,31 @@ __device__ __forceinline__ void list_insert(unsigned long long& li, unsigned lon
 }
 
 template <typename T, int R, int E>
-__global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(RouteParams p) {
+__global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   using VecT = Vec<T, E>;
   using raw = typename VecT::raw;
+  constexpr int kU = kUof<R>();
+  constexpr int kSub = kSubOf<R>();
   constexpr int V = kU * R;
   constexpr int VPL = V >= 32 ? V / 32 : 1;  // values per lane after the warp reduction
   constexpr int E2 = E / 2;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int W = p.h_kv * p.d;
-  const int LPC = W / E;          // threads per chunk (multiple of 32, <= 256)
-  const int CPG = kNT / LPC;      // chunk groups per CTA
-  const int NWG = LPC / 32;       // warps per chunk group
-  const int TC = kU * CPG;        // chunks per tile
+  const int LPC = W / E;             // threads per chunk (multiple of 32, <= kNT)
+  const int CPG = kNT / LPC;         // chunk groups per CTA
+  const int NWG = LPC / 32;          // warps per chunk group
+  const int TCS = kU * CPG;          // chunks per sub-tile
+  const int TC = kSub * TCS;         // chunks per tile
   const uint32_t tile_bytes = (uint32_t)(TC * W * (int)sizeof(T));
-  const uint32_t inv_bytes = (uint32_t)(TC * p.h_kv * 4);
 
   extern __shared__ __align__(128) unsigned char sm[];
   unsigned char* stage = sm;                                                   // [S][tile]
   float* invs = reinterpret_cast<float*>(sm + kStages * tile_bytes);          // [S][TC*h_kv]
-  float* qt = invs + kStages * TC * p.h_kv;                                    // [R][W]
-  float* red = qt + R * W;                                                     // [2][warps][V]
-  int64_t* win = reinterpret_cast<int64_t*>(red + 2 * kWarps * V);            // [kWin+1]
+  float* red = invs + kStages * TC * p.h_kv;                                   // [kSub][warps][V]
+  float* msc = red + kSub * kWarps * V;                                        // [TC][R]
+  float* qn = msc + TC * R;                                                    // [R][h_qr]
+  int64_t* win = reinterpret_cast<int64_t*>(qn + ((R * p.h_qr + 1) & ~1));    // [kWin+1]
   unsigned long long* lists = reinterpret_cast<unsigned long long*>(win + kWin + 1);  // [R][32]
   float* carry = reinterpret_cast<float*>(lists + R * 32);                    // [R]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(carry + ((R + 1) & ~1) + 2);   // [S]
@@ -141,56 +148,53 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
   if (tid == 0)
     for (int s = 0; s < kStages && s < n_tiles; ++s) issue(s, s);
 
-  // ---- doc-offset window, query fold (q̃ in shared, then registers)
+  // ---- doc-offset window; inverse norms of the router query heads
   for (int j = tid; j <= kWin; j += kNT) win[j] = (D0 + j <= D1) ? p.coff[D0 + j] : INT64_MAX;
-  {
-    const T* q = static_cast<const T*>(p.qr);
-    const int rows = p.B * p.T;
-    const int m = p.h_qr / p.h_kv;
-    const float inv_h = 1.0f / (float)p.h_qr;
-    for (int pair = warp; pair < R * p.h_kv; pair += kWarps) {
-      const int r = pair / p.h_kv, g = pair % p.h_kv;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (r < rows) {
-        for (int hm = 0; hm < m; ++hm) {
-          const int h = g * m + hm;
-          const T* qh = q + ((int64_t)r * p.h_qr + h) * p.d;
-          float x[4];
-          float ss = 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int e = lane + 32 * j;
-            x[j] = e < p.d ? Elem<T>::to_f(qh[e]) : 0.f;
-            ss += x[j] * x[j];
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          const float sc = ss > 0.f ? (1.0f / sqrtf(ss)) * inv_h : 0.f;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[j] += x[j] * sc;
-        }
+  const T* q = static_cast<const T*>(p.qr);
+  const int rows = p.B * p.T;
+  for (int pair = warp; pair < R * p.h_qr; pair += kWarps) {
+    const int r = pair / p.h_qr, h = pair % p.h_qr;
+    float ss = 0.f;
+    if (r < rows)
+      for (int e = lane; e < p.d; e += 32) {
+        const float x = Elem<T>::to_f(q[((int64_t)r * p.h_qr + h) * p.d + e]);
+        ss += x * x;
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = lane + 32 * j;
-        if (e < p.d) qt[r * W + g * p.d + e] = acc[j];
-      }
-    }
-    for (int b = warp; b < R; b += kWarps) lists[b * 32 + lane] = 0ull;
-    if (tid < R) carry[tid] = -INFINITY;
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) qn[pair] = ss > 0.f ? (1.0f / sqrtf(ss)) / (float)p.h_qr : 0.f;
   }
+  for (int b = warp; b < R; b += kWarps) lists[b * 32 + lane] = 0ull;
+  if (tid < R) carry[tid] = -INFINITY;
   __syncthreads();
 
+  // ---- this thread's slice of q̃: E elements of KV head g for every row, in registers
   const int cg = tid / LPC;
   const int li = tid % LPC;
   const int e0 = li * E;
   const int g = e0 / p.d;
+  const int ed = e0 % p.d;
   float2 qreg[R][E2];
+  {
+    const int m = p.h_qr / p.h_kv;
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+    for (int r = 0; r < R; ++r) {
+      float acc[E];
 #pragma unroll
-    for (int e = 0; e < E2; ++e)
-      qreg[r][e] = make_float2(qt[r * W + e0 + 2 * e], qt[r * W + e0 + 2 * e + 1]);
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      if (r < rows)
+        for (int hm = 0; hm < m; ++hm) {
+          const int h = g * m + hm;
+          const float sc = qn[r * p.h_qr + h];
+          float x[E];
+          VecT::unpack(*reinterpret_cast<const raw*>(q + ((int64_t)r * p.h_qr + h) * p.d + ed), x);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] += x[e] * sc;
+        }
+#pragma unroll
+      for (int e = 0; e < E2; ++e) qreg[r][e] = make_float2(acc[2 * e], acc[2 * e + 1]);
+    }
+  }
 
   bool failed = false;
   int64_t it = 0;
@@ -201,41 +205,44 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
     const int n = (int)min((int64_t)TC, ce - c0);
     const bool ok = mbar_wait_bounded(&mbar[s], par, p.err);
 
-    float v[V];
     const unsigned char* tile = stage + (size_t)s * tile_bytes;
     const float* itile = invs + s * TC * p.h_kv;
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int ci = u * CPG + cg;
-      float2 x2[E2];
-      float inv = 0.f;
-      if (ci < n) {
-        float x[E];
-        VecT::unpack(*reinterpret_cast<const raw*>(tile + ((size_t)ci * W + e0) * sizeof(T)), x);
+    for (int sub = 0; sub < kSub; ++sub) {
+      float v[V];
 #pragma unroll
-        for (int e = 0; e < E2; ++e) x2[e] = make_float2(x[2 * e], x[2 * e + 1]);
-        inv = p.inv_bulk ? itile[ci * p.h_kv + g] : __ldg(p.invk + (c0 + ci) * p.h_kv + g);
+      for (int u = 0; u < kU; ++u) {
+        const int ci = sub * TCS + u * CPG + cg;
+        float2 x2[E2];
+        float inv = 0.f;
+        if (ci < n) {
+          float x[E];
+          VecT::unpack(*reinterpret_cast<const raw*>(tile + ((size_t)ci * W + e0) * sizeof(T)), x);
+#pragma unroll
+          for (int e = 0; e < E2; ++e) x2[e] = make_float2(x[2 * e], x[2 * e + 1]);
+          inv = p.inv_bulk ? itile[ci * p.h_kv + g] : __ldg(p.invk + (c0 + ci) * p.h_kv + g);
+        } else {
+#pragma unroll
+          for (int e = 0; e < E2; ++e) x2[e] = make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < E2; ++e) a = __ffma2_rn(qreg[r][e], x2[e], a);
+          v[u * R + r] = (a.x + a.y) * inv;
+        }
+      }
+      tr_reduce<V, 16>(v, lane);
+      float* rb = red + (sub * kWarps + warp) * V;
+      if constexpr (V >= 32) {
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) rb[lane * VPL + j] = v[j];
       } else {
-#pragma unroll
-        for (int e = 0; e < E2; ++e) x2[e] = make_float2(0.f, 0.f);
-      }
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int e = 0; e < E2; ++e) a = __ffma2_rn(qreg[r][e], x2[e], a);
-        v[u * R + r] = (a.x + a.y) * inv;
+        if ((lane % (32 / V)) == 0) rb[lane / (32 / V)] = v[0];
       }
     }
-    tr_reduce<V, 16>(v, lane);
-    float* rb = red + (int)(it & 1) * kWarps * V;
-    if constexpr (V >= 32) {
-#pragma unroll
-      for (int j = 0; j < VPL; ++j) rb[warp * V + lane * VPL + j] = v[j];
-    } else {
-      if ((lane % (32 / V)) == 0) rb[warp * V + lane / (32 / V)] = v[0];
-    }
-    if (!__syncthreads_and(ok)) {  // the only block-wide barrier of a tile
+    if (!__syncthreads_and(ok)) {  // stage s consumed; partial sums complete
       failed = true;
       break;
     }
@@ -243,6 +250,23 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
       fence_proxy_async_smem();
       issue(s, it + kStages);
     }
+    // chunk score per query: sum over the chunk group's warps, max over the query tokens
+    for (int idx = tid; idx < TC * p.B; idx += kNT) {
+      const int ci = idx / p.B, b = idx % p.B;
+      const int sub = ci / TCS, cs = ci % TCS;
+      const int gi = cs % CPG, u = cs / CPG;
+      float mx = -INFINITY;
+      if (ci < n) {
+        for (int t = 0; t < p.T; ++t) {
+          const int f = u * R + b * p.T + t;
+          float sum = 0.f;
+          for (int w = 0; w < NWG; ++w) sum += red[(sub * kWarps + gi * NWG + w) * V + f];
+          mx = fmaxf(mx, sum);
+        }
+      }
+      msc[ci * R + b] = mx;
+    }
+    __syncthreads();
     // slide the doc-offset window when this tile's docs may run past it
     const int64_t dcur = docs[it & 1];
     if (dcur + TC + 2 > docs[2] + kWin) {
@@ -252,7 +276,7 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
       __syncthreads();
     }
     const int64_t w0 = docs[2];
-    // per-document max + top-k insertion; warp w serves queries w, w + 8, ...
+    // per-document max + top-k insertion; warp w serves queries w, w + kWarps, ...
     const int64_t tend = c0 + n;
     for (int b = warp; b < p.B; b += kWarps) {
       unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
@@ -271,17 +295,8 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
         bool fin = false;
         float sc = -INFINITY;
         if (valid) {
-          const int64_t lo = max(ds, c0), hi = min(de, tend);
-          for (int64_t c = lo; c < hi; ++c) {
-            const int ci = (int)(c - c0);
-            const int gi = ci % CPG, u = ci / CPG;
-            for (int t = 0; t < p.T; ++t) {
-              const int f = u * R + b * p.T + t;
-              float sum = 0.f;
-              for (int w = 0; w < NWG; ++w) sum += rb[(gi * NWG + w) * V + f];
-              sc = fmaxf(sc, sum);
-            }
-          }
+          const int lo = (int)(max(ds, c0) - c0), hi = (int)(min(de, tend) - c0);
+          for (int c = lo; c < hi; ++c) sc = fmaxf(sc, msc[c * R + b]);
           if (ds < c0) sc = fmaxf(sc, cr);
           fin = de <= tend;
         }
@@ -371,11 +386,13 @@ __global__ void __launch_bounds__(kNT, (R >= 16 ? 1 : 2)) route_scan_kernel(Rout
 
 // ------------------------------------------------------------------------------- launch
 template <typename T, int R, int E>
-static size_t route_smem_bytes(int W, int h_kv) {
-  const int LPC = W / E, CPG = kNT / LPC, TC = kU * CPG;
+static size_t route_smem_bytes(int W, int h_kv, int h_qr) {
+  constexpr int kU = kUof<R>(), kSub = kSubOf<R>();
+  const int LPC = W / E, CPG = kNT / LPC, TC = kSub * kU * CPG;
   const size_t tile = (size_t)TC * W * sizeof(T);
-  size_t s = kStages * tile + sizeof(float) * ((size_t)kStages * TC * h_kv + (size_t)R * W +
-                                               2 * kWarps * kU * R);
+  size_t s = kStages * tile + sizeof(float) * ((size_t)kStages * TC * h_kv +
+                                               (size_t)kSub * kWarps * kU * R + (size_t)TC * R +
+                                               (size_t)((R * h_qr + 1) & ~1));
   s = (s + 7) & ~(size_t)7;
   s += sizeof(int64_t) * (kWin + 1) + sizeof(unsigned long long) * R * 32;
   s += sizeof(float) * (((R + 1) & ~1) + 2);
@@ -385,7 +402,7 @@ static size_t route_smem_bytes(int W, int h_kv) {
 
 template <typename T, int R, int E>
 static cudaError_t route_launch_t(const RouteParams& p, int grid, cudaStream_t st) {
-  const size_t smem = route_smem_bytes<T, R, E>(p.h_kv * p.d, p.h_kv);
+  const size_t smem = route_smem_bytes<T, R, E>(p.h_kv * p.d, p.h_kv, p.h_qr);
   auto kfn = route_scan_kernel<T, R, E>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -394,15 +411,15 @@ static cudaError_t route_launch_t(const RouteParams& p, int grid, cudaStream_t s
 }
 
 template <typename T, int R, int E>
-static int route_grid_t(int W, int h_kv, int sms, int64_t n_chunks) {
-  const size_t smem = route_smem_bytes<T, R, E>(W, h_kv);
+static int route_grid_t(int W, int h_kv, int h_qr, int sms, int64_t n_chunks) {
+  const size_t smem = route_smem_bytes<T, R, E>(W, h_kv, h_qr);
   auto kfn = route_scan_kernel<T, R, E>;
   if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return -1;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, kNT, smem) != cudaSuccess || per_sm < 1)
     return -1;
-  const int TC = kU * (kNT / (W / E));
+  const int TC = kSubOf<R>() * kUof<R>() * (kNT / (W / E));
   int64_t want = (n_chunks + 2 * TC - 1) / (2 * TC);  // at least two tiles per CTA
   int64_t cap = (int64_t)per_sm * sms;
   if (want > cap) want = cap;
@@ -428,10 +445,10 @@ RouteChoice route_choose(int dtype, int rows, int W) {
   X(__nv_bfloat16, 8, 8) X(__nv_bfloat16, 1, 4) X(__nv_bfloat16, 2, 4)                  \
   X(__nv_bfloat16, 4, 4) X(__nv_bfloat16, 8, 4) X(__nv_bfloat16, 16, 4)
 
-int route_grid(int dtype, RouteChoice c, int W, int h_kv, int sms, int64_t n_chunks) {
+int route_grid(int dtype, RouteChoice c, int W, int h_kv, int h_qr, int sms, int64_t n_chunks) {
 #define X(TT, RR, EE)                                                                     \
   if ((dtype == 1) == std::is_same<TT, __nv_bfloat16>::value && c.R == RR && c.E == EE)   \
-    return route_grid_t<TT, RR, EE>(W, h_kv, sms, n_chunks);
+    return route_grid_t<TT, RR, EE>(W, h_kv, h_qr, sms, n_chunks);
   MSA_ROUTE_CASES(X)
 #undef X
   return -1;

@@ -1,0 +1,529 @@
+// route_tc.cu - routing for long queries (B*T rows beyond the CUDA-core scan) on the
+// 5th-generation tensor cores: the chunk-vs-query cosine matrix is a dense contraction.
+//
+// Method (as in route.cu): cosine of Q_r against every chunk's K̄_r, mean over heads, max
+// over query tokens, max over a document's chunks, top-k documents
+//   [news.neo-ai.one article, "全体設計 / アーキテクチャ"; github-eval-reports, "核心模块"].
+//
+// Because the cosine normalises each head separately, the contraction runs on per-head unit
+// vectors: K̂_r[c, g, :] = K̄_r[c, g, :] / ||K̄_r[c, g]|| (bank preparation, bf16, once per
+// bank) and q̂[r, g, :] = sum_{h in g} Q_r[r, h, :] / (||Q_r[r, h]|| h_qr) (bf16, per call).
+// Then s[c, r] = <K̂_r[c, :], q̂[r, :]> over the full h_kv * d row is exactly the head-mean
+// cosine up to the bf16 rounding of the two unit operands.
+//
+// Kernel (one CTA per SM, persistent over work units = 128 chunks x one tile of query rows):
+//   warp 0     : TMA producer (cp.async.bulk.tensor 2-D, 128-byte swizzle, no multicast)
+//                of 64-wide K slices of K̂_r (128 rows) and q̂ (N rows) into a 4-stage ring;
+//   warp 1     : one elected thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32,
+//                M = 128, N <= 256, K = 16) into one of two TMEM accumulators and commits to
+//                mbarriers (stage free / accumulator full);
+//   warps 2-5  : epilogue; each thread owns one chunk row (its TMEM lane), reads the
+//                accumulator with tcgen05.ld, takes the max over each query's T columns and
+//                writes chunk scores m[b, c] (fp32, coalesced over c).
+// A second kernel turns chunk scores into document scores and the exact top-k with the same
+// per-CTA warp-register lists and last-CTA merge as the CUDA-core scan.
+// Every wait is bounded; on expiry the CTA records an error in the workspace status word,
+// stops issuing work, drains what it issued and frees its TMEM.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace msa {
+
+constexpr int kTcStages = 4;
+constexpr int kTcBM = 128;        // chunks per tile (TMEM lanes)
+constexpr int kTcBK = 64;         // K slice (128 bytes of bf16: one swizzle row)
+constexpr int kTcThreads = 192;   // 6 warps
+
+// ------------------------------------------------------------------ PTX wrappers (sm_100a)
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand tile [rows][64 bf16] with the 128-byte swizzle: 8-row groups 1024 bytes
+// apart (SBO), leading offset unused for swizzled K-major (1), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(const void* tile) {
+  const uint64_t a = (uint64_t)(smem_u32(tile) & 0x3FFFFu) >> 4;
+  return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// ------------------------------------------------------------------ bank / query prep
+// K̂_r rows: per (chunk, head) unit vectors in bf16 (zero rows stay zero). One warp per row.
+template <typename T>
+__global__ void __launch_bounds__(256) kr_normalize_kernel(const T* __restrict__ R, int64_t rows,
+                                                           int d, __nv_bfloat16* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp; r < rows; r += nw) {
+    float x[4];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = lane + 32 * j;
+      x[j] = e < d ? Elem<T>::to_f(R[r * d + e]) : 0.f;
+      s += x[j] * x[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv = s > 0.f ? 1.0f / sqrtf(s) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = lane + 32 * j;
+      if (e < d) out[r * d + e] = __float2bfloat16_rn(x[j] * inv);
+    }
+  }
+}
+
+// q̂ [rows, h_kv * d] bf16: one warp per (row, KV head).
+template <typename T>
+__global__ void __launch_bounds__(256) q_fold_kernel(const T* __restrict__ q, int rows, int h_qr,
+                                                     int h_kv, int d,
+                                                     __nv_bfloat16* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int m = h_qr / h_kv;
+  const float inv_h = 1.0f / (float)h_qr;
+  for (int64_t pr = warp; pr < (int64_t)rows * h_kv; pr += nw) {
+    const int64_t r = pr / h_kv;
+    const int g = (int)(pr % h_kv);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int hm = 0; hm < m; ++hm) {
+      const T* qh = q + (r * h_qr + g * m + hm) * d;
+      float x[4];
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = lane + 32 * j;
+        x[j] = e < d ? Elem<T>::to_f(qh[e]) : 0.f;
+        s += x[j] * x[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const float sc = s > 0.f ? (1.0f / sqrtf(s)) * inv_h : 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] += x[j] * sc;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = lane + 32 * j;
+      if (e < d) out[(r * h_kv + g) * d + e] = __float2bfloat16_rn(acc[j]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ tcgen05 scoring GEMM
+struct TcParams {
+  int64_t n_chunks;
+  int K;                 // h_kv * d (multiple of 64)
+  int rows;              // B * T
+  int B, T, NQ, N;       // queries per row tile, row-tile width (multiple of 16, <= 256)
+  int64_t n_units, n_qtiles;
+  float* mscore;         // [B, n_chunks]
+  int* err;
+};
+
+__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* err,
+                                             volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_wait_bounded(bar, par, err)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                TcParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned operand ring: stage s = A (128 x 64) then B (N x 64)
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t a_bytes = kTcBM * kTcBK * 2;
+  const uint32_t b_bytes = (uint32_t)p.N * kTcBK * 2;
+  const uint32_t stage_bytes = (a_bytes + b_bytes + 1023) & ~1023u;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * stage_bytes);
+  uint64_t* empty = full + kTcStages;
+  uint64_t* tfull = empty + kTcStages;   // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* done = tempty + 2;           // MMA issuer: every issued MMA has completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_k = p.K / kTcBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {  // two fp32 accumulators of up to 256 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
+        const int y_a = (int)(ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
+        for (int kk = 0; kk < n_k; ++kk) {
+          if (issued >= kTcStages && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
+          unsigned char* st = base + (size_t)s * stage_bytes;
+          mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+          tma_load_2d(st, &map_k, kk * kTcBK, y_a, &full[s]);
+          tma_load_2d(st + a_bytes, &map_q, kk * kTcBK, y_b, &full[s]);
+          ++issued;
+          if (++s == kTcStages) { s = 0; ph ^= 1u; }
+        }
+        if (*abort_flag) break;
+      }
+      // drain: every issued stage must have landed before the CTA may exit
+      for (int64_t j = (issued > kTcStages ? issued - kTcStages : 0); j < issued; ++j)
+        mbar_wait_bounded(&full[j % kTcStages], (uint32_t)((j / kTcStages) & 1), p.err);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.N >> 3) << 17) |
+                             ((uint32_t)(kTcBM >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t local = 0;
+      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++local) {
+        const int a = (int)(local & 1);
+        const uint32_t aph = (uint32_t)((local >> 1) & 1);
+        if (local >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(a * 256);
+        bool ok = true;
+        for (int kk = 0; kk < n_k; ++kk) {
+          if (!wait_or_fail(&full[s], ph, p.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          unsigned char* st = base + (size_t)s * stage_bytes;
+          const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + a_bytes);
+#pragma unroll
+          for (int j = 0; j < kTcBK / 16; ++j)  // K = 16 per instruction: +32 bytes
+            tc_mma(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk | j) ? 1u : 0u);
+          tc_commit(&empty[s]);
+          if (++s == kTcStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[a]);
+      }
+      // every issued MMA must complete before the accumulators can be freed
+      tc_commit(done);
+      mbar_wait_bounded(done, 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 -> TMEM lane groups 2, 3, 0, 1)
+    const int lg = warp & 3;
+    int64_t local = 0;
+    for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++local) {
+      const int a = (int)(local & 1);
+      const uint32_t aph = (uint32_t)((local >> 1) & 1);
+      if (!wait_or_fail(&tfull[a], aph, p.err, abort_flag)) break;
+      tc_fence_after();
+      const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
+      const int64_t c = ct * kTcBM + lg * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
+      int q = 0, t = 0;
+      float cur = -INFINITY;
+      const int ncols = p.NQ * p.T;
+      for (int col = 0; col < ncols; col += 32) {
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)col, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (col + j < ncols) {
+            cur = fmaxf(cur, v[j]);
+            if (++t == p.T) {
+              const int64_t b = qt * p.NQ + q;
+              if (b < p.B && c < p.n_chunks) p.mscore[b * p.n_chunks + c] = cur;
+              cur = -INFINITY;
+              t = 0;
+              ++q;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[a]);
+    }
+  }
+
+  // ---------------- teardown: all MMAs completed (issuer waited on `done`) before TMEM is freed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+}
+
+// ------------------------------------------------------------------ documents + top-k
+// Chunk scores m[b, c] -> document max -> exact top-k (warp-register lists per CTA, last CTA
+// merges). Grid: persistent CTAs over document-aligned chunk ranges; warp w serves queries
+// w, w + 8, ...
+__device__ __forceinline__ void list_insert_tc(unsigned long long& li, unsigned long long key,
+                                               int lane, int k) {
+  const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
+  unsigned m = __ballot_sync(0xffffffffu, key > thr);
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    const unsigned long long x = __shfl_sync(0xffffffffu, key, src);
+    const unsigned gt = __ballot_sync(0xffffffffu, lane < k && li > x);
+    const int pos = __popc(gt);
+    const unsigned long long up = __shfl_up_sync(0xffffffffu, li, 1);
+    if (pos < k) {
+      if (lane > pos && lane < k) li = up;
+      if (lane == pos) li = x;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) doc_topk_kernel(DocTopkParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int last;
+  const int64_t G = gridDim.x, i = blockIdx.x;
+  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (i * p.n_chunks) / G);
+  const int64_t D1 = (i == G - 1) ? p.n_docs
+                                  : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
+  for (int b = warp; b < p.B; b += 8) {
+    unsigned long long lst = 0ull;
+    const float* mb = p.mscore + (int64_t)b * p.n_chunks;
+    for (int64_t dd = D0; dd < D1; dd += 32) {
+      const int64_t doc = dd + lane;
+      unsigned long long key = 0ull;
+      if (doc < D1) {
+        float sc = -INFINITY;
+        for (int64_t c = p.coff[doc]; c < p.coff[doc + 1]; ++c) sc = fmaxf(sc, mb[c]);
+        if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = sc;
+        const bool ex = p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
+        if (!ex) key = score_key(sc, (uint32_t)doc);
+      }
+      list_insert_tc(lst, key, lane, p.k);
+    }
+    if (lane < p.k) p.cand[(i * p.B + b) * p.k + lane] = lst;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicInc(p.counter, (unsigned)(G - 1)) == (unsigned)(G - 1));
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int64_t total = G * p.k;
+  for (int b = warp; b < p.B; b += 8) {
+    unsigned long long lst = 0ull;
+    for (int64_t base = 0; base < total; base += 32) {
+      const int64_t idx = base + lane;
+      unsigned long long key = 0ull;
+      if (idx < total) key = __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k);
+      list_insert_tc(lst, key, lane, p.k);
+    }
+    if (lane < p.k) {
+      p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
+      p.top_scores[b * p.k + lane] = lst ? key_score(lst) : -INFINITY;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, cols] row-major matrix, box {64, box_rows}, 128B swizzle.
+static bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, int k, int sms) {
+  TcPlan pl{};
+  pl.ok = (T >= 1 && T <= 256 && (h_kv * d) % kTcBK == 0);
+  if (!pl.ok) return pl;
+  pl.NQ = std::max(1, 256 / T);
+  if (pl.NQ > B) pl.NQ = B;
+  pl.N = ((pl.NQ * T + 15) / 16) * 16;
+  if (pl.N < 16) pl.N = 16;
+  pl.n_qtiles = (B + pl.NQ - 1) / pl.NQ;
+  pl.n_ctiles = (n_chunks + kTcBM - 1) / kTcBM;
+  pl.grid = (int)std::min<int64_t>(sms, std::max<int64_t>(1, pl.n_ctiles * pl.n_qtiles));
+  pl.topk_grid = (int)std::min<int64_t>((int64_t)sms, std::max<int64_t>(1, n_chunks / 256));
+  const size_t rows = (size_t)B * T;
+  pl.q_bytes = ((rows * h_kv * d * 2) + 255) & ~(size_t)255;
+  pl.m_bytes = (((size_t)B * n_chunks * 4) + 255) & ~(size_t)255;
+  pl.cand_bytes = (((size_t)pl.topk_grid * B * k * 8) + 255) & ~(size_t)255;
+  const size_t stage = (((size_t)kTcBM * kTcBK * 2 + (size_t)pl.N * kTcBK * 2) + 1023) & ~(size_t)1023;
+  pl.smem = 1024 + kTcStages * stage + 256;
+  (void)n_docs;
+  return pl;
+}
+
+cudaError_t launch_kr_normalize(const void* R, int64_t n_chunks, int h_kv, int d, int dtype,
+                                void* out, int sms, cudaStream_t st) {
+  const int64_t rows = n_chunks * h_kv;
+  if (rows == 0) return cudaSuccess;
+  int64_t grid = (rows * 32 + 255) / 256;
+  if (grid > (int64_t)sms * 32) grid = (int64_t)sms * 32;
+  if (dtype == 1)
+    kr_normalize_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(R), rows, d, static_cast<__nv_bfloat16*>(out));
+  else
+    kr_normalize_kernel<float><<<(unsigned)grid, 256, 0, st>>>(
+        static_cast<const float*>(R), rows, d, static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t st) {
+  // 1. fold the router queries into per-KV-head unit rows (bf16)
+  const int rows = a.B * a.T;
+  int64_t qgrid = ((int64_t)rows * a.h_kv * 32 + 255) / 256;
+  if (qgrid > 4096) qgrid = 4096;
+  if (a.dtype == 1)
+    q_fold_kernel<__nv_bfloat16><<<(unsigned)qgrid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(a.Q_r), rows, a.h_qr, a.h_kv, a.d, a.q_hat);
+  else
+    q_fold_kernel<float><<<(unsigned)qgrid, 256, 0, st>>>(static_cast<const float*>(a.Q_r), rows,
+                                                          a.h_qr, a.h_kv, a.d, a.q_hat);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 2. tensor-core scores -> chunk scores
+  CUtensorMap mk, mq;
+  const int K = a.h_kv * a.d;
+  if (!make_map(&mk, a.Kr_hat, a.n_chunks, K, kTcBM) || !make_map(&mq, a.q_hat, rows, K, pl.N))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.n_chunks = a.n_chunks;
+  p.K = K;
+  p.rows = rows;
+  p.B = a.B;
+  p.T = a.T;
+  p.NQ = pl.NQ;
+  p.N = pl.N;
+  p.n_qtiles = pl.n_qtiles;
+  p.n_units = pl.n_ctiles * pl.n_qtiles;
+  p.mscore = a.mscore;
+  p.err = a.err;
+  e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)pl.smem);
+  if (e != cudaSuccess) return e;
+  route_tc_kernel<<<pl.grid, kTcThreads, pl.smem, st>>>(mk, mq, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 3. documents + top-k
+  DocTopkParams t{};
+  t.mscore = a.mscore;
+  t.coff = a.coff;
+  t.excl = a.excl;
+  t.n_docs = a.n_docs;
+  t.n_chunks = a.n_chunks;
+  t.words = (a.n_docs + 31) / 32;
+  t.B = a.B;
+  t.k = a.k;
+  t.top_ids = a.top_ids;
+  t.top_scores = a.top_scores;
+  t.doc_scores = a.doc_scores;
+  t.cand = a.cand;
+  t.counter = a.counter;
+  doc_topk_kernel<<<pl.topk_grid, 256, 0, st>>>(t);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

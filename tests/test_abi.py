@@ -70,18 +70,24 @@ def test_encode_rejects_bad_arguments_on_host(msa):
 
 def test_route_rejects_bad_arguments_on_host(msa):
     fake = ctypes.c_void_p(256)
-    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, fake, 10, 80, 8, 128, 1, 11, None, fake,
+    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, None, fake, 10, 80, 8, 128, 1, 11, None, fake,
                                fake, None, fake, 1 << 20, None)
     assert r == 1 and b"k 11" in msa.lib.msa_last_error()          # k > n_docs
-    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, fake, 100, 800, 8, 128, 1, 33, None,
+    r = msa.lib.msa_route_topk(fake, 2, 1, 8, fake, fake, None, fake, 100, 800, 8, 128, 1, 33, None,
                                fake, fake, None, fake, 1 << 20, None)
     assert r == 2                                                   # k > 32 unsupported
-    r = msa.lib.msa_route_topk(fake, 2, 1, 6, fake, fake, fake, 100, 800, 8, 128, 1, 4, None, fake,
+    r = msa.lib.msa_route_topk(fake, 2, 1, 6, fake, fake, None, fake, 100, 800, 8, 128, 1, 4, None, fake,
                                fake, None, fake, 1 << 20, None)
     assert r == 1                                                   # h_qr % h_kv
-    r = msa.lib.msa_route_topk(fake, 1, 64, 8, fake, fake, fake, 100, 800, 8, 128, 1, 4, None,
+    r = msa.lib.msa_route_topk(fake, 1, 64, 8, fake, fake, None, fake, 100, 800, 8, 128, 1, 4, None,
                                fake, fake, None, fake, 1 << 20, None)
-    assert r == 2                                                   # long query: tensor path
+    assert r == 1                                                   # long query needs Kbar_r_hat
+    r = msa.lib.msa_route_topk(fake, 1, 64, 8, fake, fake, fake, fake, 100, 800, 8, 128, 0, 4, None,
+                               fake, fake, None, fake, 1 << 20, None)
+    assert r == 2                                                   # long fp32 query
+    r = msa.lib.msa_route_topk(fake, 1, 300, 8, fake, fake, fake, fake, 100, 800, 8, 128, 1, 4,
+                               None, fake, fake, None, fake, 1 << 20, None)
+    assert r == 2                                                   # T > 256
 
 
 def test_attend_and_gather_reject_bad_arguments_on_host(msa):

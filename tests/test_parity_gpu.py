@@ -435,3 +435,74 @@ def test_pipeline_tiny_config(msa, gpu, w):
     if set(ids.cpu().numpy()[0].tolist()) == set(ref["top_ids"][0].tolist()):
         assert np.array_equal(gi.cpu().numpy(), ref["gather_idx"])
         check_attention(O, ref["O64"], w.dtype)
+
+
+# ----------------------------------------------------------------------------- tensor-core scan
+def _route_tc_check(msa, gpu, Qr, Krb, coff, k, exclude=None):
+    """Long queries: bf16 tensor-core scan from the normalised bank; scores within the bf16
+    tolerance, exact top-k under the gap rule."""
+    Q_r, K_r = to_dev(Qr, gpu), to_dev(Krb, gpu)
+    cof = torch.from_numpy(np.ascontiguousarray(coff, np.int64)).to(gpu)
+    inv = msa.kr_inv_norm(K_r)
+    hat = msa.kr_normalize(K_r)
+    ex = None if exclude is None else torch.from_numpy(exclude.view(np.int32)).to(gpu)
+    ws = torch.zeros(msa.msa_route_topk_workspace(Qr.shape[0], Qr.shape[1], Qr.shape[2],
+                                                  Krb.shape[1], Krb.shape[2], 1, len(coff) - 1,
+                                                  Krb.shape[0], k), dtype=torch.uint8, device=gpu)
+    ids, sc, ds = msa.route_topk(Q_r, K_r, inv, cof, k, exclude_bits=ex, doc_scores=True, ws=ws,
+                                 Kbar_r_hat=hat)
+    torch.cuda.synchronize()
+    assert msa.msa_workspace_status(ws) == 0
+    r_ids, r_sc, r_ds = oracle.route(Qr, Krb, coff, k, exclude)
+    gds = ds.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(r_ds)
+    assert np.array_equal(np.isfinite(gds), fin)
+    err = np.max(np.abs(gds[fin] - r_ds[fin]), initial=0.0)
+    assert err <= SCORE_TOL["bf16"], err
+    masked = r_ds.copy()
+    if exclude is not None:
+        for b in range(masked.shape[0]):
+            for i in range(masked.shape[1]):
+                if (exclude[b, i // 32] >> (i % 32)) & 1:
+                    masked[b, i] = -np.inf
+    check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), r_ids, r_sc, masked,
+               SCORE_TOL["bf16"])
+    return ids.cpu().numpy(), err
+
+
+@pytest.mark.parametrize("B,T,n_docs,ragged", [
+    (1, 128, 300, True),     # 1M-bank prefill shape, partial last chunk tile
+    (3, 40, 150, False),     # several queries per row tile, padded N
+    (2, 256, 200, True),     # interleave-round query length, one query per tile
+    (1, 17, 5, False),       # shortest query on the tensor path, fewer chunks than a tile
+])
+def test_route_tensor_core_matches_oracle(msa, gpu, B, T, n_docs, ragged):
+    w = synth.C5.scaled(n_docs=n_docs, B=B, T=T, ragged=ragged, seed=T + B, k=min(8, n_docs),
+                        n_planted=1)
+    inp = synth.make_bank_workload(w)
+    ids, err = _route_tc_check(msa, gpu, inp["Q_r"], inp["Kbar_r"], inp["doc_chunk_off"], w.k)
+    assert np.array_equal(ids[:, 0], inp["planted"][:, 0])
+
+
+def test_route_tensor_core_head_groups_and_exclusion(msa, gpu):
+    rng = np.random.default_rng(12)
+    lens = rng.integers(0, 700, 90)
+    lens[[3, 89]] = 0
+    coff = synth.chunk_offsets_from_lengths(lens, 64)
+    Krb = synth.normal(3, 5, (int(coff[-1]), 4, 128), "bf16")
+    Qr = synth.normal(3, 6, (2, 64, 8, 128), "bf16")  # h_qr = 2 * h_kv
+    ex = np.zeros((2, 3), np.uint32)
+    ex[0, 0] = 0xF0F0F0F0
+    ex[1, 2] = 0x3FFFFFF
+    _route_tc_check(msa, gpu, Qr, Krb, coff, 12, exclude=ex)
+
+
+def test_route_tensor_core_full_1m_token_bank(msa, gpu):
+    """Routing at the 1M-token-bank size (16,384 chunks, 8 KV heads, d=128) for a 128-token
+    query, on a synthetic pooled bank; every document score against the oracle."""
+    w = synth.C5.scaled(n_docs=1024, doc_len=1024, B=1, T=128, k=16, n_planted=1, seed=21)
+    dv = synth.dev_bank_workload(w, gpu, with_kv=False)
+    coff = dv["doc_chunk_off"]
+    Krb = synth.host_bank_rows(w, "Kbar_r", 0, dv["n_chunks"], coff=coff, Q_r=dv["Q_r_host"])
+    ids, err = _route_tc_check(msa, gpu, dv["Q_r_host"], Krb, coff, w.k)
+    assert ids[0, 0] == dv["planted"][0, 0]
