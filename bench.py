@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m", choices=["bank100m", "bank10m"])
     ap.add_argument("--fetch", default="memcpy", choices=["memcpy", "zerocopy"])
+    ap.add_argument("--scan", default="tc", choices=["tc", "cc"],
+                    help="router scan: tensor cores over the normalised bank, or CUDA cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=3,
                     help="routed layers in the CPU-oracle sample")
@@ -118,7 +120,7 @@ class ClockSampler:
 class Decode:
     """Routed decode over a memory bank: per layer route -> fetch/gather -> attend."""
 
-    def __init__(self, w, dev, fetch: str, rank: int):
+    def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc"):
         import torch
 
         import long_context_doc_b200 as msa
@@ -134,6 +136,7 @@ class Decode:
         for l in range(self.L):
             dv = synth.dev_bank_workload(seed_w, dev, layer=l, with_kv=(self.fetch == "device"))
             dv["inv"] = msa.kr_inv_norm(dv["Kbar_r"])
+            dv["hat"] = msa.kr_normalize(dv["Kbar_r"]) if scan == "tc" else None
             self.layers.append(dv)
         self.coff_host = self.layers[0]["doc_chunk_off"]
         self.coff = torch.from_numpy(self.coff_host).to(dev)
@@ -176,10 +179,11 @@ class Decode:
         self.O = [torch.empty((B, w.T, w.h_q, w.d), dtype=torch.bfloat16, device=dev)
                   for _ in range(self.L)]
         self.route_ev = None
-        # kernels per step (own kernels only; memsets and copies excluded)
-        att_plan_S = 1
-        self.kernels_per_layer = 1 + 1 + 1 + 1  # route scan, gather, rope table, attend
-        from long_context_doc_b200 import msa_sparse_attend_workspace  # noqa: F401
+        self.scan = scan
+        # own kernels per layer (memsets and copies excluded): route (tensor path: query fold,
+        # scan, document top-k; CUDA-core path: one fused kernel), gather indices, RoPE table,
+        # attention, split combine
+        self.kernels_per_layer = (3 if scan == "tc" else 1) + 1 + 1 + 1 + 1
 
     # per-layer pieces -------------------------------------------------------------
     def route(self, l):
@@ -187,7 +191,7 @@ class Decode:
         if self.route_ev is not None:
             self.route_ev[l][0].record(self.main)
         msa.msa_route_topk(d["Q_r"], d["Kbar_r"], d["inv"], self.coff, self.w.k, None, bf["ids"],
-                           bf["sc"], None, bf["ws_r"], self.main)
+                           bf["sc"], None, bf["ws_r"], self.main, d["hat"])
         if self.route_ev is not None:
             self.route_ev[l][1].record(self.main)
 
@@ -226,7 +230,11 @@ class Decode:
             self.attend(l)
 
     def scan_bytes(self):
+        """Algorithmic bytes of one routing call: the bank it streams (K̂_r for the tensor
+        path; K̄_r plus fp32 inverse norms for the CUDA-core path)."""
         w = self.w
+        if self.scan == "tc":
+            return self.n_chunks * w.h_kv * w.d * 2 + 2 * w.B * self.n_chunks * 4
         return self.n_chunks * w.h_kv * w.d * 2 + self.n_chunks * w.h_kv * 4
 
 
@@ -244,7 +252,7 @@ def run_libmsa(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
     w = synth.C4 if args.workload == "bank100m" else synth.C3
-    wk = Decode(w, dev, args.fetch, rank)
+    wk = Decode(w, dev, args.fetch, rank, args.scan)
     torch.cuda.synchronize()
 
     def barrier():
@@ -339,9 +347,11 @@ def run_libmsa(args):
                                f"fetch={wk.fetch}") if wk.fetch != "device" else "HBM",
                    "l2": "no flush: every layer scans a 3.28 GB K̄_r, far larger than the 126 MB L2"
                    if wk.L > 1 else "no flush: the 328 MB K̄_r scan exceeds the 126 MB L2",
-                   "parallelism": f"replicas x{world}"},
+                   "scan": wk.scan, "parallelism": f"replicas x{world}"},
         "router_scan_gbs": round(achieved, 1),
-        "roofline": {"kernel": "route_scan (msa_route_topk: scan + fused top-k)", "bound": "hbm",
+        "roofline": {"kernel": ("msa_route_topk (tensor-core scan: query fold + tcgen05 scan + "
+                               "document top-k)" if wk.scan == "tc" else
+                               "msa_route_topk (CUDA-core scan with fused top-k)"), "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "traffic": None, "bytes_per_launch": wk.scan_bytes(),

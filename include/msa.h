@@ -127,10 +127,11 @@ msa_status msa_kr_normalize(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, 
  * Kbar_r     [n_chunks, h_kv, d] router-key bank (dtype), 16-byte aligned.
  * kr_inv_norm [n_chunks, h_kv] fp32 inverse norms (from msa_encode_pool / msa_kr_inv_norm).
  * Kbar_r_hat (nullable) [n_chunks, h_kv, d] bf16 per-head unit rows (msa_kr_normalize).
- *            Queries with T <= 16 are scored on CUDA cores from Kbar_r and kr_inv_norm in
- *            fp32 (B*T rows in passes of up to 16). Longer queries (17 <= T <= 256, bf16
- *            banks) are scored on the tensor cores as one bf16 contraction of Kbar_r_hat with
- *            the per-head normalised queries (fp32 accumulation); Kbar_r_hat is required there.
+ *            With Kbar_r_hat and a bf16 bank, every query length is scored on the tensor
+ *            cores as one bf16 contraction of Kbar_r_hat with the per-head normalised queries
+ *            (fp32 accumulation; Kbar_r and kr_inv_norm are not read). Without it, queries
+ *            with T <= 16 are scored on CUDA cores from Kbar_r and kr_inv_norm in fp32 (B*T rows
+ *            in passes of up to 16); longer queries (17 <= T <= 256) require Kbar_r_hat.
  * doc_chunk_off [n_docs+1] device int64 chunk offsets (non-decreasing, ends at n_chunks).
  * Score of doc i for query b:
  *     S[b,i] = max_{c in doc i} max_t (1/h_qr) sum_h cos(Q_r[b,t,h], Kbar_r[c, g(h)])

@@ -159,18 +159,19 @@ msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, i
 size_t msa_route_topk_workspace(int32_t B, int32_t T, int32_t h_qr, int32_t h_kv, int32_t d,
                                 int32_t dtype, int64_t n_docs, int64_t n_chunks, int32_t k) {
   if (B < 1 || T < 1 || k < 1 || h_kv < 1 || d < 1) return kHeader;
-  if (T > 16) {
+  size_t tc = kHeader;
+  if (dtype == MSA_BF16) {  // the tensor-core scan may serve any bf16 query length
     const msa::TcPlan pl = msa::tc_plan(B, T, h_kv, d, n_docs, n_chunks, k, sm_count());
-    if (!pl.ok) return kHeader;
-    return kHeader + pl.q_bytes + pl.m_bytes + pl.cand_bytes;
+    if (pl.ok) tc = kHeader + pl.q_bytes + pl.m_bytes + pl.cand_bytes;
   }
+  if (T > 16) return tc;
   int bp, passes;
   route_passes(B, T, &bp, &passes);
   const msa::RouteChoice c = msa::route_choose(dtype, bp * T, h_kv * d);
   if (c.R == 0) return kHeader;
   const int grid = msa::route_grid(dtype, c, h_kv * d, h_kv, h_qr, sm_count(), n_chunks);
-  if (grid < 1) return kHeader;
-  return kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long);
+  if (grid < 1) return tc;
+  return std::max(tc, kHeader + (size_t)passes * grid * bp * k * sizeof(unsigned long long));
 }
 
 msa_status msa_kr_normalize(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
@@ -212,7 +213,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
   REQUIRE(Q_r && Kbar_r && kr_inv_norm && doc_chunk_off && top_ids && top_scores,
           MSA_ERR_INVALID_ARG, "null tensor");
   REQUIRE(aligned16(Kbar_r), MSA_ERR_INVALID_ARG, "Kbar_r must be 16-byte aligned");
-  if (T > 16) {
+  if (T > 16 || (dtype == MSA_BF16 && Kbar_r_hat != nullptr)) {
     REQUIRE(aligned16(Kbar_r_hat) && aligned16(Q_r), MSA_ERR_INVALID_ARG,
             "Kbar_r_hat and Q_r must be 16-byte aligned");
     const msa::TcPlan pl = msa::tc_plan(B, T, h_kv, d, n_docs, n_chunks, k, sm_count());

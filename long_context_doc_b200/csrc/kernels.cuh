@@ -64,7 +64,7 @@ struct DocTopkParams {
 };
 struct TcPlan {
   bool ok;
-  int NQ, N, grid, topk_grid;
+  int NQ, N, grid, topk_grid, stages;
   int64_t n_qtiles, n_ctiles;
   size_t q_bytes, m_bytes, cand_bytes, smem;
 };

@@ -33,7 +33,8 @@
 
 namespace msa {
 
-constexpr int kTcStages = 4;
+constexpr int kTcMaxStages = 12;
+constexpr size_t kTcSmemBudget = 200 * 1024;  // operand ring
 constexpr int kTcBM = 128;        // chunks per tile (TMEM lanes)
 constexpr int kTcBK = 64;         // K slice (128 bytes of bf16: one swizzle row)
 constexpr int kTcThreads = 192;   // 6 warps
@@ -172,6 +173,7 @@ struct TcParams {
   int K;                 // h_kv * d (multiple of 64)
   int rows;              // B * T
   int B, T, NQ, N;       // queries per row tile, row-tile width (multiple of 16, <= 256)
+  int stages;            // operand ring depth (<= kTcMaxStages)
   int64_t n_units, n_qtiles;
   float* mscore;         // [B, n_chunks]
   int* err;
@@ -195,9 +197,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   const uint32_t a_bytes = kTcBM * kTcBK * 2;
   const uint32_t b_bytes = (uint32_t)p.N * kTcBK * 2;
   const uint32_t stage_bytes = (a_bytes + b_bytes + 1023) & ~1023u;
+  const int kTcStages = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * stage_bytes);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* tfull = empty + kTcStages;   // [2]
+  uint64_t* empty = full + kTcMaxStages;
+  uint64_t* tfull = empty + kTcMaxStages;  // [2]
   uint64_t* tempty = tfull + 2;          // [2]
   uint64_t* done = tempty + 2;           // MMA issuer: every issued MMA has completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
@@ -451,7 +454,8 @@ TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, 
   pl.m_bytes = (((size_t)B * n_chunks * 4) + 255) & ~(size_t)255;
   pl.cand_bytes = (((size_t)pl.topk_grid * B * k * 8) + 255) & ~(size_t)255;
   const size_t stage = (((size_t)kTcBM * kTcBK * 2 + (size_t)pl.N * kTcBK * 2) + 1023) & ~(size_t)1023;
-  pl.smem = 1024 + kTcStages * stage + 256;
+  pl.stages = (int)std::min<size_t>(kTcMaxStages, kTcSmemBudget / stage);
+  pl.smem = 1024 + pl.stages * stage + 512;
   (void)n_docs;
   return pl;
 }
@@ -497,6 +501,7 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t
   p.T = a.T;
   p.NQ = pl.NQ;
   p.N = pl.N;
+  p.stages = pl.stages;
   p.n_qtiles = pl.n_qtiles;
   p.n_units = pl.n_ctiles * pl.n_qtiles;
   p.mscore = a.mscore;

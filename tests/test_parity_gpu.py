@@ -481,7 +481,30 @@ def test_route_tensor_core_matches_oracle(msa, gpu, B, T, n_docs, ragged):
                         n_planted=1)
     inp = synth.make_bank_workload(w)
     ids, err = _route_tc_check(msa, gpu, inp["Q_r"], inp["Kbar_r"], inp["doc_chunk_off"], w.k)
+    if T <= 16:  # a long query's mean direction is nearly orthogonal to each of its tokens
+        assert np.array_equal(ids[:, 0], inp["planted"][:, 0])
+
+
+@pytest.mark.parametrize("B,T,n_docs,ragged", [
+    (8, 1, 3000, False),     # 10M-bank decode batch shape
+    (4, 1, 2501, True),      # 100M-bank decode batch shape, ragged docs
+    (40, 1, 700, False),     # wide decode batch: one 48-column tile
+    (3, 5, 400, True),       # short multi-token queries
+])
+def test_route_tensor_core_decode_matches_oracle(msa, gpu, B, T, n_docs, ragged):
+    w = synth.C3.scaled(n_docs=n_docs, B=B, T=T, ragged=ragged, seed=100 + B + T)
+    inp = synth.make_bank_workload(w)
+    ids, err = _route_tc_check(msa, gpu, inp["Q_r"], inp["Kbar_r"], inp["doc_chunk_off"], w.k)
     assert np.array_equal(ids[:, 0], inp["planted"][:, 0])
+
+
+def test_route_tensor_core_full_10m_token_bank_decode(msa, gpu):
+    w = synth.C3
+    dv = synth.dev_bank_workload(w, gpu, with_kv=False)
+    coff = dv["doc_chunk_off"]
+    Krb = synth.host_bank_rows(w, "Kbar_r", 0, dv["n_chunks"], coff=coff, Q_r=dv["Q_r_host"])
+    ids, err = _route_tc_check(msa, gpu, dv["Q_r_host"], Krb, coff, w.k)
+    assert np.array_equal(ids[:, 0], dv["planted"][:, 0])
 
 
 def test_route_tensor_core_head_groups_and_exclusion(msa, gpu):
