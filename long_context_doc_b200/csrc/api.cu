@@ -245,7 +245,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
     ta.top_scores = top_scores;
     ta.doc_scores = doc_scores;
     ta.q_hat = reinterpret_cast<__nv_bfloat16*>(base + kHeader);
-    ta.mscore = reinterpret_cast<float*>(base + kHeader + pl.q_bytes);
+    ta.mscore = nullptr;
     ta.cand = reinterpret_cast<unsigned long long*>(base + kHeader + pl.q_bytes + pl.m_bytes);
     ta.counter = reinterpret_cast<unsigned int*>(base) + 1;
     ta.err = reinterpret_cast<int*>(base);

@@ -50,18 +50,6 @@ int route_grid(int dtype, RouteChoice c, int W, int h_kv, int h_qr, int sms, int
 cudaError_t route_launch(int dtype, RouteChoice c, const RouteParams& p, int grid, cudaStream_t st);
 
 // ---- route_tc.cu (tensor-core scan for long queries)
-struct DocTopkParams {
-  const float* mscore;       // [B, n_chunks] chunk scores (max over tokens)
-  const int64_t* coff;
-  const uint32_t* excl;
-  int64_t n_docs, n_chunks, words;
-  int B, k;
-  int32_t* top_ids;
-  float* top_scores;
-  float* doc_scores;
-  unsigned long long* cand;  // [grid, B, k]
-  unsigned int* counter;
-};
 struct TcPlan {
   bool ok;
   int NQ, N, grid, topk_grid, stages;
@@ -79,7 +67,7 @@ struct RouteTcArgs {
   float* top_scores;
   float* doc_scores;
   __nv_bfloat16* q_hat;      // workspace [B*T, h_kv * d]
-  float* mscore;             // workspace [B, n_chunks]
+  float* mscore;             // unused (scores stay on chip)
   unsigned long long* cand;  // workspace
   unsigned int* counter;
   int* err;

@@ -11,17 +11,18 @@
 // Then s[c, r] = <K̂_r[c, :], q̂[r, :]> over the full h_kv * d row is exactly the head-mean
 // cosine up to the bf16 rounding of the two unit operands.
 //
-// Kernel (one CTA per SM, persistent over work units = 128 chunks x one tile of query rows):
+// Kernel (one CTA per SM; work units = 128 chunks x one tile of query rows):
 //   warp 0     : TMA producer (cp.async.bulk.tensor 2-D, 128-byte swizzle, no multicast)
 //                of 64-wide K slices of K̂_r (128 rows) and q̂ (N rows) into a 4-stage ring;
 //   warp 1     : one elected thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32,
 //                M = 128, N <= 256, K = 16) into one of two TMEM accumulators and commits to
 //                mbarriers (stage free / accumulator full);
 //   warps 2-5  : epilogue; each thread owns one chunk row (its TMEM lane), reads the
-//                accumulator with tcgen05.ld, takes the max over each query's T columns and
-//                writes chunk scores m[b, c] (fp32, coalesced over c).
-// A second kernel turns chunk scores into document scores and the exact top-k with the same
-// per-CTA warp-register lists and last-CTA merge as the CUDA-core scan.
+//                accumulator with tcgen05.ld and takes the max over each query's T columns.
+// Each CTA owns a document-aligned contiguous chunk range; once a chunk tile has been scored
+// against every query tile, the epilogue warps fold chunk scores into document maxima (with a
+// carry for documents that continue into the next tile) and keep an exact per-query top-k in
+// warp registers; the last CTA to finish merges the per-CTA candidates (no spinning).
 // Every wait is bounded; on expiry the CTA records an error in the workspace status word,
 // stops issuing work, drains what it issued and frees its TMEM.
 #include <cuda.h>
@@ -34,7 +35,6 @@
 namespace msa {
 
 constexpr int kTcMaxStages = 12;
-constexpr size_t kTcSmemBudget = 200 * 1024;  // operand ring
 constexpr int kTcBM = 128;        // chunks per tile (TMEM lanes)
 constexpr int kTcBK = 64;         // K slice (128 bytes of bf16: one swizzle row)
 constexpr int kTcThreads = 192;   // 6 warps
@@ -167,180 +167,24 @@ __global__ void __launch_bounds__(256) q_fold_kernel(const T* __restrict__ q, in
   }
 }
 
-// ------------------------------------------------------------------ tcgen05 scoring GEMM
+// ------------------------------------------------------------------ tcgen05 scoring + top-k
 struct TcParams {
-  int64_t n_chunks;
+  const int64_t* coff;   // [n_docs + 1]
+  const uint32_t* excl;  // nullable [B, words]
+  int64_t n_docs, n_chunks, words;
   int K;                 // h_kv * d (multiple of 64)
-  int rows;              // B * T
   int B, T, NQ, N;       // queries per row tile, row-tile width (multiple of 16, <= 256)
-  int stages;            // operand ring depth (<= kTcMaxStages)
-  int64_t n_units, n_qtiles;
-  float* mscore;         // [B, n_chunks]
+  int n_qtiles, stages, k;
+  int32_t* top_ids;      // [B, k]
+  float* top_scores;     // [B, k]
+  float* doc_scores;     // nullable [B, n_docs]
+  unsigned long long* cand;  // [grid, B, k]
+  unsigned int* counter;
   int* err;
 };
 
-__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* err,
-                                             volatile int* abort_flag) {
-  if (*abort_flag) return false;
-  if (mbar_wait_bounded(bar, par, err)) return true;
-  *abort_flag = 1;
-  return false;
-}
+constexpr int kTcWin = 1024;  // document offsets cached in shared memory
 
-__global__ void __launch_bounds__(kTcThreads, 1)
-route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
-                TcParams p) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte aligned operand ring: stage s = A (128 x 64) then B (N x 64)
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const uint32_t a_bytes = kTcBM * kTcBK * 2;
-  const uint32_t b_bytes = (uint32_t)p.N * kTcBK * 2;
-  const uint32_t stage_bytes = (a_bytes + b_bytes + 1023) & ~1023u;
-  const int kTcStages = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kTcStages * stage_bytes);
-  uint64_t* empty = full + kTcMaxStages;
-  uint64_t* tfull = empty + kTcMaxStages;  // [2]
-  uint64_t* tempty = tfull + 2;          // [2]
-  uint64_t* done = tempty + 2;           // MMA issuer: every issued MMA has completed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_k = p.K / kTcBK;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    mbar_init(done, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0) {  // two fp32 accumulators of up to 256 columns
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_holder)),
-                 "r"(512)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-
-  if (warp == 0) {
-    // ---------------- TMA producer
-    if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t issued = 0;
-      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-        const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-        const int y_a = (int)(ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
-        for (int kk = 0; kk < n_k; ++kk) {
-          if (issued >= kTcStages && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
-          unsigned char* st = base + (size_t)s * stage_bytes;
-          mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
-          tma_load_2d(st, &map_k, kk * kTcBK, y_a, &full[s]);
-          tma_load_2d(st + a_bytes, &map_q, kk * kTcBK, y_b, &full[s]);
-          ++issued;
-          if (++s == kTcStages) { s = 0; ph ^= 1u; }
-        }
-        if (*abort_flag) break;
-      }
-      // drain: every issued stage must have landed before the CTA may exit
-      for (int64_t j = (issued > kTcStages ? issued - kTcStages : 0); j < issued; ++j)
-        mbar_wait_bounded(&full[j % kTcStages], (uint32_t)((j / kTcStages) & 1), p.err);
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.N >> 3) << 17) |
-                             ((uint32_t)(kTcBM >> 4) << 24);
-      int s = 0;
-      uint32_t ph = 0;
-      int64_t local = 0;
-      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++local) {
-        const int a = (int)(local & 1);
-        const uint32_t aph = (uint32_t)((local >> 1) & 1);
-        if (local >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(a * 256);
-        bool ok = true;
-        for (int kk = 0; kk < n_k; ++kk) {
-          if (!wait_or_fail(&full[s], ph, p.err, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          unsigned char* st = base + (size_t)s * stage_bytes;
-          const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + a_bytes);
-#pragma unroll
-          for (int j = 0; j < kTcBK / 16; ++j)  // K = 16 per instruction: +32 bytes
-            tc_mma(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk | j) ? 1u : 0u);
-          tc_commit(&empty[s]);
-          if (++s == kTcStages) { s = 0; ph ^= 1u; }
-        }
-        if (!ok) break;
-        tc_commit(&tfull[a]);
-      }
-      // every issued MMA must complete before the accumulators can be freed
-      tc_commit(done);
-      mbar_wait_bounded(done, 0, p.err);
-    }
-  } else {
-    // ---------------- epilogue (warps 2..5 -> TMEM lane groups 2, 3, 0, 1)
-    const int lg = warp & 3;
-    int64_t local = 0;
-    for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++local) {
-      const int a = (int)(local & 1);
-      const uint32_t aph = (uint32_t)((local >> 1) & 1);
-      if (!wait_or_fail(&tfull[a], aph, p.err, abort_flag)) break;
-      tc_fence_after();
-      const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-      const int64_t c = ct * kTcBM + lg * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
-      int q = 0, t = 0;
-      float cur = -INFINITY;
-      const int ncols = p.NQ * p.T;
-      for (int col = 0; col < ncols; col += 32) {
-        float v[32];
-        tmem_ld32(tbase + (uint32_t)col, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (col + j < ncols) {
-            cur = fmaxf(cur, v[j]);
-            if (++t == p.T) {
-              const int64_t b = qt * p.NQ + q;
-              if (b < p.B && c < p.n_chunks) p.mscore[b * p.n_chunks + c] = cur;
-              cur = -INFINITY;
-              t = 0;
-              ++q;
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[a]);
-    }
-  }
-
-  // ---------------- teardown: all MMAs completed (issuer waited on `done`) before TMEM is freed
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
-                 : "memory");
-}
-
-// ------------------------------------------------------------------ documents + top-k
-// Chunk scores m[b, c] -> document max -> exact top-k (warp-register lists per CTA, last CTA
-// merges). Grid: persistent CTAs over document-aligned chunk ranges; warp w serves queries
-// w, w + 8, ...
 __device__ __forceinline__ void list_insert_tc(unsigned long long& li, unsigned long long key,
                                                int lane, int k) {
   const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
@@ -359,41 +203,283 @@ __device__ __forceinline__ void list_insert_tc(unsigned long long& li, unsigned 
   }
 }
 
-__global__ void __launch_bounds__(256) doc_topk_kernel(DocTopkParams p) {
+__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* err,
+                                             volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_wait_bounded(bar, par, err)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ void epi_sync() {  // the 128 epilogue threads only
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// Work of a CTA: the chunk tiles (128 rows from the CTA's first chunk) of its document-aligned
+// chunk range, each against every row tile of queries; units are (chunk tile, query tile),
+// query tiles innermost.
+__global__ void __launch_bounds__(kTcThreads, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                TcParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t a_bytes = kTcBM * kTcBK * 2;
+  const uint32_t b_bytes = (uint32_t)p.N * kTcBK * 2;
+  const uint32_t stage_bytes = (a_bytes + b_bytes + 1023) & ~1023u;
+  const int S = p.stages;
+  float* msc = reinterpret_cast<float*>(base + S * stage_bytes);                // [128][B]
+  int64_t* win = reinterpret_cast<int64_t*>(msc + kTcBM * p.B);                 // [kTcWin+1]
+  unsigned long long* lists = reinterpret_cast<unsigned long long*>(win + kTcWin + 1);  // [B][32]
+  float* carry = reinterpret_cast<float*>(lists + p.B * 32);                    // [B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(carry + ((p.B + 1) & ~1));       // [max]
+  uint64_t* empty = full + kTcMaxStages;
+  uint64_t* tfull = empty + kTcMaxStages;  // [2]
+  uint64_t* tempty = tfull + 2;            // [2]
+  uint64_t* done = tempty + 2;             // MMA issuer: every issued MMA has completed
+  int64_t* docs = reinterpret_cast<int64_t*>(done + 1);  // [0..1] current doc, [2] window start
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(docs + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* last_flag = const_cast<int*>(abort_flag) + 1;
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __shared__ int last;
-  const int64_t G = gridDim.x, i = blockIdx.x;
-  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (i * p.n_chunks) / G);
-  const int64_t D1 = (i == G - 1) ? p.n_docs
-                                  : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
-  for (int b = warp; b < p.B; b += 8) {
-    unsigned long long lst = 0ull;
-    const float* mb = p.mscore + (int64_t)b * p.n_chunks;
-    for (int64_t dd = D0; dd < D1; dd += 32) {
-      const int64_t doc = dd + lane;
-      unsigned long long key = 0ull;
-      if (doc < D1) {
-        float sc = -INFINITY;
-        for (int64_t c = p.coff[doc]; c < p.coff[doc + 1]; ++c) sc = fmaxf(sc, mb[c]);
-        if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = sc;
-        const bool ex = p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
-        if (!ex) key = score_key(sc, (uint32_t)doc);
-      }
-      list_insert_tc(lst, key, lane, p.k);
+  const int n_k = p.K / kTcBK;
+
+  // document-aligned chunk range of this CTA
+  const int64_t G = gridDim.x, ci = blockIdx.x;
+  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (ci * p.n_chunks) / G);
+  const int64_t D1 = (ci == G - 1) ? p.n_docs
+                                   : lower_bound_i64(p.coff, p.n_docs, ((ci + 1) * p.n_chunks) / G);
+  const int64_t cb = p.coff[D0], ce = p.coff[D1];
+  const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
+  const int64_t n_units = n_ct * p.n_qtiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    if (lane < p.k) p.cand[(i * p.B + b) * p.k + lane] = lst;
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    docs[0] = D0;
+    docs[2] = D0;
+    fence_mbar_init();
   }
+  for (int j = threadIdx.x; j <= kTcWin; j += kTcThreads)
+    win[j] = (D0 + j <= D1) ? p.coff[D0 + j] : INT64_MAX;
+  for (int j = threadIdx.x; j < p.B * 32; j += kTcThreads) lists[j] = 0ull;
+  for (int j = threadIdx.x; j < p.B; j += kTcThreads) carry[j] = -INFINITY;
+  if (warp == 0) {  // two fp32 accumulators of up to 256 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t u = 0; u < n_units; ++u) {
+        const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
+        const int y_a = (int)(cb + ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
+        for (int kk = 0; kk < n_k; ++kk) {
+          if (issued >= S && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
+          unsigned char* st = base + (size_t)s * stage_bytes;
+          mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+          tma_load_2d(st, &map_k, kk * kTcBK, y_a, &full[s]);
+          tma_load_2d(st + a_bytes, &map_q, kk * kTcBK, y_b, &full[s]);
+          ++issued;
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+        if (*abort_flag) break;
+      }
+      for (int64_t j = (issued > S ? issued - S : 0); j < issued; ++j)
+        mbar_wait_bounded(&full[j % S], (uint32_t)((j / S) & 1), p.err);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.N >> 3) << 17) |
+                             ((uint32_t)(kTcBM >> 4) << 24);
+      int s = 0;
+      uint32_t ph = 0;
+      for (int64_t u = 0; u < n_units; ++u) {
+        const int a = (int)(u & 1);
+        const uint32_t aph = (uint32_t)((u >> 1) & 1);
+        if (u >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(a * 256);
+        bool ok = true;
+        for (int kk = 0; kk < n_k; ++kk) {
+          if (!wait_or_fail(&full[s], ph, p.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          unsigned char* st = base + (size_t)s * stage_bytes;
+          const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + a_bytes);
+#pragma unroll
+          for (int j = 0; j < kTcBK / 16; ++j)  // K = 16 per instruction: +32 bytes
+            tc_mma(d_tmem, ad + 2 * j, bd + 2 * j, idesc, (kk | j) ? 1u : 0u);
+          tc_commit(&empty[s]);
+          if (++s == S) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[a]);
+      }
+      tc_commit(done);
+      mbar_wait_bounded(done, 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 -> TMEM lane groups 2, 3, 0, 1)
+    const int lg = warp & 3;
+    const int ew = warp - 2;                 // epilogue warp 0..3
+    const int row = lg * 32 + lane;          // chunk row of the tile (TMEM lane)
+    const int ncols = p.NQ * p.T;
+    bool aborted = false;
+    for (int64_t u = 0; u < n_units; ++u) {
+      const int a = (int)(u & 1);
+      const uint32_t aph = (uint32_t)((u >> 1) & 1);
+      const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
+      if (!wait_or_fail(&tfull[a], aph, p.err, abort_flag)) { aborted = true; break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
+      int q = 0, t = 0;
+      float cur = -INFINITY;
+      for (int col = 0; col < ncols; col += 32) {
+        float v[32];
+        tmem_ld32(tbase + (uint32_t)col, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (col + j < ncols) {
+            cur = fmaxf(cur, v[j]);
+            if (++t == p.T) {  // max over the query's tokens done
+              const int b = (int)qt * p.NQ + q;
+              if (b < p.B) msc[row * p.B + b] = cur;
+              cur = -INFINITY;
+              t = 0;
+              ++q;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[a]);
+      if (qt != p.n_qtiles - 1) continue;
+      // ---- chunk tile complete for every query: per-document max + top-k insertion
+      epi_sync();
+      const int64_t c0 = cb + ct * kTcBM;
+      const int64_t tend = min(c0 + kTcBM, ce);
+      const int64_t dcur = docs[ct & 1];
+      if (dcur + kTcBM + 2 > docs[2] + kTcWin) {  // slide the document-offset window
+        for (int j = ew * 32 + lane; j <= kTcWin; j += 128)
+          win[j] = (dcur + j <= D1) ? p.coff[dcur + j] : INT64_MAX;
+        epi_sync();
+        if (ew == 0 && lane == 0) docs[2] = dcur;
+        epi_sync();
+      }
+      const int64_t w0 = docs[2];
+      for (int b = ew; b < p.B; b += 4) {
+        unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
+        float cr = carry[b];
+        int64_t dd = dcur, next = dcur;
+        while (true) {
+          const int64_t doc = dd + lane;
+          bool valid = doc < D1;
+          int64_t ds = 0, de = 0;
+          if (valid) {
+            ds = (doc - w0 < kTcWin) ? win[doc - w0] : __ldg(p.coff + doc);
+            de = (doc + 1 - w0 <= kTcWin) ? win[doc + 1 - w0] : __ldg(p.coff + doc + 1);
+          }
+          valid = valid && ds < tend;
+          bool fin = false;
+          float sc = -INFINITY;
+          if (valid) {
+            const int lo = (int)(max(ds, c0) - c0), hi = (int)(min(de, tend) - c0);
+            for (int c = lo; c < hi; ++c) sc = fmaxf(sc, msc[c * p.B + b]);
+            if (ds < c0) sc = fmaxf(sc, cr);
+            fin = de <= tend;
+          }
+          unsigned long long key = 0ull;
+          if (fin) {
+            if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = sc;
+            const bool ex =
+                p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
+            if (!ex) key = score_key(sc, (uint32_t)doc);
+          }
+          list_insert_tc(lst, key, lane, p.k);
+          const unsigned cont = __ballot_sync(0xffffffffu, valid && !fin);
+          const unsigned vm = __ballot_sync(0xffffffffu, valid);
+          if (cont) {
+            const int src = __ffs(cont) - 1;
+            cr = __shfl_sync(0xffffffffu, sc, src);
+            next = dd + src;
+            break;
+          }
+          if (vm != 0xffffffffu) {
+            next = dd + __popc(vm);
+            break;
+          }
+          dd += 32;
+        }
+        if (lane < p.k) lists[b * 32 + lane] = lst;
+        if (lane == 0) carry[b] = cr;
+        if (b == 0 && lane == 0) docs[(ct + 1) & 1] = next;
+      }
+      epi_sync();  // msc and the document cursor are reused by the next chunk tile
+    }
+    if (!aborted) {  // documents without chunks at the end of the range score -inf
+      const int64_t dcur = docs[n_ct & 1];
+      for (int b = ew; b < p.B; b += 4) {
+        unsigned long long lst = lane < p.k ? lists[b * 32 + lane] : 0ull;
+        for (int64_t dd = dcur; dd < D1; dd += 32) {
+          const int64_t doc = dd + lane;
+          unsigned long long key = 0ull;
+          if (doc < D1) {
+            if (p.doc_scores) p.doc_scores[(int64_t)b * p.n_docs + doc] = -INFINITY;
+            const bool ex =
+                p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
+            if (!ex) key = score_key(-INFINITY, (uint32_t)doc);
+          }
+          list_insert_tc(lst, key, lane, p.k);
+        }
+        if (lane < p.k) lists[b * 32 + lane] = lst;
+      }
+    }
+  }
+
+  // ---------------- teardown: every MMA completed (the issuer waited on `done`)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+
+  // ---------------- publish this CTA's candidates; the last CTA merges
+  for (int b = warp; b < p.B; b += kTcThreads / 32)
+    if (lane < p.k) p.cand[(ci * p.B + b) * p.k + lane] = lists[b * 32 + lane];
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = (atomicInc(p.counter, (unsigned)(G - 1)) == (unsigned)(G - 1));
+  if (threadIdx.x == 0)
+    *last_flag = (atomicInc(p.counter, (unsigned)(G - 1)) == (unsigned)(G - 1));
   __syncthreads();
-  if (!last) return;
+  if (!*last_flag) return;
   __threadfence();
   const int64_t total = G * p.k;
-  for (int b = warp; b < p.B; b += 8) {
+  for (int b = warp; b < p.B; b += kTcThreads / 32) {
     unsigned long long lst = 0ull;
-    for (int64_t base = 0; base < total; base += 32) {
-      const int64_t idx = base + lane;
+    for (int64_t bs = 0; bs < total; bs += 32) {
+      const int64_t idx = bs + lane;
       unsigned long long key = 0ull;
       if (idx < total) key = __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k);
       list_insert_tc(lst, key, lane, p.k);
@@ -439,7 +525,7 @@ static bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols
 
 TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, int k, int sms) {
   TcPlan pl{};
-  pl.ok = (T >= 1 && T <= 256 && (h_kv * d) % kTcBK == 0);
+  pl.ok = (T >= 1 && T <= 256 && B >= 1 && B <= 64 && (h_kv * d) % kTcBK == 0);
   if (!pl.ok) return pl;
   pl.NQ = std::max(1, 256 / T);
   if (pl.NQ > B) pl.NQ = B;
@@ -447,15 +533,19 @@ TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, 
   if (pl.N < 16) pl.N = 16;
   pl.n_qtiles = (B + pl.NQ - 1) / pl.NQ;
   pl.n_ctiles = (n_chunks + kTcBM - 1) / kTcBM;
-  pl.grid = (int)std::min<int64_t>(sms, std::max<int64_t>(1, pl.n_ctiles * pl.n_qtiles));
-  pl.topk_grid = (int)std::min<int64_t>((int64_t)sms, std::max<int64_t>(1, n_chunks / 256));
+  pl.grid = (int)std::min<int64_t>(sms, std::max<int64_t>(1, pl.n_ctiles));
+  pl.topk_grid = pl.grid;
   const size_t rows = (size_t)B * T;
   pl.q_bytes = ((rows * h_kv * d * 2) + 255) & ~(size_t)255;
-  pl.m_bytes = (((size_t)B * n_chunks * 4) + 255) & ~(size_t)255;
-  pl.cand_bytes = (((size_t)pl.topk_grid * B * k * 8) + 255) & ~(size_t)255;
+  pl.m_bytes = 0;
+  pl.cand_bytes = (((size_t)pl.grid * B * k * 8) + 255) & ~(size_t)255;
   const size_t stage = (((size_t)kTcBM * kTcBK * 2 + (size_t)pl.N * kTcBK * 2) + 1023) & ~(size_t)1023;
-  pl.stages = (int)std::min<size_t>(kTcMaxStages, kTcSmemBudget / stage);
-  pl.smem = 1024 + pl.stages * stage + 512;
+  const size_t fixed = (size_t)kTcBM * B * 4 + (kTcWin + 1) * 8 + (size_t)B * 32 * 8 +
+                       ((B + 1) & ~1) * 4 + (2 * kTcMaxStages + 5) * 8 + 3 * 8 + 16;
+  const size_t budget = 227 * 1024 - 1024 - fixed - 64;
+  pl.stages = (int)std::min<size_t>(kTcMaxStages, budget / stage);
+  if (pl.stages < 2) pl.ok = false;
+  pl.smem = 1024 + pl.stages * stage + fixed + 64;
   (void)n_docs;
   return pl;
 }
@@ -488,46 +578,35 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t
                                                           a.h_qr, a.h_kv, a.d, a.q_hat);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // 2. tensor-core scores -> chunk scores
+  // 2. tensor-core scores fused with the per-document max and the exact top-k
   CUtensorMap mk, mq;
   const int K = a.h_kv * a.d;
   if (!make_map(&mk, a.Kr_hat, a.n_chunks, K, kTcBM) || !make_map(&mq, a.q_hat, rows, K, pl.N))
     return cudaErrorInvalidValue;
   TcParams p{};
+  p.coff = a.coff;
+  p.excl = a.excl;
+  p.n_docs = a.n_docs;
   p.n_chunks = a.n_chunks;
+  p.words = (a.n_docs + 31) / 32;
   p.K = K;
-  p.rows = rows;
   p.B = a.B;
   p.T = a.T;
   p.NQ = pl.NQ;
   p.N = pl.N;
+  p.n_qtiles = (int)pl.n_qtiles;
   p.stages = pl.stages;
-  p.n_qtiles = pl.n_qtiles;
-  p.n_units = pl.n_ctiles * pl.n_qtiles;
-  p.mscore = a.mscore;
+  p.k = a.k;
+  p.top_ids = a.top_ids;
+  p.top_scores = a.top_scores;
+  p.doc_scores = a.doc_scores;
+  p.cand = a.cand;
+  p.counter = a.counter;
   p.err = a.err;
   e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)pl.smem);
   if (e != cudaSuccess) return e;
   route_tc_kernel<<<pl.grid, kTcThreads, pl.smem, st>>>(mk, mq, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // 3. documents + top-k
-  DocTopkParams t{};
-  t.mscore = a.mscore;
-  t.coff = a.coff;
-  t.excl = a.excl;
-  t.n_docs = a.n_docs;
-  t.n_chunks = a.n_chunks;
-  t.words = (a.n_docs + 31) / 32;
-  t.B = a.B;
-  t.k = a.k;
-  t.top_ids = a.top_ids;
-  t.top_scores = a.top_scores;
-  t.doc_scores = a.doc_scores;
-  t.cand = a.cand;
-  t.counter = a.counter;
-  doc_topk_kernel<<<pl.topk_grid, 256, 0, st>>>(t);
   return cudaGetLastError();
 }
 
