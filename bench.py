@@ -44,7 +44,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m", choices=["bank100m", "bank10m"])
-    ap.add_argument("--fetch", default="memcpy", choices=["memcpy", "zerocopy"])
+    ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
+                    help="host-bank fetch: device gather over the host link on a side stream "
+                         "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
     ap.add_argument("--scan", default="tc", choices=["tc", "cc"],
                     help="router scan: tensor cores over the normalised bank, or CUDA cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -160,6 +162,8 @@ class Decode:
                     dst[c0:c0 + n].copy_(t)
             del tmp
             self.fetchers = [msa.Fetcher(w.B, w.k) for _ in range(2)]
+            self.ev_route = [torch.cuda.Event() for _ in range(2)]
+            self.ev_gather = [torch.cuda.Event() for _ in range(2)]
         B, k = w.B, w.k
         ws_r = msa.msa_route_topk_workspace(B, w.T, w.h_qr, w.h_kv, w.d, 1, self.n_docs,
                                             self.n_chunks, k)
@@ -201,14 +205,21 @@ class Decode:
             self.fetchers[l % 2].begin(bf["ids"], self.coff, self.max_ctx, bf["gi"], bf["cl"],
                                        bf["ws_g"], self.main)
         elif self.fetch == "zerocopy":
+            # the gather kernel reads the selected rows from pinned host memory on a side
+            # stream, ordered after this layer's routing and before its attention
+            self.ev_route[l % 2].record(self.main)
+            self.copy.wait_event(self.ev_route[l % 2])
             self.msa.msa_gather(bf["ids"], self.coff, self.Kh, self.Vh, self.max_ctx, bf["gi"],
-                                bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.main)
+                                bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.copy)
+            self.ev_gather[l % 2].record(self.copy)
         else:
             d = self.layers[l]
             self.msa.msa_gather(bf["ids"], self.coff, d["Kbar"], d["Vbar"], self.max_ctx,
                                 bf["gi"], bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.main)
 
     def finish(self, l):
+        if self.fetch == "zerocopy":
+            self.main.wait_event(self.ev_gather[l % 2])
         if self.fetch == "memcpy":
             bf = self.buf[l % 2]
             self.fetchers[l % 2].finish(self.coff_host, self.Kh, self.Vh, self.max_ctx, bf["cK"],

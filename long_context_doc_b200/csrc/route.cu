@@ -368,14 +368,15 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   const int64_t total = G * p.k;
   for (int b = warp; b < p.B; b += kWarps) {
     unsigned long long lst = 0ull;
-    for (int64_t base = 0; base < total; base += 32) {
-      const int64_t idx = base + lane;
-      unsigned long long key = 0ull;
-      if (idx < total) {
-        const int64_t cta = idx / p.k, j = idx % p.k;
-        key = __ldcg(p.cand + (cta * p.B + b) * p.k + j);
+    for (int64_t base = 0; base < total; base += 8 * 32) {
+      unsigned long long key[8];  // eight independent loads in flight per lane
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t idx = base + j * 32 + lane;
+        key[j] = idx < total ? __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k) : 0ull;
       }
-      list_insert(lst, key, lane, p.k);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) list_insert(lst, key[j], lane, p.k);
     }
     if (lane < p.k) {
       p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;

@@ -478,11 +478,15 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   const int64_t total = G * p.k;
   for (int b = warp; b < p.B; b += kTcThreads / 32) {
     unsigned long long lst = 0ull;
-    for (int64_t bs = 0; bs < total; bs += 32) {
-      const int64_t idx = bs + lane;
-      unsigned long long key = 0ull;
-      if (idx < total) key = __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k);
-      list_insert_tc(lst, key, lane, p.k);
+    for (int64_t bs = 0; bs < total; bs += 8 * 32) {
+      unsigned long long key[8];  // eight independent loads in flight per lane
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t idx = bs + j * 32 + lane;
+        key[j] = idx < total ? __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k) : 0ull;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) list_insert_tc(lst, key[j], lane, p.k);
     }
     if (lane < p.k) {
       p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
