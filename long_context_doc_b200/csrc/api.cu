@@ -475,7 +475,7 @@ size_t msa_sparse_attend_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_
                                    int32_t max_ctx, int32_t L_loc) {
   if (B < 1 || T < 1 || h_q < 1 || h_kv < 1 || d < 2 || max_ctx < 0 || L_loc < 1) return kHeader;
   const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
-  return kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes;
+  return kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes + pl.ctr_bytes;
 }
 
 msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
@@ -498,7 +498,7 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
               (max_ctx == 0 || (aligned16(ctxK) && aligned16(ctxV))),
           MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
-  const size_t need = kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes;
+  const size_t need = kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes + pl.ctr_bytes;
   REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
           MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
   unsigned char* base = static_cast<unsigned char*>(ws) + kHeader;
@@ -526,6 +526,8 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
   p.NRB = pl.NRB;
   p.part_o = reinterpret_cast<float*>(base + pl.cs_bytes);
   p.part_ml = reinterpret_cast<float*>(base + pl.cs_bytes + pl.part_o_bytes);
+  p.counters = reinterpret_cast<unsigned int*>(base + pl.cs_bytes + pl.part_o_bytes +
+                                               pl.part_ml_bytes);
   p.O = O;
   cudaError_t e = msa::launch_attend(p, dtype, (double)rope_base, pos0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");

@@ -109,11 +109,12 @@ struct AttendParams {
   int S, KPS, RB, NRB;  // splits, keys per split, rows per CTA, row blocks
   float* part_o;        // [B*T*h_q, S, d]
   float* part_ml;       // [B*T*h_q, S, 2]
+  unsigned int* counters;  // [B*h_kv, NRB] split tickets
   void* O;              // [B, T, h_q, d]
 };
 struct AttendPlan {
   int RB, NRB, KPS, S;
-  size_t cs_bytes, part_o_bytes, part_ml_bytes;
+  size_t cs_bytes, part_o_bytes, part_ml_bytes, ctr_bytes;
 };
 AttendPlan attend_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0, cudaStream_t st);
