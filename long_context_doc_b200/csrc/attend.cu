@@ -11,13 +11,12 @@
 //
 // Kernel: split-K flash attention on CUDA cores (fp32 accumulation, online softmax).
 // CTA = (key split, row block, batch x KV head); the rows of a CTA are RB of the G x T query
-// rows that share one KV head (GQA), ordered token-major. Each warp owns 32-key tiles: the
-// tile's key and value rows are staged with coalesced 16-byte loads into padded shared
-// memory (all loads in flight at once); then lane = key reads its key row (memory rows as
-// stored, local rows rotated in registers with the cos/sin table), dots it with the CTA's
-// rotated, pre-scaled query rows (broadcast reads), and the warp updates its running
-// max/sum; P·V is accumulated with lane = output dims. Warps are merged in shared memory;
-// the last CTA of each (query, KV head, row block) to finish merges the splits.
+// rows that share one KV head (GQA), ordered token-major. Per 64-key tile, every load is in
+// flight at once (key and value rows by cp.async, the RoPE pairs of the local keys by
+// coalesced loads); the local keys are rotated once per CTA into an fp32 tile; logits,
+// the online softmax and P·V then run from shared memory (two lanes per key for the logits,
+// one thread per output dim for P·V). The last CTA of each (query, KV head, row block) to
+// finish merges the splits.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -42,203 +41,195 @@ __global__ void rope_table_kernel(float2* cs, int L, int d, int pos0, double bas
   }
 }
 
-// One warp's 32 key rows (or value rows) of KV head g, staged with coalesced 16-byte loads
-// into a shared-memory tile with padded rows (row stride D + 16 / sizeof(T) elements), so
-// that one-row-per-lane reads are free of bank conflicts.
-template <typename T, int D>
-__device__ __forceinline__ void stage_rows(T* tile, const AttendParams& p, const void* ctx_base,
-                                           const void* loc_base, int b, int g, int kt, int nk,
-                                           int n_ctx, int lane) {
-  constexpr int SEG = D * (int)sizeof(T) / 16;       // 16-byte segments per row
-  constexpr int RPI = 32 / SEG;                      // rows per warp instruction
-  constexpr int PAD = D + 16 / (int)sizeof(T);
-  const int64_t W = (int64_t)p.h_kv * D;
-#pragma unroll
-  for (int it = 0; it < SEG; ++it) {
-    const int r = it * RPI + lane / SEG, sg = lane % SEG;
-    const int key = kt + r;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < nk) {
-      const T* src = key < n_ctx
-          ? static_cast<const T*>(ctx_base) + ((int64_t)b * p.max_ctx + key) * W + (int64_t)g * D
-          : static_cast<const T*>(loc_base) + ((int64_t)b * p.L + (key - n_ctx)) * W + (int64_t)g * D;
-      v = reinterpret_cast<const uint4*>(src)[sg];
-    }
-    *reinterpret_cast<uint4*>(tile + r * PAD + sg * (16 / (int)sizeof(T))) = v;
-  }
+// cp.async (16 bytes, L2 only) global -> shared
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+constexpr int kAttKT = 64;  // keys per tile
 
 template <typename T, int D, int RB>
 __global__ void __launch_bounds__(kAttThreads) attend_kernel(AttendParams p) {
   constexpr int HALF = D / 2;
-  constexpr int DPL = D / 32;  // output dims per lane
-  constexpr int PAD = D + 16 / (int)sizeof(T);
-  constexpr int E = 16 / (int)sizeof(T);
-  constexpr int kMaxRB = RB;
-  using VecT = Vec<T, E>;
-  // dynamic shared memory: query rows, then per-warp key/value tiles; after the key loop the
-  // tiles are reused for the warp merge
+  constexpr int KP = D + 4;                          // padded fp32 key row
+  constexpr int VEC = 16 / (int)sizeof(T);           // elements per 16-byte copy
+  constexpr int PAIRS = kAttKT * HALF / kAttThreads;  // RoPE pairs per thread per tile
+  constexpr int KPB = kAttThreads / D;               // key phases of the P.V step (1 or 2)
   extern __shared__ __align__(16) unsigned char att_smem[];
-  float (*qs)[D] = reinterpret_cast<float (*)[D]>(att_smem);
-  T* tiles = reinterpret_cast<T*>(att_smem + sizeof(float) * RB * D);
-  float (*wo)[RB][D] = reinterpret_cast<float (*)[RB][D]>(tiles);
-  __shared__ float wm[kAttWarps][RB], wl[kAttWarps][RB];
+  T* kraw = reinterpret_cast<T*>(att_smem);                               // [KT][D]
+  T* vraw = kraw + kAttKT * D;                                            // [KT][D]
+  float* krot = reinterpret_cast<float*>(vraw + kAttKT * D);              // [KT][KP]
+  float* qs = krot + kAttKT * KP;                                         // [RB][D]
+  float* ps = qs + RB * D;                                                // [RB][KT]
+  float* rowm = ps + RB * kAttKT;                                         // [RB] running max
+  float* rowl = rowm + RB;                                                // [RB] running sum
+  float* rowa = rowl + RB;                                                // [RB] rescale
   __shared__ int is_last;
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x;
   const int rb = blockIdx.y;
   const int b = blockIdx.z / p.h_kv, g = blockIdx.z % p.h_kv;
   const int G = p.h_q / p.h_kv;
   const int rows_total = G * p.T;
-  const int r0 = rb * p.RB;
-  const int nr = min(p.RB, rows_total - r0);
+  const int r0 = rb * RB;
+  const int nr = min(RB, rows_total - r0);
   const int n_ctx = min(max(p.ctx_len[b], 0), p.max_ctx);
   const int n_keys = n_ctx + p.L;
   const int ks = split * p.KPS;
   const int t_hi = (r0 + nr - 1) / G;  // last local row any row of this block can see
   const int ke = min(min(ks + p.KPS, n_keys), n_ctx + p.L - p.T + t_hi + 1);
+  const int64_t W = (int64_t)p.h_kv * D;
 
-  // rotated, pre-scaled query rows
-  for (int idx = threadIdx.x; idx < nr * HALF; idx += blockDim.x) {
+  // rotated, pre-scaled query rows; running softmax state
+  for (int idx = tid; idx < RB * HALF; idx += kAttThreads) {
     const int rr = idx / HALF, i = idx % HALF;
-    const int r = r0 + rr;
-    const int t = r / G, h = g * G + r % G;
-    const T* q = static_cast<const T*>(p.Q) + (((int64_t)b * p.T + t) * p.h_q + h) * D;
-    float x1 = Elem<T>::to_f(q[i]), x2 = Elem<T>::to_f(q[i + HALF]);
-    if (p.rope) {
-      const float2 c = p.cs[(int64_t)(p.L - p.T + t) * HALF + i];
-      const float y1 = x1 * c.x - x2 * c.y, y2 = x2 * c.x + x1 * c.y;
-      x1 = y1;
-      x2 = y2;
-    }
-    qs[rr][i] = x1 * p.scale_log2;
-    qs[rr][i + HALF] = x2 * p.scale_log2;
-  }
-  __syncthreads();
-
-  float m[kMaxRB], l[kMaxRB], acc[kMaxRB][DPL];
-#pragma unroll
-  for (int r = 0; r < kMaxRB; ++r) {
-    m[r] = -INFINITY;
-    l[r] = 0.f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[r][e] = 0.f;
-  }
-
-  T* kt_s = tiles + (size_t)(2 * warp) * 32 * PAD;
-  T* vt_s = tiles + (size_t)(2 * warp + 1) * 32 * PAD;
-  for (int kt = ks + warp * 32; kt < ke; kt += kAttWarps * 32) {
-    const int nk = min(32, ke - kt);
-    // both tiles' loads are issued before either is used
-    stage_rows<T, D>(kt_s, p, p.cK, p.Kl, b, g, kt, nk, n_ctx, lane);
-    stage_rows<T, D>(vt_s, p, p.cV, p.Vl, b, g, kt, nk, n_ctx, lane);
-    __syncwarp();
-    const int key = kt + lane;
-    const bool kin = lane < nk;
-    const bool is_ctx = key < n_ctx;
-    const int j = key - n_ctx;  // local row (if not memory)
-    float s[kMaxRB];
-#pragma unroll
-    for (int r = 0; r < kMaxRB; ++r) s[r] = 0.f;
-    if (kin) {
-      const bool rot = !is_ctx && p.rope;
-      const float4* csr = reinterpret_cast<const float4*>(p.cs + (int64_t)(rot ? j : 0) * HALF);
-      const T* krow = kt_s + lane * PAD;
-#pragma unroll 2
-      for (int v = 0; v < HALF / E; ++v) {
-        float a[E], c[E];
-        VecT::unpack(reinterpret_cast<const typename VecT::raw*>(krow)[v], a);
-        VecT::unpack(reinterpret_cast<const typename VecT::raw*>(krow + HALF)[v], c);
-        if (rot) {
-#pragma unroll
-          for (int e2 = 0; e2 < E / 2; ++e2) {
-            const float4 t2 = __ldg(csr + (v * E) / 2 + e2);  // (cos, sin) of two pairs
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 2 * e2 + h2;
-              const float co = h2 ? t2.z : t2.x, si = h2 ? t2.w : t2.y;
-              const float y1 = a[e] * co - c[e] * si, y2 = c[e] * co + a[e] * si;
-              a[e] = y1;
-              c[e] = y2;
-            }
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kMaxRB; ++r) {
-          if (r < nr) {
-            float acc_r = s[r];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-              acc_r = fmaf(qs[r][v * E + e], a[e], acc_r);
-              acc_r = fmaf(qs[r][HALF + v * E + e], c[e], acc_r);
-            }
-            s[r] = acc_r;
-          }
-        }
+    float x1 = 0.f, x2 = 0.f;
+    if (rr < nr) {
+      const int r = r0 + rr;
+      const int t = r / G, h = g * G + r % G;
+      const T* q = static_cast<const T*>(p.Q) + (((int64_t)b * p.T + t) * p.h_q + h) * D;
+      x1 = Elem<T>::to_f(q[i]);
+      x2 = Elem<T>::to_f(q[i + HALF]);
+      if (p.rope) {
+        const float2 c = p.cs[(int64_t)(p.L - p.T + t) * HALF + i];
+        const float y1 = x1 * c.x - x2 * c.y, y2 = x2 * c.x + x1 * c.y;
+        x1 = y1;
+        x2 = y2;
       }
     }
-    // mask + online softmax per row (base-2 exponent; q was pre-scaled by log2 e)
+    qs[rr * D + i] = x1 * p.scale_log2;
+    qs[rr * D + i + HALF] = x2 * p.scale_log2;
+  }
+  if (tid < RB) { rowm[tid] = -INFINITY; rowl[tid] = 0.f; }
+
+  const int e_own = tid % D;       // output dim of this thread in the P.V step
+  const int kph = tid / D;         // key phase of this thread in the P.V step
+  float acc[RB];
 #pragma unroll
-    for (int r = 0; r < kMaxRB; ++r) {
-      if (r >= nr) continue;
-      const int t = (r0 + r) / G;
-      const bool vis = kin && (is_ctx || j <= p.L - p.T + t);
-      const float sv = vis ? s[r] : -INFINITY;
-      float mx = sv;
+  for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+
+  for (int kt = ks; kt < ke; kt += kAttKT) {
+    const int nk = min(kAttKT, ke - kt);
+    // 1. all loads of the tile in flight at once: K and V rows (cp.async) and RoPE pairs
+    for (int idx = tid; idx < nk * (D / VEC); idx += kAttThreads) {
+      const int j = idx / (D / VEC), sg = idx % (D / VEC);
+      const int key = kt + j;
+      const T* ks_src = key < n_ctx
+          ? static_cast<const T*>(p.cK) + ((int64_t)b * p.max_ctx + key) * W + (int64_t)g * D
+          : static_cast<const T*>(p.Kl) + ((int64_t)b * p.L + (key - n_ctx)) * W + (int64_t)g * D;
+      const T* vs_src = key < n_ctx
+          ? static_cast<const T*>(p.cV) + ((int64_t)b * p.max_ctx + key) * W + (int64_t)g * D
+          : static_cast<const T*>(p.Vl) + ((int64_t)b * p.L + (key - n_ctx)) * W + (int64_t)g * D;
+      cp_async16(kraw + j * D + sg * VEC, ks_src + sg * VEC);
+      cp_async16(vraw + j * D + sg * VEC, vs_src + sg * VEC);
+    }
+    float2 cs[PAIRS];
+#pragma unroll
+    for (int q = 0; q < PAIRS; ++q) {
+      const int idx = q * kAttThreads + tid;
+      const int j = idx / HALF, i = idx % HALF;
+      const int key = kt + j;
+      cs[q] = make_float2(1.f, 0.f);
+      if (p.rope && j < nk && key >= n_ctx) cs[q] = __ldg(p.cs + (int64_t)(key - n_ctx) * HALF + i);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // 2. rotate the local keys once (memory rows pass through), fp32
+#pragma unroll
+    for (int q = 0; q < PAIRS; ++q) {
+      const int idx = q * kAttThreads + tid;
+      const int j = idx / HALF, i = idx % HALF;
+      float y1 = 0.f, y2 = 0.f;
+      if (j < nk) {
+        const float a = Elem<T>::to_f(kraw[j * D + i]), c = Elem<T>::to_f(kraw[j * D + i + HALF]);
+        y1 = a * cs[q].x - c * cs[q].y;
+        y2 = c * cs[q].x + a * cs[q].y;
+      }
+      krot[j * KP + i] = y1;
+      krot[j * KP + i + HALF] = y2;
+    }
+    __syncthreads();
+    // 3. logits: two lanes per key (half the dims each), 16 keys per warp
+    {
+      const int j = warp * 16 + (lane & 15);
+      const int hh = lane >> 4;
+      float s[RB];
+#pragma unroll
+      for (int r = 0; r < RB; ++r) s[r] = 0.f;
+      const float4* kr4 = reinterpret_cast<const float4*>(krot + j * KP + hh * HALF);
+#pragma unroll 4
+      for (int v = 0; v < HALF / 4; ++v) {
+        const float4 kv = kr4[v];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          const float4 qv = reinterpret_cast<const float4*>(qs + r * D + hh * HALF)[v];
+          s[r] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, s[r]))));
+        }
+      }
+      const int key = kt + j;
+      const bool kin = j < nk;
+      const bool is_ctx = key < n_ctx;
+      const int jl = key - n_ctx;
+#pragma unroll
+      for (int r = 0; r < RB; ++r) {
+        s[r] += __shfl_xor_sync(0xffffffffu, s[r], 16);
+        const int t = (r0 + r) / G;
+        const bool vis = kin && r < nr && (is_ctx || jl <= p.L - p.T + t);
+        if (hh == 0) ps[r * kAttKT + j] = vis ? s[r] : -INFINITY;
+      }
+    }
+    __syncthreads();
+    // 4. online softmax: warp w owns rows w, w + 4, ...
+    for (int r = warp; r < RB; r += kAttWarps) {
+      const float a0 = ps[r * kAttKT + lane], a1 = ps[r * kAttKT + lane + 32];
+      float mx = fmaxf(a0, a1);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float mn = fmaxf(m[r], mx);
-      if (mn == -INFINITY) { s[r] = 0.f; continue; }
-      const float pr = vis ? exp2f(sv - mn) : 0.f;
-      const float alpha = exp2f(m[r] - mn);
-      float ps = pr;
+      const float mo = rowm[r];
+      const float mn = fmaxf(mo, mx);
+      float p0 = 0.f, p1 = 0.f, alpha = 1.f;
+      if (mn != -INFINITY) {
+        p0 = a0 == -INFINITY ? 0.f : exp2f(a0 - mn);
+        p1 = a1 == -INFINITY ? 0.f : exp2f(a1 - mn);
+        alpha = mo == -INFINITY ? 0.f : exp2f(mo - mn);
+      }
+      float sum = p0 + p1;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-      l[r] = l[r] * alpha + ps;
-      m[r] = mn;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[r][e] *= alpha;
-      s[r] = pr;
-    }
-    // P V: lane owns DPL consecutive dims; value rows from the staged tile
-    using VecV = Vec<T, DPL>;
-    for (int kk = 0; kk < nk; ++kk) {
-      float vv[DPL];
-      VecV::unpack(reinterpret_cast<const typename VecV::raw*>(vt_s + kk * PAD)[lane], vv);
-#pragma unroll
-      for (int r = 0; r < kMaxRB; ++r) {
-        if (r >= nr) continue;
-        const float pr = __shfl_sync(0xffffffffu, s[r], kk);
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[r][e] = fmaf(pr, vv[e], acc[r][e]);
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      ps[r * kAttKT + lane] = p0;
+      ps[r * kAttKT + lane + 32] = p1;
+      if (lane == 0) {
+        rowl[r] = rowl[r] * alpha + sum;
+        rowm[r] = mn;
+        rowa[r] = alpha;
       }
     }
-    __syncwarp();  // the tiles are rewritten by the next iteration
+    __syncthreads();
+    // 5. P.V: thread owns one output dim (and a key phase when D < 128)
+#pragma unroll
+    for (int r = 0; r < RB; ++r) acc[r] *= rowa[r];
+    for (int j = kph; j < nk; j += KPB) {
+      const float v = Elem<T>::to_f(vraw[j * D + e_own]);
+#pragma unroll
+      for (int r = 0; r < RB; ++r) acc[r] = fmaf(ps[r * kAttKT + j], v, acc[r]);
+    }
+    __syncthreads();  // the tiles are rewritten by the next iteration
   }
 
-  // merge the warps (the tiles are free once every warp has left the key loop)
-  __syncthreads();
+  // combine the key phases (D < 128), then write this split's partial or the output
+  float* part = krot;  // free after the loop: [KPB][RB][D]
 #pragma unroll
-  for (int r = 0; r < kMaxRB; ++r) {
-    if (r >= nr) continue;
-    if (lane == 0) { wm[warp][r] = m[r]; wl[warp][r] = l[r]; }
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) wo[warp][r][lane * DPL + e] = acc[r][e];
-  }
+  for (int r = 0; r < RB; ++r) part[(kph * RB + r) * D + e_own] = acc[r];
   __syncthreads();
-  for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) {
+  for (int idx = tid; idx < nr * D; idx += kAttThreads) {
     const int r = idx / D, e = idx % D;
-    float mm = -INFINITY;
-    for (int w = 0; w < kAttWarps; ++w) mm = fmaxf(mm, wm[w][r]);
-    float ll = 0.f, oo = 0.f;
-    if (mm != -INFINITY) {
-      for (int w = 0; w < kAttWarps; ++w) {
-        const float a = exp2f(wm[w][r] - mm);
-        ll += wl[w][r] * a;
-        oo += wo[w][r][e] * a;
-      }
-    }
+    float oo = 0.f;
+    for (int k2 = 0; k2 < KPB; ++k2) oo += part[(k2 * RB + r) * D + e];
+    const float mm = rowm[r], ll = rowl[r];
     const int rr = r0 + r;
     const int t = rr / G, h = g * G + rr % G;
     const int64_t row = ((int64_t)b * p.T + t) * p.h_q + h;
@@ -256,26 +247,28 @@ __global__ void __launch_bounds__(kAttThreads) attend_kernel(AttendParams p) {
   // the last split CTA of this (query, KV head, row block) merges the splits
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     unsigned int* ctr = p.counters + ((int64_t)blockIdx.z * p.NRB + rb);
     is_last = (atomicInc(ctr, (unsigned)(p.S - 1)) == (unsigned)(p.S - 1));
   }
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) {
+  for (int idx = tid; idx < nr * D; idx += kAttThreads) {
     const int r = idx / D, e = idx % D;
     const int rr = r0 + r;
     const int t = rr / G, h = g * G + rr % G;
     const int64_t row = ((int64_t)b * p.T + t) * p.h_q + h;
     float mm = -INFINITY;
+#pragma unroll 8
     for (int sp = 0; sp < p.S; ++sp) mm = fmaxf(mm, __ldcg(p.part_ml + (row * p.S + sp) * 2));
     float ll = 0.f, oo = 0.f;
     if (mm != -INFINITY) {
+#pragma unroll 8
       for (int sp = 0; sp < p.S; ++sp) {
-        const float ms = __ldcg(p.part_ml + (row * p.S + sp) * 2);
-        const float a = ms == -INFINITY ? 0.f : exp2f(ms - mm);
-        ll += __ldcg(p.part_ml + (row * p.S + sp) * 2 + 1) * a;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (row * p.S + sp) * 2));
+        const float a = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mm);
+        ll += ml.y * a;
         oo += __ldcg(p.part_o + (row * p.S + sp) * D + e) * a;
       }
     }
@@ -291,16 +284,16 @@ AttendPlan attend_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int 
   const int rows = G * T;
   pl.RB = rows >= 8 ? 8 : rows >= 4 ? 4 : rows >= 2 ? 2 : 1;
   pl.NRB = (rows + pl.RB - 1) / pl.RB;
-  pl.KPS = 128;
+  pl.KPS = 64;
   const int keys = max_ctx + L;
   const int max_s = (keys + pl.KPS - 1) / pl.KPS;
   const int64_t base = (int64_t)B * h_kv * pl.NRB;
-  int64_t want = base > 0 ? ((int64_t)sms * 8 + base - 1) / base : 1;
+  int64_t want = base > 0 ? ((int64_t)sms * 12 + base - 1) / base : 1;
   if (want > max_s) want = max_s;
   if (want < 1) want = 1;
   pl.S = (int)want;
-  pl.KPS = ((keys + pl.S - 1) / pl.S + 127) / 128 * 128;
-  if (pl.KPS < 128) pl.KPS = 128;
+  pl.KPS = ((keys + pl.S - 1) / pl.S + 63) / 64 * 64;
+  if (pl.KPS < 64) pl.KPS = 64;
   pl.S = (keys + pl.KPS - 1) / pl.KPS;
   if (pl.S < 1) pl.S = 1;
   pl.cs_bytes = ((size_t)L * (d / 2) * sizeof(float2) + 255) & ~(size_t)255;
@@ -330,9 +323,8 @@ cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0,
   cudaError_t e = cudaSuccess;
 #define MSA_ATT(TT, DD, RR)                                                                    \
   {                                                                                            \
-    const size_t sm = sizeof(float) * RR * DD +                                                 \
-                      std::max(sizeof(TT) * 2 * kAttWarps * 32 * (DD + 16 / sizeof(TT)),       \
-                               sizeof(float) * kAttWarps * RR * DD);                           \
+    const size_t sm = sizeof(TT) * 2 * kAttKT * DD + sizeof(float) * kAttKT * (DD + 4) +         \
+                      sizeof(float) * (RR * DD + RR * kAttKT + 3 * RR);                         \
     auto kf = attend_kernel<TT, DD, RR>;                                                       \
     e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);        \
     if (e == cudaSuccess) kf<<<grid, kAttThreads, sm, st>>>(p);                               \
