@@ -156,6 +156,29 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
                           const uint32_t* exclude_bits, int32_t* top_ids, float* top_scores,
                           float* doc_scores, void* ws, size_t ws_bytes, void* stream);
 
+/* msa_route_topk_noalloc - msa_route_topk without a caller workspace, for callers that
+ * cannot allocate device memory where they call it: code running under another framework's
+ * memory planner (which owns every device allocation), paths that must not synchronise the
+ * device (cudaMalloc/cudaFree may), and serving loops that forbid allocator calls.
+ * (A library service; the pages describing MSA have no counterpart.)
+ *
+ * Same arguments and results as msa_route_topk, minus ws/ws_bytes. The scratch is a 2 MiB
+ * array inside the library, held on every GPU that loads it until the process exits; calls
+ * whose msa_route_topk_workspace(...) exceeds 2 MiB return MSA_ERR_UNSUPPORTED (use
+ * msa_route_topk). The first call on a device, made with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture. It allocates nothing (no cudaMalloc/cudaFree or allocating library
+ * routine). All calls share the one array, which keeps the last call's contents (what must
+ * start at zero is cleared by every call); calls that overlap on the GPU race and must be
+ * serialised by the caller. */
+msa_status msa_route_topk_noalloc(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
+                                  const void* Kbar_r, const float* kr_inv_norm,
+                                  const void* Kbar_r_hat, const int64_t* doc_chunk_off,
+                                  int64_t n_docs, int64_t n_chunks, int32_t h_kv, int32_t d,
+                                  int32_t dtype, int32_t k, const uint32_t* exclude_bits,
+                                  int32_t* top_ids, float* top_scores, float* doc_scores,
+                                  void* stream);
+
 /* Read the device status word of a workspace (synchronises `stream`): *code = 0 if the
  * kernels that used it recorded no error. Returns MSA_ERR_DEVICE if *code != 0. */
 msa_status msa_workspace_status(const void* ws, int32_t* code, void* stream);

@@ -29,7 +29,7 @@ LIB_PATH = _build.LIB
 # every symbol include/msa.h declares
 SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chunks",
            "msa_encode_pool", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
-           "msa_route_topk",
+           "msa_route_topk", "msa_route_topk_noalloc",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
            "msa_sparse_attend")
@@ -67,6 +67,9 @@ def _load():
     L.msa_route_topk.restype = ctypes.c_int
     L.msa_route_topk.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32,
                                  vp, vp, vp, vp, vp, sz, vp]
+    L.msa_route_topk_noalloc.restype = ctypes.c_int
+    L.msa_route_topk_noalloc.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, i64, i64, i32, i32, i32,
+                                         i32, vp, vp, vp, vp, vp]
     L.msa_workspace_status.restype = ctypes.c_int
     L.msa_workspace_status.argtypes = [vp, vp, vp]
     L.msa_gather.restype = ctypes.c_int
@@ -156,6 +159,17 @@ def msa_route_topk(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_bits, top
                               doc_chunk_off.shape[0] - 1, n_chunks, h_kv, d, dtype_code(Kbar_r), k,
                               _p(exclude_bits), _p(top_ids), _p(top_scores), _p(doc_scores),
                               _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_route_topk_noalloc(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_bits, top_ids,
+                           top_scores, doc_scores, stream=None, Kbar_r_hat=None):
+    """msa_route_topk without a workspace (the library's built-in 2 MiB scratch)."""
+    B, T, h_qr, d = Q_r.shape
+    n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
+    _check(lib.msa_route_topk_noalloc(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm),
+                                      _p(Kbar_r_hat), _p(doc_chunk_off), doc_chunk_off.shape[0] - 1,
+                                      n_chunks, h_kv, d, dtype_code(Kbar_r), k, _p(exclude_bits),
+                                      _p(top_ids), _p(top_scores), _p(doc_scores), _s(stream)))
 
 
 def msa_workspace_status(ws, stream=None) -> int:

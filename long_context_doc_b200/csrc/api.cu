@@ -78,6 +78,12 @@ void route_passes(int B, int T, int* bp, int* passes) {
 
 }  // namespace
 
+namespace msa {
+// Set the thread-local message returned by msa_last_error (for entry points defined in other
+// translation units).
+void set_last_error(const std::string& msg) { g_err = msg; }
+}  // namespace msa
+
 extern "C" {
 
 const char* msa_status_string(int s) {

@@ -5,8 +5,12 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <string>
 
 namespace msa {
+
+// api.cu: thread-local message of msa_last_error
+void set_last_error(const std::string& msg);
 
 // ---- encode_pool.cu
 struct EncodeParams {

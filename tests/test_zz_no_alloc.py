@@ -1,0 +1,63 @@
+"""msa_route_topk_noalloc: routing for callers that cannot allocate device memory at the call
+site (a framework's memory planner owns every allocation, allocation may synchronise the
+device, or the serving loop forbids allocator calls). It must return what msa_route_topk
+returns with a caller workspace, call after call, although all calls share one scratch
+array inside the library. Collected last on purpose: a failure here leaves every other test
+already run."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from _util import SCORE_TOL, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def msa(gpu):
+    import long_context_doc_b200 as m
+    return m
+
+
+def _inputs(gpu, tensor_path: bool):
+    w = synth.C3.scaled(n_docs=1500, B=8, T=1, ragged=True, seed=31)
+    inp = synth.make_bank_workload(w)
+    Krb = to_dev(inp["Kbar_r"], gpu)
+    import long_context_doc_b200 as m
+    return dict(w=w, Q_r=to_dev(inp["Q_r"], gpu), Kbar_r=Krb, inv=m.kr_inv_norm(Krb),
+                hat=m.kr_normalize(Krb) if tensor_path else None,
+                coff=torch.from_numpy(inp["doc_chunk_off"]).to(gpu))
+
+
+@pytest.mark.parametrize("tensor_path", [False, True], ids=["cuda_core_scan", "tensor_core_scan"])
+def test_noalloc_matches_workspace_route_two_calls(msa, gpu, tensor_path):
+    d = _inputs(gpu, tensor_path)
+    w = d["w"]
+    ref_ids, ref_sc, ref_ds = msa.route_topk(d["Q_r"], d["Kbar_r"], d["inv"], d["coff"], w.k,
+                                             doc_scores=True, Kbar_r_hat=d["hat"])
+    torch.cuda.synchronize()
+    n_docs = d["coff"].shape[0] - 1
+    for _ in range(2):  # the shared scratch keeps the previous call's contents
+        ids = torch.full((w.B, w.k), -7, dtype=torch.int32, device=gpu)
+        sc = torch.full((w.B, w.k), np.nan, dtype=torch.float32, device=gpu)
+        ds = torch.full((w.B, n_docs), np.nan, dtype=torch.float32, device=gpu)
+        msa.msa_route_topk_noalloc(d["Q_r"], d["Kbar_r"], d["inv"], d["coff"], w.k, None, ids, sc,
+                                   ds, Kbar_r_hat=d["hat"])
+        torch.cuda.synchronize()
+        assert torch.equal(ids, ref_ids)
+        np.testing.assert_allclose(sc.cpu().numpy(), ref_sc.cpu().numpy(), rtol=0,
+                                   atol=SCORE_TOL["bf16"])
+        np.testing.assert_allclose(ds.cpu().numpy(), ref_ds.cpu().numpy(), rtol=0,
+                                   atol=SCORE_TOL["bf16"])
+
+
+def test_noalloc_rejects_calls_beyond_its_scratch(msa, gpu):
+    d = _inputs(gpu, True)
+    Q = torch.zeros((64, 256, 8, 128), dtype=torch.bfloat16, device=gpu)  # 32 MB of folded queries
+    ids = torch.empty((64, 4), dtype=torch.int32, device=gpu)
+    sc = torch.empty((64, 4), dtype=torch.float32, device=gpu)
+    with pytest.raises(msa.MSAError) as e:
+        msa.msa_route_topk_noalloc(Q, d["Kbar_r"], d["inv"], d["coff"], 4, None, ids, sc, None,
+                                   Kbar_r_hat=d["hat"])
+    assert e.value.status == 2 and "scratch" in e.value.message
