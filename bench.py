@@ -55,6 +55,22 @@ def parse():
     return ap.parse_args()
 
 
+def captured_traffic(kernel_src: str, summary: str):
+    """DRAM bytes (read + write) of one launch from a committed ncu capture, or None when the
+    kernel source changed since the capture (the summary records its SHA-256)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, "long_context_doc_b200", "csrc", kernel_src), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("kernel_src_sha256") != sha:
+            return None
+        return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
+    except Exception:
+        return None
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -245,7 +261,7 @@ class Decode:
         path; K̄_r plus fp32 inverse norms for the CUDA-core path)."""
         w = self.w
         if self.scan == "tc":
-            return self.n_chunks * w.h_kv * w.d * 2 + 2 * w.B * self.n_chunks * 4
+            return self.n_chunks * w.h_kv * w.d * 2
         return self.n_chunks * w.h_kv * w.d * 2 + self.n_chunks * w.h_kv * 4
 
 
@@ -365,7 +381,9 @@ def run_libmsa(args):
                                "msa_route_topk (CUDA-core scan with fused top-k)"), "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": None, "bytes_per_launch": wk.scan_bytes(),
+                     "traffic": (captured_traffic("route_tc.cu", f"route_tc_{w.name}_dram.json")
+                                 if wk.scan == "tc" else None),
+                     "bytes_per_launch": wk.scan_bytes(),
                      "avg_launch_ms": round(route_avg, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},

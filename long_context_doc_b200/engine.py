@@ -1,0 +1,99 @@
+"""Routed-layer loop and Memory Interleaving rounds over the libmsa entry points.
+
+Memory Interleaving alternates generative retrieval, context extension and generation: the
+documents a round retrieves have their original text appended to the query for the next
+round, and routing repeats until the model judges the accumulated documents sufficient
+[ai-papers.net summary, "MSAの提案手法"; ruixiangma.github.io blog, "Memory Interleaving"].
+Without a model to generate document ids, a round's retrieval is read from the routing
+itself: the documents selected by the last routed layer of round r are appended (their raw
+per-token K/V, in ascending doc id, after the documents of earlier rounds and before the
+query tokens) and excluded from routing in later rounds. Every round uses pos0 = k.
+
+Only the loop lives here; every step of every round runs in libmsa's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, List, Optional, Sequence
+
+import torch
+
+from . import gather, route_topk, sparse_attend
+
+
+@dataclass
+class RoutedLayer:
+    """One routed layer's memory bank and the query's per-layer tensors."""
+    Kbar_r: torch.Tensor        # [n_chunks, h_kv, d]
+    kr_inv_norm: torch.Tensor   # [n_chunks, h_kv] fp32
+    Kbar: torch.Tensor          # [n_chunks, h_kv, d] (device or pinned host memory)
+    Vbar: torch.Tensor
+    doc_chunk_off: torch.Tensor  # [n_docs + 1] int64, device
+    Q_r: torch.Tensor           # [B, T, h_qr, d]
+    Q: torch.Tensor             # [B, T, h_q, d]
+    K_q: torch.Tensor           # [B, T, h_kv, d] the query tokens' own keys (before RoPE)
+    V_q: torch.Tensor           # [B, T, h_kv, d]
+    Kbar_r_hat: Optional[torch.Tensor] = None  # normalised bank for the tensor-core scan
+
+
+def exclusion_bits(appended: Sequence[Sequence[int]], n_docs: int, device) -> torch.Tensor:
+    """[B, ceil(n_docs/32)] int32 bitsets of the documents already appended per query."""
+    words = (n_docs + 31) // 32
+    bits = torch.zeros((len(appended), words), dtype=torch.int64)
+    for b, docs in enumerate(appended):
+        for doc in docs:
+            bits[b, doc // 32] |= 1 << (doc % 32)
+    bits = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits)
+    return bits.to(torch.int32).to(device)
+
+
+def routed_layer(layer: RoutedLayer, k: int, K_loc: torch.Tensor, V_loc: torch.Tensor,
+                 rope_base: float, exclude_bits: Optional[torch.Tensor] = None):
+    """Route -> gather -> sparse attention for one routed layer.
+    Returns (top_ids, top_scores, O)."""
+    ids, scores, _ = route_topk(layer.Q_r, layer.Kbar_r, layer.kr_inv_norm, layer.doc_chunk_off, k,
+                                exclude_bits=exclude_bits, Kbar_r_hat=layer.Kbar_r_hat)
+    cpd = int((layer.doc_chunk_off[1:] - layer.doc_chunk_off[:-1]).max().item())
+    _, ctx_len, ctxK, ctxV = gather(ids, layer.doc_chunk_off, layer.Kbar, layer.Vbar, k * cpd)
+    O = sparse_attend(layer.Q, K_loc, V_loc, ctxK, ctxV, ctx_len, k, rope_base)
+    return ids, scores, O
+
+
+def interleave_rounds(layers: List[RoutedLayer], k: int, rounds: int, rope_base: float,
+                      doc_kv: Callable[[int, int], tuple]):
+    """Memory Interleaving over ``rounds`` rounds of all routed layers.
+
+    ``doc_kv(layer, doc)`` returns the raw per-token (K, V) [len, h_kv, d] device tensors of a
+    retrieved document at that layer. Returns (ids[r][l] [B, k], scores[r][l] [B, k],
+    O[r][l] [B, T, h_q, d], appended[b] = the documents appended per query, in order).
+    """
+    B = layers[0].Q.shape[0]
+    n_docs = layers[0].doc_chunk_off.shape[0] - 1
+    appended: List[List[int]] = [[] for _ in range(B)]
+    all_ids, all_sc, all_O = [], [], []
+    for r in range(rounds):
+        ex = exclusion_bits(appended, n_docs, layers[0].Q.device) if r > 0 else None
+        ids_r, sc_r, O_r = [], [], []
+        for li, layer in enumerate(layers):
+            if r == 0:
+                K_loc, V_loc = layer.K_q, layer.V_q
+            else:
+                ks, vs = [], []
+                for b in range(B):
+                    parts = [doc_kv(li, doc) for doc in appended[b]]
+                    ks.append(torch.cat([p[0] for p in parts] + [layer.K_q[b]]))
+                    vs.append(torch.cat([p[1] for p in parts] + [layer.V_q[b]]))
+                if len({x.shape[0] for x in ks}) != 1:
+                    raise ValueError("interleaved local contexts must have one length per batch")
+                K_loc, V_loc = torch.stack(ks), torch.stack(vs)
+            ids, sc, O = routed_layer(layer, k, K_loc, V_loc, rope_base, ex)
+            ids_r.append(ids)
+            sc_r.append(sc)
+            O_r.append(O)
+        last = ids_r[-1].cpu().tolist()
+        for b in range(B):
+            appended[b].extend(sorted(i for i in last[b] if i >= 0))
+        all_ids.append(ids_r)
+        all_sc.append(sc_r)
+        all_O.append(O_r)
+    return all_ids, all_sc, all_O, appended

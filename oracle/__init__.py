@@ -216,3 +216,49 @@ def pipeline(w, inp: dict, L=None) -> dict:
     out["O64"] = O
     out["O"] = store_as(O, dt, L)
     return out
+
+
+def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=None) -> dict:
+    """Oracle of Memory Interleaving rounds (reading R18 of the design notes).
+
+    layers[l]: dict with Kbar_r, Kbar, Vbar (stored dtype), doc_chunk_off, Q_r, Q and the query
+    tokens' own K_q, V_q [B, T, h_kv, d]. doc_kv(l, doc) -> raw (K, V) [len, h_kv, d] of a
+    retrieved document. Round 0 attends to the query tokens alone; after each round the docs
+    selected by the LAST routed layer are appended (ascending id) for every later round,
+    before the query tokens, and excluded from routing. pos0 = k in every round.
+    Returns dict(ids=[r][l] int32 [B,k], scores=[r][l], doc_scores=[r][l], O64=[r][l],
+    appended=[b] list)."""
+    B = layers[0]["Q"].shape[0]
+    n_docs = len(layers[0]["doc_chunk_off"]) - 1
+    words = (n_docs + 31) // 32
+    appended = [[] for _ in range(B)]
+    res = dict(ids=[], scores=[], doc_scores=[], O64=[])
+    for r in range(rounds):
+        ex = np.zeros((B, words), dtype=np.uint32)
+        for b in range(B):
+            for doc in appended[b]:
+                ex[b, doc // 32] |= np.uint32(1) << np.uint32(doc % 32)
+        ids_r, sc_r, ds_r, O_r = [], [], [], []
+        for li, lay in enumerate(layers):
+            coff = lay["doc_chunk_off"]
+            ids, sc, ds = route(lay["Q_r"], lay["Kbar_r"], coff, k, ex if r > 0 else None, L)
+            cpd = int(np.max(np.diff(coff)))
+            gi, cl = gather(ids, coff, k * cpd, L)
+            K_loc = np.stack([np.concatenate([doc_kv(li, doc)[0] for doc in appended[b]] +
+                                             [lay["K_q"][b]]) for b in range(B)])
+            V_loc = np.stack([np.concatenate([doc_kv(li, doc)[1] for doc in appended[b]] +
+                                             [lay["V_q"][b]]) for b in range(B)])
+            O = attend(lay["Q"], K_loc, V_loc, lay["Kbar"], lay["Vbar"], gi, cl, pos0=k,
+                       rope_base=rope_base, L=L)
+            ids_r.append(ids)
+            sc_r.append(sc)
+            ds_r.append(ds)
+            O_r.append(O)
+        for b in range(B):
+            appended[b].extend(sorted(int(i) for i in ids_r[-1][b] if i >= 0))
+        res["ids"].append(ids_r)
+        res["scores"].append(sc_r)
+        res["doc_scores"].append(ds_r)
+        res["O64"].append(O_r)
+    res["appended"] = appended
+    return res

@@ -1,0 +1,102 @@
+"""Memory Interleaving rounds: properties of the oracle's loop (CPU) and parity of the
+engine over libmsa against it (GPU)."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from _util import ATT_TOL, SCORE_TOL, check_attention, check_topk, to_dev
+
+
+def _case(B=2, T=32, n_docs=150, doc_len=100, layers=2, k=4, seed=5):
+    w = synth.C5.scaled(n_docs=n_docs, doc_len=doc_len, B=B, T=T, L_loc=T, k=k, h_q=8, h_kv=2,
+                        h_qr=2, layers=layers, rounds=3, n_planted=1, seed=seed)
+    lays = []
+    for l in range(layers):
+        inp = synth.make_bank_workload(w, l)
+        lays.append(dict(Kbar_r=inp["Kbar_r"], Kbar=inp["Kbar"], Vbar=inp["Vbar"],
+                         doc_chunk_off=inp["doc_chunk_off"], Q_r=inp["Q_r"], Q=inp["Q"],
+                         K_q=inp["K_loc"], V_q=inp["V_loc"]))
+    return w, lays
+
+
+def test_oracle_interleave_round_structure():
+    w, lays = _case()
+    res = oracle.interleave(lays, w.k, 3, w.rope_base, lambda l, d: synth.appended_doc_kv(w, l, d))
+    # round 0 is the plain routed layer with the query tokens as the local context
+    for l, lay in enumerate(lays):
+        ids, _, _ = oracle.route(lay["Q_r"], lay["Kbar_r"], lay["doc_chunk_off"], w.k)
+        assert np.array_equal(res["ids"][0][l], ids)
+    for b in range(w.B):
+        app = res["appended"][b]
+        assert len(app) == 3 * w.k and len(set(app)) == len(app)  # k new docs per round
+        assert app[:w.k] == sorted(res["ids"][0][-1][b].tolist())
+        assert app[w.k:2 * w.k] == sorted(res["ids"][1][-1][b].tolist())
+        for r in (1, 2):  # appended docs are never routed again
+            for l in range(len(lays)):
+                assert not set(res["ids"][r][l][b].tolist()) & set(app[:r * w.k])
+
+
+def test_oracle_interleave_attends_to_appended_text():
+    """Round 1 equals attention over [memory ; round-0 docs' raw K/V ; query tokens]."""
+    w, lays = _case(B=1, layers=1, seed=9)
+    dk = lambda l, d: synth.appended_doc_kv(w, l, d)  # noqa: E731
+    res = oracle.interleave(lays, w.k, 2, w.rope_base, dk)
+    lay = lays[0]
+    app = res["appended"][0][:w.k]
+    K_loc = np.concatenate([dk(0, d)[0] for d in app] + [lay["K_q"][0]])[None]
+    V_loc = np.concatenate([dk(0, d)[1] for d in app] + [lay["V_q"][0]])[None]
+    assert K_loc.shape[1] == w.T + w.k * w.doc_len
+    gi, cl = oracle.gather(res["ids"][1][0], lay["doc_chunk_off"], w.k * w.cpd)
+    O = oracle.attend(lay["Q"], K_loc, V_loc, lay["Kbar"], lay["Vbar"], gi, cl, w.k, w.rope_base)
+    assert np.max(np.abs(O - res["O64"][1][0])) == 0.0
+
+
+@pytest.mark.gpu
+def test_interleave_engine_matches_oracle(gpu):
+    import torch
+
+    import long_context_doc_b200 as msa
+    from long_context_doc_b200 import engine
+    w, lays = _case()
+    dk_np = lambda l, d: synth.appended_doc_kv(w, l, d)  # noqa: E731
+    ref = oracle.interleave(lays, w.k, 3, w.rope_base, dk_np)
+    layers = []
+    for lay in lays:
+        Krb = to_dev(lay["Kbar_r"], gpu)
+        layers.append(engine.RoutedLayer(
+            Kbar_r=Krb, kr_inv_norm=msa.kr_inv_norm(Krb), Kbar=to_dev(lay["Kbar"], gpu),
+            Vbar=to_dev(lay["Vbar"], gpu),
+            doc_chunk_off=torch.from_numpy(lay["doc_chunk_off"]).to(gpu),
+            Q_r=to_dev(lay["Q_r"], gpu), Q=to_dev(lay["Q"], gpu), K_q=to_dev(lay["K_q"], gpu),
+            V_q=to_dev(lay["V_q"], gpu), Kbar_r_hat=msa.kr_normalize(Krb)))
+    cache = {}
+
+    def dk_dev(l, d):
+        if (l, d) not in cache:
+            kk, vv = dk_np(l, d)
+            cache[(l, d)] = (to_dev(kk, gpu), to_dev(vv, gpu))
+        return cache[(l, d)]
+
+    ids, scores, O, appended = engine.interleave_rounds(layers, w.k, 3, w.rope_base, dk_dev)
+    torch.cuda.synchronize()
+    tol = SCORE_TOL["bf16"]
+    for r in range(3):
+        exact = True
+        for l in range(len(lays)):
+            n = check_topk(ids[r][l].cpu().numpy(), scores[r][l].cpu().numpy().astype(np.float64),
+                           ref["ids"][r][l], ref["scores"][r][l], _masked(ref, r, l, w), tol)
+            exact &= n == w.B
+            if n == w.B:
+                check_attention(O[r][l], ref["O64"][r][l], "bf16")
+        if not exact:  # a near-tie changed the appended set; later rounds are not comparable
+            break
+        assert appended == ref["appended"] or r < 2
+
+
+def _masked(ref, r, l, w):
+    ds = ref["doc_scores"][r][l].copy()
+    if r > 0:
+        for b in range(w.B):
+            ds[b, ref["appended"][b][:r * w.k]] = -np.inf
+    return ds

@@ -529,3 +529,29 @@ def test_route_tensor_core_full_1m_token_bank(msa, gpu):
     Krb = synth.host_bank_rows(w, "Kbar_r", 0, dv["n_chunks"], coff=coff, Q_r=dv["Q_r_host"])
     ids, err = _route_tc_check(msa, gpu, dv["Q_r_host"], Krb, coff, w.k)
     assert ids[0, 0] == dv["planted"][0, 0]
+
+
+def test_pipeline_1m_bank_shape_reduced(msa, gpu):
+    """The 1M-token-bank configuration's full path at 24 documents: doc-wise RoPE + pooling,
+    tensor-core routing of the 128-token query, gather, global-RoPE attention (bf16)."""
+    w = synth.C2.scaled(n_docs=24, n_planted=2)
+    inp = synth.make_token_workload(w)
+    ref = oracle.pipeline(w, inp)
+    t = lambda x: to_dev(x, gpu)  # noqa: E731
+    enc = msa.encode_pool(t(inp["K"]), t(inp["V"]), t(inp["K_r"]), inp["doc_tok_off"], w.chunk,
+                          w.rope_base)
+    check_pooled(enc["Kbar_r"], ref["Krbar64"], "bf16", "Kbar_r")
+    hat = msa.kr_normalize(enc["Kbar_r"])
+    ids, sc, ds = msa.route_topk(t(inp["Q_r"]), enc["Kbar_r"], enc["kr_inv_norm"],
+                                 enc["doc_chunk_off"], w.k, doc_scores=True, Kbar_r_hat=hat)
+    max_ctx = ref["gather_idx"].shape[1]
+    gi, cl, cK, cV = msa.gather(ids, enc["doc_chunk_off"], enc["Kbar"], enc["Vbar"], max_ctx)
+    O = msa.sparse_attend(t(inp["Q"]), t(inp["K_loc"]), t(inp["V_loc"]), cK, cV, cl, w.k,
+                          w.rope_base)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(ds.cpu().numpy() - ref["doc_scores"])) <= SCORE_TOL["bf16"]
+    n = check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), ref["top_ids"],
+                   ref["top_scores"], ref["doc_scores"], SCORE_TOL["bf16"])
+    if n == 1:
+        assert np.array_equal(gi.cpu().numpy(), ref["gather_idx"])
+        check_attention(O, ref["O64"], "bf16")
