@@ -49,6 +49,8 @@ def parse():
                          "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
     ap.add_argument("--scan", default="tc", choices=["tc", "cc"],
                     help="router scan: tensor cores over the normalised bank, or CUDA cores")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels one by one instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=3,
                     help="routed layers in the CPU-oracle sample")
@@ -146,7 +148,7 @@ class Decode:
         self.torch, self.msa, self.w, self.dev = torch, msa, w, dev
         self.fetch = fetch if w.layers > 1 else "device"
         self.L = w.layers
-        self.main = torch.cuda.current_stream()
+        self.main = torch.cuda.Stream()  # the step's stream (capturable into a CUDA graph)
         self.copy = torch.cuda.Stream()
         self.layers = []
         seed_w = w.scaled(seed=w.seed + 1000 * rank)
@@ -200,10 +202,9 @@ class Decode:
                   for _ in range(self.L)]
         self.route_ev = None
         self.scan = scan
-        # own kernels per layer (memsets and copies excluded): route (tensor path: query fold,
-        # scan, document top-k; CUDA-core path: one fused kernel), gather indices, RoPE table,
-        # attention, split combine
-        self.kernels_per_layer = (3 if scan == "tc" else 1) + 1 + 1 + 1 + 1
+        # own kernels per layer (memsets and copies excluded): route (tensor path: query fold +
+        # scan with fused top-k; CUDA-core path: one fused kernel), gather, RoPE table, attention
+        self.kernels_per_layer = (2 if scan == "tc" else 1) + 1 + 1 + 1
 
     # per-layer pieces -------------------------------------------------------------
     def route(self, l):
@@ -290,12 +291,23 @@ def run_libmsa(args):
     for _ in range(max(args.warmup, 3)):
         wk.step()
     barrier()
-    # timed region: K steps, per-route events for the roofline
+    # the step as one CUDA graph (the zero-copy and device fetches need no host round trip)
+    use_graph = not args.no_graph and wk.fetch != "memcpy"
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=wk.main):
+            wk.step()
+        graph.replay()
+    barrier()
+
+    def run_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            wk.step()
+
     Kst = args.steps
-    wk.route_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(wk.L)] for _ in range(Kst)]
-    ev_route = wk.route_ev
-    route_ms = []
     uuid = str(torch.cuda.get_device_properties(local).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     sampler.start()
@@ -304,16 +316,23 @@ def run_libmsa(args):
     barrier()
     t0.record(wk.main)
     for s in range(Kst):
-        wk.route_ev = ev_route[s]
-        wk.step()
+        run_step()
     t1.record(wk.main)
     barrier()
     clocks = sampler.stop()
     step_ms = t0.elapsed_time(t1) / Kst
-    for s in range(Kst):
-        for l in range(wk.L):
-            route_ms.append(ev_route[s][l][0].elapsed_time(ev_route[s][l][1]))
+    # routing-call durations for the roofline: the same step launched eagerly with CUDA events
+    # around every msa_route_topk call (on the launching stream)
+    Kr = max(3, min(Kst, 20))
+    ev_route = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(wk.L)] for _ in range(Kr)]
+    for s in range(Kr):
+        wk.route_ev = ev_route[s]
+        wk.step()
+    barrier()
     wk.route_ev = None
+    route_ms = [ev_route[s][l][0].elapsed_time(ev_route[s][l][1])
+                for s in range(Kr) for l in range(wk.L)]
     # end to end: per-step query inputs copied from pinned host memory, outputs read back
     host_in = []
     for l in range(wk.L):
@@ -326,28 +345,39 @@ def run_libmsa(args):
     d2h = sum(o.numel() * o.element_size() for o in host_O) + wk.L * w.B * w.k * 4
 
     def e2e_step():
-        for l in range(wk.L):
-            d = wk.layers[l]
-            qr, q, kn, vn = host_in[l]
-            d["Q_r"].copy_(qr, non_blocking=True)
-            d["Q"].copy_(q, non_blocking=True)
-            d["K_loc"][:, -1:].copy_(kn, non_blocking=True)
-            d["V_loc"][:, -1:].copy_(vn, non_blocking=True)
-        wk.step()
-        for l in range(wk.L):
-            host_O[l].copy_(wk.O[l], non_blocking=True)
-        host_ids[0].copy_(wk.buf[0]["ids"], non_blocking=True)
-        host_ids[1].copy_(wk.buf[1]["ids"], non_blocking=True)
+        with torch.cuda.stream(wk.main):
+            for l in range(wk.L):
+                d = wk.layers[l]
+                qr, q, kn, vn = host_in[l]
+                d["Q_r"].copy_(qr, non_blocking=True)
+                d["Q"].copy_(q, non_blocking=True)
+                d["K_loc"][:, -1:].copy_(kn, non_blocking=True)
+                d["V_loc"][:, -1:].copy_(vn, non_blocking=True)
+            wk.step()
+            for l in range(wk.L):
+                host_O[l].copy_(wk.O[l], non_blocking=True)
+            host_ids[0].copy_(wk.buf[0]["ids"], non_blocking=True)
+            host_ids[1].copy_(wk.buf[1]["ids"], non_blocking=True)
 
     for _ in range(3):
         e2e_step()
     barrier()
+    e_graph = None
+    if use_graph:
+        e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e_graph, stream=wk.main):
+            e2e_step()
+        e_graph.replay()
+        barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     Ke = max(5, Kst // 2)
     e0.record(wk.main)
     for _ in range(Ke):
-        e2e_step()
+        if e_graph is not None:
+            e_graph.replay()
+        else:
+            e2e_step()
     e1.record(wk.main)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / Ke
@@ -374,7 +404,8 @@ def run_libmsa(args):
                                f"fetch={wk.fetch}") if wk.fetch != "device" else "HBM",
                    "l2": "no flush: every layer scans a 3.28 GB K̄_r, far larger than the 126 MB L2"
                    if wk.L > 1 else "no flush: the 328 MB K̄_r scan exceeds the 126 MB L2",
-                   "scan": wk.scan, "parallelism": f"replicas x{world}"},
+                   "scan": wk.scan, "cuda_graph": use_graph,
+                   "parallelism": f"replicas x{world}"},
         "router_scan_gbs": round(achieved, 1),
         "roofline": {"kernel": ("msa_route_topk (tensor-core scan: query fold + tcgen05 scan + "
                                "document top-k)" if wk.scan == "tc" else
@@ -388,12 +419,14 @@ def run_libmsa(args):
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": Kst * wk.L * wk.kernels_per_layer,
+        "route_calls_timed": len(route_ms),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_layers)
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph, e_graph  # graphs are released before the process group
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

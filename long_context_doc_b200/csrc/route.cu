@@ -367,6 +367,18 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   __threadfence();
   const int64_t total = G * p.k;
   for (int b = warp; b < p.B; b += kWarps) {
+    // tau = the largest k-th-best key over the CTAs: that CTA alone holds k keys >= tau, so no
+    // key below tau can be in the global top-k; only the keys >= tau are inserted
+    unsigned long long tau = 0ull;
+    for (int64_t c = lane; c < G; c += 32) {
+      const unsigned long long kth = __ldcg(p.cand + (c * p.B + b) * p.k + (p.k - 1));
+      tau = kth > tau ? kth : tau;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, tau, o);
+      tau = other > tau ? other : tau;
+    }
     unsigned long long lst = 0ull;
     for (int64_t base = 0; base < total; base += 8 * 32) {
       unsigned long long key[8];  // eight independent loads in flight per lane
@@ -376,7 +388,7 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
         key[j] = idx < total ? __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k) : 0ull;
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) list_insert(lst, key[j], lane, p.k);
+      for (int j = 0; j < 8; ++j) list_insert(lst, key[j] >= tau ? key[j] : 0ull, lane, p.k);
     }
     if (lane < p.k) {
       p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
