@@ -298,14 +298,17 @@ def run_libmsa(args):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=wk.main):
             wk.step()
-        graph.replay()
     barrier()
 
     def run_step():
         if graph is not None:
-            graph.replay()
+            with torch.cuda.stream(wk.main):  # replay on the stream the timing events use
+                graph.replay()
         else:
             wk.step()
+
+    run_step()
+    barrier()
 
     Kst = args.steps
     uuid = str(torch.cuda.get_device_properties(local).uuid)
@@ -367,7 +370,8 @@ def run_libmsa(args):
         e_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(e_graph, stream=wk.main):
             e2e_step()
-        e_graph.replay()
+        with torch.cuda.stream(wk.main):
+            e_graph.replay()
         barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -375,7 +379,8 @@ def run_libmsa(args):
     e0.record(wk.main)
     for _ in range(Ke):
         if e_graph is not None:
-            e_graph.replay()
+            with torch.cuda.stream(wk.main):
+                e_graph.replay()
         else:
             e2e_step()
     e1.record(wk.main)
