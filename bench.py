@@ -57,16 +57,19 @@ def parse():
     return ap.parse_args()
 
 
-def captured_traffic(kernel_src: str, summary: str):
+def captured_traffic(kernel_srcs, summary: str):
     """DRAM bytes (read + write) of one launch from a committed ncu capture, or None when the
-    kernel source changed since the capture (the summary records its SHA-256)."""
+    kernel's sources changed since the capture (the summary records the SHA-256 of the
+    sources concatenated in the order given)."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", summary)) as f:
             rec = json.load(f)
-        with open(os.path.join(ROOT, "long_context_doc_b200", "csrc", kernel_src), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        if rec.get("kernel_src_sha256") != sha:
+        h = hashlib.sha256()
+        for src in kernel_srcs:
+            with open(os.path.join(ROOT, "long_context_doc_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+        if rec.get("kernel_src_sha256") != h.hexdigest():
             return None
         return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
     except Exception:
@@ -417,7 +420,8 @@ def run_libmsa(args):
                                "msa_route_topk (CUDA-core scan with fused top-k)"), "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": (captured_traffic("route_tc.cu", f"route_tc_{w.name}_dram.json")
+                     "traffic": (captured_traffic(("route_tc.cu", "common.cuh"),
+                                                   f"route_tc_{w.name}_dram.json")
                                  if wk.scan == "tc" else None),
                      "bytes_per_launch": wk.scan_bytes(),
                      "avg_launch_ms": round(route_avg, 4)},

@@ -159,4 +159,199 @@ __device__ __forceinline__ int64_t lower_bound_i64(const int64_t* off, int64_t n
   return lo;
 }
 
+// The same search by one warp with 32-way splits: ceil(log32(n)) + 1 dependent loads instead
+// of log2(n). Needs x <= off[n]. Every lane returns j; *val = off[j].
+__device__ __forceinline__ int64_t warp_lower_bound(const int64_t* off, int64_t n, int64_t x,
+                                                    int lane, int64_t* val) {
+  int64_t lo = 0, hi = n;  // off[lo - 1] < x <= off[hi]
+  while (hi - lo >= 32) {
+    const int64_t pos = lo + ((hi - lo) * (lane + 1)) / 32;  // lane 31 probes hi
+    const unsigned m = __ballot_sync(0xffffffffu, __ldg(off + pos) >= x);
+    const int f = __ffs(m) - 1;
+    const int64_t prev = __shfl_sync(0xffffffffu, pos, f > 0 ? f - 1 : 0);
+    hi = __shfl_sync(0xffffffffu, pos, f);
+    lo = f > 0 ? prev + 1 : lo;
+  }
+  const int64_t pos = lo + lane;
+  const int64_t v = pos <= hi ? __ldg(off + pos) : INT64_MAX;
+  const int f = __ffs(__ballot_sync(0xffffffffu, v >= x)) - 1;
+  *val = __shfl_sync(0xffffffffu, v, f);
+  return lo + f;
+}
+
+// Document-aligned chunk range of CTA i of G: documents [D0, D1) whose chunks [cb, ce) start
+// in the CTA's equal share of the n_chunks rows (the last CTA takes every remaining document).
+// Run by warps 0 and 1 of the block (whole warps); writes {D0, D1, cb, ce} to out, which the
+// block reads after its next barrier.
+__device__ __forceinline__ void cta_doc_range(const int64_t* coff, int64_t n_docs,
+                                              int64_t n_chunks, int64_t i, int64_t G,
+                                              int64_t* out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp > 1) return;
+  int64_t D, cv;
+  if (warp == 1 && i == G - 1) {
+    D = n_docs;
+    cv = __ldg(coff + n_docs);
+  } else {
+    D = warp_lower_bound(coff, n_docs, ((i + warp) * n_chunks) / G, lane, &cv);
+  }
+  if (lane == 0) {
+    out[warp] = D;
+    out[2 + warp] = cv;
+  }
+}
+
+// ---------------------------------------------------------------- warp top-k lists
+// Insert the lanes' candidate keys into the warp-held sorted list (lane i < k holds the
+// i-th largest key; 0 = empty).
+__device__ __forceinline__ void list_insert(unsigned long long& li, unsigned long long key,
+                                            int lane, int k) {
+  const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
+  unsigned m = __ballot_sync(0xffffffffu, key > thr);
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    const unsigned long long x = __shfl_sync(0xffffffffu, key, src);
+    const unsigned gt = __ballot_sync(0xffffffffu, lane < k && li > x);
+    const int pos = __popc(gt);
+    const unsigned long long up = __shfl_up_sync(0xffffffffu, li, 1);
+    if (pos < k) {
+      if (lane > pos && lane < k) li = up;
+      if (lane == pos) li = x;
+    }
+  }
+}
+
+__device__ __forceinline__ void cp_async16_cg(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+
+// Merge of one query's per-CTA lists by insertion: every key >= tau enters the warp-held
+// top-k list (cand rows of CTA c for query b start at (c * B + b) * k).
+__device__ __forceinline__ unsigned long long merge_by_insertion(const unsigned long long* src,
+                                                                 bool in_smem, int G, int B, int b,
+                                                                 int k, unsigned long long tau,
+                                                                 int lane) {
+  unsigned long long lst = 0ull;
+  for (int c0 = 0; c0 < G; c0 += 32) {
+    const int c = c0 + lane;
+    const int row = (c * B + b) * k;
+    for (int j = 0; j < k; ++j) {
+      unsigned long long key = 0ull;
+      if (c < G) key = in_smem ? src[row + j] : __ldcg(src + row + j);
+      key = key >= tau ? key : 0ull;
+      if (__ballot_sync(0xffffffffu, key != 0ull) == 0u) break;  // lists are sorted
+      list_insert(lst, key, lane, k);
+    }
+  }
+  return lst;
+}
+
+constexpr int kMergeCap = 256;  // survivors ranked directly, per warp
+
+// Final merge of the per-CTA candidate lists cand[G][B][k] (run by the last CTA, every thread
+// of the block). Each list is sorted (descending keys, 0 = empty) and the keys of different
+// lists are distinct. The lists are first copied into shared memory with every copy in
+// flight; warp w then takes queries w, w + nwarps, ...:
+//   tau = max(largest k-th key of a list, largest per-lane maximum of the list heads that at
+//         least k per-lane maxima reach): either way at least k distinct keys are >= tau,
+//         so the global top-k lies in the keys >= tau;
+//   the keys >= tau (a prefix of every list) are compacted into a per-warp buffer and each
+//         one's rank is the number of larger survivors: rank r < k goes to output slot r.
+// A query with more than kMergeCap survivors (or a block without the shared memory) falls
+// back to inserting the keys >= tau into a warp-held sorted list.
+__device__ __forceinline__ void merge_candidates(const unsigned long long* cand, int G, int B,
+                                                 int k, unsigned char* smem, size_t smem_bytes,
+                                                 int32_t* top_ids, float* top_scores) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
+  const int n = G * B * k;
+  const bool staged = (size_t)(n + nwarps * kMergeCap) * 8 <= smem_bytes;
+  const unsigned long long* src = cand;
+  unsigned long long* surv = nullptr;
+  if (staged) {
+    fence_proxy_async_smem();  // the region last held bulk-copied operand tiles
+    unsigned long long* dst = reinterpret_cast<unsigned long long*>(smem);
+    for (int i = 2 * tid; i + 1 < n; i += 2 * nthreads) cp_async16_cg(dst + i, cand + i);
+    if ((n & 1) && tid == 0) dst[n - 1] = __ldcg(cand + n - 1);
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    src = dst;
+    surv = dst + n + warp * kMergeCap;
+  }
+  for (int b = warp; b < B; b += nwarps) {
+    // largest k-th key of a list
+    unsigned long long tau = 0ull;
+    for (int c = lane; c < G; c += 32) {
+      const int at = (c * B + b) * k + (k - 1);
+      const unsigned long long kth = staged ? src[at] : __ldcg(src + at);
+      tau = kth > tau ? kth : tau;
+    }
+    // lane maxima of the list heads: heads of different lists are distinct documents, so the
+    // largest lane maximum that k of the 32 lane maxima reach is a lower bound as well
+    {
+      unsigned long long hm = 0ull;
+      for (int c = lane; c < G; c += 32) {
+        const int at = (c * B + b) * k;
+        const unsigned long long h = staged ? src[at] : __ldcg(src + at);
+        hm = h > hm ? h : hm;
+      }
+      int ge = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ge += __shfl_sync(0xffffffffu, hm, j) >= hm ? 1 : 0;
+      if (hm != 0ull && ge >= k) tau = hm > tau ? hm : tau;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, tau, o);
+      tau = other > tau ? other : tau;
+    }
+    // compact the survivors
+    int total = 0;
+    if (staged) {
+      for (int c0 = 0; c0 < G; c0 += 32) {
+        const int c = c0 + lane;
+        const int row = (c * B + b) * k;
+        int m = 0;
+        if (c < G)
+          while (m < k && src[row + m] != 0ull && src[row + m] >= tau) ++m;
+        int incl = m;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const int at = total + incl - m;
+        if (at + m <= kMergeCap)
+          for (int j = 0; j < m; ++j) surv[at + j] = src[row + j];
+        total += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      __syncwarp();
+    }
+    if (staged && total <= kMergeCap) {
+      for (int i = lane; i < total; i += 32) {
+        const unsigned long long x = surv[i];
+        int r = 0;
+        for (int j = 0; j < total; ++j) r += surv[j] > x ? 1 : 0;
+        if (r < k) {
+          top_ids[b * k + r] = key_id(x);
+          top_scores[b * k + r] = key_score(x);
+        }
+      }
+      if (lane < k && lane >= total) {
+        top_ids[b * k + lane] = -1;
+        top_scores[b * k + lane] = -INFINITY;
+      }
+      __syncwarp();  // the buffer is refilled for the warp's next query
+    } else {
+      const unsigned long long lst = merge_by_insertion(src, staged, G, B, b, k, tau, lane);
+      if (lane < k) {
+        top_ids[b * k + lane] = lst ? key_id(lst) : -1;
+        top_scores[b * k + lane] = lst ? key_score(lst) : -INFINITY;
+      }
+    }
+  }
+}
+
 }  // namespace msa

@@ -65,26 +65,6 @@ __device__ __forceinline__ void tr_reduce(float* v, int lane) {
   }
 }
 
-// Insert the lanes' candidate keys into the warp-held sorted list (lane i < k holds the
-// i-th largest key; 0 = empty).
-__device__ __forceinline__ void list_insert(unsigned long long& li, unsigned long long key,
-                                            int lane, int k) {
-  const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
-  unsigned m = __ballot_sync(0xffffffffu, key > thr);
-  while (m) {
-    const int src = __ffs(m) - 1;
-    m &= m - 1;
-    const unsigned long long x = __shfl_sync(0xffffffffu, key, src);
-    const unsigned gt = __ballot_sync(0xffffffffu, lane < k && li > x);
-    const int pos = __popc(gt);
-    const unsigned long long up = __shfl_up_sync(0xffffffffu, li, 1);
-    if (pos < k) {
-      if (lane > pos && lane < k) li = up;
-      if (lane == pos) li = x;
-    }
-  }
-}
-
 template <typename T, int R, int E>
 __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   using VecT = Vec<T, E>;
@@ -114,20 +94,24 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   unsigned long long* lists = reinterpret_cast<unsigned long long*>(win + kWin + 1);  // [R][32]
   float* carry = reinterpret_cast<float*>(lists + R * 32);                    // [R]
   uint64_t* mbar = reinterpret_cast<uint64_t*>(carry + ((R + 1) & ~1) + 2);   // [S]
-  int64_t* docs = reinterpret_cast<int64_t*>(mbar + kStages);                 // [0..1] cur, [2] win0
-  int* flags = reinterpret_cast<int*>(docs + 3);                              // [0] last
+  // [0..1] current doc, [2] window start, [3..6] this CTA's {D0, D1, cb, ce}
+  int64_t* docs = reinterpret_cast<int64_t*>(mbar + kStages);
+  int* flags = reinterpret_cast<int*>(docs + 7);                              // [0] last
 
   // ---- document-aligned chunk range of this CTA
   const int64_t G = gridDim.x;
   const int64_t i = blockIdx.x;
-  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (i * p.n_chunks) / G);
-  const int64_t D1 = (i == G - 1) ? p.n_docs
-                                  : lower_bound_i64(p.coff, p.n_docs, ((i + 1) * p.n_chunks) / G);
-  const int64_t cb = p.coff[D0], ce = p.coff[D1];
-  const int64_t n_tiles = (ce - cb + TC - 1) / TC;
+  cta_doc_range(p.coff, p.n_docs, p.n_chunks, i, G, docs + 3);
   const T* kr = static_cast<const T*>(p.kr);
   const size_t row_bytes = (size_t)W * sizeof(T);
 
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t D0 = docs[3], D1 = docs[4], cb = docs[5], ce = docs[6];
+  const int64_t n_tiles = (ce - cb + TC - 1) / TC;
   auto issue = [&](int s, int64_t t) {
     const int64_t c0 = cb + t * TC;
     const int64_t n = min((int64_t)TC, ce - c0);
@@ -137,14 +121,10 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
     bulk_g2s(stage + (size_t)s * tile_bytes, kr + c0 * W, kb, &mbar[s]);
     if (ib) bulk_g2s(invs + s * TC * p.h_kv, p.invk + c0 * p.h_kv, ib, &mbar[s]);
   };
-
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
-    fence_mbar_init();
     docs[0] = D0;
     docs[2] = D0;
   }
-  __syncthreads();
   if (tid == 0)
     for (int s = 0; s < kStages && s < n_tiles; ++s) issue(s, s);
 
@@ -365,36 +345,8 @@ __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   __syncthreads();
   if (!flags[0]) return;
   __threadfence();
-  const int64_t total = G * p.k;
-  for (int b = warp; b < p.B; b += kWarps) {
-    // tau = the largest k-th-best key over the CTAs: that CTA alone holds k keys >= tau, so no
-    // key below tau can be in the global top-k; only the keys >= tau are inserted
-    unsigned long long tau = 0ull;
-    for (int64_t c = lane; c < G; c += 32) {
-      const unsigned long long kth = __ldcg(p.cand + (c * p.B + b) * p.k + (p.k - 1));
-      tau = kth > tau ? kth : tau;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, tau, o);
-      tau = other > tau ? other : tau;
-    }
-    unsigned long long lst = 0ull;
-    for (int64_t base = 0; base < total; base += 8 * 32) {
-      unsigned long long key[8];  // eight independent loads in flight per lane
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t idx = base + j * 32 + lane;
-        key[j] = idx < total ? __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k) : 0ull;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) list_insert(lst, key[j] >= tau ? key[j] : 0ull, lane, p.k);
-    }
-    if (lane < p.k) {
-      p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
-      p.top_scores[b * p.k + lane] = lst ? key_score(lst) : -INFINITY;
-    }
-  }
+  merge_candidates(p.cand, (int)G, p.B, p.k, stage, (size_t)kStages * tile_bytes, p.top_ids,
+                   p.top_scores);
 }
 
 // ------------------------------------------------------------------------------- launch
@@ -409,7 +361,7 @@ static size_t route_smem_bytes(int W, int h_kv, int h_qr) {
   s = (s + 7) & ~(size_t)7;
   s += sizeof(int64_t) * (kWin + 1) + sizeof(unsigned long long) * R * 32;
   s += sizeof(float) * (((R + 1) & ~1) + 2);
-  s += sizeof(uint64_t) * kStages + sizeof(int64_t) * 3 + sizeof(int) * 4;
+  s += sizeof(uint64_t) * kStages + sizeof(int64_t) * 7 + sizeof(int) * 4;
   return (s + 127) & ~(size_t)127;
 }
 

@@ -185,24 +185,6 @@ struct TcParams {
 
 constexpr int kTcWin = 1024;  // document offsets cached in shared memory
 
-__device__ __forceinline__ void list_insert_tc(unsigned long long& li, unsigned long long key,
-                                               int lane, int k) {
-  const unsigned long long thr = __shfl_sync(0xffffffffu, li, k - 1);
-  unsigned m = __ballot_sync(0xffffffffu, key > thr);
-  while (m) {
-    const int src = __ffs(m) - 1;
-    m &= m - 1;
-    const unsigned long long x = __shfl_sync(0xffffffffu, key, src);
-    const unsigned gt = __ballot_sync(0xffffffffu, lane < k && li > x);
-    const int pos = __popc(gt);
-    const unsigned long long up = __shfl_up_sync(0xffffffffu, li, 1);
-    if (pos < k) {
-      if (lane > pos && lane < k) li = up;
-      if (lane == pos) li = x;
-    }
-  }
-}
-
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* err,
                                              volatile int* abort_flag) {
   if (*abort_flag) return false;
@@ -237,23 +219,17 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   uint64_t* tfull = empty + kTcMaxStages;  // [2]
   uint64_t* tempty = tfull + 2;            // [2]
   uint64_t* done = tempty + 2;             // MMA issuer: every issued MMA has completed
-  int64_t* docs = reinterpret_cast<int64_t*>(done + 1);  // [0..1] current doc, [2] window start
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(docs + 3);
+  // [0..1] current doc, [2] window start, [3..6] this CTA's {D0, D1, cb, ce}
+  int64_t* docs = reinterpret_cast<int64_t*>(done + 1);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(docs + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_k = p.K / kTcBK;
 
-  // document-aligned chunk range of this CTA
   const int64_t G = gridDim.x, ci = blockIdx.x;
-  const int64_t D0 = lower_bound_i64(p.coff, p.n_docs, (ci * p.n_chunks) / G);
-  const int64_t D1 = (ci == G - 1) ? p.n_docs
-                                   : lower_bound_i64(p.coff, p.n_docs, ((ci + 1) * p.n_chunks) / G);
-  const int64_t cb = p.coff[D0], ce = p.coff[D1];
-  const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
-  const int64_t n_units = n_ct * p.n_qtiles;
-
+  cta_doc_range(p.coff, p.n_docs, p.n_chunks, ci, G, docs + 3);
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -265,12 +241,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     }
     mbar_init(done, 1);
     *abort_flag = 0;
-    docs[0] = D0;
-    docs[2] = D0;
     fence_mbar_init();
   }
-  for (int j = threadIdx.x; j <= kTcWin; j += kTcThreads)
-    win[j] = (D0 + j <= D1) ? p.coff[D0 + j] : INT64_MAX;
   for (int j = threadIdx.x; j < p.B * 32; j += kTcThreads) lists[j] = 0ull;
   for (int j = threadIdx.x; j < p.B; j += kTcThreads) carry[j] = -INFINITY;
   if (warp == 0) {  // two fp32 accumulators of up to 256 columns
@@ -284,6 +256,9 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const int64_t D0 = docs[3], D1 = docs[4], cb = docs[5], ce = docs[6];
+  const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
+  const int64_t n_units = n_ct * p.n_qtiles;
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -346,6 +321,14 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int row = lg * 32 + lane;          // chunk row of the tile (TMEM lane)
     const int ncols = p.NQ * p.T;
     bool aborted = false;
+    // document-offset window (the producer is already streaming the first tiles)
+    for (int j = ew * 32 + lane; j <= kTcWin; j += 128)
+      win[j] = (D0 + j <= D1) ? __ldg(p.coff + D0 + j) : INT64_MAX;
+    if (ew == 0 && lane == 0) {
+      docs[0] = D0;
+      docs[2] = D0;
+    }
+    epi_sync();
     for (int64_t u = 0; u < n_units; ++u) {
       const int a = (int)(u & 1);
       const uint32_t aph = (uint32_t)((u >> 1) & 1);
@@ -416,7 +399,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
             if (!ex) key = score_key(sc, (uint32_t)doc);
           }
-          list_insert_tc(lst, key, lane, p.k);
+          list_insert(lst, key, lane, p.k);
           const unsigned cont = __ballot_sync(0xffffffffu, valid && !fin);
           const unsigned vm = __ballot_sync(0xffffffffu, valid);
           if (cont) {
@@ -450,7 +433,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 p.excl && ((p.excl[(int64_t)b * p.words + (doc >> 5)] >> (doc & 31)) & 1u);
             if (!ex) key = score_key(-INFINITY, (uint32_t)doc);
           }
-          list_insert_tc(lst, key, lane, p.k);
+          list_insert(lst, key, lane, p.k);
         }
         if (lane < p.k) lists[b * 32 + lane] = lst;
       }
@@ -475,36 +458,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   __syncthreads();
   if (!*last_flag) return;
   __threadfence();
-  const int64_t total = G * p.k;
-  for (int b = warp; b < p.B; b += kTcThreads / 32) {
-    // tau = the largest k-th-best key over the CTAs: that CTA alone holds k keys >= tau, so no
-    // key below tau can be in the global top-k; only the keys >= tau are inserted
-    unsigned long long tau = 0ull;
-    for (int64_t c = lane; c < G; c += 32) {
-      const unsigned long long kth = __ldcg(p.cand + (c * p.B + b) * p.k + (p.k - 1));
-      tau = kth > tau ? kth : tau;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, tau, o);
-      tau = other > tau ? other : tau;
-    }
-    unsigned long long lst = 0ull;
-    for (int64_t bs = 0; bs < total; bs += 8 * 32) {
-      unsigned long long key[8];  // eight independent loads in flight per lane
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t idx = bs + j * 32 + lane;
-        key[j] = idx < total ? __ldcg(p.cand + ((idx / p.k) * p.B + b) * p.k + idx % p.k) : 0ull;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) list_insert_tc(lst, key[j] >= tau ? key[j] : 0ull, lane, p.k);
-    }
-    if (lane < p.k) {
-      p.top_ids[b * p.k + lane] = lst ? key_id(lst) : -1;
-      p.top_scores[b * p.k + lane] = lst ? key_score(lst) : -INFINITY;
-    }
-  }
+  merge_candidates(p.cand, (int)G, p.B, p.k, base, (size_t)S * stage_bytes, p.top_ids,
+                   p.top_scores);
 }
 
 // ------------------------------------------------------------------ host side
@@ -557,7 +512,7 @@ TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, 
   pl.cand_bytes = (((size_t)pl.grid * B * k * 8) + 255) & ~(size_t)255;
   const size_t stage = (((size_t)kTcBM * kTcBK * 2 + (size_t)pl.N * kTcBK * 2) + 1023) & ~(size_t)1023;
   const size_t fixed = (size_t)kTcBM * B * 4 + (kTcWin + 1) * 8 + (size_t)B * 32 * 8 +
-                       ((B + 1) & ~1) * 4 + (2 * kTcMaxStages + 5) * 8 + 3 * 8 + 16;
+                       ((B + 1) & ~1) * 4 + (2 * kTcMaxStages + 5) * 8 + 7 * 8 + 16;
   const size_t budget = 227 * 1024 - 1024 - fixed - 64;
   pl.stages = (int)std::min<size_t>(kTcMaxStages, budget / stage);
   if (pl.stages < 2) pl.ok = false;
