@@ -481,7 +481,13 @@ size_t msa_sparse_attend_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_
                                    int32_t max_ctx, int32_t L_loc) {
   if (B < 1 || T < 1 || h_q < 1 || h_kv < 1 || d < 2 || max_ctx < 0 || L_loc < 1) return kHeader;
   const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
-  return kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes + pl.ctr_bytes;
+  size_t need = kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes + pl.ctr_bytes;
+  if (h_q % h_kv == 0) {  // the decode kernel (bf16) lays out the same workspace differently
+    const msa::DecPlan dp = msa::attend_dec_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
+    if (dp.ok)
+      need = std::max(need, kHeader + dp.ctr_bytes + dp.part_ml_bytes + dp.part_o_bytes);
+  }
+  return need;
 }
 
 msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
@@ -503,6 +509,49 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
   REQUIRE(aligned16(Q) && aligned16(K_loc) && aligned16(V_loc) &&
               (max_ctx == 0 || (aligned16(ctxK) && aligned16(ctxV))),
           MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  if (dtype == 1) {
+    const msa::DecPlan dp = msa::attend_dec_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
+    if (dp.ok) {
+      const size_t need = kHeader + dp.ctr_bytes + dp.part_ml_bytes + dp.part_o_bytes;
+      REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+              MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes,
+              need);
+      unsigned char* w8 = static_cast<unsigned char*>(ws);
+      msa::DecParams q{};
+      q.Q = static_cast<const __nv_bfloat16*>(Q);
+      q.Kl = static_cast<const __nv_bfloat16*>(K_loc);
+      q.Vl = static_cast<const __nv_bfloat16*>(V_loc);
+      q.cK = static_cast<const __nv_bfloat16*>(ctxK);
+      q.cV = static_cast<const __nv_bfloat16*>(ctxV);
+      q.ctx_len = ctx_len;
+      q.B = B;
+      q.T = T;
+      q.h_q = h_q;
+      q.h_kv = h_kv;
+      q.L = L_loc;
+      q.max_ctx = max_ctx;
+      q.rope = rope_base > 0.f ? 1 : 0;
+      q.pos0 = pos0;
+      q.rope_base = (double)rope_base;
+      q.scale_log2 = sc * 1.4426950408889634f;
+      q.TPP = dp.TPP;
+      q.CT = dp.CT;
+      q.max_seg = dp.max_seg;
+      q.total = dp.total;
+      q.err = reinterpret_cast<int*>(w8);
+      q.counters = reinterpret_cast<unsigned int*>(w8 + kHeader);
+      q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);
+      q.part_o = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes + dp.part_ml_bytes);
+      q.O = static_cast<__nv_bfloat16*>(O);
+      cudaStream_t st = (cudaStream_t)stream;
+      // status word and segment tickets start at zero
+      cudaError_t e = cudaMemsetAsync(ws, 0, kHeader + dp.ctr_bytes, st);
+      if (e == cudaSuccess) e = msa::launch_attend_dec(q, dp, st);
+      if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
+      return ok();
+    }
+  }
   const msa::AttendPlan pl = msa::attend_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
   const size_t need = kHeader + pl.cs_bytes + pl.part_o_bytes + pl.part_ml_bytes + pl.ctr_bytes;
   REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
@@ -524,7 +573,6 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
   p.max_ctx = max_ctx;
   p.rope = rope_base > 0.f ? 1 : 0;
   p.cs = reinterpret_cast<const float2*>(base);
-  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
   p.scale_log2 = sc * 1.4426950408889634f;
   p.S = pl.S;
   p.KPS = pl.KPS;

@@ -96,6 +96,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // One-dimensional bulk copy global -> shared, completion counted on `bar` in bytes.
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
@@ -198,6 +202,32 @@ __device__ __forceinline__ void cta_doc_range(const int64_t* coff, int64_t n_doc
   if (lane == 0) {
     out[warp] = D;
     out[2 + warp] = cv;
+  }
+}
+
+// ---------------------------------------------------------------- warp reductions
+// Transposing warp reduction of N values per lane: at each of the five butterfly steps a lane
+// keeps one half of its values, sends the other half to its XOR partner and adds what it
+// receives, so the values per lane halve while every kept value gathers more lanes. After the call,
+// if N >= 32 lane l holds flat indices [l*N/32, (l+1)*N/32) in v[0..N/32); otherwise v[0]
+// holds index l / (32/N), summed over all 32 lanes.
+template <int N, int O>
+__device__ __forceinline__ void tr_reduce(float* v, int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (N >= 2) {
+      constexpr int H = N / 2;
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < H; ++i) {
+        const float send = up ? v[i] : v[i + H];
+        const float keep = up ? v[i + H] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      tr_reduce<H, O / 2>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      tr_reduce<1, O / 2>(v, lane);
+    }
   }
 }
 

@@ -1,6 +1,7 @@
 // kernels.cuh - parameter blocks and launchers of the libmsa kernels (internal).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstddef>
@@ -122,5 +123,40 @@ struct AttendPlan {
 };
 AttendPlan attend_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0, cudaStream_t st);
+
+// route_tc.cu: bf16 tensor map (no swizzle, zero fill out of bounds) of a rank-dimensional
+// array: dims innermost first, strides[rank - 1] in bytes, box in elements.
+bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box);
+
+// ---- attend_dec.cu: decode-shaped attention (bf16, d = 128, <= 8 query rows per KV head)
+struct DecParams {
+  const __nv_bfloat16* Q;   // [B, T, h_q, 128]
+  const __nv_bfloat16* Kl;  // [B, L, h_kv, 128]
+  const __nv_bfloat16* Vl;
+  const __nv_bfloat16* cK;  // [B, max_ctx, h_kv, 128]
+  const __nv_bfloat16* cV;
+  const int32_t* ctx_len;
+  int B, T, h_q, h_kv, L, max_ctx;
+  int rope, pos0;
+  double rope_base;
+  float scale_log2;
+  int TPP, CT, max_seg;     // 64-key tiles per (query, KV head) pair, of which the first CT
+                            // hold memory rows and the rest local rows; segments per pair
+  int64_t total;            // B * h_kv * TPP
+  float* part_o;            // [pairs, max_seg, RB, 128]
+  float* part_ml;           // [pairs, max_seg, RB, 2]
+  unsigned int* counters;   // [pairs] segment tickets (zeroed per call)
+  int* err;                 // workspace status word
+  __nv_bfloat16* O;         // [B, T, h_q, 128]
+};
+struct DecPlan {
+  bool ok;
+  int RB, TPP, CT, grid, max_seg;
+  int64_t n_pairs, total;
+  size_t ctr_bytes, part_ml_bytes, part_o_bytes, smem;
+};
+DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
+cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
 
 }  // namespace msa

@@ -42,29 +42,6 @@ template <int R> __host__ __device__ constexpr int kSubOf() { return 8 / kUof<R>
 constexpr int kStages = 3;  // bulk-copy pipeline depth
 constexpr int kWin = 1024;  // document offsets cached in shared memory
 
-// Transposing warp reduction of N values per lane (see header comment). After the call,
-// if N >= 32 lane l holds flat indices [l*N/32, (l+1)*N/32) in v[0..N/32); otherwise v[0]
-// holds index l / (32/N), summed over all 32 lanes.
-template <int N, int O>
-__device__ __forceinline__ void tr_reduce(float* v, int lane) {
-  if constexpr (O >= 1) {
-    if constexpr (N >= 2) {
-      constexpr int H = N / 2;
-      const bool up = (lane & O) != 0;
-#pragma unroll
-      for (int i = 0; i < H; ++i) {
-        const float send = up ? v[i] : v[i + H];
-        const float keep = up ? v[i + H] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
-      }
-      tr_reduce<H, O / 2>(v, lane);
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
-      tr_reduce<1, O / 2>(v, lane);
-    }
-  }
-}
-
 template <typename T, int R, int E>
 __global__ void __launch_bounds__(kNT, 1) route_scan_kernel(RouteParams p) {
   using VecT = Vec<T, E>;

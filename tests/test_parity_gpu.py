@@ -401,6 +401,12 @@ def _attend_case(msa, gpu, dt, B, T, h_q, h_kv, d, L, n_ctx, pos0, base, seed=0)
     ("bf16", 1, 128, 32, 8, 128, 128, [256], 16, 1e6),  # 1M-bank prefill shape
     ("fp32", 3, 5, 8, 2, 128, 40, [0, 9, 33], 7, 1e4),  # T < L, one query without memory
     ("bf16", 2, 3, 4, 4, 64, 3, [5, 300], 2, 0.0),      # RoPE off, MHA, long memory
+    # decode-shaped (bf16, d = 128, <= 8 query rows per KV head): the streaming decode kernel
+    ("bf16", 3, 2, 16, 4, 128, 100, [0, 64, 130], 16, 1e6),  # 8 rows, causal over 2 tokens
+    ("bf16", 2, 1, 8, 2, 128, 40, [20, 3], 4, 1e6),     # one tile per pair (no split merge)
+    ("bf16", 2, 1, 4, 4, 128, 300, [50, 0], 3, 1e4),    # one row per KV head, no memory
+    ("bf16", 1, 1, 8, 2, 128, 200, [70], 2, 0.0),       # RoPE off
+    ("bf16", 2, 1, 32, 8, 128, 1024, [96, 128], 5000, 1e6),  # positions up to 6k
     ("fp32", 1, 1, 2, 1, 64, 1, [1], 0, 1e6),           # one memory row + the query itself
 ])
 def test_attend_matches_oracle(msa, gpu, dt, B, T, h_q, h_kv, d, L, ctx, pos0, base):
