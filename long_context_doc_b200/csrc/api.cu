@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cstdarg>
 #include <chrono>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -533,12 +534,23 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       q.max_ctx = max_ctx;
       q.rope = rope_base > 0.f ? 1 : 0;
       q.pos0 = pos0;
-      q.rope_base = (double)rope_base;
+      for (int i = 0; i < 64; ++i) {  // theta_i / (2 pi) mod 1 in 64-bit fixed point
+        unsigned long long F = 0;
+        if (q.rope) {
+          const long double pi2 = 6.283185307179586476925286766559005768L;
+          long double f = powl((long double)rope_base, -2.0L * i / 128.0L) / pi2;
+          f -= floorl(f);
+          const long double scaled = ldexpl(f, 64);
+          F = scaled >= 18446744073709551615.0L ? ~0ull : (unsigned long long)scaled;
+        }
+        q.rope_turns[i] = F;
+      }
       q.scale_log2 = sc * 1.4426950408889634f;
       q.TPP = dp.TPP;
       q.CT = dp.CT;
       q.max_seg = dp.max_seg;
       q.total = dp.total;
+      q.grid = dp.grid;
       q.err = reinterpret_cast<int*>(w8);
       q.counters = reinterpret_cast<unsigned int*>(w8 + kHeader);
       q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);

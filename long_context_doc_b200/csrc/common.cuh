@@ -135,6 +135,33 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait by polling (non-blocking test, short sleeps between tests): for waits whose
+// phase usually completes within a microsecond or two, where a blocking try_wait can keep the
+// thread suspended well past the completion. Same limit and error as mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_wait_poll_bounded(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test_wait(bar, parity)) {
+    __nanosleep(32);
+    if (clock64() - t0 > (1ll << 31)) {
+      set_err(err, kErrWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- order-preserving keys
 // 64-bit key: larger key = larger score, then lower doc id. 0 is "empty".
 __device__ __forceinline__ unsigned long long score_key(float s, uint32_t id) {

@@ -129,7 +129,8 @@ cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0,
 bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box);
 
-// ---- attend_dec.cu: decode-shaped attention (bf16, d = 128, <= 8 query rows per KV head)
+// ---- attend_dec.cu: decode-shaped attention (bf16, d = 128, <= 8 query rows per KV head,
+// h_kv in {1, 2, 4, 8})
 struct DecParams {
   const __nv_bfloat16* Q;   // [B, T, h_q, 128]
   const __nv_bfloat16* Kl;  // [B, L, h_kv, 128]
@@ -139,21 +140,23 @@ struct DecParams {
   const int32_t* ctx_len;
   int B, T, h_q, h_kv, L, max_ctx;
   int rope, pos0;
-  double rope_base;
+  unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions,
+                                      // theta_i = base^(-2i/128); all zero without RoPE
   float scale_log2;
-  int TPP, CT, max_seg;     // 64-key tiles per (query, KV head) pair, of which the first CT
-                            // hold memory rows and the rest local rows; segments per pair
-  int64_t total;            // B * h_kv * TPP
-  float* part_o;            // [pairs, max_seg, RB, 128]
-  float* part_ml;           // [pairs, max_seg, RB, 2]
-  unsigned int* counters;   // [pairs] segment tickets (zeroed per call)
+  int TPP, CT, max_seg;     // tiles of 64/h_kv key rows per query, of which the first CT hold
+                            // memory rows and the rest local rows; segments per query
+  int64_t total;            // B * TPP
+  int grid;                 // CTAs of the attention kernel (tile ranges)
+  float* part_o;            // [B, max_seg, h_kv, RB, 128]
+  float* part_ml;           // [B, max_seg, h_kv, RB, 2]
+  unsigned int* counters;   // [B] (reserved; zeroed per call)
   int* err;                 // workspace status word
   __nv_bfloat16* O;         // [B, T, h_q, 128]
 };
 struct DecPlan {
   bool ok;
   int RB, TPP, CT, grid, max_seg;
-  int64_t n_pairs, total;
+  int64_t n_pairs, total;   // n_pairs: queries that own tiles (B)
   size_t ctr_bytes, part_ml_bytes, part_o_bytes, smem;
 };
 DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
