@@ -80,6 +80,19 @@ void route_passes(int B, int T, int* bp, int* passes) {
 }  // namespace
 
 namespace msa {
+void rope_turns(double base, int d, unsigned long long* out) {
+  const long double pi2 = 6.283185307179586476925286766559005768L;
+  for (int i = 0; i < d / 2; ++i) {
+    unsigned long long F = 0;
+    if (base > 0.0) {
+      long double f = powl((long double)base, -2.0L * i / (long double)d) / pi2;
+      f -= floorl(f);
+      const long double scaled = ldexpl(f, 64);
+      F = scaled >= 18446744073709551615.0L ? ~0ull : (unsigned long long)scaled;
+    }
+    out[i] = F;
+  }
+}
 // Set the thread-local message returned by msa_last_error (for entry points defined in other
 // translation units).
 void set_last_error(const std::string& msg) { g_err = msg; }
@@ -144,8 +157,22 @@ msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_
                 aligned16(Vbar) && aligned16(Kbar_r),
             MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   }
-  msa::EncodeParams p{K, V, K_r, doc_tok_off, doc_chunk_off, n_docs, n_chunks, chunk, h_kv,
-                      (double)rope_base, Kbar, Vbar, Kbar_r, kr_inv_norm};
+  msa::EncodeParams p{};
+  p.K = K;
+  p.V = V;
+  p.Kr = K_r;
+  p.tok_off = doc_tok_off;
+  p.chunk_off = doc_chunk_off;
+  p.n_docs = n_docs;
+  p.n_chunks = n_chunks;
+  p.chunk = chunk;
+  p.h_kv = h_kv;
+  p.rope = rope_base > 0.f ? 1 : 0;
+  msa::rope_turns(p.rope ? (double)rope_base : 0.0, d, p.rope_turns);
+  p.Kb = Kbar;
+  p.Vb = Vbar;
+  p.Rb = Kbar_r;
+  p.inv_norm = kr_inv_norm;
   cudaError_t e = msa::launch_encode_pool(p, dtype, d, sm_count(), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "msa_encode_pool launch");
   return ok();
@@ -534,17 +561,7 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       q.max_ctx = max_ctx;
       q.rope = rope_base > 0.f ? 1 : 0;
       q.pos0 = pos0;
-      for (int i = 0; i < 64; ++i) {  // theta_i / (2 pi) mod 1 in 64-bit fixed point
-        unsigned long long F = 0;
-        if (q.rope) {
-          const long double pi2 = 6.283185307179586476925286766559005768L;
-          long double f = powl((long double)rope_base, -2.0L * i / 128.0L) / pi2;
-          f -= floorl(f);
-          const long double scaled = ldexpl(f, 64);
-          F = scaled >= 18446744073709551615.0L ? ~0ull : (unsigned long long)scaled;
-        }
-        q.rope_turns[i] = F;
-      }
+      msa::rope_turns(q.rope ? (double)rope_base : 0.0, 128, q.rope_turns);
       q.scale_log2 = sc * 1.4426950408889634f;
       q.TPP = dp.TPP;
       q.CT = dp.CT;

@@ -47,18 +47,6 @@ constexpr uint32_t kDecRow = kDecD * 2;                   // bytes of one (key, 
 constexpr uint32_t kDecHalf = kDecRowsPerTile * kDecRow;  // K (or V) of a tile: 16 KB
 constexpr uint32_t kDecStage = 2 * kDecHalf;
 
-// (cos, sin) of n * theta_i for an integer position n. F = theta_i / (2 pi) mod 1 as a 64-bit
-// binary fraction (host-computed), so n * F mod 2^64 is the exact turn count of the angle mod 1
-// (two's complement for negative n); its top 32 bits, as a signed fraction of a half turn, go
-// to the single-precision sincospi. Angle error < 2^-24 half turns at any position.
-__device__ __forceinline__ float2 rot_turns(int64_t n, unsigned long long F) {
-  const unsigned long long t = (unsigned long long)n * F;
-  const float x = (float)(int)(t >> 32) * 0x1p-31f;  // angle / pi in [-1, 1)
-  float s, c;
-  sincospif(x, &s, &c);
-  return make_float2(c, s);
-}
-
 // First CTA whose tile range contains flattened tile x.
 __device__ __forceinline__ int64_t dec_cta_of(int64_t x, int64_t G, int64_t total) {
   return ((x + 1) * G + total - 1) / total - 1;

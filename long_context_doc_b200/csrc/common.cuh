@@ -162,6 +162,19 @@ __device__ __forceinline__ bool mbar_wait_poll_bounded(uint64_t* bar, uint32_t p
   return true;
 }
 
+// ---------------------------------------------------------------- RoPE angles
+// (cos, sin) of n * theta_i for an integer position n. F = theta_i / (2 pi) mod 1 as a 64-bit
+// binary fraction (host-computed), so n * F mod 2^64 is the exact turn count of the angle mod 1
+// (two's complement for negative n); its top 32 bits, as a signed fraction of a half turn, go
+// to the single-precision sincospi. Angle error < 2^-24 half turns at any position.
+__device__ __forceinline__ float2 rot_turns(int64_t n, unsigned long long F) {
+  const unsigned long long t = (unsigned long long)n * F;
+  const float x = (float)(int)(t >> 32) * 0x1p-31f;  // angle / pi in [-1, 1)
+  float s, c;
+  sincospif(x, &s, &c);
+  return make_float2(c, s);
+}
+
 // ---------------------------------------------------------------- order-preserving keys
 // 64-bit key: larger key = larger score, then lower doc id. 0 is "empty".
 __device__ __forceinline__ unsigned long long score_key(float s, uint32_t id) {

@@ -8,19 +8,24 @@
 //   RoPE whose positions restart at 0 in every document
 //   [news.neo-ai.one, "並列（ドキュメント単位）RoPE"; ruixiangma blog, "文档级RoPE"].
 //
-// Layout: one CTA per chunk (grid-stride). A thread owns one "pair group": E consecutive
+// Layout: each CTA pools a contiguous range of chunks (the owning document advances with the
+// chunk, no search per chunk). A thread owns one "pair group": E consecutive
 // elements of the first half of a head and the E elements they pair with in the second half
 // (RoPE rotates element i with i + d/2), for TP-strided tokens of the chunk; TP lanes that
 // share a pair group sit next to each other in the warp and are reduced with shuffles.
-// cos/sin of the chunk's positions are computed once per CTA in double precision into a
-// shared-memory table (padded rows: conflict-free 16-byte reads).
+// RoPE is linear, so sum_t R((P + c_t) theta) x_t = R(P theta) sum_t R(c_t theta) x_t: for chunks
+// of at most 64 tokens one shared table of R(c theta), c < 64, built once per CTA, serves every
+// chunk, and the chunk's sums are turned by its start position P once (longer chunks rebuild the
+// table per 64-token block). Every cos/sin comes from the exact angle mod 2 pi (integer
+// position x 64-bit fixed-point theta / 2 pi) through a single-precision sincospi; the padded
+// table rows give conflict-free 16-byte reads.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace msa {
 
 
-template <typename T, int E, int D, int TP>
+template <typename T, int E, int D, int TP, bool SINGLE>
 __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
   constexpr int HALF = D / 2;
   constexpr int SUBS = HALF / E;     // pair groups per head
@@ -31,8 +36,8 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   float2* cs = reinterpret_cast<float2*>(smem_raw);                 // [TB][ROW]
-  double* theta = reinterpret_cast<double*>(cs + TB * ROW);         // [HALF]
-  float* ssp = reinterpret_cast<float*>(theta + HALF);              // [PG] partial sum sq
+  unsigned long long* turns = reinterpret_cast<unsigned long long*>(cs + TB * ROW);  // [HALF]
+  float* ssp = reinterpret_cast<float*>(turns + HALF);              // [PG] partial sum sq
 
   const int PG = p.h_kv * SUBS;
   const int tid = threadIdx.x;
@@ -42,20 +47,30 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
   const int h = pg / SUBS;
   const int e1 = (pg % SUBS) * E;    // first-half element offset within the head
   const int W = p.h_kv * D;          // row length
-  const bool rope = p.rope_base > 0.0;
+  const bool rope = p.rope != 0;
 
   if (rope) {
-    for (int i = tid; i < HALF; i += blockDim.x)
-      theta[i] = pow(p.rope_base, -2.0 * (double)i / (double)D);
+    for (int i = tid; i < HALF; i += blockDim.x) turns[i] = p.rope_turns[i];
+    if constexpr (SINGLE) {  // in-chunk offsets 0 .. 63, shared by every chunk
+      __syncthreads();
+      for (int idx = tid; idx < TB * HALF; idx += blockDim.x) {
+        const int pl = idx / HALF, i = idx % HALF;
+        cs[pl * ROW + i] = rot_turns(pl, turns[i]);
+      }
+    }
   }
+  __syncthreads();
 
   const T* K = static_cast<const T*>(p.K);
   const T* Vt = static_cast<const T*>(p.V);
   const T* Kr = static_cast<const T*>(p.Kr);
 
-  for (int64_t c = blockIdx.x; c < p.n_chunks; c += gridDim.x) {
-    // document owning chunk c: off[i] <= c < off[i+1]
-    const int64_t doc = lower_bound_i64(p.chunk_off, p.n_docs, c + 1) - 1;
+  const int64_t c_begin = (int64_t)blockIdx.x * p.n_chunks / gridDim.x;
+  const int64_t c_end = ((int64_t)blockIdx.x + 1) * p.n_chunks / gridDim.x;
+  // document owning chunk c: off[doc] <= c < off[doc+1] (found once, then advanced)
+  int64_t doc = c_begin < c_end ? lower_bound_i64(p.chunk_off, p.n_docs, c_begin + 1) - 1 : 0;
+  for (int64_t c = c_begin; c < c_end; ++c) {
+    while (p.chunk_off[doc + 1] <= c) ++doc;
     const int64_t j = c - p.chunk_off[doc];
     const int64_t tdoc = p.tok_off[doc];
     const int64_t t0 = tdoc + j * p.chunk;
@@ -70,13 +85,11 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
 
     for (int sb = 0; sb < n; sb += TB) {
       const int nb = min(TB, n - sb);
-      if (rope) {
+      if (!SINGLE && rope) {
         __syncthreads();  // the previous table block is no longer read
         for (int idx = tid; idx < nb * HALF; idx += blockDim.x) {
           const int pl = idx / HALF, i = idx % HALF;
-          double s, co;
-          sincos((double)(pos0 + sb + pl) * theta[i], &s, &co);
-          cs[pl * ROW + i] = make_float2((float)co, (float)s);
+          cs[pl * ROW + i] = rot_turns(pos0 + sb + pl, turns[i]);
         }
         __syncthreads();
       }
@@ -113,6 +126,18 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
       }
     }
 
+    if (SINGLE && rope) {  // turn the sums by the chunk's start position
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float2 t = rot_turns(pos0, turns[e1 + e]);
+        const float a = k1[e] * t.x - k2[e] * t.y, b = k2[e] * t.x + k1[e] * t.y;
+        k1[e] = a;
+        k2[e] = b;
+        const float ar = r1[e] * t.x - r2[e] * t.y, br = r2[e] * t.x + r1[e] * t.y;
+        r1[e] = ar;
+        r2[e] = br;
+      }
+    }
     // reduce over the TP lanes sharing this pair group (adjacent lanes)
 #pragma unroll
     for (int o = TP / 2; o > 0; o >>= 1) {
@@ -213,22 +238,31 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int64_t* __re
 }
 
 // ------------------------------------------------------------------------------- launch
-template <typename T, int E, int D, int TP>
-static cudaError_t launch_encode_t(const EncodeParams& p, int sms, cudaStream_t st) {
+template <typename T, int E, int D, int TP, bool SINGLE>
+static cudaError_t launch_encode_s(const EncodeParams& p, int sms, cudaStream_t st) {
   constexpr int HALF = D / 2;
   const int PG = p.h_kv * (HALF / E);
-  const size_t smem = sizeof(float2) * 64 * (HALF + 2) + sizeof(double) * HALF +
+  const size_t smem = sizeof(float2) * 64 * (HALF + 2) + sizeof(unsigned long long) * HALF +
                       sizeof(float) * PG;
-  auto kfn = encode_pool_kernel<T, E, D, TP>;
+  auto kfn = encode_pool_kernel<T, E, D, TP, SINGLE>;
   cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  int64_t grid = p.n_chunks;
-  const int64_t cap = (int64_t)sms * 64;
-  if (grid > cap) grid = cap;
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kfn, PG * TP, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int64_t grid = (int64_t)sms * per_sm;  // every CTA resident; contiguous chunk ranges
+  if (grid > p.n_chunks) grid = p.n_chunks;
   if (grid < 1) grid = 1;
   kfn<<<(unsigned)grid, PG * TP, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+template <typename T, int E, int D, int TP>
+static cudaError_t launch_encode_t(const EncodeParams& p, int sms, cudaStream_t st) {
+  return p.chunk <= 64 ? launch_encode_s<T, E, D, TP, true>(p, sms, st)
+                       : launch_encode_s<T, E, D, TP, false>(p, sms, st);
 }
 
 template <typename T, int E, int D>

@@ -22,7 +22,8 @@ struct EncodeParams {
   const int64_t* chunk_off;  // [n_docs+1] (written by the chunk-offset kernel)
   int64_t n_docs, n_chunks;
   int chunk, h_kv;
-  double rope_base;          // <= 0: no rotation
+  int rope;                  // 0: no rotation
+  unsigned long long rope_turns[128];  // theta_i / (2 pi) mod 1, 64-bit fractions (i < d/2)
   void* Kb;
   void* Vb;
   void* Rb;
@@ -123,6 +124,10 @@ struct AttendPlan {
 };
 AttendPlan attend_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0, cudaStream_t st);
+
+// api.cu: theta_i / (2 pi) mod 1 as 64-bit binary fractions, theta_i = base^(-2i/d), for
+// i < d/2 (all zero when base <= 0)
+void rope_turns(double base, int d, unsigned long long* out);
 
 // route_tc.cu: bf16 tensor map (no swizzle, zero fill out of bounds) of a rank-dimensional
 // array: dims innermost first, strides[rank - 1] in bytes, box in elements.
