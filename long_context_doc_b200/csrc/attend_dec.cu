@@ -454,9 +454,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
 }
 
 // Merge of the partials of the queries split over several CTAs: CTA = one output row (query b,
-// query head h, token t); warp w folds segments w, w + 4, ... with lane l on dims 4l .. 4l+3,
-// then the four warps combine in shared memory.
-__global__ void __launch_bounds__(128) attend_dec_merge_kernel(DecParams p) {
+// query head h, token t); warp w folds segments w, w + 8, ... with lane l on dims 4l .. 4l+3,
+// then the eight warps combine in shared memory.
+constexpr int kMergeWarps = 8;
+__global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int HKV = p.h_kv, Gq = p.h_q / HKV;
   const int row = blockIdx.x;  // ((b * T + t) * h_q + h)
@@ -468,8 +469,8 @@ __global__ void __launch_bounds__(128) attend_dec_merge_kernel(DecParams p) {
   const int64_t last = dec_cta_of((int64_t)b * p.TPP + p.TPP - 1, G, total);
   const int n_seg = (int)(last - first + 1);
   if (n_seg == 1) return;  // written directly by the attention kernel
-  __shared__ float sm_l[4];
-  __shared__ float4 sm_o[4][32];
+  __shared__ float sm_l[kMergeWarps];
+  __shared__ float4 sm_o[kMergeWarps][32];
   auto slot_of = [&](int sg) { return (((int64_t)b * p.max_seg + sg) * HKV + gh) * RB + r; };
   // the row's maximum over all segments
   float M = -INFINITY;
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(128) attend_dec_merge_kernel(DecParams p) {
   float l = 0.f;
   float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
   if (M != -INFINITY) {
-#pragma unroll 4
-    for (int sg = warp; sg < n_seg; sg += 4) {
+#pragma unroll 2
+    for (int sg = warp; sg < n_seg; sg += kMergeWarps) {
       const int64_t sl = slot_of(sg);
       const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + sl * 2));
       const float4 x = __ldcg(reinterpret_cast<const float4*>(p.part_o + sl * kDecD) + lane);
@@ -499,7 +500,7 @@ __global__ void __launch_bounds__(128) attend_dec_merge_kernel(DecParams p) {
     float4 s4 = sm_o[0][lane];
     float ls = sm_l[0];
 #pragma unroll
-    for (int w = 1; w < 4; ++w) {
+    for (int w = 1; w < kMergeWarps; ++w) {
       const float4 y = sm_o[w][lane];
       s4.x += y.x; s4.y += y.y; s4.z += y.z; s4.w += y.w;
       ls += sm_l[w];
@@ -556,7 +557,7 @@ cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.max_seg == 1) return e;
   // split queries: merge their partials (one CTA per output row; y carries the grid size)
-  attend_dec_merge_kernel<<<(unsigned)(p.B * p.T * p.h_q), 128, 0, st>>>(p);
+  attend_dec_merge_kernel<<<(unsigned)(p.B * p.T * p.h_q), kMergeWarps * 32, 0, st>>>(p);
   return cudaGetLastError();
 }
 
