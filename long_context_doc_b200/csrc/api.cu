@@ -514,6 +514,9 @@ size_t msa_sparse_attend_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_
     const msa::DecPlan dp = msa::attend_dec_plan(B, T, h_q, h_kv, d, max_ctx, L_loc, sm_count());
     if (dp.ok)
       need = std::max(need, kHeader + dp.ctr_bytes + dp.part_ml_bytes + dp.part_o_bytes);
+    const msa::AtcPlan ap = msa::attend_tc_plan(B, T, h_q, h_kv, d, max_ctx, L_loc);
+    if (ap.ok)
+      need = std::max(need, kHeader + ap.q_bytes + ap.k_bytes + ap.vl_bytes + ap.vc_bytes);
   }
   return need;
 }
@@ -577,6 +580,38 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       // status word and segment tickets start at zero
       cudaError_t e = cudaMemsetAsync(ws, 0, kHeader + dp.ctr_bytes, st);
       if (e == cudaSuccess) e = msa::launch_attend_dec(q, dp, st);
+      if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
+      return ok();
+    }
+    const msa::AtcPlan ap = msa::attend_tc_plan(B, T, h_q, h_kv, d, max_ctx, L_loc);
+    if (ap.ok) {  // long queries: tensor-core attention
+      const size_t need = kHeader + ap.q_bytes + ap.k_bytes + ap.vl_bytes + ap.vc_bytes;
+      REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+              MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes,
+              need);
+      unsigned char* w8 = static_cast<unsigned char*>(ws);
+      msa::AtcParams a{};
+      a.Q = static_cast<const __nv_bfloat16*>(Q);
+      a.Kl = static_cast<const __nv_bfloat16*>(K_loc);
+      a.Vl = static_cast<const __nv_bfloat16*>(V_loc);
+      a.cK = static_cast<const __nv_bfloat16*>(ctxK);
+      a.cV = static_cast<const __nv_bfloat16*>(ctxV);
+      a.ctx_len = ctx_len;
+      a.B = B;
+      a.T = T;
+      a.h_q = h_q;
+      a.h_kv = h_kv;
+      a.L = L_loc;
+      a.max_ctx = max_ctx;
+      a.rope = rope_base > 0.f ? 1 : 0;
+      a.pos0 = pos0;
+      msa::rope_turns(a.rope ? (double)rope_base : 0.0, 128, a.rope_turns);
+      a.scale_log2 = sc * 1.4426950408889634f;
+      a.err = reinterpret_cast<int*>(w8);
+      a.O = static_cast<__nv_bfloat16*>(O);
+      cudaStream_t st = (cudaStream_t)stream;
+      cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);  // status word
+      if (e == cudaSuccess) e = msa::launch_attend_tc(a, ap, w8 + kHeader, sm_count(), st);
       if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
       return ok();
     }

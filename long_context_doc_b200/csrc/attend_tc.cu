@@ -1,0 +1,570 @@
+// attend_tc.cu - sparse attention of MSA for long queries (prefill and Memory Interleaving
+// rounds: at least 64 query rows per KV head) on the 5th-generation tensor cores.
+//
+// Method (the same operation as attend.cu): each query token attends over the compressed K/V
+// of the routed documents (memory rows, used as stored, always visible) followed by the local
+// context (causal: query token t sits at local row L - T + t), one softmax with scale 1/sqrt(d);
+// Q and the local K are rotated at positions pos0 + row, pos0 = k
+//   [news.neo-ai.one article, "グローバル RoPE（アクティブコンテキスト）" and "推論パイプライン";
+//    ruixiangma.github.io blog, "三阶段推理流程" and "Memory Interleaving"].
+//
+// Two kernels:
+//  * A pre-pass makes both tensor-core operands plain K-major tiles: Q and the local K are
+//    rotated once (bf16 out; angles as exact fixed-point turn counts through sincospi) and V
+//    (local and gathered memory rows) is transposed to [query][KV head][d][row], memory rows
+//    beyond ctx_len written as zeros.
+//  * The attention kernel, one CTA per (128 query rows of one KV head, KV head, query): the rows
+//    are 128 / (h_q / h_kv) tokens x the KV head's query heads. Warp 0 loads Q once and the
+//    key tiles (128 rows: K and V^T, two 128-byte-swizzled TMA boxes each, no multicast) into a
+//    2-stage ring; one thread of warp 1 issues tcgen05.mma (bf16 x bf16 -> fp32 in TMEM):
+//    S_j = Q K_j^T into one of two S buffers, issued one tile ahead, and O += P_j V_j into a
+//    TMEM accumulator; warps 2-5 (one query row per thread, its TMEM lane) read S_j, mask,
+//    keep the online softmax (the running maximum is raised only when a tile's maximum exceeds
+//    it by more than 8 in log2 units, and only then is O rescaled in TMEM), write P_j in bf16 to
+//    shared memory in the operand layout, and finally normalise O and store it.
+// Every wait is bounded; on expiry the CTA records kErrWaitTimeout in the workspace status word,
+// stops, lets its copies and MMAs land, frees its TMEM and writes nothing.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace msa {
+namespace atc {
+
+constexpr int kM = 128;         // query rows per tile (TMEM lanes)
+constexpr int kN = 128;         // key rows per tile
+constexpr int kD = 128;         // head dim
+constexpr int kThreads = 192;   // warp 0 copies, warp 1 MMA, warps 2-5 softmax
+constexpr uint32_t kSlice = 128 * 128;           // one 128-row x 64-element bf16 slice: 16 KB
+constexpr uint32_t kQBytes = 2 * kSlice;         // Q tile (two 64-wide K slices)
+constexpr uint32_t kKBytes = 2 * kSlice;         // K tile
+constexpr uint32_t kVBytes = 2 * kSlice;         // V^T tile (two 64-key slices)
+constexpr uint32_t kStage = kKBytes + kVBytes;   // 64 KB
+constexpr int kStages = 2;
+constexpr float kRaise = 8.f;  // log2 headroom before the running maximum is raised
+
+__device__ __forceinline__ void tma3(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                     uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma2(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// K-major operand slice [rows][64 bf16], 128-byte swizzle: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc128(const void* slice) {
+  const uint64_t a = (uint64_t)(smem_u32(slice) & 0x3FFFFu) >> 4;
+  return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+__device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t par, int* err,
+                                              volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_wait_bounded(bar, par, err)) return true;
+  *abort_flag = 1;
+  return false;
+}
+
+// ------------------------------------------------------------------------------ pre-pass
+// Rotated bf16 copies of rows [n_rows, 128]: row r sits at position base + (r / div) % mod.
+// One warp per row; lane l takes the RoPE pairs l and l + 32 (dims l, l+64, l+32, l+96).
+__global__ void __launch_bounds__(256) rope_rows_kernel(const __nv_bfloat16* __restrict__ src,
+                                                        __nv_bfloat16* __restrict__ dst,
+                                                        int64_t n_rows, int64_t div, int64_t mod,
+                                                        int64_t base, AtcParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const unsigned long long F0 = p.rope_turns[lane], F1 = p.rope_turns[lane + 32];
+  for (int64_t r = warp; r < n_rows; r += nw) {
+    const int64_t pos = base + (r / div) % mod;
+    const __nv_bfloat16* s = src + r * kD;
+    __nv_bfloat16* d = dst + r * kD;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = lane + 32 * h;
+      const float a = __bfloat162float(s[i]), c = __bfloat162float(s[i + 64]);
+      const float2 cs = p.rope ? rot_turns(pos, h ? F1 : F0) : make_float2(1.f, 0.f);
+      d[i] = __float2bfloat16_rn(a * cs.x - c * cs.y);
+      d[i + 64] = __float2bfloat16_rn(c * cs.x + a * cs.y);
+    }
+  }
+}
+
+// V [B, R, h_kv, 128] -> V^T [B, h_kv, 128, Rp]: rows >= valid(b) written as zeros. CTA per
+// (64-row block, KV head, query): the block goes through shared memory.
+__global__ void __launch_bounds__(256) transpose_v_kernel(const __nv_bfloat16* __restrict__ V,
+                                                          __nv_bfloat16* __restrict__ Vt, int R,
+                                                          int Rp, int h_kv,
+                                                          const int32_t* __restrict__ valid_len,
+                                                          int valid_cap) {
+  __shared__ __nv_bfloat16 tile[64][kD + 8];
+  const int r0 = blockIdx.x * 64, g = blockIdx.y, b = blockIdx.z;
+  const int valid = valid_len ? min(max(valid_len[b], 0), valid_cap) : R;
+  for (int idx = threadIdx.x; idx < 64 * (kD / 8); idx += blockDim.x) {
+    const int rr = idx / (kD / 8), c8 = (idx % (kD / 8)) * 8;
+    const int row = r0 + rr;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (row < R && row < valid)
+      v = *reinterpret_cast<const uint4*>(V + (((int64_t)b * R + row) * h_kv + g) * kD + c8);
+    *reinterpret_cast<uint4*>(&tile[rr][c8]) = v;
+  }
+  __syncthreads();
+  // out row = dim, 64 consecutive keys: 8 threads per dim write 8 keys each (16 bytes)
+  for (int idx = threadIdx.x; idx < kD * 8; idx += blockDim.x) {
+    const int dim = idx / 8, k8 = (idx % 8) * 8;
+    if (r0 + k8 >= R) continue;
+    __align__(16) __nv_bfloat16 w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) w[q] = tile[k8 + q][dim];
+    __nv_bfloat16* out = Vt + (((int64_t)b * h_kv + g) * kD + dim) * Rp + r0 + k8;
+    if (r0 + k8 + 8 <= Rp) *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(w);
+  }
+}
+
+// ------------------------------------------------------------------------------ attention
+__global__ void __launch_bounds__(kThreads, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kc,
+                 const __grid_constant__ CUtensorMap map_kl, const __grid_constant__ CUtensorMap map_vc,
+                 const __grid_constant__ CUtensorMap map_vl, AtcParams p) {
+  extern __shared__ __align__(1024) unsigned char sm_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* q_s = base;                                  // [2][128][64]
+  unsigned char* stages = base + kQBytes;                     // [S][K 2 slices | V^T 2 slices]
+  unsigned char* p_s = stages + kStages * kStage;             // [2][128][64] probabilities
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * kSlice);
+  uint64_t* qfull = bars;                    // Q landed
+  uint64_t* kfull = bars + 1;                // [2] stage landed
+  uint64_t* kempty = bars + 3;               // [2] stage consumed (P.V done)
+  uint64_t* sfull = bars + 5;                // [2] S buffer written
+  uint64_t* sfree = bars + 7;                // [2] S buffer read (128 threads)
+  uint64_t* pfull = bars + 9;                // P written (128 threads)
+  uint64_t* ofull = bars + 10;               // P.V of the tile completed
+  uint64_t* done = bars + 11;                // every issued MMA completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int Gq = p.h_q / p.h_kv;
+  const int TQ = kM / Gq;                         // tokens per query tile
+  const int t0 = qt * TQ;
+  const int t_last = min(t0 + TQ - 1, p.T - 1);
+  const int n_ctx = min(max(p.ctx_len[b], 0), p.max_ctx);
+  const int CT = (n_ctx + kN - 1) / kN;           // memory tiles
+  const int jmax = p.L - p.T + t_last;            // last local row the tile's rows can see
+  const int LT = jmax / kN + 1;                   // local tiles
+  const int n_tiles = CT + LT;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qfull, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sfree[s], 128);
+    }
+    mbar_init(pfull, 128);
+    mbar_init(ofull, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {  // S0 at column 0, S1 at 128, O at 256
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      mbar_arrive_expect_tx(qfull, kQBytes);
+      tma3(q_s, &map_q, 0, g * Gq, b * p.T + t0, qfull);
+      tma3(q_s + kSlice, &map_q, 64, g * Gq, b * p.T + t0, qfull);
+      const int vrow = (b * p.h_kv + g) * kD;  // first V^T row of this (query, KV head)
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !wait_or_abort(&kempty[s], (uint32_t)(((j >> 1) - 1) & 1), p.err, abort_flag))
+          break;
+        unsigned char* st = stages + s * kStage;
+        mbar_arrive_expect_tx(&kfull[s], kStage);
+        if (j < CT) {
+          const int m0 = j * kN;
+          tma3(st, &map_kc, 0, g, b * p.max_ctx + m0, &kfull[s]);
+          tma3(st + kSlice, &map_kc, 64, g, b * p.max_ctx + m0, &kfull[s]);
+          tma2(st + kKBytes, &map_vc, m0, vrow, &kfull[s]);
+          tma2(st + kKBytes + kSlice, &map_vc, m0 + 64, vrow, &kfull[s]);
+        } else {
+          const int j0 = (j - CT) * kN;
+          tma3(st, &map_kl, 0, g, b * p.L + j0, &kfull[s]);
+          tma3(st + kSlice, &map_kl, 64, g, b * p.L + j0, &kfull[s]);
+          tma2(st + kKBytes, &map_vl, j0, vrow, &kfull[s]);
+          tma2(st + kKBytes + kSlice, &map_vl, j0 + 64, vrow, &kfull[s]);
+        }
+        ++issued;
+      }
+      // the copies issued land before the CTA can exit
+      mbar_wait_bounded(qfull, 0, p.err);
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait_bounded(&kfull[j & 1], (uint32_t)((j >> 1) & 1), p.err);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
+                             ((uint32_t)(kM >> 4) << 24);
+      const uint64_t qd0 = desc128(q_s), qd1 = desc128(q_s + kSlice);
+      const uint64_t pd0 = desc128(p_s), pd1 = desc128(p_s + kSlice);
+      auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T into buffer j & 1
+        const int s = j & 1;
+        if (!wait_or_abort(&kfull[s], (uint32_t)((j >> 1) & 1), p.err, abort_flag)) return false;
+        if (j >= 2 && !wait_or_abort(&sfree[s], (uint32_t)(((j >> 1) - 1) & 1), p.err, abort_flag))
+          return false;
+        fence_after();
+        const unsigned char* st = stages + s * kStage;
+        const uint64_t kd0 = desc128(st), kd1 = desc128(st + kSlice);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // K = 16 per instruction: +32 bytes within a slice
+          const uint64_t a = (kk < 4 ? qd0 : qd1) + 2 * (kk & 3);
+          const uint64_t bb = (kk < 4 ? kd0 : kd1) + 2 * (kk & 3);
+          mma(tmem + (uint32_t)(s * kN), a, bb, idesc, kk ? 1u : 0u);
+        }
+        commit(&sfull[s]);
+        return true;
+      };
+      bool ok = wait_or_abort(qfull, 0, p.err, abort_flag) && (n_tiles == 0 || issue_s(0));
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+        if (!wait_or_abort(pfull, (uint32_t)(j & 1), p.err, abort_flag)) break;
+        fence_after();
+        const unsigned char* st = stages + (j & 1) * kStage;
+        const uint64_t vd0 = desc128(st + kKBytes), vd1 = desc128(st + kKBytes + kSlice);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // O += P_j V_j over the tile's 128 keys
+          const uint64_t a = (kk < 4 ? pd0 : pd1) + 2 * (kk & 3);
+          const uint64_t bb = (kk < 4 ? vd0 : vd1) + 2 * (kk & 3);
+          mma(tmem + 2u * kN, a, bb, idesc, (j | kk) ? 1u : 0u);
+        }
+        commit(ofull);
+        commit(&kempty[j & 1]);
+      }
+      commit(done);
+      mbar_wait_bounded(done, 0, p.err);
+    }
+  } else {
+    // ---------------- softmax: thread = query row (its TMEM lane)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int tok = t0 + row / Gq;              // query token of this row
+    const int hq = g * Gq + row % Gq;           // query head
+    const bool row_ok = tok < p.T;
+    const int vis = p.L - p.T + min(tok, p.T - 1);  // last visible local row
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float c = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool aborted = false;
+    // tcgen05.ld/st are warp-collective: every decision around them is taken warp-uniformly
+    for (int j = 0; j < n_tiles; ++j) {
+      const int sb = j & 1;
+      if (!__all_sync(0xffffffffu, wait_or_abort(&sfull[sb], (uint32_t)((j >> 1) & 1), p.err, abort_flag))) {
+        aborted = true;
+        break;
+      }
+      fence_after();
+      const bool is_ctx = j < CT;
+      const int k0 = is_ctx ? j * kN : (j - CT) * kN;
+      const int lim = is_ctx ? n_ctx - 1 - k0 : vis - k0;  // keys [0, lim] of the tile visible
+      const uint32_t sa = lane_base + (uint32_t)(sb * kN);
+      // pass 1: the tile's maximum
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        ld32(sa + ch * 32, r);
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (ch * 32 + q <= lim) mx = fmaxf(mx, __uint_as_float(r[q]) * c);
+      }
+      // the running maximum moves only by more than kRaise (then O is rescaled)
+      float alpha = 1.f;
+      const bool raise = mx > m + kRaise || m == -INFINITY;
+      const float m_new = raise ? mx : m;
+      if (raise && m != -INFINITY) alpha = exp2f(m - m_new);
+      // P_{j-1} . V_{j-1} must be done before P is rewritten and before O is rescaled
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, wait_or_abort(ofull, (uint32_t)((j - 1) & 1), p.err, abort_flag))) {
+          aborted = true;
+          break;
+        }
+        fence_after();
+        if (__any_sync(0xffffffffu, raise && m != -INFINITY)) {  // lanes not raising scale by 1
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t r[32];
+            ld32(lane_base + 2u * kN + ch * 32, r);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
+            st32(lane_base + 2u * kN + ch * 32, r);
+          }
+        }
+      }
+      m = (m_new == -INFINITY) ? m : m_new;
+      l *= alpha;
+      // pass 2: probabilities in bf16 into the operand layout (row-major 64-key slices,
+      // 16-byte chunk index XOR row % 8)
+      float sum = 0.f;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        ld32(sa + ch * 32, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int k = ch * 32 + 2 * q;
+          const float p0 = (k <= lim && m != -INFINITY) ? exp2f(__uint_as_float(r[2 * q]) * c - m) : 0.f;
+          const float p1 = (k + 1 <= lim && m != -INFINITY) ? exp2f(__uint_as_float(r[2 * q + 1]) * c - m) : 0.f;
+          sum += p0 + p1;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        unsigned char* slice = p_s + (ch >> 1) * kSlice + row * 128;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {  // 4 chunks of 16 bytes (8 keys) of this 32-key group
+          const int chunk = (ch & 1) * 4 + q4;
+          *reinterpret_cast<uint4*>(slice + ((chunk ^ (row & 7)) << 4)) =
+              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        }
+      }
+      l += sum;
+      fence_before();
+      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      mbar_arrive(&sfree[sb]);
+      mbar_arrive(pfull);
+    }
+    // epilogue: O / l of the last tile's accumulator
+    const bool fin = !aborted && n_tiles > 0 &&
+                     wait_or_abort(ofull, (uint32_t)((n_tiles - 1) & 1), p.err, abort_flag);
+    if (__all_sync(0xffffffffu, fin)) {
+      fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* out = p.O + (((int64_t)b * p.T + tok) * p.h_q + hq) * kD;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        ld32(lane_base + 2u * kN + ch * 32, r);
+        if (row_ok && !*abort_flag) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(
+                  __uint_as_float(r[8 * q8 + 2 * q]) * inv, __uint_as_float(r[8 * q8 + 2 * q + 1]) * inv);
+              w[q] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(out + ch * 32 + q8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown: every MMA completed (the issuer waited on `done`)
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+}
+
+}  // namespace atc
+
+// ------------------------------------------------------------------------------ host side
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn_atc() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+// bf16 map with the 128-byte swizzle (box rows of 64 elements), zero fill out of bounds
+bool encode_bf16_map_sw128(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn_atc();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = (cuuint64_t)dims[i];
+    bx[i] = (cuuint32_t)box[i];
+    es[i] = 1;
+    if (i + 1 < rank) st[i] = (cuuint64_t)strides[i];
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, st,
+            bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L) {
+  AtcPlan pl{};
+  const int Gq = h_kv > 0 ? h_q / h_kv : 0;
+  pl.ok = d == atc::kD && B >= 1 && T >= 1 && L >= T && Gq >= 1 && atc::kM % Gq == 0 &&
+          Gq * T >= 64;
+  if (!pl.ok) return pl;
+  pl.n_qtiles = (Gq * T + atc::kM - 1) / atc::kM;
+  pl.Lp = (L + 7) / 8 * 8;
+  pl.Mp = (max_ctx + 7) / 8 * 8;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  pl.q_bytes = al((size_t)B * T * h_q * atc::kD * 2);
+  pl.k_bytes = al((size_t)B * L * h_kv * atc::kD * 2);
+  pl.vl_bytes = al((size_t)B * h_kv * atc::kD * pl.Lp * 2);
+  pl.vc_bytes = max_ctx > 0 ? al((size_t)B * h_kv * atc::kD * pl.Mp * 2) : 0;
+  pl.smem = 1024 + atc::kQBytes + atc::kStages * atc::kStage + 2 * atc::kSlice + 16 * 8 + 16;
+  return pl;
+}
+
+cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned char* scratch,
+                             int sms, cudaStream_t st) {
+  AtcParams p = p0;
+  __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(scratch);
+  __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes);
+  __nv_bfloat16* vt_l = reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes + pl.k_bytes);
+  __nv_bfloat16* vt_c =
+      reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes + pl.k_bytes + pl.vl_bytes);
+  const int Gq = p.h_q / p.h_kv;
+  // pre-pass: rotated Q and local K, transposed V
+  {
+    const int64_t qrows = (int64_t)p.B * p.T * p.h_q, krows = (int64_t)p.B * p.L * p.h_kv;
+    const int64_t grid_q = std::min<int64_t>((qrows + 7) / 8, (int64_t)sms * 16);
+    const int64_t grid_k = std::min<int64_t>((krows + 7) / 8, (int64_t)sms * 16);
+    atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_q, 1), 256, 0, st>>>(
+        p.Q, q_rot, qrows, p.h_q, p.T, (int64_t)p.pos0 + p.L - p.T, p);
+    atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_k, 1), 256, 0, st>>>(
+        p.Kl, k_rot, krows, p.h_kv, p.L, (int64_t)p.pos0, p);
+    atc::transpose_v_kernel<<<dim3((unsigned)((p.L + 63) / 64), (unsigned)p.h_kv, (unsigned)p.B),
+                              256, 0, st>>>(p.Vl, vt_l, p.L, pl.Lp, p.h_kv, nullptr, p.L);
+    if (p.max_ctx > 0)
+      atc::transpose_v_kernel<<<dim3((unsigned)((p.max_ctx + 63) / 64), (unsigned)p.h_kv,
+                                     (unsigned)p.B),
+                                256, 0, st>>>(p.cV, vt_c, p.max_ctx, pl.Mp, p.h_kv, p.ctx_len,
+                                              p.max_ctx);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // tensor maps (bf16, 128-byte swizzle, zero fill out of bounds)
+  CUtensorMap mq, mkc, mkl, mvc, mvl;
+  const uint64_t row = atc::kD * 2;
+  {
+    const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_q, (uint64_t)p.B * p.T};
+    const uint64_t str[2] = {row, row * p.h_q};
+    const uint32_t box[3] = {64, (uint32_t)Gq, (uint32_t)(atc::kM / Gq)};
+    if (!encode_bf16_map_sw128(&mq, q_rot, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.L};
+    const uint64_t str[2] = {row, row * p.h_kv};
+    const uint32_t box[3] = {64, 1, atc::kN};
+    if (!encode_bf16_map_sw128(&mkl, k_rot, 3, dims, str, box)) return cudaErrorInvalidValue;
+    const uint64_t dv[2] = {(uint64_t)p.L, (uint64_t)p.B * p.h_kv * atc::kD};
+    const uint64_t sv[1] = {(uint64_t)pl.Lp * 2};
+    const uint32_t bv[2] = {64, atc::kD};
+    if (!encode_bf16_map_sw128(&mvl, vt_l, 2, dv, sv, bv)) return cudaErrorInvalidValue;
+  }
+  if (p.max_ctx > 0) {
+    const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.max_ctx};
+    const uint64_t str[2] = {row, row * p.h_kv};
+    const uint32_t box[3] = {64, 1, atc::kN};
+    if (!encode_bf16_map_sw128(&mkc, p.cK, 3, dims, str, box)) return cudaErrorInvalidValue;
+    const uint64_t dv[2] = {(uint64_t)p.max_ctx, (uint64_t)p.B * p.h_kv * atc::kD};
+    const uint64_t sv[1] = {(uint64_t)pl.Mp * 2};
+    const uint32_t bv[2] = {64, atc::kD};
+    if (!encode_bf16_map_sw128(&mvc, vt_c, 2, dv, sv, bv)) return cudaErrorInvalidValue;
+  } else {  // no memory tiles: never read
+    mkc = mkl;
+    mvc = mvl;
+  }
+  cudaError_t e = cudaFuncSetAttribute(atc::attend_tc_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+  if (e != cudaSuccess) return e;
+  atc::attend_tc_kernel<<<dim3((unsigned)pl.n_qtiles, (unsigned)p.h_kv, (unsigned)p.B),
+                          atc::kThreads, pl.smem, st>>>(mq, mkc, mkl, mvc, mvl, p);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

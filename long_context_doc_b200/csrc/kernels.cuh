@@ -167,4 +167,29 @@ struct DecPlan {
 DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
 
+// ---- attend_tc.cu: long-query attention on tensor cores (bf16, d = 128, (h_q/h_kv) * T >= 64,
+// h_q/h_kv dividing 128)
+struct AtcParams {
+  const __nv_bfloat16* Q;   // [B, T, h_q, 128]
+  const __nv_bfloat16* Kl;  // [B, L, h_kv, 128] (before RoPE)
+  const __nv_bfloat16* Vl;
+  const __nv_bfloat16* cK;  // [B, max_ctx, h_kv, 128]
+  const __nv_bfloat16* cV;
+  const int32_t* ctx_len;
+  int B, T, h_q, h_kv, L, max_ctx;
+  int rope, pos0;
+  unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions
+  float scale_log2;
+  int* err;                 // workspace status word
+  __nv_bfloat16* O;         // [B, T, h_q, 128]
+};
+struct AtcPlan {
+  bool ok;
+  int n_qtiles, Lp, Mp;     // query tiles per (query, KV head); padded row counts of V^T
+  size_t q_bytes, k_bytes, vl_bytes, vc_bytes, smem;  // scratch: rotated Q, rotated K, V^T
+};
+AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L);
+cudaError_t launch_attend_tc(const AtcParams& p, const AtcPlan& pl, unsigned char* scratch,
+                             int sms, cudaStream_t st);
+
 }  // namespace msa
