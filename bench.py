@@ -14,7 +14,11 @@ layer's scan), sparse attention (msa_sparse_attend). Queries/s = B / step time.
 ``--workload bank10m`` runs the 10M-token single-layer decode (20,000 docs, B = 8, device
 bank) instead. ``--workload prefill1m`` times the 1M-token prefill path (1,024 docs x 1,024
 tokens: doc-wise RoPE + chunk pooling of K, V, K_r, bank preparation, tensor-core routing of a
-128-token query, gather, attention) phase by phase; its line reports bank tokens/s. ``--impl reference`` times the CPU oracle on the host cores (a bounded
+128-token query, gather, attention) phase by phase; its line reports bank tokens/s.
+``--workload interleave10m`` runs Memory Interleaving at its full configuration (18 routed
+layers, each over its own 10M-token bank; B = 32 queries of T = 256 tokens, k = 8, 3 rounds:
+each round re-routes with the appended documents excluded and attends over their raw K/V
+placed before the query tokens); its line reports queries/s of the whole interleave. ``--impl reference`` times the CPU oracle on the host cores (a bounded
 sample of the same workload). Under torchrun every rank runs an independent replica
 (the path does not shard: no collective on the data path).
 """
@@ -45,7 +49,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
-    ap.add_argument("--workload", default="bank100m", choices=["bank100m", "bank10m", "prefill1m"])
+    ap.add_argument("--workload", default="bank100m",
+                    choices=["bank100m", "bank10m", "prefill1m", "interleave10m"])
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
                     help="host-bank fetch: device gather over the host link on a side stream "
                          "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
@@ -644,12 +649,196 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+def run_interleave(args):
+    """Memory Interleaving at full size, each phase timed with CUDA events on its stream."""
+    import torch
+    import torch.distributed as dist
+
+    import long_context_doc_b200 as msa
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=dev)
+    w = synth.C5.scaled(seed=synth.C5.seed + 1000 * rank)
+    B, T, k, R, NL = w.B, w.T, w.k, w.rounds, w.layers
+    bf = torch.bfloat16
+    lay = []
+    for l in range(NL):
+        d = synth.dev_bank_workload(w, dev, layer=l, with_kv=True)
+        d["inv"] = msa.kr_inv_norm(d["Kbar_r"])
+        d["hat"] = msa.kr_normalize(d["Kbar_r"])
+        lay.append(d)
+    coff_host = lay[0]["doc_chunk_off"]
+    coff = torch.from_numpy(coff_host).to(dev)
+    n_chunks, n_docs = int(coff_host[-1]), w.n_docs
+    max_ctx = k * int(np.max(np.diff(coff_host)))
+    words = (n_docs + 31) // 32
+    # raw per-token K/V of appended documents: a per-layer pool of P synthetic documents
+    # (document d uses pool entry d mod P; the content does not change the cost)
+    P = 16
+    pools = []
+    for l in range(NL):
+        kp = torch.empty((P, w.doc_len, w.h_kv, w.d), dtype=bf, device=dev)
+        vp = torch.empty_like(kp)
+        synth.dev_normal(kp, w.seed, synth.tag(synth.APPK, l))
+        synth.dev_normal(vp, w.seed, synth.tag(synth.APPV, l))
+        pools.append((kp, vp))
+    Ls = [T + r * k * w.doc_len for r in range(R)]
+    kloc = [torch.empty((B, Lr, w.h_kv, w.d), dtype=bf, device=dev) for Lr in Ls]
+    vloc = [torch.empty_like(t) for t in kloc]
+    ws_r = torch.empty(msa.msa_route_topk_workspace(B, T, w.h_qr, w.h_kv, w.d, 1, n_docs,
+                                                    n_chunks, k), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(max(msa.msa_sparse_attend_workspace(B, T, w.h_q, w.h_kv, w.d, max_ctx, Lr)
+                           for Lr in Ls), dtype=torch.uint8, device=dev)
+    ids = torch.empty((B, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, k), dtype=torch.float32, device=dev)
+    gi = torch.empty((B, max_ctx), dtype=torch.int32, device=dev)
+    cl = torch.empty(B, dtype=torch.int32, device=dev)
+    cK = torch.empty((B, max_ctx, w.h_kv, w.d), dtype=bf, device=dev)
+    cV = torch.empty_like(cK)
+    ws_g = torch.zeros(256, dtype=torch.uint8, device=dev)
+    O = torch.empty((B, T, w.h_q, w.d), dtype=bf, device=dev)
+    appended = torch.zeros((B, R * k), dtype=torch.int64, device=dev)
+    excl = torch.zeros((B, words), dtype=torch.int64, device=dev)
+    ex32 = torch.zeros((B, words), dtype=torch.int32, device=dev)
+    st = torch.cuda.Stream()
+    names = ["route", "gather", "assemble", "attend"]
+    nev = R * NL
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nev)]
+    rows_b = torch.arange(B, device=dev).unsqueeze(1)
+
+    def interleave(rec):
+        with torch.cuda.stream(st):
+            excl.zero_()
+            for r in range(R):
+                A = r * k * w.doc_len
+                for l in range(NL):
+                    ev = evs[r * NL + l]
+                    d = lay[l]
+                    if rec:
+                        ev[0].record(st)
+                    msa.msa_route_topk(d["Q_r"], d["Kbar_r"], d["inv"], coff, k,
+                                       ex32 if r > 0 else None, ids, sc, None, ws_r, st,
+                                       d["hat"])
+                    if rec:
+                        ev[1].record(st)
+                    msa.msa_gather(ids, coff, d["Kbar"], d["Vbar"], max_ctx, gi, cl, cK, cV,
+                                   ws_g, st)
+                    if rec:
+                        ev[2].record(st)
+                    if r > 0:  # [appended documents (round order, ascending id) ; query tokens]
+                        sel = (appended[:, :r * k] % P).reshape(-1)
+                        kloc[r][:, :A] = pools[l][0].index_select(0, sel).view(B, A, w.h_kv, w.d)
+                        vloc[r][:, :A] = pools[l][1].index_select(0, sel).view(B, A, w.h_kv, w.d)
+                    kloc[r][:, A:] = d["K_loc"]
+                    vloc[r][:, A:] = d["V_loc"]
+                    if rec:
+                        ev[3].record(st)
+                    msa.msa_sparse_attend(d["Q"], kloc[r], vloc[r], cK, cV, cl, k, w.rope_base,
+                                          0.0, O, ws_a, st)
+                    if rec:
+                        ev[4].record(st)
+                # the last routed layer's documents are appended and excluded from now on
+                new = torch.sort(ids.to(torch.int64), dim=1).values
+                appended[:, r * k:(r + 1) * k] = new
+                excl.scatter_add_(1, new // 32, torch.ones_like(new) << (new % 32))
+                ex32.copy_(excl.to(torch.int32))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        interleave(False)
+    barrier()
+    Kst = max(1, min(args.steps, 3))
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    phase = {n: 0.0 for n in names}
+    per_round_attend = [0.0] * R
+    per_round_route = [0.0] * R
+    t0.record(st)
+    for _ in range(Kst):
+        interleave(True)
+        st.synchronize()
+        for r in range(R):
+            for l in range(NL):
+                ev = evs[r * NL + l]
+                for i, n in enumerate(names):
+                    phase[n] += ev[i].elapsed_time(ev[i + 1]) / Kst
+                per_round_attend[r] += ev[3].elapsed_time(ev[4]) / Kst
+                per_round_route[r] += ev[0].elapsed_time(ev[1]) / Kst
+    t1.record(st)
+    barrier()
+    clocks = sampler.stop()
+    step_ms = t0.elapsed_time(t1) / Kst
+    if world > 1:
+        tt = torch.tensor([step_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        step_ms = float(tt[0])
+    route_flop = 2.0 * B * T * n_chunks * w.h_kv * w.d  # per routing call
+    route_call_ms = phase["route"] / (R * NL)
+    route_tf = route_flop / (route_call_ms / 1e3) / 1e12
+    # attention: QK^T and PV over the visible keys (memory rows + causal local rows)
+    att_flop = 0.0
+    for r in range(R):
+        vis = max_ctx + Ls[r] - T + (T + 1) / 2.0
+        att_flop += NL * 4.0 * B * T * w.h_q * vis * w.d
+    att_tf = att_flop / (phase["attend"] / 1e3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        tpeak, tkind = float(pk["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        tpeak, tkind = 1410.0, "fallback (sustained)"
+    line = {
+        "metric": "MSA Memory Interleaving queries/s (18 routed layers x 3 rounds, 10M-token "
+                  "bank per layer)",
+        "value": round(world * B / (step_ms / 1e3), 3), "unit": "queries/s", "n_gpus": world,
+        "steps": Kst, "warmup": max(1, min(args.warmup, 2)), "ms_per_step": round(step_ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 normals; appended documents from a per-layer pool)",
+        "config": {"workload": w.name, "bank_tokens_per_layer": n_docs * w.doc_len,
+                   "n_chunks": n_chunks, "routed_layers": NL, "rounds": R, "batch": B, "T": T,
+                   "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d, "k": k, "local_kv_per_round": Ls,
+                   "l2": "no flush: every layer reads its own 328 MB bank and 0.3-1 GB of K/V",
+                   "parallelism": f"replicas x{world}"},
+        "phases_ms": {n: round(v, 3) for n, v in phase.items()},
+        "route_ms_per_round": [round(x, 3) for x in per_round_route],
+        "attend_ms_per_round": [round(x, 3) for x in per_round_attend],
+        "roofline": {"kernel": "msa_route_topk (tcgen05 scan, 8,192 query rows per call)",
+                     "bound": "tensor", "achieved": round(route_tf, 1), "peak": tpeak,
+                     "unit": "TFLOP/s", "frac": round(route_tf / tpeak, 4), "peak_kind": tkind,
+                     "traffic": None, "flop_per_launch": route_flop,
+                     "avg_launch_ms": round(route_call_ms, 4)},
+        "attend_tflops": round(att_tf, 1),
+        "gpu_launches": Kst * R * NL * 8,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
     elif args.workload == "prefill1m":
         run_prefill(args)
+    elif args.workload == "interleave10m":
+        run_interleave(args)
     else:
         run_libmsa(args)
 
