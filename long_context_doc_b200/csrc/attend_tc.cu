@@ -18,10 +18,12 @@
 //    key tiles (128 rows: K and V^T, two 128-byte-swizzled TMA boxes each, no multicast) into a
 //    2-stage ring; one thread of warp 1 issues tcgen05.mma (bf16 x bf16 -> fp32 in TMEM):
 //    S_j = Q K_j^T into one of two S buffers, issued one tile ahead, and O += P_j V_j into a
-//    TMEM accumulator; warps 2-5 (one query row per thread, its TMEM lane) read S_j, mask,
-//    keep the online softmax (the running maximum is raised only when a tile's maximum exceeds
-//    it by more than 8 in log2 units, and only then is O rescaled in TMEM), write P_j in bf16 to
-//    shared memory in the operand layout, and finally normalise O and store it.
+//    TMEM accumulator; warps 2-9 (two per TMEM lane quarter: thread = one query row x one half
+//    of the keys and of the output dims) read S_j, mask, keep the online softmax (the halves
+//    exchange the tile's row maximum through shared memory; the running maximum is raised only
+//    when a tile's maximum exceeds it by more than 8 in log2 units, and only then is O rescaled
+//    in TMEM), write P_j in bf16 to shared memory in the operand layout, and finally normalise
+//    O and store it.
 // Every wait is bounded; on expiry the CTA records kErrWaitTimeout in the workspace status word,
 // stops, lets its copies and MMAs land, frees its TMEM and writes nothing.
 #include <cuda.h>
@@ -37,7 +39,7 @@ namespace atc {
 constexpr int kM = 128;         // query rows per tile (TMEM lanes)
 constexpr int kN = 128;         // key rows per tile
 constexpr int kD = 128;         // head dim
-constexpr int kThreads = 192;   // warp 0 copies, warp 1 MMA, warps 2-5 softmax
+constexpr int kThreads = 320;   // warp 0 copies, warp 1 MMA, warps 2-9 softmax
 constexpr uint32_t kSlice = 128 * 128;           // one 128-row x 64-element bf16 slice: 16 KB
 constexpr uint32_t kQBytes = 2 * kSlice;         // Q tile (two 64-wide K slices)
 constexpr uint32_t kKBytes = 2 * kSlice;         // K tile
@@ -112,12 +114,32 @@ __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Barrier of the 256 softmax threads (id 2), returning whether every one of them passed true.
+__device__ __forceinline__ bool named_sync_softmax_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 2, 256, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t par, int* err,
                                               volatile int* abort_flag) {
   if (*abort_flag) return false;
   if (mbar_wait_bounded(bar, par, err)) return true;
   *abort_flag = 1;
   return false;
+}
+
+// 2^x by the hardware approximation (max relative error 2^-22; the probabilities are stored
+// in bf16)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------------------ pre-pass
@@ -188,16 +210,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   unsigned char* q_s = base;                                  // [2][128][64]
   unsigned char* stages = base + kQBytes;                     // [S][K 2 slices | V^T 2 slices]
   unsigned char* p_s = stages + kStages * kStage;             // [2][128][64] probabilities
-  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + 2 * kSlice);
+  float* xmax = reinterpret_cast<float*>(p_s + 2 * kSlice);  // [2 tiles][2 halves][128 rows]
+  float* xsum = xmax + 512;                                  // [2 halves][128 rows]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xsum + 256);
   uint64_t* qfull = bars;                    // Q landed
-  uint64_t* kfull = bars + 1;                // [2] stage landed
-  uint64_t* kempty = bars + 3;               // [2] stage consumed (P.V done)
+  uint64_t* kfull = bars + 1;                // [2] K half of the stage landed
+  uint64_t* kempty = bars + 3;               // [2] K half consumed (S = Q K^T done)
   uint64_t* sfull = bars + 5;                // [2] S buffer written
-  uint64_t* sfree = bars + 7;                // [2] S buffer read (128 threads)
-  uint64_t* pfull = bars + 9;                // P written (128 threads)
+  uint64_t* sfree = bars + 7;                // [2] S buffer read (256 threads)
+  uint64_t* pfull = bars + 9;                // P written (256 threads)
   uint64_t* ofull = bars + 10;               // P.V of the tile completed
   uint64_t* done = bars + 11;                // every issued MMA completed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* vfull = bars + 12;               // [2] V^T half of the stage landed
+  uint64_t* vempty = bars + 14;              // [2] V^T half consumed (P.V done)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,10 +243,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int s = 0; s < 2; ++s) {
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
+      mbar_init(&vfull[s], 1);
+      mbar_init(&vempty[s], 1);
       mbar_init(&sfull[s], 1);
-      mbar_init(&sfree[s], 128);
+      mbar_init(&sfree[s], 256);
     }
-    mbar_init(pfull, 128);
+    mbar_init(pfull, 256);
     mbar_init(ofull, 1);
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -246,31 +274,35 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tma3(q_s, &map_q, 0, g * Gq, b * p.T + t0, qfull);
       tma3(q_s + kSlice, &map_q, 64, g * Gq, b * p.T + t0, qfull);
       const int vrow = (b * p.h_kv + g) * kD;  // first V^T row of this (query, KV head)
+      // K of tile j may load once S_{j-2} is done, V^T once P_{j-2} V_{j-2} is done
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
-        if (j >= 2 && !wait_or_abort(&kempty[s], (uint32_t)(((j >> 1) - 1) & 1), p.err, abort_flag))
-          break;
+        const uint32_t par = (uint32_t)(((j >> 1) - 1) & 1);
         unsigned char* st = stages + s * kStage;
-        mbar_arrive_expect_tx(&kfull[s], kStage);
-        if (j < CT) {
-          const int m0 = j * kN;
-          tma3(st, &map_kc, 0, g, b * p.max_ctx + m0, &kfull[s]);
-          tma3(st + kSlice, &map_kc, 64, g, b * p.max_ctx + m0, &kfull[s]);
-          tma2(st + kKBytes, &map_vc, m0, vrow, &kfull[s]);
-          tma2(st + kKBytes + kSlice, &map_vc, m0 + 64, vrow, &kfull[s]);
-        } else {
-          const int j0 = (j - CT) * kN;
-          tma3(st, &map_kl, 0, g, b * p.L + j0, &kfull[s]);
-          tma3(st + kSlice, &map_kl, 64, g, b * p.L + j0, &kfull[s]);
-          tma2(st + kKBytes, &map_vl, j0, vrow, &kfull[s]);
-          tma2(st + kKBytes + kSlice, &map_vl, j0 + 64, vrow, &kfull[s]);
+        const bool ctx = j < CT;
+        const int r0 = ctx ? j * kN : (j - CT) * kN;
+        const CUtensorMap* mk = ctx ? &map_kc : &map_kl;
+        const CUtensorMap* mv = ctx ? &map_vc : &map_vl;
+        const int krow = ctx ? b * p.max_ctx + r0 : b * p.L + r0;
+        if (j >= 2 && !wait_or_abort(&kempty[s], par, p.err, abort_flag)) break;
+        mbar_arrive_expect_tx(&kfull[s], kKBytes);
+        tma3(st, mk, 0, g, krow, &kfull[s]);
+        tma3(st + kSlice, mk, 64, g, krow, &kfull[s]);
+        if (j >= 2 && !wait_or_abort(&vempty[s], par, p.err, abort_flag)) {
+          ++issued;  // the K half is in flight
+          break;
         }
+        mbar_arrive_expect_tx(&vfull[s], kVBytes);
+        tma2(st + kKBytes, mv, r0, vrow, &vfull[s]);
+        tma2(st + kKBytes + kSlice, mv, r0 + 64, vrow, &vfull[s]);
         ++issued;
       }
       // the copies issued land before the CTA can exit
       mbar_wait_bounded(qfull, 0, p.err);
-      for (int j = max(0, issued - 2); j < issued; ++j)
+      for (int j = max(0, issued - 2); j < issued; ++j) {
         mbar_wait_bounded(&kfull[j & 1], (uint32_t)((j >> 1) & 1), p.err);
+        mbar_wait_bounded(&vfull[j & 1], (uint32_t)((j >> 1) & 1), p.err);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -294,12 +326,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           mma(tmem + (uint32_t)(s * kN), a, bb, idesc, kk ? 1u : 0u);
         }
         commit(&sfull[s]);
+        commit(&kempty[s]);
         return true;
       };
       bool ok = wait_or_abort(qfull, 0, p.err, abort_flag) && (n_tiles == 0 || issue_s(0));
       for (int j = 0; ok && j < n_tiles; ++j) {
         if (j + 1 < n_tiles && !issue_s(j + 1)) break;
         if (!wait_or_abort(pfull, (uint32_t)(j & 1), p.err, abort_flag)) break;
+        if (!wait_or_abort(&vfull[j & 1], (uint32_t)((j >> 1) & 1), p.err, abort_flag)) break;
         fence_after();
         const unsigned char* st = stages + (j & 1) * kStage;
         const uint64_t vd0 = desc128(st + kKBytes), vd1 = desc128(st + kKBytes + kSlice);
@@ -310,112 +344,146 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           mma(tmem + 2u * kN, a, bb, idesc, (j | kk) ? 1u : 0u);
         }
         commit(ofull);
-        commit(&kempty[j & 1]);
+        commit(&vempty[j & 1]);
       }
       commit(done);
       mbar_wait_bounded(done, 0, p.err);
     }
   } else {
-    // ---------------- softmax: thread = query row (its TMEM lane)
+    // ---------------- softmax: warps 2-9, two per TMEM lane quarter; thread = (query row, half
+    // of the keys and of the output dims). The halves exchange only the row maximum per tile.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const int tok = t0 + row / Gq;              // query token of this row
     const int hq = g * Gq + row % Gq;           // query head
     const bool row_ok = tok < p.T;
     const int vis = p.L - p.T + min(tok, p.T - 1);  // last visible local row
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t col0 = (uint32_t)(half * 64);
     const float c = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool aborted = false;
-    // tcgen05.ld/st are warp-collective: every decision around them is taken warp-uniformly
-    for (int j = 0; j < n_tiles; ++j) {
+    float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+    bool bad = false;              // a wait gave up: no more tensor-memory work
+    int j = 0;
+    // tcgen05.ld/st are warp-collective: decisions around them are warp-uniform; leaving the
+    // loop is a vote of all 256 softmax threads at the per-tile barrier
+    for (; j < n_tiles; ++j) {
       const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, wait_or_abort(&sfull[sb], (uint32_t)((j >> 1) & 1), p.err, abort_flag))) {
-        aborted = true;
-        break;
-      }
-      fence_after();
+      bool ok = !bad && __all_sync(0xffffffffu, wait_or_abort(&sfull[sb], (uint32_t)((j >> 1) & 1),
+                                                               p.err, abort_flag));
       const bool is_ctx = j < CT;
-      const int k0 = is_ctx ? j * kN : (j - CT) * kN;
-      const int lim = is_ctx ? n_ctx - 1 - k0 : vis - k0;  // keys [0, lim] of the tile visible
-      const uint32_t sa = lane_base + (uint32_t)(sb * kN);
-      // pass 1: the tile's maximum
+      const int k0 = (is_ctx ? j * kN : (j - CT) * kN) + half * 64;
+      const int lim = is_ctx ? n_ctx - 1 - k0 : vis - k0;  // this half's keys [0, lim] visible
+      const uint32_t sa = lane_base + (uint32_t)(sb * kN) + col0;
+      const bool all_vis = lim >= 63;  // every key of this half visible to the row
       float mx = -INFINITY;
+      if (ok) {
+        fence_after();
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t r[32];
-        ld32(sa + ch * 32, r);
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t r[32];
+          ld32(sa + ch * 32, r);
+          if (all_vis) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (ch * 32 + q <= lim) mx = fmaxf(mx, __uint_as_float(r[q]) * c);
+            for (int q = 0; q < 32; ++q) mx = fmaxf(mx, __uint_as_float(r[q]));
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (ch * 32 + q <= lim) mx = fmaxf(mx, __uint_as_float(r[q]));
+          }
+        }
+        mx *= c;  // the scale is positive: max of the scaled scores
       }
+      xmax[(j & 1) * 256 + half * 128 + row] = mx;
+      if (!named_sync_softmax_and(ok)) break;  // every softmax thread leaves together
+      mx = fmaxf(mx, xmax[(j & 1) * 256 + (half ^ 1) * 128 + row]);
       // the running maximum moves only by more than kRaise (then O is rescaled)
-      float alpha = 1.f;
       const bool raise = mx > m + kRaise || m == -INFINITY;
       const float m_new = raise ? mx : m;
+      float alpha = 1.f;
       if (raise && m != -INFINITY) alpha = exp2f(m - m_new);
       // P_{j-1} . V_{j-1} must be done before P is rewritten and before O is rescaled
       if (j > 0) {
-        if (!__all_sync(0xffffffffu, wait_or_abort(ofull, (uint32_t)((j - 1) & 1), p.err, abort_flag))) {
-          aborted = true;
-          break;
+        ok = __all_sync(0xffffffffu, wait_or_abort(ofull, (uint32_t)((j - 1) & 1), p.err, abort_flag));
+        if (!ok) {
+          bad = true;
+          continue;  // the next barrier vote ends the loop for everyone
         }
         fence_after();
         if (__any_sync(0xffffffffu, raise && m != -INFINITY)) {  // lanes not raising scale by 1
 #pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < 2; ++ch) {
             uint32_t r[32];
-            ld32(lane_base + 2u * kN + ch * 32, r);
+            ld32(lane_base + 2u * kN + col0 + ch * 32, r);
 #pragma unroll
             for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * alpha);
-            st32(lane_base + 2u * kN + ch * 32, r);
+            st32(lane_base + 2u * kN + col0 + ch * 32, r);
           }
         }
       }
       m = (m_new == -INFINITY) ? m : m_new;
       l *= alpha;
-      // pass 2: probabilities in bf16 into the operand layout (row-major 64-key slices,
+      // pass 2: this half's probabilities in bf16 into P slice `half` (row-major 64 keys,
       // 16-byte chunk index XOR row % 8)
-      float sum = 0.f;
+      float sum0 = 0.f, sum1 = 0.f;
+      unsigned char* slice = p_s + half * kSlice + row * 128;
+      const float negm = -m;
+      const bool none = m == -INFINITY;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t r[32];
         ld32(sa + ch * 32, r);
         uint32_t pk[16];
+        if (all_vis && !none) {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int k = ch * 32 + 2 * q;
-          const float p0 = (k <= lim && m != -INFINITY) ? exp2f(__uint_as_float(r[2 * q]) * c - m) : 0.f;
-          const float p1 = (k + 1 <= lim && m != -INFINITY) ? exp2f(__uint_as_float(r[2 * q + 1]) * c - m) : 0.f;
-          sum += p0 + p1;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int q = 0; q < 16; ++q) {
+            const float p0 = ex2(fmaf(__uint_as_float(r[2 * q]), c, negm));
+            const float p1 = ex2(fmaf(__uint_as_float(r[2 * q + 1]), c, negm));
+            sum0 += p0;
+            sum1 += p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int k = ch * 32 + 2 * q;
+            const float p0 = (k <= lim && !none) ? ex2(fmaf(__uint_as_float(r[2 * q]), c, negm)) : 0.f;
+            const float p1 = (k + 1 <= lim && !none) ? ex2(fmaf(__uint_as_float(r[2 * q + 1]), c, negm)) : 0.f;
+            sum0 += p0;
+            sum1 += p1;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[q] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
         }
-        unsigned char* slice = p_s + (ch >> 1) * kSlice + row * 128;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {  // 4 chunks of 16 bytes (8 keys) of this 32-key group
-          const int chunk = (ch & 1) * 4 + q4;
+          const int chunk = ch * 4 + q4;
           *reinterpret_cast<uint4*>(slice + ((chunk ^ (row & 7)) << 4)) =
               make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
         }
       }
-      l += sum;
+      l += sum0 + sum1;
       fence_before();
       fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
       mbar_arrive(&sfree[sb]);
       mbar_arrive(pfull);
     }
-    // epilogue: O / l of the last tile's accumulator
-    const bool fin = !aborted && n_tiles > 0 &&
-                     wait_or_abort(ofull, (uint32_t)((n_tiles - 1) & 1), p.err, abort_flag);
-    if (__all_sync(0xffffffffu, fin)) {
+    // epilogue: O / l of the last tile's accumulator (the halves add their shares of l)
+    const bool fin = j == n_tiles && n_tiles > 0 && !bad &&
+                     __all_sync(0xffffffffu, wait_or_abort(ofull, (uint32_t)((n_tiles - 1) & 1),
+                                                           p.err, abort_flag));
+    xsum[half * 128 + row] = l;
+    const bool all_fin = named_sync_softmax_and(fin);
+    if (all_fin) {
       fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* out = p.O + (((int64_t)b * p.T + tok) * p.h_q + hq) * kD;
+      const float lt = l + xsum[(half ^ 1) * 128 + row];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      __nv_bfloat16* out = p.O + (((int64_t)b * p.T + tok) * p.h_q + hq) * kD + half * 64;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 2; ++ch) {
         uint32_t r[32];
-        ld32(lane_base + 2u * kN + ch * 32, r);
+        ld32(lane_base + 2u * kN + col0 + ch * 32, r);
         if (row_ok && !*abort_flag) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
@@ -495,7 +563,8 @@ AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int 
   pl.k_bytes = al((size_t)B * L * h_kv * atc::kD * 2);
   pl.vl_bytes = al((size_t)B * h_kv * atc::kD * pl.Lp * 2);
   pl.vc_bytes = max_ctx > 0 ? al((size_t)B * h_kv * atc::kD * pl.Mp * 2) : 0;
-  pl.smem = 1024 + atc::kQBytes + atc::kStages * atc::kStage + 2 * atc::kSlice + 16 * 8 + 16;
+  pl.smem = 1024 + atc::kQBytes + atc::kStages * atc::kStage + 2 * atc::kSlice + 768 * 4 +
+            20 * 8 + 16;
   return pl;
 }
 
