@@ -144,27 +144,34 @@ __device__ __forceinline__ float ex2(float x) {
 
 // ------------------------------------------------------------------------------ pre-pass
 // Rotated bf16 copies of rows [n_rows, 128]: row r sits at position base + (r / div) % mod.
-// One warp per row; lane l takes the RoPE pairs l and l + 32 (dims l, l+64, l+32, l+96).
+// Eight threads per row; thread q takes the RoPE pairs 8q .. 8q+7 (dims 8q.., 64+8q..) with
+// 16-byte loads and stores.
 __global__ void __launch_bounds__(256) rope_rows_kernel(const __nv_bfloat16* __restrict__ src,
                                                         __nv_bfloat16* __restrict__ dst,
                                                         int64_t n_rows, int64_t div, int64_t mod,
                                                         int64_t base, AtcParams p) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const unsigned long long F0 = p.rope_turns[lane], F1 = p.rope_turns[lane + 32];
-  for (int64_t r = warp; r < n_rows; r += nw) {
-    const int64_t pos = base + (r / div) % mod;
-    const __nv_bfloat16* s = src + r * kD;
-    __nv_bfloat16* d = dst + r * kD;
+  const int q = threadIdx.x & 7;
+  const int64_t r0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
+  const int64_t nr = ((int64_t)gridDim.x * blockDim.x) >> 3;
+  unsigned long long F[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = lane + 32 * h;
-      const float a = __bfloat162float(s[i]), c = __bfloat162float(s[i + 64]);
-      const float2 cs = p.rope ? rot_turns(pos, h ? F1 : F0) : make_float2(1.f, 0.f);
-      d[i] = __float2bfloat16_rn(a * cs.x - c * cs.y);
-      d[i + 64] = __float2bfloat16_rn(c * cs.x + a * cs.y);
+  for (int e = 0; e < 8; ++e) F[e] = p.rope_turns[8 * q + e];
+  for (int64_t r = r0; r < n_rows; r += nr) {
+    const int64_t pos = base + (r / div) % mod;
+    const uint4 lo = *reinterpret_cast<const uint4*>(src + r * kD + 8 * q);
+    const uint4 hi = *reinterpret_cast<const uint4*>(src + r * kD + 64 + 8 * q);
+    float a[8], c[8];
+    Vec<__nv_bfloat16, 8>::unpack(lo, a);
+    Vec<__nv_bfloat16, 8>::unpack(hi, c);
+    __align__(16) __nv_bfloat16 ol[8], oh[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 cs = p.rope ? rot_turns(pos, F[e]) : make_float2(1.f, 0.f);
+      ol[e] = __float2bfloat16_rn(a[e] * cs.x - c[e] * cs.y);
+      oh[e] = __float2bfloat16_rn(c[e] * cs.x + a[e] * cs.y);
     }
+    *reinterpret_cast<uint4*>(dst + r * kD + 8 * q) = *reinterpret_cast<const uint4*>(ol);
+    *reinterpret_cast<uint4*>(dst + r * kD + 64 + 8 * q) = *reinterpret_cast<const uint4*>(oh);
   }
 }
 
@@ -580,8 +587,8 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
   // pre-pass: rotated Q and local K, transposed V
   {
     const int64_t qrows = (int64_t)p.B * p.T * p.h_q, krows = (int64_t)p.B * p.L * p.h_kv;
-    const int64_t grid_q = std::min<int64_t>((qrows + 7) / 8, (int64_t)sms * 16);
-    const int64_t grid_k = std::min<int64_t>((krows + 7) / 8, (int64_t)sms * 16);
+    const int64_t grid_q = std::min<int64_t>((qrows + 31) / 32, (int64_t)sms * 16);
+    const int64_t grid_k = std::min<int64_t>((krows + 31) / 32, (int64_t)sms * 16);
     atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_q, 1), 256, 0, st>>>(
         p.Q, q_rot, qrows, p.h_q, p.T, (int64_t)p.pos0 + p.L - p.T, p);
     atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_k, 1), 256, 0, st>>>(
