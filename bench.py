@@ -18,7 +18,10 @@ tokens: doc-wise RoPE + chunk pooling of K, V, K_r, bank preparation, tensor-cor
 ``--workload interleave10m`` runs Memory Interleaving at its full configuration (18 routed
 layers, each over its own 10M-token bank; B = 32 queries of T = 256 tokens, k = 8, 3 rounds:
 each round re-routes with the appended documents excluded and attends over their raw K/V
-placed before the query tokens); its line reports queries/s of the whole interleave. ``--impl reference`` times the CPU oracle on the host cores (a bounded
+placed before the query tokens); its line reports queries/s of the whole interleave.
+``--workload attend_long`` times one msa_sparse_attend call alone at the last interleave round's
+shape with 4 queries (256 tokens, 64 memory + 8,256 local rows): the small case for profiling
+the tensor-core attention. ``--impl reference`` times the CPU oracle on the host cores (a bounded
 sample of the same workload). Under torchrun every rank runs an independent replica
 (the path does not shard: no collective on the data path).
 """
@@ -50,7 +53,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
-                    choices=["bank100m", "bank10m", "prefill1m", "interleave10m"])
+                    choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long"])
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
                     help="host-bank fetch: device gather over the host link on a side stream "
                          "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
@@ -831,6 +834,47 @@ def run_interleave(args):
         dist.destroy_process_group()
 
 
+def run_attend_long(args):
+    """One long-query attention call (the last interleave round's shape, B = 4), CUDA events."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    import synth
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.C5
+    B, T, L, mc = 4, w.T, w.T + 2 * w.k * w.doc_len, w.k * 8
+    bf = torch.bfloat16
+    Q = synth.dev_normal(torch.empty((B, T, w.h_q, w.d), dtype=bf, device=dev), w.seed, 1)
+    Kl = synth.dev_normal(torch.empty((B, L, w.h_kv, w.d), dtype=bf, device=dev), w.seed, 2)
+    Vl = synth.dev_normal(torch.empty_like(Kl), w.seed, 3)
+    cK = synth.dev_normal(torch.empty((B, mc, w.h_kv, w.d), dtype=bf, device=dev), w.seed, 4)
+    cV = synth.dev_normal(torch.empty_like(cK), w.seed, 5)
+    cl = torch.full((B,), mc, dtype=torch.int32, device=dev)
+    ws = torch.empty(msa.msa_sparse_attend_workspace(B, T, w.h_q, w.h_kv, w.d, mc, L),
+                     dtype=torch.uint8, device=dev)
+    O = torch.empty((B, T, w.h_q, w.d), dtype=bf, device=dev)
+    st = torch.cuda.Stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(max(args.warmup, 3)):
+        msa.msa_sparse_attend(Q, Kl, Vl, cK, cV, cl, w.k, w.rope_base, 0.0, O, ws, st)
+    Kst = max(1, min(args.steps, 20))
+    e0.record(st)
+    for _ in range(Kst):
+        msa.msa_sparse_attend(Q, Kl, Vl, cK, cV, cl, w.k, w.rope_base, 0.0, O, ws, st)
+    e1.record(st)
+    st.synchronize()
+    ms = e0.elapsed_time(e1) / Kst
+    flop = 4.0 * B * T * w.h_q * (mc + L - T + (T + 1) / 2.0) * w.d
+    print(json.dumps({"metric": "long-query attention TFLOP/s (call incl. RoPE/transpose pre-pass)",
+                      "value": round(flop / (ms / 1e3) / 1e12, 1), "unit": "TFLOP/s",
+                      "ms_per_call": round(ms, 4), "steps": Kst, "dtype": "bf16",
+                      "config": {"workload": "attend_long", "batch": B, "T": T, "h_q": w.h_q,
+                                 "h_kv": w.h_kv, "d": w.d, "memory_rows": mc, "local_rows": L}}),
+          flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -839,6 +883,8 @@ def main():
         run_prefill(args)
     elif args.workload == "interleave10m":
         run_interleave(args)
+    elif args.workload == "attend_long":
+        run_attend_long(args)
     else:
         run_libmsa(args)
 
