@@ -692,8 +692,12 @@ def run_interleave(args):
         synth.dev_normal(vp, w.seed, synth.tag(synth.APPV, l))
         pools.append((kp, vp))
     Ls = [T + r * k * w.doc_len for r in range(R)]
-    kloc = [torch.empty((B, Lr, w.h_kv, w.d), dtype=bf, device=dev) for Lr in Ls]
-    vloc = [torch.empty_like(t) for t in kloc]
+    kloc = [None] + [torch.empty((B, Lr, w.h_kv, w.d), dtype=bf, device=dev) for Lr in Ls[1:]]
+    vloc = [None] + [torch.empty_like(t) for t in kloc[1:]]
+    doc_bytes = w.doc_len * w.h_kv * w.d * 2
+    seglen = [None] + [torch.full((B, r * k), w.doc_len, dtype=torch.int32, device=dev)
+                       for r in range(1, R)]
+    ws_s = torch.zeros(256, dtype=torch.uint8, device=dev)
     ws_r = torch.empty(msa.msa_route_topk_workspace(B, T, w.h_qr, w.h_kv, w.d, 1, n_docs,
                                                     n_chunks, k), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(max(msa.msa_sparse_attend_workspace(B, T, w.h_q, w.h_kv, w.d, max_ctx, Lr)
@@ -735,15 +739,17 @@ def run_interleave(args):
                     if rec:
                         ev[2].record(st)
                     if r > 0:  # [appended documents (round order, ascending id) ; query tokens]
-                        sel = (appended[:, :r * k] % P).reshape(-1)
-                        kloc[r][:, :A] = pools[l][0].index_select(0, sel).view(B, A, w.h_kv, w.d)
-                        vloc[r][:, :A] = pools[l][1].index_select(0, sel).view(B, A, w.h_kv, w.d)
-                    kloc[r][:, A:] = d["K_loc"]
-                    vloc[r][:, A:] = d["V_loc"]
+                        idx = (appended[:, :r * k] % P) * doc_bytes
+                        msa.msa_assemble_local(idx + pools[l][0].data_ptr(),
+                                               idx + pools[l][1].data_ptr(), seglen[r],
+                                               d["K_loc"], d["V_loc"], kloc[r], vloc[r], ws_s, st)
+                        kl, vl = kloc[r], vloc[r]
+                    else:  # round 0: the query tokens alone
+                        kl, vl = d["K_loc"], d["V_loc"]
                     if rec:
                         ev[3].record(st)
-                    msa.msa_sparse_attend(d["Q"], kloc[r], vloc[r], cK, cV, cl, k, w.rope_base,
-                                          0.0, O, ws_a, st)
+                    msa.msa_sparse_attend(d["Q"], kl, vl, cK, cV, cl, k, w.rope_base, 0.0, O,
+                                          ws_a, st)
                     if rec:
                         ev[4].record(st)
                 # the last routed layer's documents are appended and excluded from now on
@@ -824,7 +830,7 @@ def run_interleave(args):
                      "traffic": None, "flop_per_launch": route_flop,
                      "avg_launch_ms": round(route_call_ms, 4)},
         "attend_tflops": round(att_tf, 1),
-        "gpu_launches": Kst * R * NL * 8,
+        "gpu_launches": Kst * R * NL * 9,
         "clocks": clocks,
     }
     if rank == 0:

@@ -261,6 +261,29 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
                              int32_t pos0, float rope_base, float scale, void* O, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------------------
+ * msa_assemble_local - the local context of a Memory Interleaving round: for every query b,
+ * the raw per-token K/V of the documents appended so far (segment 0 .. n_seg-1, in the order
+ * appended) followed by the query's own T token rows, written contiguously.
+ *   [ai-papers.net summary, "MSAの提案手法"; ruixiangma.github.io blog, "Memory Interleaving":
+ *    each round's retrieved documents have their original text appended to the query's
+ *    context for the next round]
+ *
+ * seg_k, seg_v  device arrays of B * n_seg device pointers (row-major [b][segment]), each to a
+ *               segment's [seg_len, h_kv, d] rows (dtype), 16-byte aligned.
+ * seg_len       device int32 [B * n_seg].
+ * K_q, V_q      [B, T, h_kv, d] the query tokens' own K/V (before RoPE, like K_loc).
+ * K_out, V_out  [B, L_loc, h_kv, d]; caller-owned. Requires sum_q seg_len[b][q] + T == L_loc
+ *               for every query; a query for which it does not hold is left unwritten and the
+ *               workspace status word records the error (msa_workspace_status).
+ * ws            >= 256 bytes, 256-byte aligned; 0 <= n_seg <= 1024.
+ */
+msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k,
+                              const void* const* seg_v, const int32_t* seg_len, const void* K_q,
+                              const void* V_q, int32_t T, int32_t h_kv, int32_t d, int32_t dtype,
+                              int64_t L_loc, void* K_out, void* V_out, void* ws, size_t ws_bytes,
+                              void* stream);
+
 #ifdef __cplusplus
 }
 #endif

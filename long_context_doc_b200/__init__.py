@@ -32,7 +32,7 @@ SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chun
            "msa_route_topk", "msa_route_topk_noalloc",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
-           "msa_sparse_attend")
+           "msa_sparse_attend", "msa_assemble_local")
 
 
 class MSAError(RuntimeError):
@@ -88,6 +88,9 @@ def _load():
     L.msa_sparse_attend.restype = ctypes.c_int
     L.msa_sparse_attend.argtypes = [vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32,
                                     i32, f32, f32, vp, vp, sz, vp]
+    L.msa_assemble_local.restype = ctypes.c_int
+    L.msa_assemble_local.argtypes = [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, vp, vp,
+                                     vp, sz, vp]
     return L
 
 
@@ -178,6 +181,16 @@ def msa_workspace_status(ws, stream=None) -> int:
     if st not in (0, 6):
         _check(st)
     return int(code.value)
+
+
+def msa_assemble_local(seg_k_ptrs, seg_v_ptrs, seg_len, K_q, V_q, K_out, V_out, ws, stream=None):
+    """seg_k_ptrs, seg_v_ptrs: int64 device tensors [B, n_seg] of segment data pointers;
+    seg_len: int32 device [B, n_seg]; K_q, V_q: [B, T, h_kv, d]; K_out, V_out: [B, L, h_kv, d]."""
+    B, n_seg = seg_len.shape
+    T, h_kv, d = K_q.shape[1], K_q.shape[2], K_q.shape[3]
+    _check(lib.msa_assemble_local(B, n_seg, _p(seg_k_ptrs), _p(seg_v_ptrs), _p(seg_len), _p(K_q),
+                                  _p(V_q), T, h_kv, d, dtype_code(K_q), K_out.shape[1], _p(K_out),
+                                  _p(V_out), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
 def msa_gather(top_ids, doc_chunk_off, Kbar, Vbar, max_ctx, gather_idx, ctx_len, ctxK, ctxV, ws,

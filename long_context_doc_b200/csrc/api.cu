@@ -652,4 +652,42 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
   return ok();
 }
 
+// ----------------------------------------------------------------------------- interleave
+msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k,
+                              const void* const* seg_v, const int32_t* seg_len, const void* K_q,
+                              const void* V_q, int32_t T, int32_t h_kv, int32_t d, int32_t dtype,
+                              int64_t L_loc, void* K_out, void* V_out, void* ws, size_t ws_bytes,
+                              void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && n_seg >= 0 && n_seg <= 1024 && T >= 0 && L_loc >= T, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d n_seg=%d T=%d L_loc=%lld)", B, n_seg, T, (long long)L_loc);
+  REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "assemble needs a 256-byte aligned workspace of >= 256 bytes");
+  if (B == 0 || L_loc == 0) return ok();
+  REQUIRE(K_out && V_out && (T == 0 || (K_q && V_q)) && (n_seg == 0 || (seg_k && seg_v && seg_len)),
+          MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(aligned16(K_out) && aligned16(V_out) && (T == 0 || (aligned16(K_q) && aligned16(V_q))),
+          MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  msa::AssembleParams p{};
+  p.B = B;
+  p.n_seg = n_seg;
+  p.T = T;
+  p.L = L_loc;
+  p.row_bytes = (int64_t)h_kv * d * (dtype == 1 ? 2 : 4);
+  p.seg_k = seg_k;
+  p.seg_v = seg_v;
+  p.seg_len = seg_len;
+  p.K_q = K_q;
+  p.V_q = V_q;
+  p.K_out = K_out;
+  p.V_out = V_out;
+  p.err = static_cast<int*>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess) e = msa::launch_assemble_local(p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_assemble_local launch");
+  return ok();
+}
+
 }  // extern "C"

@@ -167,6 +167,22 @@ struct DecPlan {
 DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
 
+// ---- assemble.cu: local context of a Memory Interleaving round
+struct AssembleParams {
+  int B, n_seg, T;
+  int64_t L;                  // local rows per query: sum of the segment lengths + T
+  int64_t row_bytes;          // h_kv * d * element size (multiple of 16)
+  const void* const* seg_k;   // [B * n_seg] device pointers, each [seg_len, h_kv, d]
+  const void* const* seg_v;
+  const int32_t* seg_len;     // [B * n_seg]
+  const void* K_q;            // [B, T, h_kv, d]
+  const void* V_q;
+  void* K_out;                // [B, L, h_kv, d]
+  void* V_out;
+  int* err;                   // workspace status word
+};
+cudaError_t launch_assemble_local(const AssembleParams& p, cudaStream_t st);
+
 // ---- attend_tc.cu: long-query attention on tensor cores (bf16, d = 128, (h_q/h_kv) * T >= 64,
 // h_q/h_kv dividing 128)
 struct AtcParams {

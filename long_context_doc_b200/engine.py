@@ -18,7 +18,7 @@ from typing import Callable, List, Optional, Sequence
 
 import torch
 
-from . import gather, route_topk, sparse_attend
+from . import gather, msa_assemble_local, route_topk, sparse_attend
 
 
 @dataclass
@@ -45,6 +45,28 @@ def exclusion_bits(appended: Sequence[Sequence[int]], n_docs: int, device) -> to
             bits[b, doc // 32] |= 1 << (doc % 32)
     bits = torch.where(bits >= 2 ** 31, bits - 2 ** 32, bits)
     return bits.to(torch.int32).to(device)
+
+
+def assemble_local(parts, K_q, V_q):
+    """parts[b] = [(K, V) [len, h_kv, d] device tensors of the appended documents, in order];
+    returns the local K/V [B, sum(len) + T, h_kv, d] built by msa_assemble_local."""
+    B, T = K_q.shape[0], K_q.shape[1]
+    n_seg = len(parts[0])
+    if any(len(p) != n_seg for p in parts):
+        raise ValueError("every query appends the same number of documents")
+    L = {sum(kv[0].shape[0] for kv in p) + T for p in parts}
+    if len(L) != 1:
+        raise ValueError("interleaved local contexts must have one length per batch")
+    L = L.pop()
+    dev = K_q.device
+    kp = torch.tensor([[kv[0].data_ptr() for kv in p] for p in parts], dtype=torch.int64).to(dev)
+    vp = torch.tensor([[kv[1].data_ptr() for kv in p] for p in parts], dtype=torch.int64).to(dev)
+    ln = torch.tensor([[kv[0].shape[0] for kv in p] for p in parts], dtype=torch.int32).to(dev)
+    K_out = torch.empty((B, L) + tuple(K_q.shape[2:]), dtype=K_q.dtype, device=dev)
+    V_out = torch.empty_like(K_out)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    msa_assemble_local(kp, vp, ln, K_q, V_q, K_out, V_out, ws)
+    return K_out, V_out
 
 
 def routed_layer(layer: RoutedLayer, k: int, K_loc: torch.Tensor, V_loc: torch.Tensor,
@@ -77,15 +99,10 @@ def interleave_rounds(layers: List[RoutedLayer], k: int, rounds: int, rope_base:
         for li, layer in enumerate(layers):
             if r == 0:
                 K_loc, V_loc = layer.K_q, layer.V_q
-            else:
-                ks, vs = [], []
-                for b in range(B):
-                    parts = [doc_kv(li, doc) for doc in appended[b]]
-                    ks.append(torch.cat([p[0] for p in parts] + [layer.K_q[b]]))
-                    vs.append(torch.cat([p[1] for p in parts] + [layer.V_q[b]]))
-                if len({x.shape[0] for x in ks}) != 1:
-                    raise ValueError("interleaved local contexts must have one length per batch")
-                K_loc, V_loc = torch.stack(ks), torch.stack(vs)
+            else:  # [appended documents' raw K/V, in the order appended ; query tokens]
+                K_loc, V_loc = assemble_local(
+                    [[doc_kv(li, doc) for doc in appended[b]] for b in range(B)],
+                    layer.K_q, layer.V_q)
             ids, sc, O = routed_layer(layer, k, K_loc, V_loc, rope_base, ex)
             ids_r.append(ids)
             sc_r.append(sc)

@@ -100,3 +100,41 @@ def _masked(ref, r, l, w):
         for b in range(w.B):
             ds[b, ref["appended"][b][:r * w.k]] = -np.inf
     return ds
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dt", ["fp32", "bf16"])
+def test_assemble_local_matches_concatenation(gpu, dt):
+    """msa_assemble_local writes [segments in order ; query rows] bit for bit; a query whose
+    segment lengths do not add up to L_loc - T is reported through the workspace status."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    from long_context_doc_b200 import engine
+    rng = np.random.default_rng(2)
+    B, T, h, d = 3, 5, 2, 64
+    lens = [[7, 3, 12], [10, 10, 2], [1, 20, 1]]  # 22 appended rows per query
+    tdt = torch.float32 if dt == "fp32" else torch.bfloat16
+
+    def mk(*shape):
+        return torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(gpu).to(tdt)
+
+    parts = [[(mk(n, h, d), mk(n, h, d)) for n in row] for row in lens]
+    Kq, Vq = mk(B, T, h, d), mk(B, T, h, d)
+    K, V = engine.assemble_local(parts, Kq, Vq)
+    torch.cuda.synchronize()
+    assert K.shape == (B, 22 + T, h, d)
+    for b in range(B):
+        assert torch.equal(K[b], torch.cat([p[0] for p in parts[b]] + [Kq[b]]))
+        assert torch.equal(V[b], torch.cat([p[1] for p in parts[b]] + [Vq[b]]))
+    # one row too many in L_loc: every query mismatches, nothing is written, status is set
+    kp = torch.tensor([[kv[0].data_ptr() for kv in p] for p in parts], dtype=torch.int64).to(gpu)
+    vp = torch.tensor([[kv[1].data_ptr() for kv in p] for p in parts], dtype=torch.int64).to(gpu)
+    ln = torch.tensor(lens, dtype=torch.int32).to(gpu)
+    Ko = torch.full((B, 22 + T + 1, h, d), 7.0, dtype=tdt, device=gpu)
+    Vo = torch.full_like(Ko, 7.0)
+    ws = torch.zeros(256, dtype=torch.uint8, device=gpu)
+    msa.msa_assemble_local(kp, vp, ln, Kq, Vq, Ko, Vo, ws)
+    torch.cuda.synchronize()
+    assert msa.msa_workspace_status(ws) != 0
+    assert bool((Ko == 7.0).all()) and bool((Vo == 7.0).all())
