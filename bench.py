@@ -216,7 +216,8 @@ class Decode:
         self.route_ev = None
         self.scan = scan
         # own kernels per layer (memsets and copies excluded): route (tensor path: query fold +
-        # scan with fused top-k; CUDA-core path: one fused kernel), gather, RoPE table, attention
+        # scan with fused top-k; CUDA-core path: one fused kernel), gather, decode attention,
+        # the merge of its split queries
         self.kernels_per_layer = (2 if scan == "tc" else 1) + 1 + 1 + 1
 
     # per-layer pieces -------------------------------------------------------------

@@ -520,41 +520,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 }  // namespace atc
 
 // ------------------------------------------------------------------------------ host side
-namespace {
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeTiledFn encode_fn_atc() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-// bf16 map with the 128-byte swizzle (box rows of 64 elements), zero fill out of bounds
-bool encode_bf16_map_sw128(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
-                           const uint64_t* strides, const uint32_t* box) {
-  EncodeTiledFn fn = encode_fn_atc();
-  if (!fn || rank < 2 || rank > 5) return false;
-  cuuint64_t d[5], st[4];
-  cuuint32_t bx[5], es[5];
-  for (int i = 0; i < rank; ++i) {
-    d[i] = (cuuint64_t)dims[i];
-    bx[i] = (cuuint32_t)box[i];
-    es[i] = 1;
-    if (i + 1 < rank) st[i] = (cuuint64_t)strides[i];
-  }
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(ptr), d, st,
-            bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-}  // namespace
 
 AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L) {
   AtcPlan pl{};
@@ -610,27 +575,27 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
     const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_q, (uint64_t)p.B * p.T};
     const uint64_t str[2] = {row, row * p.h_q};
     const uint32_t box[3] = {64, (uint32_t)Gq, (uint32_t)(atc::kM / Gq)};
-    if (!encode_bf16_map_sw128(&mq, q_rot, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mq, q_rot, 3, dims, str, box, true)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.L};
     const uint64_t str[2] = {row, row * p.h_kv};
     const uint32_t box[3] = {64, 1, atc::kN};
-    if (!encode_bf16_map_sw128(&mkl, k_rot, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mkl, k_rot, 3, dims, str, box, true)) return cudaErrorInvalidValue;
     const uint64_t dv[2] = {(uint64_t)p.L, (uint64_t)p.B * p.h_kv * atc::kD};
     const uint64_t sv[1] = {(uint64_t)pl.Lp * 2};
     const uint32_t bv[2] = {64, atc::kD};
-    if (!encode_bf16_map_sw128(&mvl, vt_l, 2, dv, sv, bv)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mvl, vt_l, 2, dv, sv, bv, true)) return cudaErrorInvalidValue;
   }
   if (p.max_ctx > 0) {
     const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.max_ctx};
     const uint64_t str[2] = {row, row * p.h_kv};
     const uint32_t box[3] = {64, 1, atc::kN};
-    if (!encode_bf16_map_sw128(&mkc, p.cK, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mkc, p.cK, 3, dims, str, box, true)) return cudaErrorInvalidValue;
     const uint64_t dv[2] = {(uint64_t)p.max_ctx, (uint64_t)p.B * p.h_kv * atc::kD};
     const uint64_t sv[1] = {(uint64_t)pl.Mp * 2};
     const uint32_t bv[2] = {64, atc::kD};
-    if (!encode_bf16_map_sw128(&mvc, vt_c, 2, dv, sv, bv)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mvc, vt_c, 2, dv, sv, bv, true)) return cudaErrorInvalidValue;
   } else {  // no memory tiles: never read
     mkc = mkl;
     mvc = mvl;

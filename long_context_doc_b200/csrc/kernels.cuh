@@ -129,10 +129,10 @@ cudaError_t launch_attend(AttendParams p, int dtype, double rope_base, int pos0,
 // i < d/2 (all zero when base <= 0)
 void rope_turns(double base, int d, unsigned long long* out);
 
-// route_tc.cu: bf16 tensor map (no swizzle, zero fill out of bounds) of a rank-dimensional
-// array: dims innermost first, strides[rank - 1] in bytes, box in elements.
+// tmap.cu: bf16 tensor map of a rank-dimensional array (dims innermost first, strides[rank-1]
+// in bytes, box in elements; zero fill out of bounds), no swizzle or the 128-byte swizzle
 bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
-                     const uint64_t* strides, const uint32_t* box);
+                     const uint64_t* strides, const uint32_t* box, bool swizzle128);
 
 // ---- attend_dec.cu: decode-shaped attention (bf16, d = 128, <= 8 query rows per KV head,
 // h_kv in {1, 2, 4, 8})
