@@ -109,3 +109,36 @@ def test_attend_and_gather_reject_bad_arguments_on_host(msa):
 def test_fetch_finish_requires_begin(msa):
     r = msa.lib.msa_fetch_finish(None, None, 0, None, None, 8, 128, 1, 16, None, None, None, None, 0)
     assert r == 1
+
+
+def test_attend_fast_paths_check_their_workspace_on_host(msa):
+    """bf16 d=128 decode (<= 8 rows per KV head) and long-query (>= 64 rows) shapes take their
+    own kernels; each refuses a workspace smaller than its plan before touching the device."""
+    fake = ctypes.c_void_p(256)
+    for T, L in ((1, 2048), (64, 300)):  # decode kernel, tensor-core kernel
+        need = msa.msa_sparse_attend_workspace(2, T, 32, 8, 128, 128, L)
+        assert need > 256
+        r = msa.lib.msa_sparse_attend(fake, 2, T, 32, fake, fake, L, fake, fake, fake, 128, 8, 128,
+                                      1, 16, 1e6, 0.0, fake, fake, 256, None)
+        assert r == 3, (T, r)
+
+
+def test_assemble_local_rejects_bad_arguments_on_host(msa):
+    fake = ctypes.c_void_p(256)
+    ws = ctypes.c_void_p(512)
+    # more than 1024 segments per query
+    r = msa.lib.msa_assemble_local(2, 1025, fake, fake, fake, fake, fake, 4, 8, 128, 1, 10, fake,
+                                   fake, ws, 256, None)
+    assert r == 1
+    # L_loc shorter than the query rows
+    r = msa.lib.msa_assemble_local(2, 3, fake, fake, fake, fake, fake, 8, 8, 128, 1, 4, fake, fake,
+                                   ws, 256, None)
+    assert r == 1
+    # no workspace
+    r = msa.lib.msa_assemble_local(2, 3, fake, fake, fake, fake, fake, 4, 8, 128, 1, 10, fake, fake,
+                                   None, 0, None)
+    assert r == 3
+    # missing output
+    r = msa.lib.msa_assemble_local(2, 3, fake, fake, fake, fake, fake, 4, 8, 128, 1, 10, None, fake,
+                                   ws, 256, None)
+    assert r == 1
