@@ -262,3 +262,24 @@ def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=No
         res["O64"].append(O_r)
     res["appended"] = appended
     return res
+
+
+def generate(Q_steps, Kn_steps, Vn_steps, K_prompt, V_prompt, Kbar, Vbar, gather_idx, ctx_len,
+             pos0: int, rope_base: float, scale: float = 0.0, L=None):
+    """Oracle of sparse generation over an assembled context (reading R24 of the design notes).
+
+    Routing and context assembly come first and the routed memory then stays fixed while the
+    model generates autoregressively over the assembled context [news.neo-ai.one article,
+    "推論パイプライン"; ruixiangma.github.io blog, "三阶段推理流程"]. Step s brings the K/V of
+    its new tokens, Kn_steps[s], Vn_steps[s] [B, T, h_kv, d]: they join the end of the local
+    context [K_prompt ; tokens of steps 0 .. s-1], and the step's queries Q_steps[s]
+    [B, T, h_q, d] attend over [gathered memory ; that local context] exactly as ``attend``
+    (query token t is the local row L - T + t). Returns O64 [S, B, T, h_q, d]."""
+    K_loc, V_loc = np.asarray(K_prompt), np.asarray(V_prompt)
+    out = []
+    for s in range(len(Q_steps)):
+        K_loc = np.concatenate([K_loc, np.asarray(Kn_steps[s])], axis=1)
+        V_loc = np.concatenate([V_loc, np.asarray(Vn_steps[s])], axis=1)
+        out.append(attend(Q_steps[s], K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0,
+                          rope_base, scale, L))
+    return np.stack(out)

@@ -316,6 +316,63 @@ def test_msa_with_unit_chunks_and_all_docs_is_dense_causal_attention():
     assert np.max(np.abs(O[0].transpose(1, 0, 2) - ref)) < 5e-4  # fp32 angles in the reference
 
 
+# ----------------------------------------------------------------------------- generation
+def test_generate_token_by_token_is_causal_attention_over_the_whole_sequence():
+    """Sparse generation, one token per step, must equal textbook causal attention (torch's
+    SDPA, Qwen3 RoPE from transformers) over [memory rows as stored ; prompt and generated
+    tokens rotated at pos0 + j], each generated token's query at its own position."""
+    import torch.nn.functional as F
+    rng = np.random.default_rng(21)
+    B, S, L0, h_q, h_kv, d, pos0, base = 2, 5, 3, 4, 2, 8, 4, 1e4
+    n_bank = 6
+    Kb = rng.standard_normal((n_bank, h_kv, d)).astype(np.float32)
+    Vb = rng.standard_normal((n_bank, h_kv, d)).astype(np.float32)
+    n_ctx = np.array([4, 0], np.int32)
+    gi = np.full((B, 4), -1, np.int32)
+    gi[0] = [5, 0, 2, 3]
+    Kp = rng.standard_normal((B, L0, h_kv, d)).astype(np.float32)
+    Vp = rng.standard_normal((B, L0, h_kv, d)).astype(np.float32)
+    Qs = rng.standard_normal((S, B, 1, h_q, d)).astype(np.float32)
+    Ks = rng.standard_normal((S, B, 1, h_kv, d)).astype(np.float32)
+    Vs = rng.standard_normal((S, B, 1, h_kv, d)).astype(np.float32)
+    O = oracle.generate(Qs, Ks, Vs, Kp, Vp, Kb, Vb, gi, n_ctx, pos0, base)
+    assert O.shape == (S, B, 1, h_q, d)
+    for b in range(B):
+        mem_k = Kb[gi[b, :n_ctx[b]]].astype(np.float64)
+        mem_v = Vb[gi[b, :n_ctx[b]]].astype(np.float64)
+        loc_k = np.concatenate([Kp[b], Ks[:, b, 0]]).astype(np.float64)  # [L0 + S, h_kv, d]
+        loc_v = np.concatenate([Vp[b], Vs[:, b, 0]]).astype(np.float64)
+        loc_k = _qwen3_rope(loc_k.transpose(1, 0, 2), pos0 + np.arange(L0 + S),
+                            base).transpose(1, 0, 2)
+        q = _qwen3_rope(Qs[:, b, 0].astype(np.float64).transpose(1, 0, 2),
+                        pos0 + L0 + np.arange(S), base)  # [h_q, S, d]
+        keys = np.concatenate([mem_k, loc_k])
+        vals = np.concatenate([mem_v, loc_v])
+        n_mem = mem_k.shape[0]
+        mask = np.zeros((S, n_mem + L0 + S), bool)
+        for s in range(S):
+            mask[s, :n_mem + L0 + s + 1] = True
+        kt = torch.from_numpy(keys.transpose(1, 0, 2)).repeat_interleave(h_q // h_kv, 0)
+        vt = torch.from_numpy(vals.transpose(1, 0, 2)).repeat_interleave(h_q // h_kv, 0)
+        ref = F.scaled_dot_product_attention(torch.from_numpy(q), kt, vt,
+                                             attn_mask=torch.from_numpy(mask)).numpy()
+        assert np.max(np.abs(O[:, b, 0].transpose(1, 0, 2) - ref)) < 5e-4
+
+
+def test_generate_first_token_without_context_returns_its_value():
+    """No prompt, no memory: the first generated token attends to itself alone."""
+    rng = np.random.default_rng(22)
+    Qs = rng.standard_normal((1, 1, 1, 4, 8)).astype(np.float32)
+    Ks = rng.standard_normal((1, 1, 1, 2, 8)).astype(np.float32)
+    Vs = rng.standard_normal((1, 1, 1, 2, 8)).astype(np.float32)
+    empty = np.zeros((1, 0, 2, 8), np.float32)
+    bank = np.zeros((1, 2, 8), np.float32)
+    O = oracle.generate(Qs, Ks, Vs, empty, empty, bank, bank, np.full((1, 1), -1, np.int32),
+                        np.zeros(1, np.int32), pos0=2, rope_base=1e6)
+    for h in range(4):
+        assert np.array_equal(O[0, 0, 0, h], Vs[0, 0, 0, h // 2].astype(np.float64))
+
+
 def test_pipeline_tiny_config_runs_and_planted_recall_is_reported():
     w = synth.C1.scaled(n_docs=16, doc_len=128, n_planted=2)
     inp = synth.make_token_workload(w)
