@@ -21,7 +21,12 @@ each round re-routes with the appended documents excluded and attends over their
 placed before the query tokens); its line reports queries/s of the whole interleave.
 ``--workload attend_long`` times one msa_sparse_attend call alone at the last interleave round's
 shape with 4 queries (256 tokens, 64 memory + 8,256 local rows): the small case for profiling
-the tensor-core attention. ``--impl reference`` times the CPU oracle on the host cores (a bounded
+the tensor-core attention. ``--workload gen100m`` runs sparse generation at the 100M-token bank: per request the context is
+built once (the default workload's step: 18 routed layers of route + host-bank gather +
+attention of the query token), then 256 tokens are generated per query, each through 18
+decode steps (msa_decode_step: the token's K/V appended to the layer's 2,048-row local cache,
+attention over [gathered memory ; cache]); its line reports generated tokens/s.
+``--impl reference`` times the CPU oracle on the host cores (a bounded
 sample of the same workload). Under torchrun every rank runs an independent replica
 (the path does not shard: no collective on the data path).
 """
@@ -53,7 +58,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
-                    choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long"])
+                    choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long",
+                             "gen100m"])
+    ap.add_argument("--gen-tokens", type=int, default=256,
+                    help="gen100m: tokens generated per query after the context is built")
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
                     help="host-bank fetch: device gather over the host link on a side stream "
                          "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
@@ -153,7 +161,7 @@ class ClockSampler:
 class Decode:
     """Routed decode over a memory bank: per layer route -> fetch/gather -> attend."""
 
-    def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc"):
+    def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc", nbuf: int = 2):
         import torch
 
         import long_context_doc_b200 as msa
@@ -200,7 +208,8 @@ class Decode:
                                             self.n_chunks, k)
         ws_a = msa.msa_sparse_attend_workspace(B, w.T, w.h_q, w.h_kv, w.d, self.max_ctx, w.L_loc)
         self.buf = []
-        for _ in range(2):
+        self.nbuf = nbuf  # 2: layers alternate buffers; L: every layer keeps its context
+        for _ in range(nbuf):
             self.buf.append(dict(
                 ws_r=torch.empty(ws_r, dtype=torch.uint8, device=dev),
                 ws_a=torch.empty(ws_a, dtype=torch.uint8, device=dev),
@@ -222,7 +231,7 @@ class Decode:
 
     # per-layer pieces -------------------------------------------------------------
     def route(self, l):
-        msa, d, bf = self.msa, self.layers[l], self.buf[l % 2]
+        msa, d, bf = self.msa, self.layers[l], self.buf[l % self.nbuf]
         if self.route_ev is not None:
             self.route_ev[l][0].record(self.main)
         msa.msa_route_topk(d["Q_r"], d["Kbar_r"], d["inv"], self.coff, self.w.k, None, bf["ids"],
@@ -231,7 +240,7 @@ class Decode:
             self.route_ev[l][1].record(self.main)
 
     def begin(self, l):
-        bf = self.buf[l % 2]
+        bf = self.buf[l % self.nbuf]
         if self.fetch == "memcpy":
             self.fetchers[l % 2].begin(bf["ids"], self.coff, self.max_ctx, bf["gi"], bf["cl"],
                                        bf["ws_g"], self.main)
@@ -252,12 +261,12 @@ class Decode:
         if self.fetch == "zerocopy":
             self.main.wait_event(self.ev_gather[l % 2])
         if self.fetch == "memcpy":
-            bf = self.buf[l % 2]
+            bf = self.buf[l % self.nbuf]
             self.fetchers[l % 2].finish(self.coff_host, self.Kh, self.Vh, self.max_ctx, bf["cK"],
                                         bf["cV"], self.main, self.copy, 10_000)
 
     def attend(self, l):
-        d, bf, w = self.layers[l], self.buf[l % 2], self.w
+        d, bf, w = self.layers[l], self.buf[l % self.nbuf], self.w
         self.msa.msa_sparse_attend(d["Q"], d["K_loc"], d["V_loc"], bf["cK"], bf["cV"], bf["cl"],
                                    w.k, w.rope_base, 0.0, self.O[l], bf["ws_a"], self.main)
 
@@ -502,6 +511,32 @@ def run_reference(args):
         return
     import oracle
     import synth
+    if args.workload == "gen100m":
+        w = synth.C4
+        times = []
+        for s in range(args.steps):
+            times.append(oracle_generate_time(w, s % w.layers, 4) / 4 * w.layers)
+            if sum(times) > 120:
+                break
+        token = statistics.mean(times)
+        value = w.B / token
+        unit = "generated tokens/s"
+        print(json.dumps({
+            "metric": "MSA sparse generation tokens/s at the 100M-token bank (context built once "
+                      "per request, routed memory fixed while generating)",
+            "value": round(value, 4), "unit": unit, "n_gpus": 1, "steps": len(times),
+            "warmup": args.warmup, "ms_per_step": round(token * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "gen100m", "routed_layers": w.layers, "batch": w.B,
+                       "prompt_local_kv": w.L_loc},
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "kind": "oracle",
+                             "cores": oracle.num_threads(),
+                             "sample": "each step = 4 generation steps of one routed layer for "
+                                       "the batch x the layer count (construction left out)"},
+            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
     w = synth.C4 if args.workload == "bank100m" else synth.C3
     for l in range(min(args.warmup, 1)):
         oracle_layer_time(w.scaled(n_docs=2000), l)
@@ -882,6 +917,281 @@ def run_attend_long(args):
           flush=True)
 
 
+def run_generate(args):
+    """Sparse generation at the 100M-token bank: context construction once per request, then
+    ``--gen-tokens`` decode steps through all routed layers; generated tokens/s."""
+    import torch
+    import torch.distributed as dist
+
+    import long_context_doc_b200 as msa
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    w = synth.C4
+    G = max(1, args.gen_tokens)
+    # one context buffer per layer: the gathered memory stays fixed while tokens are generated
+    wk = Decode(w, dev, args.fetch, rank, args.scan, nbuf=w.layers)
+    B, L0, bf = w.B, w.L_loc, torch.bfloat16
+    cap = L0 + G
+    lens = torch.zeros(wk.L, dtype=torch.int32, device=dev)
+    lens0 = torch.full((wk.L,), L0, dtype=torch.int32, device=dev)
+    caches, tok = [], []
+    ws_bytes = msa.msa_decode_step_workspace(B, 1, w.h_q, w.h_kv, w.d, wk.max_ctx, cap)
+    for l in range(wk.L):
+        c = msa.LocalCache(B, cap, w.h_kv, w.d, device=dev, length=lens[l:l + 1])
+        c.append(wk.layers[l]["K_loc"], wk.layers[l]["V_loc"])  # the prompt's local K/V
+        caches.append(c)
+        # the generated token's query and K/V at this layer (synthetic, reused every step)
+        tok.append(dict(
+            Q=synth.dev_normal(torch.empty((B, 1, w.h_q, w.d), dtype=bf, device=dev), w.seed,
+                               synth.tag(synth.GEN_Q, l)),
+            K=synth.dev_normal(torch.empty((B, 1, w.h_kv, w.d), dtype=bf, device=dev), w.seed,
+                               synth.tag(synth.GEN_K, l)),
+            V=synth.dev_normal(torch.empty((B, 1, w.h_kv, w.d), dtype=bf, device=dev), w.seed,
+                               synth.tag(synth.GEN_V, l)),
+            O=torch.empty((B, 1, w.h_q, w.d), dtype=bf, device=dev),
+            ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+    torch.cuda.synchronize()
+    assert int(lens[0]) == L0
+    dec_ev = None
+
+    def token_step():
+        for l in range(wk.L):
+            x, c, b = tok[l], caches[l], wk.buf[l]
+            if dec_ev is not None:
+                dec_ev[l][0].record(wk.main)
+            msa.msa_decode_step(x["Q"], x["K"], x["V"], c.K, c.V, c.length, b["cK"], b["cV"],
+                                b["cl"], w.k, w.rope_base, 0.0, x["O"], x["ws"], wk.main)
+            if dec_ev is not None:
+                dec_ev[l][1].record(wk.main)
+
+    def construct():
+        lens.copy_(lens0)  # a new request: every cache holds the prompt again
+        wk.step()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(wk.main):
+        for _ in range(max(args.warmup, 3)):
+            construct()
+            for _ in range(4):
+                token_step()
+    barrier()
+    use_graph = not args.no_graph and wk.fetch != "memcpy"
+    g_con = g_tok = None
+    if use_graph:
+        g_con, g_tok = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_con, stream=wk.main):
+            construct()
+        with torch.cuda.graph(g_tok, stream=wk.main):
+            token_step()
+    barrier()
+
+    def request(ev=None):
+        with torch.cuda.stream(wk.main):
+            if g_con is not None:
+                g_con.replay()
+            else:
+                construct()
+            if ev is not None:
+                ev.record(wk.main)
+            for _ in range(G):
+                if g_tok is not None:
+                    g_tok.replay()
+                else:
+                    token_step()
+
+    request()
+    barrier()
+    assert int(lens[0]) == cap and int(lens[-1]) == cap
+    for l in range(wk.L):
+        assert msa.msa_workspace_status(tok[l]["ws"], wk.main) == 0
+    Kst = max(1, args.steps)
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(Kst)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(Kst)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(Kst)]
+    barrier()
+    t0.record(wk.main)
+    for s in range(Kst):
+        starts[s].record(wk.main)
+        request(mids[s])
+        ends[s].record(wk.main)
+    t1.record(wk.main)
+    barrier()
+    clocks = sampler.stop()
+    req_ms = t0.elapsed_time(t1) / Kst
+    con_ms = statistics.mean(starts[s].elapsed_time(mids[s]) for s in range(Kst))
+    tok_ms = statistics.mean(mids[s].elapsed_time(ends[s]) for s in range(Kst)) / G
+    # decode-step durations for the roofline: one request's tokens launched eagerly with
+    # CUDA events around every msa_decode_step call (on the launching stream)
+    with torch.cuda.stream(wk.main):
+        construct()
+    n_ev = min(G, 64)
+    dec_all = []
+    for s in range(n_ev):
+        dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(wk.L)]
+        with torch.cuda.stream(wk.main):
+            token_step()
+        dec_all.append(dec_ev)
+    dec_ev = None
+    barrier()
+    dec_ms = [e[0].elapsed_time(e[1]) for ev in dec_all for e in ev]
+    dec_avg = statistics.mean(dec_ms)
+    # algorithmic bytes of one decode step at the mean cache length of those tokens: memory
+    # and local K/V rows read once, the query read, the output written, the token's K/V
+    # appended (read + written)
+    cl_host = [wk.buf[l]["cl"].cpu().numpy() for l in range(wk.L)]
+    mem_rows = statistics.mean(float(c.sum()) for c in cl_host)
+    loc_rows = B * (L0 + (n_ev + 1) / 2.0)
+    row = w.h_kv * w.d * 2
+    step_bytes = ((mem_rows + loc_rows) * 2 * row + 2 * B * w.h_q * w.d * 2 + 4 * B * row)
+    achieved = step_bytes / (dec_avg / 1e3) / 1e9
+    # end to end: each token's per-layer inputs copied from pinned host memory and the last
+    # layer's output read back, per generated token; the request's query inputs as in the
+    # default workload
+    host_tok = [[t.cpu().pin_memory() for t in (x["Q"], x["K"], x["V"])] for x in tok]
+    host_out = tok[-1]["O"].cpu().pin_memory()
+    host_q = [[t.cpu().pin_memory() for t in (wk.layers[l]["Q_r"], wk.layers[l]["Q"])]
+              for l in range(wk.L)]
+    tok_h2d = sum(t.numel() * t.element_size() for hs in host_tok for t in hs)
+    q_h2d = sum(t.numel() * t.element_size() for hs in host_q for t in hs)
+    h2d = q_h2d + G * tok_h2d
+    d2h = G * host_out.numel() * host_out.element_size()
+
+    def e2e_token():
+        for l in range(wk.L):
+            for dst, src in zip((tok[l]["Q"], tok[l]["K"], tok[l]["V"]), host_tok[l]):
+                dst.copy_(src, non_blocking=True)
+        token_step()
+        host_out.copy_(tok[-1]["O"], non_blocking=True)
+
+    def e2e_con():
+        for l in range(wk.L):
+            wk.layers[l]["Q_r"].copy_(host_q[l][0], non_blocking=True)
+            wk.layers[l]["Q"].copy_(host_q[l][1], non_blocking=True)
+        construct()
+
+    e_con = e_tok = None
+    with torch.cuda.stream(wk.main):
+        e2e_con()
+        e2e_token()
+    barrier()
+    if use_graph:
+        e_con, e_tok = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(e_con, stream=wk.main):
+            e2e_con()
+        with torch.cuda.graph(e_tok, stream=wk.main):
+            e2e_token()
+    barrier()
+    Ke = max(1, min(Kst, 3))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(wk.main)
+    with torch.cuda.stream(wk.main):
+        for _ in range(Ke):
+            e_con.replay() if e_con is not None else e2e_con()
+            for _ in range(G):
+                e_tok.replay() if e_tok is not None else e2e_token()
+    e1.record(wk.main)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    if world > 1:
+        t = torch.tensor([req_ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        req_ms, e2e_ms = float(t[0]), float(t[1])
+    unit = "generated tokens/s"
+    value = world * B * G / (req_ms / 1e3)
+    peak, peak_kind = peaks()
+    line = {
+        "metric": "MSA sparse generation tokens/s at the 100M-token bank (context built once per "
+                  "request, routed memory fixed while generating)",
+        "value": round(value, 1), "unit": unit, "n_gpus": world, "steps": Kst,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(req_ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded SplitMix64 normals, planted docs; no dataset)",
+        "config": {"workload": "gen100m", "bank_tokens": w.n_docs * w.doc_len,
+                   "routed_layers": wk.L, "batch": B, "prompt_local_kv": L0,
+                   "generated_tokens_per_query": G, "cache_capacity": cap, "k": w.k,
+                   "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
+                   "kv_bank": f"pinned host memory, fetch={wk.fetch}",
+                   "l2": "no flush: the construction scans 18 x 3.28 GB; a token step reads 18 "
+                         "layers' caches and memory (~40 MB each), 0.7 GB in total, above the "
+                         "126 MB L2",
+                   "cuda_graph": use_graph, "parallelism": f"replicas x{world}"},
+        "construct_ms": round(con_ms, 3), "token_step_ms": round(tok_ms, 4),
+        "roofline": {"kernel": "msa_decode_step (cache append + decode attention + merge)",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": captured_traffic(("attend_dec.cu", "common.cuh"),
+                                                 "attend_dec_gen100m_dram.json"),
+                     "bytes_per_launch": round(step_bytes), "avg_launch_ms": round(dec_avg, 4)},
+        "e2e": {"value": round(world * B * G / (e2e_ms / 1e3), 1), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 3)},
+        # per request: the construction step's kernels + per token and layer append,
+        # attention and merge
+        "gpu_launches": Kst * (wk.L * wk.kernels_per_layer + G * wk.L * 3),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_generate_baseline(w, G, args.cpu_layers)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g_con, g_tok, e_con, e_tok
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def oracle_generate_time(w, layer: int, steps: int) -> float:
+    """Oracle time of ``steps`` generation steps of one routed layer for the whole batch
+    (attention over 128 memory rows + the growing local context)."""
+    import oracle
+    import synth
+    B, L0 = w.B, w.L_loc
+    Kp = synth.normal(w.seed, synth.tag(synth.KLOC, layer), (B, L0, w.h_kv, w.d), "bf16")
+    Vp = synth.normal(w.seed, synth.tag(synth.VLOC, layer), (B, L0, w.h_kv, w.d), "bf16")
+    n_mem = w.k * 8
+    Kb = synth.normal(w.seed, synth.tag(synth.KBAR, layer), (n_mem, w.h_kv, w.d), "bf16")
+    Vb = synth.normal(w.seed, synth.tag(synth.VBAR, layer), (n_mem, w.h_kv, w.d), "bf16")
+    gi = np.tile(np.arange(n_mem, dtype=np.int32), (B, 1))
+    cl = np.full(B, n_mem, np.int32)
+    Qs = [synth.normal(w.seed, synth.tag(synth.GEN_Q, layer, s), (B, 1, w.h_q, w.d), "bf16") for s in range(steps)]
+    Ks = [synth.normal(w.seed, synth.tag(synth.GEN_K, layer, s), (B, 1, w.h_kv, w.d), "bf16")
+          for s in range(steps)]
+    Vs = [synth.normal(w.seed, synth.tag(synth.GEN_V, layer, s), (B, 1, w.h_kv, w.d), "bf16")
+          for s in range(steps)]
+    t0 = time.perf_counter()
+    oracle.generate(Qs, Ks, Vs, Kp, Vp, Kb, Vb, gi, cl, w.k, w.rope_base)
+    return time.perf_counter() - t0
+
+
+def cpu_generate_baseline(w, G: int, n_layers: int) -> dict:
+    import oracle
+    steps = 8
+    per_step = statistics.mean(oracle_generate_time(w, l, steps) / steps for l in range(n_layers))
+    token = per_step * w.layers
+    return {"value": round(w.B / token, 3), "unit": "generated tokens/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{steps} generation steps of {n_layers} of {w.layers} routed layers "
+                       f"(batch {w.B}, 128 memory rows, cache from {w.L_loc} rows); token time = "
+                       f"mean step time x {w.layers}; the construction (routing) is left out, so "
+                       "this overstates the CPU rate")}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -892,6 +1202,8 @@ def main():
         run_interleave(args)
     elif args.workload == "attend_long":
         run_attend_long(args)
+    elif args.workload == "gen100m":
+        run_generate(args)
     else:
         run_libmsa(args)
 

@@ -284,6 +284,45 @@ msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k
                               int64_t L_loc, void* K_out, void* V_out, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* ------------------------------------------------------------------------------------
+ * Sparse generation over an assembled context. Once the routed memory of a layer is fixed
+ * (route -> gather, at context construction), generation proceeds token by token: each new
+ * token's K/V joins the end of the local context and the token attends over
+ * [gathered memory ; local context] with the routed memory unchanged
+ *   [news.neo-ai.one article, "推論パイプライン"; ruixiangma.github.io blog, "三阶段推理流程":
+ *    routing and context assembly are one online stage, autoregressive generation over the
+ *    assembled sparse context the next].
+ * The local context is a caller-owned cache K_cache, V_cache [B, cap, h_kv, d] whose
+ * length len (one int32 in device memory, shared by the batch) is read and advanced by the
+ * kernels, so a captured step (CUDA graph) replays unchanged while the cache grows.
+ */
+
+/* msa_kv_append - rows [len, len + T_new) of every query's cache <- K_new, V_new
+ * [B, T_new, h_kv, d] (K before RoPE, like K_loc); then len += T_new. If len + T_new > cap
+ * on the device, nothing is written, len is unchanged and the workspace status word records
+ * the overflow (msa_workspace_status). ws >= 256 bytes, 256-byte aligned. Fills a prompt
+ * into an empty cache (len = 0) as well as appending generated tokens. */
+msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, int32_t* len_dev,
+                         const void* K_new, const void* V_new, int32_t T_new, int32_t h_kv,
+                         int32_t d, int32_t dtype, void* ws, size_t ws_bytes, void* stream);
+
+/* msa_decode_step - one generation step of one routed layer: msa_kv_append of the step's T
+ * tokens (K_new, V_new [B, T, h_kv, d]) followed by msa_sparse_attend of their queries Q
+ * [B, T, h_q, d] with K_loc, V_loc = the cache's first len rows (len read on the device after
+ * the append; query token t is local row len - T + t at position pos0 + len - T + t).
+ * ctxK, ctxV, ctx_len, max_ctx, pos0, rope_base, scale and O as in msa_sparse_attend.
+ * Supported: bf16, d = 128, h_kv in {1, 2, 4, 8}, (h_q / h_kv) * T <= 8 (else
+ * MSA_ERR_UNSUPPORTED). ws: msa_decode_step_workspace(...) bytes, 256-byte aligned; its
+ * status word records a cache overflow (then O is not written) or an expired device wait. */
+size_t msa_decode_step_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv, int32_t d,
+                                 int32_t max_ctx, int32_t cap);
+msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, int32_t B,
+                           int32_t T, int32_t h_q, void* K_cache, void* V_cache, int32_t cap,
+                           int32_t* len_dev, const void* ctxK, const void* ctxV,
+                           const int32_t* ctx_len, int32_t max_ctx, int32_t h_kv, int32_t d,
+                           int32_t dtype, int32_t pos0, float rope_base, float scale, void* O,
+                           void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,7 +32,8 @@ SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chun
            "msa_route_topk", "msa_route_topk_noalloc",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
-           "msa_sparse_attend", "msa_assemble_local")
+           "msa_sparse_attend", "msa_assemble_local", "msa_kv_append",
+           "msa_decode_step_workspace", "msa_decode_step")
 
 
 class MSAError(RuntimeError):
@@ -91,6 +92,13 @@ def _load():
     L.msa_assemble_local.restype = ctypes.c_int
     L.msa_assemble_local.argtypes = [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, vp, vp,
                                      vp, sz, vp]
+    L.msa_kv_append.restype = ctypes.c_int
+    L.msa_kv_append.argtypes = [vp, vp, i32, i32, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
+    L.msa_decode_step_workspace.restype = sz
+    L.msa_decode_step_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    L.msa_decode_step.restype = ctypes.c_int
+    L.msa_decode_step.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32, i32,
+                                  i32, i32, i32, f32, f32, vp, vp, sz, vp]
     return L
 
 
@@ -191,6 +199,30 @@ def msa_assemble_local(seg_k_ptrs, seg_v_ptrs, seg_len, K_q, V_q, K_out, V_out, 
     _check(lib.msa_assemble_local(B, n_seg, _p(seg_k_ptrs), _p(seg_v_ptrs), _p(seg_len), _p(K_q),
                                   _p(V_q), T, h_kv, d, dtype_code(K_q), K_out.shape[1], _p(K_out),
                                   _p(V_out), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_kv_append(K_cache, V_cache, length, K_new, V_new, ws, stream=None):
+    """K_cache, V_cache: [B, cap, h_kv, d]; length: int32 device tensor of one element;
+    K_new, V_new: [B, T_new, h_kv, d]."""
+    B, cap, h_kv, d = K_cache.shape
+    _check(lib.msa_kv_append(_p(K_cache), _p(V_cache), B, cap, _p(length), _p(K_new), _p(V_new),
+                             K_new.shape[1], h_kv, d, dtype_code(K_cache), _p(ws),
+                             ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_decode_step_workspace(B, T, h_q, h_kv, d, max_ctx, cap) -> int:
+    return int(lib.msa_decode_step_workspace(B, T, h_q, h_kv, d, max_ctx, cap))
+
+
+def msa_decode_step(Q, K_new, V_new, K_cache, V_cache, length, ctxK, ctxV, ctx_len, pos0,
+                    rope_base, scale, O, ws, stream=None):
+    """One generation step of one routed layer (append, then attend over the cache)."""
+    B, T, h_q, d = Q.shape
+    cap, h_kv = K_cache.shape[1], K_cache.shape[2]
+    _check(lib.msa_decode_step(_p(Q), _p(K_new), _p(V_new), B, T, h_q, _p(K_cache), _p(V_cache),
+                               cap, _p(length), _p(ctxK), _p(ctxV), _p(ctx_len), ctxK.shape[1],
+                               h_kv, d, dtype_code(Q), pos0, rope_base, scale, _p(O), _p(ws),
+                               ws.numel() * ws.element_size(), _s(stream)))
 
 
 def msa_gather(top_ids, doc_chunk_off, Kbar, Vbar, max_ctx, gather_idx, ctx_len, ctxK, ctxV, ws,
@@ -331,3 +363,36 @@ class Fetcher:
             self.close()
         except Exception:
             pass
+
+
+class LocalCache:
+    """Preallocated local K/V of sparse generation: [B, cap, h_kv, d] plus its length, one
+    int32 in device memory that msa_kv_append / msa_decode_step read and advance."""
+
+    def __init__(self, B: int, cap: int, h_kv: int, d: int, dtype=torch.bfloat16, device="cuda",
+                 length=None):
+        self.K = torch.empty((B, cap, h_kv, d), dtype=dtype, device=device)
+        self.V = torch.empty_like(self.K)
+        # ``length``: an int32 device tensor of one element to use (e.g. a view of one array
+        # holding the lengths of several layers' caches); a new zero otherwise
+        self.length = (torch.zeros(1, dtype=torch.int32, device=device) if length is None
+                       else length)
+        self.ws = _ws(256, device)
+
+    def append(self, K_new, V_new, stream=None):
+        msa_kv_append(self.K, self.V, self.length, K_new, V_new, self.ws, stream)
+
+
+def decode_step(cache: LocalCache, Q, K_new, V_new, ctxK, ctxV, ctx_len, pos0: int,
+                rope_base: float, scale: float = 0.0, O=None, ws=None, stream=None):
+    """Append the step's tokens to ``cache`` and attend; returns O [B, T, h_q, d]."""
+    B, T, h_q, d = Q.shape
+    if ws is None:
+        ws = _ws(msa_decode_step_workspace(B, T, h_q, cache.K.shape[2], d, ctxK.shape[1],
+                                           cache.K.shape[1]), Q.device)
+    if O is None:
+        O = torch.empty_like(Q)
+    msa_decode_step(Q, K_new, V_new, cache.K, cache.V, cache.length, ctxK, ctxV, ctx_len, pos0,
+                    rope_base, scale, O, ws, stream)
+    return O
+

@@ -561,6 +561,8 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       q.h_q = h_q;
       q.h_kv = h_kv;
       q.L = L_loc;
+      q.Ls = L_loc;
+      q.L_dev = nullptr;
       q.max_ctx = max_ctx;
       q.rope = rope_base > 0.f ? 1 : 0;
       q.pos0 = pos0;
@@ -687,6 +689,127 @@ msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k
   cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
   if (e == cudaSuccess) e = msa::launch_assemble_local(p, st);
   if (e != cudaSuccess) return cuda_fail(e, "msa_assemble_local launch");
+  return ok();
+}
+
+
+// ------------------------------------------------------------------------ sparse generation
+msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, int32_t* len_dev,
+                         const void* K_new, const void* V_new, int32_t T_new, int32_t h_kv,
+                         int32_t d, int32_t dtype, void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && cap >= 1 && T_new >= 0, MSA_ERR_INVALID_ARG, "bad sizes (B=%d cap=%d T_new=%d)",
+          B, cap, T_new);
+  REQUIRE(T_new <= cap, MSA_ERR_INVALID_ARG, "T_new %d exceeds the capacity %d", T_new, cap);
+  REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "append needs a 256-byte aligned workspace of >= 256 bytes");
+  if (B == 0 || T_new == 0) return ok();
+  REQUIRE(K_cache && V_cache && len_dev && K_new && V_new, MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(aligned16(K_cache) && aligned16(V_cache) && aligned16(K_new) && aligned16(V_new),
+          MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  msa::AppendParams p{};
+  p.B = B;
+  p.T_new = T_new;
+  p.cap = cap;
+  p.row_bytes = (int64_t)h_kv * d * (int64_t)esize(dtype);
+  p.K_cache = K_cache;
+  p.V_cache = V_cache;
+  p.K_new = K_new;
+  p.V_new = V_new;
+  p.len = len_dev;
+  p.err = static_cast<int*>(ws);
+  p.ticket = reinterpret_cast<unsigned int*>(static_cast<unsigned char*>(ws) + 4);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), st);  // status word, ticket
+  if (e == cudaSuccess) e = msa::launch_kv_append(p, sm_count(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_kv_append launch");
+  return ok();
+}
+
+size_t msa_decode_step_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv, int32_t d,
+                                 int32_t max_ctx, int32_t cap) {
+  if (B < 1 || T < 1 || h_kv < 1 || h_q % h_kv != 0 || max_ctx < 0 || cap < T) return kHeader;
+  const msa::DecPlan dp = msa::attend_dec_plan_cap(B, T, h_q, h_kv, d, max_ctx, cap, sm_count());
+  if (!dp.ok) return kHeader;
+  return kHeader + dp.ctr_bytes + dp.part_ml_bytes + dp.part_o_bytes;
+}
+
+msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, int32_t B,
+                           int32_t T, int32_t h_q, void* K_cache, void* V_cache, int32_t cap,
+                           int32_t* len_dev, const void* ctxK, const void* ctxV,
+                           const int32_t* ctx_len, int32_t max_ctx, int32_t h_kv, int32_t d,
+                           int32_t dtype, int32_t pos0, float rope_base, float scale, void* O,
+                           void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && T >= 1 && cap >= T && max_ctx >= 0, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d T=%d cap=%d max_ctx=%d)", B, T, cap, max_ctx);
+  REQUIRE(h_q >= h_kv && h_q % h_kv == 0, MSA_ERR_INVALID_ARG, "h_q %d not a multiple of h_kv %d",
+          h_q, h_kv);
+  REQUIRE(pos0 >= 0, MSA_ERR_INVALID_ARG, "pos0 %d", pos0);
+  const msa::DecPlan dp = msa::attend_dec_plan_cap(B, T, h_q, h_kv, d, max_ctx, cap, sm_count());
+  REQUIRE(dtype == MSA_BF16 && dp.ok, MSA_ERR_UNSUPPORTED,
+          "decode step: bf16, d = 128, h_kv in {1, 2, 4, 8}, (h_q / h_kv) * T <= 8");
+  const size_t need = kHeader + dp.ctr_bytes + dp.part_ml_bytes + dp.part_o_bytes;
+  REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+  if (B == 0) return ok();
+  REQUIRE(Q && K_new && V_new && K_cache && V_cache && len_dev && ctx_len && O,
+          MSA_ERR_INVALID_ARG, "null tensor");
+  REQUIRE(max_ctx == 0 || (ctxK && ctxV), MSA_ERR_INVALID_ARG, "null context");
+  REQUIRE(aligned16(Q) && aligned16(K_new) && aligned16(V_new) && aligned16(K_cache) &&
+              aligned16(V_cache) && (max_ctx == 0 || (aligned16(ctxK) && aligned16(ctxV))),
+          MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  unsigned char* w8 = static_cast<unsigned char*>(ws);
+  cudaStream_t st = (cudaStream_t)stream;
+  // status word, append ticket and the reserved counters start at zero
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHeader + dp.ctr_bytes, st);
+  msa::AppendParams a{};
+  a.B = B;
+  a.T_new = T;
+  a.cap = cap;
+  a.row_bytes = (int64_t)h_kv * d * 2;
+  a.K_cache = K_cache;
+  a.V_cache = V_cache;
+  a.K_new = K_new;
+  a.V_new = V_new;
+  a.len = len_dev;
+  a.err = reinterpret_cast<int*>(w8);
+  a.ticket = reinterpret_cast<unsigned int*>(w8 + 4);
+  if (e == cudaSuccess) e = msa::launch_kv_append(a, sm_count(), st);
+  msa::DecParams q{};
+  q.Q = static_cast<const __nv_bfloat16*>(Q);
+  q.Kl = static_cast<const __nv_bfloat16*>(K_cache);
+  q.Vl = static_cast<const __nv_bfloat16*>(V_cache);
+  q.cK = static_cast<const __nv_bfloat16*>(ctxK);
+  q.cV = static_cast<const __nv_bfloat16*>(ctxV);
+  q.ctx_len = ctx_len;
+  q.B = B;
+  q.T = T;
+  q.h_q = h_q;
+  q.h_kv = h_kv;
+  q.L = cap;
+  q.Ls = cap;
+  q.L_dev = len_dev;
+  q.skip_on_err = 1;  // an overflowing append leaves O unwritten
+  q.max_ctx = max_ctx;
+  q.rope = rope_base > 0.f ? 1 : 0;
+  q.pos0 = pos0;
+  msa::rope_turns(q.rope ? (double)rope_base : 0.0, 128, q.rope_turns);
+  q.scale_log2 = (scale > 0.f ? scale : 1.0f / sqrtf((float)d)) * 1.4426950408889634f;
+  q.TPP = dp.TPP;
+  q.CT = dp.CT;
+  q.max_seg = dp.max_seg;
+  q.total = dp.total;
+  q.grid = dp.grid;
+  q.err = reinterpret_cast<int*>(w8);
+  q.counters = reinterpret_cast<unsigned int*>(w8 + kHeader);
+  q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);
+  q.part_o = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes + dp.part_ml_bytes);
+  q.O = static_cast<__nv_bfloat16*>(O);
+  if (e == cudaSuccess) e = msa::launch_attend_dec(q, dp, st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_decode_step launch");
   return ok();
 }
 

@@ -89,16 +89,28 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
   uint64_t* full = reinterpret_cast<uint64_t*>(wscr + kDecCW * WS);           // [NS]
   uint64_t* empty = full + NS;                                                // [NS]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  __shared__ int skip_call;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int HKV = p.h_kv;
   const int KT = kDecRowsPerTile / HKV;  // key rows per tile
   const int Gq = p.h_q / HKV;
   const int nr = Gq * p.T;  // query rows per KV head (<= RB)
-  const int64_t G = gridDim.x, ci = blockIdx.x;
-  const int64_t x0 = ci * p.total / G, x1 = (ci + 1) * p.total / G;
+  // local rows per query: fixed, or read from the device (a cache that grows between launches)
+  const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
+  if (L < p.T || L > p.Ls) {  // uniform over the grid: nothing is read or written
+    if (blockIdx.x == 0 && tid == 0) set_err(p.err, kErrBadIndex);
+    return;
+  }
+  const int TPP = p.CT + (L + KT - 1) / KT;  // tiles per query
+  const int64_t total = (int64_t)p.B * TPP;
+  // tile ranges: one per CTA, at most one per tile (a grid planned for a longer context
+  // leaves its surplus CTAs idle, so every range a query spans is non-empty)
+  const int64_t G = min((int64_t)gridDim.x, total), ci = blockIdx.x;
+  if (ci >= G) return;
+  const int64_t x0 = ci * total / G, x1 = (ci + 1) * total / G;
   const int n_tiles = (int)(x1 - x0);
-  const int b_first = (int)(x0 / p.TPP), tt_first = (int)(x0 % p.TPP);
+  const int b_first = (int)(x0 / TPP), tt_first = (int)(x0 % TPP);
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
@@ -106,10 +118,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
       mbar_init(&empty[s], kDecCW);
     }
     *abort_flag = 0;
+    // an error an earlier kernel of the same call recorded (a failed append) skips the call
+    skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
     fence_mbar_init();
   }
   if (tid < HALF) turns[tid] = p.rope_turns[tid];
   __syncthreads();
+  if (skip_call) return;  // written once before the barrier: one value for the whole CTA
 
   if (warp == kDecCW) {
     // ---------------- copy warp (lane 0): tile u -> stage u % NS
@@ -141,8 +156,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
           vs = p.cV + off;
         } else {  // local rows [KT i, KT i + KT)
           const int j0 = (tt - p.CT) * KT;
-          nk = min(p.L - j0, KT);
-          const int64_t off = ((int64_t)b * p.L + j0) * row_elems;
+          nk = min(L - j0, KT);
+          const int64_t off = ((int64_t)b * p.Ls + j0) * row_elems;
           ks = p.Kl + off;
           vs = p.Vl + off;
         }
@@ -153,7 +168,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
           bulk_g2s(st, ks, bytes, &full[s]);
           bulk_g2s(st + kDecHalf, vs, bytes, &full[s]);
         }
-        if (++tt == p.TPP) {
+        if (++tt == TPP) {
           tt = 0;
           ++b;
         }
@@ -205,8 +220,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
       *reinterpret_cast<float4*>(comb + (warp * RB + r) * D + 4 * lane) =
           make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
     const bool write = !named_sync_compute_or(*abort_flag != 0);  // one decision for all warps
-    const int64_t first = dec_cta_of((int64_t)fb * p.TPP, G, p.total);
-    const int64_t last = dec_cta_of((int64_t)fb * p.TPP + p.TPP - 1, G, p.total);
+    const int64_t first = dec_cta_of((int64_t)fb * TPP, G, total);
+    const int64_t last = dec_cta_of((int64_t)fb * TPP + TPP - 1, G, total);
     const int n_seg = (int)(last - first + 1);
     const int seg = (int)(ci - first);
     const int n_out = HKV * nr * D;
@@ -256,7 +271,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
         if (r < nr) {
           const int t = r / Gq, h = g * Gq + r % Gq;
           const __nv_bfloat16* q = p.Q + (((int64_t)b * p.T + t) * p.h_q + h) * D;
-          const int64_t pos = (int64_t)p.pos0 + p.L - p.T + t;
+          const int64_t pos = (int64_t)p.pos0 + L - p.T + t;
 #pragma unroll
           for (int m = 0; m < PPL; ++m) {
             const float a = __bfloat162float(q[i0 + m]), c = __bfloat162float(q[i0 + m + HALF]);
@@ -279,7 +294,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
       }
       __syncwarp();
     }
-    const int nk = is_ctx ? min(max(n_ctx - kt, 0), KT) : min(p.L - kt, KT);
+    const int nk = is_ctx ? min(max(n_ctx - kt, 0), KT) : min(L - kt, KT);
     if (!is_ctx && !qa_ok) {  // the query turned back by the tile's start position P
       const int64_t P = (int64_t)p.pos0 + kt;
 #pragma unroll
@@ -369,7 +384,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
       for (int e = 0; e < PER; ++e) {
         const int r = (dl * PER + e) % RB;
         const int t = r / Gq;
-        const bool vis = 8 * sl + kk < nk && r < nr && (is_ctx || jrow <= p.L - p.T + t);
+        const bool vis = 8 * sl + kk < nk && r < nr && (is_ctx || jrow <= L - p.T + t);
         float x = vis ? v[e] : -INFINITY;
         float mx = x;
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -445,7 +460,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
         }
       }
     }
-    if (++tt == p.TPP) {
+    if (++tt == TPP) {
       tt = 0;
       ++b;
     }
@@ -464,9 +479,14 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecP
   const int h = row % p.h_q, t = (row / p.h_q) % p.T, b = row / (p.h_q * p.T);
   const int gh = h / Gq, r = t * Gq + h % Gq;
   const int RB = (Gq * p.T) <= 4 ? 4 : 8;
-  const int64_t G = p.grid, total = p.total;
-  const int64_t first = dec_cta_of((int64_t)b * p.TPP, G, total);
-  const int64_t last = dec_cta_of((int64_t)b * p.TPP + p.TPP - 1, G, total);
+  const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
+  if (L < p.T || L > p.Ls) return;  // reported by the attention kernel
+  if (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) return;
+  const int KT = kDecRowsPerTile / HKV;
+  const int TPP = p.CT + (L + KT - 1) / KT;
+  const int64_t total = (int64_t)p.B * TPP, G = min((int64_t)p.grid, total);
+  const int64_t first = dec_cta_of((int64_t)b * TPP, G, total);
+  const int64_t last = dec_cta_of((int64_t)b * TPP + TPP - 1, G, total);
   const int n_seg = (int)(last - first + 1);
   if (n_seg == 1) return;  // written directly by the attention kernel
   __shared__ float sm_l[kMergeWarps];
@@ -540,6 +560,22 @@ DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int
   pl.smem = 1024 + (size_t)kDecStages * kDecStage + (size_t)64 * 32 * 16 + (kDecD / 2) * 8 +
             sizeof(float) * ((size_t)kDecCW * pl.RB * kDecD + (size_t)kDecCW * 11 * pl.RB) +
             2 * kDecStages * 8 + 16;
+  return pl;
+}
+
+// Plan for a local length known only on the device (1 <= T <= L <= cap): the grid is fixed
+// and the kernel cuts the tile list for the live length. A query's TPP tiles out of B * TPP
+// meet fewer than G / B + 2 of the G tile ranges, so ceil(G / B) + 1 partial slots suffice.
+DecPlan attend_dec_plan_cap(int B, int T, int h_q, int h_kv, int d, int max_ctx, int cap,
+                            int sms) {
+  DecPlan pl = attend_dec_plan(B, T, h_q, h_kv, d, max_ctx, cap, sms);
+  if (!pl.ok) return pl;
+  pl.grid = sms;
+  const int max_seg = std::min<int64_t>(sms, (sms + B - 1) / B + 1);
+  pl.max_seg = max_seg;
+  const size_t slots = (size_t)B * max_seg * h_kv * pl.RB;
+  pl.part_ml_bytes = (slots * 2 * sizeof(float) + 255) & ~(size_t)255;
+  pl.part_o_bytes = (slots * kDecD * sizeof(float) + 255) & ~(size_t)255;
   return pl;
 }
 

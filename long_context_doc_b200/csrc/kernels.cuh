@@ -138,18 +138,22 @@ bool encode_bf16_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* 
 // h_kv in {1, 2, 4, 8})
 struct DecParams {
   const __nv_bfloat16* Q;   // [B, T, h_q, 128]
-  const __nv_bfloat16* Kl;  // [B, L, h_kv, 128]
+  const __nv_bfloat16* Kl;  // [B, Ls, h_kv, 128], the first L rows of each query used
   const __nv_bfloat16* Vl;
   const __nv_bfloat16* cK;  // [B, max_ctx, h_kv, 128]
   const __nv_bfloat16* cV;
   const int32_t* ctx_len;
   int B, T, h_q, h_kv, L, max_ctx;
+  int Ls;                   // local rows stored per query (row stride of Kl / Vl), >= L
+  const int32_t* L_dev;     // nullable: the local length is read from here at run time
+  int skip_on_err;          // write nothing if the status word already holds an error
   int rope, pos0;
   unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions,
                                       // theta_i = base^(-2i/128); all zero without RoPE
   float scale_log2;
   int TPP, CT, max_seg;     // tiles of 64/h_kv key rows per query, of which the first CT hold
-                            // memory rows and the rest local rows; segments per query
+                            // memory rows and the rest local rows; segments per query (the
+                            // kernels recompute TPP from the live length)
   int64_t total;            // B * TPP
   int grid;                 // CTAs of the attention kernel (tile ranges)
   float* part_o;            // [B, max_seg, h_kv, RB, 128]
@@ -165,6 +169,7 @@ struct DecPlan {
   size_t ctr_bytes, part_ml_bytes, part_o_bytes, smem;
 };
 DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
+DecPlan attend_dec_plan_cap(int B, int T, int h_q, int h_kv, int d, int max_ctx, int cap, int sms);
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
 
 // ---- assemble.cu: local context of a Memory Interleaving round
@@ -181,6 +186,21 @@ struct AssembleParams {
   void* V_out;
   int* err;                   // workspace status word
 };
+// Sparse generation: rows [len, len + T_new) of every query's local cache <- the new tokens'
+// K/V, then len += T_new (len read on the device)
+struct AppendParams {
+  int B, T_new, cap;
+  int64_t row_bytes;          // h_kv * d * element size, a multiple of 16
+  void* K_cache;              // [B, cap, h_kv, d]
+  void* V_cache;
+  const void* K_new;          // [B, T_new, h_kv, d]
+  const void* V_new;
+  int32_t* len;               // device, the rows the cache holds (shared by the batch)
+  int* err;                   // workspace status word
+  unsigned int* ticket;       // zero on entry; the last CTA advances len and resets it
+};
+cudaError_t launch_kv_append(const AppendParams& p, int sms, cudaStream_t st);
+
 cudaError_t launch_assemble_local(const AssembleParams& p, cudaStream_t st);
 
 // ---- attend_tc.cu: long-query attention on tensor cores (bf16, d = 128, (h_q/h_kv) * T >= 64,

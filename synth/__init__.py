@@ -30,6 +30,7 @@ _SO_DEV = os.path.join(_HERE, "libsynth_dev.so")
 # tensor ids used in generator tags
 K, V, KR, Q, QR, KLOC, VLOC, KBAR, VBAR, KRBAR, APPK, APPV = range(1, 13)
 PLANT_DOCS, PLANT_EPS, DOC_LEN, EXTRA = 20, 21, 22, 23
+GEN_Q, GEN_K, GEN_V = 30, 31, 32  # a generated token's query and K/V
 
 
 def tag(tid: int, layer: int = 0, sub: int = 0) -> int:

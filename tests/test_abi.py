@@ -142,3 +142,31 @@ def test_assemble_local_rejects_bad_arguments_on_host(msa):
     r = msa.lib.msa_assemble_local(2, 3, fake, fake, fake, fake, fake, 4, 8, 128, 1, 10, None, fake,
                                    ws, 256, None)
     assert r == 1
+
+
+def test_generation_entry_points_reject_bad_arguments_on_host(msa):
+    fake = ctypes.c_void_p(256)
+    ws = ctypes.c_void_p(512)
+    # kv_append: more new rows than the cache holds, no workspace, missing length, misaligned
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 9, 8, 128, 1, ws, 256, None)
+    assert r == 1
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 1, 8, 128, 1, None, 0, None)
+    assert r == 3
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, None, fake, fake, 1, 8, 128, 1, ws, 256, None)
+    assert r == 1
+    r = msa.lib.msa_kv_append(fake, ctypes.c_void_p(264), 2, 8, fake, fake, fake, 1, 8, 128, 1,
+                              ws, 256, None)
+    assert r == 1
+    need = msa.msa_decode_step_workspace(4, 1, 32, 8, 128, 128, 4096)
+    assert need > 256
+
+    def step(dtype=1, h_q=32, h_kv=8, d=128, T=1, cap=4096, ws_bytes=need, L=fake):
+        return msa.lib.msa_decode_step(fake, fake, fake, 4, T, h_q, fake, fake, cap, L, fake,
+                                       fake, fake, 128, h_kv, d, dtype, 16, 1e6, 0.0, fake, ws,
+                                       ws_bytes, None)
+    assert step(dtype=0) == 2           # fp32: no decode kernel
+    assert step(T=3) == 2               # 12 query rows per KV head
+    assert step(h_kv=3, h_q=30) == 2    # 3 KV heads
+    assert step(cap=0) == 1             # capacity below T
+    assert step(ws_bytes=need - 1) == 3
+    assert step(L=None) == 1            # no device length
