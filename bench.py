@@ -944,7 +944,8 @@ def run_generate(args):
     caches, tok = [], []
     ws_bytes = msa.msa_decode_step_workspace(B, 1, w.h_q, w.h_kv, w.d, wk.max_ctx, cap)
     for l in range(wk.L):
-        c = msa.LocalCache(B, cap, w.h_kv, w.d, device=dev, length=lens[l:l + 1])
+        c = msa.LocalCache(B, cap, w.h_kv, w.d, pos0=w.k, rope_base=w.rope_base, device=dev,
+                           length=lens[l:l + 1])
         c.append(wk.layers[l]["K_loc"], wk.layers[l]["V_loc"])  # the prompt's local K/V
         caches.append(c)
         # the generated token's query and K/V at this layer (synthetic, reused every step)

@@ -294,23 +294,31 @@ msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k
  *    assembled sparse context the next].
  * The local context is a caller-owned cache K_cache, V_cache [B, cap, h_kv, d] whose
  * length len (one int32 in device memory, shared by the batch) is read and advanced by the
- * kernels, so a captured step (CUDA graph) replays unchanged while the cache grows.
+ * kernels, so a captured step (CUDA graph) replays unchanged while the cache grows. Cache
+ * row j holds its key already rotated at its global position pos0 + j (global RoPE of the
+ * active context, applied once when the row is appended), so attention over the cache
+ * rotates only the query.
  */
 
 /* msa_kv_append - rows [len, len + T_new) of every query's cache <- K_new, V_new
- * [B, T_new, h_kv, d] (K before RoPE, like K_loc); then len += T_new. If len + T_new > cap
- * on the device, nothing is written, len is unchanged and the workspace status word records
- * the overflow (msa_workspace_status). ws >= 256 bytes, 256-byte aligned. Fills a prompt
- * into an empty cache (len = 0) as well as appending generated tokens. */
+ * [B, T_new, h_kv, d] (K before RoPE, like K_loc); row j's key is stored rotated at
+ * position pos0 + j with base rope_base (rope_base <= 0: stored as given); then
+ * len += T_new. If len + T_new > cap on the device, nothing is written, len is unchanged and
+ * the workspace status word records the overflow (msa_workspace_status). ws >= 256 bytes,
+ * 256-byte aligned. Fills a prompt into an empty cache (len = 0) as well as appending
+ * generated tokens. */
 msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, int32_t* len_dev,
                          const void* K_new, const void* V_new, int32_t T_new, int32_t h_kv,
-                         int32_t d, int32_t dtype, void* ws, size_t ws_bytes, void* stream);
+                         int32_t d, int32_t dtype, int32_t pos0, float rope_base, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /* msa_decode_step - one generation step of one routed layer: msa_kv_append of the step's T
- * tokens (K_new, V_new [B, T, h_kv, d]) followed by msa_sparse_attend of their queries Q
- * [B, T, h_q, d] with K_loc, V_loc = the cache's first len rows (len read on the device after
- * the append; query token t is local row len - T + t at position pos0 + len - T + t).
- * ctxK, ctxV, ctx_len, max_ctx, pos0, rope_base, scale and O as in msa_sparse_attend.
+ * tokens (K_new, V_new [B, T, h_kv, d], pre-RoPE) followed by msa_sparse_attend of their
+ * queries Q [B, T, h_q, d] with K_loc, V_loc = the cache's first len rows (len read on the
+ * device after the append; query token t is local row len - T + t at position
+ * pos0 + len - T + t). The cache must have been filled with the same pos0 and rope_base
+ * (its keys are stored rotated). ctxK, ctxV, ctx_len, max_ctx, pos0, rope_base, scale and O
+ * as in msa_sparse_attend.
  * Supported: bf16, d = 128, h_kv in {1, 2, 4, 8}, (h_q / h_kv) * T <= 8 (else
  * MSA_ERR_UNSUPPORTED). ws: msa_decode_step_workspace(...) bytes, 256-byte aligned; its
  * status word records a cache overflow (then O is not written) or an expired device wait. */

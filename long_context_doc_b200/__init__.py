@@ -93,7 +93,8 @@ def _load():
     L.msa_assemble_local.argtypes = [i32, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i64, vp, vp,
                                      vp, sz, vp]
     L.msa_kv_append.restype = ctypes.c_int
-    L.msa_kv_append.argtypes = [vp, vp, i32, i32, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
+    L.msa_kv_append.argtypes = [vp, vp, i32, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, sz,
+                                vp]
     L.msa_decode_step_workspace.restype = sz
     L.msa_decode_step_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     L.msa_decode_step.restype = ctypes.c_int
@@ -201,13 +202,13 @@ def msa_assemble_local(seg_k_ptrs, seg_v_ptrs, seg_len, K_q, V_q, K_out, V_out, 
                                   _p(V_out), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
-def msa_kv_append(K_cache, V_cache, length, K_new, V_new, ws, stream=None):
+def msa_kv_append(K_cache, V_cache, length, K_new, V_new, pos0, rope_base, ws, stream=None):
     """K_cache, V_cache: [B, cap, h_kv, d]; length: int32 device tensor of one element;
-    K_new, V_new: [B, T_new, h_kv, d]."""
+    K_new, V_new: [B, T_new, h_kv, d] (keys stored rotated at pos0 + row when rope_base > 0)."""
     B, cap, h_kv, d = K_cache.shape
     _check(lib.msa_kv_append(_p(K_cache), _p(V_cache), B, cap, _p(length), _p(K_new), _p(V_new),
-                             K_new.shape[1], h_kv, d, dtype_code(K_cache), _p(ws),
-                             ws.numel() * ws.element_size(), _s(stream)))
+                             K_new.shape[1], h_kv, d, dtype_code(K_cache), pos0, rope_base,
+                             _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
 def msa_decode_step_workspace(B, T, h_q, h_kv, d, max_ctx, cap) -> int:
@@ -367,10 +368,12 @@ class Fetcher:
 
 class LocalCache:
     """Preallocated local K/V of sparse generation: [B, cap, h_kv, d] plus its length, one
-    int32 in device memory that msa_kv_append / msa_decode_step read and advance."""
+    int32 in device memory that msa_kv_append / msa_decode_step read and advance. Keys are
+    stored rotated at their global positions pos0 + row (RoPE base ``rope_base``)."""
 
-    def __init__(self, B: int, cap: int, h_kv: int, d: int, dtype=torch.bfloat16, device="cuda",
-                 length=None):
+    def __init__(self, B: int, cap: int, h_kv: int, d: int, pos0: int = 0,
+                 rope_base: float = 0.0, dtype=torch.bfloat16, device="cuda", length=None):
+        self.pos0, self.rope_base = int(pos0), float(rope_base)
         self.K = torch.empty((B, cap, h_kv, d), dtype=dtype, device=device)
         self.V = torch.empty_like(self.K)
         # ``length``: an int32 device tensor of one element to use (e.g. a view of one array
@@ -380,13 +383,16 @@ class LocalCache:
         self.ws = _ws(256, device)
 
     def append(self, K_new, V_new, stream=None):
-        msa_kv_append(self.K, self.V, self.length, K_new, V_new, self.ws, stream)
+        msa_kv_append(self.K, self.V, self.length, K_new, V_new, self.pos0, self.rope_base,
+                      self.ws, stream)
 
 
-def decode_step(cache: LocalCache, Q, K_new, V_new, ctxK, ctxV, ctx_len, pos0: int,
-                rope_base: float, scale: float = 0.0, O=None, ws=None, stream=None):
-    """Append the step's tokens to ``cache`` and attend; returns O [B, T, h_q, d]."""
+def decode_step(cache: LocalCache, Q, K_new, V_new, ctxK, ctxV, ctx_len, scale: float = 0.0,
+                O=None, ws=None, stream=None):
+    """Append the step's tokens to ``cache`` and attend (global RoPE with the cache's pos0 and
+    base); returns O [B, T, h_q, d]."""
     B, T, h_q, d = Q.shape
+    pos0, rope_base = cache.pos0, cache.rope_base
     if ws is None:
         ws = _ws(msa_decode_step_workspace(B, T, h_q, cache.K.shape[2], d, ctxK.shape[1],
                                            cache.K.shape[1]), Q.device)

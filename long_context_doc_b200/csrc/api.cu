@@ -696,12 +696,14 @@ msa_status msa_assemble_local(int32_t B, int32_t n_seg, const void* const* seg_k
 // ------------------------------------------------------------------------ sparse generation
 msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, int32_t* len_dev,
                          const void* K_new, const void* V_new, int32_t T_new, int32_t h_kv,
-                         int32_t d, int32_t dtype, void* ws, size_t ws_bytes, void* stream) {
+                         int32_t d, int32_t dtype, int32_t pos0, float rope_base, void* ws,
+                         size_t ws_bytes, void* stream) {
   msa_status s = check_common(h_kv, d, dtype);
   if (s != MSA_OK) return s;
   REQUIRE(B >= 0 && cap >= 1 && T_new >= 0, MSA_ERR_INVALID_ARG, "bad sizes (B=%d cap=%d T_new=%d)",
           B, cap, T_new);
   REQUIRE(T_new <= cap, MSA_ERR_INVALID_ARG, "T_new %d exceeds the capacity %d", T_new, cap);
+  REQUIRE(pos0 >= 0, MSA_ERR_INVALID_ARG, "pos0 %d", pos0);
   REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
           MSA_ERR_WORKSPACE, "append needs a 256-byte aligned workspace of >= 256 bytes");
   if (B == 0 || T_new == 0) return ok();
@@ -720,6 +722,11 @@ msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, i
   p.len = len_dev;
   p.err = static_cast<int*>(ws);
   p.ticket = reinterpret_cast<unsigned int*>(static_cast<unsigned char*>(ws) + 4);
+  p.rope = rope_base > 0.f ? 1 : 0;
+  p.pos0 = pos0;
+  p.d = d;
+  p.esize = (int)esize(dtype);
+  msa::rope_turns(p.rope ? (double)rope_base : 0.0, d, p.rope_turns);
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(int32_t), st);  // status word, ticket
   if (e == cudaSuccess) e = msa::launch_kv_append(p, sm_count(), st);
@@ -763,8 +770,8 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
           MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   unsigned char* w8 = static_cast<unsigned char*>(ws);
   cudaStream_t st = (cudaStream_t)stream;
-  // status word, append ticket and the reserved counters start at zero
-  cudaError_t e = cudaMemsetAsync(ws, 0, kHeader + dp.ctr_bytes, st);
+  // the append runs as one CTA and starts the status word (no memset node per step)
+  cudaError_t e = cudaSuccess;
   msa::AppendParams a{};
   a.B = B;
   a.T_new = T;
@@ -777,6 +784,12 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
   a.len = len_dev;
   a.err = reinterpret_cast<int*>(w8);
   a.ticket = reinterpret_cast<unsigned int*>(w8 + 4);
+  a.single = 1;
+  a.rope = rope_base > 0.f ? 1 : 0;  // the cache holds keys rotated at pos0 + row
+  a.pos0 = pos0;
+  a.d = d;
+  a.esize = 2;
+  msa::rope_turns(a.rope ? (double)rope_base : 0.0, d, a.rope_turns);
   if (e == cudaSuccess) e = msa::launch_kv_append(a, sm_count(), st);
   msa::DecParams q{};
   q.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -792,7 +805,8 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
   q.L = cap;
   q.Ls = cap;
   q.L_dev = len_dev;
-  q.skip_on_err = 1;  // an overflowing append leaves O unwritten
+  q.skip_on_err = 1;   // an overflowing append leaves O unwritten
+  q.keys_rotated = 1;  // the append stored the keys rotated
   q.max_ctx = max_ctx;
   q.rope = rope_base > 0.f ? 1 : 0;
   q.pos0 = pos0;

@@ -20,6 +20,7 @@
 namespace msa {
 
 constexpr int kAsmRows = 16;
+constexpr int kAppendTab = 8;  // appends of at most this many rows per query use a RoPE table
 constexpr int kAsmMaxSeg = 1024;
 
 __global__ void __launch_bounds__(256) assemble_local_kernel(AssembleParams p) {
@@ -76,25 +77,92 @@ __global__ void __launch_bounds__(256) assemble_local_kernel(AssembleParams p) {
 // kErrCtxOverflow and leaves cache and length unchanged.
 __global__ void __launch_bounds__(256) kv_append_kernel(AppendParams p) {
   __shared__ int len_s;
+  __shared__ unsigned long long turns[64];
+  __shared__ float2 rtab[kAppendTab * 64];  // (cos, sin) per (new row t, pair i) for short appends
   if (threadIdx.x == 0) len_s = *reinterpret_cast<volatile int32_t*>(p.len);
+  if (threadIdx.x < p.d / 2) turns[threadIdx.x] = p.rope_turns[threadIdx.x];
   __syncthreads();
   const int len = len_s;
   const bool ok = len >= 0 && (int64_t)len + p.T_new <= p.cap;
+  const bool tab = p.rope && ok && p.T_new <= kAppendTab;  // a decode step's few rows
+  if (tab) {
+    const int half = p.d / 2;
+    for (int e = threadIdx.x; e < p.T_new * half; e += blockDim.x)
+      rtab[e] = rot_turns((int64_t)p.pos0 + len + e / half, turns[e % half]);
+    __syncthreads();
+  }
+  // a one-CTA launch (a decode step) starts the call's status word itself
+  if (p.single && threadIdx.x == 0) *p.err = ok ? 0 : kErrCtxOverflow;
   if (ok) {
     const int64_t vecs = p.row_bytes / 16;
     const int64_t n = (int64_t)p.B * p.T_new * vecs;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
       const int64_t row = i / vecs, v = i % vecs;  // row = b * T_new + t
       const int64_t b = row / p.T_new, t = row % p.T_new;
       const int64_t dst = ((b * p.cap + len + t) * p.row_bytes) / 16 + v;
-      reinterpret_cast<uint4*>(p.K_cache)[dst] = reinterpret_cast<const uint4*>(p.K_new)[i];
+      if (!p.rope)
+        reinterpret_cast<uint4*>(p.K_cache)[dst] = reinterpret_cast<const uint4*>(p.K_new)[i];
       reinterpret_cast<uint4*>(p.V_cache)[dst] = reinterpret_cast<const uint4*>(p.V_new)[i];
     }
-  } else if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (p.rope) {  // keys rotated at their global positions pos0 + len + t (pairs i, i + d/2)
+      // one 16-byte vector of the first half of a (row, head) and its partner vector at + d/2
+      const int half = p.d / 2, E = 16 / p.esize, cpr = half / E;  // vectors per half row
+      const int64_t heads = p.row_bytes / ((int64_t)p.esize * p.d);
+      const int64_t n_vec = (int64_t)p.B * p.T_new * heads * cpr;
+      for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < n_vec; w += stride) {
+        const int c = (int)(w % cpr);
+        const int64_t rh = w / cpr;  // (b * T_new + t) * heads + head
+        const int64_t row = rh / heads, b = row / p.T_new, t = row % p.T_new;
+        const int64_t src = (rh * p.d + (int64_t)c * E) * p.esize / 16;  // in 16-byte vectors
+        const int64_t dst =
+            ((((b * p.cap + len + t) * heads + rh % heads) * p.d + (int64_t)c * E) * p.esize) / 16;
+        const uint4 lo = reinterpret_cast<const uint4*>(p.K_new)[src];
+        const uint4 hi = reinterpret_cast<const uint4*>(p.K_new)[src + half * p.esize / 16];
+        float x[8], y[8];
+        if (p.esize == 2) {
+          Vec<__nv_bfloat16, 8>::unpack(lo, x);
+          Vec<__nv_bfloat16, 8>::unpack(hi, y);
+        } else {
+          Vec<float, 4>::unpack(*reinterpret_cast<const float4*>(&lo), x);
+          Vec<float, 4>::unpack(*reinterpret_cast<const float4*>(&hi), y);
+        }
+        float xr[8], yr[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (e >= E) break;
+          const int i = c * E + e;
+          const float2 cs = tab ? rtab[t * half + i] : rot_turns((int64_t)p.pos0 + len + t, turns[i]);
+          xr[e] = x[e] * cs.x - y[e] * cs.y;
+          yr[e] = y[e] * cs.x + x[e] * cs.y;
+        }
+        uint4 olo, ohi;
+        if (p.esize == 2) {
+          __nv_bfloat162* a2 = reinterpret_cast<__nv_bfloat162*>(&olo);
+          __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&ohi);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            a2[e] = __floats2bfloat162_rn(xr[2 * e], xr[2 * e + 1]);
+            b2[e] = __floats2bfloat162_rn(yr[2 * e], yr[2 * e + 1]);
+          }
+        } else {
+          olo = make_uint4(__float_as_uint(xr[0]), __float_as_uint(xr[1]), __float_as_uint(xr[2]),
+                           __float_as_uint(xr[3]));
+          ohi = make_uint4(__float_as_uint(yr[0]), __float_as_uint(yr[1]), __float_as_uint(yr[2]),
+                           __float_as_uint(yr[3]));
+        }
+        reinterpret_cast<uint4*>(p.K_cache)[dst] = olo;
+        reinterpret_cast<uint4*>(p.K_cache)[dst + half * p.esize / 16] = ohi;
+      }
+    }
+  } else if (!p.single && blockIdx.x == 0 && threadIdx.x == 0) {
     set_err(p.err, kErrCtxOverflow);
   }
   __syncthreads();
+  if (p.single) {  // every thread's rows are written: publish the new length
+    if (threadIdx.x == 0 && ok) *reinterpret_cast<volatile int32_t*>(p.len) = len + p.T_new;
+    return;
+  }
   if (threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(p.ticket, 1u) == gridDim.x - 1) {
@@ -107,7 +175,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(AppendParams p) {
 
 cudaError_t launch_kv_append(const AppendParams& p, int sms, cudaStream_t st) {
   const int64_t n = (int64_t)p.B * p.T_new * (p.row_bytes / 16);
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 4LL * sms));
+  const int64_t blocks =
+      p.single ? 1 : std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 4LL * sms));
   kv_append_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
   return cudaGetLastError();
 }

@@ -8,24 +8,31 @@
 // documents, memory rows are used as stored
 //   [news.neo-ai.one article, "グローバル RoPE（アクティブコンテキスト）" and "推論パイプライン"].
 //
-// Kernel design (one CTA per SM: eight compute warps and one copy warp):
-//  * A tile is KT = 64 / h_kv consecutive key rows of one query with all their KV heads: one
-//    contiguous 16 KB block of K and one of V ([row][KV head][d] is the storage order), so the
-//    copy warp moves a tile with two one-dimensional bulk copies and DRAM sees long sequential
-//    reads. Per query the memory rows come first, then the local rows (a tile holds one kind).
-//    The flattened tile list of all queries is cut into one contiguous range per CTA; a 4-stage
-//    ring (full/empty mbarriers) keeps ~128 KB of loads in flight per SM.
+// Kernel design (one CTA of eight warps per SM):
+//  * A tile is KT = 64 / h_kv consecutive key rows of one query with all their KV heads (16 KB
+//    of K and 16 KB of V, contiguous in the [row][KV head][d] storage order). The copy warp
+//    moves it with four TMA boxes of [KV head][key row][64 dims] (each half of d of K and of V)
+//    whose 128-byte swizzle makes every later shared-memory read conflict-free. Per query the
+//    memory rows come first, then the local rows (a tile holds one kind). The flattened tile
+//    list of all queries is cut into one contiguous range per CTA; a 4-stage ring keeps
+//    128 KB of loads in flight per SM (an mbarrier per stage signals its copies' arrival;
+//    the last warp to release a stage, counted in shared memory, issues its next copies).
 //  * Compute warp w owns KV head w % h_kv and eight key rows of every tile, with its own online
-//    softmax state (running max, sum, P.V accumulators of its head's query rows); the warps
-//    meet only at the end of a query's segment (no block barrier per tile).
-//  * RoPE by angle addition: key c of a local tile whose rows start at position P is rotated by
-//    c*theta from a per-CTA table, and the rotation by P*theta moves to the query
+//    softmax state; the warps meet only at the end of a query's segment (no block barrier per
+//    tile). The logits and P.V run on the tensor cores as warp-level bf16 MMAs (fp32
+//    accumulation): the query rows of the head (<= 8) are the rows of a 16-row A operand,
+//    ldmatrix hands each lane its key and value fragments (8 MMAs of k = 16 over d for the
+//    logits, 16 MMAs of k = 8 for P.V), and the probabilities of the logits' accumulator
+//    fragment are the A fragment of P.V without leaving registers. This is a bandwidth-bound
+//    stream, not a GEMM: the MMAs replace ~100 fp32 instructions per (key, KV head) row with
+//    ~4, which is what lets eight warps keep up with HBM.
+//  * RoPE by angle addition: key c of a local tile whose rows start at position P is rotated
+//    by c*theta (per-CTA table, applied to the key fragments in registers before they are
+//    rounded back to bf16), and the rotation by P*theta moves to the query
 //    (<R((P+c)th) k, q> = <R(c th) k, R(-P th) q>); from one local tile to the next the query
-//    turns by a fixed -KT*theta, so no position table is read or built. Angles are exact
-//    integer turn counts (64-bit fixed point) fed to a single-precision sincospi.
-//  * Logits: the lanes split each key's RoPE pairs (16 lanes per key for 4 query rows, 32 for
-//    8) and a transposing reduction hands each lane finished logits; P.V: lane l owns output
-//    dims 4l .. 4l+3; packed fp32 FMA throughout.
+//    turns by a fixed -KT*theta. Angles are exact integer turn counts (64-bit fixed point) fed
+//    to a single-precision sincospi. The rotated query and keys and the probabilities are
+//    rounded to bf16 for the MMAs (fp32 accumulation, softmax in fp32).
 //  * A query split over several CTAs leaves one fp32 partial (m, l, o) per CTA in the workspace;
 //    a second, short kernel merges them with one CTA per output row spread over all SMs.
 // Every wait is bounded; on expiry the CTA records kErrWaitTimeout in the workspace status
@@ -39,7 +46,7 @@
 namespace msa {
 
 constexpr int kDecCW = 8;                        // compute warps
-constexpr int kDecThreads = (kDecCW + 1) * 32;   // + the copy warp
+constexpr int kDecThreads = kDecCW * 32;
 constexpr int kDecRowsPerTile = 64;              // key rows x KV heads per tile
 constexpr int kDecStages = 4;
 constexpr int kDecD = 128;
@@ -67,35 +74,84 @@ __device__ __forceinline__ bool named_sync_compute_or(bool pred) {
   return r != 0;
 }
 
-template <int RB>
-__global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p) {
+// ---- register-level helpers of the tensor-core (mma.sync) logits and P.V
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// D = A B + C for a 16 x 8 x 16 bf16 product whose A rows 8..15 are zero: only the row-g
+// accumulators (c0, c1) are kept.
+__device__ __forceinline__ void mma_k16(float& c0, float& c1, uint32_t a0, uint32_t a2,
+                                        uint32_t b0, uint32_t b1) {
+  float d2, d3;
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %10, %11};"
+      : "+f"(c0), "+f"(c1), "=f"(d2), "=f"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f), "f"(0.f));
+}
+// The same for a 16 x 8 x 8 product.
+__device__ __forceinline__ void mma_k8(float& c0, float& c1, uint32_t a0, uint32_t b0) {
+  float d2, d3;
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+      "{%0, %1, %7, %8};"
+      : "+f"(c0), "+f"(c1), "=f"(d2), "=f"(d3)
+      : "r"(a0), "r"(0u), "r"(b0), "f"(0.f), "f"(0.f));
+}
+__device__ __forceinline__ float2 bf2_unpack(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t bf2_pack(float2 v) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                      uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(0), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_constant__ CUtensorMap map_vc,
+                  const __grid_constant__ CUtensorMap map_kl, const __grid_constant__ CUtensorMap map_vl,
+                  DecParams p) {
   constexpr int D = kDecD, HALF = D / 2, NS = kDecStages;
-  constexpr int LPK = RB == 4 ? 16 : 32;  // lanes sharing one key's dims in the logits
-  constexpr int NG = 32 / LPK;            // key groups per warp
-  constexpr int KG = 8 / NG;              // keys per group
-  constexpr int PPL = HALF / LPK;         // RoPE pairs per lane (4 or 2)
-  constexpr int PH = PPL / 2;             // packed float2 of pairs per lane
-  constexpr int NV = KG * RB;             // logits per lane before the group reduction
-  constexpr int PER = NV / LPK;           // logits per lane after it (RB / 4)
-  constexpr int WS = 8 * RB + 3 * RB;     // per-warp scratch: probabilities, alpha, max, sum
   extern __shared__ __align__(1024) unsigned char sm_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
   unsigned char* stages = sm;                                                 // [NS][K|V]
   float4* rstep = reinterpret_cast<float4*>(sm + NS * kDecStage);             // [KT][32]
-  unsigned long long* turns = reinterpret_cast<unsigned long long*>(rstep + 64 * 32);  // [HALF]
-  float* comb = reinterpret_cast<float*>(turns + HALF);                       // [8][RB][D]
-  float* wscr = comb + kDecCW * RB * D;                                       // [8][WS]
-  uint64_t* full = reinterpret_cast<uint64_t*>(wscr + kDecCW * WS);           // [NS]
-  uint64_t* empty = full + NS;                                                // [NS]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + NS);
+  float4* kturn = rstep + 64 * 32;                                            // [32]
+  float4* qrot = kturn + 32;   // [T][32]: R(pos theta) at each query token's position
+  float4* turn0 = qrot + 8 * 32;  // [32]: R(-pos0 theta), a query's first local tile
+  float4* turn1 = turn0 + 32;     // [32]: R(-P theta), P = the CTA's first local tile start
+  unsigned long long* turns = reinterpret_cast<unsigned long long*>(turn1 + 32);  // [HALF]
+  const int RB = (p.h_q / p.h_kv) * p.T <= 4 ? 4 : 8;  // combine-buffer rows per KV head
+  constexpr int WS = 11 * 8;                            // per-warp scratch floats
+  float* comb = reinterpret_cast<float*>(turns + HALF);  // [8][RB][D]
+  float* wscr = comb + kDecCW * 8 * D;                   // [8][WS]: max at 9 RB, sum at 10 RB
+  uint64_t* full = reinterpret_cast<uint64_t*>(wscr + kDecCW * WS);  // [NS]
+  unsigned int* released = reinterpret_cast<unsigned int*>(full + NS);  // [NS] warp releases
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(released + NS);
+  volatile int* issued = abort_flag + 1;  // tiles whose copies were issued
   __shared__ int skip_call;
+  __shared__ int ctx_first[32];  // context rows of the CTA's first 32 queries
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int HKV = p.h_kv;
   const int KT = kDecRowsPerTile / HKV;  // key rows per tile
   const int Gq = p.h_q / HKV;
-  const int nr = Gq * p.T;  // query rows per KV head (<= RB)
+  const int nr = Gq * p.T;  // query rows per KV head (<= 8)
   // local rows per query: fixed, or read from the device (a cache that grows between launches)
   const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
   if (L < p.T || L > p.Ls) {  // uniform over the grid: nothing is read or written
@@ -115,139 +171,152 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kDecCW);
+      released[s] = 0u;
     }
     *abort_flag = 0;
+    *issued = 0;
     // an error an earlier kernel of the same call recorded (a failed append) skips the call
     skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
     fence_mbar_init();
   }
   if (tid < HALF) turns[tid] = p.rope_turns[tid];
+  if (tid < 32)
+    ctx_first[tid] = b_first + tid < p.B ? min(max(__ldg(p.ctx_len + b_first + tid), 0), p.max_ctx) : 0;
   __syncthreads();
-  if (skip_call) return;  // written once before the barrier: one value for the whole CTA
+  if (skip_call) return;
+  auto ctx_rows = [&](int bb) {
+    return bb - b_first < 32 ? ctx_first[bb - b_first]
+                             : min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
+  };  // written once before the barrier: one value for the whole CTA
 
-  if (warp == kDecCW) {
-    // ---------------- copy warp (lane 0): tile u -> stage u % NS
-    if (lane == 0) {
-      int b = b_first, tt = tt_first, cb = -1, n_ctx = 0;
-      const int64_t row_elems = (int64_t)HKV * D;  // one key row, all KV heads
-      int u = 0;
-      for (; u < n_tiles; ++u) {
-        const int s = u % NS;
-        if (u >= NS) {  // the compute warps released this stage
-          const bool ok = !*abort_flag &&
-                          mbar_wait_bounded(&empty[s], (uint32_t)(((u / NS) - 1) & 1), p.err);
-          if (!ok) {
-            *abort_flag = 1;
-            break;
-          }
-        }
-        if (b != cb) {
-          cb = b;
-          n_ctx = min(max(__ldg(p.ctx_len + b), 0), p.max_ctx);
-        }
-        int nk;
-        const __nv_bfloat16 *ks, *vs;
-        if (tt < p.CT) {  // memory rows [KT tt, KT tt + KT)
-          const int kt = tt * KT;
-          nk = min(max(n_ctx - kt, 0), KT);
-          const int64_t off = ((int64_t)b * p.max_ctx + kt) * row_elems;
-          ks = p.cK + off;
-          vs = p.cV + off;
-        } else {  // local rows [KT i, KT i + KT)
-          const int j0 = (tt - p.CT) * KT;
-          nk = min(L - j0, KT);
-          const int64_t off = ((int64_t)b * p.Ls + j0) * row_elems;
-          ks = p.Kl + off;
-          vs = p.Vl + off;
-        }
-        const uint32_t bytes = (uint32_t)nk * (uint32_t)HKV * kDecRow;
-        unsigned char* st = stages + (size_t)s * kDecStage;
-        mbar_arrive_expect_tx(&full[s], 2u * bytes);
-        if (bytes) {
-          bulk_g2s(st, ks, bytes, &full[s]);
-          bulk_g2s(st + kDecHalf, vs, bytes, &full[s]);
-        }
-        if (++tt == TPP) {
-          tt = 0;
-          ++b;
-        }
-      }
-      // every copy issued lands before the CTA can exit (bounded; the last NS stages)
-      for (int j = max(0, u - NS); j < u; ++j)
-        mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), p.err);
+  // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
+  // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d. Issued by one
+  // thread: the first NS tiles here, each later one by the warp that releases the stage last.
+  auto issue = [&](int v) {
+    const int64_t x = x0 + v;
+    const int bb = (int)(x / TPP), tv = (int)(x % TPP);
+    const bool ctx = tv < p.CT;
+    const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
+    // memory tiles past the query's context are not read (local tiles hold >= 1 row)
+    const bool any = !ctx || kt < ctx_rows(bb);
+    const int s = v % NS;
+    const uint32_t st = smem_u32(stages + (size_t)s * kDecStage);
+    fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
+    mbar_arrive_expect_tx(&full[s], any ? kDecStage : 0u);
+    if (any) {
+      const CUtensorMap* mk = ctx ? &map_kc : &map_kl;
+      const CUtensorMap* mv = ctx ? &map_vc : &map_vl;
+      const int y = ctx ? bb * p.max_ctx + kt : bb * p.Ls + kt;
+      tma3d(st, mk, 0, y, &full[s]);
+      tma3d(st + kDecHalf / 2, mk, HALF, y, &full[s]);
+      tma3d(st + kDecHalf, mv, 0, y, &full[s]);
+      tma3d(st + kDecHalf + kDecHalf / 2, mv, HALF, y, &full[s]);
     }
-    return;
-  }
+    *issued = v + 1;
+  };
+  if (tid == 0)
+    for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
 
   // ---------------- compute warps
   const int g = warp % HKV;    // KV head of this warp
   const int sl = warp / HKV;   // its eight key rows of a tile: [8 sl, 8 sl + 8)
-  const int grp = lane / LPK, dl = lane % LPK;
-  const int i0 = PPL * dl;     // first RoPE pair of this lane in the logits
-  // in-tile rotations: rstep[c][pp] = (cos, cos, sin, sin) of c*theta for the pairs 2pp, 2pp+1
+  const int gr = lane >> 2;    // fragment row: query row gr (logits) / key 8 sl + gr (keys)
+  const int t4 = lane & 3;     // fragment column pair
+  // in-tile rotations: rstep[c][pp] = (cos, cos, sin, sin) of c*theta for the pairs 2pp, 2pp+1,
+  // and the query's turn from one local tile to the next: kturn[pp] for -KT*theta
   for (int idx = tid; idx < KT * 32; idx += kDecCW * 32) {
     const int c = idx >> 5, pp = idx & 31;
     const float2 r0 = rot_turns(c, turns[2 * pp]), r1 = rot_turns(c, turns[2 * pp + 1]);
     rstep[idx] = make_float4(r0.x, r1.x, r0.y, r1.y);
   }
-  // the query's turn from one local tile to the next: R(-KT theta) on the lane's pairs
-  float2 stc[PH], sts[PH];  // (cos, cos), (sin, sin) of the packed pairs
-#pragma unroll
-  for (int h = 0; h < PH; ++h) {
-    const float2 r0 = rot_turns(-KT, turns[i0 + 2 * h]), r1 = rot_turns(-KT, turns[i0 + 2 * h + 1]);
-    stc[h] = make_float2(r0.x, r1.x);
-    sts[h] = make_float2(r0.y, r1.y);
+  {  // per-CTA rotations of the query: kturn, qrot[T], turn0, turn1 (32 pairs of pairs each)
+    const int64_t kt_first = (int64_t)max(tt_first - p.CT, 0) * KT;
+    for (int idx = tid; idx < (p.T + 3) * 32; idx += kDecCW * 32) {
+      const int r = idx >> 5, pp = idx & 31;
+      int64_t n;
+      float4* dst;
+      if (r < p.T) {
+        n = (int64_t)p.pos0 + L - p.T + r;
+        dst = qrot + idx;
+      } else if (r == p.T) {
+        n = -KT;
+        dst = kturn + pp;
+      } else if (r == p.T + 1) {
+        n = -(int64_t)p.pos0;
+        dst = turn0 + pp;
+      } else {
+        n = -((int64_t)p.pos0 + kt_first);
+        dst = turn1 + pp;
+      }
+      const float2 r0 = rot_turns(n, turns[2 * pp]), r1 = rot_turns(n, turns[2 * pp + 1]);
+      *dst = make_float4(r0.x, r1.x, r0.y, r1.y);
+    }
   }
-  named_sync_compute();  // rstep complete
+  named_sync_compute();  // tables complete
 
-  float* wp = wscr + warp * WS;  // [8 keys][RB] probabilities
-  float* wa = wp + 8 * RB;       // [RB] rescale of this tile
-  float* wm = wa + RB;           // [RB] running max
-  float* wl = wm + RB;           // [RB] running sum
-  // rotated, pre-scaled query on this lane's pairs, packed by two: lo = dims i0 + 2h, +1,
-  // hi = the same + 64; ql as rotated, qa turned back by the local tile's start position
-  float2 ql_lo[RB][PH], ql_hi[RB][PH], qa_lo[RB][PH], qa_hi[RB][PH];
-  float2 acc[RB][2];             // P.V: dims 4l .. 4l+3
+  // ldmatrix row addresses of this lane: key row 8 sl + (lane & 7) of KV head g, dim chunk
+  // 4 (m & 1) + (lane >> 3) of the half m >> 1 (128-byte swizzle: chunk ^ (line & 7))
+  const int line = g * KT + 8 * sl + (lane & 7);
+  uint32_t lofs[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    lofs[m] = (uint32_t)((m >> 1) * (kDecHalf / 2) + line * 128 +
+                         ((((m & 1) * 4 + (lane >> 3)) ^ (line & 7)) << 4));
+
+  // the query rows of KV head g in fragment order: element (m, q) holds dims 32m + 8q + 2 t4
+  // and +1 of row gr (zero for gr >= nr); ql rotated at the query position and pre-scaled,
+  // qa turned back by the current local tile's start position
+  float2 ql[4][4], qa[4][4];
+  float2 o[16];  // P.V accumulators of row gr: dims 8 nt + 2 t4, +1
+  float mrow = -INFINITY, lsum = 0.f;
   int b = b_first, tt = tt_first, cur = -1, n_ctx = 0;
   const int WPH = kDecCW / HKV;  // warps per KV head
 
   // combine the warps of each KV head over the open segment of query fb; write O (a query
   // within one CTA) or this CTA's partial
   auto finish_segment = [&](int fb) {
+    float l = lsum;
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (gr < RB) {
 #pragma unroll
-    for (int r = 0; r < RB; ++r)
-      *reinterpret_cast<float4*>(comb + (warp * RB + r) * D + 4 * lane) =
-          make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+      for (int nt = 0; nt < 16; ++nt)
+        *reinterpret_cast<float2*>(comb + (warp * RB + gr) * D + 8 * nt + 2 * t4) = o[nt];
+      if (t4 == 0) {
+        wscr[warp * WS + 9 * RB + gr] = mrow;
+        wscr[warp * WS + 10 * RB + gr] = l;
+      }
+    }
     const bool write = !named_sync_compute_or(*abort_flag != 0);  // one decision for all warps
     const int64_t first = dec_cta_of((int64_t)fb * TPP, G, total);
     const int64_t last = dec_cta_of((int64_t)fb * TPP + TPP - 1, G, total);
     const int n_seg = (int)(last - first + 1);
     const int seg = (int)(ci - first);
-    const int n_out = HKV * nr * D;
-    for (int idx = tid; idx < n_out; idx += kDecCW * 32) {
-      const int gh = idx / (nr * D), r = (idx / D) % nr, e = idx % D;
+    const int e = tid & (D - 1);  // output dim of this thread; rows r = tid / D, + 2, ...
+    for (int gh = 0; gh < HKV; ++gh)
+    for (int r = tid / D; r < nr; r += kDecCW * 32 / D) {
       float M = -INFINITY;
       for (int k2 = 0; k2 < WPH; ++k2) M = fmaxf(M, wscr[(gh + k2 * HKV) * WS + 9 * RB + r]);
-      float o = 0.f, l = 0.f;
+      float ov = 0.f, lv = 0.f;
       if (M != -INFINITY)
         for (int k2 = 0; k2 < WPH; ++k2) {
           const int w = gh + k2 * HKV;
           const float m = wscr[w * WS + 9 * RB + r];
           const float a = m == -INFINITY ? 0.f : exp2f(m - M);
-          o = fmaf(comb[(w * RB + r) * D + e], a, o);
-          l = fmaf(wscr[w * WS + 10 * RB + r], a, l);
+          ov = fmaf(comb[(w * RB + r) * D + e], a, ov);
+          lv = fmaf(wscr[w * WS + 10 * RB + r], a, lv);
         }
       if (!write) continue;
       const int t = r / Gq, h = gh * Gq + r % Gq;
       if (n_seg == 1) {
-        p.O[(((int64_t)fb * p.T + t) * p.h_q + h) * D + e] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+        p.O[(((int64_t)fb * p.T + t) * p.h_q + h) * D + e] =
+            __float2bfloat16_rn(lv > 0.f ? ov / lv : 0.f);
       } else {
         const int64_t slot = (((int64_t)fb * p.max_seg + seg) * HKV + gh) * RB + r;
-        p.part_o[slot * D + e] = o;
+        p.part_o[slot * D + e] = ov;
         if (e == 0) {
           p.part_ml[slot * 2] = M;
-          p.part_ml[slot * 2 + 1] = l;
+          p.part_ml[slot * 2 + 1] = lv;
         }
       }
     }
@@ -261,204 +330,148 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
     if (b != cur) {
       if (cur >= 0) finish_segment(cur);
       cur = b;
-      n_ctx = min(max(__ldg(p.ctx_len + b), 0), p.max_ctx);
-      // rotated, pre-scaled query rows of this warp's KV head
+      n_ctx = ctx_rows(b);
+      const int tq = min(gr / Gq, p.T - 1), h = g * Gq + gr % Gq;
+      const __nv_bfloat16* q = p.Q + (((int64_t)b * p.T + tq) * p.h_q + h) * D;
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        float xl[PPL], xh[PPL];
+      for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int m = 0; m < PPL; ++m) xl[m] = xh[m] = 0.f;
-        if (r < nr) {
-          const int t = r / Gq, h = g * Gq + r % Gq;
-          const __nv_bfloat16* q = p.Q + (((int64_t)b * p.T + t) * p.h_q + h) * D;
-          const int64_t pos = (int64_t)p.pos0 + L - p.T + t;
-#pragma unroll
-          for (int m = 0; m < PPL; ++m) {
-            const float a = __bfloat162float(q[i0 + m]), c = __bfloat162float(q[i0 + m + HALF]);
-            const float2 cs = rot_turns(pos, turns[i0 + m]);
-            xl[m] = (a * cs.x - c * cs.y) * p.scale_log2;
-            xh[m] = (c * cs.x + a * cs.y) * p.scale_log2;
+        for (int qq = 0; qq < 4; ++qq) {
+          const int i = 32 * m + 8 * qq + 2 * t4;  // RoPE pairs i, i + 1 (partners + 64)
+          float2 lo = make_float2(0.f, 0.f), hi = lo;
+          if (gr < nr) {
+            const float2 a = bf2_unpack(*reinterpret_cast<const uint32_t*>(q + i));
+            const float2 c = bf2_unpack(*reinterpret_cast<const uint32_t*>(q + i + HALF));
+            const float4 cs = qrot[tq * 32 + i / 2];
+            const float2 c2 = make_float2(cs.x, cs.y), s2 = make_float2(cs.z, cs.w);
+            lo = __fmul2_rn(__ffma2_rn(a, c2, __fmul2_rn(c, make_float2(-s2.x, -s2.y))), sc2);
+            hi = __fmul2_rn(__ffma2_rn(c, c2, __fmul2_rn(a, s2)), sc2);
           }
+          ql[m][qq] = lo;
+          ql[m + 2][qq] = hi;
         }
 #pragma unroll
-        for (int hh = 0; hh < PH; ++hh) {
-          ql_lo[r][hh] = make_float2(xl[2 * hh], xl[2 * hh + 1]);
-          ql_hi[r][hh] = make_float2(xh[2 * hh], xh[2 * hh + 1]);
-        }
-        acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
-      }
+      for (int nt = 0; nt < 16; ++nt) o[nt] = make_float2(0.f, 0.f);
+      mrow = -INFINITY;
+      lsum = 0.f;
       qa_ok = false;
-      if (lane < RB) {
-        wm[lane] = -INFINITY;
-        wl[lane] = 0.f;
-      }
-      __syncwarp();
     }
     const int nk = is_ctx ? min(max(n_ctx - kt, 0), KT) : min(L - kt, KT);
-    if (!is_ctx && !qa_ok) {  // the query turned back by the tile's start position P
-      const int64_t P = (int64_t)p.pos0 + kt;
+    // keys used as stored: memory rows, and local rows of a cache that holds rotated keys
+    const bool plain = is_ctx || p.keys_rotated;
+    if (!plain && !qa_ok) {  // the query turned back by the tile's start position P
+      // P = pos0 (a query's first local tile) or, for the CTA's first tile only, pos0 + kt
+      const float4* A = kt == 0 ? turn0 : turn1;
 #pragma unroll
-      for (int hh = 0; hh < PH; ++hh) {
-        const float2 r0 = rot_turns(-P, turns[i0 + 2 * hh]);
-        const float2 r1 = rot_turns(-P, turns[i0 + 2 * hh + 1]);
-        const float2 c2 = make_float2(r0.x, r1.x), s2 = make_float2(r0.y, r1.y);
-        const float2 ns2 = make_float2(-s2.x, -s2.y);
+      for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int r = 0; r < RB; ++r) {
-          qa_lo[r][hh] = __ffma2_rn(ql_lo[r][hh], c2, __fmul2_rn(ql_hi[r][hh], ns2));
-          qa_hi[r][hh] = __ffma2_rn(ql_hi[r][hh], c2, __fmul2_rn(ql_lo[r][hh], s2));
+        for (int qq = 0; qq < 4; ++qq) {
+          const float4 cs = A[16 * m + 4 * qq + t4];
+          const float2 c2 = make_float2(cs.x, cs.y), s2 = make_float2(cs.z, cs.w);
+          const float2 lo = ql[m][qq], hi = ql[m + 2][qq];
+          qa[m][qq] = __ffma2_rn(lo, c2, __fmul2_rn(hi, make_float2(-s2.x, -s2.y)));
+          qa[m + 2][qq] = __ffma2_rn(hi, c2, __fmul2_rn(lo, s2));
         }
-      }
       qa_ok = true;
     }
     const int s = u % NS;
     if (!*abort_flag && !mbar_wait_bounded(&full[s], (uint32_t)((u / NS) & 1), p.err))
       *abort_flag = 1;
-    const unsigned char* stg = stages + (size_t)s * kDecStage;
+    const uint32_t kb = smem_u32(stages + (size_t)s * kDecStage), vb = kb + kDecHalf;
 
-    // ---- logits of this warp's eight keys x RB rows: lane group grp takes keys
-    // [KG grp, KG grp + KG) of them, lane dl of the group the RoPE pairs [PPL dl, PPL dl + PPL)
-    float v[NV];
+    // ---- logits S[row gr][keys 8 sl + 2 t4, +1]: 8 MMAs over d, keys rotated in registers
+    uint32_t kr[4][4];
 #pragma unroll
-    for (int kk = 0; kk < KG; ++kk) {
-      const int j = 8 * sl + grp * KG + kk;  // key row within the tile
-      const unsigned char* row = stg + (j * HKV + g) * kDecRow;
-      float2 x2[PH], y2[PH];
-      if constexpr (PPL == 4) {
-        const uint2 lo = *reinterpret_cast<const uint2*>(row + 2 * i0);
-        const uint2 hi = *reinterpret_cast<const uint2*>(row + 2 * HALF + 2 * i0);
-        x2[0] = make_float2(__uint_as_float(lo.x << 16), __uint_as_float(lo.x & 0xFFFF0000u));
-        x2[1] = make_float2(__uint_as_float(lo.y << 16), __uint_as_float(lo.y & 0xFFFF0000u));
-        y2[0] = make_float2(__uint_as_float(hi.x << 16), __uint_as_float(hi.x & 0xFFFF0000u));
-        y2[1] = make_float2(__uint_as_float(hi.y << 16), __uint_as_float(hi.y & 0xFFFF0000u));
-      } else {
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(row + 2 * i0);
-        const uint32_t hi = *reinterpret_cast<const uint32_t*>(row + 2 * HALF + 2 * i0);
-        x2[0] = make_float2(__uint_as_float(lo << 16), __uint_as_float(lo & 0xFFFF0000u));
-        y2[0] = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
-      }
-      if (!is_ctx) {  // local row: rotate by c * theta within the tile, dot with qa
+    for (int m = 0; m < 4; ++m) ldsm_x4(kb + lofs[m], kr[m]);
+    if (!plain) {  // local keys: R(c theta), c = 8 sl + gr within the tile
+      const float4* R = rstep + (8 * sl + gr) * 32 + t4;
 #pragma unroll
-        for (int hh = 0; hh < PH; ++hh) {
-          const float4 R = rstep[j * 32 + i0 / 2 + hh];
-          const float2 c2 = make_float2(R.x, R.y), s2 = make_float2(R.z, R.w);
-          const float2 a2 = __ffma2_rn(x2[hh], c2, __fmul2_rn(y2[hh], make_float2(-s2.x, -s2.y)));
-          const float2 b2 = __ffma2_rn(y2[hh], c2, __fmul2_rn(x2[hh], s2));
-          x2[hh] = a2;
-          y2[hh] = b2;
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float4 cs = R[16 * m + 4 * qq];
+          const float2 c2 = make_float2(cs.x, cs.y), s2 = make_float2(cs.z, cs.w);
+          const float2 x = bf2_unpack(kr[m][qq]), y = bf2_unpack(kr[m + 2][qq]);
+          kr[m][qq] = bf2_pack(__ffma2_rn(x, c2, __fmul2_rn(y, make_float2(-s2.x, -s2.y))));
+          kr[m + 2][qq] = bf2_pack(__ffma2_rn(y, c2, __fmul2_rn(x, s2)));
         }
-#pragma unroll
-        for (int r = 0; r < RB; ++r) {
-          float2 t2 = __fmul2_rn(qa_lo[r][0], x2[0]);
-          t2 = __ffma2_rn(qa_hi[r][0], y2[0], t2);
-#pragma unroll
-          for (int hh = 1; hh < PH; ++hh) {
-            t2 = __ffma2_rn(qa_lo[r][hh], x2[hh], t2);
-            t2 = __ffma2_rn(qa_hi[r][hh], y2[hh], t2);
-          }
-          v[kk * RB + r] = t2.x + t2.y;
-        }
-      } else {  // memory row: as stored, against the unshifted query
-#pragma unroll
-        for (int r = 0; r < RB; ++r) {
-          float2 t2 = __fmul2_rn(ql_lo[r][0], x2[0]);
-          t2 = __ffma2_rn(ql_hi[r][0], y2[0], t2);
-#pragma unroll
-          for (int hh = 1; hh < PH; ++hh) {
-            t2 = __ffma2_rn(ql_lo[r][hh], x2[hh], t2);
-            t2 = __ffma2_rn(ql_hi[r][hh], y2[hh], t2);
-          }
-          v[kk * RB + r] = t2.x + t2.y;
-        }
-      }
     }
-    tr_reduce<NV, LPK / 2>(v, lane);
+    // four independent accumulator pairs (one per quarter of d) shorten the MMA chain
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    if (plain) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          mma_k16(sa[m], sb[m], bf2_pack(ql[m][2 * hh]), bf2_pack(ql[m][2 * hh + 1]),
+                  kr[m][2 * hh], kr[m][2 * hh + 1]);
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          mma_k16(sa[m], sb[m], bf2_pack(qa[m][2 * hh]), bf2_pack(qa[m][2 * hh + 1]),
+                  kr[m][2 * hh], kr[m][2 * hh + 1]);
+    }
+    const float s0 = (sa[0] + sa[1]) + (sa[2] + sa[3]), s1 = (sb[0] + sb[1]) + (sb[2] + sb[3]);
 
-    // ---- online softmax over the warp's 8 keys: lane holds the logits of the warp's key
-    // grp * KG + (dl * PER + e) / RB and row (dl * PER + e) % RB
-    {
-      const int kk = grp * KG + (dl * PER) / RB;
-      const int jrow = kt + 8 * sl + kk;  // memory row or local row
-      float pe[PER];
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int r = (dl * PER + e) % RB;
-        const int t = r / Gq;
-        const bool vis = 8 * sl + kk < nk && r < nr && (is_ctx || jrow <= L - p.T + t);
-        float x = vis ? v[e] : -INFINITY;
-        float mx = x;
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mo = wm[r];
-        const float mn = fmaxf(mo, mx);
-        const float pr = (x == -INFINITY) ? 0.f : exp2f(x - mn);
-        float sum = pr;
-        sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 8);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-        pe[e] = pr;
-        v[e] = mn;         // reuse: new max of row r
-        v[PER + e] = sum;  // and the tile's sum (NV >= 2 * PER)
-      }
-      __syncwarp();  // every lane read the old maxima
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int r = (dl * PER + e) % RB;
-        wp[kk * RB + r] = pe[e];
-        if (kk == 0) {
-          const float mo = wm[r], mn = v[e];
-          const float alpha = mn == -INFINITY ? 1.f : (mo == -INFINITY ? 0.f : exp2f(mo - mn));
-          wa[r] = alpha;
-          wm[r] = mn;
-          wl[r] = fmaf(wl[r], alpha, v[PER + e]);
-        }
-      }
-      __syncwarp();
-    }
-    // ---- P.V over the warp's 8 keys: dims 4l .. 4l+3
-    {
-#pragma unroll
-      for (int r = 0; r < RB; ++r) {
-        const float a = wa[r];
-        acc[r][0].x *= a; acc[r][0].y *= a; acc[r][1].x *= a; acc[r][1].y *= a;
-      }
-      const unsigned char* vt = stg + kDecHalf;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int j = 8 * sl + kk;
-        if (j >= nk) break;
-        const uint2 w = *reinterpret_cast<const uint2*>(vt + (j * HKV + g) * kDecRow + 8 * lane);
-        const float2 v01 = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u));
-        const float2 v23 = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
-#pragma unroll
-        for (int r4 = 0; r4 < RB; r4 += 4) {
-          const float4 pr = *reinterpret_cast<const float4*>(wp + kk * RB + r4);
-          const float pv[4] = {pr.x, pr.y, pr.z, pr.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 pp = make_float2(pv[i], pv[i]);
-            acc[r4 + i][0] = __ffma2_rn(pp, v01, acc[r4 + i][0]);
-            acc[r4 + i][1] = __ffma2_rn(pp, v23, acc[r4 + i][1]);
-          }
-        }
-      }
-      __syncwarp();  // probabilities and rescale are rewritten by the next tile
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    // next local tile: advance the position by KT (turn the query back by KT theta)
+    // ---- online softmax of row gr over this warp's 8 keys (a lane holds keys 2 t4, 2 t4 + 1)
+    const int jj = 8 * sl + 2 * t4;          // tile key of s0 (s1: jj + 1)
+    const bool k0 = jj < nk, k1 = jj + 1 < nk;
+    bool v0 = k0, v1 = k1;
     if (!is_ctx) {
+      const int lim = L - p.T + gr / Gq - kt;  // causal: local row kt + j visible if <= lim
+      v0 = v0 && jj <= lim;
+      v1 = v1 && jj + 1 <= lim;
+    }
+    const float xa = v0 ? s0 : -INFINITY, xb = v1 ? s1 : -INFINITY;
+    float mx = fmaxf(xa, xb);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float mn = fmaxf(mrow, mx);
+    const float alpha = mn == -INFINITY ? 1.f : exp2f(mrow - mn);
+    const float p0 = v0 ? exp2f(xa - mn) : 0.f, p1 = v1 ? exp2f(xb - mn) : 0.f;
+    lsum = fmaf(lsum, alpha, p0 + p1);
+    mrow = mn;
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-      for (int hh = 0; hh < PH; ++hh) {
-        const float2 ns2 = make_float2(-sts[hh].x, -sts[hh].y);
+      for (int nt = 0; nt < 16; ++nt) o[nt] = __fmul2_rn(o[nt], make_float2(alpha, alpha));
+    }
+    const uint32_t pa = bf2_pack(make_float2(p0, p1));
+
+    // ---- P.V: O[row gr][dims] += P[row gr][8 keys] V[8 keys][dims], 16 MMAs; V rows of keys
+    // past the tile's valid rows are cleared (their probabilities are zero, their contents
+    // are not defined)
+    const uint32_t vmask = (k0 ? 0x0000FFFFu : 0u) | (k1 ? 0xFFFF0000u : 0u);
+    const bool partial = __any_sync(0xffffffffu, vmask != 0xFFFFFFFFu);
 #pragma unroll
-        for (int r = 0; r < RB; ++r) {
-          const float2 lo = __ffma2_rn(qa_lo[r][hh], stc[hh], __fmul2_rn(qa_hi[r][hh], ns2));
-          const float2 hi = __ffma2_rn(qa_hi[r][hh], stc[hh], __fmul2_rn(qa_lo[r][hh], sts[hh]));
-          qa_lo[r][hh] = lo;
-          qa_hi[r][hh] = hi;
-        }
+    for (int m = 0; m < 4; ++m) {
+      uint32_t vr[4];
+      ldsm_x4_trans(vb + lofs[m], vr);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        const uint32_t bv = partial ? (vr[qq] & vmask) : vr[qq];
+        mma_k8(o[4 * m + qq].x, o[4 * m + qq].y, pa, bv);
       }
+    }
+    __syncwarp();
+    // release the stage; the last of the eight warps refills it with tile u + NS
+    if (lane == 0 && atomicAdd(&released[s], 1u) % kDecCW == kDecCW - 1 && u + NS < n_tiles &&
+        !*abort_flag)
+      issue(u + NS);
+    // next local tile: advance the position by KT (turn the query back by KT theta)
+    if (!plain) {
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const float4 cs = kturn[16 * m + 4 * qq + t4];
+          const float2 c2 = make_float2(cs.x, cs.y), s2 = make_float2(cs.z, cs.w);
+          const float2 lo = qa[m][qq], hi = qa[m + 2][qq];
+          qa[m][qq] = __ffma2_rn(lo, c2, __fmul2_rn(hi, make_float2(-s2.x, -s2.y)));
+          qa[m + 2][qq] = __ffma2_rn(hi, c2, __fmul2_rn(lo, s2));
+        }
     }
     if (++tt == TPP) {
       tt = 0;
@@ -466,6 +479,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) attend_dec_kernel(DecParams p)
     }
   }
   if (cur >= 0) finish_segment(cur);
+  // every copy issued lands before the CTA exits (after an expired wait some were not
+  // consumed; bounded)
+  named_sync_compute();
+  if (tid == 0)
+    for (int j = max(0, *issued - NS); j < *issued; ++j)
+      mbar_wait_bounded(&full[j % NS], (uint32_t)((j / NS) & 1), p.err);
 }
 
 // Merge of the partials of the queries split over several CTAs: CTA = one output row (query b,
@@ -557,9 +576,9 @@ DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int
   pl.ctr_bytes = ((size_t)B * sizeof(unsigned int) + 255) & ~(size_t)255;
   pl.part_ml_bytes = max_seg > 1 ? ((slots * 2 * sizeof(float) + 255) & ~(size_t)255) : 0;
   pl.part_o_bytes = max_seg > 1 ? ((slots * kDecD * sizeof(float) + 255) & ~(size_t)255) : 0;
-  pl.smem = 1024 + (size_t)kDecStages * kDecStage + (size_t)64 * 32 * 16 + (kDecD / 2) * 8 +
-            sizeof(float) * ((size_t)kDecCW * pl.RB * kDecD + (size_t)kDecCW * 11 * pl.RB) +
-            2 * kDecStages * 8 + 16;
+  pl.smem = 1024 + (size_t)kDecStages * kDecStage + (size_t)64 * 32 * 16 + 11 * 32 * 16 +
+            (kDecD / 2) * 8 + sizeof(float) * ((size_t)kDecCW * 8 * kDecD + (size_t)kDecCW * 88) +
+            kDecStages * 12 + 16;
   return pl;
 }
 
@@ -580,16 +599,31 @@ DecPlan attend_dec_plan_cap(int B, int T, int h_q, int h_kv, int d, int max_ctx,
 }
 
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st) {
-  cudaError_t e = cudaSuccess;
-  if (pl.RB == 4) {
-    e = cudaFuncSetAttribute(attend_dec_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)pl.smem);
-    if (e == cudaSuccess) attend_dec_kernel<4><<<pl.grid, kDecThreads, pl.smem, st>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(attend_dec_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)pl.smem);
-    if (e == cudaSuccess) attend_dec_kernel<8><<<pl.grid, kDecThreads, pl.smem, st>>>(p);
+  // tensor maps of [rows][KV head][d] (bf16, 128-byte swizzle, zero fill out of bounds) read
+  // as boxes of [KV head][KT rows][64 dims]: dims (d, rows of all queries, KV head)
+  const uint64_t row = (uint64_t)p.h_kv * kDecRow;
+  const uint32_t box[3] = {64, (uint32_t)(kDecRowsPerTile / p.h_kv), (uint32_t)p.h_kv};
+  const uint64_t str[2] = {row, kDecRow};
+  CUtensorMap mkl, mvl, mkc, mvc;
+  {
+    const uint64_t dims[3] = {kDecD, (uint64_t)p.B * p.Ls, (uint64_t)p.h_kv};
+    if (!encode_bf16_map(&mkl, p.Kl, 3, dims, str, box, true) ||
+        !encode_bf16_map(&mvl, p.Vl, 3, dims, str, box, true))
+      return cudaErrorInvalidValue;
   }
+  if (p.max_ctx > 0) {
+    const uint64_t dims[3] = {kDecD, (uint64_t)p.B * p.max_ctx, (uint64_t)p.h_kv};
+    if (!encode_bf16_map(&mkc, p.cK, 3, dims, str, box, true) ||
+        !encode_bf16_map(&mvc, p.cV, 3, dims, str, box, true))
+      return cudaErrorInvalidValue;
+  } else {  // no memory tiles: never read
+    mkc = mkl;
+    mvc = mvl;
+  }
+  cudaError_t e = cudaFuncSetAttribute(attend_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pl.smem);
+  if (e == cudaSuccess)
+    attend_dec_kernel<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.max_seg == 1) return e;
   // split queries: merge their partials (one CTA per output row; y carries the grid size)

@@ -147,6 +147,7 @@ struct DecParams {
   int Ls;                   // local rows stored per query (row stride of Kl / Vl), >= L
   const int32_t* L_dev;     // nullable: the local length is read from here at run time
   int skip_on_err;          // write nothing if the status word already holds an error
+  int keys_rotated;         // local keys are stored rotated at their positions pos0 + j
   int rope, pos0;
   unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions,
                                       // theta_i = base^(-2i/128); all zero without RoPE
@@ -198,6 +199,11 @@ struct AppendParams {
   int32_t* len;               // device, the rows the cache holds (shared by the batch)
   int* err;                   // workspace status word
   unsigned int* ticket;       // zero on entry; the last CTA advances len and resets it
+  int single;                 // one CTA: sets the status word itself, needs no ticket
+  int rope, pos0;             // keys stored rotated at position pos0 + row (rope != 0)
+  unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1, 64-bit fixed point
+  int d;                      // head dim (RoPE pairs i, i + d/2)
+  int esize;                  // bytes per element (2: bf16, 4: fp32)
 };
 cudaError_t launch_kv_append(const AppendParams& p, int sms, cudaStream_t st);
 

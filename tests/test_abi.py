@@ -148,14 +148,20 @@ def test_generation_entry_points_reject_bad_arguments_on_host(msa):
     fake = ctypes.c_void_p(256)
     ws = ctypes.c_void_p(512)
     # kv_append: more new rows than the cache holds, no workspace, missing length, misaligned
-    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 9, 8, 128, 1, ws, 256, None)
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 9, 8, 128, 1, 0, 0.0, ws, 256,
+                              None)
     assert r == 1
-    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 1, 8, 128, 1, None, 0, None)
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 1, 8, 128, 1, 0, 0.0, None, 0,
+                              None)
     assert r == 3
-    r = msa.lib.msa_kv_append(fake, fake, 2, 8, None, fake, fake, 1, 8, 128, 1, ws, 256, None)
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, None, fake, fake, 1, 8, 128, 1, 0, 0.0, ws, 256,
+                              None)
+    assert r == 1
+    r = msa.lib.msa_kv_append(fake, fake, 2, 8, fake, fake, fake, 1, 8, 128, 1, -1, 1e6, ws, 256,
+                              None)  # negative pos0
     assert r == 1
     r = msa.lib.msa_kv_append(fake, ctypes.c_void_p(264), 2, 8, fake, fake, fake, 1, 8, 128, 1,
-                              ws, 256, None)
+                              0, 0.0, ws, 256, None)
     assert r == 1
     need = msa.msa_decode_step_workspace(4, 1, 32, 8, 128, 128, 4096)
     assert need > 256

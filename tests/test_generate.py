@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from _util import check_attention, to_dev
+from _util import check_attention, stored_f64, to_dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -55,7 +55,7 @@ def test_decode_step_matches_oracle(msa, gpu, B, T, h_q, h_kv, L0, S, n_ctx, pos
     c = _case(7, B, T, h_q, h_kv, d, L0, S, n_ctx)
     ref = oracle.generate(c["Qs"], c["Ks"], c["Vs"], c["Kp"], c["Vp"], c["Kb"], c["Vb"], c["gi"],
                           c["n_ctx"], pos0, base)
-    cache = msa.LocalCache(B, cap, h_kv, d, device=gpu)
+    cache = msa.LocalCache(B, cap, h_kv, d, pos0=pos0, rope_base=base, device=gpu)
     if L0:
         cache.append(to_dev(c["Kp"], gpu), to_dev(c["Vp"], gpu))
     ctxK, ctxV = to_dev(c["ctxK"], gpu), to_dev(c["ctxV"], gpu)
@@ -63,21 +63,31 @@ def test_decode_step_matches_oracle(msa, gpu, B, T, h_q, h_kv, L0, S, n_ctx, pos
     worst = 0.0
     for s in range(S):
         O = msa.decode_step(cache, to_dev(c["Qs"][s], gpu), to_dev(c["Ks"][s], gpu),
-                            to_dev(c["Vs"][s], gpu), ctxK, ctxV, cl, pos0, base)
+                            to_dev(c["Vs"][s], gpu), ctxK, ctxV, cl)
         torch.cuda.synchronize()
         worst = max(worst, check_attention(O, ref[s], "bf16"))
-    assert int(cache.length.item()) == L0 + S * T
-    # the cache holds [prompt ; every step's tokens] bit for bit
-    want = np.concatenate([c["Kp"]] + c["Ks"], axis=1) if L0 else np.concatenate(c["Ks"], axis=1)
-    got = cache.K[:, :L0 + S * T].contiguous().view(torch.int16).cpu().numpy()
-    assert np.array_equal(got.view(np.uint16), want)
+    n = L0 + S * T
+    assert int(cache.length.item()) == n
+    # the cache holds [prompt ; every step's tokens]: V bit for bit, K rotated at pos0 + row
+    # (the oracle's RoPE, within one bf16 rounding)
+    K_all = np.concatenate([c["Kp"]] + c["Ks"], axis=1)
+    V_all = np.concatenate([c["Vp"]] + c["Vs"], axis=1)
+    got_v = cache.V[:, :n].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got_v, V_all)
+    got_k = to_np(cache.K[:, :n])
+    K64 = stored_f64(K_all, "bf16")
+    for b in range(B):
+        for j in range(0, n, max(1, n // 37)):
+            for hh in range(h_kv):
+                ref_k = oracle.rope(K64[b, j, hh], pos0 + j, base) if base > 0 else K64[b, j, hh]
+                assert np.all(np.abs(got_k[b, j, hh] - ref_k) <= 2.0 ** -8 * np.abs(ref_k) + 1e-6)
 
 
 def test_kv_append_fills_in_pieces_and_advances_the_length(msa, gpu):
     B, h_kv, d, cap = 3, 8, 128, 100
     K = synth.normal(3, 110, (B, 87, h_kv, d), "bf16")
     V = synth.normal(3, 111, (B, 87, h_kv, d), "bf16")
-    cache = msa.LocalCache(B, cap, h_kv, d, device=gpu)
+    cache = msa.LocalCache(B, cap, h_kv, d, device=gpu)  # no RoPE: stored as given
     cache.append(to_dev(K[:, :37], gpu), to_dev(V[:, :37], gpu))
     cache.append(to_dev(K[:, 37:], gpu), to_dev(V[:, 37:], gpu))
     torch.cuda.synchronize()
@@ -91,7 +101,7 @@ def test_kv_append_fills_in_pieces_and_advances_the_length(msa, gpu):
 def test_full_cache_is_flagged_and_left_unchanged(msa, gpu):
     B, T, h_q, h_kv, d, L0 = 2, 1, 32, 8, 128, 30
     c = _case(5, B, T, h_q, h_kv, d, L0, 2, [10, 20])
-    cache = msa.LocalCache(B, L0 + 1, h_kv, d, device=gpu)
+    cache = msa.LocalCache(B, L0 + 1, h_kv, d, pos0=16, rope_base=1e6, device=gpu)
     cache.append(to_dev(c["Kp"], gpu), to_dev(c["Vp"], gpu))
     ctxK, ctxV = to_dev(c["ctxK"], gpu), to_dev(c["ctxV"], gpu)
     cl = torch.from_numpy(c["n_ctx"]).to(gpu)
@@ -99,12 +109,12 @@ def test_full_cache_is_flagged_and_left_unchanged(msa, gpu):
                      dtype=torch.uint8, device=gpu)
     O = torch.empty((B, T, h_q, d), dtype=torch.bfloat16, device=gpu)
     msa.decode_step(cache, to_dev(c["Qs"][0], gpu), to_dev(c["Ks"][0], gpu),
-                    to_dev(c["Vs"][0], gpu), ctxK, ctxV, cl, 16, 1e6, O=O, ws=ws)
+                    to_dev(c["Vs"][0], gpu), ctxK, ctxV, cl, O=O, ws=ws)
     assert msa.msa_workspace_status(ws) == 0
     before = cache.K.clone()
     O.fill_(7.0)
     msa.decode_step(cache, to_dev(c["Qs"][1], gpu), to_dev(c["Ks"][1], gpu),
-                    to_dev(c["Vs"][1], gpu), ctxK, ctxV, cl, 16, 1e6, O=O, ws=ws)
+                    to_dev(c["Vs"][1], gpu), ctxK, ctxV, cl, O=O, ws=ws)
     assert msa.msa_workspace_status(ws) == 2      # the context overflow code
     assert int(cache.length.item()) == L0 + 1
     assert torch.equal(cache.K.view(torch.int16), before.view(torch.int16))
@@ -123,7 +133,7 @@ def test_captured_step_replays_as_the_cache_grows(msa, gpu):
     def setup():
         out = []
         for c in cases:
-            cache = msa.LocalCache(B, cap, h_kv, d, device=gpu)
+            cache = msa.LocalCache(B, cap, h_kv, d, pos0=pos0, rope_base=base, device=gpu)
             with torch.cuda.stream(st):
                 cache.append(to_dev(c["Kp"], gpu), to_dev(c["Vp"], gpu), stream=st)
             out.append(dict(cache=cache, ctxK=to_dev(c["ctxK"], gpu), ctxV=to_dev(c["ctxV"], gpu),
@@ -148,7 +158,7 @@ def test_captured_step_replays_as_the_cache_grows(msa, gpu):
     def step(layers):
         for x in layers:
             msa.decode_step(x["cache"], x["Q"], x["K"], x["V"], x["ctxK"], x["ctxV"], x["cl"],
-                            pos0, base, O=x["O"], ws=x["ws"], stream=st)
+                            O=x["O"], ws=x["ws"], stream=st)
 
     eager = setup()
     want = []
