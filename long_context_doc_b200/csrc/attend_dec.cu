@@ -222,26 +222,29 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
   const int sl = warp / HKV;   // its eight key rows of a tile: [8 sl, 8 sl + 8)
   const int gr = lane >> 2;    // fragment row: query row gr (logits) / key 8 sl + gr (keys)
   const int t4 = lane & 3;     // fragment column pair
-  // in-tile rotations: rstep[c][pp] = (cos, cos, sin, sin) of c*theta for the pairs 2pp, 2pp+1,
-  // and the query's turn from one local tile to the next: kturn[pp] for -KT*theta
-  for (int idx = tid; idx < KT * 32; idx += kDecCW * 32) {
-    const int c = idx >> 5, pp = idx & 31;
-    const float2 r0 = rot_turns(c, turns[2 * pp]), r1 = rot_turns(c, turns[2 * pp + 1]);
-    rstep[idx] = make_float4(r0.x, r1.x, r0.y, r1.y);
-  }
-  {  // per-CTA rotations of the query: kturn, qrot[T], turn0, turn1 (32 pairs of pairs each)
+  // per-CTA rotation tables, (cos, cos, sin, sin) of the pairs 2pp, 2pp + 1 (32 per row):
+  // qrot[t] R(pos theta) at each query token's position; for caches whose keys are rotated
+  // here also rstep[c] R(c theta) of the in-tile key offsets, kturn R(-KT theta) (the query's
+  // turn from one local tile to the next), turn0 R(-pos0 theta) and turn1 R(-P theta) with P
+  // the start of the CTA's first local tile
+  {
+    const bool rot_keys = p.rope && !p.keys_rotated;
+    const int n_rows = p.T + (rot_keys ? KT + 3 : 0);
     const int64_t kt_first = (int64_t)max(tt_first - p.CT, 0) * KT;
-    for (int idx = tid; idx < (p.T + 3) * 32; idx += kDecCW * 32) {
+    for (int idx = tid; idx < n_rows * 32; idx += kDecCW * 32) {
       const int r = idx >> 5, pp = idx & 31;
       int64_t n;
       float4* dst;
       if (r < p.T) {
         n = (int64_t)p.pos0 + L - p.T + r;
         dst = qrot + idx;
-      } else if (r == p.T) {
+      } else if (r < p.T + KT) {
+        n = r - p.T;
+        dst = rstep + (r - p.T) * 32 + pp;
+      } else if (r == p.T + KT) {
         n = -KT;
         dst = kturn + pp;
-      } else if (r == p.T + 1) {
+      } else if (r == p.T + KT + 1) {
         n = -(int64_t)p.pos0;
         dst = turn0 + pp;
       } else {
@@ -359,7 +362,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     }
     const int nk = is_ctx ? min(max(n_ctx - kt, 0), KT) : min(L - kt, KT);
     // keys used as stored: memory rows, and local rows of a cache that holds rotated keys
-    const bool plain = is_ctx || p.keys_rotated;
+    const bool plain = is_ctx || p.keys_rotated || !p.rope;
     if (!plain && !qa_ok) {  // the query turned back by the tile's start position P
       // P = pos0 (a query's first local tile) or, for the CTA's first tile only, pos0 + kt
       const float4* A = kt == 0 ? turn0 : turn1;

@@ -82,12 +82,16 @@ def routed_layer(layer: RoutedLayer, k: int, K_loc: torch.Tensor, V_loc: torch.T
 
 
 def interleave_rounds(layers: List[RoutedLayer], k: int, rounds: int, rope_base: float,
-                      doc_kv: Callable[[int, int], tuple]):
-    """Memory Interleaving over ``rounds`` rounds of all routed layers.
+                      doc_kv: Callable[[int, int], tuple], select=None):
+    """Memory Interleaving over up to ``rounds`` rounds of all routed layers.
 
     ``doc_kv(layer, doc)`` returns the raw per-token (K, V) [len, h_kv, d] device tensors of a
-    retrieved document at that layer. Returns (ids[r][l] [B, k], scores[r][l] [B, k],
-    O[r][l] [B, T, h_q, d], appended[b] = the documents appended per query, in order).
+    retrieved document at that layer. ``select(r, ids_r)``, if given, takes the place of the
+    model's generative retrieval: it gets the round's selections (numpy int32 [B, k] per routed
+    layer) and returns per query the doc ids to append, in order, or None to end the loop (the
+    documents suffice); without it the last routed layer's selection is appended. Returns
+    (ids[r][l] [B, k], scores[r][l] [B, k], O[r][l] [B, T, h_q, d], appended[b] = the
+    documents appended per query, in order).
     """
     B = layers[0].Q.shape[0]
     n_docs = layers[0].doc_chunk_off.shape[0] - 1
@@ -107,10 +111,18 @@ def interleave_rounds(layers: List[RoutedLayer], k: int, rounds: int, rope_base:
             ids_r.append(ids)
             sc_r.append(sc)
             O_r.append(O)
-        last = ids_r[-1].cpu().tolist()
-        for b in range(B):
-            appended[b].extend(sorted(i for i in last[b] if i >= 0))
         all_ids.append(ids_r)
         all_sc.append(sc_r)
         all_O.append(O_r)
+        if select is None:
+            last = ids_r[-1].cpu().tolist()
+            chosen = [sorted(i for i in last[b] if i >= 0) for b in range(B)]
+        else:
+            chosen = select(r, [x.cpu().numpy() for x in ids_r])
+        if chosen is None:
+            break
+        for b in range(B):
+            for doc in chosen[b]:
+                if doc >= 0 and doc not in appended[b]:
+                    appended[b].append(int(doc))
     return all_ids, all_sc, all_O, appended

@@ -218,7 +218,8 @@ def pipeline(w, inp: dict, L=None) -> dict:
     return out
 
 
-def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=None) -> dict:
+def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=None,
+               select=None) -> dict:
     """Oracle of Memory Interleaving rounds (reading R18 of the design notes).
 
     layers[l]: dict with Kbar_r, Kbar, Vbar (stored dtype), doc_chunk_off, Q_r, Q and the query
@@ -226,8 +227,14 @@ def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=No
     retrieved document. Round 0 attends to the query tokens alone; after each round the docs
     selected by the LAST routed layer are appended (ascending id) for every later round,
     before the query tokens, and excluded from routing. pos0 = k in every round.
+    ``select(r, ids_r)``, if given, stands for the model's generative retrieval: it receives the
+    round's selections (ids_r[l] int32 [B, k] per routed layer) and returns, per query, the doc
+    ids to append in order (already appended ids and ids < 0 are skipped), or None when the
+    accumulated documents suffice, which ends the loop (ai-papers.net summary, "MSAの提案手法";
+    ruixiangma.github.io blog, "Memory Interleaving": the model generates document ids, their
+    text is appended, and the loop repeats until the model judges the documents sufficient).
     Returns dict(ids=[r][l] int32 [B,k], scores=[r][l], doc_scores=[r][l], O64=[r][l],
-    appended=[b] list)."""
+    appended=[b] list, rounds=rounds run)."""
     B = layers[0]["Q"].shape[0]
     n_docs = len(layers[0]["doc_chunk_off"]) - 1
     words = (n_docs + 31) // 32
@@ -254,13 +261,20 @@ def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=No
             sc_r.append(sc)
             ds_r.append(ds)
             O_r.append(O)
-        for b in range(B):
-            appended[b].extend(sorted(int(i) for i in ids_r[-1][b] if i >= 0))
         res["ids"].append(ids_r)
         res["scores"].append(sc_r)
         res["doc_scores"].append(ds_r)
         res["O64"].append(O_r)
+        chosen = ([sorted(int(i) for i in ids_r[-1][b] if i >= 0) for b in range(B)]
+                  if select is None else select(r, ids_r))
+        if chosen is None:
+            break
+        for b in range(B):
+            for doc in chosen[b]:
+                if doc >= 0 and doc not in appended[b]:
+                    appended[b].append(int(doc))
     res["appended"] = appended
+    res["rounds"] = len(res["ids"])
     return res
 
 

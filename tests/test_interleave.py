@@ -37,6 +37,42 @@ def test_oracle_interleave_round_structure():
                 assert not set(res["ids"][r][l][b].tolist()) & set(app[:r * w.k])
 
 
+def test_oracle_interleave_follows_selected_docs_and_stops():
+    """Generative retrieval stood in for by a schedule: the docs a round selects are appended in
+    the order given (duplicates skipped), excluded from later routing, and a None ends the loop.
+    (Every query appends the same number of new documents per round: one local length per
+    batch.)"""
+    w, lays = _case()
+    dk = lambda l, d: synth.appended_doc_kv(w, l, d)  # noqa: E731
+    sched = {0: [[5, 3], [9, 4]], 1: [[3, 7], [2, 9]]}  # one new doc each in round 1
+    seen = []
+
+    def sel(r, ids_r):
+        assert len(ids_r) == len(lays) and ids_r[0].shape == (w.B, w.k)
+        seen.append(r)
+        return sched.get(r)
+
+    res = oracle.interleave(lays, w.k, 4, w.rope_base, dk, select=sel)
+    assert res["rounds"] == 3 and seen == [0, 1, 2]
+    assert res["appended"] == [[5, 3, 7], [9, 4, 2]]
+    for l in range(len(lays)):
+        assert not set(res["ids"][1][l][0].tolist()) & {5, 3}
+        assert not set(res["ids"][1][l][1].tolist()) & {9, 4}
+        assert not set(res["ids"][2][l][0].tolist()) & {5, 3, 7}
+        assert not set(res["ids"][2][l][1].tolist()) & {9, 4, 2}
+    # round 2 of layer 0, query 0, attends over [doc 5 ; doc 3 ; doc 7 ; query tokens]
+    lay = lays[0]
+    coff = lay["doc_chunk_off"]
+    cpd = int(np.max(np.diff(coff)))
+    gi, cl = oracle.gather(res["ids"][2][0], coff, w.k * cpd)
+    parts = [dk(0, doc) for doc in (5, 3, 7)]
+    K_loc = np.concatenate([p[0] for p in parts] + [lay["K_q"][0]])[None]
+    V_loc = np.concatenate([p[1] for p in parts] + [lay["V_q"][0]])[None]
+    O = oracle.attend(lay["Q"][:1], K_loc, V_loc, lay["Kbar"], lay["Vbar"], gi[:1], cl[:1], w.k,
+                      w.rope_base)
+    assert np.array_equal(O[0], res["O64"][2][0][0])
+
+
 def test_oracle_interleave_attends_to_appended_text():
     """Round 1 equals attention over [memory ; round-0 docs' raw K/V ; query tokens]."""
     w, lays = _case(B=1, layers=1, seed=9)
@@ -92,6 +128,64 @@ def test_interleave_engine_matches_oracle(gpu):
         if not exact:  # a near-tie changed the appended set; later rounds are not comparable
             break
         assert appended == ref["appended"] or r < 2
+
+
+@pytest.mark.gpu
+def test_interleave_engine_with_selected_docs_matches_oracle(gpu):
+    """The engine's loop with the appended documents chosen by a caller (here: the first routed
+    layer's two best documents, best first) and an early stop, against the oracle's loop."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    from long_context_doc_b200 import engine
+    w, lays = _case(seed=9)
+    dk_np = lambda l, d: synth.appended_doc_kv(w, l, d)  # noqa: E731
+
+    def sel(r, ids_r):
+        if r == 2:
+            return None
+        return [[int(x) for x in ids_r[0][b][:2]] for b in range(w.B)]
+
+    ref = oracle.interleave(lays, w.k, 4, w.rope_base, dk_np, select=sel)
+    assert ref["rounds"] == 3
+    layers = []
+    for lay in lays:
+        Krb = to_dev(lay["Kbar_r"], gpu)
+        layers.append(engine.RoutedLayer(
+            Kbar_r=Krb, kr_inv_norm=msa.kr_inv_norm(Krb), Kbar=to_dev(lay["Kbar"], gpu),
+            Vbar=to_dev(lay["Vbar"], gpu),
+            doc_chunk_off=torch.from_numpy(lay["doc_chunk_off"]).to(gpu),
+            Q_r=to_dev(lay["Q_r"], gpu), Q=to_dev(lay["Q"], gpu), K_q=to_dev(lay["K_q"], gpu),
+            V_q=to_dev(lay["V_q"], gpu), Kbar_r_hat=msa.kr_normalize(Krb)))
+    cache = {}
+
+    def dk_dev(l, d):
+        if (l, d) not in cache:
+            kk, vv = dk_np(l, d)
+            cache[(l, d)] = (to_dev(kk, gpu), to_dev(vv, gpu))
+        return cache[(l, d)]
+
+    ids, scores, O, appended = engine.interleave_rounds(layers, w.k, 4, w.rope_base, dk_dev,
+                                                        select=sel)
+    torch.cuda.synchronize()
+    assert len(ids) == 3
+    tol = SCORE_TOL["bf16"]
+    for r in range(3):
+        exact = True
+        for l in range(len(lays)):
+            ds = ref["doc_scores"][r][l].copy()
+            for b in range(w.B):
+                if r > 0:
+                    ds[b, [d for d in ref["appended"][b][:2 * r]]] = -np.inf
+            n = check_topk(ids[r][l].cpu().numpy(), scores[r][l].cpu().numpy().astype(np.float64),
+                           ref["ids"][r][l], ref["scores"][r][l], ds, tol)
+            exact &= n == w.B
+            if n == w.B:
+                check_attention(O[r][l], ref["O64"][r][l], "bf16")
+        if not exact:  # a near-tie changed the selection; later rounds are not comparable
+            break
+    else:
+        assert appended == ref["appended"]
 
 
 def _masked(ref, r, l, w):
