@@ -103,6 +103,48 @@ def peaks():
         return 6650.0, "fallback"
 
 
+# ------------------------------------------------------------------------------ ranks
+class Ranks:
+    """One process per GPU (torchrun's RANK / WORLD_SIZE / LOCAL_RANK; rendezvous on
+    MASTER_ADDR, 127.0.0.1 on one node). The path does not shard: every rank runs its own
+    replica, and the only collectives are the timing barrier and the max over ranks of the
+    measured times."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: int = 300):
+        import torch.distributed as dist
+        self.dist = dist
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world > 1:
+            kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, values, device):
+        """Element-wise max over ranks of a list of floats (every rank gets the result)."""
+        if self.world == 1:
+            return [float(v) for v in values]
+        import torch
+        t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return [float(v) for v in t.tolist()]
+
+    def close(self):
+        if self.world > 1:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+
+
+def replica_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Whole-job throughput of ``world`` replicas that each processed ``units_per_rank`` in at
+    most ``ms`` milliseconds (the max over ranks)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -291,24 +333,19 @@ class Decode:
 
 def run_libmsa(args):
     import torch
-    import torch.distributed as dist
 
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+    ranks = Ranks("nccl", dev)
+    rank, world = ranks.rank, ranks.world
     w = synth.C4 if args.workload == "bank100m" else synth.C3
     wk = Decode(w, dev, args.fetch, rank, args.scan)
     torch.cuda.synchronize()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
@@ -409,13 +446,9 @@ def run_libmsa(args):
     e1.record(wk.main)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / Ke
-    # max over ranks
-    if world > 1:
-        t = torch.tensor([step_ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, e2e_ms = float(t[0]), float(t[1])
-    value = world * w.B / (step_ms / 1e3)
-    e2e_value = world * w.B / (e2e_ms / 1e3)
+    step_ms, e2e_ms = ranks.max([step_ms, e2e_ms], dev)  # max over ranks
+    value = replica_rate(world, w.B, step_ms)
+    e2e_value = replica_rate(world, w.B, e2e_ms)
     route_avg = statistics.mean(route_ms)
     peak, peak_kind = peaks()
     achieved = wk.scan_bytes() / (route_avg / 1e3) / 1e9
@@ -456,9 +489,7 @@ def run_libmsa(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, e_graph  # graphs are released before the process group
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 # ------------------------------------------------------------------------------ CPU oracle
@@ -565,18 +596,14 @@ def run_reference(args):
 def run_prefill(args):
     """The 1M-token prefill path, each phase timed with CUDA events on the launching stream."""
     import torch
-    import torch.distributed as dist
 
     import long_context_doc_b200 as msa
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+    ranks = Ranks("nccl", dev, timeout_s=300)
+    rank, world = ranks.rank, ranks.world
     w = synth.C2.scaled(seed=synth.C2.seed + 1000 * rank)
     inp = synth.dev_token_workload(w, dev)
     off = inp["doc_tok_off"]
@@ -628,8 +655,7 @@ def run_prefill(args):
             ev[5].record(st)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     for _ in range(max(args.warmup, 3)):
@@ -649,10 +675,7 @@ def run_prefill(args):
         totals.append(ev[0].elapsed_time(ev[-1]))
     clocks = sampler.stop()
     step_ms = statistics.mean(totals)
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t[0])
+    step_ms, = ranks.max([step_ms], dev)  # max over ranks
     ph = {n: round(statistics.mean(v), 4) for n, v in phase.items()}
     peak, peak_kind = peaks()
     row = w.h_kv * w.d * 2
@@ -662,7 +685,7 @@ def run_prefill(args):
     line = {
         "metric": "MSA 1M-token prefill: bank tokens/s (doc-wise RoPE + pooling, routing, "
                   "gather, attention)",
-        "value": round(world * n_tok / (step_ms / 1e3), 1), "unit": "bank tokens/s",
+        "value": round(replica_rate(world, n_tok, step_ms), 1), "unit": "bank tokens/s",
         "n_gpus": world, "steps": Kst, "warmup": max(args.warmup, 3),
         "ms_per_step": round(step_ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16",
@@ -683,26 +706,20 @@ def run_prefill(args):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def run_interleave(args):
     """Memory Interleaving at full size, each phase timed with CUDA events on its stream."""
     import torch
-    import torch.distributed as dist
 
     import long_context_doc_b200 as msa
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=dev)
+    ranks = Ranks("nccl", dev, timeout_s=600)
+    rank, world = ranks.rank, ranks.world
     w = synth.C5.scaled(seed=synth.C5.seed + 1000 * rank)
     B, T, k, R, NL = w.B, w.T, w.k, w.rounds, w.layers
     bf = torch.bfloat16
@@ -795,8 +812,7 @@ def run_interleave(args):
                 ex32.copy_(excl.to(torch.int32))
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     for _ in range(max(1, min(args.warmup, 2))):
@@ -826,10 +842,7 @@ def run_interleave(args):
     barrier()
     clocks = sampler.stop()
     step_ms = t0.elapsed_time(t1) / Kst
-    if world > 1:
-        tt = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        step_ms = float(tt[0])
+    step_ms, = ranks.max([step_ms], dev)  # max over ranks
     route_flop = 2.0 * B * T * n_chunks * w.h_kv * w.d  # per routing call
     route_call_ms = phase["route"] / (R * NL)
     route_tf = route_flop / (route_call_ms / 1e3) / 1e12
@@ -848,7 +861,7 @@ def run_interleave(args):
     line = {
         "metric": "MSA Memory Interleaving queries/s (18 routed layers x 3 rounds, 10M-token "
                   "bank per layer)",
-        "value": round(world * B / (step_ms / 1e3), 3), "unit": "queries/s", "n_gpus": world,
+        "value": round(replica_rate(world, B, step_ms), 3), "unit": "queries/s", "n_gpus": world,
         "steps": Kst, "warmup": max(1, min(args.warmup, 2)), "ms_per_step": round(step_ms, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 normals; appended documents from a per-layer pool)",
@@ -871,9 +884,7 @@ def run_interleave(args):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def run_attend_long(args):
@@ -921,18 +932,14 @@ def run_generate(args):
     """Sparse generation at the 100M-token bank: context construction once per request, then
     ``--gen-tokens`` decode steps through all routed layers; generated tokens/s."""
     import torch
-    import torch.distributed as dist
 
     import long_context_doc_b200 as msa
     import synth
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+    ranks = Ranks("nccl", dev, timeout_s=300)
+    rank, world = ranks.rank, ranks.world
     w = synth.C4
     G = max(1, args.gen_tokens)
     # one context buffer per layer: the gathered memory stays fixed while tokens are generated
@@ -972,8 +979,7 @@ def run_generate(args):
         wk.step()
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     with torch.cuda.stream(wk.main):
@@ -1093,12 +1099,9 @@ def run_generate(args):
     e1.record(wk.main)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / Ke
-    if world > 1:
-        t = torch.tensor([req_ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        req_ms, e2e_ms = float(t[0]), float(t[1])
+    req_ms, e2e_ms = ranks.max([req_ms, e2e_ms], dev)  # max over ranks
     unit = "generated tokens/s"
-    value = world * B * G / (req_ms / 1e3)
+    value = replica_rate(world, B * G, req_ms)
     peak, peak_kind = peaks()
     line = {
         "metric": "MSA sparse generation tokens/s at the 100M-token bank (context built once per "
@@ -1124,7 +1127,7 @@ def run_generate(args):
                      "traffic": captured_traffic(("attend_dec.cu", "common.cuh"),
                                                  "attend_dec_gen100m_dram.json"),
                      "bytes_per_launch": round(step_bytes), "avg_launch_ms": round(dec_avg, 4)},
-        "e2e": {"value": round(world * B * G / (e2e_ms / 1e3), 1), "unit": unit,
+        "e2e": {"value": round(replica_rate(world, B * G, e2e_ms), 1), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3)},
         # per request: the construction step's kernels + per token and layer append,
@@ -1137,9 +1140,7 @@ def run_generate(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_con, g_tok, e_con, e_tok
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def oracle_generate_time(w, layer: int, steps: int) -> float:
