@@ -568,13 +568,10 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       q.pos0 = pos0;
       msa::rope_turns(q.rope ? (double)rope_base : 0.0, 128, q.rope_turns);
       q.scale_log2 = sc * 1.4426950408889634f;
-      q.TPP = dp.TPP;
       q.CT = dp.CT;
       q.max_seg = dp.max_seg;
-      q.total = dp.total;
       q.grid = dp.grid;
       q.err = reinterpret_cast<int*>(w8);
-      q.counters = reinterpret_cast<unsigned int*>(w8 + kHeader);
       q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);
       q.part_o = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes + dp.part_ml_bytes);
       q.O = static_cast<__nv_bfloat16*>(O);
@@ -812,13 +809,10 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
   q.pos0 = pos0;
   msa::rope_turns(q.rope ? (double)rope_base : 0.0, 128, q.rope_turns);
   q.scale_log2 = (scale > 0.f ? scale : 1.0f / sqrtf((float)d)) * 1.4426950408889634f;
-  q.TPP = dp.TPP;
   q.CT = dp.CT;
   q.max_seg = dp.max_seg;
-  q.total = dp.total;
   q.grid = dp.grid;
   q.err = reinterpret_cast<int*>(w8);
-  q.counters = reinterpret_cast<unsigned int*>(w8 + kHeader);
   q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);
   q.part_o = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes + dp.part_ml_bytes);
   q.O = static_cast<__nv_bfloat16*>(O);

@@ -152,14 +152,12 @@ struct DecParams {
   unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions,
                                       // theta_i = base^(-2i/128); all zero without RoPE
   float scale_log2;
-  int TPP, CT, max_seg;     // tiles of 64/h_kv key rows per query, of which the first CT hold
-                            // memory rows and the rest local rows; segments per query (the
-                            // kernels recompute TPP from the live length)
-  int64_t total;            // B * TPP
+  int CT, max_seg;          // tiles of 64/h_kv memory rows per query (the local tiles follow;
+                            // the kernels count them from the live length); partial slots
+                            // per query
   int grid;                 // CTAs of the attention kernel (tile ranges)
   float* part_o;            // [B, max_seg, h_kv, RB, 128]
   float* part_ml;           // [B, max_seg, h_kv, RB, 2]
-  unsigned int* counters;   // [B] (reserved; zeroed per call)
   int* err;                 // workspace status word
   __nv_bfloat16* O;         // [B, T, h_q, 128]
 };
