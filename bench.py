@@ -262,8 +262,18 @@ class Decode:
                 cl=torch.empty(B, dtype=torch.int32, device=dev),
                 cK=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev),
                 cV=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)))
-        self.O = [torch.empty((B, w.T, w.h_q, w.d), dtype=torch.bfloat16, device=dev)
-                  for _ in range(self.L)]
+        # every layer's query inputs (Q_r, Q) in one contiguous buffer and every layer's output
+        # in another, so that a step's host copies are one in and one out
+        nqr, nq = B * w.T * w.h_qr * w.d, B * w.T * w.h_q * w.d
+        self.qbuf = torch.empty(self.L * (nqr + nq), dtype=torch.bfloat16, device=dev)
+        for l, dv in enumerate(self.layers):
+            base = l * (nqr + nq)
+            for name, off, n in (("Q_r", base, nqr), ("Q", base + nqr, nq)):
+                v = self.qbuf[off:off + n].view(dv[name].shape)
+                v.copy_(dv[name])
+                dv[name] = v
+        self.obuf = torch.empty(self.L * nq, dtype=torch.bfloat16, device=dev)
+        self.O = [self.obuf[l * nq:(l + 1) * nq].view(B, w.T, w.h_q, w.d) for l in range(self.L)]
         self.route_ev = None
         self.scan = scan
         # own kernels per layer (memsets and copies excluded): route (tensor path: query fold +
@@ -397,28 +407,27 @@ def run_libmsa(args):
     route_ms = [ev_route[s][l][0].elapsed_time(ev_route[s][l][1])
                 for s in range(Kr) for l in range(wk.L)]
     # end to end: per-step query inputs copied from pinned host memory, outputs read back
-    host_in = []
-    for l in range(wk.L):
-        d = wk.layers[l]
-        host_in.append([t.cpu().pin_memory() for t in (d["Q_r"], d["Q"], d["K_loc"][:, -1:],
-                                                        d["V_loc"][:, -1:])])
-    host_O = [o.cpu().pin_memory() for o in wk.O]
-    host_ids = [b["ids"].cpu().pin_memory() for b in wk.buf]
-    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs)
-    d2h = sum(o.numel() * o.element_size() for o in host_O) + wk.L * w.B * w.k * 4
+    # per step: every layer's Q_r and Q (one copy), the new token's K/V row of every layer's
+    # local cache, then every layer's output (one copy) and the last two layers' top-k ids
+    host_q = wk.qbuf.cpu().pin_memory()
+    host_kv = [[t.cpu().pin_memory() for t in (d["K_loc"][:, -1:], d["V_loc"][:, -1:])]
+               for d in wk.layers]
+    host_O = wk.obuf.cpu().pin_memory()
+    host_ids = [b["ids"].cpu().pin_memory() for b in wk.buf[:2]]
+    h2d = (host_q.numel() * host_q.element_size() +
+           sum(t.numel() * t.element_size() for hs in host_kv for t in hs))
+    d2h = host_O.numel() * host_O.element_size() + 2 * w.B * w.k * 4
 
     def e2e_step():
         with torch.cuda.stream(wk.main):
+            wk.qbuf.copy_(host_q, non_blocking=True)
             for l in range(wk.L):
                 d = wk.layers[l]
-                qr, q, kn, vn = host_in[l]
-                d["Q_r"].copy_(qr, non_blocking=True)
-                d["Q"].copy_(q, non_blocking=True)
+                kn, vn = host_kv[l]
                 d["K_loc"][:, -1:].copy_(kn, non_blocking=True)
                 d["V_loc"][:, -1:].copy_(vn, non_blocking=True)
             wk.step()
-            for l in range(wk.L):
-                host_O[l].copy_(wk.O[l], non_blocking=True)
+            host_O.copy_(wk.obuf, non_blocking=True)
             host_ids[0].copy_(wk.buf[0]["ids"], non_blocking=True)
             host_ids[1].copy_(wk.buf[1]["ids"], non_blocking=True)
 
@@ -950,21 +959,25 @@ def run_generate(args):
     lens0 = torch.full((wk.L,), L0, dtype=torch.int32, device=dev)
     caches, tok = [], []
     ws_bytes = msa.msa_decode_step_workspace(B, 1, w.h_q, w.h_kv, w.d, wk.max_ctx, cap)
+    # the generated token's query and K/V of every layer, in one contiguous buffer so that a
+    # token's inputs arrive with a single host-to-device copy (synthetic, reused every step)
+    nq, nkv = B * w.h_q * w.d, B * w.h_kv * w.d
+    per_layer = nq + 2 * nkv
+    tokbuf = torch.empty(wk.L * per_layer, dtype=bf, device=dev)
     for l in range(wk.L):
         c = msa.LocalCache(B, cap, w.h_kv, w.d, pos0=w.k, rope_base=w.rope_base, device=dev,
                            length=lens[l:l + 1])
         c.append(wk.layers[l]["K_loc"], wk.layers[l]["V_loc"])  # the prompt's local K/V
         caches.append(c)
-        # the generated token's query and K/V at this layer (synthetic, reused every step)
-        tok.append(dict(
-            Q=synth.dev_normal(torch.empty((B, 1, w.h_q, w.d), dtype=bf, device=dev), w.seed,
-                               synth.tag(synth.GEN_Q, l)),
-            K=synth.dev_normal(torch.empty((B, 1, w.h_kv, w.d), dtype=bf, device=dev), w.seed,
-                               synth.tag(synth.GEN_K, l)),
-            V=synth.dev_normal(torch.empty((B, 1, w.h_kv, w.d), dtype=bf, device=dev), w.seed,
-                               synth.tag(synth.GEN_V, l)),
-            O=torch.empty((B, 1, w.h_q, w.d), dtype=bf, device=dev),
-            ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+        base = l * per_layer
+        x = dict(Q=tokbuf[base:base + nq].view(B, 1, w.h_q, w.d),
+                 K=tokbuf[base + nq:base + nq + nkv].view(B, 1, w.h_kv, w.d),
+                 V=tokbuf[base + nq + nkv:base + per_layer].view(B, 1, w.h_kv, w.d),
+                 O=torch.empty((B, 1, w.h_q, w.d), dtype=bf, device=dev),
+                 ws=torch.empty(ws_bytes, dtype=torch.uint8, device=dev))
+        for name, tid in (("Q", synth.GEN_Q), ("K", synth.GEN_K), ("V", synth.GEN_V)):
+            synth.dev_normal(x[name], w.seed, synth.tag(tid, l))
+        tok.append(x)
     torch.cuda.synchronize()
     assert int(lens[0]) == L0
 
@@ -1054,26 +1067,21 @@ def run_generate(args):
     # end to end: each token's per-layer inputs copied from pinned host memory and the last
     # layer's output read back, per generated token; the request's query inputs as in the
     # default workload
-    host_tok = [[t.cpu().pin_memory() for t in (x["Q"], x["K"], x["V"])] for x in tok]
+    host_tok = tokbuf.cpu().pin_memory()  # every layer's token inputs, one copy per token
     host_out = tok[-1]["O"].cpu().pin_memory()
-    host_q = [[t.cpu().pin_memory() for t in (wk.layers[l]["Q_r"], wk.layers[l]["Q"])]
-              for l in range(wk.L)]
-    tok_h2d = sum(t.numel() * t.element_size() for hs in host_tok for t in hs)
-    q_h2d = sum(t.numel() * t.element_size() for hs in host_q for t in hs)
+    host_q = wk.qbuf.cpu().pin_memory()  # every layer's Q_r and Q of the request
+    tok_h2d = host_tok.numel() * host_tok.element_size()
+    q_h2d = host_q.numel() * host_q.element_size()
     h2d = q_h2d + G * tok_h2d
     d2h = G * host_out.numel() * host_out.element_size()
 
     def e2e_token():
-        for l in range(wk.L):
-            for dst, src in zip((tok[l]["Q"], tok[l]["K"], tok[l]["V"]), host_tok[l]):
-                dst.copy_(src, non_blocking=True)
+        tokbuf.copy_(host_tok, non_blocking=True)
         token_step()
         host_out.copy_(tok[-1]["O"], non_blocking=True)
 
     def e2e_con():
-        for l in range(wk.L):
-            wk.layers[l]["Q_r"].copy_(host_q[l][0], non_blocking=True)
-            wk.layers[l]["Q"].copy_(host_q[l][1], non_blocking=True)
+        wk.qbuf.copy_(host_q, non_blocking=True)
         construct()
 
     e_con = e_tok = None
