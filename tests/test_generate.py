@@ -83,6 +83,26 @@ def test_decode_step_matches_oracle(msa, gpu, B, T, h_q, h_kv, L0, S, n_ctx, pos
                 assert np.all(np.abs(got_k[b, j, hh] - ref_k) <= 2.0 ** -8 * np.abs(ref_k) + 1e-6)
 
 
+def test_decode_step_without_routed_memory(msa, gpu):
+    """max_ctx = 0 (nothing gathered): the cache alone is the context."""
+    B, T, h_q, h_kv, d, L0, S, pos0, base = 2, 1, 32, 8, 128, 33, 5, 16, 1e6
+    c = _case(13, B, T, h_q, h_kv, d, L0, S, [1, 1])
+    gi = np.zeros((B, 0), np.int32)
+    cl = np.zeros(B, np.int32)
+    ref = oracle.generate(c["Qs"], c["Ks"], c["Vs"], c["Kp"], c["Vp"], c["Kb"], c["Vb"], gi, cl,
+                          pos0, base)
+    cache = msa.LocalCache(B, L0 + S, h_kv, d, pos0=pos0, rope_base=base, device=gpu)
+    cache.append(to_dev(c["Kp"], gpu), to_dev(c["Vp"], gpu))
+    empty = torch.empty((B, 0, h_kv, d), dtype=torch.bfloat16, device=gpu)
+    cl_dev = torch.from_numpy(cl).to(gpu)
+    for s in range(S):
+        O = msa.decode_step(cache, to_dev(c["Qs"][s], gpu), to_dev(c["Ks"][s], gpu),
+                            to_dev(c["Vs"][s], gpu), empty, empty, cl_dev)
+        torch.cuda.synchronize()
+        check_attention(O, ref[s], "bf16")
+    assert int(cache.length.item()) == L0 + S
+
+
 def test_kv_append_fills_in_pieces_and_advances_the_length(msa, gpu):
     B, h_kv, d, cap = 3, 8, 128, 100
     K = synth.normal(3, 110, (B, 87, h_kv, d), "bf16")
