@@ -143,6 +143,30 @@ def encode_pool(K, V, K_r, doc_tok_off, chunk: int, rope_base: float, L=None):
     return Kb, Vb, Rb, coff
 
 
+def encode_hidden(H, W_k, W_v, W_r, doc_tok_off, chunk: int, rope_base: float, h_kv: int,
+                  L=None):
+    """Offline encode from hidden states (reading R26 of the design notes): the per-token keys,
+    values and router keys are projections of the hidden states, K = H W_k, V = H W_v,
+    K_r = H W_r (the router K projector makes the routing keys: ruixiangma.github.io blog,
+    "稀疏注意力机制"), computed here as plain matrix products in double precision; they then
+    go through doc-wise RoPE and chunk mean pooling exactly as in ``encode_pool``.
+    H [N_tok, D] and W_* [D, h_kv * d] in one storage type (float32, or bf16 bits as uint16).
+    Returns (Kbar, Vbar, Krbar, doc_chunk_off) as ``encode_pool``."""
+    def f64(x):
+        x = np.ascontiguousarray(x)
+        if x.dtype == np.uint16:
+            return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        return x.astype(np.float64)
+
+    H64 = f64(H)
+    n = H64.shape[0]
+    d = f64(W_k).shape[1] // h_kv
+    # per-token projections, handed to the pooling in fp32 (the accumulation precision of the
+    # product; a fused kernel never rounds them to the storage type)
+    proj = [(H64 @ f64(W)).reshape(n, h_kv, d).astype(np.float32) for W in (W_k, W_v, W_r)]
+    return encode_pool(proj[0], proj[1], proj[2], doc_tok_off, chunk, rope_base, L)
+
+
 def route(Q_r, Kbar_r, doc_chunk_off, k: int, exclude_bits=None, L=None):
     """Cosine routing + top-k. Returns (top_ids int32 [B,k], top_scores f64 [B,k],
     doc_scores f64 [B, n_docs])."""

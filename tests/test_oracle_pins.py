@@ -316,6 +316,48 @@ def test_msa_with_unit_chunks_and_all_docs_is_dense_causal_attention():
     assert np.max(np.abs(O[0].transpose(1, 0, 2) - ref)) < 5e-4  # fp32 angles in the reference
 
 
+# ----------------------------------------------------------------------------- encode from H
+def _hidden_case(lens, D, h_kv, d, seed, dtype="fp32"):
+    off = np.zeros(len(lens) + 1, np.int64)
+    off[1:] = np.cumsum(lens)
+    H = synth.normal(seed, 40, (int(off[-1]), D), dtype)
+    Ws = [synth.normal(seed, 41 + i, (D, h_kv * d), dtype, scale=D ** -0.5) for i in range(3)]
+    return H, Ws, off
+
+
+def test_encode_hidden_value_path_is_the_projected_chunk_mean():
+    """V has no RoPE, so pooling commutes with the projection: V̄ = mean(H over the chunk) W_v."""
+    lens, chunk, D, h_kv, d = [5, 9, 1, 12], 4, 24, 2, 8
+    H, (Wk, Wv, Wr), off = _hidden_case(lens, D, h_kv, d, seed=31)
+    Kb, Vb, Rb, coff = oracle.encode_hidden(H, Wk, Wv, Wr, off, chunk, 1e4, h_kv)
+    c = 0
+    for i in range(len(lens)):
+        for s0 in range(int(off[i]), int(off[i + 1]), chunk):
+            s1 = min(s0 + chunk, int(off[i + 1]))
+            ref = (H[s0:s1].astype(np.float64).mean(0) @ Wv.astype(np.float64)).reshape(h_kv, d)
+            assert np.max(np.abs(Vb[c] - ref)) <= 1e-6 * (1 + np.max(np.abs(ref)))
+            c += 1
+    assert c == len(Vb) == int(coff[-1])
+
+
+def test_encode_hidden_brute_force_against_backbone_rope():
+    """Keys and router keys: each token projected, rotated at its within-document position by the
+    Qwen3 rotary embedding, then averaged per chunk."""
+    lens, chunk, D, h_kv, d, base = [3, 6], 4, 16, 2, 8, 1e4
+    H, (Wk, Wv, Wr), off = _hidden_case(lens, D, h_kv, d, seed=32)
+    Kb, Vb, Rb, coff = oracle.encode_hidden(H, Wk, Wv, Wr, off, chunk, base, h_kv)
+    for W, got in ((Wk, Kb), (Wr, Rb)):
+        c = 0
+        for i in range(len(lens)):
+            toks = (H[off[i]:off[i + 1]].astype(np.float64) @ W.astype(np.float64))
+            toks = toks.reshape(-1, h_kv, d).transpose(1, 0, 2)  # [h_kv, len, d]
+            rot = _qwen3_rope(toks, np.arange(lens[i]), base).transpose(1, 0, 2)
+            for s0 in range(0, lens[i], chunk):
+                ref = rot[s0:min(s0 + chunk, lens[i])].mean(0)
+                assert np.max(np.abs(got[c] - ref)) <= 1e-5 * (1 + np.max(np.abs(ref)))
+                c += 1
+
+
 # ----------------------------------------------------------------------------- generation
 def test_generate_token_by_token_is_causal_attention_over_the_whole_sequence():
     """Sparse generation, one token per step, must equal textbook causal attention (torch's
