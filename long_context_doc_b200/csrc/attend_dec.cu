@@ -10,14 +10,14 @@
 //
 // Kernel design (one CTA of eight warps per SM):
 //  * A tile is KT = 64 / h_kv consecutive key rows of one query with all their KV heads (16 KB
-//    of K and 16 KB of V, contiguous in the [row][KV head][d] storage order). The copy warp
+//    of K and 16 KB of V, contiguous in the [row][KV head][d] storage order). One thread
 //    moves it with four TMA boxes of [KV head][key row][64 dims] (each half of d of K and of V)
 //    whose 128-byte swizzle makes every later shared-memory read conflict-free. Per query the
 //    memory rows come first, then the local rows (a tile holds one kind). The flattened tile
 //    list of all queries is cut into one contiguous range per CTA; a 4-stage ring keeps
 //    128 KB of loads in flight per SM (an mbarrier per stage signals its copies' arrival;
 //    the last warp to release a stage, counted in shared memory, issues its next copies).
-//  * Compute warp w owns KV head w % h_kv and eight key rows of every tile, with its own online
+//  * Warp w owns KV head w % h_kv and eight key rows of every tile, with its own online
 //    softmax state; the warps meet only at the end of a query's segment (no block barrier per
 //    tile). The logits and P.V run on the tensor cores as warp-level bf16 MMAs (fp32
 //    accumulation): the query rows of the head (<= 8) are the rows of a 16-row A operand,
