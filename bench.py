@@ -26,7 +26,9 @@ built once (the default workload's step: 18 routed layers of route + host-bank g
 attention of the query token), then 256 tokens are generated per query, each through 18
 decode steps (msa_decode_step: the token's K/V appended to the layer's 2,048-row local cache,
 attention over [gathered memory ; cache]); its line reports generated tokens/s.
-``--impl reference`` times the CPU oracle on the host cores (a bounded
+``--workload encode_hidden1m`` times the offline encode from hidden states at the 1M-token bank
+(1,024 docs x 1,024 tokens, hidden size 2,560: the three projections on tcgen05 fused with
+doc-wise RoPE and chunk pooling). ``--impl reference`` times the CPU oracle on the host cores (a bounded
 sample of the same workload). Under torchrun every rank runs an independent replica
 (the path does not shard: no collective on the data path).
 """
@@ -59,7 +61,7 @@ def parse():
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
                     choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long",
-                             "gen100m"])
+                             "gen100m", "encode_hidden1m"])
     ap.add_argument("--gen-tokens", type=int, default=256,
                     help="gen100m: tokens generated per query after the context is built")
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
@@ -1187,6 +1189,74 @@ def cpu_generate_baseline(w, G: int, n_layers: int) -> dict:
                        "this overstates the CPU rate")}
 
 
+def run_encode_hidden(args):
+    """The offline encode from hidden states (msa_encode_hidden) at the 1M-token bank."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    import synth
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    rank, world = ranks.rank, ranks.world
+    w = synth.C2.scaled(seed=synth.C2.seed + 1000 * rank)
+    D, bf = 2560, torch.bfloat16
+    off = np.arange(w.n_docs + 1, dtype=np.int64) * w.doc_len
+    n_tok = int(off[-1])
+    H = synth.dev_normal(torch.empty((n_tok, D), dtype=bf, device=dev), w.seed, synth.tag(50))
+    Ws = [synth.dev_normal(torch.empty((w.h_kv * w.d, D), dtype=bf, device=dev), w.seed,
+                           synth.tag(51 + i), scale=D ** -0.5) for i in range(3)]
+    n_chunks = msa.msa_count_chunks(off, w.chunk)
+    shape = (n_chunks, w.h_kv, w.d)
+    outs = [torch.empty(shape, dtype=bf, device=dev) for _ in range(3)]
+    coff = torch.empty(len(off), dtype=torch.int64, device=dev)
+    ws = torch.empty(msa.msa_encode_hidden_workspace(n_chunks), dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream()
+
+    def call():
+        msa.msa_encode_hidden(H, *Ws, off, w.chunk, w.rope_base, *outs, coff, ws, st)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    ranks.barrier()
+    torch.cuda.synchronize()
+    Kst = max(1, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(Kst):
+        call()
+    e1.record(st)
+    st.synchronize()
+    ms, = ranks.max([e0.elapsed_time(e1) / Kst], dev)
+    assert msa.msa_workspace_status(ws, st) == 0
+    flop = 2.0 * n_tok * D * 3 * w.h_kv * w.d
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tpeak, tkind = float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        tpeak, tkind = 1400.0, "fallback (sustained)"
+    tf = flop / (ms / 1e3) / 1e12
+    line = {"metric": "offline encode from hidden states, bank tokens/s (projections + doc-wise "
+                      "RoPE + chunk pooling)",
+            "value": round(replica_rate(world, n_tok, ms), 1), "unit": "bank tokens/s",
+            "n_gpus": world, "steps": Kst, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normals; random "
+                                                          "projection weights)",
+            "config": {"workload": "encode_hidden1m", "bank_tokens": n_tok, "n_docs": w.n_docs,
+                       "hidden": D, "h_kv": w.h_kv, "d": w.d, "chunk": w.chunk,
+                       "l2": "no flush: 5.4 GB of hidden states per call"},
+            "roofline": {"kernel": "encode_hidden_kernel (tcgen05 projections + RoPE + pooling; "
+                                   "the call also uploads the chunk table)",
+                         "bound": "tensor", "achieved": round(tf, 1), "peak": tpeak,
+                         "unit": "TFLOP/s", "frac": round(tf / tpeak, 4), "peak_kind": tkind,
+                         "traffic": None}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -1199,6 +1269,8 @@ def main():
         run_attend_long(args)
     elif args.workload == "gen100m":
         run_generate(args)
+    elif args.workload == "encode_hidden1m":
+        run_encode_hidden(args)
     else:
         run_libmsa(args)
 

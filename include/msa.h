@@ -331,6 +331,33 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
                            int32_t dtype, int32_t pos0, float rope_base, float scale, void* O,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------------------
+ * msa_encode_hidden - offline memory encoding from hidden states: for every token, the key,
+ * value and router-key projections K = H W_k^T, V = H W_v^T, K_r = H W_r^T, then document-wise
+ * RoPE of K and K_r and chunk mean pooling as in msa_encode_pool, in one kernel whose epilogue
+ * works on the fp32 products (the per-token K, V, K_r are never written).
+ *   [ruixiangma.github.io blog, "稀疏注意力机制": the router K projector produces each
+ *    document's routing keys; news.neo-ai.one, "アーキテクチャ": chunk-wise mean pooling]
+ *
+ * H              [n_tok, D] bf16 hidden states of the documents, documents contiguous.
+ * W_k, W_v, W_r  [h_kv * 128, D] bf16 projection weights (output-major rows).
+ * doc_tok_off_host, n_docs, chunk, rope_base: as msa_encode_pool (chunk must be 64).
+ * Kbar, Vbar, Kbar_r [n_chunks, h_kv, 128] bf16 outputs (means of fp32 values, RNE);
+ * doc_chunk_off  [n_docs+1] int64 device output.
+ * ws             msa_encode_hidden_workspace(n_chunks) bytes, 256-byte aligned (chunk table;
+ *                the status word records an expired device wait).
+ * Supported: bf16, d = 128, chunk = 64, even h_kv, D a multiple of 64 (else
+ * MSA_ERR_UNSUPPORTED). Synchronises `stream` once (the chunk table is uploaded from the host).
+ * Inverse norms or the normalised routing bank come from msa_kr_inv_norm / msa_kr_normalize.
+ */
+size_t msa_encode_hidden_workspace(int64_t n_chunks);
+msa_status msa_encode_hidden(const void* H, int64_t n_tok, int32_t D, const void* W_k,
+                             const void* W_v, const void* W_r, const int64_t* doc_tok_off_host,
+                             int64_t n_docs, int32_t chunk, int32_t h_kv, int32_t d,
+                             int32_t dtype, float rope_base, void* Kbar, void* Vbar,
+                             void* Kbar_r, int64_t* doc_chunk_off, int64_t n_chunks, void* ws,
+                             size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,8 @@ SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chun
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
            "msa_sparse_attend", "msa_assemble_local", "msa_kv_append",
-           "msa_decode_step_workspace", "msa_decode_step")
+           "msa_decode_step_workspace", "msa_decode_step", "msa_encode_hidden_workspace",
+           "msa_encode_hidden")
 
 
 class MSAError(RuntimeError):
@@ -97,6 +98,11 @@ def _load():
                                 vp]
     L.msa_decode_step_workspace.restype = sz
     L.msa_decode_step_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    L.msa_encode_hidden_workspace.restype = sz
+    L.msa_encode_hidden_workspace.argtypes = [i64]
+    L.msa_encode_hidden.restype = ctypes.c_int
+    L.msa_encode_hidden.argtypes = [vp, i64, i32, vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
+                                    vp, vp, vp, i64, vp, sz, vp]
     L.msa_decode_step.restype = ctypes.c_int
     L.msa_decode_step.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32, i32,
                                   i32, i32, i32, f32, f32, vp, vp, sz, vp]
@@ -146,6 +152,42 @@ def msa_encode_pool(K, V, K_r, doc_tok_off_host, doc_tok_off, chunk, rope_base, 
                                _p(doc_tok_off), len(off) - 1, chunk, K.shape[1], K.shape[2],
                                dtype_code(K), rope_base, _p(Kbar), _p(Vbar), _p(Kbar_r),
                                _p(kr_inv_norm), _p(doc_chunk_off), Kbar.shape[0], _s(stream)))
+
+
+def msa_encode_hidden(H, W_k, W_v, W_r, doc_tok_off_host, chunk, rope_base, Kbar, Vbar, Kbar_r,
+                      doc_chunk_off, ws, stream=None):
+    """H [n_tok, D]; W_* [h_kv * 128, D]; outputs [n_chunks, h_kv, 128] and doc_chunk_off."""
+    off = np.ascontiguousarray(doc_tok_off_host, dtype=np.int64)
+    n_tok, D = H.shape
+    _check(lib.msa_encode_hidden(_p(H), n_tok, D, _p(W_k), _p(W_v), _p(W_r), off.ctypes.data,
+                                 len(off) - 1, chunk, Kbar.shape[1], Kbar.shape[2],
+                                 dtype_code(H), rope_base, _p(Kbar), _p(Vbar), _p(Kbar_r),
+                                 _p(doc_chunk_off), Kbar.shape[0], _p(ws),
+                                 ws.numel() * ws.element_size(), _s(stream)))
+
+
+def encode_hidden(H, W_k, W_v, W_r, doc_tok_off_host, chunk: int, rope_base: float, h_kv: int,
+                  stream=None):
+    """Projections of the hidden states fused with doc-wise RoPE + chunk pooling. Returns
+    dict(Kbar, Vbar, Kbar_r, doc_chunk_off)."""
+    dev = H.device
+    off = np.ascontiguousarray(doc_tok_off_host, dtype=np.int64)
+    n_chunks = msa_count_chunks(off, chunk)
+    if n_chunks < 0:
+        raise MSAError(1, "invalid document offsets")
+    shape = (n_chunks, h_kv, W_k.shape[0] // h_kv)
+    out = dict(Kbar=torch.empty(shape, dtype=H.dtype, device=dev),
+               Vbar=torch.empty(shape, dtype=H.dtype, device=dev),
+               Kbar_r=torch.empty(shape, dtype=H.dtype, device=dev),
+               doc_chunk_off=torch.empty(len(off), dtype=torch.int64, device=dev))
+    ws = _ws(msa_encode_hidden_workspace(n_chunks), dev)
+    msa_encode_hidden(H, W_k, W_v, W_r, off, chunk, rope_base, out["Kbar"], out["Vbar"],
+                      out["Kbar_r"], out["doc_chunk_off"], ws, stream)
+    return out
+
+
+def msa_encode_hidden_workspace(n_chunks) -> int:
+    return int(lib.msa_encode_hidden_workspace(n_chunks))
 
 
 def msa_kr_inv_norm(Kbar_r, out, stream=None):

@@ -821,4 +821,84 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
   return ok();
 }
 
+// ------------------------------------------------------------------ encode from hidden states
+size_t msa_encode_hidden_workspace(int64_t n_chunks) {
+  if (n_chunks < 0) return kHeader;
+  return kHeader + (((size_t)n_chunks * 3 * sizeof(int32_t) + 255) & ~(size_t)255);
+}
+
+msa_status msa_encode_hidden(const void* H, int64_t n_tok, int32_t D, const void* W_k,
+                             const void* W_v, const void* W_r, const int64_t* doc_tok_off_host,
+                             int64_t n_docs, int32_t chunk, int32_t h_kv, int32_t d,
+                             int32_t dtype, float rope_base, void* Kbar, void* Vbar,
+                             void* Kbar_r, int64_t* doc_chunk_off, int64_t n_chunks, void* ws,
+                             size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(dtype == MSA_BF16 && d == 128 && chunk == 64 && h_kv % 2 == 0 && h_kv <= 64,
+          MSA_ERR_UNSUPPORTED, "encode from hidden states: bf16, d = 128, chunk = 64, even h_kv");
+  REQUIRE(D >= 64 && D % 64 == 0, MSA_ERR_UNSUPPORTED, "hidden size %d (a multiple of 64)", D);
+  REQUIRE(n_docs >= 0 && n_tok >= 0 && n_chunks >= 0 && n_tok < (1ll << 31), MSA_ERR_INVALID_ARG,
+          "bad sizes (n_tok=%lld n_docs=%lld)", (long long)n_tok, (long long)n_docs);
+  REQUIRE(doc_tok_off_host && doc_chunk_off, MSA_ERR_INVALID_ARG, "null offset pointer");
+  REQUIRE(doc_tok_off_host[n_docs] == n_tok, MSA_ERR_INVALID_ARG,
+          "doc_tok_off[n_docs] = %lld != n_tok %lld", (long long)doc_tok_off_host[n_docs],
+          (long long)n_tok);
+  const int64_t nc = msa_count_chunks(doc_tok_off_host, n_docs, chunk);
+  REQUIRE(nc >= 0, MSA_ERR_INVALID_ARG, "doc_tok_off must start at 0 and not decrease");
+  REQUIRE(nc == n_chunks, MSA_ERR_INVALID_ARG, "n_chunks %lld != %lld implied by the offsets",
+          (long long)n_chunks, (long long)nc);
+  const size_t need = msa_encode_hidden_workspace(n_chunks);
+  REQUIRE(ws && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+  if (n_chunks > 0) {
+    REQUIRE(H && W_k && W_v && W_r && Kbar && Vbar && Kbar_r, MSA_ERR_INVALID_ARG,
+            "null tensor");
+    REQUIRE(aligned16(H) && aligned16(W_k) && aligned16(W_v) && aligned16(W_r) &&
+                aligned16(Kbar) && aligned16(Vbar) && aligned16(Kbar_r),
+            MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  }
+  // chunk table [first token row, valid rows, position of the first row in its document] and
+  // the chunk offsets, from the host offsets
+  std::vector<int32_t> tab((size_t)n_chunks * 3);
+  std::vector<int64_t> coff((size_t)n_docs + 1);
+  int64_t c = 0;
+  for (int64_t i = 0; i < n_docs; ++i) {
+    coff[i] = c;
+    for (int64_t s0 = doc_tok_off_host[i]; s0 < doc_tok_off_host[i + 1]; s0 += chunk, ++c) {
+      tab[3 * c] = (int32_t)s0;
+      tab[3 * c + 1] = (int32_t)std::min<int64_t>(chunk, doc_tok_off_host[i + 1] - s0);
+      tab[3 * c + 2] = (int32_t)(s0 - doc_tok_off_host[i]);
+    }
+  }
+  coff[n_docs] = c;
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned char* w8 = static_cast<unsigned char*>(ws);
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess && n_chunks > 0)
+    e = cudaMemcpyAsync(w8 + kHeader, tab.data(), tab.size() * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(doc_chunk_off, coff.data(), coff.size() * sizeof(int64_t),
+                        cudaMemcpyHostToDevice, st);
+  msa::EhParams p{};
+  p.n_chunks = n_chunks;
+  p.n_tiles = h_kv / 2;
+  p.n_units = ((n_chunks + 1) / 2) * 3 * p.n_tiles;
+  p.D = D;
+  p.h_kv = h_kv;
+  p.ctab = reinterpret_cast<const int32_t*>(w8 + kHeader);
+  p.rope = rope_base > 0.f ? 1 : 0;
+  msa::rope_turns(p.rope ? (double)rope_base : 0.0, d, p.rope_turns);
+  p.Kbar = static_cast<__nv_bfloat16*>(Kbar);
+  p.Vbar = static_cast<__nv_bfloat16*>(Vbar);
+  p.Kbar_r = static_cast<__nv_bfloat16*>(Kbar_r);
+  p.err = reinterpret_cast<int*>(w8);
+  if (e == cudaSuccess) e = msa::launch_encode_hidden(p, H, n_tok, W_k, W_v, W_r, sm_count(), st);
+  // the host tables above are sources of the copies: they must outlive them
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_encode_hidden");
+  return ok();
+}
+
 }  // extern "C"

@@ -171,6 +171,25 @@ DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int
 DecPlan attend_dec_plan_cap(int B, int T, int h_q, int h_kv, int d, int max_ctx, int cap, int sms);
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
 
+// ---- encode_hidden.cu: projections of hidden states fused with doc-wise RoPE + pooling
+struct EhParams {
+  int64_t n_chunks, n_units;   // units = ceil(n_chunks / 2) x 3 projections x n_tiles
+  int n_tiles;                 // head pairs: h_kv / 2
+  int D, h_kv;                 // hidden size (multiple of 64), KV heads (even); d = 128
+  const int32_t* ctab;         // [n_chunks][3]: first token row, valid rows, position of the
+                               // first row within its document
+  int rope;
+  unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1, 64-bit fixed point
+  __nv_bfloat16* Kbar;         // [n_chunks, h_kv, 128]
+  __nv_bfloat16* Vbar;
+  __nv_bfloat16* Kbar_r;
+  int* err;                    // workspace status word
+};
+size_t encode_hidden_smem();
+cudaError_t launch_encode_hidden(const EhParams& p, const void* H, int64_t n_tok,
+                                 const void* Wk, const void* Wv, const void* Wr, int sms,
+                                 cudaStream_t st);
+
 // ---- assemble.cu: local context of a Memory Interleaving round
 struct AssembleParams {
   int B, n_seg, T;
