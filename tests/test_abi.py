@@ -176,3 +176,24 @@ def test_generation_entry_points_reject_bad_arguments_on_host(msa):
     assert step(cap=0) == 1             # capacity below T
     assert step(ws_bytes=need - 1) == 3
     assert step(L=None) == 1            # no device length
+
+
+def test_encode_hidden_rejects_bad_arguments_on_host(msa):
+    import numpy as np
+    fake = ctypes.c_void_p(256)
+    off = np.array([0, 70, 80], np.int64)
+    ws_bytes = msa.msa_encode_hidden_workspace(3)
+    assert ws_bytes >= 256 + 3 * 12
+    ws = ctypes.c_void_p(512)
+
+    def call(D=256, chunk=64, h_kv=2, d=128, dtype=1, n_chunks=3, wsb=ws_bytes, offs=off):
+        return msa.lib.msa_encode_hidden(fake, int(offs[-1]), D, fake, fake, fake,
+                                         offs.ctypes.data, len(offs) - 1, chunk, h_kv, d, dtype,
+                                         1e6, fake, fake, fake, fake, n_chunks, ws, wsb, None)
+    assert call(dtype=0) == 2          # fp32
+    assert call(chunk=32) == 2         # chunk must be 64
+    assert call(h_kv=3) == 2           # odd KV heads
+    assert call(D=100) == 2            # hidden size not a multiple of 64
+    assert call(n_chunks=4) == 1       # inconsistent with the offsets
+    assert call(offs=np.array([0, 70, 60], np.int64)) == 1  # decreasing offsets
+    assert call(wsb=ws_bytes - 1) == 3
