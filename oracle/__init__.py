@@ -53,6 +53,9 @@ def _declare(L):
     L.orc_attend.restype = i32
     L.orc_attend.argtypes = [i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32, i32, i32,
                              i32, dbl, dbl, vp]
+    L.orc_attend_backward.restype = i32
+    L.orc_attend_backward.argtypes = [i32, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32,
+                                      i32, i32, i32, dbl, dbl, vp, vp, vp, vp, vp, vp]
     return L
 
 
@@ -214,6 +217,40 @@ def attend(Q, K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0: int, rope_bas
     if r != 0:
         raise ValueError("orc_attend: invalid arguments")
     return O
+
+
+def attend_backward(Q, K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0: int,
+                    rope_base: float, dO, scale: float = 0.0, L=None) -> dict:
+    """Gradients of ``attend`` w.r.t. its inputs for an output gradient dO [B, T, h_q, d]
+    (reverse mode of the same arithmetic, double precision). Returns dict(dQ, dK_loc, dV_loc,
+    dK_ctx, dV_ctx, dKbar, dVbar): dK_ctx/dV_ctx [B, max_ctx, h_kv, d] per gathered row,
+    dKbar/dVbar the same scattered into the bank rows (summed over the queries that gathered
+    them). Routing itself (top-k) has no gradient."""
+    Q, K_loc, V_loc, Kbar, Vbar = map(_c, (Q, K_loc, V_loc, Kbar, Vbar))
+    B, T, h_q, d = Q.shape
+    Lloc, h_kv = K_loc.shape[1], K_loc.shape[2]
+    gi = np.ascontiguousarray(gather_idx, dtype=np.int32)
+    cl = np.ascontiguousarray(ctx_len, dtype=np.int32)
+    max_ctx = gi.shape[1]
+    g_o = np.ascontiguousarray(dO, dtype=np.float64)
+    out = dict(dQ=np.empty((B, T, h_q, d)), dK_loc=np.empty((B, Lloc, h_kv, d)),
+               dV_loc=np.empty((B, Lloc, h_kv, d)), dK_ctx=np.empty((B, max_ctx, h_kv, d)),
+               dV_ctx=np.empty((B, max_ctx, h_kv, d)))
+    r = (L or lib()).orc_attend_backward(
+        _same(Q, K_loc, V_loc, Kbar, Vbar), _p(Q), B, T, h_q, _p(K_loc), _p(V_loc), Lloc,
+        _p(Kbar), _p(Vbar), _p(gi), _p(cl), max_ctx, h_kv, d, int(pos0), float(rope_base),
+        float(scale), _p(g_o), _p(out["dQ"]), _p(out["dK_loc"]), _p(out["dV_loc"]),
+        _p(out["dK_ctx"]), _p(out["dV_ctx"]))
+    if r != 0:
+        raise ValueError("orc_attend_backward: invalid arguments")
+    dKb = np.zeros(Kbar.shape)
+    dVb = np.zeros(Vbar.shape)
+    for b in range(B):
+        for j in range(int(cl[b])):
+            dKb[gi[b, j]] += out["dK_ctx"][b, j]
+            dVb[gi[b, j]] += out["dV_ctx"][b, j]
+    out.update(dKbar=dKb, dVbar=dVb)
+    return out
 
 
 def pipeline(w, inp: dict, L=None) -> dict:

@@ -377,3 +377,144 @@ int orc_attend(int dtype, const void* Q, int B, int T, int h_q, const void* K_lo
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------- its gradients
+ * Reverse mode of orc_attend, for training the routed layer: continued pre-training uses the
+ * standard generation loss through the sparse attention plus an auxiliary routing loss
+ * [C, 训练策略 "连续预训练阶段"].
+ * Given dO [B, T, h_q, d] (double), writes (double, zeroed here):
+ *   dQ [B, T, h_q, d]; dK_loc, dV_loc [B, L, h_kv, d] (w.r.t. the pre-RoPE local keys);
+ *   dK_ctx, dV_ctx [B, max_ctx, h_kv, d] w.r.t. the gathered memory rows as used (row j of
+ *   query b is bank row gather_idx[b, j]; rows j >= ctx_len[b] get zero).
+ * Per query row: P = softmax(scale q k^T) over the visible rows, dV_j += P_j dO,
+ * dP_j = dO . v_j, dS_j = P_j (dP_j - sum_i P_i dP_i), dq_rot = scale sum_j dS_j k_j,
+ * dk_j += scale dS_j q_rot; rotated vectors go back through the inverse rotation (RoPE is
+ * orthogonal: the rotation by -pos). Sequential over query rows (small cases). Returns 0 or -1. */
+int orc_attend_backward(int dtype, const void* Q, int B, int T, int h_q, const void* K_loc,
+                        const void* V_loc, int L, const void* Kbar, const void* Vbar,
+                        const int32_t* gather_idx, const int32_t* ctx_len, int max_ctx, int h_kv,
+                        int d, int pos0, double rope_base, double scale, const double* dO,
+                        double* dQ, double* dK_loc, double* dV_loc, double* dK_ctx,
+                        double* dV_ctx) {
+    if (T <= 0 || L < T || h_q <= 0 || h_kv <= 0 || h_q % h_kv || d <= 0 || (d & 1)) return -1;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    int grp = h_q / h_kv;
+    memset(dQ, 0, sizeof(double) * (size_t)B * T * h_q * d);
+    memset(dK_loc, 0, sizeof(double) * (size_t)B * L * h_kv * d);
+    memset(dV_loc, 0, sizeof(double) * (size_t)B * L * h_kv * d);
+    memset(dK_ctx, 0, sizeof(double) * (size_t)B * max_ctx * h_kv * d);
+    memset(dV_ctx, 0, sizeof(double) * (size_t)B * max_ctx * h_kv * d);
+    double* q = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dq = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int b = 0; b < B; ++b) {
+        int n_ctx = ctx_len[b];
+        if (n_ctx < 0 || n_ctx > max_ctx) { free(q); free(dq); return -1; }
+        int n_max = n_ctx + L;
+        /* rotated local keys and their (rotated) gradients */
+        double* kl = (double*)malloc(sizeof(double) * (size_t)L * h_kv * d);
+        double* dkl = (double*)calloc((size_t)L * h_kv * d, sizeof(double));
+        double* p = (double*)malloc(sizeof(double) * (size_t)n_max);
+        double* dp = (double*)malloc(sizeof(double) * (size_t)n_max);
+        for (int64_t j = 0; j < L; ++j)
+            for (int g = 0; g < h_kv; ++g) {
+                double* r = kl + (j * h_kv + g) * d;
+                for (int e = 0; e < d; ++e)
+                    r[e] = orc_at(K_loc, dtype, (((int64_t)b * L + j) * h_kv + g) * d + e);
+                orc_rope(r, d, (double)pos0 + (double)j, rope_base);
+            }
+        for (int t = 0; t < T; ++t)
+            for (int h = 0; h < h_q; ++h) {
+                int g = h / grp;
+                int64_t qi = (int64_t)L - T + t;
+                const double pos = (double)pos0 + (double)qi;
+                for (int e = 0; e < d; ++e)
+                    q[e] = orc_at(Q, dtype, (((int64_t)b * T + t) * h_q + h) * d + e);
+                orc_rope(q, d, pos, rope_base);
+                const double* go = dO + (((int64_t)b * T + t) * h_q + h) * d;
+                /* forward again: logits, softmax */
+                int n = 0;
+                double mx = -INFINITY;
+                for (int j = 0; j < n_ctx; ++j, ++n) {
+                    int64_t c = gather_idx[(int64_t)b * max_ctx + j];
+                    double sdot = 0.0;
+                    for (int e = 0; e < d; ++e)
+                        sdot += q[e] * orc_at(Kbar, dtype, (c * h_kv + g) * (int64_t)d + e);
+                    p[n] = sdot * scale;
+                    if (p[n] > mx) mx = p[n];
+                }
+                for (int64_t j = 0; j <= qi; ++j, ++n) {
+                    const double* r = kl + (j * h_kv + g) * d;
+                    double sdot = 0.0;
+                    for (int e = 0; e < d; ++e) sdot += q[e] * r[e];
+                    p[n] = sdot * scale;
+                    if (p[n] > mx) mx = p[n];
+                }
+                double den = 0.0;
+                for (int j = 0; j < n; ++j) { p[j] = exp(p[j] - mx); den += p[j]; }
+                for (int j = 0; j < n; ++j) p[j] /= den;
+                /* dV, dP and their weighted sum */
+                double dsum = 0.0;
+                n = 0;
+                for (int j = 0; j < n_ctx; ++j, ++n) {
+                    int64_t c = gather_idx[(int64_t)b * max_ctx + j];
+                    double* gv = dV_ctx + (((int64_t)b * max_ctx + j) * h_kv + g) * d;
+                    double acc = 0.0;
+                    for (int e = 0; e < d; ++e) {
+                        gv[e] += p[n] * go[e];
+                        acc += go[e] * orc_at(Vbar, dtype, (c * h_kv + g) * (int64_t)d + e);
+                    }
+                    dp[n] = acc;
+                    dsum += p[n] * acc;
+                }
+                for (int64_t j = 0; j <= qi; ++j, ++n) {
+                    double* gv = dV_loc + (((int64_t)b * L + j) * h_kv + g) * d;
+                    double acc = 0.0;
+                    for (int e = 0; e < d; ++e) {
+                        gv[e] += p[n] * go[e];
+                        acc += go[e] *
+                               orc_at(V_loc, dtype, (((int64_t)b * L + j) * h_kv + g) * d + e);
+                    }
+                    dp[n] = acc;
+                    dsum += p[n] * acc;
+                }
+                /* dS, then the query and key gradients (rotated frame) */
+                for (int e = 0; e < d; ++e) dq[e] = 0.0;
+                n = 0;
+                for (int j = 0; j < n_ctx; ++j, ++n) {
+                    int64_t c = gather_idx[(int64_t)b * max_ctx + j];
+                    const double ds = p[n] * (dp[n] - dsum) * scale;
+                    double* gk = dK_ctx + (((int64_t)b * max_ctx + j) * h_kv + g) * d;
+                    for (int e = 0; e < d; ++e) {
+                        dq[e] += ds * orc_at(Kbar, dtype, (c * h_kv + g) * (int64_t)d + e);
+                        gk[e] += ds * q[e];
+                    }
+                }
+                for (int64_t j = 0; j <= qi; ++j, ++n) {
+                    const double ds = p[n] * (dp[n] - dsum) * scale;
+                    const double* r = kl + (j * h_kv + g) * d;
+                    double* gk = dkl + (j * h_kv + g) * d;
+                    for (int e = 0; e < d; ++e) {
+                        dq[e] += ds * r[e];
+                        gk[e] += ds * q[e];
+                    }
+                }
+                orc_rope(dq, d, -pos, rope_base); /* back through R(pos theta) */
+                double* gq = dQ + (((int64_t)b * T + t) * h_q + h) * d;
+                for (int e = 0; e < d; ++e) gq[e] = dq[e];
+            }
+        for (int64_t j = 0; j < L; ++j)
+            for (int g = 0; g < h_kv; ++g) {
+                double* r = dkl + (j * h_kv + g) * d;
+                orc_rope(r, d, -((double)pos0 + (double)j), rope_base);
+                double* gk = dK_loc + (((int64_t)b * L + j) * h_kv + g) * d;
+                for (int e = 0; e < d; ++e) gk[e] = r[e];
+            }
+        free(kl);
+        free(dkl);
+        free(p);
+        free(dp);
+    }
+    free(q);
+    free(dq);
+    return 0;
+}

@@ -437,3 +437,87 @@ def test_bf16_rounding_is_round_to_nearest_even():
     # a double just above a midpoint rounds up (no double rounding through fp32)
     assert oracle.round_bf16(np.array([1.0 + 2 ** -8 + 2 ** -30]))[0] == 0x3F81
     assert oracle.round_bf16(np.array([-(1.0 + 2 ** -8 + 2 ** -30)]))[0] == 0xBF81
+
+
+# ----------------------------------------------------------------------------- backward
+def _bw_case(seed, B=2, T=3, h_q=4, h_kv=2, d=8, L=6, n_bank=7, max_ctx=4, ctx=(3, 0)):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((B, T, h_q, d)).astype(np.float32)
+    Kl = rng.standard_normal((B, L, h_kv, d)).astype(np.float32)
+    Vl = rng.standard_normal((B, L, h_kv, d)).astype(np.float32)
+    Kb = rng.standard_normal((n_bank, h_kv, d)).astype(np.float32)
+    Vb = rng.standard_normal((n_bank, h_kv, d)).astype(np.float32)
+    gi = np.full((B, max_ctx), -1, np.int32)
+    for b in range(B):
+        gi[b, :ctx[b]] = rng.choice(n_bank, ctx[b], replace=False)
+    cl = np.array(ctx, np.int32)
+    dO = rng.standard_normal((B, T, h_q, d))
+    return Q, Kl, Vl, Kb, Vb, gi, cl, dO
+
+
+def test_attend_backward_matches_central_differences():
+    """<dO, dO/dx . delta> from the reverse mode equals the central difference of the forward
+    oracle along a random delta, for every input."""
+    Q, Kl, Vl, Kb, Vb, gi, cl, dO = _bw_case(41)
+    pos0, base = 3, 1e4
+    g = oracle.attend_backward(Q, Kl, Vl, Kb, Vb, gi, cl, pos0, base, dO)
+    rng = np.random.default_rng(42)
+    args = dict(Q=Q, K_loc=Kl, V_loc=Vl, Kbar=Kb, Vbar=Vb)
+    grads = dict(Q=g["dQ"], K_loc=g["dK_loc"], V_loc=g["dV_loc"], Kbar=g["dKbar"], Vbar=g["dVbar"])
+    eps = 1e-2
+    for name, x in args.items():
+        delta = rng.standard_normal(x.shape).astype(np.float32)
+        hi = dict(args, **{name: (x.astype(np.float64) + eps * delta).astype(np.float32)})
+        lo = dict(args, **{name: (x.astype(np.float64) - eps * delta).astype(np.float32)})
+        o_hi = oracle.attend(hi["Q"], hi["K_loc"], hi["V_loc"], hi["Kbar"], hi["Vbar"], gi, cl,
+                             pos0, base)
+        o_lo = oracle.attend(lo["Q"], lo["K_loc"], lo["V_loc"], lo["Kbar"], lo["Vbar"], gi, cl,
+                             pos0, base)
+        fd = np.sum(dO * (o_hi - o_lo)) / (2 * eps)
+        an = np.sum(grads[name] * delta)
+        assert abs(fd - an) <= 2e-3 * (1 + abs(an)), (name, fd, an)
+
+
+def test_attend_backward_matches_autograd_of_sdpa():
+    """Gradients against torch autograd of an independent forward: transformers' Qwen3 rotary
+    embedding and scaled_dot_product_attention over [memory rows as stored ; rotated causal
+    local rows], GQA by repeating the KV heads."""
+    import torch.nn.functional as F
+    Q, Kl, Vl, Kb, Vb, gi, cl, dO = _bw_case(43, B=1, ctx=(3,))
+    B, T, h_q, d = Q.shape
+    L, h_kv = Kl.shape[1], Kl.shape[2]
+    pos0, base = 5, 1e4
+    g = oracle.attend_backward(Q, Kl, Vl, Kb, Vb, gi, cl, pos0, base, dO)
+    from transformers import Qwen3Config
+    from transformers.models.qwen3.modeling_qwen3 import Qwen3RotaryEmbedding, apply_rotary_pos_emb
+    cfg = Qwen3Config(hidden_size=d * 2, num_attention_heads=2, num_key_value_heads=2,
+                      head_dim=d, rope_theta=base)
+    re_ = Qwen3RotaryEmbedding(cfg)
+
+    def rot(x, pos):  # x [heads, n, d]
+        cos, sin = re_(x, torch.as_tensor(pos, dtype=torch.int64)[None])
+        out, _ = apply_rotary_pos_emb(x[None], x[None], cos, sin, unsqueeze_dim=1)
+        return out[0]
+
+    q = torch.tensor(Q[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    kl = torch.tensor(Kl[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    vl = torch.tensor(Vl[0].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    n_mem = int(cl[0])
+    km = torch.tensor(Kb[gi[0, :n_mem]].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    vm = torch.tensor(Vb[gi[0, :n_mem]].transpose(1, 0, 2), dtype=torch.float64, requires_grad=True)
+    qr = rot(q, pos0 + L - T + np.arange(T))
+    klr = rot(kl, pos0 + np.arange(L))
+    keys = torch.cat([km, klr], 1).repeat_interleave(h_q // h_kv, 0)
+    vals = torch.cat([vm, vl], 1).repeat_interleave(h_q // h_kv, 0)
+    mask = torch.ones((T, n_mem + L), dtype=torch.bool)
+    for t in range(T):
+        mask[t, n_mem + L - T + t + 1:] = False
+    out = F.scaled_dot_product_attention(qr, keys, vals, attn_mask=mask)
+    out.backward(torch.tensor(dO[0].transpose(1, 0, 2)))
+    tol = 1e-5
+    assert np.max(np.abs(q.grad.numpy().transpose(1, 0, 2) - g["dQ"][0])) < tol
+    assert np.max(np.abs(kl.grad.numpy().transpose(1, 0, 2) - g["dK_loc"][0])) < tol
+    assert np.max(np.abs(vl.grad.numpy().transpose(1, 0, 2) - g["dV_loc"][0])) < tol
+    assert np.max(np.abs(km.grad.numpy().transpose(1, 0, 2) - g["dK_ctx"][0, :n_mem])) < tol
+    assert np.max(np.abs(vm.grad.numpy().transpose(1, 0, 2) - g["dV_ctx"][0, :n_mem])) < tol
+    assert not g["dK_ctx"][0, n_mem:].any() and not g["dV_ctx"][0, n_mem:].any()
