@@ -1222,12 +1222,16 @@ def run_encode_hidden(args):
     ranks.barrier()
     torch.cuda.synchronize()
     Kst = max(1, min(args.steps, 20))
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
     for _ in range(Kst):
         call()
     e1.record(st)
     st.synchronize()
+    clocks = sampler.stop()
     ms, = ranks.max([e0.elapsed_time(e1) / Kst], dev)
     assert msa.msa_workspace_status(ws, st) == 0
     flop = 2.0 * n_tok * D * 3 * w.h_kv * w.d
@@ -1251,10 +1255,31 @@ def run_encode_hidden(args):
                                    "the call also uploads the chunk table)",
                          "bound": "tensor", "achieved": round(tf, 1), "peak": tpeak,
                          "unit": "TFLOP/s", "frac": round(tf / tpeak, 4), "peak_kind": tkind,
-                         "traffic": None}}
+                         "traffic": None},
+            "gpu_launches": Kst, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_encode_hidden_baseline(w, D)
     if rank == 0:
         print(json.dumps(line), flush=True)
     ranks.close()
+
+
+def cpu_encode_hidden_baseline(w, D: int, n_docs: int = 8) -> dict:
+    """The oracle's encode from hidden states on a sample of the same workload: ``n_docs``
+    documents of the bank (their hidden rows, the three projections, RoPE, pooling)."""
+    import oracle
+    import synth
+    off = np.arange(n_docs + 1, dtype=np.int64) * w.doc_len
+    n = int(off[-1])
+    H = synth.normal(w.seed, synth.tag(50), (n, D), "bf16")
+    Wt = [np.ascontiguousarray(synth.normal(w.seed, synth.tag(51 + i), (w.h_kv * w.d, D), "bf16",
+                                            scale=D ** -0.5).T) for i in range(3)]
+    t0 = time.perf_counter()
+    oracle.encode_hidden(H, Wt[0], Wt[1], Wt[2], off, w.chunk, w.rope_base, w.h_kv)
+    dt = time.perf_counter() - t0
+    return {"value": round(n / dt, 1), "unit": "bank tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{n_docs} of {w.n_docs} documents ({n} tokens), "
+                                        "projections + RoPE + pooling"}
 
 
 def main():
