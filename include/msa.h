@@ -29,7 +29,8 @@
  *    workspace whose size the matching *_workspace() query returns (256-byte aligned).
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). All
  *    device work is asynchronous on that stream. The only host waits are in
- *    msa_fetch_finish (bounded by timeout_ms) and msa_workspace_status.
+ *    msa_fetch_finish (bounded by timeout_ms), msa_workspace_status and the offline
+ *    msa_encode_hidden (one stream synchronisation after uploading its chunk table).
  *  - dtype: MSA_FP32 (float) or MSA_BF16 (bfloat16 bit patterns); all floating tensors of
  *    one call share it, except the fp32 inverse norms and scores.
  *  - Supported shapes: d in {64, 128}; h_q % h_kv == 0; h_qr % h_kv == 0; 1 <= k <= 32;
