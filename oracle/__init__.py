@@ -253,6 +253,54 @@ def attend_backward(Q, K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0: int,
     return out
 
 
+def aux_routing_loss(Q_r, Kbar_r, positive, tau: float = 0.1):
+    """Auxiliary routing loss (reading R27 of the design notes: the pages name a supervised
+    contrastive loss that separates relevant from irrelevant document chunks but give no
+    formula, so this function's parity with the authors' loss is unpinned).
+
+    Chunk scores as in routing before the document maximum: s[b, c] = max over query tokens t of
+    the mean over router heads h of cos(Q_r[b, t, h], Kbar_r[c, g(h)]), g(h) = h // (h_qr/h_kv).
+    Positives positive[b, c] (bool): the chunks of the query's relevant documents. Loss per query
+    = -mean over positives c of log softmax_c(s[b, :] / tau); averaged over the queries that
+    have positives. Returns (loss, dQ_r, dKbar_r) in float64; the maximum over tokens passes its
+    gradient to the first maximising token."""
+    Q = np.asarray(Q_r, dtype=np.float64)
+    K = np.asarray(Kbar_r, dtype=np.float64)
+    pos = np.asarray(positive, dtype=bool)
+    B, T, h_qr, d = Q.shape
+    n, h_kv = K.shape[0], K.shape[1]
+    grp = h_qr // h_kv
+    qn = np.linalg.norm(Q, axis=-1, keepdims=True)
+    kn = np.linalg.norm(K, axis=-1, keepdims=True)
+    qh = np.where(qn > 0, Q / np.where(qn > 0, qn, 1), 0.0)      # [B, T, h_qr, d]
+    kh = np.where(kn > 0, K / np.where(kn > 0, kn, 1), 0.0)      # [n, h_kv, d]
+    kg = kh[:, np.arange(h_qr) // grp]                          # [n, h_qr, d]
+    cos = np.einsum("bthd,chd->btch", qh, kg)                   # [B, T, n, h_qr]
+    s_t = cos.mean(-1)                                          # [B, T, n]
+    arg = s_t.argmax(1)                                         # [B, n] first maximising token
+    s = np.take_along_axis(s_t, arg[:, None, :], 1)[:, 0]       # [B, n]
+    loss, dQ, dK = 0.0, np.zeros_like(Q), np.zeros_like(K)
+    rows = [b for b in range(B) if pos[b].any()]
+    for b in rows:
+        z = s[b] / tau
+        z = z - z.max()
+        p = np.exp(z) / np.exp(z).sum()
+        P = pos[b]
+        loss += -np.mean(np.log(p[P]))
+        ds = (p - P / P.sum()) / tau / len(rows)                # d loss / d s[b, c]
+        for c in range(n):
+            t = arg[b, c]
+            for h in range(h_qr):
+                g = h // grp
+                # d cos(q, k) / d q = (k_hat - cos q_hat) / |q|, and symmetrically for k
+                w = ds[c] / h_qr
+                if qn[b, t, h, 0] > 0 and kn[c, g, 0] > 0:
+                    cq = cos[b, t, c, h]
+                    dQ[b, t, h] += w * (kg[c, h] - cq * qh[b, t, h]) / qn[b, t, h, 0]
+                    dK[c, g] += w * (qh[b, t, h] - cq * kh[c, g]) / kn[c, g, 0]
+    return loss / max(len(rows), 1), dQ, dK
+
+
 def pipeline(w, inp: dict, L=None) -> dict:
     """Oracle of one routed layer: (encode →) route → gather → attend, with the storage
     rounding of the configuration between steps. ``inp`` comes from synth."""

@@ -521,3 +521,45 @@ def test_attend_backward_matches_autograd_of_sdpa():
     assert np.max(np.abs(km.grad.numpy().transpose(1, 0, 2) - g["dK_ctx"][0, :n_mem])) < tol
     assert np.max(np.abs(vm.grad.numpy().transpose(1, 0, 2) - g["dV_ctx"][0, :n_mem])) < tol
     assert not g["dK_ctx"][0, n_mem:].any() and not g["dV_ctx"][0, n_mem:].any()
+
+
+# ----------------------------------------------------------------------------- aux routing loss
+def test_aux_routing_loss_equal_scores_is_log_n():
+    """All chunks score alike: the softmax is uniform, the loss is log(n_chunks) whatever the
+    positives."""
+    n, h_kv, d = 9, 2, 8
+    K = np.tile(np.random.default_rng(44).standard_normal((1, h_kv, d)), (n, 1, 1))
+    Q = np.random.default_rng(45).standard_normal((2, 3, h_kv, d))
+    pos = np.zeros((2, n), bool)
+    pos[0, [1, 4]] = True
+    pos[1, 7] = True
+    loss, _, _ = oracle.aux_routing_loss(Q, K, pos)
+    assert abs(loss - np.log(n)) < 1e-12
+
+
+def test_aux_routing_loss_gradients_match_autograd():
+    """Loss and gradients against torch autograd of an independent forward
+    (F.cosine_similarity, amax over tokens, log_softmax)."""
+    import torch.nn.functional as F
+    rng = np.random.default_rng(46)
+    B, T, h_qr, h_kv, d, n = 2, 3, 4, 2, 8, 11
+    Q = rng.standard_normal((B, T, h_qr, d))
+    K = rng.standard_normal((n, h_kv, d))
+    pos = np.zeros((B, n), bool)
+    pos[0, [2, 3]] = True
+    pos[1, [9]] = True
+    tau = 0.2
+    loss, dQ, dK = oracle.aux_routing_loss(Q, K, pos, tau)
+    q = torch.tensor(Q, requires_grad=True)
+    k = torch.tensor(K, requires_grad=True)
+    kg = k[:, torch.arange(h_qr) // (h_qr // h_kv)]                        # [n, h_qr, d]
+    cos = F.cosine_similarity(q[:, :, None], kg[None, None], dim=-1)      # [B, T, n, h_qr]
+    s = cos.mean(-1).amax(1)                                             # [B, n]
+    lsm = F.log_softmax(s / tau, dim=-1)
+    P = torch.tensor(pos)
+    ref = -torch.stack([lsm[b][P[b]].mean() for b in range(B)]).mean()
+    ref.backward()
+    assert abs(float(ref) - loss) < 1e-10
+    assert np.max(np.abs(q.grad.numpy() - dQ)) < 1e-8
+    assert np.max(np.abs(k.grad.numpy() - dK)) < 1e-8
+
