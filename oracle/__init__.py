@@ -7,6 +7,9 @@ shares no code with it; the two meet only through the seeded inputs of ``synth``
 The arithmetic lives in ``msa_oracle.c`` (plain C, double precision, one output at a time);
 this module marshals numpy arrays into it. Storage rounding of the bf16 configuration is
 mirrored with the oracle's own round-to-nearest-even (``round_bf16``).
+
+Parity unpinned: ``aux_routing_loss`` follows a reading of a loss the pages name without a
+formula (its arithmetic is pinned, its agreement with the authors' loss is not).
 """
 from __future__ import annotations
 
