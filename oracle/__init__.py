@@ -4,8 +4,10 @@ TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and bench.py's CPU
 are the only code allowed to import this package. The CUDA library never imports it and
 shares no code with it; the two meet only through the seeded inputs of ``synth``.
 
-The arithmetic lives in ``msa_oracle.c`` (plain C, double precision, one output at a time);
-this module marshals numpy arrays into it. Storage rounding of the bf16 configuration is
+The per-output arithmetic lives in ``msa_oracle.c`` (plain C, double precision, one output at
+a time) and this module marshals numpy arrays into it; the loops composing it (generation,
+interleave rounds, the encode from hidden states with numpy's matrix product as the
+projection) and the auxiliary routing loss are plain numpy here. Storage rounding of the bf16 configuration is
 mirrored with the oracle's own round-to-nearest-even (``round_bf16``).
 
 Parity unpinned: ``aux_routing_loss`` follows a reading of a loss the pages name without a
