@@ -34,6 +34,13 @@ MUTANTS = {
                               "orc_rope(r, d, (double)j, rope_base);"),
     "softmax_scale": ("scale = 1.0 / sqrt((double)d);", "scale = 1.0 / (double)d;"),
     "softmax_unnormalised": ("o[e] /= den;", "o[e] /= 1.0;"),
+    "bw_ds_sign": ("const double ds = p[n] * (dp[n] - dsum) * scale;",
+                   "const double ds = p[n] * (dsum - dp[n]) * scale;"),
+    "bw_query_not_rotated_back": ("orc_rope(dq, d, -pos, rope_base);",
+                                  "orc_rope(dq, d, pos, rope_base);"),
+    "bw_dv_unweighted": ("gv[e] += p[n] * go[e];", "gv[e] += go[e];"),
+    "bw_local_key_not_rotated_back": ("orc_rope(r, d, -((double)pos0 + (double)j), rope_base);",
+                                      ""),
 }
 
 
@@ -110,6 +117,31 @@ def _battery(L) -> list:
     ref = F.scaled_dot_product_attention(torch.from_numpy(q), keys, vals.expand(2, -1, -1),
                                          attn_mask=mask).numpy()
     check("attend", np.max(np.abs(O[0].transpose(1, 0, 2) - ref)) < 5e-4)
+    # attention gradients: central differences of the forward along random directions
+    Q = rng.standard_normal((1, 2, 2, 8)).astype(np.float32)
+    Kl = rng.standard_normal((1, 4, 1, 8)).astype(np.float32)
+    Vl = rng.standard_normal((1, 4, 1, 8)).astype(np.float32)
+    Kb = rng.standard_normal((3, 1, 8)).astype(np.float32)
+    Vb = rng.standard_normal((3, 1, 8)).astype(np.float32)
+    gi = np.array([[2, 0]], np.int32)
+    cl = np.array([2], np.int32)
+    dO = rng.standard_normal((1, 2, 2, 8))
+    g = oracle.attend_backward(Q, Kl, Vl, Kb, Vb, gi, cl, 3, 1e4, dO, L=L)
+    args = dict(Q=Q, K_loc=Kl, V_loc=Vl, Kbar=Kb, Vbar=Vb)
+    grads = dict(Q=g["dQ"], K_loc=g["dK_loc"], V_loc=g["dV_loc"], Kbar=g["dKbar"],
+                 Vbar=g["dVbar"])
+    ok = True
+    for name, x in args.items():
+        delta = rng.standard_normal(x.shape).astype(np.float32)
+        o = []
+        for sgn in (1, -1):
+            a = dict(args, **{name: (x.astype(np.float64) + sgn * 1e-2 * delta).astype(np.float32)})
+            o.append(oracle.attend(a["Q"], a["K_loc"], a["V_loc"], a["Kbar"], a["Vbar"], gi, cl,
+                                   3, 1e4, L=L))
+        fd = np.sum(dO * (o[0] - o[1])) / 2e-2
+        an = np.sum(grads[name] * delta)
+        ok &= abs(fd - an) <= 2e-3 * (1 + abs(an))
+    check("attend_backward", ok)
     return fails
 
 
