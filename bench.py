@@ -1232,8 +1232,32 @@ def run_encode_hidden(args):
     e1.record(st)
     st.synchronize()
     clocks = sampler.stop()
-    ms, = ranks.max([e0.elapsed_time(e1) / Kst], dev)
     assert msa.msa_workspace_status(ws, st) == 0
+    # end to end: the hidden states copied from pinned host memory and the pooled bank read
+    # back, every call
+    host_H = H.cpu().pin_memory()
+    host_out = [o.cpu().pin_memory() for o in outs]
+    h2d = host_H.numel() * host_H.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in host_out)
+
+    def e2e_call():
+        with torch.cuda.stream(st):
+            H.copy_(host_H, non_blocking=True)
+        call()
+        with torch.cuda.stream(st):
+            for o, ho in zip(outs, host_out):
+                ho.copy_(o, non_blocking=True)
+
+    e2e_call()
+    st.synchronize()
+    Ke = max(1, min(Kst, 3))
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(st)
+    for _ in range(Ke):
+        e2e_call()
+    e3.record(st)
+    st.synchronize()
+    ms, e2e_ms = ranks.max([e0.elapsed_time(e1) / Kst, e2.elapsed_time(e3) / Ke], dev)
     flop = 2.0 * n_tok * D * 3 * w.h_kv * w.d
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -1256,6 +1280,9 @@ def run_encode_hidden(args):
                          "bound": "tensor", "achieved": round(tf, 1), "peak": tpeak,
                          "unit": "TFLOP/s", "frac": round(tf / tpeak, 4), "peak_kind": tkind,
                          "traffic": None},
+            "e2e": {"value": round(replica_rate(world, n_tok, e2e_ms), 1), "unit": "bank tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
             "gpu_launches": Kst, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_encode_hidden_baseline(w, D)
