@@ -559,7 +559,7 @@ def test_aux_routing_loss_gradients_match_autograd():
     P = torch.tensor(pos)
     ref = -torch.stack([lsm[b][P[b]].mean() for b in range(B)]).mean()
     ref.backward()
-    assert abs(float(ref) - loss) < 1e-10
+    assert abs(float(ref.detach()) - loss) < 1e-10
     assert np.max(np.abs(q.grad.numpy() - dQ)) < 1e-8
     assert np.max(np.abs(k.grad.numpy() - dK)) < 1e-8
 
