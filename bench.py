@@ -203,136 +203,94 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ workload
 class Decode:
-    """Routed decode over a memory bank: per layer route -> fetch/gather -> attend."""
+    """The routed decode workload: synthetic banks and queries fed to the package's
+    ``engine.RoutedDecode`` (per layer route -> fetch/gather -> attend; see its docstring for
+    the overlapped schedule)."""
 
     def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc", nbuf: int = 2):
         import torch
 
         import long_context_doc_b200 as msa
         import synth
+        from long_context_doc_b200.engine import DecodeLayer, RoutedDecode
         self.torch, self.msa, self.w, self.dev = torch, msa, w, dev
-        self.fetch = fetch if w.layers > 1 else "device"
+        fetch = fetch if w.layers > 1 else "device"
         self.L = w.layers
-        self.main = torch.cuda.Stream()  # the step's stream (capturable into a CUDA graph)
-        self.copy = torch.cuda.Stream()
-        self.layers = []
+        self.scan = scan
         seed_w = w.scaled(seed=w.seed + 1000 * rank)
-        self.sw = seed_w
-        for l in range(self.L):
-            dv = synth.dev_bank_workload(seed_w, dev, layer=l, with_kv=(self.fetch == "device"))
-            dv["inv"] = msa.kr_inv_norm(dv["Kbar_r"])
-            dv["hat"] = msa.kr_normalize(dv["Kbar_r"]) if scan == "tc" else None
-            self.layers.append(dv)
-        self.coff_host = self.layers[0]["doc_chunk_off"]
-        self.coff = torch.from_numpy(self.coff_host).to(dev)
-        self.n_chunks = int(self.coff_host[-1])
-        self.n_docs = w.n_docs
-        self.max_ctx = w.k * int(np.max(np.diff(self.coff_host)))
-        if self.fetch != "device":
-            # one pinned host K̄/V̄ bank shared by the routed layers (only the selected rows
-            # ever cross the host link, so the fetch traffic does not depend on this)
-            self.Kh = torch.empty((self.n_chunks, w.h_kv, w.d), dtype=torch.bfloat16,
-                                  pin_memory=True)
-            self.Vh = torch.empty_like(self.Kh, pin_memory=True)
-            tmp = torch.empty((1 << 20, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)
-            row = w.h_kv * w.d
-            for name, dst in (("Kbar", self.Kh), ("Vbar", self.Vh)):
-                tid = synth.KBAR if name == "Kbar" else synth.VBAR
-                for c0 in range(0, self.n_chunks, tmp.shape[0]):
-                    n = min(tmp.shape[0], self.n_chunks - c0)
-                    t = tmp[:n]
-                    synth.dev_normal(t, seed_w.seed, synth.tag(tid, 0), first=c0 * row)
-                    dst[c0:c0 + n].copy_(t)
-            del tmp
-            self.fetchers = [msa.Fetcher(w.B, w.k) for _ in range(2)]
-            self.ev_route = [torch.cuda.Event() for _ in range(2)]
-            self.ev_gather = [torch.cuda.Event() for _ in range(2)]
-        B, k = w.B, w.k
-        ws_r = msa.msa_route_topk_workspace(B, w.T, w.h_qr, w.h_kv, w.d, 1, self.n_docs,
-                                            self.n_chunks, k)
-        ws_a = msa.msa_sparse_attend_workspace(B, w.T, w.h_q, w.h_kv, w.d, self.max_ctx, w.L_loc)
-        self.buf = []
-        self.nbuf = nbuf  # 2: layers alternate buffers; L: every layer keeps its context
-        for _ in range(nbuf):
-            self.buf.append(dict(
-                ws_r=torch.empty(ws_r, dtype=torch.uint8, device=dev),
-                ws_a=torch.empty(ws_a, dtype=torch.uint8, device=dev),
-                ws_g=torch.zeros(256, dtype=torch.uint8, device=dev),
-                ids=torch.empty((B, k), dtype=torch.int32, device=dev),
-                sc=torch.empty((B, k), dtype=torch.float32, device=dev),
-                gi=torch.empty((B, self.max_ctx), dtype=torch.int32, device=dev),
-                cl=torch.empty(B, dtype=torch.int32, device=dev),
-                cK=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev),
-                cV=torch.empty((B, self.max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)))
-        # every layer's query inputs (Q_r, Q) in one contiguous buffer and every layer's output
-        # in another, so that a step's host copies are one in and one out
+        B = w.B
+        # every layer's query inputs (Q_r, Q) in one contiguous buffer, so that a step's host
+        # copy of them is one transfer
         nqr, nq = B * w.T * w.h_qr * w.d, B * w.T * w.h_q * w.d
         self.qbuf = torch.empty(self.L * (nqr + nq), dtype=torch.bfloat16, device=dev)
-        for l, dv in enumerate(self.layers):
+        Kh = Vh = None
+        coff_host = None
+        layers = []
+        for l in range(self.L):
+            dv = synth.dev_bank_workload(seed_w, dev, layer=l, with_kv=(fetch == "device"))
+            coff_host = dv["doc_chunk_off"]
+            if fetch != "device" and Kh is None:
+                Kh, Vh = self._host_bank(seed_w, coff_host, dev)
             base = l * (nqr + nq)
-            for name, off, n in (("Q_r", base, nqr), ("Q", base + nqr, nq)):
-                v = self.qbuf[off:off + n].view(dv[name].shape)
-                v.copy_(dv[name])
-                dv[name] = v
-        self.obuf = torch.empty(self.L * nq, dtype=torch.bfloat16, device=dev)
-        self.O = [self.obuf[l * nq:(l + 1) * nq].view(B, w.T, w.h_q, w.d) for l in range(self.L)]
-        self.route_ev = None
-        self.scan = scan
-        # own kernels per layer (memsets and copies excluded): route (tensor path: query fold +
-        # scan with fused top-k; CUDA-core path: one fused kernel), gather, decode attention,
-        # the merge of its split queries
-        self.kernels_per_layer = (2 if scan == "tc" else 1) + 1 + 1 + 1
+            Q_r = self.qbuf[base:base + nqr].view(dv["Q_r"].shape)
+            Q = self.qbuf[base + nqr:base + nqr + nq].view(dv["Q"].shape)
+            Q_r.copy_(dv["Q_r"])
+            Q.copy_(dv["Q"])
+            kv = (Kh, Vh) if fetch != "device" else (dv["Kbar"], dv["Vbar"])
+            if scan == "tc":
+                # the tensor-core scan reads only the normalised bank: K̄_r is not kept
+                hat = msa.kr_normalize(dv.pop("Kbar_r"))
+                la = DecodeLayer(Q_r, Q, dv["K_loc"], dv["V_loc"], kv[0], kv[1], Kbar_r_hat=hat)
+            else:
+                la = DecodeLayer(Q_r, Q, dv["K_loc"], dv["V_loc"], kv[0], kv[1],
+                                 Kbar_r=dv["Kbar_r"], kr_inv_norm=msa.kr_inv_norm(dv["Kbar_r"]))
+            layers.append(la)
+            del dv
+        self.rd = RoutedDecode(layers, coff_host, w.k, w.rope_base, fetch=fetch, nbuf=nbuf)
+        self.fetch = self.rd.fetch
+        self.main = self.rd.stream
+        self.layers = layers
+        self.n_chunks = self.rd.n_chunks
+        self.max_ctx = self.rd.max_ctx
+        self.obuf = self.rd.O.view(-1)
+        self.kernels_per_step = self.rd.kernels_per_step()
 
-    # per-layer pieces -------------------------------------------------------------
-    def route(self, l):
-        msa, d, bf = self.msa, self.layers[l], self.buf[l % self.nbuf]
-        if self.route_ev is not None:
-            self.route_ev[l][0].record(self.main)
-        msa.msa_route_topk(d["Q_r"], d["Kbar_r"], d["inv"], self.coff, self.w.k, None, bf["ids"],
-                           bf["sc"], None, bf["ws_r"], self.main, d["hat"])
-        if self.route_ev is not None:
-            self.route_ev[l][1].record(self.main)
+    @staticmethod
+    def _host_bank(w, coff_host, dev):
+        """One pinned host K̄/V̄ bank shared by the routed layers (only the selected rows ever
+        cross the host link, so the fetch traffic does not depend on this)."""
+        import torch
 
-    def begin(self, l):
-        bf = self.buf[l % self.nbuf]
-        if self.fetch == "memcpy":
-            self.fetchers[l % 2].begin(bf["ids"], self.coff, self.max_ctx, bf["gi"], bf["cl"],
-                                       bf["ws_g"], self.main)
-        elif self.fetch == "zerocopy":
-            # the gather kernel reads the selected rows from pinned host memory on a side
-            # stream, ordered after this layer's routing and before its attention
-            self.ev_route[l % 2].record(self.main)
-            self.copy.wait_event(self.ev_route[l % 2])
-            self.msa.msa_gather(bf["ids"], self.coff, self.Kh, self.Vh, self.max_ctx, bf["gi"],
-                                bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.copy)
-            self.ev_gather[l % 2].record(self.copy)
-        else:
-            d = self.layers[l]
-            self.msa.msa_gather(bf["ids"], self.coff, d["Kbar"], d["Vbar"], self.max_ctx,
-                                bf["gi"], bf["cl"], bf["cK"], bf["cV"], bf["ws_g"], self.main)
+        import synth
+        n_chunks = int(coff_host[-1])
+        Kh = torch.empty((n_chunks, w.h_kv, w.d), dtype=torch.bfloat16, pin_memory=True)
+        Vh = torch.empty_like(Kh, pin_memory=True)
+        tmp = torch.empty((1 << 20, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)
+        row = w.h_kv * w.d
+        for tid, dst in ((synth.KBAR, Kh), (synth.VBAR, Vh)):
+            for c0 in range(0, n_chunks, tmp.shape[0]):
+                n = min(tmp.shape[0], n_chunks - c0)
+                t = tmp[:n]
+                synth.dev_normal(t, w.seed, synth.tag(tid, 0), first=c0 * row)
+                dst[c0:c0 + n].copy_(t)
+        del tmp
+        return Kh, Vh
 
-    def finish(self, l):
-        if self.fetch == "zerocopy":
-            self.main.wait_event(self.ev_gather[l % 2])
-        if self.fetch == "memcpy":
-            bf = self.buf[l % self.nbuf]
-            self.fetchers[l % 2].finish(self.coff_host, self.Kh, self.Vh, self.max_ctx, bf["cK"],
-                                        bf["cV"], self.main, self.copy, 10_000)
+    @property
+    def route_ev(self):
+        return self.rd.route_events
 
-    def attend(self, l):
-        d, bf, w = self.layers[l], self.buf[l % self.nbuf], self.w
-        self.msa.msa_sparse_attend(d["Q"], d["K_loc"], d["V_loc"], bf["cK"], bf["cV"], bf["cl"],
-                                   w.k, w.rope_base, 0.0, self.O[l], bf["ws_a"], self.main)
+    @route_ev.setter
+    def route_ev(self, ev):
+        self.rd.route_events = ev
 
     def step(self):
-        self.route(0)
-        self.begin(0)
-        for l in range(self.L):
-            if l + 1 < self.L:
-                self.route(l + 1)
-                self.begin(l + 1)
-            self.finish(l)
-            self.attend(l)
+        self.rd.step()
+
+    def ctx(self, l):
+        """(ctxK, ctxV, ctx_len) of layer l after a step (with one buffer set per layer)."""
+        bf = self.rd.buf[l % self.rd.nbuf]
+        return bf["cK"], bf["cV"], self.rd.ctx_len[l]
 
     def scan_bytes(self):
         """Algorithmic bytes of one routing call: the bank it streams (K̂_r for the tensor
@@ -412,13 +370,13 @@ def run_libmsa(args):
     # per step: every layer's Q_r and Q (one copy), the new token's K/V row of every layer's
     # local cache, then every layer's output (one copy) and the last two layers' top-k ids
     host_q = wk.qbuf.cpu().pin_memory()
-    host_kv = [[t.cpu().pin_memory() for t in (d["K_loc"][:, -1:], d["V_loc"][:, -1:])]
+    host_kv = [[t.cpu().pin_memory() for t in (d.K_loc[:, -1:], d.V_loc[:, -1:])]
                for d in wk.layers]
     host_O = wk.obuf.cpu().pin_memory()
-    host_ids = [b["ids"].cpu().pin_memory() for b in wk.buf[:2]]
+    host_ids = wk.rd.ids.cpu().pin_memory()
     h2d = (host_q.numel() * host_q.element_size() +
            sum(t.numel() * t.element_size() for hs in host_kv for t in hs))
-    d2h = host_O.numel() * host_O.element_size() + 2 * w.B * w.k * 4
+    d2h = host_O.numel() * host_O.element_size() + host_ids.numel() * 4
 
     def e2e_step():
         with torch.cuda.stream(wk.main):
@@ -426,12 +384,11 @@ def run_libmsa(args):
             for l in range(wk.L):
                 d = wk.layers[l]
                 kn, vn = host_kv[l]
-                d["K_loc"][:, -1:].copy_(kn, non_blocking=True)
-                d["V_loc"][:, -1:].copy_(vn, non_blocking=True)
+                d.K_loc[:, -1:].copy_(kn, non_blocking=True)
+                d.V_loc[:, -1:].copy_(vn, non_blocking=True)
             wk.step()
             host_O.copy_(wk.obuf, non_blocking=True)
-            host_ids[0].copy_(wk.buf[0]["ids"], non_blocking=True)
-            host_ids[1].copy_(wk.buf[1]["ids"], non_blocking=True)
+            host_ids.copy_(wk.rd.ids, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -491,7 +448,7 @@ def run_libmsa(args):
                      "avg_launch_ms": round(route_avg, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": Kst * wk.L * wk.kernels_per_layer,
+        "gpu_launches": Kst * wk.kernels_per_step,
         "route_calls_timed": len(route_ms),
         "clocks": clocks,
     }
@@ -555,19 +512,25 @@ def run_reference(args):
     import synth
     if args.workload == "gen100m":
         w = synth.C4
+        # each timed step = 4 generation steps of ONE routed layer (a bounded sample); the
+        # tokens/s extrapolate its mean per-token time to all routed layers
         times = []
         for s in range(args.steps):
-            times.append(oracle_generate_time(w, s % w.layers, 4) / 4 * w.layers)
+            times.append(oracle_generate_time(w, s % w.layers, 4))
             if sum(times) > 120:
                 break
-        token = statistics.mean(times)
+        sample = statistics.mean(times)
+        token = sample / 4 * w.layers
         value = w.B / token
         unit = "generated tokens/s"
         print(json.dumps({
             "metric": "MSA sparse generation tokens/s at the 100M-token bank (context built once "
                       "per request, routed memory fixed while generating)",
             "value": round(value, 4), "unit": unit, "n_gpus": 1, "steps": len(times),
-            "warmup": args.warmup, "ms_per_step": round(token * 1e3, 2), "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": round(sample * 1e3, 2),
+            "step_is": f"4 generation steps of one routed layer of {w.layers} (value = batch / "
+                       f"(mean step time / 4 x {w.layers}))",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": "gen100m", "routed_layers": w.layers, "batch": w.B,
@@ -582,23 +545,30 @@ def run_reference(args):
     w = synth.C4 if args.workload == "bank100m" else synth.C3
     for l in range(min(args.warmup, 1)):
         oracle_layer_time(w.scaled(n_docs=2000), l)
+    # each timed step is a bounded sample of the workload's step: ONE routed layer (route over
+    # every document + gather + attend for the batch); the queries/s extrapolate it to all
+    # routed layers, while steps and ms_per_step describe what was actually timed
     times = []
     for s in range(args.steps):
-        times.append(oracle_layer_time(w, s % w.layers) * w.layers)
-        if sum(times) / w.layers > 60:
+        times.append(oracle_layer_time(w, s % w.layers))
+        if sum(times) > 60:
             break
-    step = statistics.mean(times)
-    value = w.B / step
+    layer = statistics.mean(times)
+    value = w.B / (layer * w.layers)
     line = {"metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": 1,
-            "steps": len(times), "warmup": args.warmup, "ms_per_step": round(step * 1e3, 2),
+            "steps": len(times), "warmup": args.warmup, "ms_per_step": round(layer * 1e3, 2),
+            "step_is": f"one routed layer of {w.layers} (value = batch / ({w.layers} x mean "
+                       "layer time))",
+            "extrapolated_ms_per_full_step": round(layer * w.layers * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len,
                        "routed_layers": w.layers, "batch": w.B, "k": w.k},
             "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle",
                              "cores": oracle.num_threads(),
-                             "sample": "each step = one routed layer (route over every doc + "
-                                       "gather + attend for the batch) x the layer count"},
+                             "sample": "each timed step = one routed layer (route over every "
+                                       "doc + gather + attend for the batch); value "
+                                       "extrapolates the mean layer time to all routed layers"},
             "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -969,7 +939,7 @@ def run_generate(args):
     for l in range(wk.L):
         c = msa.LocalCache(B, cap, w.h_kv, w.d, pos0=w.k, rope_base=w.rope_base, device=dev,
                            length=lens[l:l + 1])
-        c.append(wk.layers[l]["K_loc"], wk.layers[l]["V_loc"])  # the prompt's local K/V
+        c.append(wk.layers[l].K_loc, wk.layers[l].V_loc)  # the prompt's local K/V
         caches.append(c)
         base = l * per_layer
         x = dict(Q=tokbuf[base:base + nq].view(B, 1, w.h_q, w.d),
@@ -985,9 +955,10 @@ def run_generate(args):
 
     def token_step():
         for l in range(wk.L):
-            x, c, b = tok[l], caches[l], wk.buf[l]
-            msa.msa_decode_step(x["Q"], x["K"], x["V"], c.K, c.V, c.length, b["cK"], b["cV"],
-                                b["cl"], w.k, w.rope_base, 0.0, x["O"], x["ws"], wk.main)
+            x, c = tok[l], caches[l]
+            cK, cV, cl = wk.ctx(l)
+            msa.msa_decode_step(x["Q"], x["K"], x["V"], c.K, c.V, c.length, cK, cV, cl, w.k,
+                                w.rope_base, 0.0, x["O"], x["ws"], wk.main)
 
     def construct():
         lens.copy_(lens0)  # a new request: every cache holds the prompt again
@@ -1060,7 +1031,7 @@ def run_generate(args):
     # algorithmic bytes of one decode step at the mean cache length of a request: memory
     # and local K/V rows read once, the query read, the output written, the token's K/V
     # appended (read + written)
-    cl_host = [wk.buf[l]["cl"].cpu().numpy() for l in range(wk.L)]
+    cl_host = [wk.rd.ctx_len[l].cpu().numpy() for l in range(wk.L)]
     mem_rows = statistics.mean(float(c.sum()) for c in cl_host)
     loc_rows = B * (L0 + (n_ev + 1) / 2.0)
     row = w.h_kv * w.d * 2
@@ -1142,7 +1113,7 @@ def run_generate(args):
                 "ms_per_step": round(e2e_ms, 3)},
         # per request: the construction step's kernels + per token and layer append,
         # attention and merge
-        "gpu_launches": Kst * (wk.L * wk.kernels_per_layer + G * wk.L * 3),
+        "gpu_launches": Kst * (wk.kernels_per_step + G * wk.L * 3),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -125,12 +125,15 @@ msa_status msa_kr_normalize(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, 
  *
  * Q_r        [B, T, h_qr, d] router queries (dtype). Router head h uses router-key head
  *            floor(h / (h_qr / h_kv)).
- * Kbar_r     [n_chunks, h_kv, d] router-key bank (dtype), 16-byte aligned.
- * kr_inv_norm [n_chunks, h_kv] fp32 inverse norms (from msa_encode_pool / msa_kr_inv_norm).
+ * Kbar_r     [n_chunks, h_kv, d] router-key bank (dtype), 16-byte aligned (nullable with
+ *            Kbar_r_hat, see below).
+ * kr_inv_norm [n_chunks, h_kv] fp32 inverse norms (from msa_encode_pool / msa_kr_inv_norm;
+ *            nullable with Kbar_r_hat).
  * Kbar_r_hat (nullable) [n_chunks, h_kv, d] bf16 per-head unit rows (msa_kr_normalize).
  *            With Kbar_r_hat and a bf16 bank, every query length is scored on the tensor
  *            cores as one bf16 contraction of Kbar_r_hat with the per-head normalised queries
- *            (fp32 accumulation; Kbar_r and kr_inv_norm are not read). Without it, queries
+ *            (fp32 accumulation; Kbar_r and kr_inv_norm are not read and may be NULL, so a
+ *            bank prepared for this scan need not keep K̄_r resident). Without it, queries
  *            with T <= 16 are scored on CUDA cores from Kbar_r and kr_inv_norm in fp32 (B*T rows
  *            in passes of up to 16); longer queries (17 <= T <= 256) require Kbar_r_hat.
  * doc_chunk_off [n_docs+1] device int64 chunk offsets (non-decreasing, ends at n_chunks).
@@ -171,7 +174,10 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
  * any stream capture. It allocates nothing (no cudaMalloc/cudaFree or allocating library
  * routine). All calls share the one array, which keeps the last call's contents (what must
  * start at zero is cleared by every call); calls that overlap on the GPU race and must be
- * serialised by the caller. */
+ * serialised by the caller. The cached address is that of the device's primary context (the
+ * CUDA runtime's): it is not valid after cudaDeviceReset or under another driver-API context.
+ * Device-side failures (a bounded wait that ran out, a bad index) are recorded in the array's
+ * status word as in a workspace; read it with msa_route_topk_noalloc_status. */
 msa_status msa_route_topk_noalloc(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
                                   const void* Kbar_r, const float* kr_inv_norm,
                                   const void* Kbar_r_hat, const int64_t* doc_chunk_off,
@@ -179,6 +185,14 @@ msa_status msa_route_topk_noalloc(const void* Q_r, int32_t B, int32_t T, int32_t
                                   int32_t dtype, int32_t k, const uint32_t* exclude_bits,
                                   int32_t* top_ids, float* top_scores, float* doc_scores,
                                   void* stream);
+
+/* msa_route_topk_noalloc_status - the status word of the built-in scratch of
+ * msa_route_topk_noalloc on the current device, read after the work queued on `stream`
+ * (synchronises `stream`; allocates nothing). *code = 0 if the last call's kernels recorded no
+ * error; otherwise returns MSA_ERR_DEVICE with *code the recorded error. The word is cleared
+ * by every msa_route_topk_noalloc call, so read it after the call it should describe and
+ * before the next. (A library service; the pages describing MSA have no counterpart.) */
+msa_status msa_route_topk_noalloc_status(int32_t* code, void* stream);
 
 /* Read the device status word of a workspace (synchronises `stream`): *code = 0 if the
  * kernels that used it recorded no error. Returns MSA_ERR_DEVICE if *code != 0. */

@@ -29,7 +29,7 @@ LIB_PATH = _build.LIB
 # every symbol include/msa.h declares
 SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chunks",
            "msa_encode_pool", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
-           "msa_route_topk", "msa_route_topk_noalloc",
+           "msa_route_topk", "msa_route_topk_noalloc", "msa_route_topk_noalloc_status",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
            "msa_sparse_attend", "msa_assemble_local", "msa_kv_append",
@@ -72,6 +72,8 @@ def _load():
     L.msa_route_topk_noalloc.restype = ctypes.c_int
     L.msa_route_topk_noalloc.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, i64, i64, i32, i32, i32,
                                          i32, vp, vp, vp, vp, vp]
+    L.msa_route_topk_noalloc_status.restype = ctypes.c_int
+    L.msa_route_topk_noalloc_status.argtypes = [vp, vp]
     L.msa_workspace_status.restype = ctypes.c_int
     L.msa_workspace_status.argtypes = [vp, vp, vp]
     L.msa_gather.restype = ctypes.c_int
@@ -204,13 +206,20 @@ def msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k) ->
     return int(lib.msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype, n_docs, n_chunks, k))
 
 
+def _bank(Kbar_r, Kbar_r_hat):
+    """(n_chunks, h_kv, dtype code) of a routing bank; Kbar_r may be None when the normalised
+    bank Kbar_r_hat is given (the tensor-core scan reads only that)."""
+    ref = Kbar_r if Kbar_r is not None else Kbar_r_hat
+    return ref.shape[0], ref.shape[1], dtype_code(ref)
+
+
 def msa_route_topk(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_bits, top_ids, top_scores,
                    doc_scores, ws, stream=None, Kbar_r_hat=None):
     B, T, h_qr, d = Q_r.shape
-    n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
+    n_chunks, h_kv, dt = _bank(Kbar_r, Kbar_r_hat)
     _check(lib.msa_route_topk(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm), _p(Kbar_r_hat),
                               _p(doc_chunk_off),
-                              doc_chunk_off.shape[0] - 1, n_chunks, h_kv, d, dtype_code(Kbar_r), k,
+                              doc_chunk_off.shape[0] - 1, n_chunks, h_kv, d, dt, k,
                               _p(exclude_bits), _p(top_ids), _p(top_scores), _p(doc_scores),
                               _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
@@ -219,11 +228,20 @@ def msa_route_topk_noalloc(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_b
                            top_scores, doc_scores, stream=None, Kbar_r_hat=None):
     """msa_route_topk without a workspace (the library's built-in 2 MiB scratch)."""
     B, T, h_qr, d = Q_r.shape
-    n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
+    n_chunks, h_kv, dt = _bank(Kbar_r, Kbar_r_hat)
     _check(lib.msa_route_topk_noalloc(_p(Q_r), B, T, h_qr, _p(Kbar_r), _p(kr_inv_norm),
                                       _p(Kbar_r_hat), _p(doc_chunk_off), doc_chunk_off.shape[0] - 1,
-                                      n_chunks, h_kv, d, dtype_code(Kbar_r), k, _p(exclude_bits),
+                                      n_chunks, h_kv, d, dt, k, _p(exclude_bits),
                                       _p(top_ids), _p(top_scores), _p(doc_scores), _s(stream)))
+
+
+def msa_route_topk_noalloc_status(stream=None) -> int:
+    """Status word of msa_route_topk_noalloc's built-in scratch (0 = no device error)."""
+    code = ctypes.c_int32(0)
+    st = lib.msa_route_topk_noalloc_status(ctypes.addressof(code), _s(stream))
+    if st not in (0, 6):
+        _check(st)
+    return int(code.value)
 
 
 def msa_workspace_status(ws, stream=None) -> int:
@@ -332,12 +350,11 @@ def route_topk(Q_r, Kbar_r, kr_inv, doc_chunk_off, k: int, exclude_bits=None,
                doc_scores: bool = False, ws=None, stream=None, Kbar_r_hat=None):
     """Returns (top_ids int32 [B,k], top_scores f32 [B,k], doc_scores f32 [B,n_docs] or None)."""
     B, T, h_qr, d = Q_r.shape
-    n_chunks, h_kv = Kbar_r.shape[:2]
+    n_chunks, h_kv, dt = _bank(Kbar_r, Kbar_r_hat)
     n_docs = doc_chunk_off.shape[0] - 1
     dev = Q_r.device
     if ws is None:
-        ws = _ws(msa_route_topk_workspace(B, T, h_qr, h_kv, d, dtype_code(Kbar_r), n_docs,
-                                          n_chunks, k), dev)
+        ws = _ws(msa_route_topk_workspace(B, T, h_qr, h_kv, d, dt, n_docs, n_chunks, k), dev)
     ids = torch.empty((B, k), dtype=torch.int32, device=dev)
     sc = torch.empty((B, k), dtype=torch.float32, device=dev)
     ds = torch.empty((B, n_docs), dtype=torch.float32, device=dev) if doc_scores else None

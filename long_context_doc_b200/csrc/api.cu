@@ -244,10 +244,13 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
             "T=%d > 16 needs the normalised bank Kbar_r_hat (msa_kr_normalize)", T);
   }
   if (B == 0) return ok();
-  REQUIRE(Q_r && Kbar_r && kr_inv_norm && doc_chunk_off && top_ids && top_scores,
+  // the tensor-core scan reads only the normalised bank: Kbar_r and its inverse norms may be
+  // null there (a bank prepared for it need not keep K̄_r resident)
+  const bool tc_scan = T > 16 || (dtype == MSA_BF16 && Kbar_r_hat != nullptr);
+  REQUIRE(Q_r && doc_chunk_off && top_ids && top_scores && (tc_scan || (Kbar_r && kr_inv_norm)),
           MSA_ERR_INVALID_ARG, "null tensor");
-  REQUIRE(aligned16(Kbar_r), MSA_ERR_INVALID_ARG, "Kbar_r must be 16-byte aligned");
-  if (T > 16 || (dtype == MSA_BF16 && Kbar_r_hat != nullptr)) {
+  REQUIRE(tc_scan || aligned16(Kbar_r), MSA_ERR_INVALID_ARG, "Kbar_r must be 16-byte aligned");
+  if (tc_scan) {
     REQUIRE(aligned16(Kbar_r_hat) && aligned16(Q_r), MSA_ERR_INVALID_ARG,
             "Kbar_r_hat and Q_r must be 16-byte aligned");
     const msa::TcPlan pl = msa::tc_plan(B, T, h_kv, d, n_docs, n_chunks, k, sm_count());

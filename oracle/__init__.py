@@ -153,8 +153,9 @@ def encode_pool(K, V, K_r, doc_tok_off, chunk: int, rope_base: float, L=None):
 
 def encode_hidden(H, W_k, W_v, W_r, doc_tok_off, chunk: int, rope_base: float, h_kv: int,
                   L=None):
-    """Offline encode from hidden states (reading R26 of the design notes): the per-token keys,
-    values and router keys are projections of the hidden states, K = H W_k, V = H W_v,
+    """Offline encode from hidden states. The pages name the projections but not where they
+    sit; the reading here is that the per-token keys, values and router keys are projections
+    of the hidden states, K = H W_k, V = H W_v,
     K_r = H W_r (the router K projector makes the routing keys: ruixiangma.github.io blog,
     "稀疏注意力机制"), computed here as plain matrix products in double precision; they then
     go through doc-wise RoPE and chunk mean pooling exactly as in ``encode_pool``.
@@ -259,7 +260,7 @@ def attend_backward(Q, K_loc, V_loc, Kbar, Vbar, gather_idx, ctx_len, pos0: int,
 
 
 def aux_routing_loss(Q_r, Kbar_r, positive, tau: float = 0.1):
-    """Auxiliary routing loss (reading R27 of the design notes: the pages name a supervised
+    """Auxiliary routing loss (a reading: the pages name a supervised
     contrastive loss that separates relevant from irrelevant document chunks but give no
     formula, so this function's parity with the authors' loss is unpinned).
 
@@ -334,7 +335,10 @@ def pipeline(w, inp: dict, L=None) -> dict:
 
 def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=None,
                select=None) -> dict:
-    """Oracle of Memory Interleaving rounds (reading R18 of the design notes).
+    """Oracle of Memory Interleaving rounds. The pages describe the loop (retrieve, append the
+    retrieved documents' text, repeat) but not which routed layer's selection is appended
+    without a model; the reading here takes the last routed layer's selection, keeps pos0 = k
+    in every round and excludes appended documents from later routing.
 
     layers[l]: dict with Kbar_r, Kbar, Vbar (stored dtype), doc_chunk_off, Q_r, Q and the query
     tokens' own K_q, V_q [B, T, h_kv, d]. doc_kv(l, doc) -> raw (K, V) [len, h_kv, d] of a
@@ -394,7 +398,9 @@ def interleave(layers: list, k: int, rounds: int, rope_base: float, doc_kv, L=No
 
 def generate(Q_steps, Kn_steps, Vn_steps, K_prompt, V_prompt, Kbar, Vbar, gather_idx, ctx_len,
              pos0: int, rope_base: float, scale: float = 0.0, L=None):
-    """Oracle of sparse generation over an assembled context (reading R24 of the design notes).
+    """Oracle of sparse generation over an assembled context. The pages route once, when the
+    context is constructed, and generate over it; the reading here keeps the routed memory fixed
+    for every generated token and appends each token's K/V to the local context.
 
     Routing and context assembly come first and the routed memory then stays fixed while the
     model generates autoregressively over the assembled context [news.neo-ai.one article,

@@ -18,7 +18,7 @@
  *       "三阶段推理流程" (three-stage inference) and "Memory Interleaving".
  *  [D]  github-eval-reports "MSA 项目评测报告", section "核心模块" (core modules).
  *
- * Readings where the pages are silent (each is listed with its reason in the design notes):
+ * Readings where the pages are silent (each one the plainest reading the rest supports):
  *  - RoPE pairs element i with element i + d/2 ("rotate half"), angle pos * base^(-2i/d);
  *    the backbone is Qwen3 [A, 実験設定]. rope_base <= 0 disables rotation.
  *  - Chunks never cross documents; a partial last chunk is the mean of its valid tokens.

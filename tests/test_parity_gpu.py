@@ -241,29 +241,47 @@ def test_route_full_10m_token_bank(msa, gpu):
     assert np.array_equal(ids.cpu().numpy()[:, 0], dv["planted"][:, 0])
 
 
-@pytest.mark.slow
-def test_route_full_100m_token_bank_layer_sampled(msa, gpu):
-    """100M-token bank layer (1.6M chunks, bf16, 3.3 GB), 4 decode queries: GPU scores of a
-    sample of documents against the oracle; the GPU top-k must be the exact top-k of its own
-    document scores and must start with the planted document."""
+@pytest.fixture(scope="module")
+def bank100m_layer(gpu):
+    """One routed layer of the 100M-token bank (200,000 docs x 8 chunks = 1.6M chunks, bf16,
+    3.3 GB) on the device, its host twin, and the oracle's routing of the 4 decode queries
+    over every chunk."""
     w = synth.C4
     dv = synth.dev_bank_workload(w, gpu, layer=0, with_kv=False)
     coff = dv["doc_chunk_off"]
-    inv = msa.kr_inv_norm(dv["Kbar_r"])
-    ids, sc, ds = msa.route_topk(dv["Q_r"], dv["Kbar_r"], inv, torch.from_numpy(coff).to(gpu), w.k,
-                                 doc_scores=True)
+    Krb = synth.host_bank_rows(w, "Kbar_r", 0, dv["n_chunks"], coff=coff, Q_r=dv["Q_r_host"])
+    ref = oracle.route(dv["Q_r_host"], Krb, coff, w.k)
+    del Krb
+    yield w, dv, ref
+    del dv
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("scan", ["tc", "cc"], ids=["tensor_core_scan", "cuda_core_scan"])
+def test_route_full_100m_token_bank_layer(msa, gpu, bank100m_layer, scan):
+    """A full 100M-token bank layer (1.6M chunks, 3.3 GB) routed for the 4 decode queries of
+    the benchmarked configuration, in the launch configuration the benchmark times for
+    ``tc`` (the tensor-core scan over the normalised bank, without K̄_r or its norms): every
+    one of the 200,000 document scores against the oracle's full routing within the bf16
+    tolerance, and the top-16 against the oracle's ids under the gap rule."""
+    w, dv, (r_ids, r_sc, r_ds) = bank100m_layer
+    coff = torch.from_numpy(dv["doc_chunk_off"]).to(gpu)
+    if scan == "tc":
+        hat = msa.kr_normalize(dv["Kbar_r"])
+        ids, sc, ds = msa.route_topk(dv["Q_r"], None, None, coff, w.k, doc_scores=True,
+                                     Kbar_r_hat=hat)
+    else:
+        inv = msa.kr_inv_norm(dv["Kbar_r"])
+        ids, sc, ds = msa.route_topk(dv["Q_r"], dv["Kbar_r"], inv, coff, w.k, doc_scores=True)
     torch.cuda.synchronize()
-    ids, sc, gds = ids.cpu().numpy(), sc.cpu().numpy(), ds.cpu().numpy()
-    for b in range(w.B):
-        order = np.lexsort((np.arange(w.n_docs), -gds[b].astype(np.float64)))[:w.k]
-        assert ids[b].tolist() == order.tolist()
-        assert ids[b, 0] == dv["planted"][b, 0]
-    sample = sorted(set(synth.uniform(3, 4, 300, w.n_docs).tolist() + ids.ravel().tolist()))
-    for dd in sample:
-        rows = synth.host_bank_rows(w, "Kbar_r", int(coff[dd]), int(coff[dd + 1]), coff=coff,
-                                    Q_r=dv["Q_r_host"])
-        _, _, r = oracle.route(dv["Q_r_host"], rows, np.array([0, len(rows)]), 1)
-        assert np.max(np.abs(r[:, 0] - gds[:, dd])) <= SCORE_TOL["bf16"]
+    gds = ds.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(gds))
+    err = np.max(np.abs(gds - r_ds))
+    assert err <= SCORE_TOL["bf16"], err
+    check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), r_ids, r_sc, r_ds,
+               SCORE_TOL["bf16"])
+    assert np.array_equal(ids.cpu().numpy()[:, 0], dv["planted"][:, 0])
 
 
 def test_route_reports_small_workspace(msa, gpu):
@@ -443,8 +461,23 @@ def test_pipeline_tiny_config(msa, gpu, w):
     torch.cuda.synchronize()
     check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), ref["top_ids"],
                ref["top_scores"], ref["doc_scores"], SCORE_TOL[w.dtype])
-    if set(ids.cpu().numpy()[0].tolist()) == set(ref["top_ids"][0].tolist()):
-        assert np.array_equal(gi.cpu().numpy(), ref["gather_idx"])
+    _check_downstream_of_selection(w, inp, ref, ids, gi, cl, O, max_ctx)
+
+
+def _check_downstream_of_selection(w, inp, ref, ids, gi, cl, O, max_ctx):
+    """Gather and attention checked on the GPU's own selection (a valid top-k under the gap
+    rule, already checked): the oracle gathers and attends with the GPU's ids, and the GPU's
+    gather indices must equal the oracle's bit for bit and its output the oracle's within the
+    attention tolerance. Runs whatever the selection, so it never skips."""
+    g_ids = ids.cpu().numpy()
+    r_gi, r_cl = oracle.gather(g_ids, ref["doc_chunk_off"], max_ctx)
+    assert np.array_equal(gi.cpu().numpy(), r_gi)
+    assert np.array_equal(cl.cpu().numpy(), r_cl)
+    O_ref = oracle.attend(inp["Q"], inp["K_loc"], inp["V_loc"], ref["Kbar"], ref["Vbar"], r_gi,
+                          r_cl, w.k, w.rope_base)
+    check_attention(O, O_ref, w.dtype)
+    if np.array_equal(g_ids, ref["top_ids"]):  # same selection: the oracle's pipeline output
+        assert np.array_equal(r_gi, ref["gather_idx"])
         check_attention(O, ref["O64"], w.dtype)
 
 
@@ -561,8 +594,6 @@ def test_pipeline_1m_bank_shape_reduced(msa, gpu):
                           w.rope_base)
     torch.cuda.synchronize()
     assert np.max(np.abs(ds.cpu().numpy() - ref["doc_scores"])) <= SCORE_TOL["bf16"]
-    n = check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), ref["top_ids"],
-                   ref["top_scores"], ref["doc_scores"], SCORE_TOL["bf16"])
-    if n == 1:
-        assert np.array_equal(gi.cpu().numpy(), ref["gather_idx"])
-        check_attention(O, ref["O64"], "bf16")
+    check_topk(ids.cpu().numpy(), sc.cpu().numpy().astype(np.float64), ref["top_ids"],
+               ref["top_scores"], ref["doc_scores"], SCORE_TOL["bf16"])
+    _check_downstream_of_selection(w, inp, ref, ids, gi, cl, O, max_ctx)
