@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
                     choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long",
-                             "gen100m", "encode_hidden1m"])
+                             "gen100m", "encode_hidden1m", "attend_bwd"])
     ap.add_argument("--gen-tokens", type=int, default=256,
                     help="gen100m: tokens generated per query after the context is built")
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
@@ -909,6 +909,133 @@ def run_attend_long(args):
           flush=True)
 
 
+def run_attend_backward(args):
+    """The backward of the sparse attention at the last interleave round's shape (B = 4 queries
+    of T = 256 tokens, 32 query heads over 8 KV heads, 64 memory rows + 8,256 local rows):
+    msa_sparse_attend_backward (forward recompute, D, the tcgen05 gradient kernel, dQ rotated
+    back) plus the scatter of the memory rows' gradients into an fp32 bank gradient, timed with
+    CUDA events on the launching stream; TFLOP/s of the five backward products over the
+    visible (query row, key) pairs."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    import synth
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev, timeout_s=300)
+    rank, world = ranks.rank, ranks.world
+    w = synth.C5
+    B, T, L, mc = 4, w.T, w.T + 2 * w.k * w.doc_len, w.k * 8
+    bf, f32 = torch.bfloat16, torch.float32
+    seed = w.seed + 1000 * rank
+    Q = synth.dev_normal(torch.empty((B, T, w.h_q, w.d), dtype=bf, device=dev), seed, 1)
+    Kl = synth.dev_normal(torch.empty((B, L, w.h_kv, w.d), dtype=bf, device=dev), seed, 2)
+    Vl = synth.dev_normal(torch.empty_like(Kl), seed, 3)
+    cK = synth.dev_normal(torch.empty((B, mc, w.h_kv, w.d), dtype=bf, device=dev), seed, 4)
+    cV = synth.dev_normal(torch.empty_like(cK), seed, 5)
+    dO = synth.dev_normal(torch.empty_like(Q), seed, 6)
+    cl = torch.full((B,), mc, dtype=torch.int32, device=dev)
+    n_chunks = 20000 * 8
+    gi = torch.stack([torch.randperm(n_chunks, device=dev)[:mc] for _ in range(B)]).to(torch.int32)
+    g = dict(dQ=torch.empty((B, T, w.h_q, w.d), dtype=f32, device=dev),
+             dK_loc=torch.empty((B, L, w.h_kv, w.d), dtype=f32, device=dev),
+             dV_loc=torch.empty((B, L, w.h_kv, w.d), dtype=f32, device=dev),
+             dK_ctx=torch.empty((B, mc, w.h_kv, w.d), dtype=f32, device=dev),
+             dV_ctx=torch.empty((B, mc, w.h_kv, w.d), dtype=f32, device=dev))
+    dKb = torch.zeros((n_chunks, w.h_kv, w.d), dtype=f32, device=dev)
+    dVb = torch.zeros_like(dKb)
+    ws = torch.empty(msa.msa_sparse_attend_backward_workspace(B, T, w.h_q, w.h_kv, w.d, mc, L),
+                     dtype=torch.uint8, device=dev)
+    ws_s = torch.zeros(256, dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream()
+
+    def step():
+        msa.msa_sparse_attend_backward(Q, Kl, Vl, cK, cV, cl, w.k, w.rope_base, 0.0, dO, g["dQ"],
+                                       g["dK_loc"], g["dV_loc"], g["dK_ctx"], g["dV_ctx"], ws, st)
+        msa.msa_scatter_bank_grad(gi, cl, g["dK_ctx"], g["dV_ctx"], dKb, dVb, ws_s, st)
+
+    def barrier():
+        ranks.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    barrier()
+    assert msa.msa_workspace_status(ws, st) == 0
+    Kst = max(1, min(args.steps, 20))
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(st)
+    for _ in range(Kst):
+        step()
+    e1.record(st)
+    barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / Kst
+    ms, = ranks.max([ms], dev)
+    # visible pairs: every row sees the memory rows and local rows up to L - T + t
+    pairs = B * w.h_q * sum(mc + L - T + t + 1 for t in range(T))
+    flop = 5 * 2.0 * pairs * w.d  # dP = dO V^T, dV = P^T dO, dK = dS^T Q, dQ = dS K (+ S again)
+    sustained = 1410.6
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            sustained = float(json.load(f)["bf16_tflops_sustained"])
+        kind = "measured (sustained)"
+    except Exception:
+        kind = "fallback (sustained)"
+    tflops = flop / (ms / 1e3) / 1e12
+    # end to end: inputs from pinned host memory, gradients read back, per step
+    hQ, hK, hV, hc, hd = (t.cpu().pin_memory() for t in (Q, Kl, Vl, cK, dO))
+    houts = {k: v.cpu().pin_memory() for k, v in g.items() if k in ("dQ", "dK_loc", "dV_loc")}
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hc, hd)) + hc.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in houts.values())
+
+    def e2e_step():
+        with torch.cuda.stream(st):
+            for dst, src in ((Q, hQ), (Kl, hK), (Vl, hV), (cK, hc), (cV, hc), (dO, hd)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for k, h in houts.items():
+                h.copy_(g[k], non_blocking=True)
+
+    e2e_step()
+    barrier()
+    Ke = max(3, Kst // 2)
+    e0.record(st)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(st)
+    barrier()
+    e_ms = e0.elapsed_time(e1) / Ke
+    e_ms, = ranks.max([e_ms], dev)
+    line = {
+        "metric": "MSA sparse-attention backward TFLOP/s (5 products over the visible pairs; "
+                  "forward recompute and bank scatter inside the timed call)",
+        "value": round(replica_rate(world, tflops, 1e3), 1), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": Kst, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normals)",
+        "config": {"workload": "attend_bwd", "batch": B, "T": T, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "d": w.d, "memory_rows": mc, "local_rows": L,
+                   "l2": "no flush: the local K/V read per call (135 MB) exceeds the 126 MB L2"},
+        "roofline": {"kernel": "msa_sparse_attend_backward (whole call)", "bound": "tensor",
+                     "achieved": round(tflops, 1), "peak": sustained, "unit": "TFLOP/s",
+                     "frac": round(tflops / sustained, 4), "peak_kind": kind, "traffic": None,
+                     "flop_per_call": flop},
+        "e2e": {"value": round(replica_rate(world, flop / 1e12, e_ms), 1), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
+        "gpu_launches": Kst * 8,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
 def run_generate(args):
     """Sparse generation at the 100M-token bank: context construction once per request, then
     ``--gen-tokens`` decode steps through all routed layers; generated tokens/s."""
@@ -1294,6 +1421,8 @@ def main():
         run_generate(args)
     elif args.workload == "encode_hidden1m":
         run_encode_hidden(args)
+    elif args.workload == "attend_bwd":
+        run_attend_backward(args)
     else:
         run_libmsa(args)
 

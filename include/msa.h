@@ -67,6 +67,16 @@ const char* msa_last_error(void);
 /* ABI version, (major << 16) | minor. */
 int msa_version(void);
 
+/* msa_set_device_wait_limit - the limit, in SM clock cycles, after which the consumer-side
+ * waits of the tensor-core routing scan (its MMA issuer waiting for operand tiles, its epilogue
+ * waiting for accumulators) give up: the kernel then records MSA_ERR_DEVICE's code 1 in the
+ * workspace status word, stops issuing, lets the copies and MMAs it issued land, frees its
+ * tensor memory and returns (outputs undefined). Copies in flight are always waited for with the
+ * default limit. cycles <= 0 restores the default (2^31 cycles, about a second). Process-wide,
+ * read when a call is enqueued; returns the previous setting (0 = default). For testing the
+ * error path; the pages describing MSA have no counterpart. */
+int64_t msa_set_device_wait_limit(int64_t cycles);
+
 /* ------------------------------------------------------------------------------------
  * Bank layout helper (host only, no device work).
  * Number of chunks of a corpus whose document d owns tokens
@@ -275,6 +285,67 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
                              int32_t max_ctx, int32_t h_kv, int32_t d, int32_t dtype,
                              int32_t pos0, float rope_base, float scale, void* O, void* ws,
                              size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * msa_sparse_attend_backward - gradients of msa_sparse_attend with respect to its inputs.
+ *   [ruixiangma.github.io blog, "训练策略": MSA is trained on the generation loss plus an
+ *    auxiliary routing loss; news.neo-ai.one article, "プロジェクト概要", Fig. 1: top-k
+ *    selection fused with the sparse attention keeps the model differentiable end to end]
+ *
+ * Same forward operation and arguments as msa_sparse_attend (Q, K_loc, V_loc, ctxK, ctxV,
+ * ctx_len, max_ctx, h_kv, d, dtype, pos0, rope_base, scale), plus the output gradient
+ * dO [B, T, h_q, d] (dtype). Writes fp32 gradients:
+ *   dQ      [B, T, h_q, d]        with respect to Q (before RoPE);
+ *   dK_loc  [B, L_loc, h_kv, d]   with respect to K_loc (before RoPE);
+ *   dV_loc  [B, L_loc, h_kv, d];
+ *   dK_ctx, dV_ctx [B, max_ctx, h_kv, d] with respect to the gathered memory rows (rows past
+ *           ctx_len[b]: 0). msa_scatter_bank_grad adds them into the bank rows.
+ * The softmax is recomputed (the forward again, in the workspace); probabilities and dS enter
+ * the tensor-core products in bf16, accumulation is fp32. Routing (top-k) has no gradient.
+ * Supported: bf16, d = 128, h_q / h_kv dividing 64 (else MSA_ERR_UNSUPPORTED). ws:
+ * msa_sparse_attend_backward_workspace(...) bytes, 256-byte aligned; its status word records
+ * an expired device wait.
+ */
+size_t msa_sparse_attend_backward_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv,
+                                            int32_t d, int32_t max_ctx, int32_t L_loc);
+msa_status msa_sparse_attend_backward(const void* Q, int32_t B, int32_t T, int32_t h_q,
+                                      const void* K_loc, const void* V_loc, int32_t L_loc,
+                                      const void* ctxK, const void* ctxV, const int32_t* ctx_len,
+                                      int32_t max_ctx, int32_t h_kv, int32_t d, int32_t dtype,
+                                      int32_t pos0, float rope_base, float scale, const void* dO,
+                                      float* dQ, float* dK_loc, float* dV_loc, float* dK_ctx,
+                                      float* dV_ctx, void* ws, size_t ws_bytes, void* stream);
+
+/* msa_scatter_bank_grad - the gathered rows' gradients flow back into the memory bank:
+ * dKbar[gather_idx[b, j]] += dK_ctx[b, j] and dVbar[...] += dV_ctx[b, j] for j < ctx_len[b]
+ * (fp32 [n_chunks, h_kv, d], accumulated with atomics: several queries may gather one
+ * document). gather_idx, ctx_len as written by msa_gather. An index outside [0, n_chunks) is
+ * skipped and recorded in the status word of ws (>= 256 bytes, 256-byte aligned). */
+msa_status msa_scatter_bank_grad(const int32_t* gather_idx, const int32_t* ctx_len, int32_t B,
+                                 int32_t max_ctx, int32_t h_kv, int32_t d, const float* dK_ctx,
+                                 const float* dV_ctx, float* dKbar, float* dVbar,
+                                 int64_t n_chunks, void* ws, size_t ws_bytes, void* stream);
+
+/* msa_aux_routing_loss - the auxiliary routing loss of training and its gradients.
+ *   [ruixiangma.github.io blog, "训练策略": the router is trained with an auxiliary loss, a
+ *    supervised contrastive loss between relevant and irrelevant document chunks, next to the
+ *    generation loss. The pages give no formula; this is a reading, so its agreement with the
+ *    authors' loss is not pinned.]
+ * Chunk scores as in routing before the document maximum:
+ *   s[b, c] = max_t (1/h_qr) sum_h cos(Q_r[b, t, h], Kbar_r[c, g(h)]);
+ * positives: bit c of positive_bits[b, ceil(n_chunks/32)] marks chunk c relevant to query b;
+ *   loss = mean over queries with positives of -(1/|P_b|) sum_{c in P_b} log softmax_c(s[b,:]/tau)
+ * written to loss (one fp32 in device memory). Gradients (fp32, nullable): dQ_r [B, T, h_qr, d]
+ * and dKbar_r [n_chunks, h_kv, d]; the token maximum passes its gradient to the first maximising
+ * token. fp32 or bf16 inputs, d in {64, 128}. ws: msa_aux_routing_loss_workspace(B, n_chunks)
+ * bytes, 256-byte aligned. The gradient of Q_r gathers over the chunks per query row (cost
+ * B*T*h_qr*n_chunks): meant for training-sized banks. */
+size_t msa_aux_routing_loss_workspace(int32_t B, int64_t n_chunks);
+msa_status msa_aux_routing_loss(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
+                                const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                                int32_t dtype, const uint32_t* positive_bits, float tau,
+                                float* loss, float* dQ_r, float* dKbar_r, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * msa_assemble_local - the local context of a Memory Interleaving round: for every query b,

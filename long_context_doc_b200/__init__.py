@@ -27,14 +27,17 @@ STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "M
 LIB_PATH = _build.LIB
 
 # every symbol include/msa.h declares
-SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_count_chunks",
+SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_set_device_wait_limit",
+           "msa_count_chunks",
            "msa_encode_pool", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
            "msa_route_topk", "msa_route_topk_noalloc", "msa_route_topk_noalloc_status",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
            "msa_sparse_attend", "msa_assemble_local", "msa_kv_append",
            "msa_decode_step_workspace", "msa_decode_step", "msa_encode_hidden_workspace",
-           "msa_encode_hidden")
+           "msa_encode_hidden", "msa_sparse_attend_backward_workspace",
+           "msa_sparse_attend_backward", "msa_scatter_bank_grad", "msa_aux_routing_loss_workspace",
+           "msa_aux_routing_loss")
 
 
 class MSAError(RuntimeError):
@@ -55,6 +58,8 @@ def _load():
     L.msa_last_error.restype = ctypes.c_char_p
     L.msa_last_error.argtypes = []
     L.msa_version.restype = ctypes.c_int
+    L.msa_set_device_wait_limit.restype = i64
+    L.msa_set_device_wait_limit.argtypes = [i64]
     L.msa_count_chunks.restype = i64
     L.msa_count_chunks.argtypes = [vp, i64, i32]
     L.msa_encode_pool.restype = ctypes.c_int
@@ -105,6 +110,19 @@ def _load():
     L.msa_encode_hidden.restype = ctypes.c_int
     L.msa_encode_hidden.argtypes = [vp, i64, i32, vp, vp, vp, vp, i64, i32, i32, i32, i32, f32, vp,
                                     vp, vp, vp, i64, vp, sz, vp]
+    L.msa_sparse_attend_backward_workspace.restype = sz
+    L.msa_sparse_attend_backward_workspace.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    L.msa_sparse_attend_backward.restype = ctypes.c_int
+    L.msa_sparse_attend_backward.argtypes = [vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, i32, i32,
+                                             i32, i32, i32, f32, f32, vp, vp, vp, vp, vp, vp, vp,
+                                             sz, vp]
+    L.msa_scatter_bank_grad.restype = ctypes.c_int
+    L.msa_scatter_bank_grad.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, i64, vp, sz, vp]
+    L.msa_aux_routing_loss_workspace.restype = sz
+    L.msa_aux_routing_loss_workspace.argtypes = [i32, i64]
+    L.msa_aux_routing_loss.restype = ctypes.c_int
+    L.msa_aux_routing_loss.argtypes = [vp, i32, i32, i32, vp, i64, i32, i32, i32, vp, f32, vp, vp,
+                                       vp, vp, sz, vp]
     L.msa_decode_step.restype = ctypes.c_int
     L.msa_decode_step.argtypes = [vp, vp, vp, i32, i32, i32, vp, vp, i32, vp, vp, vp, vp, i32, i32,
                                   i32, i32, i32, f32, f32, vp, vp, sz, vp]
@@ -235,6 +253,12 @@ def msa_route_topk_noalloc(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_b
                                       _p(top_ids), _p(top_scores), _p(doc_scores), _s(stream)))
 
 
+def msa_set_device_wait_limit(cycles: int) -> int:
+    """Consumer-side device wait limit of the tensor-core routing scan (SM clocks; 0: default).
+    Returns the previous setting."""
+    return int(lib.msa_set_device_wait_limit(int(cycles)))
+
+
 def msa_route_topk_noalloc_status(stream=None) -> int:
     """Status word of msa_route_topk_noalloc's built-in scratch (0 = no device error)."""
     code = ctypes.c_int32(0)
@@ -307,6 +331,38 @@ def msa_sparse_attend(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0, rope_base, sca
     _check(lib.msa_sparse_attend(_p(Q), B, T, h_q, _p(K_loc), _p(V_loc), L_loc, _p(ctxK), _p(ctxV),
                                  _p(ctx_len), max_ctx, h_kv, d, dtype_code(Q), pos0, rope_base,
                                  scale, _p(O), _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def msa_sparse_attend_backward_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc) -> int:
+    return int(lib.msa_sparse_attend_backward_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc))
+
+
+def msa_sparse_attend_backward(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0, rope_base, scale, dO,
+                               dQ, dK_loc, dV_loc, dK_ctx, dV_ctx, ws, stream=None):
+    B, T, h_q, d = Q.shape
+    L_loc, h_kv = K_loc.shape[1], K_loc.shape[2]
+    _check(lib.msa_sparse_attend_backward(
+        _p(Q), B, T, h_q, _p(K_loc), _p(V_loc), L_loc, _p(ctxK), _p(ctxV), _p(ctx_len),
+        ctxK.shape[1], h_kv, d, dtype_code(Q), pos0, rope_base, scale, _p(dO), _p(dQ),
+        _p(dK_loc), _p(dV_loc), _p(dK_ctx), _p(dV_ctx), _p(ws), ws.numel() * ws.element_size(),
+        _s(stream)))
+
+
+def msa_scatter_bank_grad(gather_idx, ctx_len, dK_ctx, dV_ctx, dKbar, dVbar, ws, stream=None):
+    B, max_ctx, h_kv, d = dK_ctx.shape
+    _check(lib.msa_scatter_bank_grad(_p(gather_idx), _p(ctx_len), B, max_ctx, h_kv, d,
+                                     _p(dK_ctx), _p(dV_ctx), _p(dKbar), _p(dVbar),
+                                     dKbar.shape[0], _p(ws), ws.numel() * ws.element_size(),
+                                     _s(stream)))
+
+
+def msa_aux_routing_loss(Q_r, Kbar_r, positive_bits, tau, loss, dQ_r, dKbar_r, ws, stream=None):
+    B, T, h_qr, d = Q_r.shape
+    n_chunks, h_kv = Kbar_r.shape[0], Kbar_r.shape[1]
+    _check(lib.msa_aux_routing_loss(_p(Q_r), B, T, h_qr, _p(Kbar_r), n_chunks, h_kv, d,
+                                    dtype_code(Q_r), _p(positive_bits), tau, _p(loss), _p(dQ_r),
+                                    _p(dKbar_r), _p(ws), ws.numel() * ws.element_size(),
+                                    _s(stream)))
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -461,3 +517,55 @@ def decode_step(cache: LocalCache, Q, K_new, V_new, ctxK, ctxV, ctx_len, scale: 
                     rope_base, scale, O, ws, stream)
     return O
 
+
+
+def sparse_attend_backward(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0: int, rope_base: float,
+                           dO, scale: float = 0.0, ws=None, stream=None) -> dict:
+    """Gradients of ``sparse_attend`` for the output gradient dO; returns fp32 dict(dQ, dK_loc,
+    dV_loc, dK_ctx, dV_ctx)."""
+    B, T, h_q, d = Q.shape
+    L_loc, h_kv = K_loc.shape[1], K_loc.shape[2]
+    max_ctx = ctxK.shape[1]
+    dev = Q.device
+    f32 = torch.float32
+    out = dict(dQ=torch.empty((B, T, h_q, d), dtype=f32, device=dev),
+               dK_loc=torch.empty((B, L_loc, h_kv, d), dtype=f32, device=dev),
+               dV_loc=torch.empty((B, L_loc, h_kv, d), dtype=f32, device=dev),
+               dK_ctx=torch.empty((B, max_ctx, h_kv, d), dtype=f32, device=dev),
+               dV_ctx=torch.empty((B, max_ctx, h_kv, d), dtype=f32, device=dev))
+    if ws is None:
+        ws = _ws(msa_sparse_attend_backward_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc), dev)
+    msa_sparse_attend_backward(Q, K_loc, V_loc, ctxK, ctxV, ctx_len, pos0, rope_base, scale, dO,
+                               out["dQ"], out["dK_loc"], out["dV_loc"], out["dK_ctx"],
+                               out["dV_ctx"], ws, stream)
+    return out
+
+
+def scatter_bank_grad(gather_idx, ctx_len, dK_ctx, dV_ctx, n_chunks: int, dKbar=None,
+                      dVbar=None, ws=None, stream=None):
+    """Adds the gathered rows' gradients into fp32 bank gradients [n_chunks, h_kv, d] (zeros
+    unless given); returns (dKbar, dVbar)."""
+    h_kv, d = dK_ctx.shape[2], dK_ctx.shape[3]
+    dev = dK_ctx.device
+    if dKbar is None:
+        dKbar = torch.zeros((n_chunks, h_kv, d), dtype=torch.float32, device=dev)
+    if dVbar is None:
+        dVbar = torch.zeros((n_chunks, h_kv, d), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _ws(256, dev)
+    msa_scatter_bank_grad(gather_idx, ctx_len, dK_ctx, dV_ctx, dKbar, dVbar, ws, stream)
+    return dKbar, dVbar
+
+
+def aux_routing_loss(Q_r, Kbar_r, positive_bits, tau: float = 0.1, stream=None):
+    """Auxiliary routing loss over the chunk scores and its gradients; positive_bits int32
+    [B, ceil(n_chunks/32)] (bit c: chunk c relevant). Returns (loss [1] fp32, dQ_r, dKbar_r)."""
+    B, T, h_qr, d = Q_r.shape
+    n_chunks = Kbar_r.shape[0]
+    dev = Q_r.device
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    dQ = torch.empty((B, T, h_qr, d), dtype=torch.float32, device=dev)
+    dK = torch.empty(tuple(Kbar_r.shape), dtype=torch.float32, device=dev)
+    ws = _ws(int(lib.msa_aux_routing_loss_workspace(B, n_chunks)), dev)
+    msa_aux_routing_loss(Q_r, Kbar_r, positive_bits, tau, loss, dQ, dK, ws, stream)
+    return loss, dQ, dK

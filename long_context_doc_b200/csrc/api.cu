@@ -2,6 +2,7 @@
 // validation, workspace sizing and kernel launches. No device memory is allocated here; the
 // only allocation is the pinned staging area of an msa_fetch context, made at set-up time.
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <chrono>
 #include <cmath>
@@ -96,6 +97,8 @@ void rope_turns(double base, int d, unsigned long long* out) {
 // Set the thread-local message returned by msa_last_error (for entry points defined in other
 // translation units).
 void set_last_error(const std::string& msg) { g_err = msg; }
+static std::atomic<long long> g_wait_limit{0};
+long long device_wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 }  // namespace msa
 
 extern "C" {
@@ -116,6 +119,10 @@ const char* msa_status_string(int s) {
 const char* msa_last_error(void) { return g_err.c_str(); }
 
 int msa_version(void) { return (1 << 16) | 0; }
+
+int64_t msa_set_device_wait_limit(int64_t cycles) {
+  return msa::g_wait_limit.exchange(cycles > 0 ? cycles : 0);
+}
 
 int64_t msa_count_chunks(const int64_t* off, int64_t n_docs, int32_t chunk) {
   if (off == nullptr || n_docs < 0 || chunk < 1) return -1;
@@ -286,6 +293,7 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
     ta.cand = reinterpret_cast<unsigned long long*>(base + kHeader + pl.q_bytes + pl.m_bytes);
     ta.counter = reinterpret_cast<unsigned int*>(base) + 1;
     ta.err = reinterpret_cast<int*>(base);
+    ta.wait_limit = msa::device_wait_limit();
     e = msa::launch_route_tc(ta, pl, st);
     if (e != cudaSuccess) return cuda_fail(e, "msa_route_topk (tensor-core scan) launch");
     return ok();
@@ -651,6 +659,131 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
   p.O = O;
   cudaError_t e = msa::launch_attend(p, dtype, (double)rope_base, pos0, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
+  return ok();
+}
+
+// ----------------------------------------------------------------------------- backward
+size_t msa_sparse_attend_backward_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv,
+                                            int32_t d, int32_t max_ctx, int32_t L_loc) {
+  const msa::BwdPlan pl = msa::attend_bwd_plan(B, T, h_q, h_kv, d, max_ctx, L_loc);
+  if (!pl.ok) return kHeader;
+  return kHeader + pl.fwd_bytes + pl.o_bytes + 2 * pl.lse_bytes;
+}
+
+msa_status msa_sparse_attend_backward(const void* Q, int32_t B, int32_t T, int32_t h_q,
+                                      const void* K_loc, const void* V_loc, int32_t L_loc,
+                                      const void* ctxK, const void* ctxV, const int32_t* ctx_len,
+                                      int32_t max_ctx, int32_t h_kv, int32_t d, int32_t dtype,
+                                      int32_t pos0, float rope_base, float scale, const void* dO,
+                                      float* dQ, float* dK_loc, float* dV_loc, float* dK_ctx,
+                                      float* dV_ctx, void* ws, size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 0 && T >= 1 && L_loc >= T && max_ctx >= 0 && h_q >= 1, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d T=%d L_loc=%d max_ctx=%d)", B, T, L_loc, max_ctx);
+  REQUIRE(h_q % h_kv == 0, MSA_ERR_INVALID_ARG, "h_q %d not a multiple of h_kv %d", h_q, h_kv);
+  REQUIRE(dtype == MSA_BF16 && d == 128, MSA_ERR_UNSUPPORTED,
+          "the attention backward runs on bf16 with d = 128");
+  const msa::BwdPlan pl = msa::attend_bwd_plan(B, T, h_q, h_kv, d, max_ctx, L_loc);
+  REQUIRE(pl.ok, MSA_ERR_UNSUPPORTED, "h_q / h_kv = %d must divide 64", h_q / h_kv);
+  if (B == 0) return ok();
+  REQUIRE(Q && K_loc && V_loc && ctx_len && dO && dQ && dK_loc && dV_loc, MSA_ERR_INVALID_ARG,
+          "null tensor");
+  REQUIRE(max_ctx == 0 || (ctxK && ctxV && dK_ctx && dV_ctx), MSA_ERR_INVALID_ARG,
+          "null context");
+  REQUIRE(aligned16(Q) && aligned16(K_loc) && aligned16(V_loc) && aligned16(dO) &&
+              aligned16(dQ) && aligned16(dK_loc) && aligned16(dV_loc) &&
+              (max_ctx == 0 || (aligned16(ctxK) && aligned16(ctxV) && aligned16(dK_ctx) &&
+                                aligned16(dV_ctx))),
+          MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const size_t need = msa_sparse_attend_backward_workspace(B, T, h_q, h_kv, d, max_ctx, L_loc);
+  REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
+  unsigned char* w8 = static_cast<unsigned char*>(ws);
+  msa::BwdParams p{};
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.Kl = static_cast<const __nv_bfloat16*>(K_loc);
+  p.Vl = static_cast<const __nv_bfloat16*>(V_loc);
+  p.cK = static_cast<const __nv_bfloat16*>(ctxK);
+  p.cV = static_cast<const __nv_bfloat16*>(ctxV);
+  p.ctx_len = ctx_len;
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.B = B;
+  p.T = T;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.L = L_loc;
+  p.max_ctx = max_ctx;
+  p.rope = rope_base > 0.f ? 1 : 0;
+  p.pos0 = pos0;
+  msa::rope_turns(p.rope ? (double)rope_base : 0.0, 128, p.rope_turns);
+  p.scale = sc;
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.dQ = dQ;
+  p.dKl = dK_loc;
+  p.dVl = dV_loc;
+  p.dKc = dK_ctx;
+  p.dVc = dV_ctx;
+  p.err = reinterpret_cast<int*>(w8);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);  // status word
+  if (e == cudaSuccess) e = msa::launch_attend_bwd(p, pl, w8 + kHeader, sm_count(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend_backward launch");
+  return ok();
+}
+
+msa_status msa_scatter_bank_grad(const int32_t* gather_idx, const int32_t* ctx_len, int32_t B,
+                                 int32_t max_ctx, int32_t h_kv, int32_t d, const float* dK_ctx,
+                                 const float* dV_ctx, float* dKbar, float* dVbar,
+                                 int64_t n_chunks, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE(B >= 0 && max_ctx >= 0 && h_kv >= 1 && (d == 64 || d == 128) && n_chunks >= 0,
+          MSA_ERR_INVALID_ARG, "bad sizes (B=%d max_ctx=%d h_kv=%d d=%d)", B, max_ctx, h_kv, d);
+  REQUIRE(ws && ws_bytes >= kHeader && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "needs a 256-byte aligned workspace of >= 256 bytes");
+  if (B == 0 || max_ctx == 0) return ok();
+  REQUIRE(gather_idx && ctx_len && dK_ctx && dV_ctx && dKbar && dVbar, MSA_ERR_INVALID_ARG,
+          "null tensor");
+  REQUIRE(aligned16(dK_ctx) && aligned16(dV_ctx) && aligned16(dKbar) && aligned16(dVbar),
+          MSA_ERR_INVALID_ARG, "gradients must be 16-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess)
+    e = msa::launch_scatter_bank_grad(gather_idx, ctx_len, B, max_ctx, (int64_t)h_kv * d, dK_ctx,
+                                      dV_ctx, dKbar, dVbar, n_chunks,
+                                      static_cast<int*>(ws), sm_count(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_scatter_bank_grad launch");
+  return ok();
+}
+
+size_t msa_aux_routing_loss_workspace(int32_t B, int64_t n_chunks) {
+  if (B < 1 || n_chunks < 1) return kHeader;
+  return kHeader + msa::aux_loss_scratch_bytes(B, n_chunks);
+}
+
+msa_status msa_aux_routing_loss(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
+                                const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
+                                int32_t dtype, const uint32_t* positive_bits, float tau,
+                                float* loss, float* dQ_r, float* dKbar_r, void* ws,
+                                size_t ws_bytes, void* stream) {
+  msa_status s = check_common(h_kv, d, dtype);
+  if (s != MSA_OK) return s;
+  REQUIRE(B >= 1 && T >= 1 && n_chunks >= 1, MSA_ERR_INVALID_ARG,
+          "bad sizes (B=%d T=%d n_chunks=%lld)", B, T, (long long)n_chunks);
+  REQUIRE(h_qr >= 1 && h_qr % h_kv == 0, MSA_ERR_INVALID_ARG, "h_qr %d not a multiple of h_kv %d",
+          h_qr, h_kv);
+  REQUIRE(tau > 0.f, MSA_ERR_INVALID_ARG, "tau must be positive");
+  REQUIRE(Q_r && Kbar_r && positive_bits && loss, MSA_ERR_INVALID_ARG, "null tensor");
+  const size_t need = msa_aux_routing_loss_workspace(B, n_chunks);
+  REQUIRE(ws != nullptr && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0,
+          MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu (256-byte aligned)", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int32_t), st);
+  if (e == cudaSuccess)
+    e = msa::launch_aux_routing_loss(Q_r, B, T, h_qr, Kbar_r, n_chunks, h_kv, d, dtype,
+                                     positive_bits, tau, loss, dQ_r, dKbar_r,
+                                     static_cast<unsigned char*>(ws) + kHeader, sm_count(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_aux_routing_loss launch");
   return ok();
 }
 

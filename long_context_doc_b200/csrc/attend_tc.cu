@@ -486,12 +486,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       fence_after();
       const float lt = l + xsum[(half ^ 1) * 128 + row];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      if (p.lse != nullptr && half == 0 && row_ok && !*abort_flag)  // for the backward
+        p.lse[((int64_t)b * p.h_kv + g) * p.lse_stride + qt * kM + row] = m + log2f(lt);
       __nv_bfloat16* out = p.O + (((int64_t)b * p.T + tok) * p.h_q + hq) * kD + half * 64;
 #pragma unroll 1
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t r[32];
         ld32(lane_base + 2u * kN + col0 + ch * 32, r);
-        if (row_ok && !*abort_flag) {
+        if (row_ok && !*abort_flag && p.O32 != nullptr) {
+          float* o32 = p.O32 + (((int64_t)b * p.T + tok) * p.h_q + hq) * kD + half * 64 + ch * 32;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(o32 + 4 * q4) =
+                make_float4(__uint_as_float(r[4 * q4]) * inv, __uint_as_float(r[4 * q4 + 1]) * inv,
+                            __uint_as_float(r[4 * q4 + 2]) * inv,
+                            __uint_as_float(r[4 * q4 + 3]) * inv);
+        } else if (row_ok && !*abort_flag) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
             uint32_t w[4];
@@ -521,11 +531,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
 // ------------------------------------------------------------------------------ host side
 
-AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L) {
+AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L,
+                       bool any_rows) {
   AtcPlan pl{};
   const int Gq = h_kv > 0 ? h_q / h_kv : 0;
   pl.ok = d == atc::kD && B >= 1 && T >= 1 && L >= T && Gq >= 1 && atc::kM % Gq == 0 &&
-          Gq * T >= 64;
+          (any_rows || Gq * T >= 64);
   if (!pl.ok) return pl;
   pl.n_qtiles = (Gq * T + atc::kM - 1) / atc::kM;
   pl.Lp = (L + 7) / 8 * 8;

@@ -12,6 +12,8 @@ namespace msa {
 
 // api.cu: thread-local message of msa_last_error
 void set_last_error(const std::string& msg);
+// api.cu: the device wait limit set by msa_set_device_wait_limit (0: default)
+long long device_wait_limit();
 
 // ---- encode_pool.cu
 struct EncodeParams {
@@ -77,6 +79,7 @@ struct RouteTcArgs {
   unsigned long long* cand;  // workspace
   unsigned int* counter;
   int* err;
+  long long wait_limit;      // consumer-side device waits, SM clocks (0: default)
 };
 TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, int k, int sms);
 cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t st);
@@ -241,14 +244,64 @@ struct AtcParams {
   float scale_log2;
   int* err;                 // workspace status word
   __nv_bfloat16* O;         // [B, T, h_q, 128]
+  float* O32;               // nullable: O in fp32 instead of bf16 (the backward's D)
+  float* lse;               // nullable: per query row, log2 of the softmax denominator in the
+                            // units of scale_log2 * score ([B, h_kv, lse_stride], row
+                            // t * (h_q / h_kv) + head within the KV group)
+  int lse_stride;
 };
 struct AtcPlan {
   bool ok;
   int n_qtiles, Lp, Mp;     // query tiles per (query, KV head); padded row counts of V^T
   size_t q_bytes, k_bytes, vl_bytes, vc_bytes, smem;  // scratch: rotated Q, rotated K, V^T
 };
-AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L);
+// any_rows: accept fewer than 64 query rows per KV head (the backward's recompute)
+AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L,
+                       bool any_rows = false);
 cudaError_t launch_attend_tc(const AtcParams& p, const AtcPlan& pl, unsigned char* scratch,
                              int sms, cudaStream_t st);
+
+// ---- attend_bwd.cu: backward of the sparse attention on tensor cores (bf16, d = 128,
+// h_q / h_kv dividing 64)
+struct BwdParams {
+  const __nv_bfloat16* Q;   // [B, T, h_q, 128] (before RoPE)
+  const __nv_bfloat16* Kl;  // [B, L, h_kv, 128] (before RoPE)
+  const __nv_bfloat16* Vl;
+  const __nv_bfloat16* cK;  // [B, max_ctx, h_kv, 128]
+  const __nv_bfloat16* cV;
+  const int32_t* ctx_len;
+  const __nv_bfloat16* dO;  // [B, T, h_q, 128]
+  int B, T, h_q, h_kv, L, max_ctx;
+  int rope, pos0;
+  unsigned long long rope_turns[64];
+  float scale, scale_log2;
+  float* dQ;                // [B, T, h_q, 128] fp32 outputs
+  float* dKl;               // [B, L, h_kv, 128]
+  float* dVl;
+  float* dKc;               // [B, max_ctx, h_kv, 128]
+  float* dVc;
+  int* err;
+};
+struct BwdPlan {
+  bool ok;
+  AtcPlan fwd;              // the forward recompute (rotated Q and K, O, log-sum-exp)
+  int Gq, NQT, Rpad, CT, LT;
+  size_t fwd_bytes, o_bytes, lse_bytes, dq_bytes, smem;
+};
+BwdPlan attend_bwd_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L);
+cudaError_t launch_attend_bwd(const BwdParams& p, const BwdPlan& pl, unsigned char* scratch,
+                              int sms, cudaStream_t st);
+cudaError_t launch_scatter_bank_grad(const int32_t* gidx, const int32_t* ctx_len, int B,
+                                     int max_ctx, int64_t row_elems, const float* dKc,
+                                     const float* dVc, float* dKbar, float* dVbar, int64_t n_chunks,
+                                     int* err, int sms, cudaStream_t st);
+
+// ---- aux_loss.cu: auxiliary routing loss over the chunk scores and its gradients
+size_t aux_loss_scratch_bytes(int B, int64_t n_chunks);
+cudaError_t launch_aux_routing_loss(const void* Q_r, int B, int T, int h_qr, const void* Kbar_r,
+                                    int64_t n_chunks, int h_kv, int d, int dtype,
+                                    const uint32_t* pos, float tau, float* loss, float* dQ_r,
+                                    float* dKbar_r, unsigned char* scratch, int sms,
+                                    cudaStream_t st);
 
 }  // namespace msa

@@ -24,7 +24,10 @@
 // carry for documents that continue into the next tile) and keep an exact per-query top-k in
 // warp registers; the last CTA to finish merges the per-CTA candidates (no spinning).
 // Every wait is bounded; on expiry the CTA records an error in the workspace status word,
-// stops issuing work, drains what it issued and frees its TMEM.
+// stops issuing work, drains what it issued and frees its TMEM. The consumer-side waits (MMA
+// issuer, epilogue) take the limit msa_set_device_wait_limit sets; the producer's drain and the
+// wait for the last MMAs keep the default limit, so that no copy or MMA is in flight when the
+// CTA frees its TMEM and exits, and the epilogue warps decide to leave by a barrier vote.
 #include <cuda.h>
 
 #include <algorithm>
@@ -177,20 +180,35 @@ struct TcParams {
   unsigned long long* cand;  // [grid, B, k]
   unsigned int* counter;
   int* err;
+  long long wait_limit;  // consumer-side waits (MMA issuer, epilogue), SM clocks; 0: default
 };
 
 constexpr int kTcWin = 1024;  // document offsets cached in shared memory
 
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* err,
-                                             volatile int* abort_flag) {
+                                             volatile int* abort_flag,
+                                             long long limit = kDefaultWaitLimit) {
   if (*abort_flag) return false;
-  if (mbar_wait_bounded(bar, par, err)) return true;
+  if (mbar_wait_limited(bar, par, err, limit)) return true;
   *abort_flag = 1;
   return false;
 }
 
 __device__ __forceinline__ void epi_sync() {  // the 128 epilogue threads only
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// The same barrier, returning on every epilogue thread whether all 128 passed true: the
+// epilogue warps leave their loop together (their named barriers wait for all of them, and
+// tcgen05.ld is warp-collective).
+__device__ __forceinline__ bool epi_sync_and(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
 }
 
 // Work of a CTA: the chunk tiles (128 rows from the CTA's first chunk) of its document-aligned
@@ -255,6 +273,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   const int64_t D0 = docs[3], D1 = docs[4], cb = docs[5], ce = docs[6];
   const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
   const int64_t n_units = n_ct * p.n_qtiles;
+  // first chunk row a tile loads: tile ct covers chunks [cb + 128 ct, ...); the last tile of a
+  // range of at least 128 chunks is loaded ending at ce (its first rows repeat the previous
+  // tile's, just read and still in L2) instead of reading into the next CTA's range
+  auto load_row = [&](int64_t ct) -> int64_t {
+    return (ct == n_ct - 1 && ce - cb >= kTcBM) ? ce - kTcBM : cb + ct * kTcBM;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -264,7 +288,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       int64_t issued = 0;
       for (int64_t u = 0; u < n_units; ++u) {
         const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-        const int y_a = (int)(cb + ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
+        const int y_a = (int)load_row(ct), y_b = (int)(qt * p.NQ * p.T);
         for (int kk = 0; kk < n_k; ++kk) {
           if (issued >= S && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
           unsigned char* st = base + (size_t)s * stage_bytes;
@@ -289,12 +313,16 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       for (int64_t u = 0; u < n_units; ++u) {
         const int a = (int)(u & 1);
         const uint32_t aph = (uint32_t)((u >> 1) & 1);
-        if (u >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
+        if (u >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag, p.wait_limit))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * 256);
         bool ok = true;
         for (int kk = 0; kk < n_k; ++kk) {
-          if (!wait_or_fail(&full[s], ph, p.err, abort_flag)) { ok = false; break; }
+          if (!wait_or_fail(&full[s], ph, p.err, abort_flag, p.wait_limit)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           unsigned char* st = base + (size_t)s * stage_bytes;
           const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + a_bytes);
@@ -329,7 +357,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       const int a = (int)(u & 1);
       const uint32_t aph = (uint32_t)((u >> 1) & 1);
       const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-      if (!wait_or_fail(&tfull[a], aph, p.err, abort_flag)) { aborted = true; break; }
+      if (!epi_sync_and(wait_or_fail(&tfull[a], aph, p.err, abort_flag, p.wait_limit))) {
+        aborted = true;  // every epilogue thread leaves here
+        break;
+      }
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
       int q = 0, t = 0;
@@ -356,7 +387,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       if (qt != p.n_qtiles - 1) continue;
       // ---- chunk tile complete for every query: per-document max + top-k insertion
       epi_sync();
-      const int64_t c0 = cb + ct * kTcBM;
+      const int64_t c0 = cb + ct * kTcBM;     // first chunk new to this tile
+      const int64_t cl = load_row(ct);        // chunk of the tile's row 0 (<= c0)
       const int64_t tend = min(c0 + kTcBM, ce);
       const int64_t dcur = docs[ct & 1];
       if (dcur + kTcBM + 2 > docs[2] + kTcWin) {  // slide the document-offset window
@@ -383,7 +415,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
           bool fin = false;
           float sc = -INFINITY;
           if (valid) {
-            const int lo = (int)(max(ds, c0) - c0), hi = (int)(min(de, tend) - c0);
+            const int lo = (int)(max(ds, c0) - cl), hi = (int)(min(de, tend) - cl);
             for (int c = lo; c < hi; ++c) sc = fmaxf(sc, msc[c * p.B + b]);
             if (ds < c0) sc = fmaxf(sc, cr);
             fin = de <= tend;
@@ -547,6 +579,7 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t
   p.cand = a.cand;
   p.counter = a.counter;
   p.err = a.err;
+  p.wait_limit = a.wait_limit;
   e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)pl.smem);
   if (e != cudaSuccess) return e;

@@ -77,3 +77,27 @@ def test_noalloc_rejects_calls_beyond_its_scratch(msa, gpu):
         msa.msa_route_topk_noalloc(Q, d["Kbar_r"], d["inv"], d["coff"], 4, None, ids, sc, None,
                                    Kbar_r_hat=d["hat"])
     assert e.value.status == 2 and "scratch" in e.value.message
+
+
+def test_noalloc_status_reports_a_device_error_then_clears(msa, gpu):
+    """A device wait of the built-in-scratch call that runs out (the consumer-side limit cut to
+    a few dozen cycles) shows in msa_route_topk_noalloc_status; the next normal call clears it
+    and routes correctly."""
+    d = _inputs(gpu, True)
+    w = d["w"]
+    ref_ids, _, _ = msa.route_topk(d["Q_r"], d["Kbar_r"], d["inv"], d["coff"], w.k,
+                                   Kbar_r_hat=d["hat"])
+    ids = torch.empty((w.B, w.k), dtype=torch.int32, device=gpu)
+    sc = torch.empty((w.B, w.k), dtype=torch.float32, device=gpu)
+    prev = msa.msa_set_device_wait_limit(64)
+    try:
+        msa.msa_route_topk_noalloc(d["Q_r"], d["Kbar_r"], d["inv"], d["coff"], w.k, None, ids,
+                                   sc, None, Kbar_r_hat=d["hat"])
+        code = msa.msa_route_topk_noalloc_status()
+    finally:
+        msa.msa_set_device_wait_limit(prev)
+    assert code == 1
+    msa.msa_route_topk_noalloc(d["Q_r"], d["Kbar_r"], d["inv"], d["coff"], w.k, None, ids, sc,
+                               None, Kbar_r_hat=d["hat"])
+    assert msa.msa_route_topk_noalloc_status() == 0
+    assert torch.equal(ids, ref_ids)
