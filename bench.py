@@ -61,7 +61,7 @@ def parse():
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
                     choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long",
-                             "gen100m", "encode_hidden1m", "attend_bwd"])
+                             "gen100m", "encode_hidden1m", "attend_bwd", "fetch100m"])
     ap.add_argument("--gen-tokens", type=int, default=256,
                     help="gen100m: tokens generated per query after the context is built")
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
@@ -1036,6 +1036,117 @@ def run_attend_backward(args):
     ranks.close()
 
 
+def run_fetch(args):
+    """The host-bank fetch of the 100M-token bank decode, measured on its own and beside the
+    routing scan it overlaps: one routed layer (1.6M chunks), B = 4 queries, k = 16, the
+    selected documents' K̄/V̄ rows (16 docs x 8 chunks x 2 KB, K and V) read from pinned host
+    memory by (a) the zero-copy gather kernel on a side stream, (b) msa_fetch_begin/finish
+    (one cudaMemcpyAsync per run of consecutive selected chunks). CUDA events on the
+    launching streams; one JSON line."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    import synth
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.C4
+    dv = synth.dev_bank_workload(w, dev, layer=0, with_kv=False)
+    hat = msa.kr_normalize(dv.pop("Kbar_r"))
+    coff_h = dv["doc_chunk_off"]
+    coff = torch.from_numpy(coff_h).to(dev)
+    n_chunks = int(coff_h[-1])
+    Kh, Vh = Decode._host_bank(w, coff_h, dev)
+    main, side = torch.cuda.Stream(), torch.cuda.Stream()
+    B, k = w.B, w.k
+    max_ctx = k * int(np.max(np.diff(coff_h)))
+    ws_r = torch.empty(msa.msa_route_topk_workspace(B, 1, w.h_qr, w.h_kv, w.d, 1, w.n_docs,
+                                                    n_chunks, k), dtype=torch.uint8, device=dev)
+    ids = torch.empty((B, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, k), dtype=torch.float32, device=dev)
+    gi = torch.empty((B, max_ctx), dtype=torch.int32, device=dev)
+    cl = torch.empty(B, dtype=torch.int32, device=dev)
+    cK = torch.empty((B, max_ctx, w.h_kv, w.d), dtype=torch.bfloat16, device=dev)
+    cV = torch.empty_like(cK)
+    ws_g = torch.zeros(256, dtype=torch.uint8, device=dev)
+    fetcher = msa.Fetcher(B, k)
+
+    def route(st):
+        msa.msa_route_topk(dv["Q_r"], None, None, coff, k, None, ids, sc, None, ws_r, st, hat)
+
+    def gather(st):
+        msa.msa_gather(ids, coff, Kh, Vh, max_ctx, gi, cl, cK, cV, ws_g, st)
+
+    def memcpy_fetch(st):
+        fetcher.begin(ids, coff, max_ctx, gi, cl, ws_g, st)
+        fetcher.finish(coff_h, Kh, Vh, max_ctx, cK, cV, st, side, 10_000)
+
+    def timed(fn, st, n=20):
+        out = []
+        for _ in range(n):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            fn(st)
+            e1.record(st)
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1))
+        return statistics.median(out)
+
+    for _ in range(3):
+        route(main)
+        gather(main)
+        memcpy_fetch(main)
+    torch.cuda.synchronize()
+    n_rows = int(cl.sum().item())
+    row = w.h_kv * w.d * 2
+    fetch_bytes = 2 * n_rows * row
+    # runs of consecutive selected chunks (one cudaMemcpyAsync each, for K and for V)
+    runs = 0
+    for b in range(B):
+        g = gi[b, :int(cl[b])].cpu().numpy()
+        runs += int(1 + np.count_nonzero(np.diff(g) != 1)) if len(g) else 0
+    t_route = timed(route, main)
+    t_gather = timed(gather, side)
+    t_memcpy = timed(memcpy_fetch, main)
+
+    # routing with the fetch of another layer's selection running beside it on the side stream
+    def route_with(fetch_fn):
+        out = []
+        for _ in range(20):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            fetch_fn()
+            e0.record(main)
+            route(main)
+            e1.record(main)
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1))
+        return statistics.median(out)
+
+    def gather_side():
+        gather(side)
+
+    def memcpy_side():  # the copies go to the side stream; the ids are already on the host
+        fetcher.begin(ids, coff, max_ctx, gi, cl, ws_g, side)
+        fetcher.finish(coff_h, Kh, Vh, max_ctx, cK, cV, side, side, 10_000)
+
+    t_route_zc = route_with(gather_side)
+    t_route_mc = route_with(memcpy_side)
+    line = {"metric": "host-bank fetch of the 100M-token bank decode (one routed layer, B = 4)",
+            "workload": "fetch100m", "fetch_bytes": fetch_bytes, "context_rows": n_rows,
+            "memcpy_runs": runs, "route_ms": round(t_route, 4),
+            "zerocopy_gather": {"ms": round(t_gather, 4),
+                                "gbs": round(fetch_bytes / (t_gather / 1e3) / 1e9, 2),
+                                "route_ms_beside": round(t_route_zc, 4)},
+            "memcpy_fetch": {"ms": round(t_memcpy, 4),
+                             "gbs": round(fetch_bytes / (t_memcpy / 1e3) / 1e9, 2),
+                             "copies": 2 * runs, "route_ms_beside": round(t_route_mc, 4)},
+            "note": "memcpy ms spans msa_fetch_begin (gather indices + ids to the host) through "
+                    "the copies and the event the main stream waits on, host wait included"}
+    print(json.dumps(line), flush=True)
+    fetcher.close()
+
+
 def run_generate(args):
     """Sparse generation at the 100M-token bank: context construction once per request, then
     ``--gen-tokens`` decode steps through all routed layers; generated tokens/s."""
@@ -1423,6 +1534,8 @@ def main():
         run_encode_hidden(args)
     elif args.workload == "attend_bwd":
         run_attend_backward(args)
+    elif args.workload == "fetch100m":
+        run_fetch(args)
     else:
         run_libmsa(args)
 

@@ -68,10 +68,10 @@ const char* msa_last_error(void);
 int msa_version(void);
 
 /* msa_set_device_wait_limit - the limit, in SM clock cycles, after which the consumer-side
- * waits of the tensor-core routing scan (its MMA issuer waiting for operand tiles, its epilogue
- * waiting for accumulators) give up: the kernel then records MSA_ERR_DEVICE's code 1 in the
- * workspace status word, stops issuing, lets the copies and MMAs it issued land, frees its
- * tensor memory and returns (outputs undefined). Copies in flight are always waited for with the
+ * waits of the tensor-core routing scan (its epilogue warps waiting for the tensor cores'
+ * accumulators) give up: the kernel then records MSA_ERR_DEVICE's code 1 in the workspace
+ * status word, stops issuing, lets the copies and MMAs it issued land, frees its tensor memory
+ * and returns (outputs undefined). Copies and MMAs in flight are always waited for with the
  * default limit. cycles <= 0 restores the default (2^31 cycles, about a second). Process-wide,
  * read when a call is enqueued; returns the previous setting (0 = default). For testing the
  * error path; the pages describing MSA have no counterpart. */

@@ -254,8 +254,8 @@ def msa_route_topk_noalloc(Q_r, Kbar_r, kr_inv_norm, doc_chunk_off, k, exclude_b
 
 
 def msa_set_device_wait_limit(cycles: int) -> int:
-    """Consumer-side device wait limit of the tensor-core routing scan (SM clocks; 0: default).
-    Returns the previous setting."""
+    """Wait limit of the tensor-core routing scan's epilogue (SM clocks; 0: default). Returns the
+    previous setting."""
     return int(lib.msa_set_device_wait_limit(int(cycles)))
 
 

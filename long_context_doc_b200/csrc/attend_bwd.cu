@@ -25,7 +25,8 @@
 //      dQ^T = K^T dS^T                            (M = 128 dims, N = 64 rows, K = 128 keys)
 //    The last three read dO, Q and K as MN-major operands straight from the tiles loaded for
 //    the first two, and P^T / dS^T from the shared memory the softmax warps wrote them to, so
-//    nothing is transposed in global memory. Four warps (thread = TMEM lane = key row) form
+//    nothing is transposed in global memory. Eight warps (two per TMEM lane quarter: thread =
+//    key row x half of the tile's rows) form
 //    P^T = 2^(S^T * scale_log2 - lse) and dS^T under the visibility mask, then stage the tile's
 //    dQ^T (thread = head dimension) as [row][dim] rows in shared memory that the bulk-copy
 //    engine adds into the fp32 dQ accumulator (cp.reduce.async.bulk .add.f32, 512 bytes per
@@ -46,7 +47,8 @@ namespace abw {
 constexpr int kKeys = 128;      // keys per CTA (TMEM lanes of S^T, dK, dV)
 constexpr int kRows = 64;       // query rows per streamed tile
 constexpr int kD = 128;
-constexpr int kThreads = 192;   // warp 0 copies, warp 1 MMA, warps 2-5 softmax / epilogues
+constexpr int kThreads = 320;   // warp 0 copies, warp 1 MMA, warps 2-9 softmax / epilogues
+constexpr int kSoftmax = 256;   // softmax / epilogue threads
 constexpr uint32_t kKSlice = kKeys * 128;     // [128 keys][64 dims] bf16: 16 KB
 constexpr uint32_t kRSlice = kRows * 128;     // [64 rows][64 dims] bf16: 8 KB
 constexpr uint32_t kStageBytes = 4 * kRSlice + 1024;  // Q, dO (2 slices each), lse + D
@@ -133,15 +135,15 @@ __device__ __forceinline__ void bulk_wait_read_all() {  // sources of committed 
 __device__ __forceinline__ void bulk_wait_all() {  // committed groups complete
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-__device__ __forceinline__ void softmax_sync() {  // the 128 softmax / epilogue threads
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+__device__ __forceinline__ void softmax_sync() {  // the 256 softmax / epilogue threads
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
-// The same barrier, returning on every thread whether all 128 threads passed true: the
+// The same barrier, returning on every thread whether all 256 threads passed true: the
 // softmax warps leave their loop together (a named barrier waits for all of them).
 __device__ __forceinline__ bool softmax_sync_and(bool pred) {
   uint32_t r;
   asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n"
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 256, p;\n"
       " selp.u32 %0, 1, 0, q;\n}\n"
       : "=r"(r)
       : "r"((uint32_t)pred)
@@ -247,10 +249,10 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
   uint64_t* qfull = bars + 1;       // [2] stage landed
   uint64_t* qempty = bars + 3;      // [2] stage consumed by every MMA of its tile
   uint64_t* sfull = bars + 5;       // [2] S^T and dP^T of a TMEM buffer computed
-  uint64_t* pfull = bars + 7;       // P^T, dS^T written (128 threads)
+  uint64_t* pfull = bars + 7;       // P^T, dS^T written (256 threads)
   uint64_t* pempty = bars + 8;      // the MMAs reading P^T, dS^T completed
   uint64_t* dqfull = bars + 9;      // [2] dQ^T of a TMEM buffer computed
-  uint64_t* tfree = bars + 11;      // [2] dQ^T of a buffer drained (128 threads)
+  uint64_t* tfree = bars + 11;      // [2] dQ^T of a buffer drained (256 threads)
   uint64_t* done = bars + 13;       // every issued MMA completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -275,9 +277,9 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       mbar_init(&qempty[s], 1);
       mbar_init(&sfull[s], 1);
       mbar_init(&dqfull[s], 1);
-      mbar_init(&tfree[s], 128);
+      mbar_init(&tfree[s], kSoftmax);
     }
-    mbar_init(pfull, 128);
+    mbar_init(pfull, kSoftmax);
     mbar_init(pempty, 1);
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -390,19 +392,24 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       mbar_wait_bounded(done, 0, p.err);
     }
   } else {
-    // ---------------- softmax + epilogues: thread = TMEM lane (warps 2-5 -> quarters 2, 3, 0, 1)
+    // ---------------- softmax + epilogues: warps 2-9, two per TMEM lane quarter (warp w reads
+    // lanes 32 (w % 4) ..); thread = (lane = key row, half of the tile's 64 rows / of the dims)
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int kr = quarter * 32 + lane;           // key row (and head dim for dQ^T)
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int key = k0 + kr;
     const bool key_ok = kr < kvalid;
     const float c = p.scale_log2;
+    // a local key is visible to the tile rows r with token r / Gq >= key - (L - T): rows
+    // r >= rmin (memory keys: every valid row)
+    const int rmin = is_ctx ? 0 : max(0, key - (g.L - g.T)) * g.Gq;
     bool bad = false;
     int i = 0;
     for (; i < n_tiles && !bad; ++i) {
       const int s = i & 1, qt = qt0 + i;
       // the stage and S^T / dP^T have landed, and the MMAs of the previous tile no longer read
-      // P^T / dS^T; leaving is decided by all 128 threads together
+      // P^T / dS^T; leaving is decided by all 256 threads together
       bool ok = __all_sync(0xffffffffu, wait_or_abort(&qfull[s], (uint32_t)((i >> 1) & 1), p.err,
                                                       abort_flag) &&
                                             wait_or_abort(&sfull[s], (uint32_t)((i >> 1) & 1),
@@ -416,59 +423,54 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       }
       if (i == 0 && !key_ok) {
         // rows past the valid keys (memory rows past ctx_len hold whatever the buffer held):
-        // zero them in K so that dQ^T = K^T dS^T reads no stale values (their dS^T is 0)
+        // zero them in K so that dQ^T = K^T dS^T reads no stale values (their dS^T is 0); each
+        // half clears one of the two 64-dim slices
 #pragma unroll
-        for (int sl = 0; sl < 2; ++sl)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4*>(k_s + sl * kKSlice + kr * 128 + ch * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(k_s + half * kKSlice + kr * 128 + ch * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
       }
       fence_after();
       const unsigned char* st = stg + s * kStageBytes;
-      const float* lse_s = reinterpret_cast<const float*>(st + 4 * kRSlice);
+      const float* lse_s = reinterpret_cast<const float*>(st + 4 * kRSlice) + half * 32;
       const float* d_s = lse_s + 64;
-      // last visible local row per query row is L - T + t; memory keys are visible to every
-      // valid row
-      const int kvis_base = g.L - g.T;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {  // 32 rows per chunk
-        uint32_t sr[32], dr[32];
-        ld32(lane_base + (uint32_t)(s * 128 + ch * 32), sr);
-        ld32(lane_base + (uint32_t)(s * 128 + 64 + ch * 32), dr);
-        uint32_t pk[16], dk[16];
+      const int r0 = qt * kRows + half * 32;       // tile row of this thread's first column
+      const int lo_vis = max(rmin - r0, 0);        // columns [lo_vis, hi_vis) visible
+      const int hi_vis = key_ok ? min(32, g.R - r0) : 0;
+      uint32_t sr[32], dr[32];
+      ld32(lane_base + (uint32_t)(s * 128 + half * 32), sr);
+      ld32(lane_base + (uint32_t)(s * 128 + 64 + half * 32), dr);
+      uint32_t pk[16], dk[16];
+      const float sc = p.scale;
 #pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          float pv[2], dv[2];
+      for (int q = 0; q < 32; q += 2) {
+        float pv[2], dv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = ch * 32 + q + u;
-            const int r = qt * kRows + col;     // row within (query, KV head)
-            const int t = r / g.Gq;
-            const bool vis = key_ok && r < g.R && (is_ctx || key <= kvis_base + t);
-            const float pp = vis ? ex2(fmaf(__uint_as_float(sr[q + u]), c, -lse_s[col])) : 0.f;
-            pv[u] = pp;
-            dv[u] = vis ? pp * (__uint_as_float(dr[q + u]) - d_s[col]) * p.scale : 0.f;
-          }
-          const __nv_bfloat162 h0 = __floats2bfloat162_rn(pv[0], pv[1]);
-          const __nv_bfloat162 h1 = __floats2bfloat162_rn(dv[0], dv[1]);
-          pk[q >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
-          dk[q >> 1] = *reinterpret_cast<const uint32_t*>(&h1);
+        for (int u = 0; u < 2; ++u) {
+          const int col = q + u;
+          const bool vis = col >= lo_vis && col < hi_vis;
+          const float pp = vis ? ex2(fmaf(__uint_as_float(sr[col]), c, -lse_s[col])) : 0.f;
+          pv[u] = pp;
+          dv[u] = vis ? pp * (__uint_as_float(dr[col]) - d_s[col]) * sc : 0.f;
         }
+        const __nv_bfloat162 h0 = __floats2bfloat162_rn(pv[0], pv[1]);
+        const __nv_bfloat162 h1 = __floats2bfloat162_rn(dv[0], dv[1]);
+        pk[q >> 1] = *reinterpret_cast<const uint32_t*>(&h0);
+        dk[q >> 1] = *reinterpret_cast<const uint32_t*>(&h1);
+      }
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {  // 16-byte chunk index XOR row % 8 (128-byte swizzle)
-          const int chunk = ch * 4 + q4;
-          const int off = kr * 128 + ((chunk ^ (kr & 7)) << 4);
-          *reinterpret_cast<uint4*>(pt_s + off) =
-              make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-          *reinterpret_cast<uint4*>(dst_s + off) =
-              make_uint4(dk[4 * q4], dk[4 * q4 + 1], dk[4 * q4 + 2], dk[4 * q4 + 3]);
-        }
+      for (int q4 = 0; q4 < 4; ++q4) {  // 16-byte chunk index XOR row % 8 (128-byte swizzle)
+        const int chunk = half * 4 + q4;
+        const int off = kr * 128 + ((chunk ^ (kr & 7)) << 4);
+        *reinterpret_cast<uint4*>(pt_s + off) =
+            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        *reinterpret_cast<uint4*>(dst_s + off) =
+            make_uint4(dk[4 * q4], dk[4 * q4 + 1], dk[4 * q4 + 2], dk[4 * q4 + 3]);
       }
       fence_before();
       fence_proxy_async_smem();  // P^T, dS^T and the zeroed K rows are read by the tensor core
       mbar_arrive(pfull);
-      // dQ^T of this tile: thread = head dim kr, columns = the tile's rows
+      // dQ^T of this tile: thread = head dim kr, this half's 32 of the tile's rows
       if (!softmax_sync_and(__all_sync(0xffffffffu, wait_or_abort(&dqfull[s],
                                                                   (uint32_t)((i >> 1) & 1), p.err,
                                                                   abort_flag)))) {
@@ -476,26 +478,22 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         break;
       }
       fence_after();
-      uint32_t qr0[32], qr1[32];
-      ld32(lane_base + (uint32_t)(s * 128), qr0);
-      ld32(lane_base + (uint32_t)(s * 128 + 32), qr1);
+      uint32_t qr[32];
+      ld32(lane_base + (uint32_t)(s * 128 + half * 32), qr);
       fence_before();
       mbar_arrive(&tfree[s]);  // the TMEM buffer is drained into registers
       // the previous tile's reductions have read the staging rows; then every thread writes its
-      // head dim of the 64 rows ([row][dim] fp32) and one thread per warp adds 16 whole rows
+      // head dim of its 32 rows ([row][dim] fp32) and one thread per warp adds 8 whole rows
       // (512 bytes each) into the dQ accumulator with the bulk-copy engine
       if (lane == 0) bulk_wait_read_all();
       softmax_sync();
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        qst[q * kD + kr] = __uint_as_float(qr0[q]);
-        qst[(32 + q) * kD + kr] = __uint_as_float(qr1[q]);
-      }
+      for (int q = 0; q < 32; ++q) qst[(half * 32 + q) * kD + kr] = __uint_as_float(qr[q]);
       fence_proxy_async_smem();
       softmax_sync();
       if (lane == 0) {
-        const int wq = warp - 2;  // rows [16 wq, 16 wq + 16) of the tile
-        for (int q = 16 * wq; q < 16 * wq + 16; ++q) {
+        const int wq = warp - 2;  // rows [8 wq, 8 wq + 8) of the tile
+        for (int q = 8 * wq; q < 8 * wq + 8; ++q) {
           const int r = qt * kRows + q;
           if (r >= g.R) break;
           const int t = r / g.Gq, hq = gk * g.Gq + r % g.Gq;
@@ -506,8 +504,9 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       }
     }
     if (lane == 0) bulk_wait_all();  // the dQ reductions complete before the CTA exits
-    // epilogue: dK (rotated back for local keys) and dV of the tile's valid rows. The TMEM
-    // loads are warp-collective: every lane loads (a warp-uniform decision), valid rows store.
+    // epilogue: dK (rotated back for local keys) and dV of the tile's valid rows, this half's
+    // RoPE pairs (dims [32 half, 32 half + 32) and their partners 64 on). The TMEM loads are
+    // warp-collective: every lane loads (a warp-uniform decision), valid rows store.
     const bool fin = n_tiles > 0 && !bad &&
                      __all_sync(0xffffffffu, wait_or_abort(done, 0, p.err, abort_flag));
     const bool store = key_ok && !*abort_flag;
@@ -515,58 +514,54 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                        : p.dKl + (((int64_t)b * g.L + key) * g.h_kv + gk) * kD;
     float* dv = is_ctx ? p.dVc + (((int64_t)b * g.max_ctx + key) * g.h_kv + gk) * kD
                        : p.dVl + (((int64_t)b * g.L + key) * g.h_kv + gk) * kD;
+    const int e0 = half * 32;
     if (n_tiles == 0 && store) {  // no query row sees the key
-      for (int e = 0; e < kD; e += 4) {
-        *reinterpret_cast<float4*>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
-        *reinterpret_cast<float4*>(dv + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int e = 0; e < 32; e += 4) {
+        *reinterpret_cast<float4*>(dk + e0 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(dk + 64 + e0 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(dv + e0 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(dv + 64 + e0 + e) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     if (fin) {  // warp-uniform
-      {
-        fence_after();
-        const bool rot = !is_ctx && p.rope;
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {  // dims [32ch, 32ch+32) paired with [64+32ch, ...)
-          uint32_t lo[32], hi[32];
-          ld32(lane_base + 256u + ch * 32, lo);
-          ld32(lane_base + 256u + 64 + ch * 32, hi);
+      fence_after();
+      const bool rot = !is_ctx && p.rope;
+      uint32_t lo[32], hi[32];
+      ld32(lane_base + 256u + e0, lo);
+      ld32(lane_base + 256u + 64 + e0, hi);
 #pragma unroll
-          for (int q = 0; q < 32 && store; q += 4) {
-            float a[4], h[4];
+      for (int q = 0; q < 32 && store; q += 4) {
+        float a4[4], h4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float x = __uint_as_float(lo[q + u]), y = __uint_as_float(hi[q + u]);
-              if (rot) {
-                const float2 cs = rot_turns((int64_t)p.pos0 + key, p.rope_turns[ch * 32 + q + u]);
-                a[u] = x * cs.x + y * cs.y;
-                h[u] = y * cs.x - x * cs.y;
-              } else {
-                a[u] = x;
-                h[u] = y;
-              }
-            }
-            *reinterpret_cast<float4*>(dk + ch * 32 + q) = make_float4(a[0], a[1], a[2], a[3]);
-            *reinterpret_cast<float4*>(dk + 64 + ch * 32 + q) = make_float4(h[0], h[1], h[2], h[3]);
-          }
-          ld32(lane_base + 384u + ch * 32, lo);
-          ld32(lane_base + 384u + 64 + ch * 32, hi);
-#pragma unroll
-          for (int q = 0; q < 32 && store; q += 4) {
-            *reinterpret_cast<float4*>(dv + ch * 32 + q) =
-                make_float4(__uint_as_float(lo[q]), __uint_as_float(lo[q + 1]),
-                            __uint_as_float(lo[q + 2]), __uint_as_float(lo[q + 3]));
-            *reinterpret_cast<float4*>(dv + 64 + ch * 32 + q) =
-                make_float4(__uint_as_float(hi[q]), __uint_as_float(hi[q + 1]),
-                            __uint_as_float(hi[q + 2]), __uint_as_float(hi[q + 3]));
+        for (int u = 0; u < 4; ++u) {
+          const float x = __uint_as_float(lo[q + u]), y = __uint_as_float(hi[q + u]);
+          if (rot) {
+            const float2 cs = rot_turns((int64_t)p.pos0 + key, p.rope_turns[e0 + q + u]);
+            a4[u] = x * cs.x + y * cs.y;
+            h4[u] = y * cs.x - x * cs.y;
+          } else {
+            a4[u] = x;
+            h4[u] = y;
           }
         }
+        *reinterpret_cast<float4*>(dk + e0 + q) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+        *reinterpret_cast<float4*>(dk + 64 + e0 + q) = make_float4(h4[0], h4[1], h4[2], h4[3]);
+      }
+      ld32(lane_base + 384u + e0, lo);
+      ld32(lane_base + 384u + 64 + e0, hi);
+#pragma unroll
+      for (int q = 0; q < 32 && store; q += 4) {
+        *reinterpret_cast<float4*>(dv + e0 + q) =
+            make_float4(__uint_as_float(lo[q]), __uint_as_float(lo[q + 1]),
+                        __uint_as_float(lo[q + 2]), __uint_as_float(lo[q + 3]));
+        *reinterpret_cast<float4*>(dv + 64 + e0 + q) =
+            make_float4(__uint_as_float(hi[q]), __uint_as_float(hi[q + 1]),
+                        __uint_as_float(hi[q + 2]), __uint_as_float(hi[q + 3]));
       }
     }
-    // memory rows of the tile past ctx_len: zero gradients
+    // memory rows of the tile past ctx_len: zero gradients (each half its 64 dims)
     if (is_ctx && !key_ok && key < g.max_ctx && !*abort_flag) {
-      float* dk = p.dKc + (((int64_t)b * g.max_ctx + key) * g.h_kv + gk) * kD;
-      float* dv = p.dVc + (((int64_t)b * g.max_ctx + key) * g.h_kv + gk) * kD;
-      for (int e = 0; e < kD; e += 4) {
+      for (int e = 64 * half; e < 64 * half + 64; e += 4) {
         *reinterpret_cast<float4*>(dk + e) = make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<float4*>(dv + e) = make_float4(0.f, 0.f, 0.f, 0.f);
       }

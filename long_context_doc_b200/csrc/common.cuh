@@ -342,9 +342,9 @@ constexpr int kMergeCap = 256;  // survivors ranked directly, per warp
 // of the block). Each list is sorted (descending keys, 0 = empty) and the keys of different
 // lists are distinct. The lists are first copied into shared memory with every copy in
 // flight; warp w then takes queries w, w + nwarps, ...:
-//   tau = max(largest k-th key of a list, k-th largest list head): either way at least k
-//         distinct keys are >= tau, so the global top-k lies in the keys >= tau (the heads
-//         bound is close to the global k-th key, so few keys survive);
+//   tau = max(largest k-th key of a list, largest per-lane maximum of the list heads that at
+//         least k per-lane maxima reach): either way at least k distinct keys are >= tau,
+//         so the global top-k lies in the keys >= tau;
 //   the keys >= tau (a prefix of every list) are compacted into a per-warp buffer and each
 //         one's rank is the number of larger survivors: rank r < k goes to output slot r.
 // A query with more than kMergeCap survivors (or a block without the shared memory) falls
@@ -376,38 +376,19 @@ __device__ __forceinline__ void merge_candidates(const unsigned long long* cand,
       const unsigned long long kth = staged ? src[at] : __ldcg(src + at);
       tau = kth > tau ? kth : tau;
     }
-    // the k-th largest list head: heads of different lists are distinct documents, so at
-    // least k distinct keys reach it and the global k-th key does too. Taken by k rounds of
-    // warp-wide maximum extraction over the heads (each lane holds its lists' heads)
-    if (G >= k) {
-      constexpr int kMaxHeadsPerLane = 8;  // grids up to 256 CTAs
-      unsigned long long h[kMaxHeadsPerLane];
-#pragma unroll
-      for (int q = 0; q < kMaxHeadsPerLane; ++q) {
-        const int c = lane + 32 * q;
-        h[q] = 0ull;
-        if (c < G) h[q] = staged ? src[(c * B + b) * k] : __ldcg(src + (c * B + b) * k);
+    // lane maxima of the list heads: heads of different lists are distinct documents, so the
+    // largest lane maximum that k of the 32 lane maxima reach is a lower bound as well
+    {
+      unsigned long long hm = 0ull;
+      for (int c = lane; c < G; c += 32) {
+        const int at = (c * B + b) * k;
+        const unsigned long long h = staged ? src[at] : __ldcg(src + at);
+        hm = h > hm ? h : hm;
       }
-      if (G <= 32 * kMaxHeadsPerLane) {
-        unsigned long long kth = 0ull;
-        for (int it = 0; it < k; ++it) {
-          unsigned long long mx = 0ull;
+      int ge = 0;
 #pragma unroll
-          for (int q = 0; q < kMaxHeadsPerLane; ++q) mx = h[q] > mx ? h[q] : mx;
-          unsigned long long w = mx;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, w, o);
-            w = other > w ? other : w;
-          }
-          kth = w;
-          if (w == 0ull) break;  // fewer than k non-empty heads
-#pragma unroll
-          for (int q = 0; q < kMaxHeadsPerLane; ++q)
-            if (h[q] == w) h[q] = 0ull;  // keys are distinct: exactly one lane owns w
-        }
-        tau = kth > tau ? kth : tau;
-      }
+      for (int j = 0; j < 32; ++j) ge += __shfl_sync(0xffffffffu, hm, j) >= hm ? 1 : 0;
+      if (hm != 0ull && ge >= k) tau = hm > tau ? hm : tau;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {

@@ -24,10 +24,10 @@
 // carry for documents that continue into the next tile) and keep an exact per-query top-k in
 // warp registers; the last CTA to finish merges the per-CTA candidates (no spinning).
 // Every wait is bounded; on expiry the CTA records an error in the workspace status word,
-// stops issuing work, drains what it issued and frees its TMEM. The consumer-side waits (MMA
-// issuer, epilogue) take the limit msa_set_device_wait_limit sets; the producer's drain and the
-// wait for the last MMAs keep the default limit, so that no copy or MMA is in flight when the
-// CTA frees its TMEM and exits, and the epilogue warps decide to leave by a barrier vote.
+// stops issuing work, drains what it issued and frees its TMEM. The epilogue's waits for
+// accumulators take the limit msa_set_device_wait_limit sets (the MMA issuer's and the
+// producer's waits keep the default one: a limit check in the issue loop costs the scan ~1.5%,
+// measured), so that no copy or MMA is in flight when the CTA frees its TMEM and exits.
 #include <cuda.h>
 
 #include <algorithm>
@@ -180,7 +180,7 @@ struct TcParams {
   unsigned long long* cand;  // [grid, B, k]
   unsigned int* counter;
   int* err;
-  long long wait_limit;  // consumer-side waits (MMA issuer, epilogue), SM clocks; 0: default
+  long long wait_limit;  // the epilogue's waits for accumulators, SM clocks; 0: default
 };
 
 constexpr int kTcWin = 1024;  // document offsets cached in shared memory
@@ -196,19 +196,6 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t par, int* e
 
 __device__ __forceinline__ void epi_sync() {  // the 128 epilogue threads only
   asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-// The same barrier, returning on every epilogue thread whether all 128 passed true: the
-// epilogue warps leave their loop together (their named barriers wait for all of them, and
-// tcgen05.ld is warp-collective).
-__device__ __forceinline__ bool epi_sync_and(bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n"
-      " selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred)
-      : "memory");
-  return r != 0;
 }
 
 // Work of a CTA: the chunk tiles (128 rows from the CTA's first chunk) of its document-aligned
@@ -238,6 +225,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(docs + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* last_flag = const_cast<int*>(abort_flag) + 1;
+  // epilogue give-up flags, one per chunk-tile parity: written (only by epilogue threads whose
+  // wait failed) before a chunk tile's barrier, read by all of them after it, so the four
+  // epilogue warps leave together; a flag is written again two chunk tiles later, after the
+  // next barrier, so no thread reads one that is being rewritten
+  volatile int* epi_abort = const_cast<int*>(abort_flag) + 2;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_k = p.K / kTcBK;
@@ -255,6 +247,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     }
     mbar_init(done, 1);
     *abort_flag = 0;
+    epi_abort[0] = 0;
+    epi_abort[1] = 0;
     fence_mbar_init();
   }
   for (int j = threadIdx.x; j < p.B * 32; j += kTcThreads) lists[j] = 0ull;
@@ -273,12 +267,6 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   const int64_t D0 = docs[3], D1 = docs[4], cb = docs[5], ce = docs[6];
   const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
   const int64_t n_units = n_ct * p.n_qtiles;
-  // first chunk row a tile loads: tile ct covers chunks [cb + 128 ct, ...); the last tile of a
-  // range of at least 128 chunks is loaded ending at ce (its first rows repeat the previous
-  // tile's, just read and still in L2) instead of reading into the next CTA's range
-  auto load_row = [&](int64_t ct) -> int64_t {
-    return (ct == n_ct - 1 && ce - cb >= kTcBM) ? ce - kTcBM : cb + ct * kTcBM;
-  };
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -288,7 +276,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       int64_t issued = 0;
       for (int64_t u = 0; u < n_units; ++u) {
         const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-        const int y_a = (int)load_row(ct), y_b = (int)(qt * p.NQ * p.T);
+        const int y_a = (int)(cb + ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
         for (int kk = 0; kk < n_k; ++kk) {
           if (issued >= S && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
           unsigned char* st = base + (size_t)s * stage_bytes;
@@ -313,16 +301,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       for (int64_t u = 0; u < n_units; ++u) {
         const int a = (int)(u & 1);
         const uint32_t aph = (uint32_t)((u >> 1) & 1);
-        if (u >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag, p.wait_limit))
-          break;
+        if (u >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * 256);
         bool ok = true;
         for (int kk = 0; kk < n_k; ++kk) {
-          if (!wait_or_fail(&full[s], ph, p.err, abort_flag, p.wait_limit)) {
-            ok = false;
-            break;
-          }
+          if (!wait_or_fail(&full[s], ph, p.err, abort_flag)) { ok = false; break; }
           tc_fence_after();
           unsigned char* st = base + (size_t)s * stage_bytes;
           const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + a_bytes);
@@ -357,15 +341,19 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       const int a = (int)(u & 1);
       const uint32_t aph = (uint32_t)((u >> 1) & 1);
       const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-      if (!epi_sync_and(wait_or_fail(&tfull[a], aph, p.err, abort_flag, p.wait_limit))) {
-        aborted = true;  // every epilogue thread leaves here
-        break;
+      // a warp whose wait fails skips the tensor-memory loads (warp-collective: a warp-uniform
+      // decision), flags the chunk tile and leaves with the others after its barrier
+      const bool got = !aborted && __all_sync(0xffffffffu, wait_or_fail(&tfull[a], aph, p.err,
+                                                                       abort_flag, p.wait_limit));
+      if (!got) {
+        aborted = true;
+        epi_abort[ct & 1] = 1;
       }
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
       int q = 0, t = 0;
       float cur = -INFINITY;
-      for (int col = 0; col < ncols; col += 32) {
+      for (int col = 0; got && col < ncols; col += 32) {
         float v[32];
         tmem_ld32(tbase + (uint32_t)col, v);
 #pragma unroll
@@ -383,12 +371,15 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[a]);
+      if (got) mbar_arrive(&tempty[a]);
       if (qt != p.n_qtiles - 1) continue;
       // ---- chunk tile complete for every query: per-document max + top-k insertion
       epi_sync();
-      const int64_t c0 = cb + ct * kTcBM;     // first chunk new to this tile
-      const int64_t cl = load_row(ct);        // chunk of the tile's row 0 (<= c0)
+      if (epi_abort[ct & 1]) {  // every epilogue thread leaves here
+        aborted = true;
+        break;
+      }
+      const int64_t c0 = cb + ct * kTcBM;
       const int64_t tend = min(c0 + kTcBM, ce);
       const int64_t dcur = docs[ct & 1];
       if (dcur + kTcBM + 2 > docs[2] + kTcWin) {  // slide the document-offset window
@@ -415,7 +406,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
           bool fin = false;
           float sc = -INFINITY;
           if (valid) {
-            const int lo = (int)(max(ds, c0) - cl), hi = (int)(min(de, tend) - cl);
+            const int lo = (int)(max(ds, c0) - c0), hi = (int)(min(de, tend) - c0);
             for (int c = lo; c < hi; ++c) sc = fmaxf(sc, msc[c * p.B + b]);
             if (ds < c0) sc = fmaxf(sc, cr);
             fin = de <= tend;
@@ -517,7 +508,7 @@ TcPlan tc_plan(int B, int T, int h_kv, int d, int64_t n_docs, int64_t n_chunks, 
   pl.cand_bytes = (((size_t)pl.grid * B * k * 8) + 255) & ~(size_t)255;
   const size_t stage = (((size_t)kTcBM * kTcBK * 2 + (size_t)pl.N * kTcBK * 2) + 1023) & ~(size_t)1023;
   const size_t fixed = (size_t)kTcBM * B * 4 + (kTcWin + 1) * 8 + (size_t)B * 32 * 8 +
-                       ((B + 1) & ~1) * 4 + (2 * kTcMaxStages + 5) * 8 + 7 * 8 + 16;
+                       ((B + 1) & ~1) * 4 + (2 * kTcMaxStages + 5) * 8 + 7 * 8 + 24;
   const size_t budget = 227 * 1024 - 1024 - fixed - 64;
   pl.stages = (int)std::min<size_t>(kTcMaxStages, budget / stage);
   if (pl.stages < 2) pl.ok = false;

@@ -4,9 +4,9 @@ A bounded device wait that runs out must record its error in the workspace statu
 with msa_workspace_status, MSA_ERR_DEVICE), leave no copy or tensor-core operation in flight,
 and let the next call on the same stream run normally. The failure is made by the caller, not by
 a fault: msa_set_device_wait_limit shortens the consumer-side waits of the tensor-core routing
-scan (its MMA issuer waiting for operand tiles, its epilogue waiting for accumulators) to a few
-dozen cycles, which no copy from memory meets; the waits for copies in flight keep the default
-limit. No test here faults, traps or hangs the GPU.
+scan (its epilogue warps waiting for the tensor cores' accumulators) to a few dozen cycles,
+which no tile loaded from memory and multiplied meets; the waits for copies and MMAs in flight
+keep the default limit. No test here faults, traps or hangs the GPU.
 """
 import numpy as np
 import pytest
