@@ -69,6 +69,10 @@ def parse():
                          "(zerocopy) or host-issued cudaMemcpyAsync per selected run (memcpy)")
     ap.add_argument("--scan", default="tc", choices=["tc", "cc"],
                     help="router scan: tensor cores over the normalised bank, or CUDA cores")
+    ap.add_argument("--cached", action="store_true",
+                    help="routed decode: keep each layer's local K/V as a rotated cache that the "
+                         "step appends the query token to (msa_decode_step) instead of passing it "
+                         "before RoPE to msa_sparse_attend every step")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels one by one instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -207,7 +211,8 @@ class Decode:
     ``engine.RoutedDecode`` (per layer route -> fetch/gather -> attend; see its docstring for
     the overlapped schedule)."""
 
-    def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc", nbuf: int = 2):
+    def __init__(self, w, dev, fetch: str, rank: int, scan: str = "tc", nbuf: int = 2,
+                 cached: bool = False):
         import torch
 
         import long_context_doc_b200 as msa
@@ -217,12 +222,19 @@ class Decode:
         fetch = fetch if w.layers > 1 else "device"
         self.L = w.layers
         self.scan = scan
+        self.cached = cached
         seed_w = w.scaled(seed=w.seed + 1000 * rank)
         B = w.B
-        # every layer's query inputs (Q_r, Q) in one contiguous buffer, so that a step's host
-        # copy of them is one transfer
+        # every layer's query inputs (Q_r, Q, and with caches the token's K/V) in one contiguous
+        # buffer, so that a step's host copy of them is one transfer
         nqr, nq = B * w.T * w.h_qr * w.d, B * w.T * w.h_q * w.d
-        self.qbuf = torch.empty(self.L * (nqr + nq), dtype=torch.bfloat16, device=dev)
+        nkv = B * w.T * w.h_kv * w.d if cached else 0
+        self.per_layer = nqr + nq + 2 * nkv
+        self.qbuf = torch.empty(self.L * self.per_layer, dtype=torch.bfloat16, device=dev)
+        # rotated local caches of L_loc rows: the first L_loc - 1 hold the prompt, the step
+        # appends the query token's own K/V; a step starts by resetting every length
+        self.lens = torch.zeros(self.L, dtype=torch.int32, device=dev)
+        self.lens0 = torch.full((self.L,), w.L_loc - w.T, dtype=torch.int32, device=dev)
         Kh = Vh = None
         coff_host = None
         layers = []
@@ -231,7 +243,7 @@ class Decode:
             coff_host = dv["doc_chunk_off"]
             if fetch != "device" and Kh is None:
                 Kh, Vh = self._host_bank(seed_w, coff_host, dev)
-            base = l * (nqr + nq)
+            base = l * self.per_layer
             Q_r = self.qbuf[base:base + nqr].view(dv["Q_r"].shape)
             Q = self.qbuf[base + nqr:base + nqr + nq].view(dv["Q"].shape)
             Q_r.copy_(dv["Q_r"])
@@ -239,11 +251,23 @@ class Decode:
             kv = (Kh, Vh) if fetch != "device" else (dv["Kbar"], dv["Vbar"])
             if scan == "tc":
                 # the tensor-core scan reads only the normalised bank: K̄_r is not kept
-                hat = msa.kr_normalize(dv.pop("Kbar_r"))
-                la = DecodeLayer(Q_r, Q, dv["K_loc"], dv["V_loc"], kv[0], kv[1], Kbar_r_hat=hat)
+                rkw = dict(Kbar_r_hat=msa.kr_normalize(dv.pop("Kbar_r")))
             else:
-                la = DecodeLayer(Q_r, Q, dv["K_loc"], dv["V_loc"], kv[0], kv[1],
-                                 Kbar_r=dv["Kbar_r"], kr_inv_norm=msa.kr_inv_norm(dv["Kbar_r"]))
+                rkw = dict(Kbar_r=dv["Kbar_r"], kr_inv_norm=msa.kr_inv_norm(dv["Kbar_r"]))
+            if cached:
+                T = w.T
+                c = msa.LocalCache(B, w.L_loc, w.h_kv, w.d, pos0=w.k, rope_base=w.rope_base,
+                                   device=dev, length=self.lens[l:l + 1])
+                c.append(dv["K_loc"][:, :-T].contiguous(), dv["V_loc"][:, :-T].contiguous())
+                o = base + nqr + nq
+                K_new = self.qbuf[o:o + nkv].view(B, T, w.h_kv, w.d)
+                V_new = self.qbuf[o + nkv:o + 2 * nkv].view(B, T, w.h_kv, w.d)
+                K_new.copy_(dv["K_loc"][:, -T:])
+                V_new.copy_(dv["V_loc"][:, -T:])
+                la = DecodeLayer(Q_r, Q, None, None, kv[0], kv[1], cache=c, K_new=K_new,
+                                 V_new=V_new, **rkw)
+            else:
+                la = DecodeLayer(Q_r, Q, dv["K_loc"], dv["V_loc"], kv[0], kv[1], **rkw)
             layers.append(la)
             del dv
         self.rd = RoutedDecode(layers, coff_host, w.k, w.rope_base, fetch=fetch, nbuf=nbuf)
@@ -285,6 +309,8 @@ class Decode:
         self.rd.route_events = ev
 
     def step(self):
+        if self.cached:  # every cache back to its prompt; the step appends the token
+            self.lens.copy_(self.lens0)
         self.rd.step()
 
     def ctx(self, l):
@@ -311,7 +337,7 @@ def run_libmsa(args):
     ranks = Ranks("nccl", dev)
     rank, world = ranks.rank, ranks.world
     w = synth.C4 if args.workload == "bank100m" else synth.C3
-    wk = Decode(w, dev, args.fetch, rank, args.scan)
+    wk = Decode(w, dev, args.fetch, rank, args.scan, cached=args.cached)
     torch.cuda.synchronize()
 
     def barrier():
@@ -369,9 +395,10 @@ def run_libmsa(args):
     # end to end: per-step query inputs copied from pinned host memory, outputs read back
     # per step: every layer's Q_r and Q (one copy), the new token's K/V row of every layer's
     # local cache, then every layer's output (one copy) and the last two layers' top-k ids
-    host_q = wk.qbuf.cpu().pin_memory()
-    host_kv = [[t.cpu().pin_memory() for t in (d.K_loc[:, -1:], d.V_loc[:, -1:])]
-               for d in wk.layers]
+    host_q = wk.qbuf.cpu().pin_memory()  # every layer's Q_r, Q (and the token's K/V if cached)
+    host_kv = ([] if wk.cached else
+               [[t.cpu().pin_memory() for t in (d.K_loc[:, -1:], d.V_loc[:, -1:])]
+                for d in wk.layers])
     host_O = wk.obuf.cpu().pin_memory()
     host_ids = wk.rd.ids.cpu().pin_memory()
     h2d = (host_q.numel() * host_q.element_size() +
@@ -381,7 +408,7 @@ def run_libmsa(args):
     def e2e_step():
         with torch.cuda.stream(wk.main):
             wk.qbuf.copy_(host_q, non_blocking=True)
-            for l in range(wk.L):
+            for l in range(len(host_kv)):
                 d = wk.layers[l]
                 kn, vn = host_kv[l]
                 d.K_loc[:, -1:].copy_(kn, non_blocking=True)
@@ -434,6 +461,11 @@ def run_libmsa(args):
                    "l2": "no flush: every layer scans a 3.28 GB K̄_r, far larger than the 126 MB L2"
                    if wk.L > 1 else "no flush: the 328 MB K̄_r scan exceeds the 126 MB L2",
                    "scan": wk.scan, "cuda_graph": use_graph,
+                   "local_kv_form": ("rotated cache: the step appends the query token's K/V "
+                                     "(RoPE at pos0 + 2047) to a 2047-row cache and attends "
+                                     "(msa_decode_step)") if wk.cached else
+                                    "K_loc before RoPE, all 2048 keys rotated per step "
+                                    "(msa_sparse_attend)",
                    "parallelism": f"replicas x{world}"},
         "router_scan_gbs": round(achieved, 1),
         "roofline": {"kernel": ("msa_route_topk (tensor-core scan: query fold + tcgen05 scan + "

@@ -623,11 +623,16 @@ cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_
     mkc = mkl;
     mvc = mvl;
   }
-  cudaError_t e = cudaFuncSetAttribute(attend_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)pl.smem);
-  if (e == cudaSuccess)
-    attend_dec_kernel<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
-  if (e == cudaSuccess) e = cudaGetLastError();
+  cudaError_t e;
+  if (p.keys_rotated || !p.rope) {  // keys used as stored: the 16-warp kernel
+    e = launch_attend_dec_plain(p, pl, mkc, mvc, mkl, mvl, st);
+  } else {
+    e = cudaFuncSetAttribute(attend_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)pl.smem);
+    if (e == cudaSuccess)
+      attend_dec_kernel<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
   if (e != cudaSuccess || pl.max_seg == 1) return e;
   // split queries: merge their partials (one CTA per output row; y carries the grid size)
   attend_dec_merge_kernel<<<(unsigned)(p.B * p.T * p.h_q), kMergeWarps * 32, 0, st>>>(p);

@@ -173,6 +173,12 @@ struct DecPlan {
 DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L, int sms);
 DecPlan attend_dec_plan_cap(int B, int T, int h_q, int h_kv, int d, int max_ctx, int cap, int sms);
 cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_t st);
+// attend_dec_plain.cu: the same attention when every key is used as stored (rotated cache or
+// no RoPE), 16 compute warps
+size_t attend_dec_plain_smem(int RB);
+cudaError_t launch_attend_dec_plain(const DecParams& p, const DecPlan& pl, const CUtensorMap& mkc,
+                                    const CUtensorMap& mvc, const CUtensorMap& mkl,
+                                    const CUtensorMap& mvl, cudaStream_t st);
 
 // ---- encode_hidden.cu: projections of hidden states fused with doc-wise RoPE + pooling
 struct EhParams {

@@ -27,9 +27,9 @@ from typing import Callable, List, Optional, Sequence
 import numpy as np
 import torch
 
-from . import (Fetcher, gather, msa_assemble_local, msa_gather, msa_route_topk,
-               msa_route_topk_workspace, msa_sparse_attend, msa_sparse_attend_workspace,
-               route_topk, sparse_attend)
+from . import (Fetcher, LocalCache, gather, msa_assemble_local, msa_decode_step,
+               msa_decode_step_workspace, msa_gather, msa_route_topk, msa_route_topk_workspace,
+               msa_sparse_attend, msa_sparse_attend_workspace, route_topk, sparse_attend)
 
 
 @dataclass
@@ -147,16 +147,25 @@ class DecodeLayer:
     Routing reads ``Kbar_r_hat`` (bf16 per-head unit rows, the tensor-core scan) when given,
     else ``Kbar_r`` with ``kr_inv_norm`` (the CUDA-core scan). ``Kbar``/``Vbar`` are either
     device tensors or pinned host tensors [n_chunks, h_kv, d]; several layers may share one
-    host bank."""
+    host bank.
+
+    The local context is either ``K_loc``/``V_loc`` (keys before RoPE, rotated by the attention
+    on every call) or a ``cache`` (a ``LocalCache`` whose keys are stored rotated at their global
+    positions pos0 + j, pos0 = k) into which the step first appends the query tokens' own
+    ``K_new``/``V_new`` (before RoPE) and then attends: the decode loop of a model, where every
+    key is rotated once, when it is appended."""
     Q_r: torch.Tensor                  # [B, T, h_qr, d]
     Q: torch.Tensor                    # [B, T, h_q, d]
-    K_loc: torch.Tensor                # [B, L_loc, h_kv, d] (before RoPE)
-    V_loc: torch.Tensor                # [B, L_loc, h_kv, d]
+    K_loc: Optional[torch.Tensor]      # [B, L_loc, h_kv, d] (before RoPE), or None with a cache
+    V_loc: Optional[torch.Tensor]      # [B, L_loc, h_kv, d]
     Kbar: torch.Tensor                 # [n_chunks, h_kv, d], device or pinned host memory
     Vbar: torch.Tensor
     Kbar_r_hat: Optional[torch.Tensor] = None
     Kbar_r: Optional[torch.Tensor] = None
     kr_inv_norm: Optional[torch.Tensor] = None
+    cache: Optional[LocalCache] = None  # rotated local cache (pos0 = k, the same RoPE base)
+    K_new: Optional[torch.Tensor] = None  # [B, T, h_kv, d] appended to the cache by the step
+    V_new: Optional[torch.Tensor] = None
 
 
 class RoutedDecode:
@@ -212,8 +221,15 @@ class RoutedDecode:
         la0 = layers[0]
         B, T, h_q, d = la0.Q.shape
         h_qr = la0.Q_r.shape[2]
-        h_kv = la0.K_loc.shape[2]
-        L_loc = la0.K_loc.shape[1]
+        self.cached = la0.cache is not None
+        if any((la.cache is not None) != self.cached for la in layers):
+            raise ValueError("either every layer has a local cache or none has")
+        for la in layers:
+            if la.cache is not None and (la.cache.pos0 != int(k) or la.K_new is None or
+                                         la.V_new is None):
+                raise ValueError("a cached layer needs pos0 = k and the step's K_new/V_new")
+        h_kv = (la0.cache.K if self.cached else la0.K_loc).shape[2]
+        L_loc = la0.cache.K.shape[1] if self.cached else la0.K_loc.shape[1]
         self.B, self.T, self.h_q, self.h_kv, self.d = B, T, h_q, h_kv, d
         cpd = int(np.max(np.diff(self.coff_host))) if self.n_docs else 0
         self.max_ctx = self.k * cpd
@@ -224,7 +240,8 @@ class RoutedDecode:
                                             self.n_chunks, self.k),
                    msa_route_topk_workspace(B, T, h_qr, h_kv, d, 0, self.n_docs, self.n_chunks,
                                             self.k))
-        ws_a = msa_sparse_attend_workspace(B, T, h_q, h_kv, d, self.max_ctx, L_loc)
+        ws_a = (msa_decode_step_workspace(B, T, h_q, h_kv, d, self.max_ctx, L_loc) if self.cached
+                else msa_sparse_attend_workspace(B, T, h_q, h_kv, d, self.max_ctx, L_loc))
         dt = la0.Q.dtype
         dev = self.dev
         self.ids = torch.empty((self.L, B, self.k), dtype=torch.int32, device=dev)
@@ -287,8 +304,15 @@ class RoutedDecode:
 
     def _attend(self, l: int):
         la, bf = self.layers[l], self.buf[l % self.nbuf]
-        msa_sparse_attend(la.Q, la.K_loc, la.V_loc, bf["cK"], bf["cV"], self.ctx_len[l], self.k,
-                          self.rope_base, self.scale, self.O[l], bf["ws_a"], self.stream)
+        if self.cached:  # append the step's tokens (rotated), then attend over the cache
+            c = la.cache
+            msa_decode_step(la.Q, la.K_new, la.V_new, c.K, c.V, c.length, bf["cK"], bf["cV"],
+                            self.ctx_len[l], self.k, self.rope_base, self.scale, self.O[l],
+                            bf["ws_a"], self.stream)
+        else:
+            msa_sparse_attend(la.Q, la.K_loc, la.V_loc, bf["cK"], bf["cV"], self.ctx_len[l],
+                              self.k, self.rope_base, self.scale, self.O[l], bf["ws_a"],
+                              self.stream)
 
     # ----------------------------------------------------------------- the step
     def step(self):
@@ -325,10 +349,11 @@ class RoutedDecode:
         """Launches of libmsa kernels per step (memsets and copies excluded): per layer the
         routing call (tensor-core scan: query fold + scan with fused top-k; CUDA-core scan: one
         kernel per pass of up to 16 query rows), the gather (none with fetch='memcpy': the
-        gather indices kernel only), the decode attention and the merge of its splits."""
+        gather indices kernel only), the decode attention and the merge of its splits, and with a
+        cache the append."""
         n = 0
         for la in self.layers:
             tc = la.Kbar_r_hat is not None and la.Q_r.dtype == torch.bfloat16
             route = 2 if tc else -(-self.B * self.T // 16)
-            n += route + 1 + 2
+            n += route + 1 + 2 + (1 if self.cached else 0)
         return n

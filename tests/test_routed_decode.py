@@ -34,10 +34,14 @@ def host_layers():
     return [synth.make_bank_workload(W, layer=l) for l in range(W.layers)]
 
 
-def _build(msa, gpu, host_layers, fetch, scan):
+def _build(msa, gpu, host_layers, fetch, scan, cached=False):
+    """With ``cached``, every layer's local context is a rotated cache holding the first
+    L_loc - 1 rows, and the step appends the last row (the query token's own K/V) before
+    attending: the same attention as the uncached step over K_loc/V_loc."""
     from long_context_doc_b200.engine import DecodeLayer, RoutedDecode
     layers = []
-    for inp in host_layers:
+    lens = torch.zeros(len(host_layers), dtype=torch.int32, device=gpu)
+    for l, inp in enumerate(host_layers):
         if fetch == "device":
             Kb, Vb = to_dev(inp["Kbar"], gpu), to_dev(inp["Vbar"], gpu)
         else:
@@ -45,10 +49,18 @@ def _build(msa, gpu, host_layers, fetch, scan):
         Krb = to_dev(inp["Kbar_r"], gpu)
         kw = (dict(Kbar_r_hat=msa.kr_normalize(Krb)) if scan == "tc" else
               dict(Kbar_r=Krb, kr_inv_norm=msa.kr_inv_norm(Krb)))
-        layers.append(DecodeLayer(to_dev(inp["Q_r"], gpu), to_dev(inp["Q"], gpu),
-                                  to_dev(inp["K_loc"], gpu), to_dev(inp["V_loc"], gpu), Kb, Vb,
+        Kl, Vl = to_dev(inp["K_loc"], gpu), to_dev(inp["V_loc"], gpu)
+        if cached:
+            c = msa.LocalCache(W.B, W.L_loc, W.h_kv, W.d, pos0=W.k, rope_base=W.rope_base,
+                               device=gpu, length=lens[l:l + 1])
+            c.append(Kl[:, :-1].contiguous(), Vl[:, :-1].contiguous())
+            kw.update(cache=c, K_new=Kl[:, -1:].contiguous(), V_new=Vl[:, -1:].contiguous())
+            Kl = Vl = None
+        layers.append(DecodeLayer(to_dev(inp["Q_r"], gpu), to_dev(inp["Q"], gpu), Kl, Vl, Kb, Vb,
                                   **kw))
-    return RoutedDecode(layers, host_layers[0]["doc_chunk_off"], W.k, W.rope_base, fetch=fetch)
+    rd = RoutedDecode(layers, host_layers[0]["doc_chunk_off"], W.k, W.rope_base, fetch=fetch)
+    rd.test_lens = lens  # the caches' lengths, reset to L_loc - 1 before every step
+    return rd
 
 
 def _check_against_oracle(rd, host_layers):
@@ -81,33 +93,45 @@ def _poison(rd):
         bf["cV"].fill_(float("nan"))
 
 
-@pytest.mark.parametrize("fetch,scan,graph", [
-    ("zerocopy", "tc", False),   # the benchmarked schedule, launched eagerly
-    ("zerocopy", "tc", True),    # ... and replayed from a CUDA graph (as the bench times it)
-    ("memcpy", "tc", False),     # host-issued cudaMemcpyAsync runs
-    ("device", "cc", True),      # device bank, CUDA-core scan, graph
-], ids=["zerocopy_eager", "zerocopy_graph", "memcpy_eager", "device_cc_graph"])
-def test_routed_decode_step_matches_oracle(msa, gpu, host_layers, fetch, scan, graph):
-    rd = _build(msa, gpu, host_layers, fetch, scan)
+@pytest.mark.parametrize("fetch,scan,graph,cached", [
+    ("zerocopy", "tc", False, False),  # the host-bank schedule, launched eagerly
+    ("zerocopy", "tc", True, False),   # ... and replayed from a CUDA graph
+    ("memcpy", "tc", False, False),    # host-issued cudaMemcpyAsync runs
+    ("device", "cc", True, False),     # device bank, CUDA-core scan, graph
+    ("zerocopy", "tc", True, True),    # rotated local caches, the benchmarked form
+    ("memcpy", "tc", False, True),
+], ids=["zerocopy_eager", "zerocopy_graph", "memcpy_eager", "device_cc_graph",
+        "zerocopy_graph_cached", "memcpy_eager_cached"])
+def test_routed_decode_step_matches_oracle(msa, gpu, host_layers, fetch, scan, graph, cached):
+    rd = _build(msa, gpu, host_layers, fetch, scan, cached)
     assert rd.nbuf == 2 and rd.L == 4
+    reset = lambda: rd.test_lens.fill_(W.L_loc - 1)  # noqa: E731
+    reset()
+    torch.cuda.synchronize()
     rd.step()
     torch.cuda.synchronize()
     if graph:
         rd.capture()
         _poison(rd)
         torch.cuda.synchronize()
-        rd.replay()
-        rd.replay()  # a second step on the same buffers (cross-step ordering)
+        for _ in range(2):  # a second step on the same buffers (cross-step ordering)
+            with torch.cuda.stream(rd.stream):
+                reset()
+            rd.replay()
     else:
         _poison(rd)
         torch.cuda.synchronize()
         with torch.cuda.stream(rd.stream):
-            rd.step()
-            rd.step()
+            for _ in range(2):
+                reset()
+                rd.step()
     torch.cuda.synchronize()
+    if cached:
+        assert rd.test_lens.cpu().tolist() == [W.L_loc] * rd.L
     for bf in rd.buf:
         assert msa.msa_workspace_status(bf["ws_r"]) == 0
         assert msa.msa_workspace_status(bf["ws_g"]) == 0
+        assert msa.msa_workspace_status(bf["ws_a"]) == 0
     _check_against_oracle(rd, host_layers)
 
 
