@@ -168,27 +168,6 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
   const int n_tiles = (int)(x1 - x0);
   const int b_first = (int)(x0 / TPP), tt_first = (int)(x0 % TPP);
 
-  if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      released[s] = 0u;
-    }
-    *abort_flag = 0;
-    *issued = 0;
-    // an error an earlier kernel of the same call recorded (a failed append) skips the call
-    skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
-    fence_mbar_init();
-  }
-  if (tid < HALF) turns[tid] = p.rope_turns[tid];
-  if (tid < 32)
-    ctx_first[tid] = b_first + tid < p.B ? min(max(__ldg(p.ctx_len + b_first + tid), 0), p.max_ctx) : 0;
-  __syncthreads();
-  if (skip_call) return;
-  auto ctx_rows = [&](int bb) {
-    return bb - b_first < 32 ? ctx_first[bb - b_first]
-                             : min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
-  };  // written once before the barrier: one value for the whole CTA
-
   // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
   // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d. Issued by one
   // thread: the first NS tiles here, each later one by the warp that releases the stage last.
@@ -198,7 +177,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     const bool ctx = tv < p.CT;
     const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
     // memory tiles past the query's context are not read (local tiles hold >= 1 row)
-    const bool any = !ctx || kt < ctx_rows(bb);
+    const bool any = !ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
     const int s = v % NS;
     const uint32_t st = smem_u32(stages + (size_t)s * kDecStage);
     fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
@@ -214,8 +193,31 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     }
     *issued = v + 1;
   };
-  if (tid == 0)
-    for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      released[s] = 0u;
+    }
+    *abort_flag = 0;
+    *issued = 0;
+    // an error an earlier kernel of the same call recorded (a failed append) skips the call
+    skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+    fence_mbar_init();
+    // the first copies go out before the tables are built, so the prologue overlaps them
+    // (none when the call is skipped: a CTA never exits with a copy in flight)
+    if (!skip_call)
+      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
+  }
+  if (tid < HALF) turns[tid] = p.rope_turns[tid];
+  if (tid < 32)
+    ctx_first[tid] = b_first + tid < p.B ? min(max(__ldg(p.ctx_len + b_first + tid), 0), p.max_ctx) : 0;
+  __syncthreads();
+  if (skip_call) return;
+  auto ctx_rows = [&](int bb) {
+    return bb - b_first < 32 ? ctx_first[bb - b_first]
+                             : min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
+  };  // written once before the barrier: one value for the whole CTA
+
 
   // ---------------- compute warps
   const int g = warp % HKV;    // KV head of this warp

@@ -141,6 +141,30 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
   const int n_tiles = (int)(x1 - x0);
   const int b_first = (int)(x0 / TPP);
 
+  // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
+  // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d.
+  auto issue = [&](int v) {
+    const int64_t x = x0 + v;
+    const int bb = (int)(x / TPP), tv = (int)(x % TPP);
+    const bool ctx = tv < p.CT;
+    const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
+    // memory tiles past the query's context are not read (local tiles hold >= 1 row)
+    const bool any = !ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
+    const int s = v % NS;
+    const uint32_t st = smem_u32(stages + (size_t)s * kStage);
+    fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
+    mbar_arrive_expect_tx(&full[s], any ? kStage : 0u);
+    if (any) {
+      const CUtensorMap* mk = ctx ? &map_kc : &map_kl;
+      const CUtensorMap* mv = ctx ? &map_vc : &map_vl;
+      const int y = ctx ? bb * p.max_ctx + kt : bb * p.Ls + kt;
+      tma3d(st, mk, 0, y, &full[s]);
+      tma3d(st + kHalf / 2, mk, HALF, y, &full[s]);
+      tma3d(st + kHalf, mv, 0, y, &full[s]);
+      tma3d(st + kHalf + kHalf / 2, mv, HALF, y, &full[s]);
+    }
+    atomicAdd(&issued[s], 1u);
+  };
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
@@ -150,6 +174,10 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
     *abort_flag = 0;
     skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
     fence_mbar_init();
+    // the first copies go out before the tables are built, so the prologue overlaps them
+    // (none when the call is skipped: a CTA never exits with a copy in flight)
+    if (!skip_call)
+      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
   }
   if (tid < 32)
     ctx_first[tid] =
@@ -169,31 +197,6 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
                              : min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
   };
 
-  // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
-  // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d.
-  auto issue = [&](int v) {
-    const int64_t x = x0 + v;
-    const int bb = (int)(x / TPP), tv = (int)(x % TPP);
-    const bool ctx = tv < p.CT;
-    const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
-    const bool any = !ctx || kt < ctx_rows(bb);  // memory tiles past the context: not read
-    const int s = v % NS;
-    const uint32_t st = smem_u32(stages + (size_t)s * kStage);
-    fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
-    mbar_arrive_expect_tx(&full[s], any ? kStage : 0u);
-    if (any) {
-      const CUtensorMap* mk = ctx ? &map_kc : &map_kl;
-      const CUtensorMap* mv = ctx ? &map_vc : &map_vl;
-      const int y = ctx ? bb * p.max_ctx + kt : bb * p.Ls + kt;
-      tma3d(st, mk, 0, y, &full[s]);
-      tma3d(st + kHalf / 2, mk, HALF, y, &full[s]);
-      tma3d(st + kHalf, mv, 0, y, &full[s]);
-      tma3d(st + kHalf + kHalf / 2, mv, HALF, y, &full[s]);
-    }
-    atomicAdd(&issued[s], 1u);
-  };
-  if (tid == 0)
-    for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
 
   // ---------------- compute warps
   const int g = lw % HKV;      // KV head of this warp
