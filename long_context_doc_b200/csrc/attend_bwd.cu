@@ -236,8 +236,7 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                   const __grid_constant__ CUtensorMap map_vc, const __grid_constant__ CUtensorMap map_vl,
                   MainArgs p) {
   extern __shared__ __align__(1024) unsigned char sm_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* base = smem_align1024(sm_raw);
   unsigned char* k_s = base;                          // [2 slices][128 keys][64 dims]
   unsigned char* v_s = base + 2 * kKSlice;            // [2 slices][128 keys][64 dims]
   unsigned char* stg = base + 4 * kKSlice;            // [2 stages][Q 2 slices | dO 2 | lse | D]

@@ -127,8 +127,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
                   DecParams p) {
   constexpr int D = kDecD, HALF = D / 2, NS = kDecStages;
   extern __shared__ __align__(1024) unsigned char sm_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sm = smem_align1024(sm_raw);
   unsigned char* stages = sm;                                                 // [NS][K|V]
   float4* rstep = reinterpret_cast<float4*>(sm + NS * kDecStage);             // [KT][32]
   float4* kturn = rstep + 64 * 32;                                            // [32]
@@ -283,6 +282,31 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     float l = lsum;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (WPH == 1) {  // one warp per KV head: nothing to combine, rows written from registers
+      const bool write = !named_sync_compute_or(*abort_flag != 0);  // one decision for all warps
+      if (!write || gr >= nr) return;
+      const int64_t first = dec_cta_of((int64_t)fb * TPP, G, total);
+      const int64_t last = dec_cta_of((int64_t)fb * TPP + TPP - 1, G, total);
+      const int t = gr / Gq, h = g * Gq + gr % Gq;
+      if (first == last) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* out = p.O + (((int64_t)fb * p.T + t) * p.h_q + h) * D + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+          *reinterpret_cast<uint32_t*>(out + 8 * nt) =
+              bf2_pack(make_float2(o[nt].x * inv, o[nt].y * inv));
+      } else {
+        const int64_t slot = (((int64_t)fb * p.max_seg + (ci - first)) * HKV + g) * RB + gr;
+        float* out = p.part_o + slot * D + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) *reinterpret_cast<float2*>(out + 8 * nt) = o[nt];
+        if (t4 == 0) {
+          p.part_ml[slot * 2] = mrow;
+          p.part_ml[slot * 2 + 1] = l;
+        }
+      }
+      return;
+    }
     if (gr < RB) {
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt)

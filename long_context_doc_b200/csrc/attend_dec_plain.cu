@@ -107,8 +107,7 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
                         const __grid_constant__ CUtensorMap map_vl, DecParams p) {
   constexpr int D = kD, HALF = D / 2, NS = kStages;
   extern __shared__ __align__(1024) unsigned char sm_raw[];
-  unsigned char* sm = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* sm = smem_align1024(sm_raw);
   unsigned char* stages = sm;                                              // [NS][K | V]
   float4* qrot = reinterpret_cast<float4*>(sm + NS * kStage);              // [T][32]
   const int RB = (p.h_q / p.h_kv) * p.T <= 4 ? 4 : 8;  // combine-buffer rows per KV head

@@ -212,8 +212,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                  const __grid_constant__ CUtensorMap map_kl, const __grid_constant__ CUtensorMap map_vc,
                  const __grid_constant__ CUtensorMap map_vl, AtcParams p) {
   extern __shared__ __align__(1024) unsigned char sm_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* base = smem_align1024(sm_raw);
   unsigned char* q_s = base;                                  // [2][128][64]
   unsigned char* stages = base + kQBytes;                     // [S][K 2 slices | V^T 2 slices]
   unsigned char* p_s = stages + kStages * kStage;             // [2][128][64] probabilities

@@ -77,6 +77,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory array advanced to the next 1024-byte boundary of the shared window
+// (the 128-byte swizzle atoms of TMA boxes and tensor-core operands). The pad is added to the
+// array itself, so every pointer derived from the result stays in the shared state space and
+// compiles to shared loads and stores with 32-bit addresses (a detour through an integer
+// address makes them generic 64-bit accesses).
+__device__ __forceinline__ unsigned char* smem_align1024(unsigned char* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");

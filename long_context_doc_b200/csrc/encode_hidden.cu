@@ -135,8 +135,7 @@ encode_hidden_kernel(const __grid_constant__ CUtensorMap map_h,
                      const __grid_constant__ CUtensorMap map_wv,
                      const __grid_constant__ CUtensorMap map_wr, EhParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* base = smem_align1024(smem_raw);
   float* pool = reinterpret_cast<float*>(base + kStages * kStage);   // [2 chunks][256]
   uint64_t* full = reinterpret_cast<uint64_t*>(pool + 2 * kBN);      // [kStages]
   uint64_t* empty = full + kStages;                                  // [kStages]

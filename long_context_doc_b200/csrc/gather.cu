@@ -3,11 +3,12 @@
 // chunks in order [news.neo-ai.one article, "推論パイプライン": the selected K̄/V̄ are loaded
 // and concatenated with the local context].
 //
-// One CTA per (selected slot j, query b). The CTA ranks its doc among the query's valid ids
-// (a k x k comparison, k <= 32), which gives its row offset in the context, writes the gather
-// indices of its chunks and copies its chunks' rows with 16-byte vector loads/stores (the
-// source may be HBM or pinned host memory mapped into the device address space). Slot 0
-// also writes ctx_len and pads gather_idx with -1.
+// One CTA per (selected slot j, query b). Its first warp ranks the doc among the query's valid
+// ids (lane q holds id q, k <= 32; sums by shuffles), which gives its row offset in the context;
+// the CTA writes the gather indices of its chunks and copies its chunks' rows with 16-byte
+// vector loads/stores, four of each tensor in flight per thread (the source may be HBM or
+// pinned host memory mapped into the device address space). Slot 0 also writes ctx_len and pads
+// gather_idx with -1.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -18,23 +19,32 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
   const int j = blockIdx.x, b = blockIdx.y;
   const int32_t* ids = p.ids + (int64_t)b * p.k;
   __shared__ int64_t s_off, s_n, s_src, s_total;
-  if (threadIdx.x == 0) {
-    const int32_t me = ids[j];
+  if (threadIdx.x < 32) {
+    const int q = threadIdx.x;
+    const int32_t o = q < p.k ? ids[q] : -1;
+    const bool ok = o >= 0 && o < p.n_docs;
+    const int64_t c0 = ok ? p.coff[o] : 0;
+    const int64_t n = ok ? p.coff[o + 1] - c0 : 0;
+    const int32_t me = __shfl_sync(0xffffffffu, o, j);
     const bool ok_me = me >= 0 && me < p.n_docs;
-    if (me >= p.n_docs) set_err(p.err, kErrBadIndex);
-    int64_t off = 0, total = 0;
-    for (int q = 0; q < p.k; ++q) {
-      const int32_t o = ids[q];
-      if (o < 0 || o >= p.n_docs) continue;
-      const int64_t n = p.coff[o + 1] - p.coff[o];
-      total += n;
-      if (ok_me && (o < me || (o == me && q < j))) off += n;
+    // rows of the valid docs before this one: smaller id, or the same id at an earlier slot
+    int64_t before = ok && ok_me && (o < me || (o == me && q < j)) ? n : 0;
+    int64_t total = n;
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, s);
+      total += __shfl_xor_sync(0xffffffffu, total, s);
     }
-    s_off = off;
-    s_n = ok_me ? p.coff[me + 1] - p.coff[me] : 0;
-    s_src = ok_me ? p.coff[me] : 0;
-    s_total = total;
-    if (total > p.max_ctx && j == 0) set_err(p.err, kErrCtxOverflow);
+    const int64_t n_me = __shfl_sync(0xffffffffu, n, j);
+    const int64_t src_me = __shfl_sync(0xffffffffu, c0, j);
+    if (q == 0) {
+      if (me >= p.n_docs) set_err(p.err, kErrBadIndex);
+      s_off = before;
+      s_n = ok_me ? n_me : 0;
+      s_src = ok_me ? src_me : 0;
+      s_total = total;
+      if (total > p.max_ctx && j == 0) set_err(p.err, kErrCtxOverflow);
+    }
   }
   __syncthreads();
   const int64_t off = s_off, src = s_src, total = s_total;
@@ -56,11 +66,22 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
   const uint4* sv = static_cast<const uint4*>(p.Vb) + src0;
   uint4* dk = static_cast<uint4*>(p.ctxK) + dst0;
   uint4* dv = static_cast<uint4*>(p.ctxV) + dst0;
-  for (int64_t x = threadIdx.x; x < vecs; x += blockDim.x) {
-    const uint4 a = sk[x];
-    const uint4 c = sv[x];
-    dk[x] = a;
-    dv[x] = c;
+  constexpr int U = 4;  // vectors of each tensor in flight per thread
+  const int64_t nt = blockDim.x;
+  for (int64_t x0 = threadIdx.x; x0 < vecs; x0 += U * nt) {
+    uint4 a[U], c[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (x0 + u * nt < vecs) {
+        a[u] = sk[x0 + u * nt];
+        c[u] = sv[x0 + u * nt];
+      }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (x0 + u * nt < vecs) {
+        dk[x0 + u * nt] = a[u];
+        dv[x0 + u * nt] = c[u];
+      }
   }
 }
 
