@@ -223,49 +223,60 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
     float l = lsum;
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if (gr < RB) {
+    // the warps of head g other than its leader (warp g) leave (m, l, o) of their rows in shared
+    // memory, o in fragment order ([warp][nt][lane], conflict-free); the leader folds them into
+    // its registers and writes the rows
+    const bool leader = warp == g;
+    if (!leader && gr < RB) {
+      float2* cw = reinterpret_cast<float2*>(comb) + warp * 16 * (RB * 4);
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
-        *reinterpret_cast<float2*>(comb + (warp * RB + gr) * D + 8 * nt + 2 * t4) = o[nt];
+      for (int nt = 0; nt < 16; ++nt) cw[nt * (RB * 4) + lane] = o[nt];
       if (t4 == 0) {
         wscr[warp * kWS + 9 * RB + gr] = mrow;
         wscr[warp * kWS + 10 * RB + gr] = l;
       }
     }
     const bool write = !sync_compute_or(*abort_flag != 0);  // one decision for all warps
-    const int64_t first = cta_of((int64_t)fb * TPP, G, total);
-    const int64_t last = cta_of((int64_t)fb * TPP + TPP - 1, G, total);
-    const int n_seg = (int)(last - first + 1);
-    const int seg = (int)(ci - first);
-    const int e = tid & (D - 1);  // output dim of this thread; rows r = tid / D, + 4, ...
-    for (int gh = 0; gh < HKV; ++gh)
-      for (int r = tid / D; r < nr; r += kThreads / D) {
-        float M = -INFINITY;
-        for (int k2 = 0; k2 < WPH; ++k2) M = fmaxf(M, wscr[(gh + k2 * HKV) * kWS + 9 * RB + r]);
-        float ov = 0.f, lv = 0.f;
-        if (M != -INFINITY)
-          for (int k2 = 0; k2 < WPH; ++k2) {
-            const int w = gh + k2 * HKV;
-            const float m = wscr[w * kWS + 9 * RB + r];
-            const float a = m == -INFINITY ? 0.f : exp2f(m - M);
-            ov = fmaf(comb[(w * RB + r) * D + e], a, ov);
-            lv = fmaf(wscr[w * kWS + 10 * RB + r], a, lv);
-          }
-        if (!write) continue;
-        const int t = r / Gq, h = gh * Gq + r % Gq;
-        if (n_seg == 1) {
-          p.O[(((int64_t)fb * p.T + t) * p.h_q + h) * D + e] =
-              __float2bfloat16_rn(lv > 0.f ? ov / lv : 0.f);
-        } else {
-          const int64_t slot = (((int64_t)fb * p.max_seg + seg) * HKV + gh) * RB + r;
-          p.part_o[slot * D + e] = ov;
-          if (e == 0) {
-            p.part_ml[slot * 2] = M;
-            p.part_ml[slot * 2 + 1] = lv;
-          }
+    if (leader && write && gr < nr) {
+      float M = mrow;
+      for (int k2 = 1; k2 < WPH; ++k2) M = fmaxf(M, wscr[(g + k2 * HKV) * kWS + 9 * RB + gr]);
+      const float a0 = mrow == -INFINITY ? 0.f : exp2f(mrow - M);
+      float2* ov = o;  // the segment's accumulators are folded in place
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) ov[nt] = __fmul2_rn(o[nt], make_float2(a0, a0));
+      float lv = l * a0;
+      for (int k2 = 1; k2 < WPH; ++k2) {
+        const int w = g + k2 * HKV;
+        const float m = wscr[w * kWS + 9 * RB + gr];
+        const float a = m == -INFINITY ? 0.f : exp2f(m - M);
+        const float2* cw = reinterpret_cast<const float2*>(comb) + w * 16 * (RB * 4);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+          ov[nt] = __ffma2_rn(cw[nt * (RB * 4) + lane], make_float2(a, a), ov[nt]);
+        lv = fmaf(wscr[w * kWS + 10 * RB + gr], a, lv);
+      }
+      const int64_t first = cta_of((int64_t)fb * TPP, G, total);
+      const int64_t last = cta_of((int64_t)fb * TPP + TPP - 1, G, total);
+      const int t = gr / Gq, h = g * Gq + gr % Gq;
+      if (first == last) {  // the whole query in this CTA: O itself
+        const float inv = lv > 0.f ? 1.f / lv : 0.f;
+        __nv_bfloat16* out = p.O + (((int64_t)fb * p.T + t) * p.h_q + h) * D + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt)
+          *reinterpret_cast<uint32_t*>(out + 8 * nt) =
+              bf2_pack(make_float2(ov[nt].x * inv, ov[nt].y * inv));
+      } else {  // this CTA's partial of a split query
+        const int64_t slot = (((int64_t)fb * p.max_seg + (ci - first)) * HKV + g) * RB + gr;
+        float* out = p.part_o + slot * D + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) *reinterpret_cast<float2*>(out + 8 * nt) = ov[nt];
+        if (t4 == 0) {
+          p.part_ml[slot * 2] = M;
+          p.part_ml[slot * 2 + 1] = lv;
         }
       }
-    sync_compute();  // comb and the warps' scratch are reused by the next segment
+    }
+    if (WPH > 1) sync_compute();  // the shared fragments are refilled by the next segment
   };
 
   int64_t x = x0;
