@@ -407,7 +407,11 @@ msa_status msa_kv_append(void* K_cache, void* V_cache, int32_t B, int32_t cap, i
  * as in msa_sparse_attend.
  * Supported: bf16, d = 128, h_kv in {1, 2, 4, 8}, (h_q / h_kv) * T <= 8 (else
  * MSA_ERR_UNSUPPORTED). ws: msa_decode_step_workspace(...) bytes, 256-byte aligned; its
- * status word records a cache overflow (then O is not written) or an expired device wait. */
+ * status word records a cache overflow (then O is not written and len stays) or an expired
+ * device wait. The step is two launches: the attention kernel, which appends the new rows
+ * itself (each in the one tile that holds it, and into the cache) and starts the status word,
+ * then the merge of split queries, which advances len; ws must not be shared with a call
+ * running concurrently. */
 size_t msa_decode_step_workspace(int32_t B, int32_t T, int32_t h_q, int32_t h_kv, int32_t d,
                                  int32_t max_ctx, int32_t cap);
 msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, int32_t B,

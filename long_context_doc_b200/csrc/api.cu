@@ -903,27 +903,9 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
           MSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   unsigned char* w8 = static_cast<unsigned char*>(ws);
   cudaStream_t st = (cudaStream_t)stream;
-  // the append runs as one CTA and starts the status word (no memset node per step)
+  // the append is fused into the attention launch: its first CTA starts the status word, the
+  // merge kernel advances the length (no memset node, no append kernel per step)
   cudaError_t e = cudaSuccess;
-  msa::AppendParams a{};
-  a.B = B;
-  a.T_new = T;
-  a.cap = cap;
-  a.row_bytes = (int64_t)h_kv * d * 2;
-  a.K_cache = K_cache;
-  a.V_cache = V_cache;
-  a.K_new = K_new;
-  a.V_new = V_new;
-  a.len = len_dev;
-  a.err = reinterpret_cast<int*>(w8);
-  a.ticket = reinterpret_cast<unsigned int*>(w8 + 4);
-  a.single = 1;
-  a.rope = rope_base > 0.f ? 1 : 0;  // the cache holds keys rotated at pos0 + row
-  a.pos0 = pos0;
-  a.d = d;
-  a.esize = 2;
-  msa::rope_turns(a.rope ? (double)rope_base : 0.0, d, a.rope_turns);
-  if (e == cudaSuccess) e = msa::launch_kv_append(a, sm_count(), st);
   msa::DecParams q{};
   q.Q = static_cast<const __nv_bfloat16*>(Q);
   q.Kl = static_cast<const __nv_bfloat16*>(K_cache);
@@ -939,7 +921,10 @@ msa_status msa_decode_step(const void* Q, const void* K_new, const void* V_new, 
   q.Ls = cap;
   q.L_dev = len_dev;
   q.skip_on_err = 1;   // an overflowing append leaves O unwritten
-  q.keys_rotated = 1;  // the append stored the keys rotated
+  q.keys_rotated = 1;  // the cache holds keys rotated at pos0 + row
+  q.K_new = static_cast<const __nv_bfloat16*>(K_new);
+  q.V_new = static_cast<const __nv_bfloat16*>(V_new);
+  q.L_out = reinterpret_cast<int*>(w8 + 8);
   q.max_ctx = max_ctx;
   q.rope = rope_base > 0.f ? 1 : 0;
   q.pos0 = pos0;

@@ -513,7 +513,15 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecP
   const int h = row % p.h_q, t = (row / p.h_q) % p.T, b = row / (p.h_q * p.T);
   const int gh = h / Gq, r = t * Gq + h % Gq;
   const int RB = (Gq * p.T) <= 4 ? 4 : 8;
-  const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
+  int L;
+  if (p.K_new != nullptr) {  // fused append: the length the attention kernel used
+    L = *reinterpret_cast<volatile int*>(p.L_out);
+    if (L < 0) return;  // overflow: the cache length stays
+    // the cache length advances here, after every attention CTA has read it
+    if (blockIdx.x == 0 && threadIdx.x == 0) *const_cast<int32_t*>(p.L_dev) = L;
+  } else {
+    L = p.L_dev != nullptr ? *p.L_dev : p.L;
+  }
   if (L < p.T || L > p.Ls) return;  // reported by the attention kernel
   if (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) return;
   const int KT = kDecRowsPerTile / HKV;
@@ -645,7 +653,8 @@ cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_
       attend_dec_kernel<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
-  if (e != cudaSuccess || pl.max_seg == 1) return e;
+  // (a fused append needs the merge kernel for the length update even with no split query)
+  if (e != cudaSuccess || (pl.max_seg == 1 && p.K_new == nullptr)) return e;
   // split queries: merge their partials (one CTA per output row; y carries the grid size)
   attend_dec_merge_kernel<<<(unsigned)(p.B * p.T * p.h_q), kMergeWarps * 32, 0, st>>>(p);
   return cudaGetLastError();

@@ -127,9 +127,21 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
   const int KT = kRowsPerTile / HKV;  // key rows per tile
   const int Gq = p.h_q / HKV;
   const int nr = Gq * p.T;            // query rows per KV head (<= 8)
-  const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
-  if (L < p.T || L > p.Ls) {  // uniform over the grid: nothing is read or written
-    if (blockIdx.x == 0 && tid == 0) set_err(p.err, kErrBadIndex);
+  // local rows per query: fixed, read from the device, or (fused append) the device length
+  // plus the T tokens this call appends
+  const bool fused = p.K_new != nullptr;
+  const int L = fused ? *reinterpret_cast<const volatile int32_t*>(p.L_dev) + p.T
+                      : (p.L_dev != nullptr ? *p.L_dev : p.L);
+  const bool bad = L < p.T || L > p.Ls;  // uniform over the grid: nothing is read or written
+  if (fused && blockIdx.x == 0 && tid == 0) {
+    // the first CTA starts the call's status word (another CTA records an error only after a
+    // bounded wait has run out, long after every CTA started) and hands the new length to the
+    // merge kernel
+    *p.err = bad ? kErrCtxOverflow : 0;
+    *p.L_out = bad ? -1 : L;
+  }
+  if (bad) {
+    if (!fused && blockIdx.x == 0 && tid == 0) set_err(p.err, kErrBadIndex);
     return;
   }
   const int TPP = p.CT + (L + KT - 1) / KT;  // tiles per query
@@ -171,7 +183,7 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
       issued[s] = 0u;
     }
     *abort_flag = 0;
-    skip_call = (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
+    skip_call = (!fused && p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) ? 1 : 0;
     fence_mbar_init();
     // the first copies go out before the tables are built, so the prologue overlaps them
     // (none when the call is skipped: a CTA never exits with a copy in flight)
@@ -212,6 +224,37 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
     return (uint32_t)((m >> 1) * (kHalf / 2)) + lbase + ((m & 1) ? lx1 : lx0);
   };
   const int WPH = kCW / HKV;  // warps per KV head
+  // Fused append of new local row j (token t = j - (L - T)) of query bb, KV head g, line
+  // g * KT + r of the tile: K rotated at its position pos0 + j (the query's table entry t; the
+  // formula of kv_append), V as given; written into the tile in shared memory (128-byte
+  // swizzle: 16-byte chunk c of a line at c ^ (line & 7)) and into the cache. Lane l: RoPE
+  // pairs 2l, 2l+1 (dims 2l, 2l+1 and their partners + 64) of K, dims 4l..4l+3 of V.
+  auto append_row = [&](int bb, int j, int r, uint32_t kb, uint32_t vb) {
+    const int t = j - (L - p.T);
+    const int line = g * KT + r;
+    const int64_t src = (((int64_t)bb * p.T + t) * HKV + g) * D;
+    const int64_t dst = (((int64_t)bb * p.Ls + j) * HKV + g) * D;
+    const float2 x = bf2_unpack(__ldg(reinterpret_cast<const unsigned int*>(p.K_new + src) + lane));
+    const float2 y =
+        bf2_unpack(__ldg(reinterpret_cast<const unsigned int*>(p.K_new + src + HALF) + lane));
+    const float4 cs = qrot[t * 32 + lane];  // (cos, cos, sin, sin) of pairs 2l, 2l+1
+    const uint32_t xr = bf2_pack(make_float2(x.x * cs.x - y.x * cs.z, x.y * cs.y - y.y * cs.w));
+    const uint32_t yr = bf2_pack(make_float2(y.x * cs.x + x.x * cs.z, y.y * cs.y + x.y * cs.w));
+    const uint32_t ko = (uint32_t)(line * 128 + ((((lane >> 2) ^ (line & 7))) << 4) + (lane & 3) * 4);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(kb + ko), "r"(xr) : "memory");
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(kb + kHalf / 2 + ko), "r"(yr) : "memory");
+    unsigned int* kc = reinterpret_cast<unsigned int*>(const_cast<__nv_bfloat16*>(p.Kl) + dst);
+    kc[lane] = xr;
+    kc[HALF / 2 + lane] = yr;
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.V_new + src) + lane);
+    const int hv = lane >> 4, cv = (lane & 15) >> 1;  // half of d, 16-byte chunk in the half
+    const uint32_t vo = (uint32_t)(hv * (kHalf / 2) + line * 128 + ((cv ^ (line & 7)) << 4) +
+                                   (lane & 1) * 8);
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(vb + vo), "r"(v.x), "r"(v.y)
+                 : "memory");
+    reinterpret_cast<uint2*>(const_cast<__nv_bfloat16*>(p.Vl) + dst)[lane] = v;
+    __syncwarp();  // the row is in the tile before the warp's fragment loads
+  };
 
   uint32_t qa[4][4];  // the query rows of head g in fragment order, rotated, scaled, bf16
   float2 o[16];       // P.V accumulators of row gr: dims 8 nt + 2 t4, +1
@@ -321,6 +364,11 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
       if (!*abort_flag && !mbar_wait_bounded(&full[s], (uint32_t)((u / NS) & 1), p.err))
         *abort_flag = 1;
       const uint32_t kb = smem_u32(stages + (size_t)s * kStage), vb = kb + kHalf;
+      if (fused && !is_ctx) {  // this warp's rows of the tile that the call appends
+        const int r0 = kt + 8 * sl;
+        const int j1 = min(r0 + 8, L);
+        for (int j = max(r0, L - p.T); j < j1; ++j) append_row(b, j, j - kt, kb, vb);
+      }
 
       // ---- logits S[row gr][keys 8 sl + 2 t4, +1]: 8 MMAs over d in four chains
       uint32_t kr[4][4];

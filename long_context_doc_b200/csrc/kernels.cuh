@@ -163,6 +163,14 @@ struct DecParams {
   float* part_ml;           // [B, max_seg, h_kv, RB, 2]
   int* err;                 // workspace status word
   __nv_bfloat16* O;         // [B, T, h_q, 128]
+  // decode step with the append fused in (16-warp kernel, L_dev set, keys_rotated): the T new
+  // tokens' K/V [B, T, h_kv, 128] become local rows L_dev..L_dev+T-1, K rotated at pos0 + row;
+  // the attention kernel writes them into Kl/Vl (and into the tiles it attends), starts the
+  // status word and leaves the new length (-1 on overflow) in L_out; the merge kernel then
+  // stores that length into L_dev
+  const __nv_bfloat16* K_new;  // nullable: no fused append
+  const __nv_bfloat16* V_new;
+  int* L_out;
 };
 struct DecPlan {
   bool ok;
