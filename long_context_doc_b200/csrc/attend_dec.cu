@@ -504,7 +504,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
 
 // Merge of the partials of the queries split over several CTAs: CTA = one output row (query b,
 // query head h, token t); warp w folds segments w, w + 8, ... with lane l on dims 4l .. 4l+3,
-// then the eight warps combine in shared memory.
+// each with its own running maximum, then the eight warps combine in shared memory.
 constexpr int kMergeWarps = 8;
 __global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -513,17 +513,17 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecP
   const int h = row % p.h_q, t = (row / p.h_q) % p.T, b = row / (p.h_q * p.T);
   const int gh = h / Gq, r = t * Gq + h % Gq;
   const int RB = (Gq * p.T) <= 4 ? 4 : 8;
-  int L;
-  if (p.K_new != nullptr) {  // fused append: the length the attention kernel used
-    L = *reinterpret_cast<volatile int*>(p.L_out);
+  // the length and the status word, loaded together
+  const int L = p.K_new != nullptr ? __ldcg(p.L_out)  // fused append: the length it used
+                                   : (p.L_dev != nullptr ? __ldcg(p.L_dev) : p.L);
+  const int err = p.skip_on_err ? __ldcg(p.err) : 0;
+  if (p.K_new != nullptr) {
     if (L < 0) return;  // overflow: the cache length stays
     // the cache length advances here, after every attention CTA has read it
     if (blockIdx.x == 0 && threadIdx.x == 0) *const_cast<int32_t*>(p.L_dev) = L;
-  } else {
-    L = p.L_dev != nullptr ? *p.L_dev : p.L;
   }
   if (L < p.T || L > p.Ls) return;  // reported by the attention kernel
-  if (p.skip_on_err && *reinterpret_cast<volatile int*>(p.err) != 0) return;
+  if (err != 0) return;
   const int KT = kDecRowsPerTile / HKV;
   const int TPP = p.CT + (L + KT - 1) / KT;
   const int64_t total = (int64_t)p.B * TPP, G = min((int64_t)p.grid, total);
@@ -531,42 +531,68 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attend_dec_merge_kernel(DecP
   const int64_t last = dec_cta_of((int64_t)b * TPP + TPP - 1, G, total);
   const int n_seg = (int)(last - first + 1);
   if (n_seg == 1) return;  // written directly by the attention kernel
-  __shared__ float sm_l[kMergeWarps];
+  __shared__ float sm_m[kMergeWarps], sm_l[kMergeWarps];
   __shared__ float4 sm_o[kMergeWarps][32];
   auto slot_of = [&](int sg) { return (((int64_t)b * p.max_seg + sg) * HKV + gh) * RB + r; };
-  // the row's maximum over all segments
-  float M = -INFINITY;
-  for (int sg = lane; sg < n_seg; sg += 32) M = fmaxf(M, __ldcg(p.part_ml + slot_of(sg) * 2));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float l = 0.f;
+  // warp w folds segments w, w + 8, ... four at a time (their loads in flight together) with
+  // its own running maximum; the eight warps are then combined in shared memory
+  float M = -INFINITY, l = 0.f;
   float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (M != -INFINITY) {
-#pragma unroll 2
-    for (int sg = warp; sg < n_seg; sg += kMergeWarps) {
-      const int64_t sl = slot_of(sg);
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + sl * 2));
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.part_o + sl * kDecD) + lane);
-      const float a = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-      l = fmaf(ml.y, a, l);
-      o4.x = fmaf(x.x, a, o4.x);
-      o4.y = fmaf(x.y, a, o4.y);
-      o4.z = fmaf(x.z, a, o4.z);
-      o4.w = fmaf(x.w, a, o4.w);
+  for (int sg0 = warp; sg0 < n_seg; sg0 += 4 * kMergeWarps) {
+    float2 ml[4];
+    float4 x[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int sg = sg0 + i * kMergeWarps;
+      ml[i] = make_float2(-INFINITY, 0.f);
+      x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (sg < n_seg) {
+        const int64_t sl = slot_of(sg);
+        ml[i] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + sl * 2));
+        x[i] = __ldcg(reinterpret_cast<const float4*>(p.part_o + sl * kDecD) + lane);
+      }
     }
+    float mb = M;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mb = fmaxf(mb, ml[i].x);
+    if (mb == -INFINITY) continue;
+    const float a = M == -INFINITY ? 0.f : exp2f(M - mb);
+    l *= a;
+    o4 = make_float4(o4.x * a, o4.y * a, o4.z * a, o4.w * a);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float w = ml[i].x == -INFINITY ? 0.f : exp2f(ml[i].x - mb);
+      l = fmaf(ml[i].y, w, l);
+      o4.x = fmaf(x[i].x, w, o4.x);
+      o4.y = fmaf(x[i].y, w, o4.y);
+      o4.z = fmaf(x[i].z, w, o4.z);
+      o4.w = fmaf(x[i].w, w, o4.w);
+    }
+    M = mb;
   }
   sm_o[warp][lane] = o4;
-  if (lane == 0) sm_l[warp] = l;
+  if (lane == 0) {
+    sm_m[warp] = M;
+    sm_l[warp] = l;
+  }
   __syncthreads();
   if (warp == 0) {
-    float4 s4 = sm_o[0][lane];
-    float ls = sm_l[0];
+    float Mt = -INFINITY;
 #pragma unroll
-    for (int w = 1; w < kMergeWarps; ++w) {
-      const float4 y = sm_o[w][lane];
-      s4.x += y.x; s4.y += y.y; s4.z += y.z; s4.w += y.w;
-      ls += sm_l[w];
-    }
+    for (int w = 0; w < kMergeWarps; ++w) Mt = fmaxf(Mt, sm_m[w]);
+    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    float ls = 0.f;
+    if (Mt != -INFINITY)
+#pragma unroll
+      for (int w = 0; w < kMergeWarps; ++w) {
+        const float a = sm_m[w] == -INFINITY ? 0.f : exp2f(sm_m[w] - Mt);
+        const float4 y = sm_o[w][lane];
+        s4.x = fmaf(y.x, a, s4.x);
+        s4.y = fmaf(y.y, a, s4.y);
+        s4.z = fmaf(y.z, a, s4.z);
+        s4.w = fmaf(y.w, a, s4.w);
+        ls = fmaf(sm_l[w], a, ls);
+      }
     __nv_bfloat162* out = reinterpret_cast<__nv_bfloat162*>(p.O + (int64_t)row * kDecD + 4 * lane);
     out[0] = __floats2bfloat162_rn(ls > 0.f ? s4.x / ls : 0.f, ls > 0.f ? s4.y / ls : 0.f);
     out[1] = __floats2bfloat162_rn(ls > 0.f ? s4.z / ls : 0.f, ls > 0.f ? s4.w / ls : 0.f);
