@@ -75,6 +75,10 @@ def parse():
                          "before RoPE to msa_sparse_attend every step")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the step's kernels one by one instead of replaying a CUDA graph")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="routed decode (bank100m, bank10m): routed layers per step (0: the "
+                         "configuration's; one layer of the 100M-token bank is the 3.3 GB case "
+                         "the DRAM counters are captured on)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=3,
                     help="routed layers in the CPU-oracle sample")
@@ -219,7 +223,8 @@ class Decode:
         import synth
         from long_context_doc_b200.engine import DecodeLayer, RoutedDecode
         self.torch, self.msa, self.w, self.dev = torch, msa, w, dev
-        fetch = fetch if w.layers > 1 else "device"
+        # the 10M-token bank keeps K̄/V̄ in HBM; the 100M-token bank's live in pinned host memory
+        fetch = fetch if w.n_docs * w.doc_len > 50_000_000 else "device"
         self.L = w.layers
         self.scan = scan
         self.cached = cached
@@ -337,6 +342,9 @@ def run_libmsa(args):
     ranks = Ranks("nccl", dev)
     rank, world = ranks.rank, ranks.world
     w = synth.C4 if args.workload == "bank100m" else synth.C3
+    if args.layers > 0 and args.layers != w.layers:
+        w = w.scaled(layers=args.layers, name=w.name.replace(f"_{w.layers}l", "") +
+                     f"_{args.layers}l")
     wk = Decode(w, dev, args.fetch, rank, args.scan, cached=args.cached)
     torch.cuda.synchronize()
 
@@ -1192,6 +1200,9 @@ def run_generate(args):
     ranks = Ranks("nccl", dev, timeout_s=300)
     rank, world = ranks.rank, ranks.world
     w = synth.C4
+    if args.layers > 0 and args.layers != w.layers:
+        w = w.scaled(layers=args.layers, name=w.name.replace(f"_{w.layers}l", "") +
+                     f"_{args.layers}l")
     G = max(1, args.gen_tokens)
     # one context buffer per layer: the gathered memory stays fixed while tokens are generated
     wk = Decode(w, dev, args.fetch, rank, args.scan, nbuf=w.layers)
@@ -1361,7 +1372,8 @@ def run_generate(args):
         "warmup": max(args.warmup, 3), "ms_per_step": round(req_ms, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 normals, planted docs; no dataset)",
-        "config": {"workload": "gen100m", "bank_tokens": w.n_docs * w.doc_len,
+        "config": {"workload": "gen100m" if wk.L == 18 else f"gen100m_{wk.L}l",
+                   "bank_tokens": w.n_docs * w.doc_len,
                    "routed_layers": wk.L, "batch": B, "prompt_local_kv": L0,
                    "generated_tokens_per_query": G, "cache_capacity": cap, "k": w.k,
                    "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d,
@@ -1371,19 +1383,20 @@ def run_generate(args):
                          "126 MB L2",
                    "cuda_graph": use_graph, "parallelism": f"replicas x{world}"},
         "construct_ms": round(con_ms, 3), "token_step_ms": round(tok_ms, 4),
-        "roofline": {"kernel": "msa_decode_step (cache append + decode attention + merge), per "
-                               "routed layer of the graph-replayed token step",
+        "roofline": {"kernel": "msa_decode_step (decode attention with the cache append fused "
+                               "in + merge), per routed layer of the graph-replayed token step",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                     "traffic": captured_traffic(("attend_dec.cu", "common.cuh"),
-                                                 "attend_dec_gen100m_dram.json"),
+                     "traffic": captured_traffic(("attend_dec_plain.cu", "attend_dec.cu",
+                                                  "common.cuh"),
+                                                 "attend_dec_plain_gen100m_dram.json"),
                      "bytes_per_launch": round(step_bytes), "avg_launch_ms": round(dec_avg, 4)},
         "e2e": {"value": round(replica_rate(world, B * G, e2e_ms), 1), "unit": unit,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 3)},
-        # per request: the construction step's kernels + per token and layer append,
-        # attention and merge
-        "gpu_launches": Kst * (wk.kernels_per_step + G * wk.L * 3),
+        # per request: the construction step's kernels + per token and layer the attention
+        # (with the token's append) and the merge
+        "gpu_launches": Kst * (wk.kernels_per_step + G * wk.L * 2),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -349,11 +349,11 @@ class RoutedDecode:
         """Launches of libmsa kernels per step (memsets and copies excluded): per layer the
         routing call (tensor-core scan: query fold + scan with fused top-k; CUDA-core scan: one
         kernel per pass of up to 16 query rows), the gather (none with fetch='memcpy': the
-        gather indices kernel only), the decode attention and the merge of its splits, and with a
-        cache the append."""
+        gather indices kernel only), the decode attention (with a cache, the token's append
+        is fused into it) and the merge of its splits."""
         n = 0
         for la in self.layers:
             tc = la.Kbar_r_hat is not None and la.Q_r.dtype == torch.bfloat16
             route = 2 if tc else -(-self.B * self.T // 16)
-            n += route + 1 + 2 + (1 if self.cached else 0)
+            n += route + 1 + 2
         return n
