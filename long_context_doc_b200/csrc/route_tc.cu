@@ -269,6 +269,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
   const int64_t D0 = docs[3], D1 = docs[4], cb = docs[5], ce = docs[6];
   const int64_t n_ct = (ce - cb + kTcBM - 1) / kTcBM;
   const int64_t n_units = n_ct * p.n_qtiles;
+  // a range's partial last tile is loaded ending at the range's end: its first `shift` rows
+  // repeat rows of the tile before (just read, in L2) and are dropped, so no row past the range
+  // (the next CTA's) is read from memory; a range shorter than a tile reads past its end
+  auto tile_shift = [&](int64_t ct) -> int64_t {
+    return (ct == n_ct - 1 && ce - cb >= kTcBM) ? cb + (ct + 1) * kTcBM - ce : 0;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer
@@ -278,7 +284,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       int64_t issued = 0;
       for (int64_t u = 0; u < n_units; ++u) {
         const int64_t ct = u / p.n_qtiles, qt = u % p.n_qtiles;
-        const int y_a = (int)(cb + ct * kTcBM), y_b = (int)(qt * p.NQ * p.T);
+        const int y_a = (int)(cb + ct * kTcBM - tile_shift(ct)), y_b = (int)(qt * p.NQ * p.T);
         for (int kk = 0; kk < n_k; ++kk) {
           if (issued >= S && !wait_or_fail(&empty[s], ph ^ 1u, p.err, abort_flag)) break;
           unsigned char* st = base + (size_t)s * stage_bytes;
@@ -353,6 +359,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       }
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(a * 256);
+      const int mrow = row - (int)tile_shift(ct);  // the row's chunk offset in the tile
       int q = 0, t = 0;
       float cur = -INFINITY;
       for (int col = 0; got && col < ncols; col += 32) {
@@ -364,7 +371,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             cur = fmaxf(cur, v[j]);
             if (++t == p.T) {  // max over the query's tokens done
               const int b = (int)qt * p.NQ + q;
-              if (b < p.B) msc[row * p.B + b] = cur;
+              if (b < p.B && mrow >= 0) msc[mrow * p.B + b] = cur;
               cur = -INFINITY;
               t = 0;
               ++q;
