@@ -268,8 +268,8 @@ msa_status msa_route_topk(const void* Q_r, int32_t B, int32_t T, int32_t h_qr,
             MSA_ERR_WORKSPACE, "workspace %zu bytes at %p, need %zu (256-byte aligned)",
             ws_bytes, ws, need);
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = cudaMemsetAsync(ws, 0, kHeader, st);
-    if (e != cudaSuccess) return cuda_fail(e, "workspace header reset");
+    cudaError_t e = cudaSuccess;
+    // no memset node: the query fold (the call's first kernel) zeroes the header
     unsigned char* base = static_cast<unsigned char*>(ws);
     msa::RouteTcArgs ta{};
     ta.Q_r = Q_r;
@@ -586,10 +586,9 @@ msa_status msa_sparse_attend(const void* Q, int32_t B, int32_t T, int32_t h_q,
       q.part_ml = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes);
       q.part_o = reinterpret_cast<float*>(w8 + kHeader + dp.ctr_bytes + dp.part_ml_bytes);
       q.O = static_cast<__nv_bfloat16*>(O);
+      q.start_status = 1;  // no memset node: the attention kernel starts the status word
       cudaStream_t st = (cudaStream_t)stream;
-      // status word and segment tickets start at zero
-      cudaError_t e = cudaMemsetAsync(ws, 0, kHeader + dp.ctr_bytes, st);
-      if (e == cudaSuccess) e = msa::launch_attend_dec(q, dp, st);
+      cudaError_t e = msa::launch_attend_dec(q, dp, st);
       if (e != cudaSuccess) return cuda_fail(e, "msa_sparse_attend launch");
       return ok();
     }

@@ -152,6 +152,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
   const int Gq = p.h_q / HKV;
   const int nr = Gq * p.T;  // query rows per KV head (<= 8)
   // local rows per query: fixed, or read from the device (a cache that grows between launches)
+  if (p.start_status && blockIdx.x == 0 && tid == 0) *p.err = 0;
   const int L = p.L_dev != nullptr ? *p.L_dev : p.L;
   if (L < p.T || L > p.Ls) {  // uniform over the grid: nothing is read or written
     if (blockIdx.x == 0 && tid == 0) set_err(p.err, kErrBadIndex);
@@ -170,13 +171,15 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
   // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
   // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d. Issued by one
   // thread: the first NS tiles here, each later one by the warp that releases the stage last.
-  auto issue = [&](int v) {
+  auto issue = [&](int v, bool check_ctx) {
     const int64_t x = x0 + v;
     const int bb = (int)(x / TPP), tv = (int)(x % TPP);
     const bool ctx = tv < p.CT;
     const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
     // memory tiles past the query's context are not read (local tiles hold >= 1 row)
-    const bool any = !ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
+    // (the first tiles go out before ctx_len is read: rows past it are masked like a partial
+    // tile's)
+    const bool any = !ctx || !check_ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
     const int s = v % NS;
     const uint32_t st = smem_u32(stages + (size_t)s * kDecStage);
     fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
@@ -205,7 +208,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     // the first copies go out before the tables are built, so the prologue overlaps them
     // (none when the call is skipped: a CTA never exits with a copy in flight)
     if (!skip_call)
-      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
+      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v, false);
   }
   if (tid < HALF) turns[tid] = p.rope_turns[tid];
   if (tid < 32)
@@ -474,7 +477,7 @@ attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_const
     // release the stage; the last of the eight warps refills it with tile u + NS
     if (lane == 0 && atomicAdd(&released[s], 1u) % kDecCW == kDecCW - 1 && u + NS < n_tiles &&
         !*abort_flag)
-      issue(u + NS);
+      issue(u + NS, true);
     // next local tile: advance the position by KT (turn the query back by KT theta)
     if (!plain) {
 #pragma unroll

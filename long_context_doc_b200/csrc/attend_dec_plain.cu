@@ -130,6 +130,7 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
   // local rows per query: fixed, read from the device, or (fused append) the device length
   // plus the T tokens this call appends
   const bool fused = p.K_new != nullptr;
+  if (p.start_status && !fused && blockIdx.x == 0 && tid == 0) *p.err = 0;
   const int L = fused ? *reinterpret_cast<const volatile int32_t*>(p.L_dev) + p.T
                       : (p.L_dev != nullptr ? *p.L_dev : p.L);
   const bool bad = L < p.T || L > p.Ls;  // uniform over the grid: nothing is read or written
@@ -154,13 +155,15 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
 
   // Copies of tile v of this CTA's range into stage v % NS: four TMA boxes of
   // [KV head][key row][64 dims] (128-byte swizzle), the K and V halves of d.
-  auto issue = [&](int v) {
+  auto issue = [&](int v, bool check_ctx) {
     const int64_t x = x0 + v;
     const int bb = (int)(x / TPP), tv = (int)(x % TPP);
     const bool ctx = tv < p.CT;
     const int kt = ctx ? tv * KT : (tv - p.CT) * KT;
     // memory tiles past the query's context are not read (local tiles hold >= 1 row)
-    const bool any = !ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
+    // (the first tiles go out before ctx_len is read: rows past it are masked like a partial
+    // tile's)
+    const bool any = !ctx || !check_ctx || kt < min(max(__ldg(p.ctx_len + bb), 0), p.max_ctx);
     const int s = v % NS;
     const uint32_t st = smem_u32(stages + (size_t)s * kStage);
     fence_proxy_async_smem();  // the stage's earlier reads come before the new writes
@@ -188,7 +191,7 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
     // the first copies go out before the tables are built, so the prologue overlaps them
     // (none when the call is skipped: a CTA never exits with a copy in flight)
     if (!skip_call)
-      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v);
+      for (int v = 0; v < min(NS, n_tiles); ++v) issue(v, false);
   }
   if (tid < 32)
     ctx_first[tid] =
@@ -426,7 +429,7 @@ attend_dec_plain_kernel(const __grid_constant__ CUtensorMap map_kc,
       if (lane == 0 &&
           atomicAdd(&released[s], 1u) % kGroupWarps == kGroupWarps - 1 && u + NS < n_tiles &&
           !*abort_flag)
-        issue(u + NS);
+        issue(u + NS, true);
     }
     finish_segment(b);
     x = xe;

@@ -150,6 +150,9 @@ struct DecParams {
   int Ls;                   // local rows stored per query (row stride of Kl / Vl), >= L
   const int32_t* L_dev;     // nullable: the local length is read from here at run time
   int skip_on_err;          // write nothing if the status word already holds an error
+  int start_status;         // the first CTA starts the status word (the call's first kernel;
+                            // another CTA records an error only after a bounded wait has run
+                            // out, long after every CTA started)
   int keys_rotated;         // local keys are stored rotated at their positions pos0 + j
   int rope, pos0;
   unsigned long long rope_turns[64];  // theta_i / (2 pi) mod 1 as 64-bit binary fractions,

@@ -132,8 +132,11 @@ __global__ void __launch_bounds__(256) kr_normalize_kernel(const T* __restrict__
 template <typename T>
 __global__ void __launch_bounds__(256) q_fold_kernel(const T* __restrict__ q, int rows, int h_qr,
                                                      int h_kv, int d,
-                                                     __nv_bfloat16* __restrict__ out) {
+                                                     __nv_bfloat16* __restrict__ out,
+                                                     int* __restrict__ header) {
   const int lane = threadIdx.x & 31;
+  // the call's workspace header (status word, merge ticket) starts at zero for the scan
+  if (blockIdx.x == 0 && threadIdx.x < 64) header[threadIdx.x] = 0;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int m = h_qr / h_kv;
@@ -548,10 +551,10 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t
   if (qgrid > 4096) qgrid = 4096;
   if (a.dtype == 1)
     q_fold_kernel<__nv_bfloat16><<<(unsigned)qgrid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(a.Q_r), rows, a.h_qr, a.h_kv, a.d, a.q_hat);
+        static_cast<const __nv_bfloat16*>(a.Q_r), rows, a.h_qr, a.h_kv, a.d, a.q_hat, a.err);
   else
     q_fold_kernel<float><<<(unsigned)qgrid, 256, 0, st>>>(static_cast<const float*>(a.Q_r), rows,
-                                                          a.h_qr, a.h_kv, a.d, a.q_hat);
+                                                          a.h_qr, a.h_kv, a.d, a.q_hat, a.err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 2. tensor-core scores fused with the per-document max and the exact top-k
