@@ -79,6 +79,9 @@ def parse():
                     help="routed decode (bank100m, bank10m): routed layers per step (0: the "
                          "configuration's; one layer of the 100M-token bank is the 3.3 GB case "
                          "the DRAM counters are captured on)")
+    ap.add_argument("--docs", type=int, default=0,
+                    help="encode_hidden1m: documents of 1,024 tokens (0: the configuration's "
+                         "1,024; fewer make the small case the kernel's counters are captured on)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-layers", type=int, default=3,
                     help="routed layers in the CPU-oracle sample")
@@ -1455,6 +1458,8 @@ def run_encode_hidden(args):
     ranks = Ranks("nccl", dev)
     rank, world = ranks.rank, ranks.world
     w = synth.C2.scaled(seed=synth.C2.seed + 1000 * rank)
+    if args.docs > 0:
+        w = w.scaled(n_docs=args.docs)
     D, bf = 2560, torch.bfloat16
     off = np.arange(w.n_docs + 1, dtype=np.int64) * w.doc_len
     n_tok = int(off[-1])
@@ -1526,9 +1531,11 @@ def run_encode_hidden(args):
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normals; random "
                                                           "projection weights)",
-            "config": {"workload": "encode_hidden1m", "bank_tokens": n_tok, "n_docs": w.n_docs,
+            "config": {"workload": ("encode_hidden1m" if w.n_docs == 1024 else
+                                    f"encode_hidden_{w.n_docs}docs"),
+                       "bank_tokens": n_tok, "n_docs": w.n_docs,
                        "hidden": D, "h_kv": w.h_kv, "d": w.d, "chunk": w.chunk,
-                       "l2": "no flush: 5.4 GB of hidden states per call"},
+                       "l2": f"no flush: {n_tok * D * 2 / 1e9:.1f} GB of hidden states per call"},
             "roofline": {"kernel": "encode_hidden_kernel (tcgen05 projections + RoPE + pooling; "
                                    "the call also uploads the chunk table)",
                          "bound": "tensor", "achieved": round(tf, 1), "peak": tpeak,
