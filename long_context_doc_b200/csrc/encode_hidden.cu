@@ -21,8 +21,9 @@
 //                position (keys and router keys), masked to the chunk's valid rows, summed over
 //                the warp's 32 rows by a transposing shuffle reduction and added into a
 //                shared-memory row per chunk; the means are stored in bf16.
-// Units are ordered chunk pair by chunk pair, so the hidden rows of a pair are read from HBM
-// once and from L2 by its other units. Every wait is bounded; on expiry the CTA records an
+// Units are ordered chunk pair by chunk pair and dealt to the CTAs in turn, so the twelve
+// units of a pair run at about the same time and the pair's hidden rows are read from HBM once
+// and from L2 by its other units. Every wait is bounded; on expiry the CTA records an
 // error in the status word, stops issuing work, drains what it issued and frees its TMEM.
 #include <cuda.h>
 
@@ -148,7 +149,9 @@ encode_hidden_kernel(const __grid_constant__ CUtensorMap map_h,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t G = gridDim.x, ci = blockIdx.x;
-  const int64_t u0 = ci * p.n_units / G, u1 = (ci + 1) * p.n_units / G;
+  // units u = ci, ci + G, ...: at any time the CTAs work on about G consecutive units, the
+  // twelve units of a chunk pair among them, so a pair's hidden rows come from HBM once and
+  // from L2 for the other units (a contiguous range per CTA re-read them from HBM per unit)
   const int n_k = p.D / kBK;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -184,7 +187,7 @@ encode_hidden_kernel(const __grid_constant__ CUtensorMap map_h,
       int s = 0;
       uint32_t ph = 0;
       int64_t issued = 0;
-      for (int64_t u = u0; u < u1; ++u) {
+      for (int64_t u = ci; u < p.n_units; u += G) {
         const int64_t pr = u / per_pair;
         const int rest = (int)(u % per_pair), j = rest / p.n_tiles, t = rest % p.n_tiles;
         const int64_t ca = 2 * pr, cb = min(2 * pr + 1, p.n_chunks - 1);
@@ -215,8 +218,7 @@ encode_hidden_kernel(const __grid_constant__ CUtensorMap map_h,
                              ((uint32_t)(kBM >> 4) << 24);
       int s = 0;
       uint32_t ph = 0;
-      for (int64_t u = u0; u < u1; ++u) {
-        const int64_t i = u - u0;
+      for (int64_t u = ci, i = 0; u < p.n_units; u += G, ++i) {
         const int a = (int)(i & 1);
         const uint32_t aph = (uint32_t)((i >> 1) & 1);
         if (i >= 2 && !wait_or_fail(&tempty[a], aph ^ 1u, p.err, abort_flag)) break;
@@ -253,8 +255,7 @@ encode_hidden_kernel(const __grid_constant__ CUtensorMap map_h,
     const int slot = row >> 6;        // chunk 0 or 1 of the pair
     const int ri = row & 63;          // row within the chunk
     const int HALF = kBN / 4;         // 64: RoPE partner offset within a head of d = 128
-    for (int64_t u = u0; u < u1; ++u) {
-      const int64_t i = u - u0;
+    for (int64_t u = ci, i = 0; u < p.n_units; u += G, ++i) {
       const int a = (int)(i & 1);
       const uint32_t aph = (uint32_t)((i >> 1) & 1);
       const int64_t pr = u / per_pair;
