@@ -121,24 +121,38 @@ __device__ __forceinline__ void tma3d(uint32_t dst, const CUtensorMap* map, int 
       : "memory");
 }
 
+// Shared memory of the 8-warp kernel with an NS-stage ring: the stages, then the rotation
+// tables (R(c theta) for the KT = 64 / h_kv in-tile key offsets and 11 rows of 32 entries),
+// the RoPE turn counts, the combine buffer of the warps of a KV head (none when each warp owns
+// a KV head, h_kv = 8), the per-warp scratch and the ring's barriers and counters.
+__host__ __device__ constexpr size_t dec_comb_floats(int h_kv) {
+  return h_kv == 8 ? 0 : (size_t)kDecCW * 8 * kDecD;
+}
+__host__ __device__ constexpr size_t dec_smem(int NS, int h_kv) {
+  return 1024 + (size_t)NS * kDecStage + (size_t)(64 / h_kv) * 32 * 16 + 11 * 32 * 16 +
+         (kDecD / 2) * 8 + sizeof(float) * (dec_comb_floats(h_kv) + (size_t)kDecCW * 88) +
+         (size_t)NS * 12 + 16;
+}
+
+template <int NS>
 __global__ void __launch_bounds__(kDecThreads, 1)
 attend_dec_kernel(const __grid_constant__ CUtensorMap map_kc, const __grid_constant__ CUtensorMap map_vc,
                   const __grid_constant__ CUtensorMap map_kl, const __grid_constant__ CUtensorMap map_vl,
                   DecParams p) {
-  constexpr int D = kDecD, HALF = D / 2, NS = kDecStages;
+  constexpr int D = kDecD, HALF = D / 2;
   extern __shared__ __align__(1024) unsigned char sm_raw[];
   unsigned char* sm = smem_align1024(sm_raw);
   unsigned char* stages = sm;                                                 // [NS][K|V]
   float4* rstep = reinterpret_cast<float4*>(sm + NS * kDecStage);             // [KT][32]
-  float4* kturn = rstep + 64 * 32;                                            // [32]
+  float4* kturn = rstep + (64 / p.h_kv) * 32;                                 // [32]
   float4* qrot = kturn + 32;   // [T][32]: R(pos theta) at each query token's position
   float4* turn0 = qrot + 8 * 32;  // [32]: R(-pos0 theta), a query's first local tile
   float4* turn1 = turn0 + 32;     // [32]: R(-P theta), P = the CTA's first local tile start
   unsigned long long* turns = reinterpret_cast<unsigned long long*>(turn1 + 32);  // [HALF]
   const int RB = (p.h_q / p.h_kv) * p.T <= 4 ? 4 : 8;  // combine-buffer rows per KV head
   constexpr int WS = 11 * 8;                            // per-warp scratch floats
-  float* comb = reinterpret_cast<float*>(turns + HALF);  // [8][RB][D]
-  float* wscr = comb + kDecCW * 8 * D;                   // [8][WS]: max at 9 RB, sum at 10 RB
+  float* comb = reinterpret_cast<float*>(turns + HALF);  // [8][RB][D] (h_kv < 8 only)
+  float* wscr = comb + dec_comb_floats(p.h_kv);          // [8][WS]: max at 9 RB, sum at 10 RB
   uint64_t* full = reinterpret_cast<uint64_t*>(wscr + kDecCW * WS);  // [NS]
   unsigned int* released = reinterpret_cast<unsigned int*>(full + NS);  // [NS] warp releases
   volatile int* abort_flag = reinterpret_cast<volatile int*>(released + NS);
@@ -628,9 +642,9 @@ DecPlan attend_dec_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int
   pl.ctr_bytes = ((size_t)B * sizeof(unsigned int) + 255) & ~(size_t)255;
   pl.part_ml_bytes = max_seg > 1 ? ((slots * 2 * sizeof(float) + 255) & ~(size_t)255) : 0;
   pl.part_o_bytes = max_seg > 1 ? ((slots * kDecD * sizeof(float) + 255) & ~(size_t)255) : 0;
-  pl.smem = 1024 + (size_t)kDecStages * kDecStage + (size_t)64 * 32 * 16 + 11 * 32 * 16 +
-            (kDecD / 2) * 8 + sizeof(float) * ((size_t)kDecCW * 8 * kDecD + (size_t)kDecCW * 88) +
-            kDecStages * 12 + 16;
+  // a deeper ring where the shared memory allows it (no combine buffer at h_kv = 8)
+  pl.NS = dec_smem(6, h_kv) <= 227 * 1024 ? 6 : kDecStages;
+  pl.smem = dec_smem(pl.NS, h_kv);
   return pl;
 }
 
@@ -676,10 +690,9 @@ cudaError_t launch_attend_dec(const DecParams& p, const DecPlan& pl, cudaStream_
   if (p.keys_rotated || !p.rope) {  // keys used as stored: the 16-warp kernel
     e = launch_attend_dec_plain(p, pl, mkc, mvc, mkl, mvl, st);
   } else {
-    e = cudaFuncSetAttribute(attend_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)pl.smem);
-    if (e == cudaSuccess)
-      attend_dec_kernel<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
+    auto kfn = pl.NS == 6 ? attend_dec_kernel<6> : attend_dec_kernel<kDecStages>;
+    e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+    if (e == cudaSuccess) kfn<<<pl.grid, kDecThreads, pl.smem, st>>>(mkc, mvc, mkl, mvl, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   // (a fused append needs the merge kernel for the length update even with no split query)

@@ -178,6 +178,7 @@ struct DecParams {
 struct DecPlan {
   bool ok;
   int RB, TPP, CT, grid, max_seg;
+  int NS;                   // stages of the 8-warp kernel's copy ring (4, or 6 when h_kv = 8)
   int64_t n_pairs, total;   // n_pairs: queries that own tiles (B)
   size_t ctr_bytes, part_ml_bytes, part_o_bytes, smem;
 };
