@@ -9,21 +9,22 @@
 //    ruixiangma.github.io blog, "三阶段推理流程" and "Memory Interleaving"].
 //
 // Two kernels:
-//  * A pre-pass makes both tensor-core operands plain K-major tiles: Q and the local K are
-//    rotated once (bf16 out; angles as exact fixed-point turn counts through sincospi) and V
-//    (local and gathered memory rows) is transposed to [query][KV head][d][row], memory rows
-//    beyond ctx_len written as zeros.
+//  * A pre-pass rotates Q and the local K once (bf16 out; angles as exact fixed-point turn
+//    counts through sincospi).
 //  * The attention kernel, one CTA per (128 query rows of one KV head, KV head, query): the rows
 //    are 128 / (h_q / h_kv) tokens x the KV head's query heads. Warp 0 loads Q once and the
-//    key tiles (128 rows: K and V^T, two 128-byte-swizzled TMA boxes each, no multicast) into a
-//    2-stage ring; one thread of warp 1 issues tcgen05.mma (bf16 x bf16 -> fp32 in TMEM):
-//    S_j = Q K_j^T into one of two S buffers, issued one tile ahead, and O += P_j V_j into a
-//    TMEM accumulator; warps 2-9 (two per TMEM lane quarter: thread = one query row x one half
+//    key tiles (128 rows of K and of V as stored, two 128-byte-swizzled TMA boxes of 64 dims
+//    each, no multicast) into a 2-stage ring; one thread of warp 1 issues tcgen05.mma (bf16 x
+//    bf16 -> fp32 in TMEM): S_j = Q K_j^T into one of two S buffers, issued one tile ahead, and
+//    O += P_j V_j into a TMEM accumulator, V_j read as an MN-major operand straight from its
+//    [key][dim] tile (nothing is transposed in memory); warps 2-9 (two per TMEM lane quarter:
+//    thread = one query row x one half
 //    of the keys and of the output dims) read S_j, mask, keep the online softmax (the halves
 //    exchange the tile's row maximum through shared memory; the running maximum is raised only
 //    when a tile's maximum exceeds it by more than 8 in log2 units, and only then is O rescaled
-//    in TMEM), write P_j in bf16 to shared memory in the operand layout, and finally normalise
-//    O and store it.
+//    in TMEM), write P_j in bf16 to shared memory in the operand layout (and clear the V rows
+//    of a memory tile past ctx_len, whose contents are not defined: 0 * NaN would reach O),
+//    and finally normalise O and store it.
 // Every wait is bounded; on expiry the CTA records kErrWaitTimeout in the workspace status word,
 // stops, lets its copies and MMAs land, frees its TMEM and writes nothing.
 #include <cuda.h>
@@ -43,7 +44,7 @@ constexpr int kThreads = 320;   // warp 0 copies, warp 1 MMA, warps 2-9 softmax
 constexpr uint32_t kSlice = 128 * 128;           // one 128-row x 64-element bf16 slice: 16 KB
 constexpr uint32_t kQBytes = 2 * kSlice;         // Q tile (two 64-wide K slices)
 constexpr uint32_t kKBytes = 2 * kSlice;         // K tile
-constexpr uint32_t kVBytes = 2 * kSlice;         // V^T tile (two 64-key slices)
+constexpr uint32_t kVBytes = 2 * kSlice;         // V tile (two 64-dim slices)
 constexpr uint32_t kStage = kKBytes + kVBytes;   // 64 KB
 constexpr int kStages = 2;
 constexpr float kRaise = 8.f;  // log2 headroom before the running maximum is raised
@@ -56,13 +57,6 @@ __device__ __forceinline__ void tma3(void* dst, const CUtensorMap* map, int x, i
       "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void tma2(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
 __device__ __forceinline__ void fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -73,6 +67,13 @@ __device__ __forceinline__ void fence_after() {
 __device__ __forceinline__ uint64_t desc128(const void* slice) {
   const uint64_t a = (uint64_t)(smem_u32(slice) & 0x3FFFFu) >> 4;
   return a | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+// MN-major operand over [rows][64 bf16] swizzled slices read the other way: the 64 elements of
+// a 128-byte row run along N, the rows along K; 8-row K groups are 1024 bytes apart, the next
+// 64 elements along N start `lbo` bytes on (the next slice); a K step of 16 rows is +2048 bytes.
+__device__ __forceinline__ uint64_t desc_mn(const void* slice, uint32_t lbo) {
+  const uint64_t a = (uint64_t)(smem_u32(slice) & 0x3FFFFu) >> 4;
+  return a | ((uint64_t)(lbo >> 4) << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -175,36 +176,6 @@ __global__ void __launch_bounds__(256) rope_rows_kernel(const __nv_bfloat16* __r
   }
 }
 
-// V [B, R, h_kv, 128] -> V^T [B, h_kv, 128, Rp]: rows >= valid(b) written as zeros. CTA per
-// (64-row block, KV head, query): the block goes through shared memory.
-__global__ void __launch_bounds__(256) transpose_v_kernel(const __nv_bfloat16* __restrict__ V,
-                                                          __nv_bfloat16* __restrict__ Vt, int R,
-                                                          int Rp, int h_kv,
-                                                          const int32_t* __restrict__ valid_len,
-                                                          int valid_cap) {
-  __shared__ __nv_bfloat16 tile[64][kD + 8];
-  const int r0 = blockIdx.x * 64, g = blockIdx.y, b = blockIdx.z;
-  const int valid = valid_len ? min(max(valid_len[b], 0), valid_cap) : R;
-  for (int idx = threadIdx.x; idx < 64 * (kD / 8); idx += blockDim.x) {
-    const int rr = idx / (kD / 8), c8 = (idx % (kD / 8)) * 8;
-    const int row = r0 + rr;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (row < R && row < valid)
-      v = *reinterpret_cast<const uint4*>(V + (((int64_t)b * R + row) * h_kv + g) * kD + c8);
-    *reinterpret_cast<uint4*>(&tile[rr][c8]) = v;
-  }
-  __syncthreads();
-  // out row = dim, 64 consecutive keys: 8 threads per dim write 8 keys each (16 bytes)
-  for (int idx = threadIdx.x; idx < kD * 8; idx += blockDim.x) {
-    const int dim = idx / 8, k8 = (idx % 8) * 8;
-    if (r0 + k8 >= R) continue;
-    __align__(16) __nv_bfloat16 w[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) w[q] = tile[k8 + q][dim];
-    __nv_bfloat16* out = Vt + (((int64_t)b * h_kv + g) * kD + dim) * Rp + r0 + k8;
-    if (r0 + k8 + 8 <= Rp) *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(w);
-  }
-}
 
 // ------------------------------------------------------------------------------ attention
 __global__ void __launch_bounds__(kThreads, 1)
@@ -214,7 +185,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   extern __shared__ __align__(1024) unsigned char sm_raw[];
   unsigned char* base = smem_align1024(sm_raw);
   unsigned char* q_s = base;                                  // [2][128][64]
-  unsigned char* stages = base + kQBytes;                     // [S][K 2 slices | V^T 2 slices]
+  unsigned char* stages = base + kQBytes;                     // [S][K 2 slices | V 2 slices]
   unsigned char* p_s = stages + kStages * kStage;             // [2][128][64] probabilities
   float* xmax = reinterpret_cast<float*>(p_s + 2 * kSlice);  // [2 tiles][2 halves][128 rows]
   float* xsum = xmax + 512;                                  // [2 halves][128 rows]
@@ -279,8 +250,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_arrive_expect_tx(qfull, kQBytes);
       tma3(q_s, &map_q, 0, g * Gq, b * p.T + t0, qfull);
       tma3(q_s + kSlice, &map_q, 64, g * Gq, b * p.T + t0, qfull);
-      const int vrow = (b * p.h_kv + g) * kD;  // first V^T row of this (query, KV head)
-      // K of tile j may load once S_{j-2} is done, V^T once P_{j-2} V_{j-2} is done
+      // K of tile j may load once S_{j-2} is done, V once P_{j-2} V_{j-2} is done
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j & 1;
         const uint32_t par = (uint32_t)(((j >> 1) - 1) & 1);
@@ -299,8 +269,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           break;
         }
         mbar_arrive_expect_tx(&vfull[s], kVBytes);
-        tma2(st + kKBytes, mv, r0, vrow, &vfull[s]);
-        tma2(st + kKBytes + kSlice, mv, r0 + 64, vrow, &vfull[s]);
+        tma3(st + kKBytes, mv, 0, g, krow, &vfull[s]);
+        tma3(st + kKBytes + kSlice, mv, 64, g, krow, &vfull[s]);
         ++issued;
       }
       // the copies issued land before the CTA can exit
@@ -315,6 +285,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (lane == 0) {
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kN >> 3) << 17) |
                              ((uint32_t)(kM >> 4) << 24);
+      const uint32_t idesc_pv = idesc | (1u << 16);  // B (V) MN-major
       const uint64_t qd0 = desc128(q_s), qd1 = desc128(q_s + kSlice);
       const uint64_t pd0 = desc128(p_s), pd1 = desc128(p_s + kSlice);
       auto issue_s = [&](int j) -> bool {  // S_j = Q K_j^T into buffer j & 1
@@ -342,12 +313,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (!wait_or_abort(&vfull[j & 1], (uint32_t)((j >> 1) & 1), p.err, abort_flag)) break;
         fence_after();
         const unsigned char* st = stages + (j & 1) * kStage;
-        const uint64_t vd0 = desc128(st + kKBytes), vd1 = desc128(st + kKBytes + kSlice);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // O += P_j V_j over the tile's 128 keys
+        for (int kk = 0; kk < 8; ++kk) {  // O += P_j V_j over the tile's 128 keys, 16 per step
           const uint64_t a = (kk < 4 ? pd0 : pd1) + 2 * (kk & 3);
-          const uint64_t bb = (kk < 4 ? vd0 : vd1) + 2 * (kk & 3);
-          mma(tmem + 2u * kN, a, bb, idesc, (j | kk) ? 1u : 0u);
+          const uint64_t bb = desc_mn(st + kKBytes + kk * 2048, kSlice);
+          mma(tmem + 2u * kN, a, bb, idesc_pv, (j | kk) ? 1u : 0u);
         }
         commit(ofull);
         commit(&vempty[j & 1]);
@@ -470,8 +440,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
       }
       l += sum0 + sum1;
+      // a memory tile reaching past ctx_len: its V rows there are cleared once the tile has
+      // landed, before P_j V_j (thread: key row `row` of the tile, its half of the dims)
+      if (is_ctx && (j + 1) * kN > n_ctx) {
+        bad = bad || !__all_sync(0xffffffffu, wait_or_abort(&vfull[sb], (uint32_t)((j >> 1) & 1),
+                                                            p.err, abort_flag));
+        if (!bad && j * kN + row >= n_ctx) {
+          uint4* vr = reinterpret_cast<uint4*>(stages + sb * kStage + kKBytes + half * kSlice +
+                                               row * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) vr[q] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       fence_before();
-      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      fence_proxy_async_smem();  // P (and the cleared V rows) are read by the tensor core
       mbar_arrive(&sfree[sb]);
       mbar_arrive(pfull);
     }
@@ -538,13 +520,11 @@ AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int 
           (any_rows || Gq * T >= 64);
   if (!pl.ok) return pl;
   pl.n_qtiles = (Gq * T + atc::kM - 1) / atc::kM;
-  pl.Lp = (L + 7) / 8 * 8;
-  pl.Mp = (max_ctx + 7) / 8 * 8;
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
   pl.q_bytes = al((size_t)B * T * h_q * atc::kD * 2);
   pl.k_bytes = al((size_t)B * L * h_kv * atc::kD * 2);
-  pl.vl_bytes = al((size_t)B * h_kv * atc::kD * pl.Lp * 2);
-  pl.vc_bytes = max_ctx > 0 ? al((size_t)B * h_kv * atc::kD * pl.Mp * 2) : 0;
+  pl.vl_bytes = 0;  // V is read as stored (no transposed copy)
+  pl.vc_bytes = 0;
   pl.smem = 1024 + atc::kQBytes + atc::kStages * atc::kStage + 2 * atc::kSlice + 768 * 4 +
             20 * 8 + 16;
   return pl;
@@ -555,11 +535,8 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
   AtcParams p = p0;
   __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(scratch);
   __nv_bfloat16* k_rot = reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes);
-  __nv_bfloat16* vt_l = reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes + pl.k_bytes);
-  __nv_bfloat16* vt_c =
-      reinterpret_cast<__nv_bfloat16*>(scratch + pl.q_bytes + pl.k_bytes + pl.vl_bytes);
   const int Gq = p.h_q / p.h_kv;
-  // pre-pass: rotated Q and local K, transposed V
+  // pre-pass: rotated Q and local K
   {
     const int64_t qrows = (int64_t)p.B * p.T * p.h_q, krows = (int64_t)p.B * p.L * p.h_kv;
     const int64_t grid_q = std::min<int64_t>((qrows + 31) / 32, (int64_t)sms * 16);
@@ -568,13 +545,6 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
         p.Q, q_rot, qrows, p.h_q, p.T, (int64_t)p.pos0 + p.L - p.T, p);
     atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_k, 1), 256, 0, st>>>(
         p.Kl, k_rot, krows, p.h_kv, p.L, (int64_t)p.pos0, p);
-    atc::transpose_v_kernel<<<dim3((unsigned)((p.L + 63) / 64), (unsigned)p.h_kv, (unsigned)p.B),
-                              256, 0, st>>>(p.Vl, vt_l, p.L, pl.Lp, p.h_kv, nullptr, p.L);
-    if (p.max_ctx > 0)
-      atc::transpose_v_kernel<<<dim3((unsigned)((p.max_ctx + 63) / 64), (unsigned)p.h_kv,
-                                     (unsigned)p.B),
-                                256, 0, st>>>(p.cV, vt_c, p.max_ctx, pl.Mp, p.h_kv, p.ctx_len,
-                                              p.max_ctx);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -591,21 +561,17 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
     const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.L};
     const uint64_t str[2] = {row, row * p.h_kv};
     const uint32_t box[3] = {64, 1, atc::kN};
-    if (!encode_bf16_map(&mkl, k_rot, 3, dims, str, box, true)) return cudaErrorInvalidValue;
-    const uint64_t dv[2] = {(uint64_t)p.L, (uint64_t)p.B * p.h_kv * atc::kD};
-    const uint64_t sv[1] = {(uint64_t)pl.Lp * 2};
-    const uint32_t bv[2] = {64, atc::kD};
-    if (!encode_bf16_map(&mvl, vt_l, 2, dv, sv, bv, true)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mkl, k_rot, 3, dims, str, box, true) ||
+        !encode_bf16_map(&mvl, p.Vl, 3, dims, str, box, true))
+      return cudaErrorInvalidValue;
   }
   if (p.max_ctx > 0) {
     const uint64_t dims[3] = {atc::kD, (uint64_t)p.h_kv, (uint64_t)p.B * p.max_ctx};
     const uint64_t str[2] = {row, row * p.h_kv};
     const uint32_t box[3] = {64, 1, atc::kN};
-    if (!encode_bf16_map(&mkc, p.cK, 3, dims, str, box, true)) return cudaErrorInvalidValue;
-    const uint64_t dv[2] = {(uint64_t)p.max_ctx, (uint64_t)p.B * p.h_kv * atc::kD};
-    const uint64_t sv[1] = {(uint64_t)pl.Mp * 2};
-    const uint32_t bv[2] = {64, atc::kD};
-    if (!encode_bf16_map(&mvc, vt_c, 2, dv, sv, bv, true)) return cudaErrorInvalidValue;
+    if (!encode_bf16_map(&mkc, p.cK, 3, dims, str, box, true) ||
+        !encode_bf16_map(&mvc, p.cV, 3, dims, str, box, true))
+      return cudaErrorInvalidValue;
   } else {  // no memory tiles: never read
     mkc = mkl;
     mvc = mvl;

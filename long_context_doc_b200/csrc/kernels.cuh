@@ -270,8 +270,9 @@ struct AtcParams {
 };
 struct AtcPlan {
   bool ok;
-  int n_qtiles, Lp, Mp;     // query tiles per (query, KV head); padded row counts of V^T
-  size_t q_bytes, k_bytes, vl_bytes, vc_bytes, smem;  // scratch: rotated Q, rotated K, V^T
+  int n_qtiles;             // query tiles per (query, KV head)
+  // scratch: rotated Q, rotated K (V is read as stored: vl_bytes = vc_bytes = 0)
+  size_t q_bytes, k_bytes, vl_bytes, vc_bytes, smem;
 };
 // any_rows: accept fewer than 64 query rows per KV head (the backward's recompute)
 AtcPlan attend_tc_plan(int B, int T, int h_q, int h_kv, int d, int max_ctx, int L,
