@@ -144,35 +144,39 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ------------------------------------------------------------------------------ pre-pass
-// Rotated bf16 copies of rows [n_rows, 128]: row r sits at position base + (r / div) % mod.
-// Eight threads per row; thread q takes the RoPE pairs 8q .. 8q+7 (dims 8q.., 64+8q..) with
-// 16-byte loads and stores.
+// Rotated bf16 copies of Q and the local K.
+// RoPE of the rows of one position at a time (Q: the h_q heads of a token; local K: the h_kv
+// heads of a row): warp per position, lane l on the pairs 2l, 2l + 1 (dims 2l, 2l+1 and their
+// partners + 64), so each cos/sin is computed once per position and reused for every head, and
+// a head row is two coalesced 128-byte reads and writes. Position of position-row r:
+// base + r % mod.
 __global__ void __launch_bounds__(256) rope_rows_kernel(const __nv_bfloat16* __restrict__ src,
                                                         __nv_bfloat16* __restrict__ dst,
-                                                        int64_t n_rows, int64_t div, int64_t mod,
+                                                        int64_t n_pos, int heads, int64_t mod,
                                                         int64_t base, AtcParams p) {
-  const int q = threadIdx.x & 7;
-  const int64_t r0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 3;
-  const int64_t nr = ((int64_t)gridDim.x * blockDim.x) >> 3;
-  unsigned long long F[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) F[e] = p.rope_turns[8 * q + e];
-  for (int64_t r = r0; r < n_rows; r += nr) {
-    const int64_t pos = base + (r / div) % mod;
-    const uint4 lo = *reinterpret_cast<const uint4*>(src + r * kD + 8 * q);
-    const uint4 hi = *reinterpret_cast<const uint4*>(src + r * kD + 64 + 8 * q);
-    float a[8], c[8];
-    Vec<__nv_bfloat16, 8>::unpack(lo, a);
-    Vec<__nv_bfloat16, 8>::unpack(hi, c);
-    __align__(16) __nv_bfloat16 ol[8], oh[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float2 cs = p.rope ? rot_turns(pos, F[e]) : make_float2(1.f, 0.f);
-      ol[e] = __float2bfloat16_rn(a[e] * cs.x - c[e] * cs.y);
-      oh[e] = __float2bfloat16_rn(c[e] * cs.x + a[e] * cs.y);
+  const int lane = threadIdx.x & 31;
+  const int64_t w0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const unsigned long long F0 = p.rope_turns[2 * lane], F1 = p.rope_turns[2 * lane + 1];
+  for (int64_t r = w0; r < n_pos; r += nw) {
+    const int64_t pos = base + r % mod;
+    const float2 c0 = p.rope ? rot_turns(pos, F0) : make_float2(1.f, 0.f);
+    const float2 c1 = p.rope ? rot_turns(pos, F1) : make_float2(1.f, 0.f);
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(src + r * heads * kD);
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + r * heads * kD);
+#pragma unroll 8
+    for (int h = 0; h < heads; ++h) {
+      const uint32_t lo = __ldg(s32 + h * (kD / 2) + lane);
+      const uint32_t hi = __ldg(s32 + h * (kD / 2) + 32 + lane);
+      const float a0 = __uint_as_float(lo << 16), a1 = __uint_as_float(lo & 0xFFFF0000u);
+      const float b0 = __uint_as_float(hi << 16), b1 = __uint_as_float(hi & 0xFFFF0000u);
+      const __nv_bfloat162 ol =
+          __floats2bfloat162_rn(a0 * c0.x - b0 * c0.y, a1 * c1.x - b1 * c1.y);
+      const __nv_bfloat162 oh =
+          __floats2bfloat162_rn(b0 * c0.x + a0 * c0.y, b1 * c1.x + a1 * c1.y);
+      d32[h * (kD / 2) + lane] = *reinterpret_cast<const uint32_t*>(&ol);
+      d32[h * (kD / 2) + 32 + lane] = *reinterpret_cast<const uint32_t*>(&oh);
     }
-    *reinterpret_cast<uint4*>(dst + r * kD + 8 * q) = *reinterpret_cast<const uint4*>(ol);
-    *reinterpret_cast<uint4*>(dst + r * kD + 64 + 8 * q) = *reinterpret_cast<const uint4*>(oh);
   }
 }
 
@@ -538,13 +542,13 @@ cudaError_t launch_attend_tc(const AtcParams& p0, const AtcPlan& pl, unsigned ch
   const int Gq = p.h_q / p.h_kv;
   // pre-pass: rotated Q and local K
   {
-    const int64_t qrows = (int64_t)p.B * p.T * p.h_q, krows = (int64_t)p.B * p.L * p.h_kv;
-    const int64_t grid_q = std::min<int64_t>((qrows + 31) / 32, (int64_t)sms * 16);
-    const int64_t grid_k = std::min<int64_t>((krows + 31) / 32, (int64_t)sms * 16);
+    const int64_t qpos = (int64_t)p.B * p.T, kpos = (int64_t)p.B * p.L;  // warp per position
+    const int64_t grid_q = std::min<int64_t>((qpos + 7) / 8, (int64_t)sms * 8);
+    const int64_t grid_k = std::min<int64_t>((kpos + 7) / 8, (int64_t)sms * 8);
     atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_q, 1), 256, 0, st>>>(
-        p.Q, q_rot, qrows, p.h_q, p.T, (int64_t)p.pos0 + p.L - p.T, p);
+        p.Q, q_rot, qpos, p.h_q, p.T, (int64_t)p.pos0 + p.L - p.T, p);
     atc::rope_rows_kernel<<<(unsigned)std::max<int64_t>(grid_k, 1), 256, 0, st>>>(
-        p.Kl, k_rot, krows, p.h_kv, p.L, (int64_t)p.pos0, p);
+        p.Kl, k_rot, kpos, p.h_kv, p.L, (int64_t)p.pos0, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
