@@ -114,6 +114,13 @@ msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_
                            void* Kbar_r, float* kr_inv_norm, int64_t* doc_chunk_off,
                            int64_t n_chunks, void* stream);
 
+/* msa_encode_pool_status - the status of the last msa_encode_pool call on any stream of this
+ * device, read on `stream` (which it synchronises): *code = 0, or the code a bounded device
+ * wait recorded when it ran out (then MSA_ERR_DEVICE; the call's outputs are not defined).
+ * The bf16, d = 128 pooling streams its input through bulk copies and waits on them with a
+ * bound; each msa_encode_pool call starts the word at zero. No allocation. */
+msa_status msa_encode_pool_status(int32_t* code, void* stream);
+
 /* msa_kr_inv_norm - inverse L2 norms of a pre-pooled router-key bank (bank preparation for
  * banks that were not produced by msa_encode_pool): out[c,h] = 1/||Kbar_r[c,h,:]|| (0 for a
  * zero row), fp32 [n_chunks, h_kv]. */

@@ -29,7 +29,7 @@ LIB_PATH = _build.LIB
 # every symbol include/msa.h declares
 SYMBOLS = ("msa_status_string", "msa_last_error", "msa_version", "msa_set_device_wait_limit",
            "msa_count_chunks",
-           "msa_encode_pool", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
+           "msa_encode_pool", "msa_encode_pool_status", "msa_kr_inv_norm", "msa_kr_normalize", "msa_route_topk_workspace",
            "msa_route_topk", "msa_route_topk_noalloc", "msa_route_topk_noalloc_status",
            "msa_workspace_status", "msa_gather", "msa_fetch_create", "msa_fetch_destroy",
            "msa_fetch_begin", "msa_fetch_finish", "msa_sparse_attend_workspace",
@@ -62,6 +62,8 @@ def _load():
     L.msa_set_device_wait_limit.argtypes = [i64]
     L.msa_count_chunks.restype = i64
     L.msa_count_chunks.argtypes = [vp, i64, i32]
+    L.msa_encode_pool_status.restype = ctypes.c_int
+    L.msa_encode_pool_status.argtypes = [vp, vp]
     L.msa_encode_pool.restype = ctypes.c_int
     L.msa_encode_pool.argtypes = [vp, vp, vp, i64, vp, vp, i64, i32, i32, i32, i32, f32, vp, vp,
                                   vp, vp, vp, i64, vp]
@@ -271,6 +273,16 @@ def msa_route_topk_noalloc_status(stream=None) -> int:
 def msa_workspace_status(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     st = lib.msa_workspace_status(_p(ws), ctypes.addressof(code), _s(stream))
+    if st not in (0, 6):
+        _check(st)
+    return int(code.value)
+
+
+def msa_encode_pool_status(stream=None) -> int:
+    """Status word of the last msa_encode_pool call (0, or the code of an expired device
+    wait); synchronises `stream`."""
+    code = ctypes.c_int32(0)
+    st = lib.msa_encode_pool_status(ctypes.addressof(code), _s(stream))
     if st not in (0, 6):
         _check(st)
     return int(code.value)

@@ -185,6 +185,16 @@ msa_status msa_encode_pool(const void* K, const void* V, const void* K_r, int64_
   return ok();
 }
 
+msa_status msa_encode_pool_status(int32_t* code, void* stream) {
+  REQUIRE(code, MSA_ERR_INVALID_ARG, "null code");
+  int v = 0;
+  cudaError_t e = msa::read_encode_status(&v, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "msa_encode_pool_status");
+  *code = v;
+  if (v != 0) return fail(MSA_ERR_DEVICE, "device status %d recorded by the pooling encode", v);
+  return ok();
+}
+
 msa_status msa_kr_inv_norm(const void* Kbar_r, int64_t n_chunks, int32_t h_kv, int32_t d,
                            int32_t dtype, float* out, void* stream) {
   msa_status s = check_common(h_kv, d, dtype);

@@ -19,6 +19,8 @@
 // table per 64-token block). Every cos/sin comes from the exact angle mod 2 pi (integer
 // position x 64-bit fixed-point theta / 2 pi) through a single-precision sincospi; the padded
 // table rows give conflict-free 16-byte reads.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -192,6 +194,204 @@ __global__ void __launch_bounds__(256) encode_pool_kernel(EncodeParams p) {
   }
 }
 
+// Status word of the pooling encode (bounded waits of encode_pool_tma_kernel), zeroed by
+// each call's chunk-offset kernel, read by msa_encode_pool_status.
+__device__ int g_encode_status;
+
+// The same pooling for bf16, d = 128, chunks of at most 64 tokens and h_kv <= 8, fed by the
+// bulk-copy engine: one CTA per SM over a contiguous chunk range; warp 0 copies each chunk's
+// token rows (contiguous in [token][KV head][d]) of K, V and K_r in blocks of kEpTB tokens into
+// a kEpNS-stage ring (one 1-D bulk copy per tensor and block, completion counted in bytes on
+// the stage's mbarrier); consumer warp h owns KV head h, lane l its RoPE pairs 2l, 2l+1 (dims
+// 2l, 2l+1 and their partners + 64), and reads a block's rows from shared memory (a warp reads
+// 128 contiguous bytes per row half). Each thread sums its pairs over the chunk's tokens in
+// order (keys rotated by c*theta from the per-CTA table, c the offset in the chunk), turns the
+// sums by the chunk's start position, divides by the token count and stores the means; the
+// warp reduces the squares of its head's bf16 K̄_r for the inverse norm. No shuffle
+// reduction and no barrier between chunks: the copies of the next blocks are in flight while a
+// chunk is finished.
+constexpr int kEpTB = 8;   // tokens per copy block
+constexpr int kEpNS = 4;   // ring stages
+__global__ void __launch_bounds__(32 + 8 * 32, 1) encode_pool_tma_kernel(EncodeParams p) {
+  constexpr int D = 128, HALF = 64;
+  const int W = p.h_kv * D;                  // elements of a token row
+  const uint32_t row_bytes = (uint32_t)W * 2;
+  const uint32_t blk_bytes = kEpTB * row_bytes;  // one tensor's block in a stage
+  extern __shared__ __align__(1024) unsigned char sm_raw[];
+  unsigned char* stages = smem_align1024(sm_raw);                          // [NS][K|V|Kr]
+  float2* cs = reinterpret_cast<float2*>(stages + kEpNS * 3 * blk_bytes);  // [64][64]
+  unsigned long long* turns = reinterpret_cast<unsigned long long*>(cs + 64 * HALF);  // [64]
+  uint64_t* full = reinterpret_cast<uint64_t*>(turns + HALF);             // [NS]
+  uint64_t* empty = full + kEpNS;                                           // [NS]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kEpNS);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool rope = p.rope != 0;
+  const int64_t c_begin = (int64_t)blockIdx.x * p.n_chunks / gridDim.x;
+  const int64_t c_end = ((int64_t)blockIdx.x + 1) * p.n_chunks / gridDim.x;
+  if (tid == 0) {
+    for (int s = 0; s < kEpNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], p.h_kv);  // one arrival per consumer warp
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (rope) {
+    for (int i = tid; i < HALF; i += blockDim.x) turns[i] = p.rope_turns[i];
+    __syncthreads();
+    for (int idx = tid; idx < 64 * HALF; idx += blockDim.x)
+      cs[idx] = rot_turns(idx / HALF, turns[idx % HALF]);  // R(c theta), c < 64
+  }
+  __syncthreads();
+  int64_t doc = c_begin < c_end ? lower_bound_i64(p.chunk_off, p.n_docs, c_begin + 1) - 1 : 0;
+
+  if (warp == 0) {
+    // ---------------- copies
+    if (lane == 0) {
+      const unsigned char* src[3] = {static_cast<const unsigned char*>(p.K),
+                                     static_cast<const unsigned char*>(p.V),
+                                     static_cast<const unsigned char*>(p.Kr)};
+      int s = 0;
+      uint32_t ph = 0;
+      int64_t issued = 0;
+      for (int64_t c = c_begin; c < c_end && !*abort_flag; ++c) {
+        while (p.chunk_off[doc + 1] <= c) ++doc;
+        const int64_t t0 = p.tok_off[doc] + (c - p.chunk_off[doc]) * p.chunk;
+        const int n = (int)(min(t0 + p.chunk, p.tok_off[doc + 1]) - t0);
+        for (int tb = 0; tb < n; tb += kEpTB) {
+          const uint32_t bytes = (uint32_t)min(kEpTB, n - tb) * row_bytes;
+          if (issued >= kEpNS && !mbar_wait_bounded(&empty[s], ph ^ 1u, &g_encode_status)) {
+            *abort_flag = 1;
+            break;
+          }
+          unsigned char* st = stages + (size_t)s * 3 * blk_bytes;
+          mbar_arrive_expect_tx(&full[s], 3 * bytes);
+#pragma unroll
+          for (int q = 0; q < 3; ++q)
+            bulk_g2s(st + q * blk_bytes, src[q] + (t0 + tb) * (int64_t)row_bytes, bytes, &full[s]);
+          ++issued;
+          if (++s == kEpNS) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // every copy issued lands before the CTA exits (bounded)
+      for (int64_t j = (issued > kEpNS ? issued - kEpNS : 0); j < issued; ++j)
+        mbar_wait_bounded(&full[j % kEpNS], (uint32_t)((j / kEpNS) & 1), &g_encode_status);
+    }
+    return;
+  }
+  // ---------------- consumers: warp h = KV head h - 1 + 1 (warps 1..h_kv)
+  const int h = warp - 1;
+  if (h >= p.h_kv) return;
+  const int e1 = 2 * lane;  // first-half dims e1, e1 + 1 of the head; partners + 64
+  const uint32_t col = (uint32_t)(h * D + e1) * 2;  // byte offset of dims e1, e1+1 in a row
+  int s = 0;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int64_t c = c_begin; c < c_end; ++c) {
+    while (p.chunk_off[doc + 1] <= c) ++doc;
+    const int64_t j = c - p.chunk_off[doc];
+    const int64_t t0 = p.tok_off[doc] + j * p.chunk;
+    const int n = (int)(min(t0 + p.chunk, p.tok_off[doc + 1]) - t0);
+    float k1[2] = {0.f, 0.f}, k2[2] = {0.f, 0.f}, r1[2] = {0.f, 0.f}, r2[2] = {0.f, 0.f};
+    float v1[2] = {0.f, 0.f}, v2[2] = {0.f, 0.f};
+    for (int tb = 0; tb < n; tb += kEpTB) {
+      const int nt = min(kEpTB, n - tb);
+      if (ok && !mbar_wait_bounded(&full[s], ph, &g_encode_status)) {
+        ok = false;
+        *abort_flag = 1;
+      }
+      if (ok) {
+        const unsigned char* st = stages + (size_t)s * 3 * blk_bytes + col;
+#pragma unroll 4
+        for (int t = 0; t < nt; ++t) {
+          const unsigned char* rk = st + t * row_bytes;
+          const uint32_t ka = *reinterpret_cast<const uint32_t*>(rk);
+          const uint32_t kb = *reinterpret_cast<const uint32_t*>(rk + HALF * 2);
+          const uint32_t va = *reinterpret_cast<const uint32_t*>(rk + blk_bytes);
+          const uint32_t vb = *reinterpret_cast<const uint32_t*>(rk + blk_bytes + HALF * 2);
+          const uint32_t ra = *reinterpret_cast<const uint32_t*>(rk + 2 * blk_bytes);
+          const uint32_t rb = *reinterpret_cast<const uint32_t*>(rk + 2 * blk_bytes + HALF * 2);
+          const float a[2] = {__uint_as_float(ka << 16), __uint_as_float(ka & 0xFFFF0000u)};
+          const float b[2] = {__uint_as_float(kb << 16), __uint_as_float(kb & 0xFFFF0000u)};
+          const float x[2] = {__uint_as_float(ra << 16), __uint_as_float(ra & 0xFFFF0000u)};
+          const float y[2] = {__uint_as_float(rb << 16), __uint_as_float(rb & 0xFFFF0000u)};
+          v1[0] += __uint_as_float(va << 16);
+          v1[1] += __uint_as_float(va & 0xFFFF0000u);
+          v2[0] += __uint_as_float(vb << 16);
+          v2[1] += __uint_as_float(vb & 0xFFFF0000u);
+          if (rope) {
+            const float4 t2 = *reinterpret_cast<const float4*>(cs + (tb + t) * HALF + e1);
+            const float2 c0 = make_float2(t2.x, t2.y), c1 = make_float2(t2.z, t2.w);
+            k1[0] += a[0] * c0.x - b[0] * c0.y;
+            k2[0] += b[0] * c0.x + a[0] * c0.y;
+            k1[1] += a[1] * c1.x - b[1] * c1.y;
+            k2[1] += b[1] * c1.x + a[1] * c1.y;
+            r1[0] += x[0] * c0.x - y[0] * c0.y;
+            r2[0] += y[0] * c0.x + x[0] * c0.y;
+            r1[1] += x[1] * c1.x - y[1] * c1.y;
+            r2[1] += y[1] * c1.x + x[1] * c1.y;
+          } else {
+            k1[0] += a[0]; k1[1] += a[1]; k2[0] += b[0]; k2[1] += b[1];
+            r1[0] += x[0]; r1[1] += x[1]; r2[0] += y[0]; r2[1] += y[1];
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);  // the stage's rows of this head are consumed
+      if (++s == kEpNS) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    if (!ok) continue;  // an expired wait: nothing more is written
+    if (rope) {  // turn the sums by the chunk's start position
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float2 t = rot_turns(j * p.chunk, turns[e1 + e]);
+        const float a = k1[e] * t.x - k2[e] * t.y, b = k2[e] * t.x + k1[e] * t.y;
+        k1[e] = a;
+        k2[e] = b;
+        const float ar = r1[e] * t.x - r2[e] * t.y, br = r2[e] * t.x + r1[e] * t.y;
+        r1[e] = ar;
+        r2[e] = br;
+      }
+    }
+    const float fn = (float)n;
+    const int64_t ob = c * (int64_t)W + h * D + e1;
+    const __nv_bfloat162 ok1 = __floats2bfloat162_rn(k1[0] / fn, k1[1] / fn);
+    const __nv_bfloat162 ok2 = __floats2bfloat162_rn(k2[0] / fn, k2[1] / fn);
+    const __nv_bfloat162 or1 = __floats2bfloat162_rn(r1[0] / fn, r1[1] / fn);
+    const __nv_bfloat162 or2 = __floats2bfloat162_rn(r2[0] / fn, r2[1] / fn);
+    const __nv_bfloat162 ov1 = __floats2bfloat162_rn(v1[0] / fn, v1[1] / fn);
+    const __nv_bfloat162 ov2 = __floats2bfloat162_rn(v2[0] / fn, v2[1] / fn);
+    __nv_bfloat16* Kb = static_cast<__nv_bfloat16*>(p.Kb);
+    __nv_bfloat16* Vb = static_cast<__nv_bfloat16*>(p.Vb);
+    __nv_bfloat16* Rb = static_cast<__nv_bfloat16*>(p.Rb);
+    *reinterpret_cast<__nv_bfloat162*>(Kb + ob) = ok1;
+    *reinterpret_cast<__nv_bfloat162*>(Kb + ob + HALF) = ok2;
+    *reinterpret_cast<__nv_bfloat162*>(Rb + ob) = or1;
+    *reinterpret_cast<__nv_bfloat162*>(Rb + ob + HALF) = or2;
+    *reinterpret_cast<__nv_bfloat162*>(Vb + ob) = ov1;
+    *reinterpret_cast<__nv_bfloat162*>(Vb + ob + HALF) = ov2;
+    if (p.inv_norm != nullptr) {  // of the stored bf16 K̄_r row of this head
+      const float2 f1 = __bfloat1622float2(or1), f2 = __bfloat1622float2(or2);
+      float ss = f1.x * f1.x + f1.y * f1.y + f2.x * f2.x + f2.y * f2.y;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) p.inv_norm[c * p.h_kv + h] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+    }
+  }
+}
+
+size_t encode_pool_tma_smem(int h_kv) {
+  const size_t blk = (size_t)kEpTB * h_kv * 128 * 2;
+  return 1024 + kEpNS * 3 * blk + sizeof(float2) * 64 * 64 + 64 * 8 + 2 * kEpNS * 8 + 16;
+}
+
 // Inverse norms of a pre-pooled bank: one warp per (chunk, head) row.
 template <typename T>
 __global__ void __launch_bounds__(256) inv_norm_kernel(const T* __restrict__ R, int64_t rows,
@@ -217,6 +417,7 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int64_t* __re
                                                              int64_t* __restrict__ out) {
   __shared__ int64_t part[1024];
   const int tid = threadIdx.x;
+  if (tid == 0) g_encode_status = 0;  // the call's status word starts at zero
   const int64_t per = (n_docs + blockDim.x - 1) / blockDim.x;
   const int64_t a = min(n_docs, (int64_t)tid * per), b = min(n_docs, a + per);
   int64_t s = 0;
@@ -285,19 +486,42 @@ static cudaError_t launch_encode_e(const EncodeParams& p, int sms, cudaStream_t 
 cudaError_t launch_encode_pool(const EncodeParams& p, int dtype, int d, int sms,
                                cudaStream_t st) {
   cudaError_t e = cudaSuccess;
-  if (p.n_docs > 0) {
+  if (p.n_docs > 0) {  // (also starts the status word)
     chunk_offsets_kernel<<<1, 1024, 0, st>>>(p.tok_off, p.n_docs, p.chunk,
                                              const_cast<int64_t*>(p.chunk_off));
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+  } else {
+    void* sw = nullptr;
+    e = cudaGetSymbolAddress(&sw, g_encode_status);
+    if (e == cudaSuccess) e = cudaMemsetAsync(sw, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
   }
   if (p.n_chunks == 0) return cudaSuccess;
+  if (dtype == 1 && d == 128 && p.chunk <= 64 && p.h_kv >= 1 && p.h_kv <= 8) {
+    const size_t smem = encode_pool_tma_smem(p.h_kv);
+    e = cudaFuncSetAttribute(encode_pool_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(sms, p.n_chunks);
+    encode_pool_tma_kernel<<<(unsigned)grid, 32 + 32 * p.h_kv, smem, st>>>(p);
+    return cudaGetLastError();
+  }
   if (dtype == 1) {
     return d == 128 ? launch_encode_e<__nv_bfloat16, 8, 128>(p, sms, st)
                     : launch_encode_e<__nv_bfloat16, 8, 64>(p, sms, st);
   }
   return d == 128 ? launch_encode_e<float, 4, 128>(p, sms, st)
                   : launch_encode_e<float, 4, 64>(p, sms, st);
+}
+
+cudaError_t read_encode_status(int* code, cudaStream_t st) {
+  int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_encode_status, sizeof v, 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  *code = v;
+  return e;
 }
 
 cudaError_t launch_inv_norm(const void* R, int64_t n_chunks, int h_kv, int d, int dtype,

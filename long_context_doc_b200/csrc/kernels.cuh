@@ -32,6 +32,8 @@ struct EncodeParams {
   float* inv_norm;           // nullable
 };
 cudaError_t launch_encode_pool(const EncodeParams& p, int dtype, int d, int sms, cudaStream_t st);
+// encode_pool.cu: the pooling encode's status word (an expired bounded wait), read on `st`
+cudaError_t read_encode_status(int* code, cudaStream_t st);
 cudaError_t launch_inv_norm(const void* R, int64_t n_chunks, int h_kv, int d, int dtype, float* out,
                             int sms, cudaStream_t st);
 

@@ -44,6 +44,7 @@ def _encode_case(msa, gpu, w):
     out = msa.encode_pool(to_dev(inp["K"], gpu), to_dev(inp["V"], gpu), to_dev(inp["K_r"], gpu),
                           inp["doc_tok_off"], w.chunk, w.rope_base)
     torch.cuda.synchronize()
+    assert msa.msa_encode_pool_status() == 0  # no device wait ran out
     assert np.array_equal(out["doc_chunk_off"].cpu().numpy(), coff)
     check_pooled(out["Kbar"], Kb, w.dtype, "Kbar")
     check_pooled(out["Vbar"], Vb, w.dtype, "Vbar")
@@ -61,23 +62,31 @@ def _encode_case(msa, gpu, w):
     synth.C2.scaled(n_docs=12, doc_len=300, ragged=True, n_planted=2),   # Qwen3-4B heads, bf16
     synth.C2.scaled(n_docs=6, doc_len=1024, n_planted=1, chunk=128),     # chunk > table block
     synth.C1.scaled(n_docs=9, doc_len=5, chunk=1, n_planted=0),          # chunk = 1
-], ids=["c1_full", "ragged_fp32", "qwen3_bf16_ragged", "chunk128", "chunk1"])
+    synth.C2.scaled(n_docs=40, doc_len=90, ragged=True, h_q=16, h_kv=4, h_qr=4, n_planted=1,
+                    seed=5),                                             # bf16, 4 KV heads
+    synth.C2.scaled(n_docs=17, doc_len=200, ragged=True, n_planted=1, rope_base=0.0,
+                    chunk=48, seed=6),                                   # bf16, no RoPE, chunk 48
+], ids=["c1_full", "ragged_fp32", "qwen3_bf16_ragged", "chunk128", "chunk1", "bf16_hkv4",
+        "bf16_norope_chunk48"])
 def test_encode_pool_matches_oracle(msa, gpu, w):
     _encode_case(msa, gpu, w)
 
 
-def test_encode_pool_constant_chunk_and_empty_docs(msa, gpu):
+@pytest.mark.parametrize("dt,h_kv,d", [(torch.float32, 2, 64), (torch.bfloat16, 8, 128)],
+                         ids=["fp32", "bf16_bulk_copies"])
+def test_encode_pool_constant_chunk_and_empty_docs(msa, gpu, dt, h_kv, d):
     lens = np.array([7, 0, 64, 65, 0])
     off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
     n = int(off[-1])
-    c = torch.full((n, 2, 64), 0.75, dtype=torch.float32, device=gpu)
+    c = torch.full((n, h_kv, d), 0.75, dtype=dt, device=gpu)
     out = msa.encode_pool(c, c, c, off, 64, 0.0)  # RoPE disabled
     torch.cuda.synchronize()
+    assert msa.msa_encode_pool_status() == 0
     for key in ("Kbar", "Vbar", "Kbar_r"):
         assert torch.all(out[key] == 0.75)
     assert out["doc_chunk_off"].cpu().tolist() == [0, 1, 1, 2, 4, 4]
     inv = out["kr_inv_norm"].cpu().numpy()
-    np.testing.assert_allclose(inv, 1.0 / np.sqrt(64 * 0.75 ** 2), rtol=1e-6)
+    np.testing.assert_allclose(inv, 1.0 / np.sqrt(d * 0.75 ** 2), rtol=1e-6)
 
 
 def test_encode_pool_full_1m_token_bank_sampled(msa, gpu):
