@@ -40,7 +40,11 @@ namespace msa {
 constexpr int kTcMaxStages = 12;
 constexpr int kTcBM = 128;        // chunks per tile (TMEM lanes)
 constexpr int kTcBK = 64;         // K slice (128 bytes of bf16: one swizzle row)
-constexpr int kTcThreads = 192;   // 6 warps
+// 6 warps (copies, MMA issue, 4 epilogue warps), or 8 for decode batches of more than 6
+// queries: the 2 more wait for the final merge, which then takes a query per warp in one round
+// (measured: 3 us less at 8 decode queries; 13 us more per call at 4 queries over the 100M-token
+// bank, where the 6-warp form keeps the scan at the copy peak)
+constexpr int kTcWarpsMerge = 8;
 
 // ------------------------------------------------------------------ PTX wrappers (sm_100a)
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -204,7 +208,8 @@ __device__ __forceinline__ void epi_sync() {  // the 128 epilogue threads only
 // Work of a CTA: the chunk tiles (128 rows from the CTA's first chunk) of its document-aligned
 // chunk range, each against every row tile of queries; units are (chunk tile, query tile),
 // query tiles innermost.
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                 TcParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -256,8 +261,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     epi_abort[1] = 0;
     fence_mbar_init();
   }
-  for (int j = threadIdx.x; j < p.B * 32; j += kTcThreads) lists[j] = 0ull;
-  for (int j = threadIdx.x; j < p.B; j += kTcThreads) carry[j] = -INFINITY;
+  for (int j = threadIdx.x; j < p.B * 32; j += NW * 32) lists[j] = 0ull;
+  for (int j = threadIdx.x; j < p.B; j += NW * 32) carry[j] = -INFINITY;
   if (warp == 0) {  // two fp32 accumulators of up to 256 columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_holder)),
@@ -333,7 +338,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
       tc_commit(done);
       mbar_wait_bounded(done, 0, p.err);
     }
-  } else {
+  } else if (warp < 6) {
     // ---------------- epilogue (warps 2..5 -> TMEM lane groups 2, 3, 0, 1)
     const int lg = warp & 3;
     const int ew = warp - 2;                 // epilogue warp 0..3
@@ -480,7 +485,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                  : "memory");
 
   // ---------------- publish this CTA's candidates; the last CTA merges
-  for (int b = warp; b < p.B; b += kTcThreads / 32)
+  for (int b = warp; b < p.B; b += NW)
     if (lane < p.k) p.cand[(ci * p.B + b) * p.k + lane] = lists[b * 32 + lane];
   __threadfence();
   __syncthreads();
@@ -583,10 +588,12 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, const TcPlan& pl, cudaStream_t
   p.counter = a.counter;
   p.err = a.err;
   p.wait_limit = a.wait_limit;
-  e = cudaFuncSetAttribute(route_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)pl.smem);
+  // decode batches of more than 6 queries: 8 warps, one merge round
+  const int nw = (pl.n_qtiles == 1 && a.B > 6 && a.B <= kTcWarpsMerge) ? kTcWarpsMerge : 6;
+  auto kfn = nw == kTcWarpsMerge ? route_tc_kernel<kTcWarpsMerge> : route_tc_kernel<6>;
+  e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
   if (e != cudaSuccess) return e;
-  route_tc_kernel<<<pl.grid, kTcThreads, pl.smem, st>>>(mk, mq, p);
+  kfn<<<pl.grid, nw * 32, pl.smem, st>>>(mk, mq, p);
   return cudaGetLastError();
 }
 
