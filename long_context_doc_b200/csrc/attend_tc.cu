@@ -101,6 +101,22 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The same load without the wait: several loads in flight, then one tmem_wait_ld().
+__device__ __forceinline__ void ld32_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -357,20 +373,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const uint32_t sa = lane_base + (uint32_t)(sb * kN) + col0;
       const bool all_vis = lim >= 63;  // every key of this half visible to the row
       float mx = -INFINITY;
+      uint32_t sr[64];  // this half's 64 scores of the row, loaded once for both passes
       if (ok) {
         fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t r[32];
-          ld32(sa + ch * 32, r);
-          if (all_vis) {
+        ld32_nowait(sa, sr);
+        ld32_nowait(sa + 32, sr + 32);
+        tmem_wait_ld();
+        if (all_vis) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) mx = fmaxf(mx, __uint_as_float(r[q]));
-          } else {
+          for (int q = 0; q < 64; ++q) mx = fmaxf(mx, __uint_as_float(sr[q]));
+        } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (ch * 32 + q <= lim) mx = fmaxf(mx, __uint_as_float(r[q]));
-          }
+          for (int q = 0; q < 64; ++q)
+            if (q <= lim) mx = fmaxf(mx, __uint_as_float(sr[q]));
         }
         mx *= c;  // the scale is positive: max of the scaled scores
       }
@@ -409,10 +424,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       unsigned char* slice = p_s + half * kSlice + row * 128;
       const float negm = -m;
       const bool none = m == -INFINITY;
-#pragma unroll 1
-      for (int ch = 0; ch < 2; ++ch) {
-        uint32_t r[32];
-        ld32(sa + ch * 32, r);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {  // the scores loaded in pass 1
+        const uint32_t* r = sr + ch * 32;
         uint32_t pk[16];
         if (all_vis && !none) {
 #pragma unroll
