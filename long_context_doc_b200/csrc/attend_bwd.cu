@@ -110,6 +110,22 @@ __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The same load without the wait: several loads in flight, then one tmem_wait_ld().
+__device__ __forceinline__ void ld32_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -437,8 +453,9 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       const int lo_vis = max(rmin - r0, 0);        // columns [lo_vis, hi_vis) visible
       const int hi_vis = key_ok ? min(32, g.R - r0) : 0;
       uint32_t sr[32], dr[32];
-      ld32(lane_base + (uint32_t)(s * 128 + half * 32), sr);
-      ld32(lane_base + (uint32_t)(s * 128 + 64 + half * 32), dr);
+      ld32_nowait(lane_base + (uint32_t)(s * 128 + half * 32), sr);  // S^T and dP^T together
+      ld32_nowait(lane_base + (uint32_t)(s * 128 + 64 + half * 32), dr);
+      tmem_wait_ld();
       uint32_t pk[16], dk[16];
       const float sc = p.scale;
 #pragma unroll
@@ -526,8 +543,9 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
       fence_after();
       const bool rot = !is_ctx && p.rope;
       uint32_t lo[32], hi[32];
-      ld32(lane_base + 256u + e0, lo);
-      ld32(lane_base + 256u + 64 + e0, hi);
+      ld32_nowait(lane_base + 256u + e0, lo);
+      ld32_nowait(lane_base + 256u + 64 + e0, hi);
+      tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 32 && store; q += 4) {
         float a4[4], h4[4];
@@ -546,8 +564,9 @@ attend_bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         *reinterpret_cast<float4*>(dk + e0 + q) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         *reinterpret_cast<float4*>(dk + 64 + e0 + q) = make_float4(h4[0], h4[1], h4[2], h4[3]);
       }
-      ld32(lane_base + 384u + e0, lo);
-      ld32(lane_base + 384u + 64 + e0, hi);
+      ld32_nowait(lane_base + 384u + e0, lo);
+      ld32_nowait(lane_base + 384u + 64 + e0, hi);
+      tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < 32 && store; q += 4) {
         *reinterpret_cast<float4*>(dv + e0 + q) =
