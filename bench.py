@@ -951,7 +951,7 @@ def run_attend_long(args):
     st.synchronize()
     ms = e0.elapsed_time(e1) / Kst
     flop = 4.0 * B * T * w.h_q * (mc + L - T + (T + 1) / 2.0) * w.d
-    print(json.dumps({"metric": "long-query attention TFLOP/s (call incl. RoPE/transpose pre-pass)",
+    print(json.dumps({"metric": "long-query attention TFLOP/s (call incl. the RoPE pre-pass)",
                       "value": round(flop / (ms / 1e3) / 1e12, 1), "unit": "TFLOP/s",
                       "ms_per_call": round(ms, 4), "steps": Kst, "dtype": "bf16",
                       "config": {"workload": "attend_long", "batch": B, "T": T, "h_q": w.h_q,

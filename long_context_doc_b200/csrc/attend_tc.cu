@@ -218,8 +218,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint64_t* pfull = bars + 9;                // P written (256 threads)
   uint64_t* ofull = bars + 10;               // P.V of the tile completed
   uint64_t* done = bars + 11;                // every issued MMA completed
-  uint64_t* vfull = bars + 12;               // [2] V^T half of the stage landed
-  uint64_t* vempty = bars + 14;              // [2] V^T half consumed (P.V done)
+  uint64_t* vfull = bars + 12;               // [2] V half of the stage landed
+  uint64_t* vempty = bars + 14;              // [2] V half consumed (P.V done)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
