@@ -540,6 +540,7 @@ def test_route_tensor_core_matches_oracle(msa, gpu, B, T, n_docs, ragged):
 
 @pytest.mark.parametrize("B,T,n_docs,ragged", [
     (8, 1, 3000, False),     # 10M-bank decode batch shape
+    (7, 1, 1900, True),      # 7 queries: the 8-warp form, a warp with no query in the merge
     (4, 1, 2501, True),      # 100M-bank decode batch shape, ragged docs
     (40, 1, 700, False),     # wide decode batch: one 48-column tile
     (3, 5, 400, True),       # short multi-token queries
