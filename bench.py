@@ -164,6 +164,15 @@ def replica_rate(world: int, units_per_rank: float, ms: float) -> float:
     return world * units_per_rank / (ms / 1e3)
 
 
+def queue_ahead(stream, ms: float = 20.0):
+    """Hold ``stream`` in a GPU spin of about ``ms`` milliseconds (cycles at up to 2 GHz) so
+    that the eager launches made after it are queued before the GPU reaches them: the CUDA
+    events placed between them then time device work alone, with no host launch gap inside."""
+    import torch
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(ms * 2e6))
+
+
 # ------------------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -323,8 +332,10 @@ class Decode:
         self.rd.route_events = ev
 
     def step(self):
+        import torch
         if self.cached:  # every cache back to its prompt; the step appends the token
-            self.lens.copy_(self.lens0)
+            with torch.cuda.stream(self.main):
+                self.lens.copy_(self.lens0)
         self.rd.step()
 
     def ctx(self, l):
@@ -398,13 +409,16 @@ def run_libmsa(args):
     clocks = sampler.stop()
     step_ms = t0.elapsed_time(t1) / Kst
     # routing-call durations for the roofline: the same step launched eagerly with CUDA events
-    # around every msa_route_topk call (on the launching stream)
+    # around every msa_route_topk call (on the launching stream), the launches queued ahead of
+    # the GPU so that the events time the call's kernels and not the host's launch latency
     Kr = max(3, min(Kst, 20))
     ev_route = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for _ in range(wk.L)] for _ in range(Kr)]
-    for s in range(Kr):
-        wk.route_ev = ev_route[s]
-        wk.step()
+    queue_ahead(wk.main)  # the eager launches queue up behind a spin: no host gap in a call
+    with torch.cuda.stream(wk.main):
+        for s in range(Kr):
+            wk.route_ev = ev_route[s]
+            wk.step()
     barrier()
     wk.route_ev = None
     route_ms = [ev_route[s][l][0].elapsed_time(ev_route[s][l][1])
@@ -699,6 +713,7 @@ def run_prefill(args):
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     sampler.start()
     for _ in range(Kst):
+        queue_ahead(st, 5.0)  # the step's launches queue up behind a spin: device time alone
         step(True)
         st.synchronize()
         for i, n in enumerate(names):
@@ -725,6 +740,8 @@ def run_prefill(args):
                    "n_chunks": n_chunks, "chunk": w.chunk, "batch": w.B, "T": w.T,
                    "h_q": w.h_q, "h_kv": w.h_kv, "d": w.d, "k": w.k, "local_kv": w.L_loc,
                    "l2": "no flush: the encode reads 6.4 GB per step, 51x the 126 MB L2",
+                   "launch": "eager; each timed step's launches queued behind a short GPU spin, "
+                             "so its events time device work and no host launch gap",
                    "parallelism": f"replicas x{world}"},
         "phases_ms": ph,
         "roofline": {"kernel": "msa_encode_pool (doc-wise RoPE + chunk mean of K, V, K_r)",
