@@ -400,14 +400,22 @@ def run_libmsa(args):
     sampler.start()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    marks = [torch.cuda.Event(enable_timing=True) for _ in range(Kst - 1)]  # between steps
     barrier()
     t0.record(wk.main)
     for s in range(Kst):
         run_step()
+        if s + 1 < Kst:
+            marks[s].record(wk.main)
     t1.record(wk.main)
     barrier()
     clocks = sampler.stop()
     step_ms = t0.elapsed_time(t1) / Kst
+    bounds = [t0] + marks + [t1]
+    per_step = sorted(bounds[i].elapsed_time(bounds[i + 1]) for i in range(Kst))
+    step_dist = {"p10": round(float(np.percentile(per_step, 10)), 4),
+                 "median": round(float(np.percentile(per_step, 50)), 4),
+                 "p90": round(float(np.percentile(per_step, 90)), 4)}
     # routing-call durations for the roofline: the same step launched eagerly with CUDA events
     # around every msa_route_topk call (on the launching stream), the launches queued ahead of
     # the GPU so that the events time the call's kernels and not the host's launch latency
@@ -480,7 +488,9 @@ def run_libmsa(args):
     achieved = wk.scan_bytes() / (route_avg / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": Kst,
-        "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "warmup": max(args.warmup, 3), "ms_per_step": round(step_ms, 4),
+        "step_ms_dist": step_dist,  # per timed step (rank 0), CUDA events between the steps
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded SplitMix64 normals, planted docs; no dataset)",
         "config": {"workload": w.name, "bank_tokens": w.n_docs * w.doc_len, "n_docs": w.n_docs,
