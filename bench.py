@@ -331,12 +331,12 @@ class Decode:
     def route_ev(self, ev):
         self.rd.route_events = ev
 
-    def step(self):
+    def step(self, local_ready=None):
         import torch
         if self.cached:  # every cache back to its prompt; the step appends the token
             with torch.cuda.stream(self.main):
                 self.lens.copy_(self.lens0)
-        self.rd.step()
+        self.rd.step(local_ready)
 
     def ctx(self, l):
         """(ctxK, ctxV, ctx_len) of layer l after a step (with one buffer set per layer)."""
@@ -433,7 +433,7 @@ def run_libmsa(args):
                 for s in range(Kr) for l in range(wk.L)]
     # end to end: per-step query inputs copied from pinned host memory, outputs read back
     # per step: every layer's Q_r and Q (one copy), the new token's K/V row of every layer's
-    # local cache, then every layer's output (one copy) and the last two layers' top-k ids
+    # local cache, then every layer's output (one copy) and every layer's top-k ids (one copy)
     host_q = wk.qbuf.cpu().pin_memory()  # every layer's Q_r, Q (and the token's K/V if cached)
     host_kv = ([] if wk.cached else
                [[t.cpu().pin_memory() for t in (d.K_loc[:, -1:], d.V_loc[:, -1:])]
@@ -444,15 +444,27 @@ def run_libmsa(args):
            sum(t.numel() * t.element_size() for hs in host_kv for t in hs))
     d2h = host_O.numel() * host_O.element_size() + host_ids.numel() * 4
 
+    kv_stream = torch.cuda.Stream(dev)
+    kv_ready = torch.cuda.Event()
+
     def e2e_step():
         with torch.cuda.stream(wk.main):
             wk.qbuf.copy_(host_q, non_blocking=True)
-            for l in range(len(host_kv)):
-                d = wk.layers[l]
-                kn, vn = host_kv[l]
-                d.K_loc[:, -1:].copy_(kn, non_blocking=True)
-                d.V_loc[:, -1:].copy_(vn, non_blocking=True)
-            wk.step()
+        ready = None
+        if host_kv:
+            # the new token's K/V rows go in on a side stream while the first layers route
+            # (only the attention reads them); the previous step's attention comes before
+            kv_stream.wait_stream(wk.main)
+            with torch.cuda.stream(kv_stream):
+                for l in range(len(host_kv)):
+                    d = wk.layers[l]
+                    kn, vn = host_kv[l]
+                    d.K_loc[:, -1:].copy_(kn, non_blocking=True)
+                    d.V_loc[:, -1:].copy_(vn, non_blocking=True)
+                kv_ready.record(kv_stream)
+            ready = kv_ready
+        with torch.cuda.stream(wk.main):
+            wk.step(ready)
             host_O.copy_(wk.obuf, non_blocking=True)
             host_ids.copy_(wk.rd.ids, non_blocking=True)
 

@@ -315,8 +315,12 @@ class RoutedDecode:
                               self.stream)
 
     # ----------------------------------------------------------------- the step
-    def step(self):
-        """Enqueue one decode step of every routed layer on ``self.stream``."""
+    def step(self, local_ready: "torch.cuda.Event" = None):
+        """Enqueue one decode step of every routed layer on ``self.stream``.
+
+        ``local_ready``: optional CUDA event that the stream waits on before the first
+        attention, for attention inputs (the local K/V, a cache's new token) that another stream
+        writes while the first layers route; routing reads none of them."""
         self._route(0)
         self._fetch_begin(0)
         for l in range(self.L):
@@ -324,6 +328,8 @@ class RoutedDecode:
                 self._route(l + 1)
                 self._fetch_begin(l + 1)
             self._fetch_finish(l)
+            if l == 0 and local_ready is not None:
+                self.stream.wait_event(local_ready)
             self._attend(l)
 
     @property

@@ -135,6 +135,37 @@ def test_routed_decode_step_matches_oracle(msa, gpu, host_layers, fetch, scan, g
     _check_against_oracle(rd, host_layers)
 
 
+def test_routed_decode_waits_for_local_inputs(msa, gpu, host_layers):
+    """``step(local_ready=ev)``: the local K/V rows of the query token, written on another
+    stream behind a ~25 ms spin (long after the first layers have routed), reach the first
+    attention because the step's stream waits on the event: the outputs equal, bit for bit,
+    those of the same step with the rows already in place."""
+    rd = _build(msa, gpu, host_layers, "zerocopy", "tc")
+    torch.cuda.synchronize()
+    rd.step()
+    torch.cuda.synchronize()
+    O_ref = rd.O.clone()
+    ids_ref = rd.ids.clone()
+    rows = [(la.K_loc[:, -1:].clone(), la.V_loc[:, -1:].clone()) for la in rd.layers]
+    for la in rd.layers:
+        la.K_loc[:, -1:].zero_()
+        la.V_loc[:, -1:].zero_()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream(gpu)
+    ready = torch.cuda.Event()
+    with torch.cuda.stream(side):
+        torch.cuda._sleep(50_000_000)
+        for la, (k, v) in zip(rd.layers, rows):
+            la.K_loc[:, -1:].copy_(k)
+            la.V_loc[:, -1:].copy_(v)
+        ready.record(side)
+    rd.step(local_ready=ready)
+    torch.cuda.synchronize()
+    assert torch.equal(rd.ids, ids_ref)
+    assert torch.equal(rd.O, O_ref)
+    _check_against_oracle(rd, host_layers)
+
+
 def test_routed_decode_rejects_bad_configurations(msa, gpu, host_layers):
     """A fetch mode that does not match where the bank lives is refused, and so is capturing the
     cudaMemcpyAsync fetch (it waits on the host for every layer's ids)."""
