@@ -248,12 +248,16 @@ class Decode:
         self.cached = cached
         seed_w = w.scaled(seed=w.seed + 1000 * rank)
         B = w.B
-        # every layer's query inputs (Q_r, Q, and with caches the token's K/V) in one contiguous
-        # buffer, so that a step's host copy of them is one transfer
+        # every layer's query inputs in one contiguous buffer: first the router queries Q_r of
+        # all layers (what the routing reads), then per layer Q and, with caches, the token's K/V
+        # (what only the attention reads), so that a step's host copy is two transfers and the
+        # second can go in beside the routing
         nqr, nq = B * w.T * w.h_qr * w.d, B * w.T * w.h_q * w.d
         nkv = B * w.T * w.h_kv * w.d if cached else 0
-        self.per_layer = nqr + nq + 2 * nkv
-        self.qbuf = torch.empty(self.L * self.per_layer, dtype=torch.bfloat16, device=dev)
+        self.n_route_in = self.L * nqr
+        att_per_layer = nq + 2 * nkv
+        self.qbuf = torch.empty(self.n_route_in + self.L * att_per_layer, dtype=torch.bfloat16,
+                                device=dev)
         # rotated local caches of L_loc rows: the first L_loc - 1 hold the prompt, the step
         # appends the query token's own K/V; a step starts by resetting every length
         self.lens = torch.zeros(self.L, dtype=torch.int32, device=dev)
@@ -266,9 +270,9 @@ class Decode:
             coff_host = dv["doc_chunk_off"]
             if fetch != "device" and Kh is None:
                 Kh, Vh = self._host_bank(seed_w, coff_host, dev)
-            base = l * self.per_layer
-            Q_r = self.qbuf[base:base + nqr].view(dv["Q_r"].shape)
-            Q = self.qbuf[base + nqr:base + nqr + nq].view(dv["Q"].shape)
+            base = self.n_route_in + l * att_per_layer
+            Q_r = self.qbuf[l * nqr:(l + 1) * nqr].view(dv["Q_r"].shape)
+            Q = self.qbuf[base:base + nq].view(dv["Q"].shape)
             Q_r.copy_(dv["Q_r"])
             Q.copy_(dv["Q"])
             kv = (Kh, Vh) if fetch != "device" else (dv["Kbar"], dv["Vbar"])
@@ -282,7 +286,7 @@ class Decode:
                 c = msa.LocalCache(B, w.L_loc, w.h_kv, w.d, pos0=w.k, rope_base=w.rope_base,
                                    device=dev, length=self.lens[l:l + 1])
                 c.append(dv["K_loc"][:, :-T].contiguous(), dv["V_loc"][:, :-T].contiguous())
-                o = base + nqr + nq
+                o = base + nq
                 K_new = self.qbuf[o:o + nkv].view(B, T, w.h_kv, w.d)
                 V_new = self.qbuf[o + nkv:o + 2 * nkv].view(B, T, w.h_kv, w.d)
                 K_new.copy_(dv["K_loc"][:, -T:])
@@ -445,28 +449,32 @@ def run_libmsa(args):
     d2h = host_O.numel() * host_O.element_size() + host_ids.numel() * 4
 
     kv_stream = torch.cuda.Stream(dev)
-    kv_ready = torch.cuda.Event()
+    att_ready, step_done = torch.cuda.Event(), torch.cuda.Event()
+    nr = wk.n_route_in
 
     def e2e_step():
         with torch.cuda.stream(wk.main):
-            wk.qbuf.copy_(host_q, non_blocking=True)
-        ready = None
-        if host_kv:
-            # the new token's K/V rows go in on a side stream while the first layers route
-            # (only the attention reads them); the previous step's attention comes before
-            kv_stream.wait_stream(wk.main)
-            with torch.cuda.stream(kv_stream):
-                for l in range(len(host_kv)):
-                    d = wk.layers[l]
-                    kn, vn = host_kv[l]
-                    d.K_loc[:, -1:].copy_(kn, non_blocking=True)
-                    d.V_loc[:, -1:].copy_(vn, non_blocking=True)
-                kv_ready.record(kv_stream)
-            ready = kv_ready
+            wk.qbuf[:nr].copy_(host_q[:nr], non_blocking=True)  # the router queries
+        # what only the attention reads (Q, the new token's K/V) goes in on a side stream while
+        # the first layers route; the previous step's attention, which read it, comes before
+        kv_stream.wait_stream(wk.main)
+        with torch.cuda.stream(kv_stream):
+            wk.qbuf[nr:].copy_(host_q[nr:], non_blocking=True)
+            for l in range(len(host_kv)):
+                d = wk.layers[l]
+                kn, vn = host_kv[l]
+                d.K_loc[:, -1:].copy_(kn, non_blocking=True)
+                d.V_loc[:, -1:].copy_(vn, non_blocking=True)
+            att_ready.record(kv_stream)
         with torch.cuda.stream(wk.main):
-            wk.step(ready)
+            wk.step(att_ready)
+            step_done.record(wk.main)
             host_O.copy_(wk.obuf, non_blocking=True)
+        # the two reads back run side by side
+        kv_stream.wait_event(step_done)
+        with torch.cuda.stream(kv_stream):
             host_ids.copy_(wk.rd.ids, non_blocking=True)
+        wk.main.wait_stream(kv_stream)
 
     for _ in range(3):
         e2e_step()
