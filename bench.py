@@ -1291,8 +1291,10 @@ def run_generate(args):
     torch.cuda.synchronize()
     assert int(lens[0]) == L0
 
-    def token_step():
+    def token_step(rest_ready=None):
         for l in range(wk.L):
+            if l == 1 and rest_ready is not None:  # the inputs of layers 1.. arrive beside layer 0
+                wk.main.wait_event(rest_ready)
             x, c = tok[l], caches[l]
             cK, cV, cl = wk.ctx(l)
             msa.msa_decode_step(x["Q"], x["K"], x["V"], c.K, c.V, c.length, cK, cV, cl, w.k,
@@ -1386,9 +1388,21 @@ def run_generate(args):
     h2d = q_h2d + G * tok_h2d
     d2h = G * host_out.numel() * host_out.element_size()
 
+    tok_stream = torch.cuda.Stream(dev)
+    rest_ready = torch.cuda.Event()
+
     def e2e_token():
-        tokbuf.copy_(host_tok, non_blocking=True)
-        token_step()
+        # layer 0's token inputs first; those of the other layers on a side stream while layer
+        # 0 attends (the previous token's steps, which read them, come before)
+        tokbuf[:per_layer].copy_(host_tok[:per_layer], non_blocking=True)
+        ready = None
+        if wk.L > 1:
+            tok_stream.wait_stream(wk.main)
+            with torch.cuda.stream(tok_stream):
+                tokbuf[per_layer:].copy_(host_tok[per_layer:], non_blocking=True)
+                rest_ready.record(tok_stream)
+            ready = rest_ready
+        token_step(ready)
         host_out.copy_(tok[-1]["O"], non_blocking=True)
 
     def e2e_con():
