@@ -539,7 +539,10 @@ def run_libmsa(args):
                                                    f"route_tc_{w.name}_dram.json")
                                  if wk.scan == "tc" else None),
                      "bytes_per_launch": wk.scan_bytes(),
-                     "avg_launch_ms": round(route_avg, 4)},
+                     "avg_launch_ms": round(route_avg, 4),
+                     "timing": "CUDA events around every routing call of an eager pass of the "
+                               "same step after the timed replays, its launches queued behind "
+                               "a GPU spin (no host launch gap inside a call)"},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": Kst * wk.kernels_per_step,
