@@ -197,3 +197,61 @@ def test_encode_hidden_rejects_bad_arguments_on_host(msa):
     assert call(n_chunks=4) == 1       # inconsistent with the offsets
     assert call(offs=np.array([0, 70, 60], np.int64)) == 1  # decreasing offsets
     assert call(wsb=ws_bytes - 1) == 3
+
+
+C_CALLER = r"""
+/* A plain C11 caller of the boundary: header compiled as C, library linked as a C library. */
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+#include "msa.h"
+
+static int fail(const char* what) { fprintf(stderr, "FAIL %s\n", what); return 1; }
+
+int main(void) {
+  if ((msa_version() >> 16) != 1) return fail("version");
+  if (strcmp(msa_status_string(MSA_OK), "MSA_OK") != 0) return fail("status MSA_OK");
+  if (strcmp(msa_status_string(MSA_ERR_DEVICE), "MSA_ERR_DEVICE") != 0) return fail("status");
+  /* documents of 1, 64, 65 and 0 tokens in chunks of 64: 1 + 1 + 2 + 0 chunks */
+  const int64_t off[5] = {0, 1, 65, 130, 130};
+  if (msa_count_chunks(off, 4, 64) != 4) return fail("count_chunks");
+  const int64_t bad[3] = {0, 5, 3};
+  if (msa_count_chunks(bad, 2, 64) != -1) return fail("count_chunks order");
+  /* k larger than the bank: refused on the host before any device work */
+  const int64_t coff[3] = {0, 2, 4};
+  int32_t ids[8];
+  float sc[8];
+  char ws[256];
+  const msa_status s = msa_route_topk((const void*)ws, 1, 1, 8, (const void*)ws, NULL, NULL, coff,
+                                      2, 4, 8, 128, MSA_BF16, 3, NULL, ids, sc, NULL, ws,
+                                      sizeof ws, NULL);
+  if (s != MSA_ERR_INVALID_ARG) return fail("route k > n_docs");
+  if (strlen(msa_last_error()) == 0) return fail("last_error");
+  printf("ok\n");
+  return 0;
+}
+"""
+
+
+def test_header_compiles_and_links_as_c(msa, tmp_path):
+    """The boundary from plain C: msa.h compiles as C11 with -pedantic -Werror, the program links
+    against libmsa.so, and host-side calls (version, status strings, the chunk count, a
+    rejected routing call with its message) behave as documented, without a GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(msa.LIB_PATH)
+    libname = os.path.basename(msa.LIB_PATH)
+    assert libname.startswith("lib") and libname.endswith(".so")
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-l" + libname[3:-3], "-Wl,-rpath," + libdir],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
