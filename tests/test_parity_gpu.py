@@ -552,6 +552,27 @@ def test_route_tensor_core_decode_matches_oracle(msa, gpu, B, T, n_docs, ragged)
     assert np.array_equal(ids[:, 0], inp["planted"][:, 0])
 
 
+@pytest.mark.parametrize("scan,B,n_docs,k", [
+    ("tc", 8, 900, 32),    # the largest k: a full 32-lane list per query
+    ("cc", 8, 900, 32),
+    ("tc", 64, 600, 32),   # the largest tensor-core batch (one 64-column query tile)
+    ("tc", 4, 20, 20),     # every document selected, fewer chunk tiles than SMs
+], ids=["tc_k32", "cc_k32", "tc_b64_k32", "tc_all_docs"])
+def test_route_largest_k_and_batch(msa, gpu, scan, B, n_docs, k):
+    """Maximum sizes of the routing call: k = 32 (the fused top-k's one-warp list), 64 decode
+    queries in one tensor-core tile, and k = n_docs (every document ranked)."""
+    w = synth.C3.scaled(n_docs=n_docs, B=B, T=1, ragged=True, seed=500 + B + k, k=k)
+    inp = synth.make_bank_workload(w)
+    if scan == "tc":
+        ids, _ = _route_tc_check(msa, gpu, inp["Q_r"], inp["Kbar_r"], inp["doc_chunk_off"], k)
+    else:
+        ids = _route_check(msa, gpu, inp["Q_r"], inp["Kbar_r"], inp["doc_chunk_off"], k,
+                           "bf16")[0]
+    assert np.array_equal(ids[:, 0], inp["planted"][:, 0])
+    if k == n_docs:
+        assert all(sorted(r) == list(range(n_docs)) for r in ids.tolist())
+
+
 def test_route_tensor_core_full_10m_token_bank_decode(msa, gpu):
     w = synth.C3
     dv = synth.dev_bank_workload(w, gpu, with_kv=False)
