@@ -304,13 +304,15 @@ def test_route_reports_small_workspace(msa, gpu):
 
 
 # ----------------------------------------------------------------------------- gather
-def test_gather_indices_exact_and_rows_copied(msa, gpu):
-    w = synth.C3.scaled(n_docs=300, B=5, ragged=True, seed=5)
+@pytest.mark.parametrize("k", [16, 32])  # 32: every lane of the ranking warp holds an id
+def test_gather_indices_exact_and_rows_copied(msa, gpu, k):
+    w = synth.C3.scaled(n_docs=300, B=5, ragged=True, seed=5, k=k)
     inp, d = _bank_inputs(w, gpu)
     coff = inp["doc_chunk_off"]
     rng = np.random.default_rng(3)
     ids = np.stack([rng.choice(w.n_docs, w.k, replace=False) for _ in range(w.B)]).astype(np.int32)
     ids[2, 3] = -1
+    ids[4, k - 1] = -1  # an empty last slot
     max_ctx = int(w.k * np.max(np.diff(coff)))
     gi, cl, cK, cV = msa.gather(torch.from_numpy(ids).to(gpu), d["doc_chunk_off"], d["Kbar"],
                                 d["Vbar"], max_ctx)
