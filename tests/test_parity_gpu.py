@@ -437,11 +437,13 @@ def _attend_case(msa, gpu, dt, B, T, h_q, h_kv, d, L, n_ctx, pos0, base, seed=0)
     ("bf16", 1, 1, 8, 2, 128, 200, [70], 2, 0.0),       # RoPE off
     ("bf16", 2, 1, 32, 8, 128, 1024, [96, 128], 5000, 1e6),  # positions up to 6k
     ("fp32", 1, 1, 2, 1, 64, 1, [1], 0, 1e6),           # one memory row + the query itself
+    ("bf16", 2, 1, 32, 8, 128, 2048, [256, 200], 32, 1e6),  # k = 32 docs of 8 chunks (max k)
     # long queries (bf16, d = 128, >= 64 query rows per KV head): the tensor-core kernel
     ("bf16", 2, 64, 16, 4, 128, 300, [0, 200], 9, 1e6),  # 2 query tiles, padded L, no memory
     ("bf16", 1, 40, 64, 8, 128, 40, [70], 3, 1e4),      # 8 heads per KV head, partial tile, L = T
     ("bf16", 2, 128, 8, 8, 128, 256, [64, 5], 0, 0.0),  # one head per KV head, RoPE off
     ("bf16", 1, 256, 32, 8, 128, 1300, [64], 8, 1e6),   # interleave-round shape, 11 local tiles
+    ("bf16", 1, 128, 32, 8, 128, 128, [512], 32, 1e6),  # prefill shape at k = 32 (512 memory rows)
 ])
 def test_attend_matches_oracle(msa, gpu, dt, B, T, h_q, h_kv, d, L, ctx, pos0, base):
     _attend_case(msa, gpu, dt, B, T, h_q, h_kv, d, L, np.array(ctx), pos0, base)
