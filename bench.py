@@ -209,8 +209,14 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
+        return self.summarize(self.lines)
+
+    @classmethod
+    def summarize(cls, lines):
+        """Median SM clock, the highest max clock and the throttle reasons seen active, from
+        ``nvidia-smi --format=csv,noheader,nounits`` lines of FIELDS (malformed lines skipped)."""
         sm, mx, reasons = [], [], set()
-        for ln in self.lines:
+        for ln in lines:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -219,7 +225,7 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
-            for name, v in zip(self.NAMES, parts[3:7]):
+            for name, v in zip(cls.NAMES, parts[3:7]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
