@@ -37,3 +37,34 @@ def test_clock_summary_without_samples():
 def test_replica_rate_is_the_whole_job():
     assert bench.replica_rate(1, 4, 10.0) == pytest.approx(400.0)
     assert bench.replica_rate(8, 4, 10.0) == pytest.approx(3200.0)  # 8 replicas, the max time
+
+
+def test_captured_traffic_only_for_the_captured_sources(tmp_path, monkeypatch):
+    """The bench reports a committed capture's DRAM bytes only while the kernel's sources
+    hash to the value recorded with the capture; otherwise (or with no capture) null."""
+    import hashlib
+    import json
+    csrc = tmp_path / "long_context_doc_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cu").write_text("kernel one\n")
+    (csrc / "c.cuh").write_text("common\n")
+    sha = hashlib.sha256(b"kernel one\n" + b"common\n").hexdigest()
+    rec = {"kernel_src_sha256": sha, "dram_bytes_read": 1000, "dram_bytes_write": 24}
+    (tmp_path / "profiles" / "cap.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic(("k.cu", "c.cuh"), "cap.json") == 1024
+    assert bench.captured_traffic(("c.cuh", "k.cu"), "cap.json") is None  # order is part of it
+    (csrc / "k.cu").write_text("kernel two\n")
+    assert bench.captured_traffic(("k.cu", "c.cuh"), "cap.json") is None
+    assert bench.captured_traffic(("k.cu",), "missing.json") is None
+
+
+def test_committed_captures_name_their_sources():
+    import json
+    for name in os.listdir(os.path.join(ROOT, "profiles")):
+        if name.endswith("_dram.json"):
+            with open(os.path.join(ROOT, "profiles", name)) as f:
+                rec = json.load(f)
+            assert len(rec["kernel_src_sha256"]) == 64, name
+            assert int(rec["dram_bytes_read"]) > 0 and int(rec["dram_bytes_write"]) >= 0, name
