@@ -61,7 +61,8 @@ def parse():
     ap.add_argument("--impl", default="libmsa", choices=["libmsa", "reference"])
     ap.add_argument("--workload", default="bank100m",
                     choices=["bank100m", "bank10m", "prefill1m", "interleave10m", "attend_long",
-                             "gen100m", "encode_hidden1m", "attend_bwd", "fetch100m"])
+                             "gen100m", "encode_hidden1m", "attend_bwd", "fetch100m",
+                             "aux_loss"])
     ap.add_argument("--gen-tokens", type=int, default=256,
                     help="gen100m: tokens generated per query after the context is built")
     ap.add_argument("--fetch", default="zerocopy", choices=["memcpy", "zerocopy"],
@@ -1015,6 +1016,72 @@ def run_attend_long(args):
           flush=True)
 
 
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # 148 SMs x 128 fp32 lanes x FMA at 1965 MHz
+
+
+def run_aux_loss(args):
+    """The auxiliary routing loss with its gradients (msa_aux_routing_loss: the chunk scores and
+    their maximising tokens, the per-query loss and dL/ds, dK̄_r, dQ_r) over the 1M-token prefill
+    bank (16,384 chunks of 8 KV heads x 128), B = 4 training queries of 128 tokens with 8 router
+    heads, the chunks of 16 documents relevant per query; CUDA events on the launching stream,
+    the calls queued behind a GPU spin."""
+    import torch
+
+    import long_context_doc_b200 as msa
+    import synth
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.C2
+    B, T = 4, w.T
+    cpd = (w.doc_len + w.chunk - 1) // w.chunk
+    n_chunks = w.n_docs * cpd
+    bf = torch.bfloat16
+    Q_r = synth.dev_normal(torch.empty((B, T, w.h_qr, w.d), dtype=bf, device=dev), w.seed, 11)
+    K_r = synth.dev_normal(torch.empty((n_chunks, w.h_kv, w.d), dtype=bf, device=dev), w.seed, 12)
+    words = (n_chunks + 31) // 32
+    pos = np.zeros((B, words), np.uint32)
+    rng = np.random.default_rng(w.seed)
+    for b in range(B):  # the chunks of 16 relevant documents per query
+        for doc in rng.choice(w.n_docs, 16, replace=False):
+            for c in range(int(doc) * cpd, (int(doc) + 1) * cpd):
+                pos[b, c // 32] |= np.uint32(1) << np.uint32(c % 32)
+    bits = torch.from_numpy(pos.view(np.int32)).to(dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    dQ = torch.empty((B, T, w.h_qr, w.d), dtype=torch.float32, device=dev)
+    dK = torch.empty((n_chunks, w.h_kv, w.d), dtype=torch.float32, device=dev)
+    ws_bytes = int(msa.lib.msa_aux_routing_loss_workspace(B, n_chunks))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = torch.cuda.Stream()
+    for _ in range(max(args.warmup, 3)):
+        msa.msa_aux_routing_loss(Q_r, K_r, bits, 0.1, loss, dQ, dK, ws, st)
+    st.synchronize()
+    assert np.isfinite(float(loss.item()))
+    Kst = max(1, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    queue_ahead(st, 5.0)
+    e0.record(st)
+    for _ in range(Kst):
+        msa.msa_aux_routing_loss(Q_r, K_r, bits, 0.1, loss, dQ, dK, ws, st)
+    e1.record(st)
+    st.synchronize()
+    ms = e0.elapsed_time(e1) / Kst
+    flop = 2.0 * B * T * w.h_qr * w.d * n_chunks  # the cosines' dot products (the bulk)
+    tf = flop / (ms / 1e3) / 1e12
+    print(json.dumps({
+        "metric": "auxiliary routing loss with gradients, TFLOP/s of the chunk-score cosines",
+        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4), "steps": Kst,
+        "dtype": "bf16 in, f32 arithmetic",
+        "config": {"workload": "aux_loss", "batch": B, "T": T, "h_qr": w.h_qr, "h_kv": w.h_kv,
+                   "d": w.d, "n_chunks": n_chunks, "relevant_docs_per_query": 16, "tau": 0.1},
+        "roofline": {"kernel": "msa_aux_routing_loss (4 launches: scores, loss, dK, dQ)",
+                     "bound": "alu", "achieved": round(tf, 2),
+                     "peak": round(FP32_ALU_TFLOPS, 1), "unit": "TFLOP/s",
+                     "frac": round(tf / FP32_ALU_TFLOPS, 4),
+                     "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 at 1965 MHz",
+                     "traffic": None}}), flush=True)
+
+
 def run_attend_backward(args):
     """The backward of the sparse attention at the last interleave round's shape (B = 4 queries
     of T = 256 tokens, 32 query heads over 8 KV heads, 64 memory rows + 8,256 local rows):
@@ -1663,6 +1730,8 @@ def main():
         run_encode_hidden(args)
     elif args.workload == "attend_bwd":
         run_attend_backward(args)
+    elif args.workload == "aux_loss":
+        run_aux_loss(args)
     elif args.workload == "fetch100m":
         run_fetch(args)
     else:
