@@ -1068,6 +1068,7 @@ def run_aux_loss(args):
     ms = e0.elapsed_time(e1) / Kst
     flop = 2.0 * B * T * w.h_qr * w.d * n_chunks  # the cosines' dot products (the bulk)
     tf = flop / (ms / 1e3) / 1e12
+    cpu = None if args.no_cpu_baseline else cpu_aux_loss_baseline(w, B, T, n_chunks, flop)
     print(json.dumps({
         "metric": "auxiliary routing loss with gradients, TFLOP/s of the chunk-score cosines",
         "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_call": round(ms, 4), "steps": Kst,
@@ -1079,7 +1080,31 @@ def run_aux_loss(args):
                      "peak": round(FP32_ALU_TFLOPS, 1), "unit": "TFLOP/s",
                      "frac": round(tf / FP32_ALU_TFLOPS, 4),
                      "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 at 1965 MHz",
-                     "traffic": None}}), flush=True)
+                     "traffic": None},
+        "cpu_baseline": cpu}), flush=True)
+
+
+def cpu_aux_loss_baseline(w, B: int, T: int, n_chunks: int, flop: float,
+                          n_sample: int = 512) -> dict:
+    """The oracle's auxiliary loss with its gradients on a bank of ``n_sample`` chunks (the same
+    queries' shape, 16 relevant documents' worth of positives scaled down), its time scaled to
+    the full bank by the chunk count (the oracle is linear in it)."""
+    import oracle
+    import synth
+    Q = synth.normal(w.seed, 11, (B, T, w.h_qr, w.d), "bf16")
+    K = synth.normal(w.seed, 12, (n_sample, w.h_kv, w.d), "bf16")
+    pos = np.zeros((B, n_sample), bool)
+    rng = np.random.default_rng(w.seed)
+    for b in range(B):
+        pos[b, rng.choice(n_sample, max(1, n_sample // 64), replace=False)] = True
+    t0 = time.perf_counter()
+    oracle.aux_routing_loss(synth.as_f32(Q, "bf16"), synth.as_f32(K, "bf16"), pos, 0.1)
+    dt = time.perf_counter() - t0
+    full = dt * n_chunks / n_sample
+    return {"value": round(flop / full / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"the same call on {n_sample} of {n_chunks} chunks, time scaled by the "
+                       f"chunk count ({dt:.2f} s measured, {full:.1f} s per full call)")}
 
 
 def run_attend_backward(args):
